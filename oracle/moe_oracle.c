@@ -1,0 +1,249 @@
+/*
+ * moe_oracle.c -- plain, slow, single-threaded fp64 CPU oracle of the
+ * sparse Mixture-of-Experts block forward.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path may call, link or
+ * load this file: only the test suite, the smoke check and the benchmark's
+ * CPU-baseline leg use it.  It shares no code, header, table or helper with
+ * the CUDA library.
+ *
+ * What it computes is the definition printed in the article
+ * "Qwen3MoeSparseMoeBlock performance optimisation in practice" (parallelising
+ * a sparse mixture-of-experts system), section 1, the forward() listing and
+ * the four-stage workflow above it:
+ *   stage 1  router logits = x . W_router (+ per-expert bias), softmax over E
+ *   stage 2  top-k experts per token by probability; the listing keeps the
+ *            top-k probabilities as routing weights and does NOT renormalise
+ *   stage 3  each selected expert processes its tokens
+ *   stage 4  the expert outputs are summed per token, weighted by the routing
+ *            weights (the prose of stage 4; the listing's index_add_ omits the
+ *            multiply, the prose requires it)
+ * The per-expert bias follows the gating formula G(x) = Softmax(W_g x + b_g)
+ * of the Hunyuan-Large overview page, section 2.1.  The expert MLP is the
+ * SwiGLU form down(silu(gate(x)) * up(x)) with silu(z) = z / (1 + exp(-z));
+ * the routing weight multiplies the expert's output (after the down
+ * projection).
+ *
+ * Readings where the pages are silent:
+ *   - ties in probability: the lower expert index ranks first; the k slots of
+ *     a token are ordered by descending probability;
+ *   - the order of tokens inside one expert group: ascending flat assignment
+ *     index t*k + j (a stable counting sort);
+ *   - every sum runs in ascending index order, in fp64, with no intermediate
+ *     rounding; bf16 inputs are widened exactly.
+ *
+ * Layouts (row-major, contiguous; bf16 given as raw uint16 bit patterns):
+ *   x [T][d], W_router [d][E], bias [E] (fp32, may be NULL),
+ *   W_gate [E][d][f], W_up [E][d][f], W_down [E][f][d].
+ *
+ * Parity status: every function here is pinned by CPU tests against
+ * independent computations (brute force, library routines, invariants and
+ * special cases); nothing is "parity unpinned".
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORACLE_OK 0
+#define ORACLE_BAD_ARG 1
+#define ORACLE_NO_MEMORY 2
+
+/* Exact widening of one bf16 bit pattern: bf16 is the top half of an fp32. */
+static double bf16_to_double(uint16_t bits)
+{
+    uint32_t u = (uint32_t)bits << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/* One (probability, expert index) pair, for the top-k sort. */
+typedef struct {
+    double p;
+    int32_t e;
+} ranked_t;
+
+/* Descending probability; equal probabilities: lower expert index first. */
+static int by_prob_desc_then_index(const void* a, const void* b)
+{
+    const ranked_t* ra = (const ranked_t*)a;
+    const ranked_t* rb = (const ranked_t*)b;
+    if (ra->p > rb->p) return -1;
+    if (ra->p < rb->p) return 1;
+    return (ra->e > rb->e) - (ra->e < rb->e);
+}
+
+/*
+ * Stages 1 and 2 for every token.
+ *   logits_out [T][E]  (may be NULL)  x . W_router + bias, fp64
+ *   probs_out  [T][E]  (may be NULL)  softmax over the E experts
+ *   ids        [T][k]                 selected experts, descending probability
+ *   weights    [T][k]                 their probabilities, not renormalised
+ */
+int oracle_route(const uint16_t* x, const uint16_t* w_router, const float* bias,
+                 int64_t T, int64_t d, int64_t E, int64_t k,
+                 double* logits_out, double* probs_out,
+                 int32_t* ids, double* weights)
+{
+    if (!x || !w_router || !ids || !weights || T < 0 || d < 1 || E < 1 || k < 1 || k > E)
+        return ORACLE_BAD_ARG;
+    double* logit = (double*)malloc(sizeof(double) * E);
+    double* prob = (double*)malloc(sizeof(double) * E);
+    ranked_t* ranked = (ranked_t*)malloc(sizeof(ranked_t) * E);
+    if (!logit || !prob || !ranked) {
+        free(logit); free(prob); free(ranked);
+        return ORACLE_NO_MEMORY;
+    }
+    for (int64_t t = 0; t < T; ++t) {
+        /* router logits: sum over the hidden index i, ascending */
+        for (int64_t e = 0; e < E; ++e) logit[e] = 0.0;
+        for (int64_t i = 0; i < d; ++i) {
+            double xi = bf16_to_double(x[t * d + i]);
+            const uint16_t* wrow = w_router + i * E;
+            for (int64_t e = 0; e < E; ++e) logit[e] += xi * bf16_to_double(wrow[e]);
+        }
+        if (bias)
+            for (int64_t e = 0; e < E; ++e) logit[e] += (double)bias[e];
+
+        /* softmax over experts, shifted by the maximum logit */
+        double m = logit[0];
+        for (int64_t e = 1; e < E; ++e) if (logit[e] > m) m = logit[e];
+        double s = 0.0;
+        for (int64_t e = 0; e < E; ++e) {
+            prob[e] = exp(logit[e] - m);
+            s += prob[e];
+        }
+        for (int64_t e = 0; e < E; ++e) prob[e] /= s;
+
+        /* top-k: sort all experts by (probability desc, index asc) */
+        for (int64_t e = 0; e < E; ++e) {
+            ranked[e].p = prob[e];
+            ranked[e].e = (int32_t)e;
+        }
+        qsort(ranked, (size_t)E, sizeof(ranked_t), by_prob_desc_then_index);
+        for (int64_t j = 0; j < k; ++j) {
+            ids[t * k + j] = ranked[j].e;
+            weights[t * k + j] = ranked[j].p;
+        }
+        if (logits_out) memcpy(logits_out + t * E, logit, sizeof(double) * E);
+        if (probs_out) memcpy(probs_out + t * E, prob, sizeof(double) * E);
+    }
+    free(logit); free(prob); free(ranked);
+    return ORACLE_OK;
+}
+
+/*
+ * Grouping of the T*k assignments by expert (the "token reordering" step of
+ * the article's section 2.2: sort_tokens_by_expert, then gather).
+ *   counts  [E]    assignments per expert
+ *   offsets [E+1]  exclusive prefix sum of counts; offsets[E] = T*k
+ *   perm    [T*k]  perm[pos] = t*k + j of the assignment at grouped row pos
+ *   inv     [T*k]  inv[t*k + j] = pos
+ * Inside one expert group the assignments keep ascending flat order.
+ */
+int oracle_permute(const int32_t* ids, int64_t T, int64_t E, int64_t k,
+                   int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* inv)
+{
+    if (!ids || !counts || !offsets || !perm || !inv || T < 0 || E < 1 || k < 1)
+        return ORACLE_BAD_ARG;
+    const int64_t n = T * k;
+    for (int64_t a = 0; a < n; ++a)
+        if (ids[a] < 0 || ids[a] >= E) return ORACLE_BAD_ARG;
+    for (int64_t e = 0; e < E; ++e) counts[e] = 0;
+    for (int64_t a = 0; a < n; ++a) counts[ids[a]] += 1;
+    offsets[0] = 0;
+    for (int64_t e = 0; e < E; ++e) offsets[e + 1] = offsets[e] + counts[e];
+    int32_t* next = (int32_t*)malloc(sizeof(int32_t) * E);
+    if (!next) return ORACLE_NO_MEMORY;
+    for (int64_t e = 0; e < E; ++e) next[e] = offsets[e];
+    for (int64_t a = 0; a < n; ++a) {
+        int32_t pos = next[ids[a]]++;
+        perm[pos] = (int32_t)a;
+        inv[a] = pos;
+    }
+    free(next);
+    return ORACLE_OK;
+}
+
+/*
+ * One expert's SwiGLU MLP on one token row (stage 3):
+ *   g = x . W_gate[e],  u = x . W_up[e]          (sums over i ascending)
+ *   h = silu(g) * u,    silu(z) = z / (1 + exp(-z))
+ *   o = h . W_down[e]                            (sum over n ascending)
+ */
+static void expert_swiglu(const double* xrow, const uint16_t* wg, const uint16_t* wu,
+                          const uint16_t* wd, int64_t d, int64_t f,
+                          double* g, double* u, double* h, double* o)
+{
+    for (int64_t n = 0; n < f; ++n) { g[n] = 0.0; u[n] = 0.0; }
+    for (int64_t i = 0; i < d; ++i) {
+        const double xi = xrow[i];
+        const uint16_t* grow = wg + i * f;
+        const uint16_t* urow = wu + i * f;
+        for (int64_t n = 0; n < f; ++n) {
+            g[n] += xi * bf16_to_double(grow[n]);
+            u[n] += xi * bf16_to_double(urow[n]);
+        }
+    }
+    for (int64_t n = 0; n < f; ++n) h[n] = g[n] / (1.0 + exp(-g[n])) * u[n];
+    for (int64_t c = 0; c < d; ++c) o[c] = 0.0;
+    for (int64_t n = 0; n < f; ++n) {
+        const double hn = h[n];
+        const uint16_t* drow = wd + n * d;
+        for (int64_t c = 0; c < d; ++c) o[c] += hn * bf16_to_double(drow[c]);
+    }
+}
+
+/*
+ * Stages 3 and 4 for a chosen list of tokens, given the routing from
+ * oracle_route:
+ *   out   [n_rows][d]     out[r] = sum_{j ascending} w[t][j] * expert_{ids[t][j]}(x[t]),
+ *                         t = rows[r]
+ *   y_out [n_rows][k][d]  (may be NULL)  the weighted per-slot expert outputs
+ *   h_out [n_rows][k][f]  (may be NULL)  silu(g) * u per slot
+ * Every output row depends only on its own token, so any subset of tokens
+ * gives exactly the rows a full evaluation would.
+ */
+int oracle_expert_rows(const uint16_t* x, const uint16_t* w_gate, const uint16_t* w_up,
+                       const uint16_t* w_down, int64_t T, int64_t d, int64_t E, int64_t k,
+                       int64_t f, const int32_t* ids, const double* weights,
+                       int64_t n_rows, const int64_t* rows,
+                       double* out, double* y_out, double* h_out)
+{
+    if (!x || !w_gate || !w_up || !w_down || !ids || !weights || !rows || !out ||
+        T < 0 || d < 1 || E < 1 || k < 1 || f < 1 || n_rows < 0)
+        return ORACLE_BAD_ARG;
+    double* xrow = (double*)malloc(sizeof(double) * d);
+    double* g = (double*)malloc(sizeof(double) * f);
+    double* u = (double*)malloc(sizeof(double) * f);
+    double* h = (double*)malloc(sizeof(double) * f);
+    double* o = (double*)malloc(sizeof(double) * d);
+    if (!xrow || !g || !u || !h || !o) {
+        free(xrow); free(g); free(u); free(h); free(o);
+        return ORACLE_NO_MEMORY;
+    }
+    int status = ORACLE_OK;
+    for (int64_t r = 0; r < n_rows && status == ORACLE_OK; ++r) {
+        const int64_t t = rows[r];
+        if (t < 0 || t >= T) { status = ORACLE_BAD_ARG; break; }
+        for (int64_t i = 0; i < d; ++i) xrow[i] = bf16_to_double(x[t * d + i]);
+        double* orow = out + r * d;
+        for (int64_t c = 0; c < d; ++c) orow[c] = 0.0;
+        for (int64_t j = 0; j < k; ++j) {
+            const int32_t e = ids[t * k + j];
+            if (e < 0 || e >= E) { status = ORACLE_BAD_ARG; break; }
+            expert_swiglu(xrow, w_gate + (int64_t)e * d * f, w_up + (int64_t)e * d * f,
+                          w_down + (int64_t)e * f * d, d, f, g, u, h, o);
+            const double wj = weights[t * k + j];
+            for (int64_t c = 0; c < d; ++c) {
+                const double yc = wj * o[c];
+                orow[c] += yc;
+                if (y_out) y_out[(r * k + j) * d + c] = yc;
+            }
+            if (h_out) memcpy(h_out + (r * k + j) * f, h, sizeof(double) * f);
+        }
+    }
+    free(xrow); free(g); free(u); free(h); free(o);
+    return status;
+}

@@ -1,0 +1,193 @@
+"""Python wrapper of the fp64 C oracle (``moe_oracle.c``).
+
+TEST INFRASTRUCTURE ONLY: the tests, the smoke check and the benchmark's
+CPU-baseline leg may import this module; the product path never does.
+
+The C source is compiled with plain ``gcc -O2`` (no fast-math, so every sum
+keeps its written order) into ``liboracle.so`` beside it, on first use or
+when the source changed.  Inputs are numpy arrays: bf16 tensors as uint16 bit
+patterns, the bias as float32.
+"""
+from __future__ import annotations
+
+import ctypes
+import hashlib
+import os
+import subprocess
+from dataclasses import dataclass
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "moe_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_STAMP = _LIB + ".srchash"
+
+
+def _source_hash(src: str) -> str:
+    with open(src, "rb") as fh:
+        return hashlib.sha256(fh.read()).hexdigest()
+
+
+def compile_oracle(src: str = _SRC, out: str = _LIB, extra_flags=(), force: bool = False) -> str:
+    """Compile an oracle source file to a shared library; returns its path."""
+    stamp = out + ".srchash"
+    h = _source_hash(src) + " " + " ".join(extra_flags)
+    if not force and os.path.exists(out) and os.path.exists(stamp):
+        with open(stamp) as fh:
+            if fh.read() == h:
+                return out
+    cmd = ["gcc", "-O2", "-std=c99", "-fPIC", "-shared", "-o", out, src, "-lm", *extra_flags]
+    subprocess.run(cmd, check=True)
+    with open(stamp, "w") as fh:
+        fh.write(h)
+    return out
+
+
+_P = ctypes.c_void_p
+_I64 = ctypes.c_int64
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+class Oracle:
+    """Handle on one compiled oracle library (the real one, or a test mutant)."""
+
+    def __init__(self, lib_path: str | None = None):
+        self.path = lib_path or compile_oracle()
+        lib = ctypes.CDLL(self.path)
+        lib.oracle_route.argtypes = [_P, _P, _P, _I64, _I64, _I64, _I64, _P, _P, _P, _P]
+        lib.oracle_permute.argtypes = [_P, _I64, _I64, _I64, _P, _P, _P, _P]
+        lib.oracle_expert_rows.argtypes = [_P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64,
+                                           _P, _P, _I64, _P, _P, _P, _P]
+        for fn in (lib.oracle_route, lib.oracle_permute, lib.oracle_expert_rows):
+            fn.restype = ctypes.c_int
+        self.lib = lib
+
+    # -- stage 1 + 2 ------------------------------------------------------
+    def route(self, x, w_router, bias, k, want_logits=False, want_probs=True):
+        x = np.ascontiguousarray(x, dtype=np.uint16)
+        w_router = np.ascontiguousarray(w_router, dtype=np.uint16)
+        T, d = x.shape
+        d2, E = w_router.shape
+        assert d == d2
+        b = None if bias is None else np.ascontiguousarray(bias, dtype=np.float32)
+        logits = np.empty((T, E), np.float64) if want_logits else None
+        probs = np.empty((T, E), np.float64) if want_probs else None
+        ids = np.empty((T, k), np.int32)
+        w = np.empty((T, k), np.float64)
+        rc = self.lib.oracle_route(_ptr(x), _ptr(w_router), _ptr(b), T, d, E, k,
+                                   _ptr(logits), _ptr(probs), _ptr(ids), _ptr(w))
+        if rc != 0:
+            raise ValueError(f"oracle_route failed ({rc})")
+        return RouteResult(ids=ids, weights=w, probs=probs, logits=logits)
+
+    # -- grouping -----------------------------------------------------------
+    def permute(self, ids, E):
+        ids = np.ascontiguousarray(ids, dtype=np.int32)
+        T, k = ids.shape
+        counts = np.empty(E, np.int32)
+        offsets = np.empty(E + 1, np.int32)
+        perm = np.empty(T * k, np.int32)
+        inv = np.empty(T * k, np.int32)
+        rc = self.lib.oracle_permute(_ptr(ids), T, E, k, _ptr(counts), _ptr(offsets),
+                                     _ptr(perm), _ptr(inv))
+        if rc != 0:
+            raise ValueError(f"oracle_permute failed ({rc})")
+        return PermuteResult(counts, offsets, perm, inv)
+
+    # -- stage 3 + 4 ----------------------------------------------------------
+    def expert_rows(self, x, w_gate, w_up, w_down, ids, weights, rows,
+                    want_y=False, want_h=False):
+        x = np.ascontiguousarray(x, dtype=np.uint16)
+        w_gate = np.ascontiguousarray(w_gate, dtype=np.uint16)
+        w_up = np.ascontiguousarray(w_up, dtype=np.uint16)
+        w_down = np.ascontiguousarray(w_down, dtype=np.uint16)
+        ids = np.ascontiguousarray(ids, dtype=np.int32)
+        weights = np.ascontiguousarray(weights, dtype=np.float64)
+        rows = np.ascontiguousarray(rows, dtype=np.int64)
+        T, d = x.shape
+        E, _, f = w_gate.shape
+        k = ids.shape[1]
+        n = rows.shape[0]
+        out = np.empty((n, d), np.float64)
+        y = np.empty((n, k, d), np.float64) if want_y else None
+        h = np.empty((n, k, f), np.float64) if want_h else None
+        rc = self.lib.oracle_expert_rows(_ptr(x), _ptr(w_gate), _ptr(w_up), _ptr(w_down),
+                                         T, d, E, k, f, _ptr(ids), _ptr(weights), n,
+                                         _ptr(rows), _ptr(out), _ptr(y), _ptr(h))
+        if rc != 0:
+            raise ValueError(f"oracle_expert_rows failed ({rc})")
+        return ExpertResult(out=out, y=y, h=h)
+
+    # -- whole block ----------------------------------------------------------
+    def forward(self, x, w_router, bias, w_gate, w_up, w_down, k, rows=None,
+                want_y=False, want_h=False):
+        """Route every token; evaluate the expert MLPs for ``rows`` (all if None)."""
+        r = self.route(x, w_router, bias, k)
+        if rows is None:
+            rows = np.arange(x.shape[0], dtype=np.int64)
+        ex = self.expert_rows(x, w_gate, w_up, w_down, r.ids, r.weights, rows,
+                              want_y=want_y, want_h=want_h)
+        return r, ex
+
+
+@dataclass
+class RouteResult:
+    ids: np.ndarray        # [T, k] int32
+    weights: np.ndarray    # [T, k] float64
+    probs: np.ndarray | None   # [T, E] float64
+    logits: np.ndarray | None  # [T, E] float64
+
+
+@dataclass
+class PermuteResult:
+    counts: np.ndarray     # [E]
+    offsets: np.ndarray    # [E+1]
+    perm: np.ndarray       # [T*k]
+    inv: np.ndarray        # [T*k]
+
+
+@dataclass
+class ExpertResult:
+    out: np.ndarray                # [n, d] float64
+    y: np.ndarray | None = None    # [n, k, d]
+    h: np.ndarray | None = None    # [n, k, f]
+
+
+def topk_gap(probs: np.ndarray, k: int) -> np.ndarray:
+    """p_(k) - p_(k+1) per token (inf when k == E): the near-tie margin."""
+    T, E = probs.shape
+    if k >= E:
+        return np.full(T, np.inf)
+    s = -np.sort(-probs, axis=1)
+    return s[:, k - 1] - s[:, k]
+
+
+def inner_gap(probs: np.ndarray, k: int) -> np.ndarray:
+    """Smallest gap between consecutive probabilities among the top k+... slots.
+
+    min over j < k-1 of p_(j) - p_(j+1): a near tie here may swap the order of
+    two selected slots without changing the selected set.
+    """
+    T, E = probs.shape
+    if k < 2:
+        return np.full(T, np.inf)
+    s = -np.sort(-probs, axis=1)[:, :k]
+    return np.min(s[:, :-1] - s[:, 1:], axis=1)
+
+
+_default: Oracle | None = None
+
+
+def default_oracle() -> Oracle:
+    global _default
+    if _default is None:
+        _default = Oracle()
+    return _default
+
+
+__all__ = ["Oracle", "compile_oracle", "default_oracle", "topk_gap", "inner_gap",
+           "RouteResult", "PermuteResult", "ExpertResult"]

@@ -1,0 +1,274 @@
+"""Checks that pin the fp64 oracle to computations other than itself.
+
+Each ``check_*`` function takes an ``Oracle`` handle and raises
+AssertionError on a mismatch.  test_oracle_pins.py runs them on the real
+oracle; test_oracle_mutants.py runs them on copies of the oracle with a
+planted mistake and requires that at least one check fails for every mutant.
+
+The independent computations used here:
+  * a dense brute force: every expert evaluated for every token with numpy
+    matmuls, masked by a one-hot of the top-k chosen by numpy's lexsort over
+    scipy's softmax, weighted and summed -- a different algorithm from the
+    oracle's sparse per-token loop;
+  * library routines for single steps: numpy matmul, scipy.special.softmax,
+    scipy.special.expit (for silu(z) = z * expit(z)), numpy's stable argsort;
+  * special cases with closed forms: E = 1, k = 1 is a dense SwiGLU MLP;
+    k = E with identical experts is that MLP times sum(p) = 1; exact ties;
+  * invariants: counts sum to T*k, the permutation is a bijection, etc.
+"""
+from __future__ import annotations
+
+import numpy as np
+import scipy.special as sps
+import torch
+
+from top_routing_grouped_softmax_b200.synth import bf16_bits, make_inputs
+
+
+def widen(bits: np.ndarray) -> np.ndarray:
+    """bf16 bit patterns -> float64, exactly."""
+    return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def _rand_case(T, d, E, k, f, seed, bias=False, sigma=0.05):
+    from top_routing_grouped_softmax_b200.synth import MoEConfig
+    cfg = MoEConfig("pin", T=T, d=d, E=E, k=k, f=f, sigma=sigma, seed=seed, skew=bias)
+    return make_inputs(cfg)
+
+
+def _args(inp):
+    return (inp.bits("x"), inp.bits("W_router"), inp.bias_np(), inp.bits("W_gate"),
+            inp.bits("W_up"), inp.bits("W_down"))
+
+
+def dense_reference(x, wr, bias, wg, wu, wd, k):
+    """Brute force: evaluate all E experts densely, mask with one-hot top-k."""
+    X, Wr = widen(x), widen(wr)
+    Wg, Wu, Wd = widen(wg), widen(wu), widen(wd)
+    T = X.shape[0]
+    E = Wr.shape[1]
+    logits = X @ Wr
+    if bias is not None:
+        logits = logits + bias.astype(np.float64)[None, :]
+    p = sps.softmax(logits, axis=1)
+    idx = np.broadcast_to(np.arange(E), (T, E))
+    order = np.lexsort((idx, -p), axis=1)       # primary -p, then index
+    top = order[:, :k]
+    mask = np.zeros((T, E))
+    np.put_along_axis(mask, top, 1.0, axis=1)
+    out = np.zeros((T, X.shape[1]))
+    for e in range(E):
+        G = X @ Wg[e]
+        U = X @ Wu[e]
+        H = G * sps.expit(G) * U
+        out += (mask[:, e] * p[:, e])[:, None] * (H @ Wd[e])
+    return out, p, top, logits
+
+
+def _rel(a, b):
+    scale = max(np.sqrt(np.mean(b * b)), 1e-300)
+    return float(np.max(np.abs(a - b)) / scale)
+
+
+# ---------------------------------------------------------------------------
+def check_brute_force(o):
+    for (T, d, E, k, f, seed, bias) in [(48, 64, 8, 2, 32, 11, False), (33, 32, 5, 3, 48, 12, True),
+                                        (64, 96, 8, 1, 64, 13, False), (17, 64, 4, 4, 16, 14, True)]:
+        inp = _rand_case(T, d, E, k, f, seed, bias=bias)
+        r, ex = o.forward(*_args(inp), k)
+        ref, p, top, _ = dense_reference(*_args(inp), k)
+        assert _rel(ex.out, ref) < 1e-10, ("brute force", T, d, E, k, f)
+        assert np.array_equal(r.ids, top), "top-k ids differ from lexsort"
+
+
+def check_softmax_library(o):
+    inp = _rand_case(40, 64, 16, 4, 16, 21, bias=True, sigma=0.3)
+    r = o.route(inp.bits("x"), inp.bits("W_router"), inp.bias_np(), 4, want_logits=True)
+    logits = widen(inp.bits("x")) @ widen(inp.bits("W_router")) + inp.bias_np().astype(np.float64)
+    assert np.allclose(r.logits, logits, rtol=1e-12, atol=1e-12), "logits != x @ Wr + b"
+    assert np.allclose(r.probs, sps.softmax(logits, axis=1), rtol=1e-12, atol=1e-15), "softmax"
+    assert np.allclose(r.probs.sum(axis=1), 1.0, atol=1e-14)
+
+
+def check_topk_library_sort(o):
+    inp = _rand_case(64, 64, 32, 6, 16, 22, sigma=0.2)
+    r = o.route(inp.bits("x"), inp.bits("W_router"), None, 6)
+    p = r.probs
+    T, E = p.shape
+    order = np.lexsort((np.broadcast_to(np.arange(E), (T, E)), -p), axis=1)[:, :6]
+    assert np.array_equal(r.ids, order), "top-k ids"
+    assert np.array_equal(r.weights, np.take_along_axis(p, r.ids.astype(np.int64), 1)), \
+        "weights are not the softmax entries at the selected ids (renormalised?)"
+    assert np.all(np.diff(r.weights, axis=1) <= 0), "slots not in descending probability"
+    for t in range(T):
+        assert len(set(r.ids[t].tolist())) == 6, "duplicate expert in one token"
+
+
+def check_topk_of_logits(o):
+    """Softmax is monotone: top-k of the logits picks the same experts."""
+    inp = _rand_case(64, 64, 16, 3, 16, 23, bias=True, sigma=0.2)
+    r = o.route(inp.bits("x"), inp.bits("W_router"), inp.bias_np(), 3, want_logits=True)
+    T, E = r.logits.shape
+    order = np.lexsort((np.broadcast_to(np.arange(E), (T, E)), -r.logits), axis=1)[:, :3]
+    assert np.array_equal(np.sort(r.ids, 1), np.sort(order, 1)), "topk(logits) != topk(p)"
+
+
+def check_exact_ties(o):
+    """All router columns identical: p = 1/E exactly, ids are 0..k-1."""
+    inp = _rand_case(16, 32, 8, 3, 16, 24)
+    wr = inp.bits("W_router").copy()
+    wr[:, :] = wr[:, :1]
+    r = o.route(inp.bits("x"), wr, None, 3)
+    assert np.all(r.ids == np.arange(3)[None, :]), "tie-break is not lowest index first"
+    assert np.all(r.weights == 0.125), "equal logits must give p = 1/E"
+    # a two-way tie at the top: columns 5 and 2 equal and largest
+    wr = np.zeros((32, 8), np.uint16)
+    one = np.uint16(0x3F80)       # bf16 1.0
+    half = np.uint16(0x3F00)      # bf16 0.5
+    wr[0, 5] = one
+    wr[0, 2] = one
+    wr[0, 7] = half
+    xb = np.zeros((4, 32), np.uint16)
+    xb[:, 0] = one
+    r = o.route(xb, wr, None, 3)
+    assert np.all(r.ids == np.array([2, 5, 7])[None, :]), r.ids
+
+
+def check_dense_special_case(o):
+    """E = 1, k = 1: p = 1 exactly and the block is one dense SwiGLU MLP."""
+    inp = _rand_case(24, 64, 1, 1, 96, 25)
+    r, ex = o.forward(*_args(inp), 1)
+    assert np.all(r.ids == 0) and np.all(r.weights == 1.0)
+    X = widen(inp.bits("x"))
+    G = X @ widen(inp.bits("W_gate"))[0]
+    U = X @ widen(inp.bits("W_up"))[0]
+    ref = (G * sps.expit(G) * U) @ widen(inp.bits("W_down"))[0]
+    assert _rel(ex.out, ref) < 1e-12, "E=1,k=1 != dense SwiGLU"
+
+
+def check_all_experts_identical(o):
+    """k = E with every expert identical: out = MLP(x) * sum_e p_e = MLP(x)."""
+    inp = _rand_case(20, 32, 4, 4, 48, 26)
+    wg, wu, wd = inp.bits("W_gate").copy(), inp.bits("W_up").copy(), inp.bits("W_down").copy()
+    wg[:] = wg[0]
+    wu[:] = wu[0]
+    wd[:] = wd[0]
+    r, ex = o.forward(inp.bits("x"), inp.bits("W_router"), None, wg, wu, wd, 4)
+    X = widen(inp.bits("x"))
+    G = X @ widen(wg[0])
+    U = X @ widen(wu[0])
+    ref = (G * sps.expit(G) * U) @ widen(wd[0])
+    assert _rel(ex.out, ref) < 1e-12, "k=E identical experts != MLP(x)"
+
+
+def check_zero_expert(o):
+    """An expert with W_down = 0 contributes nothing; unselected experts are inert."""
+    inp = _rand_case(40, 64, 8, 2, 32, 27)
+    x, wr, _, wg, wu, wd = _args(inp)
+    r, ex = o.forward(x, wr, None, wg, wu, wd, 2)
+    wd0 = wd.copy()
+    wd0[3] = 0
+    r0, ex0 = o.forward(x, wr, None, wg, wu, wd0, 2)
+    ref, p, top, _ = dense_reference(x, wr, None, wg, wu, wd, 2)
+    # remove expert 3's term from the brute force
+    X = widen(x)
+    G = X @ widen(wg[3])
+    U = X @ widen(wu[3])
+    term = ((top == 3).any(axis=1) * p[:, 3])[:, None] * ((G * sps.expit(G) * U) @ widen(wd[3]))
+    assert _rel(ex0.out, ref - term) < 1e-10, "zeroed expert still contributes"
+    # change the weights of an expert that no token selects: bit-identical out
+    # a strongly negative bias keeps expert 6 out of every token's top-k
+    bias = np.zeros(8, np.float32)
+    bias[6] = -1.0e4
+    r, ex = o.forward(x, wr, bias, wg, wu, wd, 2)
+    assert 6 not in set(r.ids.ravel().tolist())
+    e = 6
+    wg2, wu2, wd2 = wg.copy(), wu.copy(), wd.copy()
+    wg2[e] = wg2[(e + 1) % 8]
+    wu2[e] = 0
+    wd2[e] = wd2[(e + 2) % 8]
+    _, ex2 = o.forward(x, wr, bias, wg2, wu2, wd2, 2)
+    assert np.array_equal(ex2.out, ex.out), "unselected expert changed the output"
+
+
+def check_scale_down(o):
+    """Doubling W_down (exact in bf16) doubles the output exactly."""
+    inp = _rand_case(16, 64, 8, 2, 32, 28)
+    x, wr, _, wg, wu, wd = _args(inp)
+    _, ex = o.forward(x, wr, None, wg, wu, wd, 2)
+    wd2 = bf16_bits(torch.from_numpy(widen(wd).astype(np.float32) * 2).to(torch.bfloat16))
+    _, ex2 = o.forward(x, wr, None, wg, wu, wd2, 2)
+    assert np.array_equal(ex2.out, 2.0 * ex.out), "2*W_down did not double out"
+
+
+def check_permute_library(o):
+    """Grouping equals numpy's stable argsort of the flat expert ids."""
+    rng = np.random.default_rng(5)
+    for (T, E, k) in [(100, 8, 2), (257, 16, 4), (1, 4, 4), (64, 32, 1)]:
+        ids = np.stack([rng.permutation(E)[:k] for _ in range(T)]).astype(np.int32)
+        pr = o.permute(ids, E)
+        flat = ids.ravel()
+        assert np.array_equal(pr.counts, np.bincount(flat, minlength=E))
+        assert pr.offsets[0] == 0 and pr.offsets[-1] == T * k
+        assert np.all(np.diff(pr.offsets) >= 0)
+        assert np.array_equal(pr.perm, np.argsort(flat, kind="stable")), "not a stable grouping"
+        assert np.array_equal(np.sort(pr.perm), np.arange(T * k)), "perm not a bijection"
+        assert np.array_equal(pr.inv[pr.perm], np.arange(T * k)), "inv o perm != id"
+        for e in range(E):
+            seg = pr.perm[pr.offsets[e]:pr.offsets[e + 1]]
+            assert np.all(flat[seg] == e)
+
+
+def check_page_listing_torch(o):
+    """The article's forward() rendered in PyTorch fp64 on the CPU.
+
+    Structure as printed (router linear, softmax over dim 1, topk, one-hot
+    expert mask permuted to [E, k, T], a loop over experts with where / gather
+    / expert / index_add_) plus the multiply by the routing weight that the
+    article's stage 4 requires.  Random inputs, no ties.
+    """
+    inp = _rand_case(37, 64, 8, 2, 48, 29, bias=True)
+    x, wr, b, wg, wu, wd = _args(inp)
+    _, ex = o.forward(x, wr, b, wg, wu, wd, 2)
+    hs = torch.from_numpy(widen(x))
+    Wr = torch.from_numpy(widen(wr))
+    Wg, Wu, Wd = (torch.from_numpy(widen(a)) for a in (wg, wu, wd))
+    router_logits = hs @ Wr + torch.from_numpy(b.astype(np.float64))
+    routing_weights = torch.softmax(router_logits, dim=1)
+    routing_weights, selected = torch.topk(routing_weights, 2)
+    mask = torch.nn.functional.one_hot(selected, num_classes=8).permute(2, 1, 0)
+    final = torch.zeros_like(hs)
+    for e in range(8):
+        idx, top_x = torch.where(mask[e])
+        cur = hs[top_x]
+        g = cur @ Wg[e]
+        h = torch.nn.functional.silu(g) * (cur @ Wu[e])
+        cur_out = (h @ Wd[e]) * routing_weights[top_x, idx, None]
+        final.index_add_(0, top_x, cur_out)
+    assert _rel(ex.out, final.numpy()) < 1e-10, "page forward (torch) != oracle"
+
+
+def check_expert_rows_outputs(o):
+    """y and h side outputs agree with the dense pieces for each slot."""
+    inp = _rand_case(12, 32, 4, 2, 40, 30)
+    x, wr, _, wg, wu, wd = _args(inp)
+    r = o.route(x, wr, None, 2)
+    rows = np.array([0, 5, 11])
+    ex = o.expert_rows(x, wg, wu, wd, r.ids, r.weights, rows, want_y=True, want_h=True)
+    X = widen(x)
+    for i, t in enumerate(rows):
+        for j in range(2):
+            e = r.ids[t, j]
+            g = X[t] @ widen(wg[e])
+            u = X[t] @ widen(wu[e])
+            h = g * sps.expit(g) * u
+            assert np.allclose(ex.h[i, j], h, rtol=1e-12, atol=1e-14)
+            assert np.allclose(ex.y[i, j], r.weights[t, j] * (h @ widen(wd[e])), rtol=1e-12, atol=1e-15)
+        assert np.allclose(ex.out[i], ex.y[i].sum(axis=0), rtol=1e-13, atol=1e-15)
+
+
+ALL_CHECKS = [
+    check_brute_force, check_softmax_library, check_topk_library_sort, check_topk_of_logits,
+    check_exact_ties, check_dense_special_case, check_all_experts_identical, check_zero_expert,
+    check_scale_down, check_permute_library, check_page_listing_torch, check_expert_rows_outputs,
+]

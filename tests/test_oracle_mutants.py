@@ -1,0 +1,48 @@
+"""Plant one mistake at a time in a copy of the oracle source and require the
+pin suite to catch every one of them.  The mutants are compiled on the CPU
+and never touch a GPU."""
+import os
+
+import pytest
+
+from oracle.oracle import Oracle, compile_oracle
+from tests import oracle_pins
+
+SRC = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+                   "oracle", "moe_oracle.c")
+
+# (name, exact source text, replacement): each a plausible slip.
+MUTANTS = [
+    ("drop_bias", "logit[e] += (double)bias[e];", "logit[e] += 0.0 * (double)bias[e];"),
+    ("no_routing_weight", "const double yc = wj * o[c];", "const double yc = o[c];"),
+    ("silu_sign", "h[n] = g[n] / (1.0 + exp(-g[n])) * u[n];", "h[n] = g[n] / (1.0 + exp(g[n])) * u[n];"),
+    ("renormalise", "weights[t * k + j] = ranked[j].p;",
+     "weights[t * k + j] = ranked[j].p / (ranked[0].p + ranked[k - 1].p);"),
+    ("transposed_down", "o[c] += hn * bf16_to_double(drow[c]);", "o[c] += hn * bf16_to_double(wd[c * f + n]);"),
+    ("tie_highest_index", "return (ra->e > rb->e) - (ra->e < rb->e);", "return (ra->e < rb->e) - (ra->e > rb->e);"),
+    ("reverse_group_order", "for (int64_t a = 0; a < n; ++a) {\n        int32_t pos",
+     "for (int64_t a = n - 1; a >= 0; --a) {\n        int32_t pos"),
+    ("up_uses_gate", "u[n] += xi * bf16_to_double(urow[n]);", "u[n] += xi * bf16_to_double(grow[n]);"),
+    ("dropped_last_hidden_term", "for (int64_t i = 0; i < d; ++i) {\n            double xi",
+     "for (int64_t i = 0; i < d - 1; ++i) {\n            double xi"),
+    ("softmax_no_norm", "for (int64_t e = 0; e < E; ++e) prob[e] /= s;", "for (int64_t e = 0; e < E; ++e) prob[e] /= 1.0;"),
+    ("weights_from_wrong_slot", "weights[t * k + j] = ranked[j].p;", "weights[t * k + j] = ranked[0].p;"),
+    ("sum_only_first_slot", "orow[c] += yc;", "orow[c] += (j == 0) ? yc : 0.0;"),
+]
+
+
+@pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_pins_catch_mutant(tmp_path, name, old, new):
+    src = open(SRC).read()
+    assert src.count(old) == 1, f"mutation site for {name} not found exactly once"
+    mut_src = tmp_path / f"mut_{name}.c"
+    mut_src.write_text(src.replace(old, new))
+    lib = compile_oracle(str(mut_src), str(tmp_path / f"lib_{name}.so"), force=True)
+    o = Oracle(lib)
+    failed = []
+    for check in oracle_pins.ALL_CHECKS:
+        try:
+            check(o)
+        except AssertionError:
+            failed.append(check.__name__)
+    assert failed, f"no pin caught mutant {name}"
