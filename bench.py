@@ -1,0 +1,371 @@
+"""Benchmark of the sparse-MoE block forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload qwen]
+    python bench.py --impl reference ...      # the fp64 CPU oracle, timed
+
+One step = one moe_forward (router GEMM + softmax + top-k, permutation,
+grouped gate/up + SwiGLU GEMM, grouped down GEMM + routing weight, combine)
+over one batch of T tokens of the named workload, with every input already
+resident in HBM.  L2 is flushed (a 256 MiB write) between timed steps, and
+each step is timed with CUDA events on the launching stream; the stage
+boundaries inside a step are timed with events the library records on the
+same stream.  `e2e` repeats the measurement through the public API with the
+token batch copied host->device from pinned memory and the output copied
+back inside the timed region.
+
+Multi-GPU: one process per GPU (torchrun); every rank runs its own replica
+on its own batch (the block is independent per token, so the path shards by
+tokens with no data-path collective: weak scaling).  Ranks meet at a barrier
+before and after the timed region and the slowest rank's time is used.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "MoE-layer fwd tokens/s & grouped-GEMM TFLOP/s vs roofline, 1×B200"
+UNIT = "tokens/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 << 20
+STAGES = ("route", "permute", "gateup_gemm", "down_gemm", "combine")
+
+
+# ------------------------------------------------------------- host logic
+def dist_env():
+    """(rank, local_rank, world) from the torchrun environment (1 process if unset)."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", str(rank)))
+    return rank, local, world
+
+
+def replica_seed(base_seed: int, rank: int) -> int:
+    """Each rank draws its own token batch (weights use the same recipe)."""
+    return base_seed + 1000 * rank
+
+
+def whole_job_rate(units_per_rank: float, world: int, seconds_per_rank) -> float:
+    """Aggregate throughput: all ranks' units over the slowest rank's time."""
+    return units_per_rank * world / max(seconds_per_rank)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as fh:
+            p = json.load(fh)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "measured"}
+    return dict(FALLBACK_PEAKS, source="fallback")
+
+
+def algorithmic(cfg, active_experts=None):
+    """FLOPs and compulsory HBM bytes of one forward, and of its gate/up GEMM."""
+    T, d, E, k, f = cfg.T, cfg.d, cfg.E, cfg.k, cfg.f
+    flops = 2 * T * (d * E + 3 * k * d * f)
+    gateup_flops = 2 * T * k * d * 2 * f
+    down_flops = 2 * T * k * f * d
+    nact = E if active_experts is None else active_experts
+    # x read + out write (fp32) + router weights + weights of the experts in use
+    compulsory = T * d * 2 + T * d * 4 + d * E * 2 + nact * 3 * d * f * 2
+    return {"flops": flops, "gateup_flops": gateup_flops, "down_flops": down_flops, "bytes": compulsory}
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100",
+                 "-i", str(self.dev)], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        if self.path and os.path.exists(self.path):
+            for line in open(self.path):
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append((float(parts[1]), float(parts[2]), float(parts[3]), parts[5:9]))
+                except ValueError:
+                    continue
+            os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        reasons = sorted({names[i] for r in rows for i, v in enumerate(r[3]) if v.lower() == "active"})
+        loaded = [r for r in rows if r[2] > 250.0] or rows
+        return {"sm_mhz": statistics.median(r[0] for r in loaded), "sm_max_mhz": max(r[1] for r in rows),
+                "power_w_max": max(r[2] for r in rows), "samples": len(rows), "reasons": reasons}
+
+
+# ------------------------------------------------------------ CPU oracle
+def time_oracle(cfg, n_tokens: int, seed: int, inp=None):
+    """Run the fp64 oracle (single thread) on the first n_tokens of the workload.
+
+    Returns (seconds, n_tokens).  Same recipe, same shapes; only the token
+    count is bounded so the CPU leg takes seconds, not hours.
+    """
+    import numpy as np
+    from oracle.oracle import default_oracle
+    from top_routing_grouped_softmax_b200.synth import make_inputs
+
+    if inp is None:
+        inp = make_inputs(cfg.with_(seed=seed))
+    o = default_oracle()
+    x = inp.bits("x")[:n_tokens]
+    t0 = time.perf_counter()
+    r = o.route(x, inp.bits("W_router"), inp.bias_np(), cfg.k)
+    o.permute(r.ids, cfg.E)
+    o.expert_rows(x, inp.bits("W_gate"), inp.bits("W_up"), inp.bits("W_down"), r.ids, r.weights,
+                  np.arange(n_tokens, dtype=np.int64))
+    return time.perf_counter() - t0, n_tokens
+
+
+def cpu_baseline(cfg, n_tokens: int, seed: int, inp=None):
+    secs, n = time_oracle(cfg, n_tokens, seed, inp)
+    return {"value": n / secs, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"first {n} of {cfg.T} tokens of the {cfg.name} workload, full block "
+                      f"(route, permute, expert MLPs, combine), fp64, one thread"}
+
+
+# ------------------------------------------------------------- reference
+def run_reference(args, cfg):
+    rank, _, world = dist_env()
+    if rank != 0:
+        return 0
+    from top_routing_grouped_softmax_b200.synth import make_inputs
+    inp = make_inputs(cfg.with_(seed=replica_seed(cfg.seed, 0)))
+    n = args.ref_tokens
+    for _ in range(args.warmup):
+        time_oracle(cfg, n, cfg.seed, inp)
+    secs = [time_oracle(cfg, n, cfg.seed, inp)[0] for _ in range(args.steps)]
+    total = sum(secs)
+    value = n * args.steps / total
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": workload_config(cfg, extra={"tokens_per_step": n}),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": f"first {n} of {cfg.T} tokens per step, full block, fp64, one thread"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(cfg, extra=None):
+    c = {"workload": cfg.name, "T": cfg.T, "d": cfg.d, "E": cfg.E, "k": cfg.k, "f": cfg.f,
+         "router_bias": "zipf" if cfg.skew else None, "weights_sigma": cfg.sigma,
+         "inputs": "seeded synthetic (x ~ N(0,1), weights ~ N(0, sigma^2), bf16)",
+         "l2": "flushed between timed steps (256 MiB write)", "parallelism": "replicas"}
+    if extra:
+        c.update(extra)
+    return c
+
+
+# ------------------------------------------------------------------- GPU
+def run_gpu(args, cfg):
+    import torch
+    import torch.distributed as dist
+
+    import top_routing_grouped_softmax_b200 as moe
+    from top_routing_grouped_softmax_b200.synth import make_inputs
+
+    rank, local, world = dist_env()
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+
+    inp = make_inputs(cfg.with_(seed=replica_seed(cfg.seed, rank)))
+    x = inp.x.to(dev)
+    w = {n: getattr(inp, n).to(dev) for n in ("W_router", "W_gate", "W_up", "W_down")}
+    bias = None if inp.bias is None else inp.bias.to(dev)
+    blk = moe.MoEBlock(w["W_router"], w["W_gate"], w["W_up"], w["W_down"], cfg.k, bias=bias)
+    out = torch.empty(cfg.T, cfg.d, dtype=torch.float32, device=dev)
+    ids = torch.empty(cfg.T, cfg.k, dtype=torch.int32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(events=None):
+        blk(x, out=out, topk_ids=ids, events=events)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert moe.get_status() == moe.MOE_OK
+
+    n_ev = 6
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        wall0 = time.perf_counter()
+        for i in range(args.steps):
+            flush.zero_()
+            step(evs[i])
+        torch.cuda.synchronize()
+        wall = time.perf_counter() - wall0
+    if world > 1:
+        dist.barrier()
+    status = moe.get_status()
+    assert status == moe.MOE_OK, moe.strerror(status)
+    clocks = clk.summary()
+
+    step_ms = [e[0].elapsed_time(e[n_ev - 1]) for e in evs]
+    stage_ms = {s: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs) for i, s in enumerate(STAGES)}
+    total_s = sum(step_ms) / 1e3
+
+    # expert load statistics of the batch
+    counts = torch.bincount(ids.flatten().long(), minlength=cfg.E).cpu()
+    active = int((counts > 0).sum())
+    tiles = int(((counts + 127) // 128).sum())
+    padding = 1.0 - cfg.T * cfg.k / (tiles * 128)
+
+    # ---- end to end through the public API, host buffers, copies timed
+    x_host = inp.x.pin_memory()
+    out_host = torch.empty(cfg.T, cfg.d, dtype=torch.float32).pin_memory()
+    x_dev = torch.empty_like(x)
+    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for _ in range(2):
+        x_dev.copy_(x_host, non_blocking=True)
+        blk(x_dev, out=out)
+        out_host.copy_(out, non_blocking=True)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    for i in range(args.steps):
+        flush.zero_()
+        e2e_ev[i][0].record(stream)
+        x_dev.copy_(x_host, non_blocking=True)
+        blk(x_dev, out=out)
+        out_host.copy_(out, non_blocking=True)
+        e2e_ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    e2e_s = sum(a.elapsed_time(b) for a, b in e2e_ev) / 1e3
+    if world > 1:
+        dist.barrier()
+
+    # max over ranks
+    if world > 1:
+        t = torch.tensor([total_s, e2e_s, stage_ms["gateup_gemm"]], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_s, e2e_s, gateup_ms_max = t.tolist()
+    else:
+        gateup_ms_max = stage_ms["gateup_gemm"]
+
+    result = None
+    if rank == 0:
+        peaks = load_peaks()
+        alg = algorithmic(cfg, active)
+        ms = 1e3 * total_s / args.steps
+        tok_s = whole_job_rate(cfg.T * args.steps, world, [total_s])
+        achieved = alg["gateup_flops"] / (gateup_ms_max * 1e-3) / 1e12
+        roof_time = max(alg["flops"] / (peaks["bf16_tflops"] * 1e12), alg["bytes"] / (peaks["hbm_gbs"] * 1e9))
+        traffic = None
+        tpath = os.path.join(ROOT, "profiles", "gateup_traffic.json")
+        if os.path.exists(tpath):
+            with open(tpath) as fh:
+                tr = json.load(fh)
+            from top_routing_grouped_softmax_b200 import _build
+            if tr.get("source_hash") == _build.kernel_hash() and tr.get("workload") == cfg.name:
+                traffic = tr.get("dram_bytes_per_launch")
+        result = {
+            "metric": METRIC, "value": tok_s, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": workload_config(cfg, extra={"out_dtype": "fp32"}),
+            "tflops": alg["flops"] / (ms * 1e-3) / 1e12,
+            "grouped_gemm_tflops": (alg["gateup_flops"] + alg["down_flops"]) /
+                                   ((stage_ms["gateup_gemm"] + stage_ms["down_gemm"]) * 1e-3) / 1e12,
+            "roofline": {"bound": "tensor", "kernel": "grouped_gemm_kernel<SwiGLU> (gate/up + SwiGLU)",
+                         "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": achieved / peaks["bf16_tflops"], "traffic": traffic,
+                         "peak_source": f"{peaks['source']} burst bf16"},
+            "forward_roofline": {"roofline_ms": roof_time * 1e3, "frac": roof_time / (ms * 1e-3),
+                                 "flops": alg["flops"], "compulsory_bytes": alg["bytes"]},
+            "stage_ms": stage_ms,
+            "experts": {"active": active, "max_count": int(counts.max()), "min_count": int(counts.min()),
+                        "tile_padding": padding},
+            "e2e": {"value": whole_job_rate(cfg.T * args.steps, world, [e2e_s]), "unit": UNIT,
+                    "h2d_bytes_per_step": cfg.T * cfg.d * 2, "d2h_bytes_per_step": cfg.T * cfg.d * 4},
+            "gpu_launches": 8 * args.steps,
+            "clocks": clocks,
+            "wall_s_timed_region": wall,
+        }
+    if world > 1:
+        dist.destroy_process_group()
+    return result
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", default="qwen")
+    ap.add_argument("--cpu-tokens", type=int, default=384,
+                    help="tokens of the workload the CPU-oracle baseline leg evaluates")
+    ap.add_argument("--ref-tokens", type=int, default=32, help="tokens per step of the reference arm")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+
+    from top_routing_grouped_softmax_b200.synth import CONFIGS
+    cfg = CONFIGS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, cfg)
+
+    from top_routing_grouped_softmax_b200 import _build
+    _build.build_library()
+    res = run_gpu(args, cfg)
+    rank, _, world = dist_env()
+    if rank == 0 and res is not None:
+        if world == 1 and not args.no_cpu_baseline:
+            res["cpu_baseline"] = cpu_baseline(cfg, args.cpu_tokens, replica_seed(cfg.seed, 0))
+        print(json.dumps(res), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

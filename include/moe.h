@@ -1,0 +1,214 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) sparse Mixture-of-Experts block forward.
+ *
+ * The operation is the forward pass of a top-k routed MoE block as defined by
+ * the article "Qwen3MoeSparseMoeBlock performance optimisation in practice"
+ * (parallelising a sparse mixture-of-experts system), section 1: the forward()
+ * listing and the four-stage workflow above it (router linear + softmax,
+ * top-k selection, per-expert computation, routing-weighted aggregation),
+ * restaged in its section 2.2 as route -> sort tokens by expert -> batched
+ * expert compute -> scatter back.  Notation: T tokens, d hidden size, E
+ * experts, k experts per token, f expert intermediate size, M = T*k
+ * token-expert assignments.
+ *
+ *   logits[t,e] = sum_i x[t,i] * W_router[i,e] + bias[e]     (fp32)
+ *   p[t,:]      = softmax over e of logits[t,:]                (fp32)
+ *   ids[t,:]    = the k experts with the largest p, in descending order;
+ *                 equal values rank the lower expert index first
+ *   w[t,j]      = p[t, ids[t,j]]                      (NOT renormalised)
+ *   h           = silu(x[t] . W_gate[e]) * (x[t] . W_up[e]),  silu(z) = z/(1+e^-z)
+ *   y[t,j]      = w[t,j] * (h . W_down[e]),  e = ids[t,j]      (fp32)
+ *   out[t]      = sum_j y[t,j]                                  (fp32)
+ * Precision: bf16 inputs, fp32 accumulation everywhere.  h is rounded to
+ * bf16 once, because it is the operand of the second bf16 tensor-core GEMM;
+ * y and out are never rounded below fp32.
+ * The optional per-expert bias follows the gate G(x) = Softmax(W_g x + b_g)
+ * of the Hunyuan-Large overview page, section 2.1.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Pointers named x, w_*, h, x_perm are DEVICE pointers to bf16 (IEEE
+ *   bfloat16 bit patterns, type moe_bf16); y and out are DEVICE pointers to
+ *   fp32.  All are row-major, contiguous and 16-byte aligned.  Other int32 /
+ *   fp32 arrays are device pointers, 4-byte aligned.
+ *   The caller owns every buffer; the library never allocates, frees or
+ *   synchronises (except moe_get_status), in line with the article's
+ *   "memory pre-allocation" point (section 2.1, point 3).
+ * - Work is enqueued on `stream` and runs asynchronously; a return value of
+ *   MOE_OK means the arguments were valid and every launch was accepted.
+ * - Errors detected on the device (an expert id out of range, corrupt group
+ *   offsets, a pipeline wait that ran past its time limit) are written to a
+ *   per-device status word and reported by moe_get_status.  The kernel that
+ *   detects one skips the offending access and finishes without faulting.
+ * - Shapes (MOE_ERR_UNSUPPORTED_SHAPE otherwise):
+ *     d % 64 == 0 and 64 <= d <= 32768;  f % 64 == 0 and 64 <= f <= 65536;
+ *     E % 8 == 0 and 8 <= E <= 512;  1 <= k <= min(E, 32);
+ *     0 <= T and T*k < 2^31.  T == 0 is a valid no-op.
+ * - The device must be compute capability 10.0 (B200); the library carries
+ *   sm_100a code only (MOE_ERR_UNSUPPORTED_DEVICE otherwise).
+ */
+#ifndef MOE_H_
+#define MOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* IEEE bfloat16 bit pattern. */
+typedef uint16_t moe_bf16;
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1,         /* null / misaligned pointer, negative size */
+    MOE_ERR_UNSUPPORTED_SHAPE = 2,   /* shape outside the limits listed above */
+    MOE_ERR_WORKSPACE_TOO_SMALL = 3, /* workspace_bytes below the *_workspace_size value */
+    MOE_ERR_CUDA = 4,                /* a CUDA runtime call or a launch failed */
+    MOE_ERR_DEVICE_TIMEOUT = 5,      /* device: a pipeline wait ran past its limit */
+    MOE_ERR_DEVICE_BOUNDS = 6,       /* device: index data out of range (ids, offsets, inv) */
+    MOE_ERR_UNSUPPORTED_DEVICE = 7   /* not a compute-capability 10.0 GPU */
+} moe_status_t;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* moe_strerror(int status);
+
+/* ABI version of this header (major * 100 + minor). */
+int moe_version(void);
+
+/*
+ * Bytes of scratch that moe_forward needs for these sizes (0 if the shape is
+ * unsupported).  The pieces, each 256-byte aligned, are: topk ids and
+ * weights [M], counts [E], offsets [E+1], per-chunk group bases, perm / inv /
+ * w_perm [M], x_perm [M,d] bf16, h [M,f] bf16 and y [M,d] fp32.
+ */
+size_t moe_workspace_size(int64_t T, int64_t d, int64_t E, int64_t k, int64_t f);
+
+/* Bytes of scratch that moe_permute needs (per-chunk group bases). */
+size_t moe_permute_workspace_size(int64_t T, int64_t E, int64_t k);
+
+/*
+ * Stage 1-2: router GEMM, fp32 softmax over E, top-k (section 1 listing:
+ * gate linear, softmax over dim 1, topk; no renormalisation follows).
+ *   x        [T, d]    bf16
+ *   w_router [d, E]    bf16
+ *   bias     [E]       fp32, or NULL for no bias
+ *   topk_ids [T, k]    int32 out, slot j = j-th largest probability
+ *   topk_w   [T, k]    fp32  out, the softmax probability of that expert
+ * Logits are accumulated in fp32 on the tensor cores and never rounded to
+ * bf16.  Selection compares the fp32 logits (softmax is monotone); ties go
+ * to the lower expert index.
+ */
+int moe_route(const moe_bf16* x, const moe_bf16* w_router, const float* bias,
+              int64_t T, int64_t d, int64_t E, int64_t k,
+              int32_t* topk_ids, float* topk_w, cudaStream_t stream);
+
+/*
+ * Token reordering by expert (section 2.2: sort_tokens_by_expert, then
+ * gather hidden states and routing weights in that order).
+ *   topk_ids [T, k] int32 in (each in [0, E); otherwise MOE_ERR_DEVICE_BOUNDS
+ *                   is reported and those assignments are skipped)
+ *   topk_w   [T, k] fp32 in
+ *   counts   [E]    int32 out: assignments per expert
+ *   offsets  [E+1]  int32 out: exclusive prefix sum, offsets[E] = T*k
+ *   perm     [T*k]  int32 out: perm[pos] = t*k + j (grouped row -> assignment)
+ *   inv      [T*k]  int32 out: inv[t*k + j] = pos
+ *   x_perm   [T*k, d] bf16 out: x_perm[pos] = x[perm[pos] / k]; may be NULL
+ *                   to skip the row gather
+ *   w_perm   [T*k]  fp32 out: w_perm[pos] = topk_w[perm[pos]]
+ *   workspace       device scratch of moe_permute_workspace_size bytes
+ * Inside one expert's group the assignments keep ascending t*k + j order,
+ * so the result is deterministic and bit-reproducible.
+ */
+int moe_permute(const moe_bf16* x, const int32_t* topk_ids, const float* topk_w,
+                int64_t T, int64_t d, int64_t E, int64_t k,
+                int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* inv,
+                moe_bf16* x_perm, float* w_perm,
+                void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * Batched expert compute (section 2.1, point 1: the experts' weights stacked
+ * into one buffer and evaluated together; section 2.2 parallel_expert_compute)
+ * as two grouped GEMMs on the tcgen05 tensor cores:
+ *   h[pos] = silu(x_perm[pos] . W_gate[e]) * (x_perm[pos] . W_up[e])
+ *   y[pos] = w_perm[pos] * (h[pos] . W_down[e])
+ * for offsets[e] <= pos < offsets[e+1].
+ *   x_perm  [M, d] bf16,  w_perm [M] fp32,  offsets [E+1] int32 (device)
+ *   w_gate, w_up [E, d, f] bf16;  w_down [E, f, d] bf16
+ *   h [M, f] bf16 out (also the caller's scratch),  y [M, d] fp32 out
+ * offsets must be non-decreasing with offsets[0] = 0 and offsets[E] = M;
+ * otherwise MOE_ERR_DEVICE_BOUNDS is reported and nothing is written.
+ */
+int moe_expert_ffn(const moe_bf16* x_perm, const float* w_perm, const int32_t* offsets,
+                   const moe_bf16* w_gate, const moe_bf16* w_up, const moe_bf16* w_down,
+                   int64_t M, int64_t d, int64_t E, int64_t f,
+                   moe_bf16* h, float* y, cudaStream_t stream);
+
+/*
+ * Weighted aggregation back to token order (section 1, stage 4; section 2.2
+ * scatter_outputs), without atomics:
+ *   out[t] = sum_{j = 0..k-1} y[inv[t*k + j]]   (fp32 sum in slot order)
+ *   y [T*k, d] fp32 (already multiplied by the routing weight),
+ *   inv [T*k] int32 (entries outside [0, T*k) are reported as
+ *   MOE_ERR_DEVICE_BOUNDS and skipped), out [T, d] fp32.
+ */
+int moe_combine(const float* y, const int32_t* inv, int64_t T, int64_t d, int64_t k,
+                float* out, cudaStream_t stream);
+
+/*
+ * The whole block: moe_route -> moe_permute -> moe_expert_ffn -> moe_combine
+ * on one stream, with every intermediate in `workspace`
+ * (moe_workspace_size bytes).  Gives bit-identical results to calling the
+ * four stages one by one.
+ *   out          [T, d] fp32 out
+ *   topk_ids_out [T, k] int32 out, or NULL (kept in the workspace)
+ *   topk_w_out   [T, k] fp32 out, or NULL
+ */
+int moe_forward(const moe_bf16* x, const moe_bf16* w_router, const float* bias,
+                const moe_bf16* w_gate, const moe_bf16* w_up, const moe_bf16* w_down,
+                int64_t T, int64_t d, int64_t E, int64_t k, int64_t f,
+                float* out, int32_t* topk_ids_out, float* topk_w_out,
+                void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * moe_forward that also records n_events (>= 6) caller-created CUDA events
+ * on `stream`: before routing, after routing, after the permutation, after
+ * the gate/up GEMM, after the down GEMM and after the combine.  For timing
+ * individual stages; the arithmetic is identical to moe_forward.
+ */
+int moe_forward_profiled(const moe_bf16* x, const moe_bf16* w_router, const float* bias,
+                         const moe_bf16* w_gate, const moe_bf16* w_up, const moe_bf16* w_down,
+                         int64_t T, int64_t d, int64_t E, int64_t k, int64_t f,
+                         float* out, int32_t* topk_ids_out, float* topk_w_out,
+                         void* workspace, size_t workspace_bytes, cudaStream_t stream,
+                         cudaEvent_t* events, int n_events);
+
+/*
+ * Synchronises `stream`, then returns and clears the current device's status
+ * word (MOE_OK if no device-side error was recorded since the last call).
+ */
+int moe_get_status(cudaStream_t stream);
+
+/*
+ * Upper bound, in nanoseconds, on any single pipeline wait inside the
+ * library's kernels on the current device (default 1e9).  A wait that runs
+ * past it records MOE_ERR_DEVICE_TIMEOUT and the kernel winds down
+ * without faulting.  Values <= 0 restore the default.
+ */
+int moe_set_wait_limit_ns(int64_t limit_ns);
+
+/*
+ * Failure-path self test: launches one block whose bounded wait on a barrier
+ * that nothing signals runs out after `limit_ns`; afterwards
+ * moe_get_status reports MOE_ERR_DEVICE_TIMEOUT.  Needs no input data.
+ */
+int moe_selftest_wait_timeout(int64_t limit_ns, cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_H_ */

@@ -1,0 +1,63 @@
+"""Shared helpers for the GPU parity tests: seeded inputs on the device and
+cached oracle results (the oracle is slow, so each configuration's routing
+and sampled expert rows are computed once per session)."""
+from __future__ import annotations
+
+import functools
+
+import numpy as np
+import torch
+
+from oracle.oracle import default_oracle
+from top_routing_grouped_softmax_b200.synth import CONFIGS, MoEConfig, make_inputs, sample_tokens
+
+
+def small_cfg(T, d, E, k, f, seed=7, skew=False, sigma=0.02):
+    return MoEConfig(f"T{T}_d{d}_E{E}_k{k}_f{f}", T=T, d=d, E=E, k=k, f=f, sigma=sigma, seed=seed, skew=skew)
+
+
+@functools.lru_cache(maxsize=4)
+def inputs(cfg: MoEConfig):
+    return make_inputs(cfg)
+
+
+def on_device(inp):
+    dev = torch.device("cuda")
+    return {
+        "x": inp.x.to(dev), "w_router": inp.W_router.to(dev), "w_gate": inp.W_gate.to(dev),
+        "w_up": inp.W_up.to(dev), "w_down": inp.W_down.to(dev),
+        "bias": None if inp.bias is None else inp.bias.to(dev),
+    }
+
+
+@functools.lru_cache(maxsize=8)
+def oracle_route(cfg: MoEConfig):
+    inp = inputs(cfg)
+    return default_oracle().route(inp.bits("x"), inp.bits("W_router"), inp.bias_np(), cfg.k)
+
+
+def sample_for(cfg: MoEConfig, n: int):
+    """Sampled tokens, always including one token of the largest and of the
+    smallest non-empty expert group."""
+    r = oracle_route(cfg)
+    counts = np.bincount(r.ids.ravel(), minlength=cfg.E)
+    big = int(np.argmax(counts))
+    nz = np.nonzero(counts)[0]
+    small = int(nz[np.argmin(counts[nz])])
+    t_big = int(np.nonzero((r.ids == big).any(axis=1))[0][0])
+    t_small = int(np.nonzero((r.ids == small).any(axis=1))[0][0])
+    return sample_tokens(cfg.T, n, cfg.seed, must_include=(t_big, t_small, 0, cfg.T - 1))
+
+
+@functools.lru_cache(maxsize=8)
+def oracle_rows(cfg: MoEConfig, n: int):
+    inp = inputs(cfg)
+    r = oracle_route(cfg)
+    rows = sample_for(cfg, n)
+    ex = default_oracle().expert_rows(inp.bits("x"), inp.bits("W_gate"), inp.bits("W_up"), inp.bits("W_down"),
+                                      r.ids, r.weights, rows)
+    return rows, ex.out
+
+
+SAMPLES = {"tiny": 256, "qwen": 384, "fine": 384, "coarse": 24, "skew": 256}
+FULL = [CONFIGS[n] for n in ("tiny", "qwen", "fine", "coarse", "skew")]

@@ -1,0 +1,32 @@
+"""Failure detection on the GPU without a fault: a bounded wait that nothing
+satisfies gives up, reports MOE_ERR_DEVICE_TIMEOUT, and the context stays
+usable."""
+import pytest
+import torch
+
+import top_routing_grouped_softmax_b200 as moe
+from tests import gpu_cases as gc
+
+pytestmark = pytest.mark.gpu
+
+
+def test_bounded_wait_times_out_and_context_survives():
+    assert moe.get_status() == moe.MOE_OK
+    moe.selftest_wait_timeout(20_000_000)   # 20 ms
+    assert moe.get_status() == moe.MOE_ERR_DEVICE_TIMEOUT
+    assert moe.get_status() == moe.MOE_OK
+    cfg = gc.small_cfg(256, 128, 8, 2, 128)
+    d = gc.on_device(gc.inputs(cfg))
+    out = moe.forward(d["x"], d["w_router"], d["w_gate"], d["w_up"], d["w_down"], 2)
+    torch.cuda.synchronize()
+    assert moe.get_status() == moe.MOE_OK
+    assert torch.isfinite(out.float()).all().item()
+
+
+def test_wait_limit_setting_roundtrip():
+    moe.set_wait_limit_ns(500_000_000)
+    moe.set_wait_limit_ns(0)   # back to the default
+    cfg = gc.small_cfg(128, 64, 8, 2, 64)
+    d = gc.on_device(gc.inputs(cfg))
+    moe.forward(d["x"], d["w_router"], d["w_gate"], d["w_up"], d["w_down"], 2)
+    assert moe.get_status() == moe.MOE_OK

@@ -1,0 +1,118 @@
+"""The fused moe_forward against the oracle, on the GPU: small cases on every
+token, the five workloads at full size on sampled tokens (the launch
+configuration the benchmark times), and the equalities the path must keep."""
+import numpy as np
+import pytest
+import torch
+
+import top_routing_grouped_softmax_b200 as moe
+from tests import gpu_cases as gc
+from tests.parity import route_check, value_check
+
+pytestmark = pytest.mark.gpu
+
+SMALL = [
+    gc.small_cfg(1000, 256, 16, 4, 320),
+    gc.small_cfg(513, 192, 8, 2, 256, skew=True),
+    gc.small_cfg(130, 64, 8, 8, 64),
+    gc.small_cfg(2000, 128, 264, 8, 128),
+]
+
+
+def _forward(cfg, d):
+    ids = torch.empty(cfg.T, cfg.k, dtype=torch.int32, device="cuda")
+    w = torch.empty(cfg.T, cfg.k, dtype=torch.float32, device="cuda")
+    out = moe.forward(d["x"], d["w_router"], d["w_gate"], d["w_up"], d["w_down"], cfg.k, bias=d["bias"],
+                      topk_ids=ids, topk_w=w)
+    torch.cuda.synchronize()
+    assert moe.get_status() == moe.MOE_OK
+    return out, ids, w
+
+
+def _check(cfg, out, ids, w, rows, ref_out):
+    r = gc.oracle_route(cfg)
+    excluded, stats = route_check(ids.cpu().numpy(), w.cpu().numpy(), r.probs, r.ids, cfg.k)
+    keep = ~excluded[rows]
+    got = out.double().cpu().numpy()[rows]
+    return value_check(got[keep], ref_out[keep], f"out[{cfg.name}]"), stats
+
+
+@pytest.mark.parametrize("cfg", SMALL, ids=lambda c: c.name)
+def test_forward_small_all_tokens(cfg):
+    d = gc.on_device(gc.inputs(cfg))
+    out, ids, w = _forward(cfg, d)
+    rows, ref = gc.oracle_rows(cfg, cfg.T)
+    _check(cfg, out, ids, w, rows, ref)
+
+
+@pytest.mark.parametrize("cfg", gc.FULL, ids=lambda c: c.name)
+def test_forward_full_size_sampled(cfg):
+    d = gc.on_device(gc.inputs(cfg))
+    out, ids, w = _forward(cfg, d)
+    rows, ref = gc.oracle_rows(cfg, gc.SAMPLES[cfg.name])
+    (mx, mean), stats = _check(cfg, out, ids, w, rows, ref)
+    print(cfg.name, "sampled", len(rows), "max/rms", mx, "mean_rel", mean, stats)
+
+
+def test_forward_equals_stages_bitwise():
+    cfg = gc.small_cfg(1000, 256, 16, 4, 320, skew=True)
+    d = gc.on_device(gc.inputs(cfg))
+    out, ids, w = _forward(cfg, d)
+    ids2, w2 = moe.route(d["x"], d["w_router"], cfg.k, bias=d["bias"])
+    pm = moe.permute(d["x"], ids2, w2, cfg.E)
+    h, y = moe.expert_ffn(pm["x_perm"], pm["w_perm"], pm["offsets"], d["w_gate"], d["w_up"], d["w_down"])
+    out2 = moe.combine(y, pm["inv"], cfg.T, cfg.k)
+    torch.cuda.synchronize()
+    assert torch.equal(ids, ids2) and torch.equal(w, w2)
+    assert torch.equal(out, out2)
+
+
+def test_forward_deterministic_and_block_api():
+    cfg = gc.small_cfg(900, 128, 32, 4, 128)
+    d = gc.on_device(gc.inputs(cfg))
+    blk = moe.MoEBlock(d["w_router"], d["w_gate"], d["w_up"], d["w_down"], cfg.k)
+    a = blk(d["x"]).clone()
+    b = blk(d["x"]).clone()
+    c, _, _ = _forward(cfg, d)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+    assert torch.equal(a, c)
+
+
+def test_forward_single_expert_is_dense_swiglu():
+    """All tokens forced onto expert 0 with k = 1 through a dominant bias: the
+    block is one dense SwiGLU MLP scaled by p_0 (checked against the oracle)."""
+    cfg = gc.small_cfg(256, 128, 8, 1, 128)
+    inp = gc.inputs(cfg)
+    d = gc.on_device(inp)
+    bias = torch.full((8,), -30.0, device="cuda")
+    bias[0] = 30.0
+    d["bias"] = bias
+    out, ids, w = _forward(cfg, d)
+    assert torch.all(ids == 0).item()
+    from oracle.oracle import default_oracle
+    r, ex = default_oracle().forward(inp.bits("x"), inp.bits("W_router"), bias.cpu().numpy(), inp.bits("W_gate"),
+                                     inp.bits("W_up"), inp.bits("W_down"), 1)
+    value_check(out.double().cpu().numpy(), ex.out, "dense")
+
+
+def test_forward_empty_batch():
+    cfg = gc.small_cfg(8, 64, 8, 2, 64)
+    d = gc.on_device(gc.inputs(cfg))
+    x0 = d["x"][:0]
+    out = moe.forward(x0, d["w_router"], d["w_gate"], d["w_up"], d["w_down"], 2)
+    torch.cuda.synchronize()
+    assert out.shape == (0, 64)
+    assert moe.get_status() == moe.MOE_OK
+
+
+def test_forward_profiled_events():
+    cfg = gc.small_cfg(512, 128, 8, 2, 128)
+    d = gc.on_device(gc.inputs(cfg))
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
+    out = moe.forward(d["x"], d["w_router"], d["w_gate"], d["w_up"], d["w_down"], 2, events=evs)
+    torch.cuda.synchronize()
+    times = [evs[i].elapsed_time(evs[i + 1]) for i in range(5)]
+    assert all(t >= 0 for t in times)
+    ref, _, _ = _forward(cfg, d)
+    assert torch.equal(out, ref)

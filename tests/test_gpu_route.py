@@ -1,0 +1,72 @@
+"""Router kernel (GEMM + fp32 softmax + top-k) against the oracle, on the GPU.
+
+Expert ids bit-exact (near ties excepted, see tests/parity.py), weights to
+1e-5 relative."""
+import numpy as np
+import pytest
+import torch
+
+import top_routing_grouped_softmax_b200 as moe
+from tests import gpu_cases as gc
+from tests.parity import route_check
+
+pytestmark = pytest.mark.gpu
+
+SMALL = [
+    gc.small_cfg(1000, 256, 16, 4, 320, sigma=0.1),       # ragged T, several tiles
+    gc.small_cfg(129, 128, 8, 2, 64, sigma=0.1),          # one full tile + 1 token
+    gc.small_cfg(1, 64, 8, 1, 64, sigma=0.1),             # single token, minimal d
+    gc.small_cfg(300, 192, 264, 8, 64, sigma=0.1),        # E not a multiple of 64: two MMAs per k-step
+    gc.small_cfg(257, 128, 512, 32, 64, sigma=0.1),       # maximum E and k
+    gc.small_cfg(200, 64, 8, 8, 64, sigma=0.1),           # k = E
+    gc.small_cfg(640, 256, 64, 6, 64, sigma=0.1, skew=True),  # per-expert bias
+]
+
+
+def _route(cfg):
+    d = gc.on_device(gc.inputs(cfg))
+    ids, w = moe.route(d["x"], d["w_router"], cfg.k, bias=d["bias"])
+    torch.cuda.synchronize()
+    assert moe.get_status() == moe.MOE_OK
+    return ids.cpu().numpy(), w.cpu().numpy()
+
+
+@pytest.mark.parametrize("cfg", SMALL, ids=lambda c: c.name)
+def test_route_small(cfg):
+    ids, w = _route(cfg)
+    r = gc.oracle_route(cfg)
+    route_check(ids, w, r.probs, r.ids, cfg.k)
+
+
+@pytest.mark.parametrize("cfg", gc.FULL, ids=lambda c: c.name)
+def test_route_full_size(cfg):
+    ids, w = _route(cfg)
+    r = gc.oracle_route(cfg)
+    excluded, stats = route_check(ids, w, r.probs, r.ids, cfg.k)
+    print(cfg.name, stats)
+    assert stats["excluded_near_tie"] < max(1, cfg.T // 100)
+
+
+def test_route_exact_ties_lowest_index():
+    """Identical router columns: every probability is 1/E and ids are 0..k-1."""
+    cfg = gc.small_cfg(300, 128, 16, 4, 64)
+    inp = gc.inputs(cfg)
+    d = gc.on_device(inp)
+    wr = d["w_router"].clone()
+    wr[:] = wr[:, :1]
+    ids, w = moe.route(d["x"], wr, 4)
+    torch.cuda.synchronize()
+    assert np.all(ids.cpu().numpy() == np.arange(4)[None, :])
+    assert torch.all(w == 1.0 / 16).item()
+
+
+def test_route_rejects_bad_shapes():
+    x = torch.zeros(4, 64, dtype=torch.bfloat16, device="cuda")
+    wr = torch.zeros(64, 12, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(moe.MoEError) as e:
+        moe.route(x, wr, 2)
+    assert e.value.status == moe.MOE_ERR_UNSUPPORTED_SHAPE
+    wr = torch.zeros(64, 8, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(moe.MoEError) as e:
+        moe.route(x, wr, 9)
+    assert e.value.status == moe.MOE_ERR_UNSUPPORTED_SHAPE

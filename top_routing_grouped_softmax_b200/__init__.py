@@ -1,0 +1,293 @@
+"""B200-native sparse Mixture-of-Experts block forward (sm_100a CUDA).
+
+A thin ctypes binding over the C ABI of ``libmoe.so`` (declared in
+``include/moe.h``).  Every step of the block runs in the library's CUDA
+kernels; this module only checks tensor properties, allocates outputs and
+workspace through PyTorch, and passes raw device pointers and the current
+CUDA stream.  There is no CPU or PyTorch fallback: if the library is missing
+or the device is not a B200, the calls raise.
+
+Functions mirror the ABI entry points:
+  route, permute, expert_ffn, combine, forward (and forward_profiled),
+  workspace_size, permute_workspace_size, get_status, set_wait_limit_ns.
+``MoEBlock`` keeps the weights and a reusable workspace for repeated calls.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmoe.so")
+
+MOE_OK = 0
+MOE_ERR_INVALID_ARG = 1
+MOE_ERR_UNSUPPORTED_SHAPE = 2
+MOE_ERR_WORKSPACE_TOO_SMALL = 3
+MOE_ERR_CUDA = 4
+MOE_ERR_DEVICE_TIMEOUT = 5
+MOE_ERR_DEVICE_BOUNDS = 6
+MOE_ERR_UNSUPPORTED_DEVICE = 7
+
+# Every symbol include/moe.h declares.
+ABI_SYMBOLS = (
+    "moe_strerror", "moe_version", "moe_workspace_size", "moe_permute_workspace_size",
+    "moe_route", "moe_permute", "moe_expert_ffn", "moe_combine", "moe_forward",
+    "moe_forward_profiled", "moe_get_status", "moe_set_wait_limit_ns", "moe_selftest_wait_timeout",
+)
+
+
+class MoEError(RuntimeError):
+    """A non-zero status from the C ABI."""
+
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {strerror(status)} (status {status})")
+
+
+_P = ctypes.c_void_p
+_I64 = ctypes.c_int64
+_SZ = ctypes.c_size_t
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libmoe.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(
+                f"{LIB_PATH} is missing: build it with `python -m top_routing_grouped_softmax_b200._build` "
+                "or __graft_entry__.build(); there is no fallback implementation")
+        L = ctypes.CDLL(LIB_PATH)
+        L.moe_strerror.restype = ctypes.c_char_p
+        L.moe_strerror.argtypes = [ctypes.c_int]
+        L.moe_version.restype = ctypes.c_int
+        L.moe_workspace_size.restype = _SZ
+        L.moe_workspace_size.argtypes = [_I64] * 5
+        L.moe_permute_workspace_size.restype = _SZ
+        L.moe_permute_workspace_size.argtypes = [_I64] * 3
+        L.moe_route.argtypes = [_P, _P, _P, _I64, _I64, _I64, _I64, _P, _P, _P]
+        L.moe_permute.argtypes = [_P, _P, _P, _I64, _I64, _I64, _I64, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]
+        L.moe_expert_ffn.argtypes = [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _P, _P, _P]
+        L.moe_combine.argtypes = [_P, _P, _I64, _I64, _I64, _P, _P]
+        L.moe_forward.argtypes = [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64, _P, _P, _P, _P, _SZ, _P]
+        L.moe_forward_profiled.argtypes = L.moe_forward.argtypes + [_P, ctypes.c_int]
+        L.moe_get_status.argtypes = [_P]
+        L.moe_set_wait_limit_ns.argtypes = [_I64]
+        L.moe_selftest_wait_timeout.argtypes = [_I64, _P]
+        for name in ("moe_route", "moe_permute", "moe_expert_ffn", "moe_combine", "moe_forward",
+                     "moe_forward_profiled", "moe_get_status", "moe_set_wait_limit_ns",
+                     "moe_selftest_wait_timeout"):
+            getattr(L, name).restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def strerror(status: int) -> str:
+    try:
+        return lib().moe_strerror(int(status)).decode()
+    except ImportError:
+        return f"status {status}"
+
+
+def _check(rc: int, where: str):
+    if rc != MOE_OK:
+        raise MoEError(rc, where)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _need(t, name, dtype, ndim=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims, got {t.dim()}")
+    return t
+
+
+# ------------------------------------------------------------------ sizes
+def workspace_size(T: int, d: int, E: int, k: int, f: int) -> int:
+    return int(lib().moe_workspace_size(T, d, E, k, f))
+
+
+def permute_workspace_size(T: int, E: int, k: int) -> int:
+    return int(lib().moe_permute_workspace_size(T, E, k))
+
+
+def _workspace(nbytes: int, device) -> torch.Tensor:
+    return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+
+
+# ----------------------------------------------------------------- stages
+def route(x, w_router, k, bias=None, topk_ids=None, topk_w=None):
+    """Router GEMM + fp32 softmax + top-k; returns (topk_ids int32 [T,k], topk_w fp32 [T,k])."""
+    _need(x, "x", torch.bfloat16, 2)
+    _need(w_router, "w_router", torch.bfloat16, 2)
+    T, d = x.shape
+    E = w_router.shape[1]
+    if bias is not None:
+        _need(bias, "bias", torch.float32, 1)
+    if topk_ids is None:
+        topk_ids = torch.empty(T, k, dtype=torch.int32, device=x.device)
+    if topk_w is None:
+        topk_w = torch.empty(T, k, dtype=torch.float32, device=x.device)
+    _check(lib().moe_route(_ptr(x), _ptr(w_router), _ptr(bias), T, d, E, k, _ptr(topk_ids),
+                           _ptr(topk_w), _stream()), "moe_route")
+    return topk_ids, topk_w
+
+
+def permute(x, topk_ids, topk_w, E, gather=True):
+    """Stable grouping by expert; returns dict(counts, offsets, perm, inv, x_perm, w_perm)."""
+    _need(topk_ids, "topk_ids", torch.int32, 2)
+    _need(topk_w, "topk_w", torch.float32, 2)
+    T, k = topk_ids.shape
+    dev = topk_ids.device
+    d = x.shape[1] if x is not None else 64
+    if x is not None:
+        _need(x, "x", torch.bfloat16, 2)
+    M = T * k
+    out = {
+        "counts": torch.empty(E, dtype=torch.int32, device=dev),
+        "offsets": torch.empty(E + 1, dtype=torch.int32, device=dev),
+        "perm": torch.empty(M, dtype=torch.int32, device=dev),
+        "inv": torch.empty(M, dtype=torch.int32, device=dev),
+        "w_perm": torch.empty(M, dtype=torch.float32, device=dev),
+        "x_perm": torch.empty(M, d, dtype=torch.bfloat16, device=dev) if (gather and x is not None) else None,
+    }
+    nbytes = permute_workspace_size(T, E, k)
+    ws = _workspace(nbytes, dev)
+    _check(lib().moe_permute(_ptr(x), _ptr(topk_ids), _ptr(topk_w), T, d, E, k, _ptr(out["counts"]),
+                             _ptr(out["offsets"]), _ptr(out["perm"]), _ptr(out["inv"]), _ptr(out["x_perm"]),
+                             _ptr(out["w_perm"]), _ptr(ws), ws.numel(), _stream()), "moe_permute")
+    return out
+
+
+def expert_ffn(x_perm, w_perm, offsets, w_gate, w_up, w_down, h=None, y=None):
+    """Grouped gate/up + SwiGLU and grouped down + routing weight; returns (h bf16, y fp32)."""
+    _need(x_perm, "x_perm", torch.bfloat16, 2)
+    _need(w_perm, "w_perm", torch.float32, 1)
+    _need(offsets, "offsets", torch.int32, 1)
+    for n, t in (("w_gate", w_gate), ("w_up", w_up), ("w_down", w_down)):
+        _need(t, n, torch.bfloat16, 3)
+    M, d = x_perm.shape
+    E, _, f = w_gate.shape
+    if h is None:
+        h = torch.empty(M, f, dtype=torch.bfloat16, device=x_perm.device)
+    if y is None:
+        y = torch.empty(M, d, dtype=torch.float32, device=x_perm.device)
+    _need(y, "y", torch.float32, 2)
+    _check(lib().moe_expert_ffn(_ptr(x_perm), _ptr(w_perm), _ptr(offsets), _ptr(w_gate), _ptr(w_up),
+                                _ptr(w_down), M, d, E, f, _ptr(h), _ptr(y), _stream()), "moe_expert_ffn")
+    return h, y
+
+
+def combine(y, inv, T, k, out=None):
+    """out[t] = sum_j y[inv[t*k+j]] (fp32 rows, fp32 sum, fp32 result)."""
+    _need(y, "y", torch.float32, 2)
+    _need(inv, "inv", torch.int32, 1)
+    d = y.shape[1]
+    if out is None:
+        out = torch.empty(T, d, dtype=torch.float32, device=y.device)
+    _need(out, "out", torch.float32, 2)
+    _check(lib().moe_combine(_ptr(y), _ptr(inv), T, d, k, _ptr(out), _stream()), "moe_combine")
+    return out
+
+
+def _forward_args(x, w_router, w_gate, w_up, w_down, bias):
+    _need(x, "x", torch.bfloat16, 2)
+    _need(w_router, "w_router", torch.bfloat16, 2)
+    for n, t in (("w_gate", w_gate), ("w_up", w_up), ("w_down", w_down)):
+        _need(t, n, torch.bfloat16, 3)
+    if bias is not None:
+        _need(bias, "bias", torch.float32, 1)
+    T, d = x.shape
+    E, _, f = w_gate.shape
+    return T, d, E, f
+
+
+def forward(x, w_router, w_gate, w_up, w_down, k, bias=None, out=None, workspace=None,
+            topk_ids=None, topk_w=None, events=None):
+    """The whole MoE block; returns out [T, d] fp32.
+
+    ``events`` (optional): a list of >= 6 torch.cuda.Event objects recorded at
+    the stage boundaries (before route, after route, after permute, after
+    gate/up, after down, after combine).
+    """
+    T, d, E, f = _forward_args(x, w_router, w_gate, w_up, w_down, bias)
+    if out is None:
+        out = torch.empty(T, d, dtype=torch.float32, device=x.device)
+    _need(out, "out", torch.float32, 2)
+    nbytes = workspace_size(T, d, E, k, f)
+    if nbytes == 0:
+        raise MoEError(MOE_ERR_UNSUPPORTED_SHAPE, "moe_workspace_size")
+    if workspace is None:
+        workspace = _workspace(nbytes, x.device)
+    args = [_ptr(x), _ptr(w_router), _ptr(bias), _ptr(w_gate), _ptr(w_up), _ptr(w_down), T, d, E, k, f,
+            _ptr(out), _ptr(topk_ids), _ptr(topk_w), _ptr(workspace), workspace.numel(), _stream()]
+    if events is None:
+        _check(lib().moe_forward(*args), "moe_forward")
+    else:
+        arr = (ctypes.c_void_p * len(events))()
+        for i, ev in enumerate(events):
+            if ev.cuda_event == 0:
+                ev.record()  # the event handle is created lazily by torch
+            arr[i] = ev.cuda_event
+        _check(lib().moe_forward_profiled(*args, arr, len(events)), "moe_forward_profiled")
+    return out
+
+
+def get_status() -> int:
+    """Synchronise the current stream; return and clear the device status word."""
+    return int(lib().moe_get_status(_stream()))
+
+
+def set_wait_limit_ns(limit_ns: int):
+    _check(lib().moe_set_wait_limit_ns(int(limit_ns)), "moe_set_wait_limit_ns")
+
+
+def selftest_wait_timeout(limit_ns: int):
+    _check(lib().moe_selftest_wait_timeout(int(limit_ns), _stream()), "moe_selftest_wait_timeout")
+
+
+class MoEBlock:
+    """Weights of one MoE block on the GPU plus a reusable workspace."""
+
+    def __init__(self, w_router, w_gate, w_up, w_down, k, bias=None):
+        self.w_router, self.w_gate, self.w_up, self.w_down = w_router, w_gate, w_up, w_down
+        self.bias = bias
+        self.k = int(k)
+        self.E, self.d, self.f = w_gate.shape
+        self._ws = None
+
+    def workspace(self, T: int) -> torch.Tensor:
+        need = workspace_size(T, self.d, self.E, self.k, self.f)
+        if self._ws is None or self._ws.numel() < need:
+            self._ws = _workspace(need, self.w_gate.device)
+        return self._ws
+
+    def __call__(self, x, out=None, topk_ids=None, topk_w=None, events=None):
+        return forward(x, self.w_router, self.w_gate, self.w_up, self.w_down, self.k, bias=self.bias,
+                       out=out, workspace=self.workspace(x.shape[0]), topk_ids=topk_ids, topk_w=topk_w,
+                       events=events)
+
+
+__all__ = [
+    "lib", "strerror", "MoEError", "ABI_SYMBOLS", "workspace_size", "permute_workspace_size", "route",
+    "permute", "expert_ffn", "combine", "forward", "get_status", "set_wait_limit_ns",
+    "selftest_wait_timeout", "MoEBlock",
+]

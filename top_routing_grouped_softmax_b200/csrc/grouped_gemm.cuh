@@ -1,0 +1,376 @@
+// grouped_gemm.cuh -- persistent grouped GEMM over variable-size expert
+// groups on the tcgen05 tensor cores, with the two epilogues of the expert
+// MLP fused in.
+//
+// This is the "batched expert compute" of "Qwen3MoeSparseMoeBlock
+// performance optimisation in practice": the experts' weight matrices are
+// stacked in one buffer and evaluated together (section 2.1, point 1), with
+// work spread over the SMs dynamically (section 2.1, point 2) and operands
+// staged in shared memory (section 2.2, point 3).  The compute/IO overlap
+// through a producer-consumer queue that the SonicMoE comparison page
+// describes for Hopper is realised here with Blackwell's own machinery.
+//
+// Rows of the A operand are grouped by expert: group e is rows
+// [offsets[e], offsets[e+1]).  Each group is cut into 128-row M tiles (the
+// last may be partial; its extra rows belong to the next group or are past
+// the end, are computed, and are not stored).  A work item is one M tile x
+// one N tile; persistent CTAs take items blockIdx.x, +gridDim.x, ...  Each
+// CTA rebuilds the tile list from the device offsets itself, so nothing is
+// read back to the host.
+//
+// Warp roles (192 threads):
+//   warp 0       TMA producer: A [128 rows x 64 k] K-major, B 4 x [64 k x 64 n]
+//                (weights are [K, N] with N contiguous: MN-major operand)
+//   warp 1       TMEM allocation + single-thread tcgen05.mma issuer,
+//                M=128 N=256 K=16 per instruction, fp32 accumulators
+//   warps 2..5   epilogue: tcgen05.ld of the 128 x 256 accumulator, one row
+//                per thread, fused math, bf16 stores
+// Two accumulator buffers (2 x 256 TMEM columns) let the epilogue of one
+// tile overlap the MMAs of the next.
+//
+// Epilogues:
+//   kSwiGLU   : B columns 0..127 come from W_gate, 128..255 from W_up for the
+//               same 128 output columns; h = silu(g) * u, silu(z) = z/(1+e^-z)
+//   kWeighted : y = w_perm[row] * acc in fp32 (the routing weight applied
+//               after the down projection; y stays fp32 so that the k-way sum
+//               in the combine is an fp32 accumulation of unrounded terms)
+#pragma once
+
+#include <cuda_bf16.h>
+
+#include "ptx.cuh"
+
+namespace moe {
+namespace gemm {
+
+constexpr int kBM = 128;
+constexpr int kBN = 256;
+constexpr int kBK = 64;
+constexpr int kStages = 4;
+constexpr int kThreads = 192;
+constexpr int kABytes = kBM * kBK * 2;      // 16 KB
+constexpr int kChunkBytes = 64 * kBK * 2;   // 8 KB: 64 n x 64 k
+constexpr int kBBytes = 4 * kChunkBytes;    // 32 KB
+constexpr int kStageBytes = kABytes + kBBytes;
+constexpr uint32_t kTmemCols = 512;         // 2 accumulators x 256 columns
+constexpr int kMaxE = 512;
+
+enum EpiKind { kSwiGLU = 0, kWeighted = 1 };
+
+struct Params {
+    const int32_t* offsets;  // [E+1] group boundaries (device)
+    const float* w_perm;     // [M] routing weight per grouped row (kWeighted)
+    void* out;               // [M, n_out]: bf16 h (kSwiGLU) or fp32 y (kWeighted)
+    int E;
+    int M;        // rows of A
+    int K;        // reduction length (multiple of 64)
+    int n_out;    // output columns (multiple of 64)
+    int n_tiles;  // N tiles per M tile
+};
+
+// Shared memory after the stage ring.
+struct alignas(8) Ctrl {
+    uint64_t full[kStages];
+    uint64_t empty[kStages];
+    uint64_t acc_full[2];
+    uint64_t acc_empty[2];
+    uint64_t done;
+    uint32_t tmem_slot;
+    volatile int abort_flag;
+    int bad;
+    int total_mtiles;
+    int off[kMaxE + 1];   // group offsets
+    int tp[kMaxE + 1];    // exclusive prefix of M tiles per group
+};
+
+__host__ inline size_t smem_bytes() { return 1024 + (size_t)kStages * kStageBytes + sizeof(Ctrl); }
+
+// Work item -> (expert, first row, group end, N tile).
+__device__ __forceinline__ void decode(int64_t w, int n_tiles, const Ctrl& c, int E, int& e, int& row0,
+                                       int& row_end, int& nt)
+{
+    const int mt = (int)(w / n_tiles);
+    nt = (int)(w - (int64_t)mt * n_tiles);
+    int lo = 0, hi = E;  // tp[lo] <= mt < tp[hi]
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (c.tp[mid] <= mt)
+            lo = mid;
+        else
+            hi = mid;
+    }
+    e = lo;
+    row0 = c.off[e] + (mt - c.tp[e]) * kBM;
+    row_end = c.off[e + 1];
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b)
+{
+    const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+__device__ __forceinline__ float silu(float z) { return z / (1.0f + __expf(-z)); }
+
+template <int EPI>
+__global__ void __launch_bounds__(kThreads, 1)
+    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b0,
+                        const __grid_constant__ CUtensorMap tm_b1, Params p)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    Ctrl& c = *reinterpret_cast<Ctrl*>(smem + (size_t)kStages * kStageBytes);
+
+    const int warp = threadIdx.x / 32;
+    const int lane = threadIdx.x % 32;
+    const uint64_t limit = g_wait_limit_ns;
+    const int E = p.E;
+
+    // ---- tile list from the device offsets (validated) ----
+    for (int i = threadIdx.x; i <= E; i += kThreads) c.off[i] = p.offsets[i];
+    __syncthreads();
+    if (warp == 0) {
+        int run = 0;
+        bool bad = false;
+        for (int base = 0; base < E; base += 32) {
+            const int e = base + lane;
+            int tiles = 0;
+            if (e < E) {
+                const int cnt = c.off[e + 1] - c.off[e];
+                if (cnt < 0) bad = true;
+                tiles = cnt > 0 ? (cnt + kBM - 1) / kBM : 0;
+            }
+            int incl = tiles;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int nb = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += nb;
+            }
+            if (e < E) c.tp[e] = run + incl - tiles;
+            run += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        bad = __any_sync(0xffffffffu, bad);
+        if (lane == 0) {
+            c.tp[E] = run;
+            c.bad = (bad || c.off[0] != 0 || c.off[E] != p.M) ? 1 : 0;
+            c.total_mtiles = run;
+            if (c.bad && blockIdx.x == 0) record_status(kStatusDeviceBounds);
+        }
+    }
+    if (threadIdx.x == 32) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&c.full[s], 1);
+            mbar_init(&c.empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&c.acc_full[b], 1);
+            mbar_init(&c.acc_empty[b], 4 * 32);
+        }
+        mbar_init(&c.done, 1);
+        c.abort_flag = 0;
+        fence_mbar_init();
+        tma_prefetch_map(&tm_a);
+        tma_prefetch_map(&tm_b0);
+        if (EPI == kSwiGLU) tma_prefetch_map(&tm_b1);
+    }
+    if (warp == 1) {
+        __syncwarp();
+        tmem_alloc(&c.tmem_slot, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem = c.tmem_slot;
+    const int64_t total_work = c.bad ? 0 : (int64_t)c.total_mtiles * p.n_tiles;
+    const int num_kb = p.K / kBK;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ------------------------------------------------ TMA producer
+            int s = 0;
+            uint32_t ph = 0;
+            int64_t issued = 0;
+            for (int64_t w = blockIdx.x; w < total_work && !c.abort_flag; w += gridDim.x) {
+                int e, row0, row_end, nt;
+                decode(w, p.n_tiles, c, E, e, row0, row_end, nt);
+                const int krow0 = e * p.K;
+                bool ok = true;
+                for (int kb = 0; kb < num_kb; ++kb) {
+                    if (!mbar_wait(&c.empty[s], ph ^ 1u, limit)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t* sa = smem + (size_t)s * kStageBytes;
+                    uint8_t* sb = sa + kABytes;
+                    mbar_arrive_expect_tx(&c.full[s], (uint32_t)kStageBytes);
+                    tma_load_2d(sa, &tm_a, &c.full[s], kb * kBK, row0);
+                    const int kr = krow0 + kb * kBK;
+                    if (EPI == kSwiGLU) {
+                        const int n0 = nt * 128;
+                        tma_load_2d(sb + 0 * kChunkBytes, &tm_b0, &c.full[s], n0, kr);
+                        tma_load_2d(sb + 1 * kChunkBytes, &tm_b0, &c.full[s], n0 + 64, kr);
+                        tma_load_2d(sb + 2 * kChunkBytes, &tm_b1, &c.full[s], n0, kr);
+                        tma_load_2d(sb + 3 * kChunkBytes, &tm_b1, &c.full[s], n0 + 64, kr);
+                    } else {
+                        const int n0 = nt * kBN;
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+                            tma_load_2d(sb + q * kChunkBytes, &tm_b0, &c.full[s], n0 + 64 * q, kr);
+                    }
+                    ++issued;
+                    if (++s == kStages) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
+                }
+                if (!ok) {
+                    c.abort_flag = 1;
+                    break;
+                }
+            }
+            // Never leave the CTA with a copy still landing in its shared memory.
+            for (int q = 0; q < kStages; ++q) {
+                const int64_t cnt = issued / kStages + (q < issued % kStages ? 1 : 0);
+                if (cnt > 0) mbar_wait(&c.full[q], (uint32_t)(cnt - 1) & 1u, limit);
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ------------------------------------------------ MMA issuer
+            constexpr uint32_t idesc = idesc_bf16_f32(kBM, kBN, false, true);
+            int s = 0;
+            uint32_t ph = 0;
+            int acc = 0;
+            uint32_t acc_ph = 0;
+            for (int64_t w = blockIdx.x; w < total_work && !c.abort_flag; w += gridDim.x) {
+                if (!mbar_wait(&c.acc_empty[acc], acc_ph ^ 1u, limit)) {
+                    c.abort_flag = 1;
+                    break;
+                }
+                tc_fence_after_sync();
+                const uint32_t d_tmem = tmem + (uint32_t)(acc * kBN);
+                bool ok = true;
+                for (int kb = 0; kb < num_kb; ++kb) {
+                    if (!mbar_wait(&c.full[s], ph, limit)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after_sync();
+                    const uint32_t a_base = smem_u32(smem + (size_t)s * kStageBytes);
+                    const uint32_t b_base = a_base + kABytes;
+#pragma unroll
+                    for (int kk = 0; kk < kBK / 16; ++kk) {
+                        const uint64_t adesc = smem_desc_sw128(a_base + kk * 32, 16, 1024);
+                        const uint64_t bdesc = smem_desc_sw128(b_base + kk * 2048, kChunkBytes, 1024);
+                        mma_bf16_ss(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
+                    }
+                    mma_commit(&c.empty[s]);  // frees the stage once these MMAs are done
+                    if (++s == kStages) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
+                }
+                if (!ok) {
+                    c.abort_flag = 1;
+                    break;
+                }
+                mma_commit(&c.acc_full[acc]);
+                if (++acc == 2) {
+                    acc = 0;
+                    acc_ph ^= 1u;
+                }
+            }
+            mma_commit(&c.done);
+            mbar_wait(&c.done, 0, limit);
+        }
+        __syncwarp();
+    } else {
+        // ---------------------------------------------------- epilogue
+        const int q = warp & 3;          // TMEM lane quarter this warp may access
+        const int r = q * 32 + lane;     // tile row owned by this thread
+        int acc = 0;
+        uint32_t acc_ph = 0;
+        for (int64_t w = blockIdx.x; w < total_work; w += gridDim.x) {
+            int e, row0, row_end, nt;
+            decode(w, p.n_tiles, c, E, e, row0, row_end, nt);
+            // Every lane polls; the warp continues only together, since the
+            // TMEM loads below are warp-collective.
+            const bool ready = __all_sync(0xffffffffu, mbar_wait(&c.acc_full[acc], acc_ph, limit));
+            if (!ready) {
+                c.abort_flag = 1;
+                break;
+            }
+            tc_fence_after_sync();
+            const uint32_t tbase = tmem + (uint32_t)(acc * kBN) + ((uint32_t)(q * 32) << 16);
+            const int row = row0 + r;
+            const bool valid = row < row_end;
+            if (EPI == kSwiGLU) {
+                __nv_bfloat16* orow =
+                    static_cast<__nv_bfloat16*>(p.out) + (int64_t)row * p.n_out + nt * 128;
+                const int ncols = min(128, p.n_out - nt * 128);
+#pragma unroll 1
+                for (int c0 = 0; c0 < 128; c0 += 16) {
+                    uint32_t g[16], u[16];
+                    tmem_ld16(tbase + c0, g);
+                    tmem_ld16(tbase + 128 + c0, u);
+                    tmem_ld_wait();
+                    if (valid && c0 < ncols) {
+                        uint32_t packed[8];
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            const float h0 = silu(__uint_as_float(g[2 * i])) * __uint_as_float(u[2 * i]);
+                            const float h1 = silu(__uint_as_float(g[2 * i + 1])) * __uint_as_float(u[2 * i + 1]);
+                            packed[i] = pack_bf16x2(h0, h1);
+                        }
+                        uint4* dst = reinterpret_cast<uint4*>(orow + c0);
+                        dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+                        dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+                    }
+                }
+            } else {
+                const float wgt = valid ? __ldg(p.w_perm + row) : 0.0f;
+                float* orow = static_cast<float*>(p.out) + (int64_t)row * p.n_out + nt * kBN;
+                const int ncols = min(kBN, p.n_out - nt * kBN);
+#pragma unroll 1
+                for (int c0 = 0; c0 < kBN; c0 += 32) {
+                    uint32_t a0[16], a1[16];
+                    tmem_ld16(tbase + c0, a0);
+                    tmem_ld16(tbase + c0 + 16, a1);
+                    tmem_ld_wait();
+                    if (valid && c0 < ncols) {
+                        float4* dst = reinterpret_cast<float4*>(orow + c0);
+#pragma unroll
+                        for (int v = 0; v < 4; ++v)
+                            dst[v] = make_float4(wgt * __uint_as_float(a0[4 * v]), wgt * __uint_as_float(a0[4 * v + 1]),
+                                                 wgt * __uint_as_float(a0[4 * v + 2]),
+                                                 wgt * __uint_as_float(a0[4 * v + 3]));
+#pragma unroll
+                        for (int v = 0; v < 4; ++v)
+                            dst[4 + v] = make_float4(wgt * __uint_as_float(a1[4 * v]),
+                                                     wgt * __uint_as_float(a1[4 * v + 1]),
+                                                     wgt * __uint_as_float(a1[4 * v + 2]),
+                                                     wgt * __uint_as_float(a1[4 * v + 3]));
+                    }
+                }
+            }
+            tc_fence_before_sync();
+            mbar_arrive(&c.acc_empty[acc]);
+            if (++acc == 2) {
+                acc = 0;
+                acc_ph ^= 1u;
+            }
+        }
+    }
+
+    tc_fence_before_sync();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after_sync();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+}  // namespace gemm
+}  // namespace moe

@@ -1,0 +1,490 @@
+// moe.cu -- the C ABI declared in include/moe.h: argument validation,
+// workspace planning, TMA descriptor encoding and kernel launches.  All
+// device code is included here so the library is one translation unit.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "moe.h"
+
+#include "status.cuh"
+#include "ptx.cuh"
+#include "route.cuh"
+#include "permute.cuh"
+#include "grouped_gemm.cuh"
+#include "combine.cuh"
+
+namespace {
+
+// ------------------------------------------------------------ self test
+__global__ void wait_timeout_kernel(unsigned long long limit_ns)
+{
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        moe::mbar_init(&bar, 1);
+        moe::fence_mbar_init();
+    }
+    __syncthreads();
+    // Nothing ever arrives on `bar`: the bounded wait must give up.
+    if (threadIdx.x == 0) moe::mbar_wait(&bar, 0, limit_ns);
+    __syncthreads();
+}
+
+// ------------------------------------------------------ per-device state
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceState {
+    bool init = false;
+    bool supported = false;
+    int sm_count = 0;
+};
+
+std::mutex g_mu;
+DeviceState g_dev[kMaxDevices];
+EncodeTiledFn g_encode = nullptr;
+
+constexpr int kMaxDynSmem = 227 * 1024;
+
+int setup_device(DeviceState** out)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MOE_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_mu);
+    DeviceState& st = g_dev[dev];
+    if (!st.init) {
+        int major = 0, minor = 0, sms = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        st.supported = (major == 10 && minor == 0);
+        st.sm_count = sms;
+        if (st.supported) {
+            if (!g_encode) {
+                void* fn = nullptr;
+                cudaDriverEntryPointQueryResult q;
+                if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault, &q) !=
+                        cudaSuccess ||
+                    q != cudaDriverEntryPointSuccess || !fn)
+                    return MOE_ERR_CUDA;
+                g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+            }
+            cudaError_t e = cudaSuccess;
+            e = e ? e : cudaFuncSetAttribute(moe::route::route_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
+            e = e ? e : cudaFuncSetAttribute(moe::route::route_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
+            e = e ? e : cudaFuncSetAttribute(moe::route::route_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
+            e = e ? e : cudaFuncSetAttribute(moe::route::route_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
+            e = e ? e : cudaFuncSetAttribute(moe::route::route_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
+            e = e ? e : cudaFuncSetAttribute(moe::route::route_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
+            e = e ? e : cudaFuncSetAttribute(moe::gemm::grouped_gemm_kernel<moe::gemm::kSwiGLU>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
+            e = e ? e : cudaFuncSetAttribute(moe::gemm::grouped_gemm_kernel<moe::gemm::kWeighted>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
+            if (e != cudaSuccess) return MOE_ERR_CUDA;
+        }
+        st.init = true;
+    }
+    if (!st.supported) return MOE_ERR_UNSUPPORTED_DEVICE;
+    *out = &st;
+    return MOE_OK;
+}
+
+// ------------------------------------------------------------ validation
+inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+int check_common(int64_t T, int64_t d, int64_t E, int64_t k)
+{
+    if (T < 0 || d <= 0 || E <= 0 || k <= 0) return MOE_ERR_INVALID_ARG;
+    if (d % 64 != 0 || d > 32768) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (E % 8 != 0 || E < 8 || E > moe::gemm::kMaxE) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (k > E || k > 32) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (T * k >= (int64_t(1) << 31)) return MOE_ERR_UNSUPPORTED_SHAPE;
+    return MOE_OK;
+}
+
+int check_f(int64_t f)
+{
+    if (f <= 0) return MOE_ERR_INVALID_ARG;
+    if (f % 64 != 0 || f > 65536) return MOE_ERR_UNSUPPORTED_SHAPE;
+    return MOE_OK;
+}
+
+int launch_status()
+{
+    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+// 2-D bf16 tensor map, 128-byte swizzle, zero fill outside the tensor.
+int make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner,
+             uint32_t box_outer)
+{
+    cuuint64_t dims[2] = {inner, outer};
+    cuuint64_t strides[1] = {inner * 2};
+    cuuint32_t box[2] = {box_inner, box_outer};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
+}
+
+inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+inline int64_t permute_chunks(int64_t n) { return (n + moe::permute::kChunk - 1) / moe::permute::kChunk; }
+
+size_t permute_ws_bytes(int64_t T, int64_t E, int64_t k)
+{
+    return align256((size_t)permute_chunks(T * k) * (size_t)E * 4);
+}
+
+// Workspace carve-up for moe_forward.
+struct Layout {
+    size_t ids, wts, counts, offsets, chunk, perm, inv, w_perm, x_perm, h, y, total;
+};
+
+Layout plan(int64_t T, int64_t d, int64_t E, int64_t k, int64_t f)
+{
+    const size_t M = (size_t)(T * k);
+    Layout L{};
+    size_t o = 0;
+    L.ids = o;     o += align256(M * 4);
+    L.wts = o;     o += align256(M * 4);
+    L.counts = o;  o += align256((size_t)E * 4);
+    L.offsets = o; o += align256((size_t)(E + 1) * 4);
+    L.chunk = o;   o += permute_ws_bytes(T, E, k);
+    L.perm = o;    o += align256(M * 4);
+    L.inv = o;     o += align256(M * 4);
+    L.w_perm = o;  o += align256(M * 4);
+    L.x_perm = o;  o += align256(M * (size_t)d * 2);
+    L.h = o;       o += align256(M * (size_t)f * 2);
+    L.y = o;       o += align256(M * (size_t)d * 4);
+    L.total = o;
+    return L;
+}
+
+// ------------------------------------------------------------ launchers
+int run_route(const DeviceState& st, const moe_bf16* x, const moe_bf16* w_router, const float* bias, int64_t T,
+              int64_t d, int64_t E, int64_t k, int32_t* ids, float* wts, cudaStream_t s)
+{
+    (void)st;
+    if (T == 0) return MOE_OK;
+    CUtensorMap tx, tw;
+    int rc = make_map(&tx, x, (uint64_t)d, (uint64_t)T, 64, moe::route::kBM);
+    if (rc) return rc;
+    rc = make_map(&tw, w_router, (uint64_t)E, (uint64_t)d, 64, 64);
+    if (rc) return rc;
+    moe::route::Params p;
+    p.bias = bias;
+    p.ids = ids;
+    p.wts = wts;
+    p.T = (int)T;
+    p.d = (int)d;
+    p.E = (int)E;
+    p.k = (int)k;
+    p.n_chunks = (int)((E + 63) / 64);
+    const int sb = moe::route::stage_bytes(p.n_chunks);
+    p.stages = 4;
+    while (p.stages > 2 && moe::route::smem_bytes(p.n_chunks, p.stages, (int)E) > (size_t)kMaxDynSmem) --p.stages;
+    uint32_t cols = 64;
+    while (cols < (uint32_t)(64 * p.n_chunks)) cols <<= 1;
+    p.tmem_cols = cols;
+    (void)sb;
+    const size_t smem = moe::route::smem_bytes(p.n_chunks, p.stages, (int)E);
+    const dim3 grid((unsigned)((T + moe::route::kBM - 1) / moe::route::kBM));
+    const dim3 block(moe::route::kThreads);
+    int kmax = 1;
+    while (kmax < k) kmax <<= 1;
+    switch (kmax) {
+        case 1: moe::route::route_kernel<1><<<grid, block, smem, s>>>(tx, tw, p); break;
+        case 2: moe::route::route_kernel<2><<<grid, block, smem, s>>>(tx, tw, p); break;
+        case 4: moe::route::route_kernel<4><<<grid, block, smem, s>>>(tx, tw, p); break;
+        case 8: moe::route::route_kernel<8><<<grid, block, smem, s>>>(tx, tw, p); break;
+        case 16: moe::route::route_kernel<16><<<grid, block, smem, s>>>(tx, tw, p); break;
+        default: moe::route::route_kernel<32><<<grid, block, smem, s>>>(tx, tw, p); break;
+    }
+    return launch_status();
+}
+
+int run_permute(const moe_bf16* x, const int32_t* ids, const float* wts, int64_t T, int64_t d, int64_t E,
+                int64_t k, int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* inv, moe_bf16* x_perm,
+                float* w_perm, int32_t* chunk, cudaStream_t s)
+{
+    const int64_t n = T * k;
+    if (n == 0) {
+        // Empty batch: every group is empty.
+        if (cudaMemsetAsync(counts, 0, (size_t)E * 4, s) != cudaSuccess) return MOE_ERR_CUDA;
+        if (cudaMemsetAsync(offsets, 0, (size_t)(E + 1) * 4, s) != cudaSuccess) return MOE_ERR_CUDA;
+        return MOE_OK;
+    }
+    using namespace moe::permute;
+    const int nchunks = (int)permute_chunks(n);
+    hist_kernel<<<nchunks, kThreads, (size_t)E * 4, s>>>(ids, n, (int)E, chunk);
+    scan_kernel<<<1, kScanThreads, 0, s>>>(chunk, nchunks, (int)E, counts, offsets);
+    rank_kernel<<<nchunks, kThreads, (size_t)kWarps * E * 4, s>>>(ids, wts, n, (int)E, chunk, perm, inv, w_perm);
+    if (x_perm) {
+        const unsigned blocks = (unsigned)((n + kWarps - 1) / kWarps);
+        gather_kernel<<<blocks, kThreads, 0, s>>>(reinterpret_cast<const uint4*>(x), perm, n, (int)(d / 8), (int)k,
+                                                  reinterpret_cast<uint4*>(x_perm));
+    }
+    return launch_status();
+}
+
+int run_ffn(const DeviceState& st, const moe_bf16* x_perm, const float* w_perm, const int32_t* offsets,
+            const moe_bf16* w_gate, const moe_bf16* w_up, const moe_bf16* w_down, int64_t M, int64_t d, int64_t E,
+            int64_t f, moe_bf16* h, float* y, cudaStream_t s, cudaEvent_t mid_event)
+{
+    if (M == 0) {
+        if (mid_event && cudaEventRecord(mid_event, s) != cudaSuccess) return MOE_ERR_CUDA;
+        return MOE_OK;
+    }
+    using namespace moe::gemm;
+    CUtensorMap ta1, tg, tu, ta2, td;
+    int rc = make_map(&ta1, x_perm, (uint64_t)d, (uint64_t)M, 64, kBM);
+    rc = rc ? rc : make_map(&tg, w_gate, (uint64_t)f, (uint64_t)(E * d), 64, 64);
+    rc = rc ? rc : make_map(&tu, w_up, (uint64_t)f, (uint64_t)(E * d), 64, 64);
+    rc = rc ? rc : make_map(&ta2, h, (uint64_t)f, (uint64_t)M, 64, kBM);
+    rc = rc ? rc : make_map(&td, w_down, (uint64_t)d, (uint64_t)(E * f), 64, 64);
+    if (rc) return rc;
+    const size_t smem = smem_bytes();
+    const int64_t max_mtiles = (M + kBM - 1) / kBM + E;
+
+    Params p1;
+    p1.offsets = offsets;
+    p1.w_perm = nullptr;
+    p1.out = h;
+    p1.E = (int)E;
+    p1.M = (int)M;
+    p1.K = (int)d;
+    p1.n_out = (int)f;
+    p1.n_tiles = (int)((f + 127) / 128);
+    const int64_t work1 = max_mtiles * p1.n_tiles;
+    const unsigned grid1 = (unsigned)(work1 < st.sm_count ? work1 : st.sm_count);
+    grouped_gemm_kernel<kSwiGLU><<<grid1, kThreads, smem, s>>>(ta1, tg, tu, p1);
+    if (launch_status()) return MOE_ERR_CUDA;
+    if (mid_event && cudaEventRecord(mid_event, s) != cudaSuccess) return MOE_ERR_CUDA;
+
+    Params p2;
+    p2.offsets = offsets;
+    p2.w_perm = w_perm;
+    p2.out = y;
+    p2.E = (int)E;
+    p2.M = (int)M;
+    p2.K = (int)f;
+    p2.n_out = (int)d;
+    p2.n_tiles = (int)((d + kBN - 1) / kBN);
+    const int64_t work2 = max_mtiles * p2.n_tiles;
+    const unsigned grid2 = (unsigned)(work2 < st.sm_count ? work2 : st.sm_count);
+    grouped_gemm_kernel<kWeighted><<<grid2, kThreads, smem, s>>>(ta2, td, td, p2);
+    return launch_status();
+}
+
+int run_combine(const float* y, const int32_t* inv, int64_t T, int64_t d, int64_t k, float* out, cudaStream_t s)
+{
+    if (T == 0) return MOE_OK;
+    const int nvec = (int)(d / 4);
+    const int threads = nvec < 256 ? ((nvec + 31) / 32) * 32 : 256;
+    moe::combine::combine_kernel<<<(unsigned)T, threads, 0, s>>>(reinterpret_cast<const float4*>(y), inv, T * k,
+                                                                 nvec, (int)k, reinterpret_cast<float4*>(out));
+    return launch_status();
+}
+
+int forward_impl(const moe_bf16* x, const moe_bf16* w_router, const float* bias, const moe_bf16* w_gate,
+                 const moe_bf16* w_up, const moe_bf16* w_down, int64_t T, int64_t d, int64_t E, int64_t k, int64_t f,
+                 float* out, int32_t* ids_out, float* w_out, void* ws, size_t ws_bytes, cudaStream_t s,
+                 cudaEvent_t* ev, int n_ev)
+{
+    int rc = check_common(T, d, E, k);
+    if (rc) return rc;
+    if ((rc = check_f(f))) return rc;
+    if (!x || !w_router || !w_gate || !w_up || !w_down || !out) return MOE_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(w_router, 16) || !aligned(w_gate, 16) || !aligned(w_up, 16) ||
+        !aligned(w_down, 16) || !aligned(out, 16) || !aligned(bias, 4) || !aligned(ids_out, 4) ||
+        !aligned(w_out, 4))
+        return MOE_ERR_INVALID_ARG;
+    if (ev && n_ev < 6) return MOE_ERR_INVALID_ARG;
+    const Layout L = plan(T, d, E, k, f);
+    if (T > 0 && (!ws || !aligned(ws, 256))) return MOE_ERR_INVALID_ARG;
+    if (ws_bytes < L.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
+    DeviceState* st = nullptr;
+    if ((rc = setup_device(&st))) return rc;
+    auto rec = [&](int i) { return (ev && cudaEventRecord(ev[i], s) != cudaSuccess) ? MOE_ERR_CUDA : MOE_OK; };
+    if ((rc = rec(0))) return rc;
+    if (T == 0) {
+        for (int i = 1; i < 6; ++i)
+            if ((rc = rec(i))) return rc;
+        return MOE_OK;
+    }
+    uint8_t* w = static_cast<uint8_t*>(ws);
+    int32_t* ids = ids_out ? ids_out : reinterpret_cast<int32_t*>(w + L.ids);
+    float* wts = w_out ? w_out : reinterpret_cast<float*>(w + L.wts);
+    int32_t* counts = reinterpret_cast<int32_t*>(w + L.counts);
+    int32_t* offsets = reinterpret_cast<int32_t*>(w + L.offsets);
+    int32_t* chunk = reinterpret_cast<int32_t*>(w + L.chunk);
+    int32_t* perm = reinterpret_cast<int32_t*>(w + L.perm);
+    int32_t* inv = reinterpret_cast<int32_t*>(w + L.inv);
+    float* w_perm = reinterpret_cast<float*>(w + L.w_perm);
+    moe_bf16* x_perm = reinterpret_cast<moe_bf16*>(w + L.x_perm);
+    moe_bf16* h = reinterpret_cast<moe_bf16*>(w + L.h);
+    float* y = reinterpret_cast<float*>(w + L.y);
+
+    if ((rc = run_route(*st, x, w_router, bias, T, d, E, k, ids, wts, s))) return rc;
+    if ((rc = rec(1))) return rc;
+    if ((rc = run_permute(x, ids, wts, T, d, E, k, counts, offsets, perm, inv, x_perm, w_perm, chunk, s))) return rc;
+    if ((rc = rec(2))) return rc;
+    if ((rc = run_ffn(*st, x_perm, w_perm, offsets, w_gate, w_up, w_down, T * k, d, E, f, h, y, s,
+                      ev ? ev[3] : nullptr)))
+        return rc;
+    if ((rc = rec(4))) return rc;
+    if ((rc = run_combine(y, inv, T, d, k, out, s))) return rc;
+    return rec(5);
+}
+
+}  // namespace
+
+// ===================================================================== ABI
+extern "C" {
+
+const char* moe_strerror(int status)
+{
+    switch (status) {
+        case MOE_OK: return "MOE_OK";
+        case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG: null or misaligned pointer, or negative size";
+        case MOE_ERR_UNSUPPORTED_SHAPE: return "MOE_ERR_UNSUPPORTED_SHAPE: shape outside the supported limits";
+        case MOE_ERR_WORKSPACE_TOO_SMALL: return "MOE_ERR_WORKSPACE_TOO_SMALL";
+        case MOE_ERR_CUDA: return "MOE_ERR_CUDA: a CUDA call or kernel launch failed";
+        case MOE_ERR_DEVICE_TIMEOUT: return "MOE_ERR_DEVICE_TIMEOUT: a device pipeline wait ran past its limit";
+        case MOE_ERR_DEVICE_BOUNDS: return "MOE_ERR_DEVICE_BOUNDS: index data out of range on the device";
+        case MOE_ERR_UNSUPPORTED_DEVICE: return "MOE_ERR_UNSUPPORTED_DEVICE: needs a compute capability 10.0 GPU";
+        default: return "unknown moe status";
+    }
+}
+
+int moe_version(void) { return 100; }
+
+size_t moe_workspace_size(int64_t T, int64_t d, int64_t E, int64_t k, int64_t f)
+{
+    if (check_common(T, d, E, k) || check_f(f)) return 0;
+    return plan(T, d, E, k, f).total;
+}
+
+size_t moe_permute_workspace_size(int64_t T, int64_t E, int64_t k)
+{
+    if (T < 0 || E <= 0 || k <= 0 || E > moe::gemm::kMaxE || k > E) return 0;
+    return permute_ws_bytes(T, E, k);
+}
+
+int moe_route(const moe_bf16* x, const moe_bf16* w_router, const float* bias, int64_t T, int64_t d, int64_t E,
+              int64_t k, int32_t* topk_ids, float* topk_w, cudaStream_t stream)
+{
+    int rc = check_common(T, d, E, k);
+    if (rc) return rc;
+    if (!x || !w_router || !topk_ids || !topk_w) return MOE_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(w_router, 16) || !aligned(bias, 4) || !aligned(topk_ids, 4) ||
+        !aligned(topk_w, 4))
+        return MOE_ERR_INVALID_ARG;
+    DeviceState* st = nullptr;
+    if ((rc = setup_device(&st))) return rc;
+    return run_route(*st, x, w_router, bias, T, d, E, k, topk_ids, topk_w, stream);
+}
+
+int moe_permute(const moe_bf16* x, const int32_t* topk_ids, const float* topk_w, int64_t T, int64_t d, int64_t E,
+                int64_t k, int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* inv, moe_bf16* x_perm,
+                float* w_perm, void* workspace, size_t workspace_bytes, cudaStream_t stream)
+{
+    int rc = check_common(T, d, E, k);
+    if (rc) return rc;
+    if (!topk_ids || !topk_w || !counts || !offsets || !perm || !inv || !w_perm) return MOE_ERR_INVALID_ARG;
+    if (x_perm && !x) return MOE_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(x_perm, 16) || !aligned(topk_ids, 4) || !aligned(topk_w, 4) ||
+        !aligned(counts, 4) || !aligned(offsets, 4) || !aligned(perm, 4) || !aligned(inv, 4) || !aligned(w_perm, 4))
+        return MOE_ERR_INVALID_ARG;
+    const size_t need = permute_ws_bytes(T, E, k);
+    if (workspace_bytes < need) return MOE_ERR_WORKSPACE_TOO_SMALL;
+    if (T > 0 && (!workspace || !aligned(workspace, 4))) return MOE_ERR_INVALID_ARG;
+    DeviceState* st = nullptr;
+    if ((rc = setup_device(&st))) return rc;
+    return run_permute(x, topk_ids, topk_w, T, d, E, k, counts, offsets, perm, inv, x_perm, w_perm,
+                       static_cast<int32_t*>(workspace), stream);
+}
+
+int moe_expert_ffn(const moe_bf16* x_perm, const float* w_perm, const int32_t* offsets, const moe_bf16* w_gate,
+                   const moe_bf16* w_up, const moe_bf16* w_down, int64_t M, int64_t d, int64_t E, int64_t f,
+                   moe_bf16* h, float* y, cudaStream_t stream)
+{
+    if (M < 0 || d <= 0 || E <= 0) return MOE_ERR_INVALID_ARG;
+    int rc = check_common(M, d, E, 1);
+    if (rc) return rc;
+    if ((rc = check_f(f))) return rc;
+    if (!x_perm || !w_perm || !offsets || !w_gate || !w_up || !w_down || !h || !y) return MOE_ERR_INVALID_ARG;
+    if (!aligned(x_perm, 16) || !aligned(w_gate, 16) || !aligned(w_up, 16) || !aligned(w_down, 16) ||
+        !aligned(h, 16) || !aligned(y, 16) || !aligned(w_perm, 4) || !aligned(offsets, 4))
+        return MOE_ERR_INVALID_ARG;
+    DeviceState* st = nullptr;
+    if ((rc = setup_device(&st))) return rc;
+    return run_ffn(*st, x_perm, w_perm, offsets, w_gate, w_up, w_down, M, d, E, f, h, y, stream, nullptr);
+}
+
+int moe_combine(const float* y, const int32_t* inv, int64_t T, int64_t d, int64_t k, float* out,
+                cudaStream_t stream)
+{
+    if (T < 0 || d <= 0 || k <= 0) return MOE_ERR_INVALID_ARG;
+    if (d % 64 != 0 || d > 32768 || k > 32 || T * k >= (int64_t(1) << 31)) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (!y || !inv || !out) return MOE_ERR_INVALID_ARG;
+    if (!aligned(y, 16) || !aligned(out, 16) || !aligned(inv, 4)) return MOE_ERR_INVALID_ARG;
+    DeviceState* st = nullptr;
+    int rc = setup_device(&st);
+    if (rc) return rc;
+    return run_combine(y, inv, T, d, k, out, stream);
+}
+
+int moe_forward(const moe_bf16* x, const moe_bf16* w_router, const float* bias, const moe_bf16* w_gate,
+                const moe_bf16* w_up, const moe_bf16* w_down, int64_t T, int64_t d, int64_t E, int64_t k, int64_t f,
+                float* out, int32_t* topk_ids_out, float* topk_w_out, void* workspace, size_t workspace_bytes,
+                cudaStream_t stream)
+{
+    return forward_impl(x, w_router, bias, w_gate, w_up, w_down, T, d, E, k, f, out, topk_ids_out, topk_w_out,
+                        workspace, workspace_bytes, stream, nullptr, 0);
+}
+
+int moe_forward_profiled(const moe_bf16* x, const moe_bf16* w_router, const float* bias, const moe_bf16* w_gate,
+                         const moe_bf16* w_up, const moe_bf16* w_down, int64_t T, int64_t d, int64_t E, int64_t k,
+                         int64_t f, float* out, int32_t* topk_ids_out, float* topk_w_out, void* workspace,
+                         size_t workspace_bytes, cudaStream_t stream, cudaEvent_t* events, int n_events)
+{
+    if (!events) return MOE_ERR_INVALID_ARG;
+    return forward_impl(x, w_router, bias, w_gate, w_up, w_down, T, d, E, k, f, out, topk_ids_out, topk_w_out,
+                        workspace, workspace_bytes, stream, events, n_events);
+}
+
+int moe_get_status(cudaStream_t stream)
+{
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return MOE_ERR_CUDA;
+    int v = 0;
+    const int zero = 0;
+    if (cudaMemcpyFromSymbol(&v, moe::g_status, sizeof(int)) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cudaMemcpyToSymbol(moe::g_status, &zero, sizeof(int)) != cudaSuccess) return MOE_ERR_CUDA;
+    return v;
+}
+
+int moe_set_wait_limit_ns(int64_t limit_ns)
+{
+    const unsigned long long v = limit_ns > 0 ? (unsigned long long)limit_ns : 1000000000ull;
+    return cudaMemcpyToSymbol(moe::g_wait_limit_ns, &v, sizeof(v)) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+int moe_selftest_wait_timeout(int64_t limit_ns, cudaStream_t stream)
+{
+    if (limit_ns <= 0 || limit_ns > 10000000000ll) return MOE_ERR_INVALID_ARG;
+    DeviceState* st = nullptr;
+    int rc = setup_device(&st);
+    if (rc) return rc;
+    wait_timeout_kernel<<<1, 32, 0, stream>>>((unsigned long long)limit_ns);
+    return launch_status();
+}
+
+}  // extern "C"
