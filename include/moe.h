@@ -83,7 +83,8 @@ int moe_version(void);
  * Bytes of scratch that moe_forward needs for these sizes (0 if the shape is
  * unsupported).  The pieces, each 256-byte aligned, are: topk ids and
  * weights [M], counts [E], offsets [E+1], per-chunk group bases, perm / inv /
- * w_perm [M], x_perm [M,d] bf16, h [M,f] bf16 and y [M,d] fp32.
+ * w_perm [M], h [M,f] bf16 and y [M,d] fp32.  (moe_forward never builds
+ * x_perm: its gate/up GEMM gathers the rows of x through perm directly.)
  */
 size_t moe_workspace_size(int64_t T, int64_t d, int64_t E, int64_t k, int64_t f);
 

@@ -20,20 +20,28 @@
 //
 // Warp roles (192 threads):
 //   warp 0       TMA producer: A [128 rows x 64 k] K-major, B 4 x [64 k x 64 n]
-//                (weights are [K, N] with N contiguous: MN-major operand)
+//                (weights are [K, N] with N contiguous: MN-major operand).
+//                With GATHER, the A rows are fetched straight from the token
+//                matrix x through the permutation (row pos -> token
+//                perm[pos] / k) with tile::gather4 loads, one per lane, so
+//                the permuted copy of x is never written.
 //   warp 1       TMEM allocation + single-thread tcgen05.mma issuer,
 //                M=128 N=256 K=16 per instruction, fp32 accumulators
 //   warps 2..5   epilogue: tcgen05.ld of the 128 x 256 accumulator, one row
-//                per thread, fused math, bf16 stores
+//                per thread, fused math, stores
 // Two accumulator buffers (2 x 256 TMEM columns) let the epilogue of one
 // tile overlap the MMAs of the next.
 //
 // Epilogues:
 //   kSwiGLU   : B columns 0..127 come from W_gate, 128..255 from W_up for the
-//               same 128 output columns; h = silu(g) * u, silu(z) = z/(1+e^-z)
+//               same 128 output columns; h = silu(g) * u, silu(z) = z/(1+e^-z),
+//               stored as bf16 (h is the next GEMM's bf16 operand)
 //   kWeighted : y = w_perm[row] * acc in fp32 (the routing weight applied
 //               after the down projection; y stays fp32 so that the k-way sum
-//               in the combine is an fp32 accumulation of unrounded terms)
+//               in the combine is an fp32 accumulation of unrounded terms).
+//               Each warp stages 32 rows x 16 columns in shared memory and
+//               writes them with one TMA store, so global writes are whole
+//               64-byte row segments instead of per-thread scattered stores.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -54,21 +62,26 @@ constexpr int kBBytes = 4 * kChunkBytes;    // 32 KB
 constexpr int kStageBytes = kABytes + kBBytes;
 constexpr uint32_t kTmemCols = 512;         // 2 accumulators x 256 columns
 constexpr int kMaxE = 512;
+constexpr int kSlabCols = 16;               // fp32 columns per TMA-store slab (64 B rows)
+constexpr int kSlabBytes = 32 * kSlabCols * 4;     // 32 rows x 16 fp32 = 2 KB
+constexpr int kStoreBytes = 4 * 2 * kSlabBytes;    // 4 epilogue warps x 2 buffers
 
 enum EpiKind { kSwiGLU = 0, kWeighted = 1 };
 
 struct Params {
     const int32_t* offsets;  // [E+1] group boundaries (device)
     const float* w_perm;     // [M] routing weight per grouped row (kWeighted)
+    const int32_t* perm;     // [M] grouped row -> flat assignment t*k + j (GATHER)
     void* out;               // [M, n_out]: bf16 h (kSwiGLU) or fp32 y (kWeighted)
     int E;
-    int M;        // rows of A
+    int M;        // grouped rows
     int K;        // reduction length (multiple of 64)
     int n_out;    // output columns (multiple of 64)
     int n_tiles;  // N tiles per M tile
+    int k_top;    // experts per token (GATHER: token = perm[row] / k_top)
 };
 
-// Shared memory after the stage ring.
+// Shared memory after the stage ring and the store staging buffers.
 struct alignas(8) Ctrl {
     uint64_t full[kStages];
     uint64_t empty[kStages];
@@ -83,7 +96,7 @@ struct alignas(8) Ctrl {
     int tp[kMaxE + 1];    // exclusive prefix of M tiles per group
 };
 
-__host__ inline size_t smem_bytes() { return 1024 + (size_t)kStages * kStageBytes + sizeof(Ctrl); }
+__host__ inline size_t smem_bytes() { return 1024 + (size_t)kStages * kStageBytes + kStoreBytes + sizeof(Ctrl); }
 
 // Work item -> (expert, first row, group end, N tile).
 __device__ __forceinline__ void decode(int64_t w, int n_tiles, const Ctrl& c, int E, int& e, int& row0,
@@ -112,14 +125,29 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b)
 
 __device__ __forceinline__ float silu(float z) { return z / (1.0f + __expf(-z)); }
 
-template <int EPI>
+// Token row of x for grouped row r (clamped into range; rows past the group
+// end only feed accumulator rows that are never stored).
+__device__ __forceinline__ int gather_token(const Params& p, int r)
+{
+    r = r < p.M ? r : p.M - 1;
+    int a = __ldg(p.perm + r);
+    if ((unsigned)a >= (unsigned)p.M) {
+        record_status(kStatusDeviceBounds);
+        a = 0;
+    }
+    return a / p.k_top;
+}
+
+template <int EPI, bool GATHER>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b0,
-                        const __grid_constant__ CUtensorMap tm_b1, Params p)
+                        const __grid_constant__ CUtensorMap tm_b1, const __grid_constant__ CUtensorMap tm_out,
+                        Params p)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    Ctrl& c = *reinterpret_cast<Ctrl*>(smem + (size_t)kStages * kStageBytes);
+    uint8_t* stage_out = smem + (size_t)kStages * kStageBytes;
+    Ctrl& c = *reinterpret_cast<Ctrl*>(stage_out + kStoreBytes);
 
     const int warp = threadIdx.x / 32;
     const int lane = threadIdx.x % 32;
@@ -172,6 +200,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_prefetch_map(&tm_a);
         tma_prefetch_map(&tm_b0);
         if (EPI == kSwiGLU) tma_prefetch_map(&tm_b1);
+        if (EPI == kWeighted) tma_prefetch_map(&tm_out);
     }
     if (warp == 1) {
         __syncwarp();
@@ -186,25 +215,40 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int num_kb = p.K / kBK;
 
     if (warp == 0) {
-        if (lane == 0) {
-            // ------------------------------------------------ TMA producer
-            int s = 0;
-            uint32_t ph = 0;
-            int64_t issued = 0;
-            for (int64_t w = blockIdx.x; w < total_work && !c.abort_flag; w += gridDim.x) {
-                int e, row0, row_end, nt;
-                decode(w, p.n_tiles, c, E, e, row0, row_end, nt);
-                const int krow0 = e * p.K;
-                bool ok = true;
-                for (int kb = 0; kb < num_kb; ++kb) {
-                    if (!mbar_wait(&c.empty[s], ph ^ 1u, limit)) {
-                        ok = false;
-                        break;
-                    }
-                    uint8_t* sa = smem + (size_t)s * kStageBytes;
-                    uint8_t* sb = sa + kABytes;
-                    mbar_arrive_expect_tx(&c.full[s], (uint32_t)kStageBytes);
-                    tma_load_2d(sa, &tm_a, &c.full[s], kb * kBK, row0);
+        // ---------------------------------------------------- TMA producer
+        int s = 0;
+        uint32_t ph = 0;
+        int64_t issued = 0;
+        for (int64_t w = blockIdx.x; w < total_work; w += gridDim.x) {
+            if (__shfl_sync(0xffffffffu, c.abort_flag, 0)) break;  // warp-uniform exit
+            int e, row0, row_end, nt;
+            decode(w, p.n_tiles, c, E, e, row0, row_end, nt);
+            int tok0 = 0, tok1 = 0, tok2 = 0, tok3 = 0;
+            if (GATHER) {
+                tok0 = gather_token(p, row0 + lane * 4 + 0);
+                tok1 = gather_token(p, row0 + lane * 4 + 1);
+                tok2 = gather_token(p, row0 + lane * 4 + 2);
+                tok3 = gather_token(p, row0 + lane * 4 + 3);
+            }
+            const int krow0 = e * p.K;
+            bool ok = true;
+            for (int kb = 0; kb < num_kb; ++kb) {
+                bool ready = true;
+                if (lane == 0) ready = mbar_wait(&c.empty[s], ph ^ 1u, limit);
+                if (!__shfl_sync(0xffffffffu, ready ? 1 : 0, 0)) {
+                    ok = false;
+                    break;
+                }
+                uint8_t* sa = smem + (size_t)s * kStageBytes;
+                uint8_t* sb = sa + kABytes;
+                if (lane == 0) mbar_arrive_expect_tx(&c.full[s], (uint32_t)kStageBytes);
+                __syncwarp();
+                if (GATHER) {
+                    // lane l brings tile rows 4l .. 4l+3 (128 B each)
+                    tma_gather4(sa + lane * 4 * 128, &tm_a, &c.full[s], kb * kBK, tok0, tok1, tok2, tok3);
+                }
+                if (lane == 0) {
+                    if (!GATHER) tma_load_2d(sa, &tm_a, &c.full[s], kb * kBK, row0);
                     const int kr = krow0 + kb * kBK;
                     if (EPI == kSwiGLU) {
                         const int n0 = nt * 128;
@@ -218,18 +262,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                         for (int q = 0; q < 4; ++q)
                             tma_load_2d(sb + q * kChunkBytes, &tm_b0, &c.full[s], n0 + 64 * q, kr);
                     }
-                    ++issued;
-                    if (++s == kStages) {
-                        s = 0;
-                        ph ^= 1u;
-                    }
                 }
-                if (!ok) {
-                    c.abort_flag = 1;
-                    break;
+                ++issued;
+                if (++s == kStages) {
+                    s = 0;
+                    ph ^= 1u;
                 }
             }
-            // Never leave the CTA with a copy still landing in its shared memory.
+            if (!ok) {
+                if (lane == 0) c.abort_flag = 1;
+                break;
+            }
+        }
+        // Never leave the CTA with a copy still landing in its shared memory.
+        if (lane == 0) {
             for (int q = 0; q < kStages; ++q) {
                 const int64_t cnt = issued / kStages + (q < issued % kStages ? 1 : 0);
                 if (cnt > 0) mbar_wait(&c.full[q], (uint32_t)(cnt - 1) & 1u, limit);
@@ -290,6 +336,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ---------------------------------------------------- epilogue
         const int q = warp & 3;          // TMEM lane quarter this warp may access
         const int r = q * 32 + lane;     // tile row owned by this thread
+        float* slab = reinterpret_cast<float*>(stage_out + q * 2 * kSlabBytes);
+        int slab_buf = 0;
         int acc = 0;
         uint32_t acc_ph = 0;
         for (int64_t w = blockIdx.x; w < total_work; w += gridDim.x) {
@@ -331,27 +379,42 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             } else {
                 const float wgt = valid ? __ldg(p.w_perm + row) : 0.0f;
+                const int wrow0 = row0 + q * 32;                   // first row of this warp's slab
+                const bool whole = wrow0 + 31 < row_end;           // all 32 rows belong to the group
                 float* orow = static_cast<float*>(p.out) + (int64_t)row * p.n_out + nt * kBN;
                 const int ncols = min(kBN, p.n_out - nt * kBN);
 #pragma unroll 1
-                for (int c0 = 0; c0 < kBN; c0 += 32) {
-                    uint32_t a0[16], a1[16];
-                    tmem_ld16(tbase + c0, a0);
-                    tmem_ld16(tbase + c0 + 16, a1);
+                for (int c0 = 0; c0 < kBN; c0 += kSlabCols) {
+                    uint32_t a[16];
+                    tmem_ld16(tbase + c0, a);
                     tmem_ld_wait();
-                    if (valid && c0 < ncols) {
+                    if (c0 >= ncols) continue;  // warp-uniform
+                    if (whole) {
+                        float* buf = slab + slab_buf * (kSlabBytes / 4);
+                        if (lane == 0) bulk_wait_group_read<1>();  // the store that last read `buf` is done
+                        __syncwarp();
+                        // row `lane` of the slab: 4 x 16 B chunks, 64-byte swizzle
+                        float4* rowp = reinterpret_cast<float4*>(buf + lane * kSlabCols);
+                        const int sw = (lane >> 1) & 3;
+#pragma unroll
+                        for (int v = 0; v < 4; ++v)
+                            rowp[v ^ sw] = make_float4(wgt * __uint_as_float(a[4 * v]), wgt * __uint_as_float(a[4 * v + 1]),
+                                                       wgt * __uint_as_float(a[4 * v + 2]),
+                                                       wgt * __uint_as_float(a[4 * v + 3]));
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) {
+                            tma_store_2d(&tm_out, buf, nt * kBN + c0, wrow0);
+                            bulk_commit_group();
+                        }
+                        slab_buf ^= 1;
+                    } else if (valid) {
                         float4* dst = reinterpret_cast<float4*>(orow + c0);
 #pragma unroll
                         for (int v = 0; v < 4; ++v)
-                            dst[v] = make_float4(wgt * __uint_as_float(a0[4 * v]), wgt * __uint_as_float(a0[4 * v + 1]),
-                                                 wgt * __uint_as_float(a0[4 * v + 2]),
-                                                 wgt * __uint_as_float(a0[4 * v + 3]));
-#pragma unroll
-                        for (int v = 0; v < 4; ++v)
-                            dst[4 + v] = make_float4(wgt * __uint_as_float(a1[4 * v]),
-                                                     wgt * __uint_as_float(a1[4 * v + 1]),
-                                                     wgt * __uint_as_float(a1[4 * v + 2]),
-                                                     wgt * __uint_as_float(a1[4 * v + 3]));
+                            dst[v] = make_float4(wgt * __uint_as_float(a[4 * v]), wgt * __uint_as_float(a[4 * v + 1]),
+                                                 wgt * __uint_as_float(a[4 * v + 2]),
+                                                 wgt * __uint_as_float(a[4 * v + 3]));
                     }
                 }
             }
@@ -362,6 +425,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 acc_ph ^= 1u;
             }
         }
+        if (EPI == kWeighted && lane == 0) bulk_wait_group_all();
+        __syncwarp();
     }
 
     tc_fence_before_sync();

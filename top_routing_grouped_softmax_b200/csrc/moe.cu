@@ -83,8 +83,9 @@ int setup_device(DeviceState** out)
             e = e ? e : cudaFuncSetAttribute(moe::route::route_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
             e = e ? e : cudaFuncSetAttribute(moe::route::route_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
             e = e ? e : cudaFuncSetAttribute(moe::route::route_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
-            e = e ? e : cudaFuncSetAttribute(moe::gemm::grouped_gemm_kernel<moe::gemm::kSwiGLU>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
-            e = e ? e : cudaFuncSetAttribute(moe::gemm::grouped_gemm_kernel<moe::gemm::kWeighted>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
+            e = e ? e : cudaFuncSetAttribute(moe::gemm::grouped_gemm_kernel<moe::gemm::kSwiGLU, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
+            e = e ? e : cudaFuncSetAttribute(moe::gemm::grouped_gemm_kernel<moe::gemm::kSwiGLU, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
+            e = e ? e : cudaFuncSetAttribute(moe::gemm::grouped_gemm_kernel<moe::gemm::kWeighted, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
             if (e != cudaSuccess) return MOE_ERR_CUDA;
         }
         st.init = true;
@@ -119,17 +120,19 @@ int launch_status()
     return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
-// 2-D bf16 tensor map, 128-byte swizzle, zero fill outside the tensor.
+// 2-D row-major tensor map, zero fill outside the tensor.  Default: bf16
+// with 128-byte swizzle (the layout the tcgen05 descriptors expect).
 int make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint32_t box_inner,
-             uint32_t box_outer)
+             uint32_t box_outer, CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+             uint32_t elem_bytes = 2, CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B)
 {
     cuuint64_t dims[2] = {inner, outer};
-    cuuint64_t strides[1] = {inner * 2};
+    cuuint64_t strides[1] = {inner * elem_bytes};
     cuuint32_t box[2] = {box_inner, box_outer};
     cuuint32_t estr[2] = {1, 1};
-    CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    CUresult r = g_encode(m, dtype, 2, const_cast<void*>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
 }
 
@@ -144,7 +147,7 @@ size_t permute_ws_bytes(int64_t T, int64_t E, int64_t k)
 
 // Workspace carve-up for moe_forward.
 struct Layout {
-    size_t ids, wts, counts, offsets, chunk, perm, inv, w_perm, x_perm, h, y, total;
+    size_t ids, wts, counts, offsets, chunk, perm, inv, w_perm, h, y, total;
 };
 
 Layout plan(int64_t T, int64_t d, int64_t E, int64_t k, int64_t f)
@@ -160,7 +163,6 @@ Layout plan(int64_t T, int64_t d, int64_t E, int64_t k, int64_t f)
     L.perm = o;    o += align256(M * 4);
     L.inv = o;     o += align256(M * 4);
     L.w_perm = o;  o += align256(M * 4);
-    L.x_perm = o;  o += align256(M * (size_t)d * 2);
     L.h = o;       o += align256(M * (size_t)f * 2);
     L.y = o;       o += align256(M * (size_t)d * 4);
     L.total = o;
@@ -234,21 +236,29 @@ int run_permute(const moe_bf16* x, const int32_t* ids, const float* wts, int64_t
     return launch_status();
 }
 
-int run_ffn(const DeviceState& st, const moe_bf16* x_perm, const float* w_perm, const int32_t* offsets,
-            const moe_bf16* w_gate, const moe_bf16* w_up, const moe_bf16* w_down, int64_t M, int64_t d, int64_t E,
-            int64_t f, moe_bf16* h, float* y, cudaStream_t s, cudaEvent_t mid_event)
+// The two grouped GEMMs.  With x_gather/perm set, the gate/up GEMM reads its
+// A rows straight from x through perm (row pos -> token perm[pos] / k) and
+// x_perm is not used.
+int run_ffn(const DeviceState& st, const moe_bf16* x_perm, const moe_bf16* x_gather, const int32_t* perm,
+            int64_t T, int64_t k, const float* w_perm, const int32_t* offsets, const moe_bf16* w_gate,
+            const moe_bf16* w_up, const moe_bf16* w_down, int64_t M, int64_t d, int64_t E, int64_t f, moe_bf16* h,
+            float* y, cudaStream_t s, cudaEvent_t mid_event)
 {
     if (M == 0) {
         if (mid_event && cudaEventRecord(mid_event, s) != cudaSuccess) return MOE_ERR_CUDA;
         return MOE_OK;
     }
     using namespace moe::gemm;
-    CUtensorMap ta1, tg, tu, ta2, td;
-    int rc = make_map(&ta1, x_perm, (uint64_t)d, (uint64_t)M, 64, kBM);
+    const bool gather = x_gather != nullptr;
+    CUtensorMap ta1, tg, tu, ta2, td, ty;
+    int rc = gather ? make_map(&ta1, x_gather, (uint64_t)d, (uint64_t)T, 64, 1)
+                    : make_map(&ta1, x_perm, (uint64_t)d, (uint64_t)M, 64, kBM);
     rc = rc ? rc : make_map(&tg, w_gate, (uint64_t)f, (uint64_t)(E * d), 64, 64);
     rc = rc ? rc : make_map(&tu, w_up, (uint64_t)f, (uint64_t)(E * d), 64, 64);
     rc = rc ? rc : make_map(&ta2, h, (uint64_t)f, (uint64_t)M, 64, kBM);
     rc = rc ? rc : make_map(&td, w_down, (uint64_t)d, (uint64_t)(E * f), 64, 64);
+    rc = rc ? rc : make_map(&ty, y, (uint64_t)d, (uint64_t)M, kSlabCols, 32, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4,
+                            CU_TENSOR_MAP_SWIZZLE_64B);
     if (rc) return rc;
     const size_t smem = smem_bytes();
     const int64_t max_mtiles = (M + kBM - 1) / kBM + E;
@@ -256,30 +266,37 @@ int run_ffn(const DeviceState& st, const moe_bf16* x_perm, const float* w_perm, 
     Params p1;
     p1.offsets = offsets;
     p1.w_perm = nullptr;
+    p1.perm = perm;
     p1.out = h;
     p1.E = (int)E;
     p1.M = (int)M;
     p1.K = (int)d;
     p1.n_out = (int)f;
     p1.n_tiles = (int)((f + 127) / 128);
+    p1.k_top = (int)k;
     const int64_t work1 = max_mtiles * p1.n_tiles;
     const unsigned grid1 = (unsigned)(work1 < st.sm_count ? work1 : st.sm_count);
-    grouped_gemm_kernel<kSwiGLU><<<grid1, kThreads, smem, s>>>(ta1, tg, tu, p1);
+    if (gather)
+        grouped_gemm_kernel<kSwiGLU, true><<<grid1, kThreads, smem, s>>>(ta1, tg, tu, ty, p1);
+    else
+        grouped_gemm_kernel<kSwiGLU, false><<<grid1, kThreads, smem, s>>>(ta1, tg, tu, ty, p1);
     if (launch_status()) return MOE_ERR_CUDA;
     if (mid_event && cudaEventRecord(mid_event, s) != cudaSuccess) return MOE_ERR_CUDA;
 
     Params p2;
     p2.offsets = offsets;
     p2.w_perm = w_perm;
+    p2.perm = nullptr;
     p2.out = y;
     p2.E = (int)E;
     p2.M = (int)M;
     p2.K = (int)f;
     p2.n_out = (int)d;
     p2.n_tiles = (int)((d + kBN - 1) / kBN);
+    p2.k_top = 1;
     const int64_t work2 = max_mtiles * p2.n_tiles;
     const unsigned grid2 = (unsigned)(work2 < st.sm_count ? work2 : st.sm_count);
-    grouped_gemm_kernel<kWeighted><<<grid2, kThreads, smem, s>>>(ta2, td, td, p2);
+    grouped_gemm_kernel<kWeighted, false><<<grid2, kThreads, smem, s>>>(ta2, td, td, ty, p2);
     return launch_status();
 }
 
@@ -301,7 +318,7 @@ int forward_impl(const moe_bf16* x, const moe_bf16* w_router, const float* bias,
     int rc = check_common(T, d, E, k);
     if (rc) return rc;
     if ((rc = check_f(f))) return rc;
-    if (!x || !w_router || !w_gate || !w_up || !w_down || !out) return MOE_ERR_INVALID_ARG;
+    if (T > 0 && (!x || !w_router || !w_gate || !w_up || !w_down || !out)) return MOE_ERR_INVALID_ARG;
     if (!aligned(x, 16) || !aligned(w_router, 16) || !aligned(w_gate, 16) || !aligned(w_up, 16) ||
         !aligned(w_down, 16) || !aligned(out, 16) || !aligned(bias, 4) || !aligned(ids_out, 4) ||
         !aligned(w_out, 4))
@@ -328,15 +345,17 @@ int forward_impl(const moe_bf16* x, const moe_bf16* w_router, const float* bias,
     int32_t* perm = reinterpret_cast<int32_t*>(w + L.perm);
     int32_t* inv = reinterpret_cast<int32_t*>(w + L.inv);
     float* w_perm = reinterpret_cast<float*>(w + L.w_perm);
-    moe_bf16* x_perm = reinterpret_cast<moe_bf16*>(w + L.x_perm);
     moe_bf16* h = reinterpret_cast<moe_bf16*>(w + L.h);
     float* y = reinterpret_cast<float*>(w + L.y);
 
     if ((rc = run_route(*st, x, w_router, bias, T, d, E, k, ids, wts, s))) return rc;
     if ((rc = rec(1))) return rc;
-    if ((rc = run_permute(x, ids, wts, T, d, E, k, counts, offsets, perm, inv, x_perm, w_perm, chunk, s))) return rc;
+    // The grouped rows of x are never materialised: the gate/up GEMM gathers
+    // them from x through perm as it loads its operand tiles.
+    if ((rc = run_permute(x, ids, wts, T, d, E, k, counts, offsets, perm, inv, nullptr, w_perm, chunk, s)))
+        return rc;
     if ((rc = rec(2))) return rc;
-    if ((rc = run_ffn(*st, x_perm, w_perm, offsets, w_gate, w_up, w_down, T * k, d, E, f, h, y, s,
+    if ((rc = run_ffn(*st, nullptr, x, perm, T, k, w_perm, offsets, w_gate, w_up, w_down, T * k, d, E, f, h, y, s,
                       ev ? ev[3] : nullptr)))
         return rc;
     if ((rc = rec(4))) return rc;
@@ -383,7 +402,7 @@ int moe_route(const moe_bf16* x, const moe_bf16* w_router, const float* bias, in
 {
     int rc = check_common(T, d, E, k);
     if (rc) return rc;
-    if (!x || !w_router || !topk_ids || !topk_w) return MOE_ERR_INVALID_ARG;
+    if (T > 0 && (!x || !w_router || !topk_ids || !topk_w)) return MOE_ERR_INVALID_ARG;
     if (!aligned(x, 16) || !aligned(w_router, 16) || !aligned(bias, 4) || !aligned(topk_ids, 4) ||
         !aligned(topk_w, 4))
         return MOE_ERR_INVALID_ARG;
@@ -398,7 +417,8 @@ int moe_permute(const moe_bf16* x, const int32_t* topk_ids, const float* topk_w,
 {
     int rc = check_common(T, d, E, k);
     if (rc) return rc;
-    if (!topk_ids || !topk_w || !counts || !offsets || !perm || !inv || !w_perm) return MOE_ERR_INVALID_ARG;
+    if (!counts || !offsets) return MOE_ERR_INVALID_ARG;
+    if (T > 0 && (!topk_ids || !topk_w || !perm || !inv || !w_perm)) return MOE_ERR_INVALID_ARG;
     if (x_perm && !x) return MOE_ERR_INVALID_ARG;
     if (!aligned(x, 16) || !aligned(x_perm, 16) || !aligned(topk_ids, 4) || !aligned(topk_w, 4) ||
         !aligned(counts, 4) || !aligned(offsets, 4) || !aligned(perm, 4) || !aligned(inv, 4) || !aligned(w_perm, 4))
@@ -420,13 +440,15 @@ int moe_expert_ffn(const moe_bf16* x_perm, const float* w_perm, const int32_t* o
     int rc = check_common(M, d, E, 1);
     if (rc) return rc;
     if ((rc = check_f(f))) return rc;
-    if (!x_perm || !w_perm || !offsets || !w_gate || !w_up || !w_down || !h || !y) return MOE_ERR_INVALID_ARG;
+    if (M > 0 && (!x_perm || !w_perm || !offsets || !w_gate || !w_up || !w_down || !h || !y))
+        return MOE_ERR_INVALID_ARG;
     if (!aligned(x_perm, 16) || !aligned(w_gate, 16) || !aligned(w_up, 16) || !aligned(w_down, 16) ||
         !aligned(h, 16) || !aligned(y, 16) || !aligned(w_perm, 4) || !aligned(offsets, 4))
         return MOE_ERR_INVALID_ARG;
     DeviceState* st = nullptr;
     if ((rc = setup_device(&st))) return rc;
-    return run_ffn(*st, x_perm, w_perm, offsets, w_gate, w_up, w_down, M, d, E, f, h, y, stream, nullptr);
+    return run_ffn(*st, x_perm, nullptr, nullptr, 0, 1, w_perm, offsets, w_gate, w_up, w_down, M, d, E, f, h, y,
+                   stream, nullptr);
 }
 
 int moe_combine(const float* y, const int32_t* inv, int64_t T, int64_t d, int64_t k, float* out,
@@ -434,7 +456,7 @@ int moe_combine(const float* y, const int32_t* inv, int64_t T, int64_t d, int64_
 {
     if (T < 0 || d <= 0 || k <= 0) return MOE_ERR_INVALID_ARG;
     if (d % 64 != 0 || d > 32768 || k > 32 || T * k >= (int64_t(1) << 31)) return MOE_ERR_UNSUPPORTED_SHAPE;
-    if (!y || !inv || !out) return MOE_ERR_INVALID_ARG;
+    if (T > 0 && (!y || !inv || !out)) return MOE_ERR_INVALID_ARG;
     if (!aligned(y, 16) || !aligned(out, 16) || !aligned(inv, 4)) return MOE_ERR_INVALID_ARG;
     DeviceState* st = nullptr;
     int rc = setup_device(&st);
