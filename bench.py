@@ -38,6 +38,8 @@ UNIT = "tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_FLUSH_BYTES = 256 << 20
 STAGES = ("route", "permute", "gateup_gemm", "down_gemm", "combine")
+# router GEMM, softmax/top-k, chunk scan, rank, row gather, gate/up GEMM, down GEMM, combine
+KERNELS_PER_FORWARD = 8
 
 
 # ------------------------------------------------------------- host logic
@@ -226,8 +228,36 @@ def run_gpu(args, cfg):
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
-    def step(events=None):
-        blk(x, out=out, topk_ids=ids, events=events)
+    if args.path == "stages":
+        # the four ABI stages called one by one (x_perm materialised)
+        st_ids = torch.empty(cfg.T, cfg.k, dtype=torch.int32, device=dev)
+        st_w = torch.empty(cfg.T, cfg.k, dtype=torch.float32, device=dev)
+        st_h = torch.empty(cfg.T * cfg.k, cfg.f, dtype=torch.bfloat16, device=dev)
+        st_y = torch.empty(cfg.T * cfg.k, cfg.d, dtype=torch.float32, device=dev)
+
+        def step(events=None):
+            if events:
+                events[0].record()
+            moe.route(x, w["W_router"], cfg.k, bias=bias, topk_ids=st_ids, topk_w=st_w)
+            if events:
+                events[1].record()
+            pm = moe.permute(x, st_ids, st_w, cfg.E)
+            if events:
+                events[2].record()
+            h_, y_ = moe.expert_ffn(pm["x_perm"], pm["w_perm"], pm["offsets"], w["W_gate"], w["W_up"],
+                                    w["W_down"], h=st_h, y=st_y)
+            if events:
+                events[4].record()
+                events[3].record()  # gate/up and down are not split on this path
+            moe.combine(y_, pm["inv"], cfg.T, cfg.k, out=out)
+            if events:
+                events[5].record()
+            ids.copy_(st_ids)
+    else:
+        flags = moe.MOE_FLAG_FUSED_GATHER if args.gather else 0
+
+        def step(events=None):
+            blk(x, out=out, topk_ids=ids, events=events, flags=flags)
 
     for _ in range(args.warmup):
         step()
@@ -329,7 +359,7 @@ def run_gpu(args, cfg):
                         "tile_padding": padding},
             "e2e": {"value": whole_job_rate(cfg.T * args.steps, world, [e2e_s]), "unit": UNIT,
                     "h2d_bytes_per_step": cfg.T * cfg.d * 2, "d2h_bytes_per_step": cfg.T * cfg.d * 4},
-            "gpu_launches": 8 * args.steps,
+            "gpu_launches": KERNELS_PER_FORWARD * args.steps,
             "clocks": clocks,
             "wall_s_timed_region": wall,
         }
@@ -345,6 +375,10 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default="qwen")
+    ap.add_argument("--path", choices=("fused", "stages"), default="fused",
+                    help="fused: moe_forward; stages: moe_route/permute/expert_ffn/combine one by one")
+    ap.add_argument("--gather", action="store_true",
+                    help="fused path: the gate/up GEMM gathers x rows itself (MOE_FLAG_FUSED_GATHER)")
     ap.add_argument("--cpu-tokens", type=int, default=384,
                     help="tokens of the workload the CPU-oracle baseline leg evaluates")
     ap.add_argument("--ref-tokens", type=int, default=32, help="tokens per step of the reference arm")

@@ -88,7 +88,10 @@ int moe_version(void);
  */
 size_t moe_workspace_size(int64_t T, int64_t d, int64_t E, int64_t k, int64_t f);
 
-/* Bytes of scratch that moe_permute needs (per-chunk group bases). */
+/* Bytes of scratch that moe_route needs (fp32 partial router logits). */
+size_t moe_route_workspace_size(int64_t T, int64_t d, int64_t E);
+
+/* Bytes of scratch that moe_permute needs (per-chunk expert counts). */
 size_t moe_permute_workspace_size(int64_t T, int64_t E, int64_t k);
 
 /*
@@ -99,13 +102,17 @@ size_t moe_permute_workspace_size(int64_t T, int64_t E, int64_t k);
  *   bias     [E]       fp32, or NULL for no bias
  *   topk_ids [T, k]    int32 out, slot j = j-th largest probability
  *   topk_w   [T, k]    fp32  out, the softmax probability of that expert
- * Logits are accumulated in fp32 on the tensor cores and never rounded to
- * bf16.  Selection compares the fp32 logits (softmax is monotone); ties go
- * to the lower expert index.
+ *   workspace          device scratch of moe_route_workspace_size bytes,
+ *                      16-byte aligned
+ * Logits are accumulated in fp32 on the tensor cores (in a few slices of the
+ * hidden dimension, summed in a fixed order) and never rounded to bf16.
+ * Selection compares the fp32 logits (softmax is monotone); ties go to the
+ * lower expert index.
  */
 int moe_route(const moe_bf16* x, const moe_bf16* w_router, const float* bias,
               int64_t T, int64_t d, int64_t E, int64_t k,
-              int32_t* topk_ids, float* topk_w, cudaStream_t stream);
+              int32_t* topk_ids, float* topk_w,
+              void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /*
  * Token reordering by expert (section 2.2: sort_tokens_by_expert, then
@@ -174,18 +181,25 @@ int moe_forward(const moe_bf16* x, const moe_bf16* w_router, const float* bias,
                 float* out, int32_t* topk_ids_out, float* topk_w_out,
                 void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
+/* moe_forward_ex flag: the gate/up GEMM gathers its operand rows from x
+ * through the permutation while it loads them, instead of reading a
+ * materialised x_perm.  Same results bit for bit. */
+#define MOE_FLAG_FUSED_GATHER 1u
+
 /*
- * moe_forward that also records n_events (>= 6) caller-created CUDA events
- * on `stream`: before routing, after routing, after the permutation, after
- * the gate/up GEMM, after the down GEMM and after the combine.  For timing
- * individual stages; the arithmetic is identical to moe_forward.
+ * moe_forward with options.  events (may be NULL): n_events >= 6
+ * caller-created CUDA events recorded on `stream` before routing, after
+ * routing, after the permutation, after the gate/up GEMM, after the down
+ * GEMM and after the combine, for timing stages.  flags: 0 or
+ * MOE_FLAG_FUSED_GATHER (other bits: MOE_ERR_INVALID_ARG).  The arithmetic
+ * is identical to moe_forward.
  */
-int moe_forward_profiled(const moe_bf16* x, const moe_bf16* w_router, const float* bias,
-                         const moe_bf16* w_gate, const moe_bf16* w_up, const moe_bf16* w_down,
-                         int64_t T, int64_t d, int64_t E, int64_t k, int64_t f,
-                         float* out, int32_t* topk_ids_out, float* topk_w_out,
-                         void* workspace, size_t workspace_bytes, cudaStream_t stream,
-                         cudaEvent_t* events, int n_events);
+int moe_forward_ex(const moe_bf16* x, const moe_bf16* w_router, const float* bias,
+                   const moe_bf16* w_gate, const moe_bf16* w_up, const moe_bf16* w_down,
+                   int64_t T, int64_t d, int64_t E, int64_t k, int64_t f,
+                   float* out, int32_t* topk_ids_out, float* topk_w_out,
+                   void* workspace, size_t workspace_bytes, cudaStream_t stream,
+                   cudaEvent_t* events, int n_events, unsigned flags);
 
 /*
  * Synchronises `stream`, then returns and clears the current device's status

@@ -48,25 +48,33 @@ def test_workspace_sizes(moe_lib):
     assert moe.workspace_size(8192, 2000, 128, 8, 768) == 0      # d % 64 != 0
     assert moe.workspace_size(8192, 2048, 128, 33, 768) == 0     # k > 32
     assert moe.workspace_size(0, 2048, 128, 8, 768) > 0
-    assert moe.permute_workspace_size(8192, 128, 8) == 16 * 128 * 4
+    assert moe.permute_workspace_size(8192, 128, 8) == (8192 // 64) * 128 * 4
+    assert moe.route_workspace_size(8192, 2048, 128) % 256 == 0
+    assert moe.route_workspace_size(8192, 2048, 128) >= 8192 * 128 * 4
+    assert moe.route_workspace_size(8192, 2048, 12) == 0
 
 
 def test_validation_happens_before_any_device_call(moe_lib):
     L = moe_lib
     null = ctypes.c_void_p(0)
     # null pointers
-    assert L.moe_route(null, null, null, 16, 64, 8, 2, null, null, null) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_route(null, null, null, 16, 64, 8, 2, null, null, null, 0, null) == moe.MOE_ERR_INVALID_ARG
     # unsupported shapes are rejected before pointers are even looked at
-    assert L.moe_route(null, null, null, 16, 64, 12, 2, null, null, null) == moe.MOE_ERR_UNSUPPORTED_SHAPE
-    assert L.moe_route(null, null, null, 16, 64, 8, 9, null, null, null) == moe.MOE_ERR_UNSUPPORTED_SHAPE
-    assert L.moe_route(null, null, null, -1, 64, 8, 2, null, null, null) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_route(null, null, null, 16, 64, 12, 2, null, null, null, 0, null) == moe.MOE_ERR_UNSUPPORTED_SHAPE
+    assert L.moe_route(null, null, null, 16, 64, 8, 9, null, null, null, 0, null) == moe.MOE_ERR_UNSUPPORTED_SHAPE
+    assert L.moe_route(null, null, null, -1, 64, 8, 2, null, null, null, 0, null) == moe.MOE_ERR_INVALID_ARG
     # misaligned (odd) pointer
     odd = ctypes.c_void_p(0x1001)
-    assert L.moe_route(odd, odd, null, 16, 64, 8, 2, odd, odd, null) == moe.MOE_ERR_INVALID_ARG
+    assert L.moe_route(odd, odd, null, 16, 64, 8, 2, odd, odd, odd, 1 << 20, null) == moe.MOE_ERR_INVALID_ARG
+    fake = ctypes.c_void_p(0x10000)
+    assert L.moe_route(fake, fake, null, 16, 64, 8, 2, fake, fake, fake, 16, null) == \
+        moe.MOE_ERR_WORKSPACE_TOO_SMALL
+    # unknown flag bits
+    assert L.moe_forward_ex(fake, fake, null, fake, fake, fake, 16, 64, 8, 2, 64, fake, null, null, fake, 1 << 30,
+                            null, null, 0, 6) == moe.MOE_ERR_INVALID_ARG
     assert L.moe_combine(null, null, 4, 64, 2, null, null) == moe.MOE_ERR_INVALID_ARG
     assert L.moe_combine(null, null, 4, 65, 2, null, null) == moe.MOE_ERR_UNSUPPORTED_SHAPE
     # workspace too small is caught on the host
-    fake = ctypes.c_void_p(0x10000)
     assert L.moe_forward(fake, fake, null, fake, fake, fake, 16, 64, 8, 2, 64, fake, null, null, fake, 16,
                          null) == moe.MOE_ERR_WORKSPACE_TOO_SMALL
 

@@ -19,11 +19,14 @@ SMALL = [
 ]
 
 
-def _forward(cfg, d):
+VARIANTS = {"x_perm": 0, "fused_gather": moe.MOE_FLAG_FUSED_GATHER}
+
+
+def _forward(cfg, d, flags=0):
     ids = torch.empty(cfg.T, cfg.k, dtype=torch.int32, device="cuda")
     w = torch.empty(cfg.T, cfg.k, dtype=torch.float32, device="cuda")
     out = moe.forward(d["x"], d["w_router"], d["w_gate"], d["w_up"], d["w_down"], cfg.k, bias=d["bias"],
-                      topk_ids=ids, topk_w=w)
+                      topk_ids=ids, topk_w=w, flags=flags)
     torch.cuda.synchronize()
     assert moe.get_status() == moe.MOE_OK
     return out, ids, w
@@ -37,12 +40,22 @@ def _check(cfg, out, ids, w, rows, ref_out):
     return value_check(got[keep], ref_out[keep], f"out[{cfg.name}]"), stats
 
 
+@pytest.mark.parametrize("variant", list(VARIANTS))
 @pytest.mark.parametrize("cfg", SMALL, ids=lambda c: c.name)
-def test_forward_small_all_tokens(cfg):
+def test_forward_small_all_tokens(cfg, variant):
     d = gc.on_device(gc.inputs(cfg))
-    out, ids, w = _forward(cfg, d)
+    out, ids, w = _forward(cfg, d, VARIANTS[variant])
     rows, ref = gc.oracle_rows(cfg, cfg.T)
     _check(cfg, out, ids, w, rows, ref)
+
+
+def test_forward_full_size_fused_gather_matches_default():
+    """The fused-gather variant on the Qwen3-shaped layer: bit-identical to the default."""
+    cfg = gc.FULL[1]
+    d = gc.on_device(gc.inputs(cfg))
+    a, _, _ = _forward(cfg, d, 0)
+    b, _, _ = _forward(cfg, d, moe.MOE_FLAG_FUSED_GATHER)
+    assert torch.equal(a, b)
 
 
 @pytest.mark.parametrize("cfg", gc.FULL, ids=lambda c: c.name)
@@ -54,10 +67,11 @@ def test_forward_full_size_sampled(cfg):
     print(cfg.name, "sampled", len(rows), "max/rms", mx, "mean_rel", mean, stats)
 
 
-def test_forward_equals_stages_bitwise():
+@pytest.mark.parametrize("variant", list(VARIANTS))
+def test_forward_equals_stages_bitwise(variant):
     cfg = gc.small_cfg(1000, 256, 16, 4, 320, skew=True)
     d = gc.on_device(gc.inputs(cfg))
-    out, ids, w = _forward(cfg, d)
+    out, ids, w = _forward(cfg, d, VARIANTS[variant])
     ids2, w2 = moe.route(d["x"], d["w_router"], cfg.k, bias=d["bias"])
     pm = moe.permute(d["x"], ids2, w2, cfg.E)
     h, y = moe.expert_ffn(pm["x_perm"], pm["w_perm"], pm["offsets"], d["w_gate"], d["w_up"], d["w_down"])

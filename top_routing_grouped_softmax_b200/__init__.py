@@ -33,9 +33,9 @@ MOE_ERR_UNSUPPORTED_DEVICE = 7
 
 # Every symbol include/moe.h declares.
 ABI_SYMBOLS = (
-    "moe_strerror", "moe_version", "moe_workspace_size", "moe_permute_workspace_size",
-    "moe_route", "moe_permute", "moe_expert_ffn", "moe_combine", "moe_forward",
-    "moe_forward_profiled", "moe_get_status", "moe_set_wait_limit_ns", "moe_selftest_wait_timeout",
+    "moe_strerror", "moe_version", "moe_workspace_size", "moe_route_workspace_size",
+    "moe_permute_workspace_size", "moe_route", "moe_permute", "moe_expert_ffn", "moe_combine", "moe_forward",
+    "moe_forward_ex", "moe_get_status", "moe_set_wait_limit_ns", "moe_selftest_wait_timeout",
 )
 
 
@@ -67,19 +67,21 @@ def lib() -> ctypes.CDLL:
         L.moe_version.restype = ctypes.c_int
         L.moe_workspace_size.restype = _SZ
         L.moe_workspace_size.argtypes = [_I64] * 5
+        L.moe_route_workspace_size.restype = _SZ
+        L.moe_route_workspace_size.argtypes = [_I64] * 3
         L.moe_permute_workspace_size.restype = _SZ
         L.moe_permute_workspace_size.argtypes = [_I64] * 3
-        L.moe_route.argtypes = [_P, _P, _P, _I64, _I64, _I64, _I64, _P, _P, _P]
+        L.moe_route.argtypes = [_P, _P, _P, _I64, _I64, _I64, _I64, _P, _P, _P, _SZ, _P]
         L.moe_permute.argtypes = [_P, _P, _P, _I64, _I64, _I64, _I64, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]
         L.moe_expert_ffn.argtypes = [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _P, _P, _P]
         L.moe_combine.argtypes = [_P, _P, _I64, _I64, _I64, _P, _P]
         L.moe_forward.argtypes = [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64, _P, _P, _P, _P, _SZ, _P]
-        L.moe_forward_profiled.argtypes = L.moe_forward.argtypes + [_P, ctypes.c_int]
+        L.moe_forward_ex.argtypes = L.moe_forward.argtypes + [_P, ctypes.c_int, ctypes.c_uint]
         L.moe_get_status.argtypes = [_P]
         L.moe_set_wait_limit_ns.argtypes = [_I64]
         L.moe_selftest_wait_timeout.argtypes = [_I64, _P]
         for name in ("moe_route", "moe_permute", "moe_expert_ffn", "moe_combine", "moe_forward",
-                     "moe_forward_profiled", "moe_get_status", "moe_set_wait_limit_ns",
+                     "moe_forward_ex", "moe_get_status", "moe_set_wait_limit_ns",
                      "moe_selftest_wait_timeout"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
@@ -125,6 +127,10 @@ def workspace_size(T: int, d: int, E: int, k: int, f: int) -> int:
     return int(lib().moe_workspace_size(T, d, E, k, f))
 
 
+def route_workspace_size(T: int, d: int, E: int) -> int:
+    return int(lib().moe_route_workspace_size(T, d, E))
+
+
 def permute_workspace_size(T: int, E: int, k: int) -> int:
     return int(lib().moe_permute_workspace_size(T, E, k))
 
@@ -134,7 +140,7 @@ def _workspace(nbytes: int, device) -> torch.Tensor:
 
 
 # ----------------------------------------------------------------- stages
-def route(x, w_router, k, bias=None, topk_ids=None, topk_w=None):
+def route(x, w_router, k, bias=None, topk_ids=None, topk_w=None, workspace=None):
     """Router GEMM + fp32 softmax + top-k; returns (topk_ids int32 [T,k], topk_w fp32 [T,k])."""
     _need(x, "x", torch.bfloat16, 2)
     _need(w_router, "w_router", torch.bfloat16, 2)
@@ -146,8 +152,13 @@ def route(x, w_router, k, bias=None, topk_ids=None, topk_w=None):
         topk_ids = torch.empty(T, k, dtype=torch.int32, device=x.device)
     if topk_w is None:
         topk_w = torch.empty(T, k, dtype=torch.float32, device=x.device)
+    need = route_workspace_size(T, d, E)
+    if need == 0 and T > 0:
+        raise MoEError(MOE_ERR_UNSUPPORTED_SHAPE, "moe_route_workspace_size")
+    if workspace is None or workspace.numel() < need:
+        workspace = _workspace(need, x.device)
     _check(lib().moe_route(_ptr(x), _ptr(w_router), _ptr(bias), T, d, E, k, _ptr(topk_ids),
-                           _ptr(topk_w), _stream()), "moe_route")
+                           _ptr(topk_w), _ptr(workspace), workspace.numel(), _stream()), "moe_route")
     return topk_ids, topk_w
 
 
@@ -220,13 +231,18 @@ def _forward_args(x, w_router, w_gate, w_up, w_down, bias):
     return T, d, E, f
 
 
+MOE_FLAG_FUSED_GATHER = 1
+
+
 def forward(x, w_router, w_gate, w_up, w_down, k, bias=None, out=None, workspace=None,
-            topk_ids=None, topk_w=None, events=None):
+            topk_ids=None, topk_w=None, events=None, flags=None):
     """The whole MoE block; returns out [T, d] fp32.
 
     ``events`` (optional): a list of >= 6 torch.cuda.Event objects recorded at
     the stage boundaries (before route, after route, after permute, after
-    gate/up, after down, after combine).
+    gate/up, after down, after combine).  ``flags`` (optional):
+    MOE_FLAG_FUSED_GATHER selects the variant whose gate/up GEMM gathers the
+    rows of x itself; both variants give identical results.
     """
     T, d, E, f = _forward_args(x, w_router, w_gate, w_up, w_down, bias)
     if out is None:
@@ -239,15 +255,19 @@ def forward(x, w_router, w_gate, w_up, w_down, k, bias=None, out=None, workspace
         workspace = _workspace(nbytes, x.device)
     args = [_ptr(x), _ptr(w_router), _ptr(bias), _ptr(w_gate), _ptr(w_up), _ptr(w_down), T, d, E, k, f,
             _ptr(out), _ptr(topk_ids), _ptr(topk_w), _ptr(workspace), workspace.numel(), _stream()]
-    if events is None:
+    if events is None and flags is None:
         _check(lib().moe_forward(*args), "moe_forward")
     else:
-        arr = (ctypes.c_void_p * len(events))()
-        for i, ev in enumerate(events):
-            if ev.cuda_event == 0:
-                ev.record()  # the event handle is created lazily by torch
-            arr[i] = ev.cuda_event
-        _check(lib().moe_forward_profiled(*args, arr, len(events)), "moe_forward_profiled")
+        arr = None
+        n = 0
+        if events is not None:
+            arr = (ctypes.c_void_p * len(events))()
+            for i, ev in enumerate(events):
+                if ev.cuda_event == 0:
+                    ev.record()  # the event handle is created lazily by torch
+                arr[i] = ev.cuda_event
+            n = len(events)
+        _check(lib().moe_forward_ex(*args, arr, n, int(flags or 0)), "moe_forward_ex")
     return out
 
 
@@ -280,14 +300,15 @@ class MoEBlock:
             self._ws = _workspace(need, self.w_gate.device)
         return self._ws
 
-    def __call__(self, x, out=None, topk_ids=None, topk_w=None, events=None):
+    def __call__(self, x, out=None, topk_ids=None, topk_w=None, events=None, flags=None):
         return forward(x, self.w_router, self.w_gate, self.w_up, self.w_down, self.k, bias=self.bias,
                        out=out, workspace=self.workspace(x.shape[0]), topk_ids=topk_ids, topk_w=topk_w,
-                       events=events)
+                       events=events, flags=flags)
 
 
 __all__ = [
-    "lib", "strerror", "MoEError", "ABI_SYMBOLS", "workspace_size", "permute_workspace_size", "route",
+    "lib", "strerror", "MoEError", "ABI_SYMBOLS", "workspace_size", "route_workspace_size",
+    "permute_workspace_size", "MOE_FLAG_FUSED_GATHER", "route",
     "permute", "expert_ffn", "combine", "forward", "get_status", "set_wait_limit_ns",
     "selftest_wait_timeout", "MoEBlock",
 ]

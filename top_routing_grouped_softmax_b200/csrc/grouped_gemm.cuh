@@ -23,8 +23,13 @@
 //                (weights are [K, N] with N contiguous: MN-major operand).
 //                With GATHER, the A rows are fetched straight from the token
 //                matrix x through the permutation (row pos -> token
-//                perm[pos] / k) with tile::gather4 loads, one per lane, so
-//                the permuted copy of x is never written.
+//                perm[pos] / k): the 32 lanes issue 16-byte cp.async copies,
+//                8 lanes per 128-byte row segment so each warp instruction
+//                reads four whole segments, write them in the 128-byte
+//                swizzled layout the MMA expects, and each lane's completion
+//                is counted on the stage barrier.  The permuted copy of x is
+//                never written.  (A tile::gather4 TMA per 4 rows was measured
+//                3x slower here: too many small TMA requests per stage.)
 //   warp 1       TMEM allocation + single-thread tcgen05.mma issuer,
 //                M=128 N=256 K=16 per instruction, fp32 accumulators
 //   warps 2..5   epilogue: tcgen05.ld of the 128 x 256 accumulator, one row
@@ -72,6 +77,8 @@ struct Params {
     const int32_t* offsets;  // [E+1] group boundaries (device)
     const float* w_perm;     // [M] routing weight per grouped row (kWeighted)
     const int32_t* perm;     // [M] grouped row -> flat assignment t*k + j (GATHER)
+    const __nv_bfloat16* x;  // [T, ldx] token matrix the A rows are gathered from (GATHER)
+    int64_t ldx;             // row length of x in elements (= K for the gate/up GEMM)
     void* out;               // [M, n_out]: bf16 h (kSwiGLU) or fp32 y (kWeighted)
     int E;
     int M;        // grouped rows
@@ -94,6 +101,7 @@ struct alignas(8) Ctrl {
     int total_mtiles;
     int off[kMaxE + 1];   // group offsets
     int tp[kMaxE + 1];    // exclusive prefix of M tiles per group
+    int tok[kBM];         // GATHER: token row of x for each row of the current M tile
 };
 
 __host__ inline size_t smem_bytes() { return 1024 + (size_t)kStages * kStageBytes + kStoreBytes + sizeof(Ctrl); }
@@ -187,7 +195,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (threadIdx.x == 32) {
         for (int s = 0; s < kStages; ++s) {
-            mbar_init(&c.full[s], 1);
+            // GATHER: the TMA arrival plus one cp.async completion per lane
+            mbar_init(&c.full[s], GATHER ? 1 + 32 : 1);
             mbar_init(&c.empty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
@@ -214,38 +223,45 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int64_t total_work = c.bad ? 0 : (int64_t)c.total_mtiles * p.n_tiles;
     const int num_kb = p.K / kBK;
 
-    if (warp == 0) {
+    if (warp == 0 && (GATHER || lane == 0)) {
         // ---------------------------------------------------- TMA producer
+        // GATHER: the whole warp (it copies the A rows); otherwise lane 0.
+        constexpr unsigned pmask = GATHER ? 0xffffffffu : 1u;
         int s = 0;
         uint32_t ph = 0;
         int64_t issued = 0;
         for (int64_t w = blockIdx.x; w < total_work; w += gridDim.x) {
-            if (__shfl_sync(0xffffffffu, c.abort_flag, 0)) break;  // warp-uniform exit
+            if (__shfl_sync(pmask, c.abort_flag, 0)) break;  // uniform exit
             int e, row0, row_end, nt;
             decode(w, p.n_tiles, c, E, e, row0, row_end, nt);
-            int tok0 = 0, tok1 = 0, tok2 = 0, tok3 = 0;
             if (GATHER) {
-                tok0 = gather_token(p, row0 + lane * 4 + 0);
-                tok1 = gather_token(p, row0 + lane * 4 + 1);
-                tok2 = gather_token(p, row0 + lane * 4 + 2);
-                tok3 = gather_token(p, row0 + lane * 4 + 3);
+                __syncwarp(pmask);  // every lane is done issuing copies that read c.tok
+#pragma unroll
+                for (int i = 0; i < kBM / 32; ++i) c.tok[lane + 32 * i] = gather_token(p, row0 + lane + 32 * i);
+                __syncwarp(pmask);
             }
             const int krow0 = e * p.K;
             bool ok = true;
             for (int kb = 0; kb < num_kb; ++kb) {
                 bool ready = true;
                 if (lane == 0) ready = mbar_wait(&c.empty[s], ph ^ 1u, limit);
-                if (!__shfl_sync(0xffffffffu, ready ? 1 : 0, 0)) {
+                if (!__shfl_sync(pmask, ready ? 1 : 0, 0)) {
                     ok = false;
                     break;
                 }
                 uint8_t* sa = smem + (size_t)s * kStageBytes;
                 uint8_t* sb = sa + kABytes;
-                if (lane == 0) mbar_arrive_expect_tx(&c.full[s], (uint32_t)kStageBytes);
-                __syncwarp();
+                if (lane == 0) mbar_arrive_expect_tx(&c.full[s], (uint32_t)(GATHER ? kBBytes : kStageBytes));
                 if (GATHER) {
-                    // lane l brings tile rows 4l .. 4l+3 (128 B each)
-                    tma_gather4(sa + lane * 4 * 128, &tm_a, &c.full[s], kb * kBK, tok0, tok1, tok2, tok3);
+                    // lane = 8 * g + ch: 16-byte chunk ch of rows 4i + g, i = 0..31
+                    const int g = lane >> 3, ch = lane & 7;
+                    const __nv_bfloat16* xk = p.x + (size_t)kb * kBK + ch * 8;
+#pragma unroll 8
+                    for (int i = 0; i < kBM / 4; ++i) {
+                        const int r = 4 * i + g;
+                        cp_async_16(sa + r * 128 + ((ch ^ (r & 7)) << 4), xk + (size_t)c.tok[r] * p.ldx);
+                    }
+                    cp_async_arrive_noinc(&c.full[s]);
                 }
                 if (lane == 0) {
                     if (!GATHER) tma_load_2d(sa, &tm_a, &c.full[s], kb * kBK, row0);
@@ -275,13 +291,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
         // Never leave the CTA with a copy still landing in its shared memory.
+        if (GATHER) cp_async_wait_all();
         if (lane == 0) {
             for (int q = 0; q < kStages; ++q) {
                 const int64_t cnt = issued / kStages + (q < issued % kStages ? 1 : 0);
                 if (cnt > 0) mbar_wait(&c.full[q], (uint32_t)(cnt - 1) & 1u, limit);
             }
         }
-        __syncwarp();
+        __syncwarp(pmask);
+    } else if (warp == 0) {
+        // lanes 1..31 of the producer warp have nothing to do without GATHER
     } else if (warp == 1) {
         if (lane == 0) {
             // ------------------------------------------------ MMA issuer

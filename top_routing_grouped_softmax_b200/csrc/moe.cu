@@ -52,6 +52,10 @@ EncodeTiledFn g_encode = nullptr;
 
 constexpr int kMaxDynSmem = 227 * 1024;
 
+// moe_forward's variant: the gate/up GEMM reads a materialised x_perm (the
+// fused row gather measured slower on B200, see MOE_FLAG_FUSED_GATHER).
+constexpr unsigned kDefaultForwardFlags = 0;
+
 int setup_device(DeviceState** out)
 {
     int dev = 0;
@@ -77,12 +81,7 @@ int setup_device(DeviceState** out)
                 g_encode = reinterpret_cast<EncodeTiledFn>(fn);
             }
             cudaError_t e = cudaSuccess;
-            e = e ? e : cudaFuncSetAttribute(moe::route::route_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
-            e = e ? e : cudaFuncSetAttribute(moe::route::route_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
-            e = e ? e : cudaFuncSetAttribute(moe::route::route_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
-            e = e ? e : cudaFuncSetAttribute(moe::route::route_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
-            e = e ? e : cudaFuncSetAttribute(moe::route::route_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
-            e = e ? e : cudaFuncSetAttribute(moe::route::route_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
+            e = e ? e : cudaFuncSetAttribute(moe::route::logits_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
             e = e ? e : cudaFuncSetAttribute(moe::gemm::grouped_gemm_kernel<moe::gemm::kSwiGLU, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
             e = e ? e : cudaFuncSetAttribute(moe::gemm::grouped_gemm_kernel<moe::gemm::kSwiGLU, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
             e = e ? e : cudaFuncSetAttribute(moe::gemm::grouped_gemm_kernel<moe::gemm::kWeighted, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
@@ -138,16 +137,37 @@ int make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, u
 
 inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
-inline int64_t permute_chunks(int64_t n) { return (n + moe::permute::kChunk - 1) / moe::permute::kChunk; }
+// ---------------------------------------------------------- work shapes
+// Router: CTAs own 128 tokens and one of `slices` parts of the hidden
+// dimension.  The split aims at about two CTAs per SM of a 148-SM B200 and
+// keeps at least four 64-wide k-blocks per CTA.  It depends on the shape
+// only, so workspace sizes can be computed without a device.
+constexpr int64_t kRouterTargetCtas = 296;
 
-size_t permute_ws_bytes(int64_t T, int64_t E, int64_t k)
+int router_slices(int64_t T, int64_t d)
 {
-    return align256((size_t)permute_chunks(T * k) * (size_t)E * 4);
+    const int64_t tiles = (T + moe::route::kBM - 1) / moe::route::kBM;
+    const int64_t num_kb = d / moe::route::kBK;
+    int64_t s = tiles > 0 ? kRouterTargetCtas / tiles : 1;
+    int64_t cap = num_kb / 4 > 0 ? num_kb / 4 : 1;
+    if (cap > moe::route::kMaxSlices) cap = moe::route::kMaxSlices;
+    if (s > cap) s = cap;
+    if (s < 1) s = 1;
+    return (int)s;
 }
+
+inline int64_t token_chunks(int64_t T) { return (T + moe::permute::kTokensPerChunk - 1) / moe::permute::kTokensPerChunk; }
+
+size_t route_ws_bytes(int64_t T, int64_t d, int64_t E)
+{
+    return align256((size_t)router_slices(T, d) * (size_t)T * (size_t)E * 4);
+}
+
+size_t permute_ws_bytes(int64_t T, int64_t E) { return align256((size_t)token_chunks(T) * (size_t)E * 4); }
 
 // Workspace carve-up for moe_forward.
 struct Layout {
-    size_t ids, wts, counts, offsets, chunk, perm, inv, w_perm, h, y, total;
+    size_t ids, wts, counts, offsets, chunk, part, perm, inv, w_perm, x_perm, h, y, total;
 };
 
 Layout plan(int64_t T, int64_t d, int64_t E, int64_t k, int64_t f)
@@ -159,10 +179,12 @@ Layout plan(int64_t T, int64_t d, int64_t E, int64_t k, int64_t f)
     L.wts = o;     o += align256(M * 4);
     L.counts = o;  o += align256((size_t)E * 4);
     L.offsets = o; o += align256((size_t)(E + 1) * 4);
-    L.chunk = o;   o += permute_ws_bytes(T, E, k);
+    L.chunk = o;   o += permute_ws_bytes(T, E);
+    L.part = o;    o += route_ws_bytes(T, d, E);
     L.perm = o;    o += align256(M * 4);
     L.inv = o;     o += align256(M * 4);
     L.w_perm = o;  o += align256(M * 4);
+    L.x_perm = o;  o += align256(M * (size_t)d * 2);
     L.h = o;       o += align256(M * (size_t)f * 2);
     L.y = o;       o += align256(M * (size_t)d * 4);
     L.total = o;
@@ -170,10 +192,12 @@ Layout plan(int64_t T, int64_t d, int64_t E, int64_t k, int64_t f)
 }
 
 // ------------------------------------------------------------ launchers
-int run_route(const DeviceState& st, const moe_bf16* x, const moe_bf16* w_router, const float* bias, int64_t T,
-              int64_t d, int64_t E, int64_t k, int32_t* ids, float* wts, cudaStream_t s)
+// Router GEMM (partial logits into `part`) and the softmax / top-k.  With
+// chunk_counts set, the softmax kernel also fills the per-chunk expert
+// histogram the permutation needs.
+int run_route(const moe_bf16* x, const moe_bf16* w_router, const float* bias, int64_t T, int64_t d, int64_t E,
+              int64_t k, int32_t* ids, float* wts, float* part, int32_t* chunk_counts, cudaStream_t s)
 {
-    (void)st;
     if (T == 0) return MOE_OK;
     CUtensorMap tx, tw;
     int rc = make_map(&tx, x, (uint64_t)d, (uint64_t)T, 64, moe::route::kBM);
@@ -181,57 +205,65 @@ int run_route(const DeviceState& st, const moe_bf16* x, const moe_bf16* w_router
     rc = make_map(&tw, w_router, (uint64_t)E, (uint64_t)d, 64, 64);
     if (rc) return rc;
     moe::route::Params p;
-    p.bias = bias;
-    p.ids = ids;
-    p.wts = wts;
+    p.part = part;
     p.T = (int)T;
     p.d = (int)d;
     p.E = (int)E;
-    p.k = (int)k;
     p.n_chunks = (int)((E + 63) / 64);
-    const int sb = moe::route::stage_bytes(p.n_chunks);
+    p.slices = router_slices(T, d);
+    p.zero = chunk_counts;
+    p.zero_count = chunk_counts ? (int64_t)E * token_chunks(T) : 0;
+    // deepest ring that still lets two CTAs share an SM (at least 2 stages)
     p.stages = 4;
-    while (p.stages > 2 && moe::route::smem_bytes(p.n_chunks, p.stages, (int)E) > (size_t)kMaxDynSmem) --p.stages;
+    while (p.stages > 2 && moe::route::smem_bytes(p.n_chunks, p.stages) > (size_t)(113 * 1024)) --p.stages;
     uint32_t cols = 64;
     while (cols < (uint32_t)(64 * p.n_chunks)) cols <<= 1;
     p.tmem_cols = cols;
-    (void)sb;
-    const size_t smem = moe::route::smem_bytes(p.n_chunks, p.stages, (int)E);
-    const dim3 grid((unsigned)((T + moe::route::kBM - 1) / moe::route::kBM));
-    const dim3 block(moe::route::kThreads);
-    int kmax = 1;
-    while (kmax < k) kmax <<= 1;
-    switch (kmax) {
-        case 1: moe::route::route_kernel<1><<<grid, block, smem, s>>>(tx, tw, p); break;
-        case 2: moe::route::route_kernel<2><<<grid, block, smem, s>>>(tx, tw, p); break;
-        case 4: moe::route::route_kernel<4><<<grid, block, smem, s>>>(tx, tw, p); break;
-        case 8: moe::route::route_kernel<8><<<grid, block, smem, s>>>(tx, tw, p); break;
-        case 16: moe::route::route_kernel<16><<<grid, block, smem, s>>>(tx, tw, p); break;
-        default: moe::route::route_kernel<32><<<grid, block, smem, s>>>(tx, tw, p); break;
-    }
+    const size_t smem = moe::route::smem_bytes(p.n_chunks, p.stages);
+    const int64_t tiles = (T + moe::route::kBM - 1) / moe::route::kBM;
+    moe::route::logits_kernel<<<(unsigned)(tiles * p.slices), moe::route::kThreads, smem, s>>>(tx, tw, p);
+    if (launch_status()) return MOE_ERR_CUDA;
+
+    const int64_t nch = token_chunks(T);
+    const size_t hist_smem = 0;
+    const unsigned blocks = (unsigned)((T + moe::route::kSoftmaxWarps - 1) / moe::route::kSoftmaxWarps);
+    const int threads = moe::route::kSoftmaxWarps * 32;
+    const int vpl = (int)((E + 31) / 32);
+    if (vpl <= 1)
+        moe::route::softmax_topk_kernel<1><<<blocks, threads, hist_smem, s>>>(part, bias, (int)T, (int)E, (int)k, p.slices, ids, wts, chunk_counts, (int)nch);
+    else if (vpl <= 2)
+        moe::route::softmax_topk_kernel<2><<<blocks, threads, hist_smem, s>>>(part, bias, (int)T, (int)E, (int)k, p.slices, ids, wts, chunk_counts, (int)nch);
+    else if (vpl <= 4)
+        moe::route::softmax_topk_kernel<4><<<blocks, threads, hist_smem, s>>>(part, bias, (int)T, (int)E, (int)k, p.slices, ids, wts, chunk_counts, (int)nch);
+    else if (vpl <= 8)
+        moe::route::softmax_topk_kernel<8><<<blocks, threads, hist_smem, s>>>(part, bias, (int)T, (int)E, (int)k, p.slices, ids, wts, chunk_counts, (int)nch);
+    else
+        moe::route::softmax_topk_kernel<16><<<blocks, threads, hist_smem, s>>>(part, bias, (int)T, (int)E, (int)k, p.slices, ids, wts, chunk_counts, (int)nch);
     return launch_status();
 }
 
+// Grouping by expert.  have_hist: chunk_em already holds the per-chunk
+// histogram (from the router); otherwise it is computed here.
 int run_permute(const moe_bf16* x, const int32_t* ids, const float* wts, int64_t T, int64_t d, int64_t E,
                 int64_t k, int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* inv, moe_bf16* x_perm,
-                float* w_perm, int32_t* chunk, cudaStream_t s)
+                float* w_perm, int32_t* chunk_em, bool have_hist, cudaStream_t s)
 {
-    const int64_t n = T * k;
-    if (n == 0) {
+    if (T == 0) {
         // Empty batch: every group is empty.
         if (cudaMemsetAsync(counts, 0, (size_t)E * 4, s) != cudaSuccess) return MOE_ERR_CUDA;
         if (cudaMemsetAsync(offsets, 0, (size_t)(E + 1) * 4, s) != cudaSuccess) return MOE_ERR_CUDA;
         return MOE_OK;
     }
     using namespace moe::permute;
-    const int nchunks = (int)permute_chunks(n);
-    hist_kernel<<<nchunks, kThreads, (size_t)E * 4, s>>>(ids, n, (int)E, chunk);
-    scan_kernel<<<1, kScanThreads, 0, s>>>(chunk, nchunks, (int)E, counts, offsets);
-    rank_kernel<<<nchunks, kThreads, (size_t)kWarps * E * 4, s>>>(ids, wts, n, (int)E, chunk, perm, inv, w_perm);
+    const int nch = (int)token_chunks(T);
+    if (!have_hist) hist_kernel<<<nch, kThreads, 0, s>>>(ids, T, (int)k, (int)E, chunk_em, nch);
+    chunk_scan_kernel<<<(unsigned)E, kThreads, 0, s>>>(chunk_em, nch, counts);
+    rank_kernel<<<nch, kThreads, 0, s>>>(ids, wts, T, (int)k, (int)E, chunk_em, nch, counts, offsets, perm, inv,
+                                         w_perm);
     if (x_perm) {
-        const unsigned blocks = (unsigned)((n + kWarps - 1) / kWarps);
-        gather_kernel<<<blocks, kThreads, 0, s>>>(reinterpret_cast<const uint4*>(x), perm, n, (int)(d / 8), (int)k,
-                                                  reinterpret_cast<uint4*>(x_perm));
+        const int64_t n = T * k;
+        gather_kernel<<<(unsigned)((n + kWarps - 1) / kWarps), kThreads, 0, s>>>(
+            reinterpret_cast<const uint4*>(x), perm, n, (int)(d / 8), (int)k, reinterpret_cast<uint4*>(x_perm));
     }
     return launch_status();
 }
@@ -251,7 +283,9 @@ int run_ffn(const DeviceState& st, const moe_bf16* x_perm, const moe_bf16* x_gat
     using namespace moe::gemm;
     const bool gather = x_gather != nullptr;
     CUtensorMap ta1, tg, tu, ta2, td, ty;
-    int rc = gather ? make_map(&ta1, x_gather, (uint64_t)d, (uint64_t)T, 64, 1)
+    // In gather mode the A rows are copied by the producer warp itself; the
+    // A map is unused (the x_perm map is encoded over x only as a placeholder).
+    int rc = gather ? make_map(&ta1, x_gather, (uint64_t)d, (uint64_t)T, 64, kBM)
                     : make_map(&ta1, x_perm, (uint64_t)d, (uint64_t)M, 64, kBM);
     rc = rc ? rc : make_map(&tg, w_gate, (uint64_t)f, (uint64_t)(E * d), 64, 64);
     rc = rc ? rc : make_map(&tu, w_up, (uint64_t)f, (uint64_t)(E * d), 64, 64);
@@ -267,6 +301,8 @@ int run_ffn(const DeviceState& st, const moe_bf16* x_perm, const moe_bf16* x_gat
     p1.offsets = offsets;
     p1.w_perm = nullptr;
     p1.perm = perm;
+    p1.x = reinterpret_cast<const __nv_bfloat16*>(x_gather);
+    p1.ldx = d;
     p1.out = h;
     p1.E = (int)E;
     p1.M = (int)M;
@@ -287,6 +323,8 @@ int run_ffn(const DeviceState& st, const moe_bf16* x_perm, const moe_bf16* x_gat
     p2.offsets = offsets;
     p2.w_perm = w_perm;
     p2.perm = nullptr;
+    p2.x = nullptr;
+    p2.ldx = 0;
     p2.out = y;
     p2.E = (int)E;
     p2.M = (int)M;
@@ -313,11 +351,12 @@ int run_combine(const float* y, const int32_t* inv, int64_t T, int64_t d, int64_
 int forward_impl(const moe_bf16* x, const moe_bf16* w_router, const float* bias, const moe_bf16* w_gate,
                  const moe_bf16* w_up, const moe_bf16* w_down, int64_t T, int64_t d, int64_t E, int64_t k, int64_t f,
                  float* out, int32_t* ids_out, float* w_out, void* ws, size_t ws_bytes, cudaStream_t s,
-                 cudaEvent_t* ev, int n_ev)
+                 cudaEvent_t* ev, int n_ev, unsigned flags)
 {
     int rc = check_common(T, d, E, k);
     if (rc) return rc;
     if ((rc = check_f(f))) return rc;
+    if (flags & ~(unsigned)MOE_FLAG_FUSED_GATHER) return MOE_ERR_INVALID_ARG;
     if (T > 0 && (!x || !w_router || !w_gate || !w_up || !w_down || !out)) return MOE_ERR_INVALID_ARG;
     if (!aligned(x, 16) || !aligned(w_router, 16) || !aligned(w_gate, 16) || !aligned(w_up, 16) ||
         !aligned(w_down, 16) || !aligned(out, 16) || !aligned(bias, 4) || !aligned(ids_out, 4) ||
@@ -342,21 +381,23 @@ int forward_impl(const moe_bf16* x, const moe_bf16* w_router, const float* bias,
     int32_t* counts = reinterpret_cast<int32_t*>(w + L.counts);
     int32_t* offsets = reinterpret_cast<int32_t*>(w + L.offsets);
     int32_t* chunk = reinterpret_cast<int32_t*>(w + L.chunk);
+    float* part = reinterpret_cast<float*>(w + L.part);
     int32_t* perm = reinterpret_cast<int32_t*>(w + L.perm);
     int32_t* inv = reinterpret_cast<int32_t*>(w + L.inv);
     float* w_perm = reinterpret_cast<float*>(w + L.w_perm);
+    moe_bf16* x_perm = reinterpret_cast<moe_bf16*>(w + L.x_perm);
     moe_bf16* h = reinterpret_cast<moe_bf16*>(w + L.h);
     float* y = reinterpret_cast<float*>(w + L.y);
+    const bool gather = (flags & MOE_FLAG_FUSED_GATHER) != 0;
 
-    if ((rc = run_route(*st, x, w_router, bias, T, d, E, k, ids, wts, s))) return rc;
+    if ((rc = run_route(x, w_router, bias, T, d, E, k, ids, wts, part, chunk, s))) return rc;
     if ((rc = rec(1))) return rc;
-    // The grouped rows of x are never materialised: the gate/up GEMM gathers
-    // them from x through perm as it loads its operand tiles.
-    if ((rc = run_permute(x, ids, wts, T, d, E, k, counts, offsets, perm, inv, nullptr, w_perm, chunk, s)))
+    if ((rc = run_permute(x, ids, wts, T, d, E, k, counts, offsets, perm, inv, gather ? nullptr : x_perm, w_perm,
+                          chunk, true, s)))
         return rc;
     if ((rc = rec(2))) return rc;
-    if ((rc = run_ffn(*st, nullptr, x, perm, T, k, w_perm, offsets, w_gate, w_up, w_down, T * k, d, E, f, h, y, s,
-                      ev ? ev[3] : nullptr)))
+    if ((rc = run_ffn(*st, gather ? nullptr : x_perm, gather ? x : nullptr, perm, T, k, w_perm, offsets, w_gate,
+                      w_up, w_down, T * k, d, E, f, h, y, s, ev ? ev[3] : nullptr)))
         return rc;
     if ((rc = rec(4))) return rc;
     if ((rc = run_combine(y, inv, T, d, k, out, s))) return rc;
@@ -391,24 +432,34 @@ size_t moe_workspace_size(int64_t T, int64_t d, int64_t E, int64_t k, int64_t f)
     return plan(T, d, E, k, f).total;
 }
 
+size_t moe_route_workspace_size(int64_t T, int64_t d, int64_t E)
+{
+    if (check_common(T, d, E, 1)) return 0;
+    return route_ws_bytes(T, d, E);
+}
+
 size_t moe_permute_workspace_size(int64_t T, int64_t E, int64_t k)
 {
     if (T < 0 || E <= 0 || k <= 0 || E > moe::gemm::kMaxE || k > E) return 0;
-    return permute_ws_bytes(T, E, k);
+    return permute_ws_bytes(T, E);
 }
 
 int moe_route(const moe_bf16* x, const moe_bf16* w_router, const float* bias, int64_t T, int64_t d, int64_t E,
-              int64_t k, int32_t* topk_ids, float* topk_w, cudaStream_t stream)
+              int64_t k, int32_t* topk_ids, float* topk_w, void* workspace, size_t workspace_bytes,
+              cudaStream_t stream)
 {
     int rc = check_common(T, d, E, k);
     if (rc) return rc;
     if (T > 0 && (!x || !w_router || !topk_ids || !topk_w)) return MOE_ERR_INVALID_ARG;
     if (!aligned(x, 16) || !aligned(w_router, 16) || !aligned(bias, 4) || !aligned(topk_ids, 4) ||
-        !aligned(topk_w, 4))
+        !aligned(topk_w, 4) || !aligned(workspace, 16))
         return MOE_ERR_INVALID_ARG;
+    if (workspace_bytes < route_ws_bytes(T, d, E)) return MOE_ERR_WORKSPACE_TOO_SMALL;
+    if (T > 0 && !workspace) return MOE_ERR_INVALID_ARG;
     DeviceState* st = nullptr;
     if ((rc = setup_device(&st))) return rc;
-    return run_route(*st, x, w_router, bias, T, d, E, k, topk_ids, topk_w, stream);
+    return run_route(x, w_router, bias, T, d, E, k, topk_ids, topk_w, static_cast<float*>(workspace), nullptr,
+                     stream);
 }
 
 int moe_permute(const moe_bf16* x, const int32_t* topk_ids, const float* topk_w, int64_t T, int64_t d, int64_t E,
@@ -423,13 +474,13 @@ int moe_permute(const moe_bf16* x, const int32_t* topk_ids, const float* topk_w,
     if (!aligned(x, 16) || !aligned(x_perm, 16) || !aligned(topk_ids, 4) || !aligned(topk_w, 4) ||
         !aligned(counts, 4) || !aligned(offsets, 4) || !aligned(perm, 4) || !aligned(inv, 4) || !aligned(w_perm, 4))
         return MOE_ERR_INVALID_ARG;
-    const size_t need = permute_ws_bytes(T, E, k);
+    const size_t need = permute_ws_bytes(T, E);
     if (workspace_bytes < need) return MOE_ERR_WORKSPACE_TOO_SMALL;
     if (T > 0 && (!workspace || !aligned(workspace, 4))) return MOE_ERR_INVALID_ARG;
     DeviceState* st = nullptr;
     if ((rc = setup_device(&st))) return rc;
     return run_permute(x, topk_ids, topk_w, T, d, E, k, counts, offsets, perm, inv, x_perm, w_perm,
-                       static_cast<int32_t*>(workspace), stream);
+                       static_cast<int32_t*>(workspace), false, stream);
 }
 
 int moe_expert_ffn(const moe_bf16* x_perm, const float* w_perm, const int32_t* offsets, const moe_bf16* w_gate,
@@ -470,17 +521,16 @@ int moe_forward(const moe_bf16* x, const moe_bf16* w_router, const float* bias, 
                 cudaStream_t stream)
 {
     return forward_impl(x, w_router, bias, w_gate, w_up, w_down, T, d, E, k, f, out, topk_ids_out, topk_w_out,
-                        workspace, workspace_bytes, stream, nullptr, 0);
+                        workspace, workspace_bytes, stream, nullptr, 0, kDefaultForwardFlags);
 }
 
-int moe_forward_profiled(const moe_bf16* x, const moe_bf16* w_router, const float* bias, const moe_bf16* w_gate,
-                         const moe_bf16* w_up, const moe_bf16* w_down, int64_t T, int64_t d, int64_t E, int64_t k,
-                         int64_t f, float* out, int32_t* topk_ids_out, float* topk_w_out, void* workspace,
-                         size_t workspace_bytes, cudaStream_t stream, cudaEvent_t* events, int n_events)
+int moe_forward_ex(const moe_bf16* x, const moe_bf16* w_router, const float* bias, const moe_bf16* w_gate,
+                   const moe_bf16* w_up, const moe_bf16* w_down, int64_t T, int64_t d, int64_t E, int64_t k,
+                   int64_t f, float* out, int32_t* topk_ids_out, float* topk_w_out, void* workspace,
+                   size_t workspace_bytes, cudaStream_t stream, cudaEvent_t* events, int n_events, unsigned flags)
 {
-    if (!events) return MOE_ERR_INVALID_ARG;
     return forward_impl(x, w_router, bias, w_gate, w_up, w_down, T, d, E, k, f, out, topk_ids_out, topk_w_out,
-                        workspace, workspace_bytes, stream, events, n_events);
+                        workspace, workspace_bytes, stream, events, n_events, flags);
 }
 
 int moe_get_status(cudaStream_t stream)

@@ -3,14 +3,21 @@
 // The "token reordering" step of "Qwen3MoeSparseMoeBlock performance
 // optimisation in practice" (section 2.2: sort_tokens_by_expert, then gather
 // the hidden states and routing weights in that order), done as a stable
-// counting sort over the T*k flat assignments a = t*k + j:
-//   hist  : per-chunk expert histograms (chunk = 4096 assignments)
-//   scan  : per-expert totals, exclusive offsets, and each chunk's starting
-//           position inside every expert group
-//   rank  : inside a chunk, eight warps walk their 512 assignments in order;
-//           __match_any_sync gives each lane its rank among same-expert lanes
-//           so group order is ascending a -- deterministic, no global atomics
-//   gather: one warp per grouped row copies x[t] with 16-byte vectors
+// counting sort over the T*k flat assignments a = t*k + j, in 64-token chunks:
+//   hist       : each chunk's assignment count per expert, stored expert-major
+//                counts[e][chunk] (the router's softmax kernel can produce
+//                the same table as a by-product)
+//   chunk_scan : one block per expert turns its row of chunk counts into
+//                exclusive chunk bases inside the expert's group and writes
+//                the expert's total
+//   rank       : one block per chunk recomputes the group offsets (an
+//                exclusive scan of the totals), then eight warps walk their
+//                slices of the chunk in order; __match_any_sync ranks each
+//                lane among same-expert lanes, so every group lists its
+//                assignments in ascending a -- deterministic, no global
+//                atomics.
+//   gather     : x_perm[pos] = x[perm[pos] / k], one warp per row, 16-byte
+//                vectors, many rows in flight per SM.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -20,20 +27,20 @@
 namespace moe {
 namespace permute {
 
-constexpr int kChunk = 4096;        // assignments per chunk
+constexpr int kTokensPerChunk = 64;
 constexpr int kThreads = 256;       // 8 warps
 constexpr int kWarps = kThreads / 32;
-constexpr int kPerWarp = kChunk / kWarps;
-constexpr int kScanThreads = 512;   // >= max E
+constexpr int kMaxE = 512;
 
-__global__ void __launch_bounds__(kThreads) hist_kernel(const int32_t* __restrict__ ids, int64_t n, int E,
-                                                        int32_t* __restrict__ chunk_counts)
+// Chunk histogram for callers that bring their own expert ids.
+__global__ void __launch_bounds__(kThreads) hist_kernel(const int32_t* __restrict__ ids, int64_t T, int k, int E,
+                                                        int32_t* __restrict__ counts_em, int n_tchunks)
 {
-    extern __shared__ int s_hist[];
+    __shared__ int s_hist[kMaxE];
     for (int e = threadIdx.x; e < E; e += kThreads) s_hist[e] = 0;
     __syncthreads();
-    const int64_t a0 = (int64_t)blockIdx.x * kChunk;
-    const int64_t a1 = min(n, a0 + kChunk);
+    const int64_t a0 = (int64_t)blockIdx.x * kTokensPerChunk * k;
+    const int64_t a1 = min(T * k, a0 + (int64_t)kTokensPerChunk * k);
     bool bad = false;
     for (int64_t a = a0 + threadIdx.x; a < a1; a += kThreads) {
         const int e = __ldg(ids + a);
@@ -44,77 +51,133 @@ __global__ void __launch_bounds__(kThreads) hist_kernel(const int32_t* __restric
     }
     if (bad) record_status(kStatusDeviceBounds);
     __syncthreads();
-    for (int e = threadIdx.x; e < E; e += kThreads) chunk_counts[(int64_t)blockIdx.x * E + e] = s_hist[e];
+    for (int e = threadIdx.x; e < E; e += kThreads) counts_em[(int64_t)e * n_tchunks + blockIdx.x] = s_hist[e];
 }
 
-// One block.  Thread e walks the chunks of expert e (running sum), then a
-// block-wide exclusive scan over experts gives the group offsets.
-// chunk_counts is rewritten in place into absolute chunk starting positions.
-__global__ void __launch_bounds__(kScanThreads) scan_kernel(int32_t* __restrict__ chunk_counts, int nchunks, int E,
-                                                            int32_t* __restrict__ counts,
-                                                            int32_t* __restrict__ offsets)
+// Block e: exclusive scan of counts_em[e][0..n_tchunks) in place; totals[e].
+__global__ void __launch_bounds__(kThreads) chunk_scan_kernel(int32_t* __restrict__ counts_em, int n_tchunks,
+                                                              int32_t* __restrict__ totals)
 {
-    __shared__ int s_warp[kScanThreads / 32];
-    const int e = threadIdx.x;
-    const int lane = e % 32, warp = e / 32;
-    int total = 0;
-    if (e < E) {
-#pragma unroll 8
-        for (int c = 0; c < nchunks; ++c) {
-            const int v = chunk_counts[(int64_t)c * E + e];
-            chunk_counts[(int64_t)c * E + e] = total;
-            total += v;
-        }
-        counts[e] = total;
-    }
-    int incl = total;
+    __shared__ int s_warp[32];
+    int32_t* row = counts_em + (int64_t)blockIdx.x * n_tchunks;
+    const int tid = threadIdx.x, lane = tid % 32, warp = tid / 32;
+    int carry = 0;
+    for (int base = 0; base < n_tchunks; base += 4 * kThreads) {
+        const int n = min(4 * kThreads, n_tchunks - base);
+        int v[4], local = 0;
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int nb = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += nb;
-    }
-    if (lane == 31) s_warp[warp] = incl;
-    __syncthreads();
-    if (warp == 0) {
-        int w = lane < kScanThreads / 32 ? s_warp[lane] : 0;
-        int wi = w;
+        for (int i = 0; i < 4; ++i) {
+            const int idx = tid * 4 + i;
+            v[i] = idx < n ? row[base + idx] : 0;
+            local += v[i];
+        }
+        int incl = local;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
-            const int nb = __shfl_up_sync(0xffffffffu, wi, o);
-            if (lane >= o) wi += nb;
+            const int nb = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += nb;
         }
-        if (lane < kScanThreads / 32) s_warp[lane] = wi - w;  // exclusive warp prefix
+        if (lane == 31) s_warp[warp] = incl;
+        __syncthreads();
+        if (warp == 0) {
+            const int w = lane < kWarps ? s_warp[lane] : 0;
+            int wi = w;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int nb = __shfl_up_sync(0xffffffffu, wi, o);
+                if (lane >= o) wi += nb;
+            }
+            s_warp[lane] = wi;  // inclusive over warps
+        }
+        __syncthreads();
+        int run = carry + (warp > 0 ? s_warp[warp - 1] : 0) + incl - local;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int idx = tid * 4 + i;
+            if (idx < n) row[base + idx] = run;
+            run += v[i];
+        }
+        carry += s_warp[kWarps - 1];
+        __syncthreads();
     }
-    __syncthreads();
-    const int excl = s_warp[warp] + incl - total;
-    if (e < E) {
-        offsets[e] = excl;
-        if (e == E - 1) offsets[E] = excl + total;
-#pragma unroll 8
-        for (int c = 0; c < nchunks; ++c) chunk_counts[(int64_t)c * E + e] += excl;
-    }
+    if (tid == 0) totals[blockIdx.x] = carry;
 }
 
+// One block per 64-token chunk.  chunk_base_em[e][c] holds the chunk's first
+// position inside group e (relative to the group start); totals[e] the group
+// sizes.  Block 0 also writes offsets[0..E].
 __global__ void __launch_bounds__(kThreads) rank_kernel(const int32_t* __restrict__ ids,
-                                                        const float* __restrict__ wts, int64_t n, int E,
-                                                        const int32_t* __restrict__ chunk_base,
-                                                        int32_t* __restrict__ perm, int32_t* __restrict__ inv,
-                                                        float* __restrict__ w_perm)
+                                                        const float* __restrict__ wts, int64_t T, int k, int E,
+                                                        const int32_t* __restrict__ chunk_base_em, int n_tchunks,
+                                                        const int32_t* __restrict__ totals,
+                                                        int32_t* __restrict__ offsets, int32_t* __restrict__ perm,
+                                                        int32_t* __restrict__ inv, float* __restrict__ w_perm)
 {
-    extern __shared__ int s_next[];  // [kWarps][E]: next free position per warp and expert
-    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    for (int i = threadIdx.x; i < kWarps * E; i += kThreads) s_next[i] = 0;
+    __shared__ int s_off[kMaxE + 1];
+    __shared__ int s_next[kWarps * kMaxE];   // next free position per warp and expert
+    __shared__ int s_warp[32];
+    const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+    const int chunk = blockIdx.x;
+
+    // group offsets = exclusive scan of the totals (E <= 512 <= 4 * 256)
+    for (int e = tid; e < E; e += kThreads) s_off[e] = totals[e];
     __syncthreads();
-    const int64_t w0 = (int64_t)blockIdx.x * kChunk + (int64_t)warp * kPerWarp;
-    const int64_t w1 = min(n, w0 + kPerWarp);
+    {
+        int v[4], local = 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int idx = tid * 4 + i;
+            v[i] = idx < E ? s_off[idx] : 0;
+            local += v[i];
+        }
+        int incl = local;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int nb = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += nb;
+        }
+        if (lane == 31) s_warp[warp] = incl;
+        __syncthreads();
+        if (warp == 0) {
+            const int w = lane < kWarps ? s_warp[lane] : 0;
+            int wi = w;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int nb = __shfl_up_sync(0xffffffffu, wi, o);
+                if (lane >= o) wi += nb;
+            }
+            s_warp[lane] = wi;
+        }
+        __syncthreads();
+        int run = (warp > 0 ? s_warp[warp - 1] : 0) + incl - local;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int idx = tid * 4 + i;
+            if (idx < E) s_off[idx] = run;
+            run += v[i];
+        }
+        if (tid == 0) s_off[E] = s_warp[kWarps - 1];
+        __syncthreads();
+    }
+    if (chunk == 0)
+        for (int e = tid; e <= E; e += kThreads) offsets[e] = s_off[e];
+
+    // per-warp slices of this chunk's assignments
+    const int64_t a_begin = (int64_t)chunk * kTokensPerChunk * k;
+    const int64_t a_end = min(T * k, a_begin + (int64_t)kTokensPerChunk * k);
+    const int per_warp = (kTokensPerChunk * k + kWarps - 1) / kWarps;
+    const int64_t w0 = min(a_end, a_begin + (int64_t)warp * per_warp);
+    const int64_t w1 = min(a_end, w0 + per_warp);
     int* mine = s_next + warp * E;
+    for (int i = tid; i < kWarps * E; i += kThreads) s_next[i] = 0;
+    __syncthreads();
     for (int64_t a = w0 + lane; a < w1; a += 32) {
         const int e = __ldg(ids + a);
         if ((unsigned)e < (unsigned)E) atomicAdd(&mine[e], 1);
     }
     __syncthreads();
-    for (int e = threadIdx.x; e < E; e += kThreads) {
-        int run = chunk_base[(int64_t)blockIdx.x * E + e];
+    for (int e = tid; e < E; e += kThreads) {
+        int run = s_off[e] + chunk_base_em[(int64_t)e * n_tchunks + chunk];
         for (int w = 0; w < kWarps; ++w) {
             const int c = s_next[w * E + e];
             s_next[w * E + e] = run;
@@ -143,7 +206,7 @@ __global__ void __launch_bounds__(kThreads) rank_kernel(const int32_t* __restric
     }
 }
 
-// x_perm[pos] = x[perm[pos] / k]; one warp per row, 16-byte vectors.
+// x_perm[pos] = x[perm[pos] / k]; one warp per grouped row.
 __global__ void __launch_bounds__(kThreads) gather_kernel(const uint4* __restrict__ x,
                                                           const int32_t* __restrict__ perm, int64_t n, int nvec,
                                                           int k, uint4* __restrict__ x_perm)
@@ -158,7 +221,7 @@ __global__ void __launch_bounds__(kThreads) gather_kernel(const uint4* __restric
     }
     const uint4* src = x + (int64_t)(a / k) * nvec;
     uint4* dst = x_perm + row * nvec;
-#pragma unroll 4
+#pragma unroll 8
     for (int v = lane; v < nvec; v += 32) dst[v] = __ldg(src + v);
 }
 
