@@ -70,7 +70,8 @@ typedef enum {
     MOE_ERR_CUDA = 4,                /* a CUDA runtime call or a launch failed */
     MOE_ERR_DEVICE_TIMEOUT = 5,      /* device: a pipeline wait ran past its limit */
     MOE_ERR_DEVICE_BOUNDS = 6,       /* device: index data out of range (ids, offsets, inv) */
-    MOE_ERR_UNSUPPORTED_DEVICE = 7   /* not a compute-capability 10.0 GPU */
+    MOE_ERR_UNSUPPORTED_DEVICE = 7,  /* not a compute-capability 10.0 GPU */
+    MOE_ERR_STATIC_SCRATCH_TOO_SMALL = 8 /* moe_permute_static: E * ceil(T/64) > 262144 */
 } moe_status_t;
 
 /* Human-readable name of a status code (static string, never NULL). */
@@ -136,6 +137,31 @@ int moe_permute(const moe_bf16* x, const int32_t* topk_ids, const float* topk_w,
                 int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* inv,
                 moe_bf16* x_perm, float* w_perm,
                 void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * moe_permute for callers that cannot allocate device memory when they call
+ * it -- for example a plugin inside an inference engine that plans all
+ * device memory ahead of time and may not allocate while enqueueing work, or
+ * a latency-critical loop that cannot afford cudaMalloc's implicit device
+ * synchronisation.  (The pages have no counterpart: this is an interface
+ * convenience, not part of the method.)  Same arguments, outputs and
+ * results as moe_permute, without the workspace: the per-chunk expert counts
+ * live in a fixed 1 MiB array inside the library, which every GPU that loads
+ * the library keeps until the process exits.
+ *   Limit: E * ceil(T / 64) <= 262144 (for E = 128: T <= 131072); larger
+ *          sizes return MOE_ERR_STATIC_SCRATCH_TOO_SMALL.
+ *   The call allocates nothing and calls no allocating routine.  The first
+ *   call on each device looks up the array's device address (a one-time
+ *   set-up for that device); make that first call before any stream capture.
+ *   All calls share the one array and it keeps the last call's contents;
+ *   each call writes every entry it later reads, so nothing needs clearing,
+ *   but calls whose work overlaps on the GPU (for example on two streams)
+ *   race on the array and must be serialised by the caller.
+ */
+int moe_permute_static(const moe_bf16* x, const int32_t* topk_ids, const float* topk_w,
+                       int64_t T, int64_t d, int64_t E, int64_t k,
+                       int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* inv,
+                       moe_bf16* x_perm, float* w_perm, cudaStream_t stream);
 
 /*
  * Batched expert compute (section 2.1, point 1: the experts' weights stacked

@@ -30,12 +30,14 @@ MOE_ERR_CUDA = 4
 MOE_ERR_DEVICE_TIMEOUT = 5
 MOE_ERR_DEVICE_BOUNDS = 6
 MOE_ERR_UNSUPPORTED_DEVICE = 7
+MOE_ERR_STATIC_SCRATCH_TOO_SMALL = 8
 
 # Every symbol include/moe.h declares.
 ABI_SYMBOLS = (
     "moe_strerror", "moe_version", "moe_workspace_size", "moe_route_workspace_size",
     "moe_permute_workspace_size", "moe_route", "moe_permute", "moe_expert_ffn", "moe_combine", "moe_forward",
     "moe_forward_ex", "moe_get_status", "moe_set_wait_limit_ns", "moe_selftest_wait_timeout",
+    "moe_permute_static",
 )
 
 
@@ -73,6 +75,7 @@ def lib() -> ctypes.CDLL:
         L.moe_permute_workspace_size.argtypes = [_I64] * 3
         L.moe_route.argtypes = [_P, _P, _P, _I64, _I64, _I64, _I64, _P, _P, _P, _SZ, _P]
         L.moe_permute.argtypes = [_P, _P, _P, _I64, _I64, _I64, _I64, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]
+        L.moe_permute_static.argtypes = [_P, _P, _P, _I64, _I64, _I64, _I64, _P, _P, _P, _P, _P, _P, _P]
         L.moe_expert_ffn.argtypes = [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _P, _P, _P]
         L.moe_combine.argtypes = [_P, _P, _I64, _I64, _I64, _P, _P]
         L.moe_forward.argtypes = [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64, _P, _P, _P, _P, _SZ, _P]
@@ -82,7 +85,7 @@ def lib() -> ctypes.CDLL:
         L.moe_selftest_wait_timeout.argtypes = [_I64, _P]
         for name in ("moe_route", "moe_permute", "moe_expert_ffn", "moe_combine", "moe_forward",
                      "moe_forward_ex", "moe_get_status", "moe_set_wait_limit_ns",
-                     "moe_selftest_wait_timeout"):
+                     "moe_selftest_wait_timeout", "moe_permute_static"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib

@@ -404,6 +404,37 @@ int forward_impl(const moe_bf16* x, const moe_bf16* w_router, const float* bias,
     return rec(5);
 }
 
+// ------------------------------------------- fixed scratch for moe_permute_static
+// Some callers cannot allocate device memory when they run the permutation:
+// for example a plugin inside an inference engine that plans all device
+// memory ahead of time and must not allocate while it enqueues work, or a
+// latency-critical loop where cudaMalloc's implicit synchronisation is not
+// acceptable.  moe_permute_static serves them from this array instead of a
+// caller-provided workspace.  It holds the per-chunk expert counts, one
+// int32 per (expert, 64-token chunk), so it caps E * ceil(T / 64).  Every
+// GPU that loads the library keeps the array (1 MiB) until the process ends.
+constexpr int64_t kStaticPermuteScratchInts = int64_t(1) << 18;
+static __device__ __align__(256) int32_t g_static_permute_scratch[kStaticPermuteScratchInts];
+
+int32_t* g_static_scratch_addr[kMaxDevices] = {};
+
+// The array's device address for the current device.  In host code the
+// symbol name is only a host-side stand-in, so the address is looked up once
+// per device with that device current, checked, and cached.
+int static_permute_scratch(int32_t** out)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MOE_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!g_static_scratch_addr[dev]) {
+        void* addr = nullptr;
+        if (cudaGetSymbolAddress(&addr, g_static_permute_scratch) != cudaSuccess || !addr) return MOE_ERR_CUDA;
+        g_static_scratch_addr[dev] = static_cast<int32_t*>(addr);
+    }
+    *out = g_static_scratch_addr[dev];
+    return MOE_OK;
+}
+
 }  // namespace
 
 // ===================================================================== ABI
@@ -420,6 +451,8 @@ const char* moe_strerror(int status)
         case MOE_ERR_DEVICE_TIMEOUT: return "MOE_ERR_DEVICE_TIMEOUT: a device pipeline wait ran past its limit";
         case MOE_ERR_DEVICE_BOUNDS: return "MOE_ERR_DEVICE_BOUNDS: index data out of range on the device";
         case MOE_ERR_UNSUPPORTED_DEVICE: return "MOE_ERR_UNSUPPORTED_DEVICE: needs a compute capability 10.0 GPU";
+        case MOE_ERR_STATIC_SCRATCH_TOO_SMALL:
+            return "MOE_ERR_STATIC_SCRATCH_TOO_SMALL: moe_permute_static needs E * ceil(T / 64) <= 262144";
         default: return "unknown moe status";
     }
 }
@@ -481,6 +514,30 @@ int moe_permute(const moe_bf16* x, const int32_t* topk_ids, const float* topk_w,
     if ((rc = setup_device(&st))) return rc;
     return run_permute(x, topk_ids, topk_w, T, d, E, k, counts, offsets, perm, inv, x_perm, w_perm,
                        static_cast<int32_t*>(workspace), false, stream);
+}
+
+int moe_permute_static(const moe_bf16* x, const int32_t* topk_ids, const float* topk_w, int64_t T, int64_t d,
+                       int64_t E, int64_t k, int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* inv,
+                       moe_bf16* x_perm, float* w_perm, cudaStream_t stream)
+{
+    int rc = check_common(T, d, E, k);
+    if (rc) return rc;
+    if (!counts || !offsets) return MOE_ERR_INVALID_ARG;
+    if (T > 0 && (!topk_ids || !topk_w || !perm || !inv || !w_perm)) return MOE_ERR_INVALID_ARG;
+    if (x_perm && !x) return MOE_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(x_perm, 16) || !aligned(topk_ids, 4) || !aligned(topk_w, 4) ||
+        !aligned(counts, 4) || !aligned(offsets, 4) || !aligned(perm, 4) || !aligned(inv, 4) || !aligned(w_perm, 4))
+        return MOE_ERR_INVALID_ARG;
+    if (E * token_chunks(T) > kStaticPermuteScratchInts) return MOE_ERR_STATIC_SCRATCH_TOO_SMALL;
+    DeviceState* st = nullptr;
+    if ((rc = setup_device(&st))) return rc;
+    int32_t* scratch = nullptr;
+    if ((rc = static_permute_scratch(&scratch))) return rc;
+    // The histogram kernel writes every (expert, chunk) entry that the scan
+    // and rank kernels later read, so nothing left by an earlier call needs
+    // clearing first.
+    return run_permute(x, topk_ids, topk_w, T, d, E, k, counts, offsets, perm, inv, x_perm, w_perm, scratch, false,
+                       stream);
 }
 
 int moe_expert_ffn(const moe_bf16* x_perm, const float* w_perm, const int32_t* offsets, const moe_bf16* w_gate,
