@@ -33,7 +33,8 @@
 //   warp 1       TMEM allocation + single-thread tcgen05.mma issuer,
 //                M=128 N=256 K=16 per instruction, fp32 accumulators
 //   warps 2..5   epilogue: tcgen05.ld of the 128 x 256 accumulator, one row
-//                per thread, fused math, stores
+//                per thread, fused math, stores.  (With 8 warps the two warps
+//                of a lane quarter split the columns; 4 measured faster.)
 // Two accumulator buffers (2 x 256 TMEM columns) let the epilogue of one
 // tile overlap the MMAs of the next.
 //
@@ -59,8 +60,20 @@ namespace gemm {
 constexpr int kBM = 128;
 constexpr int kBN = 256;
 constexpr int kBK = 64;
-constexpr int kStages = 4;
-constexpr int kThreads = 192;
+constexpr int kMaxStages = 4;
+// Tuning constants (overridable at build time for measurements).  Measured
+// on the Qwen3-shaped layer: 4 epilogue warps beat 8, and 4 down-GEMM stages
+// beat 3 stages with double store buffers for 8 warps.
+#ifndef MOE_GEMM_EPI_WARPS
+#define MOE_GEMM_EPI_WARPS 4
+#endif
+#ifndef MOE_GEMM_DOWN_STAGES
+#define MOE_GEMM_DOWN_STAGES 4
+#endif
+constexpr int kEpiWarps = MOE_GEMM_EPI_WARPS;      // 4 or 8: 1 or 2 warps per TMEM lane quarter
+constexpr int kColGroups = kEpiWarps / 4;          // warps sharing a lane quarter split the columns
+constexpr int kThreads = 64 + kEpiWarps * 32;
+static_assert(kEpiWarps == 4 || kEpiWarps == 8, "epilogue warps");
 constexpr int kABytes = kBM * kBK * 2;      // 16 KB
 constexpr int kChunkBytes = 64 * kBK * 2;   // 8 KB: 64 n x 64 k
 constexpr int kBBytes = 4 * kChunkBytes;    // 32 KB
@@ -69,7 +82,15 @@ constexpr uint32_t kTmemCols = 512;         // 2 accumulators x 256 columns
 constexpr int kMaxE = 512;
 constexpr int kSlabCols = 16;               // fp32 columns per TMA-store slab (64 B rows)
 constexpr int kSlabBytes = 32 * kSlabCols * 4;     // 32 rows x 16 fp32 = 2 KB
-constexpr int kStoreBytes = 4 * 2 * kSlabBytes;    // 4 epilogue warps x 2 buffers
+constexpr int kStoreBytes = kEpiWarps * 2 * kSlabBytes;  // 2 buffers per epilogue warp
+
+// Ring depth and store staging per epilogue: the down GEMM gives up one
+// stage to the staging buffers its TMA stores read from.
+template <int EPI>
+struct Stages {
+    static constexpr int value = EPI == 0 ? 4 : MOE_GEMM_DOWN_STAGES;
+    static constexpr int store_bytes = EPI == 0 ? 0 : kStoreBytes;
+};
 
 enum EpiKind { kSwiGLU = 0, kWeighted = 1 };
 
@@ -90,8 +111,8 @@ struct Params {
 
 // Shared memory after the stage ring and the store staging buffers.
 struct alignas(8) Ctrl {
-    uint64_t full[kStages];
-    uint64_t empty[kStages];
+    uint64_t full[kMaxStages];
+    uint64_t empty[kMaxStages];
     uint64_t acc_full[2];
     uint64_t acc_empty[2];
     uint64_t done;
@@ -104,25 +125,78 @@ struct alignas(8) Ctrl {
     int tok[kBM];         // GATHER: token row of x for each row of the current M tile
 };
 
-__host__ inline size_t smem_bytes() { return 1024 + (size_t)kStages * kStageBytes + kStoreBytes + sizeof(Ctrl); }
+template <int EPI>
+__host__ inline size_t smem_bytes()
+{
+    return 1024 + (size_t)Stages<EPI>::value * kStageBytes + Stages<EPI>::store_bytes + sizeof(Ctrl);
+}
 
-// Work item -> (expert, first row, group end, N tile).
-__device__ __forceinline__ void decode(int64_t w, int n_tiles, const Ctrl& c, int E, int& e, int& row0,
-                                       int& row_end, int& nt)
+// Work item -> (expert, first row, group end, N tile), for M tiles of
+// TILE_ROWS rows: tp[e] is the exclusive prefix of M tiles per group.
+template <int TILE_ROWS = kBM>
+__device__ __forceinline__ void decode_tile(int64_t w, int n_tiles, const int* tp, const int* off, int E, int& e,
+                                            int& row0, int& row_end, int& nt)
 {
     const int mt = (int)(w / n_tiles);
     nt = (int)(w - (int64_t)mt * n_tiles);
     int lo = 0, hi = E;  // tp[lo] <= mt < tp[hi]
     while (hi - lo > 1) {
         const int mid = (lo + hi) >> 1;
-        if (c.tp[mid] <= mt)
+        if (tp[mid] <= mt)
             lo = mid;
         else
             hi = mid;
     }
     e = lo;
-    row0 = c.off[e] + (mt - c.tp[e]) * kBM;
-    row_end = c.off[e + 1];
+    row0 = off[e] + (mt - tp[e]) * TILE_ROWS;
+    row_end = off[e + 1];
+}
+
+__device__ __forceinline__ void decode(int64_t w, int n_tiles, const Ctrl& c, int E, int& e, int& row0,
+                                       int& row_end, int& nt)
+{
+    decode_tile<kBM>(w, n_tiles, c.tp, c.off, E, e, row0, row_end, nt);
+}
+
+// Reads the group offsets into off[0..E] and, with warp 0, builds tp (the
+// exclusive prefix of ceil(count / TILE_ROWS) per group).  The offsets are
+// validated: non-decreasing, off[0] = 0, off[E] = M; *bad is set otherwise.
+// Contains __syncthreads: every thread of the block must call it.
+template <int TILE_ROWS>
+__device__ __forceinline__ void build_tile_list(const int32_t* offsets, int E, int M, int* off, int* tp,
+                                                int* total, int* bad_out)
+{
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    for (int i = threadIdx.x; i <= E; i += blockDim.x) off[i] = offsets[i];
+    __syncthreads();
+    if (warp == 0) {
+        int run = 0;
+        bool bad = false;
+        for (int base = 0; base < E; base += 32) {
+            const int e = base + lane;
+            int tiles = 0;
+            if (e < E) {
+                const int cnt = off[e + 1] - off[e];
+                if (cnt < 0) bad = true;
+                tiles = cnt > 0 ? (cnt + TILE_ROWS - 1) / TILE_ROWS : 0;
+            }
+            int incl = tiles;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int nb = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += nb;
+            }
+            if (e < E) tp[e] = run + incl - tiles;
+            run += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        bad = __any_sync(0xffffffffu, bad);
+        if (lane == 0) {
+            tp[E] = run;
+            *bad_out = (bad || off[0] != 0 || off[E] != M) ? 1 : 0;
+            *total = run;
+            if (*bad_out && blockIdx.x == 0) record_status(kStatusDeviceBounds);
+        }
+    }
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b)
@@ -146,16 +220,115 @@ __device__ __forceinline__ int gather_token(const Params& p, int r)
     return a / p.k_top;
 }
 
+// Drains one 128 x 256 fp32 accumulator tile from TMEM and stores it.  The
+// calling warp reads TMEM lane quarter q (rows q*32 .. +31 of the tile, row
+// row0 + r for thread r) and column group hf; rows at or past row_end are
+// not stored.  tbase addresses the accumulator at this warp's lane quarter.
+template <int EPI>
+__device__ __forceinline__ void epilogue_tile(const Params& p, const CUtensorMap* tm_out, uint32_t tbase, int row0,
+                                              int row_end, int nt, int q, int lane, int hf, float* slab,
+                                              int& slab_buf)
+{
+    const int r = q * 32 + lane;        // tile row owned by this thread
+    const int row = row0 + r;
+    const bool valid = row < row_end;
+    if (EPI == kSwiGLU) {
+        // this warp: output columns [cbeg, cbeg + 128 / kColGroups) of the tile
+        constexpr int kIters = 128 / kColGroups / 16;
+        const int cbeg = hf * (128 / kColGroups);
+        __nv_bfloat16* orow =
+            static_cast<__nv_bfloat16*>(p.out) + (int64_t)row * p.n_out + nt * 128;
+        const int ncols = min(128, p.n_out - nt * 128);
+        uint32_t g[2][16], u[2][16];
+        tmem_ld16(tbase + cbeg, g[0]);
+        tmem_ld16(tbase + 128 + cbeg, u[0]);
+        tmem_ld_wait();
+#pragma unroll
+        for (int it = 0; it < kIters; ++it) {
+            const int c0 = cbeg + 16 * it;
+            if (it + 1 < kIters) {  // next chunk in flight while this one is processed
+                tmem_ld16(tbase + c0 + 16, g[(it + 1) & 1]);
+                tmem_ld16(tbase + 128 + c0 + 16, u[(it + 1) & 1]);
+            }
+            if (valid && c0 < ncols) {
+                const uint32_t* gg = g[it & 1];
+                const uint32_t* uu = u[it & 1];
+                uint32_t packed[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const float h0 = silu(__uint_as_float(gg[2 * i])) * __uint_as_float(uu[2 * i]);
+                    const float h1 = silu(__uint_as_float(gg[2 * i + 1])) * __uint_as_float(uu[2 * i + 1]);
+                    packed[i] = pack_bf16x2(h0, h1);
+                }
+                uint4* dst = reinterpret_cast<uint4*>(orow + c0);
+                dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+                dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+            }
+            tmem_ld_wait();
+        }
+    } else {
+        // this warp: columns [cbeg, cbeg + 256 / kColGroups) of the tile, in slabs of 16
+        constexpr int kIters = kBN / kColGroups / kSlabCols;
+        const int cbeg = hf * (kBN / kColGroups);
+        const float wgt = valid ? __ldg(p.w_perm + row) : 0.0f;
+        const int wrow0 = row0 + q * 32;                   // first row of this warp's slab
+        const bool whole = wrow0 + 31 < row_end;           // all 32 rows belong to the group
+        float* orow = static_cast<float*>(p.out) + (int64_t)row * p.n_out + nt * kBN;
+        const int ncols = min(kBN, p.n_out - nt * kBN);
+        uint32_t a[2][16];
+        tmem_ld16(tbase + cbeg, a[0]);
+        tmem_ld_wait();
+#pragma unroll
+        for (int it = 0; it < kIters; ++it) {
+            const int c0 = cbeg + kSlabCols * it;
+            if (it + 1 < kIters) tmem_ld16(tbase + c0 + kSlabCols, a[(it + 1) & 1]);
+            const uint32_t* av = a[it & 1];
+            if (c0 < ncols) {  // warp-uniform
+                if (whole) {
+                    float* buf = slab + slab_buf * (kSlabBytes / 4);
+                    if (lane == 0) bulk_wait_group_read<1>();  // the store that last read `buf` is done
+                    __syncwarp();
+                    // row `lane` of the slab: 4 x 16 B chunks, 64-byte swizzle
+                    float4* rowp = reinterpret_cast<float4*>(buf + lane * kSlabCols);
+                    const int sw = (lane >> 1) & 3;
+#pragma unroll
+                    for (int v = 0; v < 4; ++v)
+                        rowp[v ^ sw] = make_float4(wgt * __uint_as_float(av[4 * v]),
+                                                   wgt * __uint_as_float(av[4 * v + 1]),
+                                                   wgt * __uint_as_float(av[4 * v + 2]),
+                                                   wgt * __uint_as_float(av[4 * v + 3]));
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_2d(tm_out, buf, nt * kBN + c0, wrow0);
+                        bulk_commit_group();
+                    }
+                    slab_buf ^= 1;
+                } else if (valid) {
+                    float4* dst = reinterpret_cast<float4*>(orow + c0);
+#pragma unroll
+                    for (int v = 0; v < 4; ++v)
+                        dst[v] = make_float4(wgt * __uint_as_float(av[4 * v]), wgt * __uint_as_float(av[4 * v + 1]),
+                                             wgt * __uint_as_float(av[4 * v + 2]),
+                                             wgt * __uint_as_float(av[4 * v + 3]));
+                }
+            }
+            tmem_ld_wait();
+        }
+    }
+}
+
 template <int EPI, bool GATHER>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b0,
                         const __grid_constant__ CUtensorMap tm_b1, const __grid_constant__ CUtensorMap tm_out,
                         Params p)
 {
+    constexpr int kStages = Stages<EPI>::value;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* stage_out = smem + (size_t)kStages * kStageBytes;
-    Ctrl& c = *reinterpret_cast<Ctrl*>(stage_out + kStoreBytes);
+    Ctrl& c = *reinterpret_cast<Ctrl*>(stage_out + Stages<EPI>::store_bytes);
 
     const int warp = threadIdx.x / 32;
     const int lane = threadIdx.x % 32;
@@ -163,36 +336,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int E = p.E;
 
     // ---- tile list from the device offsets (validated) ----
-    for (int i = threadIdx.x; i <= E; i += kThreads) c.off[i] = p.offsets[i];
-    __syncthreads();
-    if (warp == 0) {
-        int run = 0;
-        bool bad = false;
-        for (int base = 0; base < E; base += 32) {
-            const int e = base + lane;
-            int tiles = 0;
-            if (e < E) {
-                const int cnt = c.off[e + 1] - c.off[e];
-                if (cnt < 0) bad = true;
-                tiles = cnt > 0 ? (cnt + kBM - 1) / kBM : 0;
-            }
-            int incl = tiles;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int nb = __shfl_up_sync(0xffffffffu, incl, o);
-                if (lane >= o) incl += nb;
-            }
-            if (e < E) c.tp[e] = run + incl - tiles;
-            run += __shfl_sync(0xffffffffu, incl, 31);
-        }
-        bad = __any_sync(0xffffffffu, bad);
-        if (lane == 0) {
-            c.tp[E] = run;
-            c.bad = (bad || c.off[0] != 0 || c.off[E] != p.M) ? 1 : 0;
-            c.total_mtiles = run;
-            if (c.bad && blockIdx.x == 0) record_status(kStatusDeviceBounds);
-        }
-    }
+    build_tile_list<kBM>(p.offsets, E, p.M, c.off, c.tp, &c.total_mtiles, &c.bad);
     if (threadIdx.x == 32) {
         for (int s = 0; s < kStages; ++s) {
             // GATHER: the TMA arrival plus one cp.async completion per lane
@@ -201,7 +345,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&c.acc_full[b], 1);
-            mbar_init(&c.acc_empty[b], 4 * 32);
+            mbar_init(&c.acc_empty[b], kEpiWarps * 32);
         }
         mbar_init(&c.done, 1);
         c.abort_flag = 0;
@@ -353,90 +497,31 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
     } else {
         // ---------------------------------------------------- epilogue
-        const int q = warp & 3;          // TMEM lane quarter this warp may access
-        const int r = q * 32 + lane;     // tile row owned by this thread
-        float* slab = reinterpret_cast<float*>(stage_out + q * 2 * kSlabBytes);
+        // Warp w may only touch TMEM lanes 32*(w%4)..+31: warps 2..5 and 6..9
+        // each cover the four lane quarters; the two groups split the columns.
+        const int ew = warp - 2;            // 0..7
+        const int q = warp & 3;             // TMEM lane quarter
+        const int hf = ew >> 2;             // column group (0 when kColGroups == 1)
+        float* slab = reinterpret_cast<float*>(stage_out + ew * 2 * kSlabBytes);
         int slab_buf = 0;
         int acc = 0;
         uint32_t acc_ph = 0;
         for (int64_t w = blockIdx.x; w < total_work; w += gridDim.x) {
             int e, row0, row_end, nt;
             decode(w, p.n_tiles, c, E, e, row0, row_end, nt);
-            // Every lane polls; the warp continues only together, since the
+            // Lane 0 polls (so idle epilogue warps do not steal issue slots
+            // from the MMA thread); the warp continues together, since the
             // TMEM loads below are warp-collective.
-            const bool ready = __all_sync(0xffffffffu, mbar_wait(&c.acc_full[acc], acc_ph, limit));
+            bool ready = true;
+            if (lane == 0) ready = mbar_wait(&c.acc_full[acc], acc_ph, limit);
+            ready = __shfl_sync(0xffffffffu, ready ? 1 : 0, 0) != 0;
             if (!ready) {
                 c.abort_flag = 1;
                 break;
             }
             tc_fence_after_sync();
             const uint32_t tbase = tmem + (uint32_t)(acc * kBN) + ((uint32_t)(q * 32) << 16);
-            const int row = row0 + r;
-            const bool valid = row < row_end;
-            if (EPI == kSwiGLU) {
-                __nv_bfloat16* orow =
-                    static_cast<__nv_bfloat16*>(p.out) + (int64_t)row * p.n_out + nt * 128;
-                const int ncols = min(128, p.n_out - nt * 128);
-#pragma unroll 1
-                for (int c0 = 0; c0 < 128; c0 += 16) {
-                    uint32_t g[16], u[16];
-                    tmem_ld16(tbase + c0, g);
-                    tmem_ld16(tbase + 128 + c0, u);
-                    tmem_ld_wait();
-                    if (valid && c0 < ncols) {
-                        uint32_t packed[8];
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            const float h0 = silu(__uint_as_float(g[2 * i])) * __uint_as_float(u[2 * i]);
-                            const float h1 = silu(__uint_as_float(g[2 * i + 1])) * __uint_as_float(u[2 * i + 1]);
-                            packed[i] = pack_bf16x2(h0, h1);
-                        }
-                        uint4* dst = reinterpret_cast<uint4*>(orow + c0);
-                        dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-                        dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
-                    }
-                }
-            } else {
-                const float wgt = valid ? __ldg(p.w_perm + row) : 0.0f;
-                const int wrow0 = row0 + q * 32;                   // first row of this warp's slab
-                const bool whole = wrow0 + 31 < row_end;           // all 32 rows belong to the group
-                float* orow = static_cast<float*>(p.out) + (int64_t)row * p.n_out + nt * kBN;
-                const int ncols = min(kBN, p.n_out - nt * kBN);
-#pragma unroll 1
-                for (int c0 = 0; c0 < kBN; c0 += kSlabCols) {
-                    uint32_t a[16];
-                    tmem_ld16(tbase + c0, a);
-                    tmem_ld_wait();
-                    if (c0 >= ncols) continue;  // warp-uniform
-                    if (whole) {
-                        float* buf = slab + slab_buf * (kSlabBytes / 4);
-                        if (lane == 0) bulk_wait_group_read<1>();  // the store that last read `buf` is done
-                        __syncwarp();
-                        // row `lane` of the slab: 4 x 16 B chunks, 64-byte swizzle
-                        float4* rowp = reinterpret_cast<float4*>(buf + lane * kSlabCols);
-                        const int sw = (lane >> 1) & 3;
-#pragma unroll
-                        for (int v = 0; v < 4; ++v)
-                            rowp[v ^ sw] = make_float4(wgt * __uint_as_float(a[4 * v]), wgt * __uint_as_float(a[4 * v + 1]),
-                                                       wgt * __uint_as_float(a[4 * v + 2]),
-                                                       wgt * __uint_as_float(a[4 * v + 3]));
-                        fence_proxy_async_smem();
-                        __syncwarp();
-                        if (lane == 0) {
-                            tma_store_2d(&tm_out, buf, nt * kBN + c0, wrow0);
-                            bulk_commit_group();
-                        }
-                        slab_buf ^= 1;
-                    } else if (valid) {
-                        float4* dst = reinterpret_cast<float4*>(orow + c0);
-#pragma unroll
-                        for (int v = 0; v < 4; ++v)
-                            dst[v] = make_float4(wgt * __uint_as_float(a[4 * v]), wgt * __uint_as_float(a[4 * v + 1]),
-                                                 wgt * __uint_as_float(a[4 * v + 2]),
-                                                 wgt * __uint_as_float(a[4 * v + 3]));
-                    }
-                }
-            }
+            epilogue_tile<EPI>(p, &tm_out, tbase, row0, row_end, nt, q, lane, hf, slab, slab_buf);
             tc_fence_before_sync();
             mbar_arrive(&c.acc_empty[acc]);
             if (++acc == 2) {

@@ -1,0 +1,253 @@
+// grouped_gemm_pair.cuh -- the grouped expert GEMM on CTA pairs
+// (tcgen05 cta_group::2), for the same work and epilogues as
+// grouped_gemm_kernel.
+//
+// A cluster of two CTAs on two SMs owns a 256-row M tile of one expert group
+// and a 256-column N tile.  Each CTA loads its own 128 rows of A and its own
+// half of the B tile (128 columns), so per SM a pipeline stage is 32 KB
+// instead of 48 KB for the same tensor work: less shared-memory fill and
+// L2->SM traffic per flop, and a deeper ring (6 stages).  The even CTA
+// issues the pair MMAs (M=256, N=256, K=16); each CTA's TMEM receives its own
+// 128 rows of the accumulator, so each CTA's epilogue drains its own rows
+// exactly like the single-CTA kernel.
+//
+// Synchronisation across the pair:
+//   full[s]      lives in the even CTA; both CTAs' TMA loads complete on it
+//                (the even CTA's producer expects the bytes of both halves)
+//   empty[s]     one per CTA; the MMA commit is multicast to both
+//   acc_full[b]  one per CTA; multicast commit
+//   acc_empty[b] lives in the even CTA; the four epilogue warps of each CTA
+//                arrive on it (remotely, for the odd CTA)
+// The pair meets at a cluster barrier after set-up and before releasing TMEM.
+// No TMA load uses multicast.
+#pragma once
+
+#include "grouped_gemm.cuh"
+
+namespace moe {
+namespace gemm {
+
+constexpr int kPairRows = 256;                        // M rows per CTA pair
+constexpr int kPairBHalfBytes = 2 * kChunkBytes;      // 128 columns x 64 k
+constexpr int kPairStageBytes = kABytes + kPairBHalfBytes;  // 32 KB per CTA
+constexpr int kPairStages = 6;
+
+struct alignas(8) PairCtrl {
+    uint64_t full[kPairStages];
+    uint64_t empty[kPairStages];
+    uint64_t acc_full[2];
+    uint64_t acc_empty[2];
+    uint64_t done;
+    uint32_t tmem_slot;
+    volatile int abort_flag;
+    int bad;
+    int total_mtiles;
+    int off[kMaxE + 1];
+    int tp[kMaxE + 1];
+};
+
+template <int EPI>
+__host__ inline size_t pair_smem_bytes()
+{
+    return 1024 + (size_t)kPairStages * kPairStageBytes + Stages<EPI>::store_bytes + sizeof(PairCtrl);
+}
+
+template <int EPI>
+__global__ void __launch_bounds__(kThreads, 1)
+    grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b0,
+                             const __grid_constant__ CUtensorMap tm_b1, const __grid_constant__ CUtensorMap tm_out,
+                             Params p)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* stage_out = smem + (size_t)kPairStages * kPairStageBytes;
+    PairCtrl& c = *reinterpret_cast<PairCtrl*>(stage_out + Stages<EPI>::store_bytes);
+
+    const int warp = threadIdx.x / 32;
+    const int lane = threadIdx.x % 32;
+    const uint64_t limit = g_wait_limit_ns;
+    const int E = p.E;
+    const uint32_t rank = cluster_ctarank();  // 0: issues the MMAs
+    const bool leader = rank == 0;
+    const int64_t pair = cluster_id_x();
+    const int64_t npairs = num_clusters_x();
+
+    build_tile_list<kPairRows>(p.offsets, E, p.M, c.off, c.tp, &c.total_mtiles, &c.bad);
+    if (threadIdx.x == 32) {
+        for (int s = 0; s < kPairStages; ++s) {
+            mbar_init(&c.full[s], 1);
+            mbar_init(&c.empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&c.acc_full[b], 1);
+            mbar_init(&c.acc_empty[b], 2 * kEpiWarps);
+        }
+        mbar_init(&c.done, 1);
+        c.abort_flag = 0;
+        fence_mbar_init();
+        tma_prefetch_map(&tm_a);
+        tma_prefetch_map(&tm_b0);
+        if (EPI == kSwiGLU) tma_prefetch_map(&tm_b1);
+        if (EPI == kWeighted) tma_prefetch_map(&tm_out);
+    }
+    if (warp == 1) {
+        __syncwarp();
+        tmem_alloc_pair(&c.tmem_slot, kTmemCols);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before_sync();
+    cluster_sync();  // both CTAs' barriers initialised and TMEM allocated
+    tc_fence_after_sync();
+    const uint32_t tmem = c.tmem_slot;
+    const int64_t total_work = c.bad ? 0 : (int64_t)c.total_mtiles * p.n_tiles;
+    const int num_kb = p.K / kBK;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ------------------------------------------------ TMA producer (both CTAs)
+            int s = 0;
+            uint32_t ph = 0;
+            int64_t issued = 0;
+            for (int64_t w = pair; w < total_work && !c.abort_flag; w += npairs) {
+                int e, row0, row_end, nt;
+                decode_tile<kPairRows>(w, p.n_tiles, c.tp, c.off, E, e, row0, row_end, nt);
+                const int krow0 = e * p.K;
+                const int arow = row0 + (int)rank * kBM;
+                bool ok = true;
+                for (int kb = 0; kb < num_kb; ++kb) {
+                    if (!mbar_wait(&c.empty[s], ph ^ 1u, limit)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t* sa = smem + (size_t)s * kPairStageBytes;
+                    uint8_t* sb = sa + kABytes;
+                    if (leader) mbar_arrive_expect_tx(&c.full[s], (uint32_t)(2 * kPairStageBytes));
+                    const uint32_t bar = mapa_shared(&c.full[s], 0);
+                    const int kr = krow0 + kb * kBK;
+                    tma_load_2d_pair(sa, &tm_a, bar, kb * kBK, arow);
+                    if (EPI == kSwiGLU) {
+                        // even CTA: the gate columns, odd CTA: the matching up columns
+                        const CUtensorMap* tb = leader ? &tm_b0 : &tm_b1;
+                        const int n0 = nt * 128;
+                        tma_load_2d_pair(sb, tb, bar, n0, kr);
+                        tma_load_2d_pair(sb + kChunkBytes, tb, bar, n0 + 64, kr);
+                    } else {
+                        const int n0 = nt * kBN + (int)rank * 128;
+                        tma_load_2d_pair(sb, &tm_b0, bar, n0, kr);
+                        tma_load_2d_pair(sb + kChunkBytes, &tm_b0, bar, n0 + 64, kr);
+                    }
+                    ++issued;
+                    if (++s == kPairStages) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
+                }
+                if (!ok) {
+                    c.abort_flag = 1;
+                    break;
+                }
+            }
+            // Never leave a copy landing in shared memory.  The even CTA's full
+            // barriers count both CTAs' copies; the odd CTA instead waits until
+            // the MMAs that read each of its stages released it (which they do
+            // only after the stage's bytes arrived).
+            for (int q = 0; q < kPairStages; ++q) {
+                const int64_t cnt = issued / kPairStages + (q < issued % kPairStages ? 1 : 0);
+                if (cnt > 0) mbar_wait(leader ? &c.full[q] : &c.empty[q], (uint32_t)(cnt - 1) & 1u, limit);
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        if (lane == 0 && leader) {
+            // ------------------------------------------------ MMA issuer (even CTA)
+            constexpr uint32_t idesc = idesc_bf16_f32(kPairRows, kBN, false, true);
+            int s = 0;
+            uint32_t ph = 0;
+            int acc = 0;
+            uint32_t acc_ph = 0;
+            for (int64_t w = pair; w < total_work && !c.abort_flag; w += npairs) {
+                if (!mbar_wait(&c.acc_empty[acc], acc_ph ^ 1u, limit)) {
+                    c.abort_flag = 1;
+                    break;
+                }
+                tc_fence_after_sync();
+                const uint32_t d_tmem = tmem + (uint32_t)(acc * kBN);
+                bool ok = true;
+                for (int kb = 0; kb < num_kb; ++kb) {
+                    if (!mbar_wait(&c.full[s], ph, limit)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after_sync();
+                    const uint32_t a_base = smem_u32(smem + (size_t)s * kPairStageBytes);
+                    const uint32_t b_base = a_base + kABytes;
+#pragma unroll
+                    for (int kk = 0; kk < kBK / 16; ++kk) {
+                        const uint64_t adesc = smem_desc_sw128(a_base + kk * 32, 16, 1024);
+                        const uint64_t bdesc = smem_desc_sw128(b_base + kk * 2048, kChunkBytes, 1024);
+                        mma_bf16_ss_pair(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
+                    }
+                    mma_commit_pair_multicast(&c.empty[s], 0x3);  // frees the stage in both CTAs
+                    if (++s == kPairStages) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
+                }
+                if (!ok) {
+                    c.abort_flag = 1;
+                    break;
+                }
+                mma_commit_pair_multicast(&c.acc_full[acc], 0x3);
+                if (++acc == 2) {
+                    acc = 0;
+                    acc_ph ^= 1u;
+                }
+            }
+            mma_commit_pair(&c.done);
+            mbar_wait(&c.done, 0, limit);
+        }
+        __syncwarp();
+    } else {
+        // ---------------------------------------------------- epilogue (both CTAs)
+        const int ew = warp - 2;
+        const int q = warp & 3;
+        const int hf = ew >> 2;
+        float* slab = reinterpret_cast<float*>(stage_out + ew * 2 * kSlabBytes);
+        int slab_buf = 0;
+        int acc = 0;
+        uint32_t acc_ph = 0;
+        for (int64_t w = pair; w < total_work; w += npairs) {
+            int e, row0, row_end, nt;
+            decode_tile<kPairRows>(w, p.n_tiles, c.tp, c.off, E, e, row0, row_end, nt);
+            bool ready = true;
+            if (lane == 0) ready = mbar_wait(&c.acc_full[acc], acc_ph, limit);
+            ready = __shfl_sync(0xffffffffu, ready ? 1 : 0, 0) != 0;
+            if (!ready) {
+                c.abort_flag = 1;
+                break;
+            }
+            tc_fence_after_sync();
+            const uint32_t tbase = tmem + (uint32_t)(acc * kBN) + ((uint32_t)(q * 32) << 16);
+            epilogue_tile<EPI>(p, &tm_out, tbase, row0 + (int)rank * kBM, row_end, nt, q, lane, hf, slab, slab_buf);
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(mapa_shared(&c.acc_empty[acc], 0));
+            if (++acc == 2) {
+                acc = 0;
+                acc_ph ^= 1u;
+            }
+        }
+        if (EPI == kWeighted && lane == 0) bulk_wait_group_all();
+        __syncwarp();
+    }
+
+    tc_fence_before_sync();
+    cluster_sync();  // both CTAs are done with TMEM and with each other's barriers
+    if (warp == 1) {
+        tc_fence_after_sync();
+        tmem_dealloc_pair(tmem, kTmemCols);
+    }
+}
+
+}  // namespace gemm
+}  // namespace moe

@@ -15,6 +15,7 @@
 #include "route.cuh"
 #include "permute.cuh"
 #include "grouped_gemm.cuh"
+#include "grouped_gemm_pair.cuh"
 #include "combine.cuh"
 
 namespace {
@@ -44,6 +45,7 @@ struct DeviceState {
     bool init = false;
     bool supported = false;
     int sm_count = 0;
+    int max_pairs = 0;  // co-resident 2-CTA clusters of the pair GEMM
 };
 
 std::mutex g_mu;
@@ -55,6 +57,35 @@ constexpr int kMaxDynSmem = 227 * 1024;
 // moe_forward's variant: the gate/up GEMM reads a materialised x_perm (the
 // fused row gather measured slower on B200, see MOE_FLAG_FUSED_GATHER).
 constexpr unsigned kDefaultForwardFlags = 0;
+
+// Grouped GEMMs on CTA pairs (tcgen05 cta_group::2) instead of single CTAs.
+#ifndef MOE_GEMM_PAIR
+#define MOE_GEMM_PAIR 1
+#endif
+
+template <int EPI>
+int launch_pair_gemm(const DeviceState& st, int64_t work, const CUtensorMap& ta, const CUtensorMap& tb0,
+                     const CUtensorMap& tb1, const CUtensorMap& tout, const moe::gemm::Params& p, cudaStream_t s)
+{
+    int64_t pairs = st.max_pairs > 0 ? st.max_pairs : st.sm_count / 2;
+    if (work < pairs) pairs = work;
+    if (pairs < 1) pairs = 1;
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3((unsigned)(2 * pairs));
+    cfg.blockDim = dim3(moe::gemm::kThreads);
+    cfg.dynamicSmemBytes = moe::gemm::pair_smem_bytes<EPI>();
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, moe::gemm::grouped_gemm_pair_kernel<EPI>, ta, tb0, tb1, tout, p) == cudaSuccess
+               ? MOE_OK
+               : MOE_ERR_CUDA;
+}
 
 int setup_device(DeviceState** out)
 {
@@ -85,6 +116,30 @@ int setup_device(DeviceState** out)
             e = e ? e : cudaFuncSetAttribute(moe::gemm::grouped_gemm_kernel<moe::gemm::kSwiGLU, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
             e = e ? e : cudaFuncSetAttribute(moe::gemm::grouped_gemm_kernel<moe::gemm::kSwiGLU, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
             e = e ? e : cudaFuncSetAttribute(moe::gemm::grouped_gemm_kernel<moe::gemm::kWeighted, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
+            e = e ? e : cudaFuncSetAttribute(moe::gemm::grouped_gemm_pair_kernel<moe::gemm::kSwiGLU>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
+            e = e ? e : cudaFuncSetAttribute(moe::gemm::grouped_gemm_pair_kernel<moe::gemm::kWeighted>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
+            if (e == cudaSuccess) {
+                // CTA pairs that can be resident at once (clusters need two
+                // SMs of one GPC, so this can be below sm_count / 2)
+                cudaLaunchConfig_t cfg = {};
+                cudaLaunchAttribute attr[1];
+                attr[0].id = cudaLaunchAttributeClusterDimension;
+                attr[0].val.clusterDim.x = 2;
+                attr[0].val.clusterDim.y = 1;
+                attr[0].val.clusterDim.z = 1;
+                cfg.gridDim = dim3(2 * (sms / 2));
+                cfg.blockDim = dim3(moe::gemm::kThreads);
+                cfg.dynamicSmemBytes = moe::gemm::pair_smem_bytes<moe::gemm::kSwiGLU>();
+                cfg.attrs = attr;
+                cfg.numAttrs = 1;
+                int n = 0;
+                if (cudaOccupancyMaxActiveClusters(&n, moe::gemm::grouped_gemm_pair_kernel<moe::gemm::kSwiGLU>,
+                                                   &cfg) != cudaSuccess) {
+                    cudaGetLastError();  // not fatal: fall back to sm_count / 2 pairs
+                    n = 0;
+                }
+                st.max_pairs = n;
+            }
             if (e != cudaSuccess) return MOE_ERR_CUDA;
         }
         st.init = true;
@@ -294,7 +349,8 @@ int run_ffn(const DeviceState& st, const moe_bf16* x_perm, const moe_bf16* x_gat
     rc = rc ? rc : make_map(&ty, y, (uint64_t)d, (uint64_t)M, kSlabCols, 32, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4,
                             CU_TENSOR_MAP_SWIZZLE_64B);
     if (rc) return rc;
-    const size_t smem = smem_bytes();
+    const size_t smem1 = smem_bytes<kSwiGLU>();
+    const size_t smem2 = smem_bytes<kWeighted>();
     const int64_t max_mtiles = (M + kBM - 1) / kBM + E;
 
     Params p1;
@@ -312,10 +368,13 @@ int run_ffn(const DeviceState& st, const moe_bf16* x_perm, const moe_bf16* x_gat
     p1.k_top = (int)k;
     const int64_t work1 = max_mtiles * p1.n_tiles;
     const unsigned grid1 = (unsigned)(work1 < st.sm_count ? work1 : st.sm_count);
-    if (gather)
-        grouped_gemm_kernel<kSwiGLU, true><<<grid1, kThreads, smem, s>>>(ta1, tg, tu, ty, p1);
+    const int64_t max_pair_tiles = (M + kPairRows - 1) / kPairRows + E;
+    if (MOE_GEMM_PAIR && !gather) {
+        if (launch_pair_gemm<kSwiGLU>(st, max_pair_tiles * p1.n_tiles, ta1, tg, tu, ty, p1, s)) return MOE_ERR_CUDA;
+    } else if (gather)
+        grouped_gemm_kernel<kSwiGLU, true><<<grid1, kThreads, smem1, s>>>(ta1, tg, tu, ty, p1);
     else
-        grouped_gemm_kernel<kSwiGLU, false><<<grid1, kThreads, smem, s>>>(ta1, tg, tu, ty, p1);
+        grouped_gemm_kernel<kSwiGLU, false><<<grid1, kThreads, smem1, s>>>(ta1, tg, tu, ty, p1);
     if (launch_status()) return MOE_ERR_CUDA;
     if (mid_event && cudaEventRecord(mid_event, s) != cudaSuccess) return MOE_ERR_CUDA;
 
@@ -334,7 +393,11 @@ int run_ffn(const DeviceState& st, const moe_bf16* x_perm, const moe_bf16* x_gat
     p2.k_top = 1;
     const int64_t work2 = max_mtiles * p2.n_tiles;
     const unsigned grid2 = (unsigned)(work2 < st.sm_count ? work2 : st.sm_count);
-    grouped_gemm_kernel<kWeighted, false><<<grid2, kThreads, smem, s>>>(ta2, td, td, ty, p2);
+    if (MOE_GEMM_PAIR) {
+        if (launch_pair_gemm<kWeighted>(st, max_pair_tiles * p2.n_tiles, ta2, td, td, ty, p2, s)) return MOE_ERR_CUDA;
+        return launch_status();
+    }
+    grouped_gemm_kernel<kWeighted, false><<<grid2, kThreads, smem2, s>>>(ta2, td, td, ty, p2);
     return launch_status();
 }
 
