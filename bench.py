@@ -38,8 +38,8 @@ UNIT = "tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_FLUSH_BYTES = 256 << 20
 STAGES = ("route", "permute", "gateup_gemm", "down_gemm", "combine")
-# router GEMM, softmax/top-k, chunk scan, rank, row gather, gate/up GEMM, down GEMM, combine
-KERNELS_PER_FORWARD = 8
+# router (GEMM + softmax + top-k), chunk scan, rank, row gather, gate/up GEMM, down GEMM, combine
+KERNELS_PER_FORWARD = 7
 
 
 # ------------------------------------------------------------- host logic

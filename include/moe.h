@@ -89,24 +89,27 @@ int moe_version(void);
  */
 size_t moe_workspace_size(int64_t T, int64_t d, int64_t E, int64_t k, int64_t f);
 
-/* Bytes of scratch that moe_route needs (fp32 partial router logits). */
+/* Bytes of scratch that moe_route needs: 0 for every supported shape (the
+ * logits stay on chip).  Kept so that callers size the argument the same
+ * way for every entry point. */
 size_t moe_route_workspace_size(int64_t T, int64_t d, int64_t E);
 
 /* Bytes of scratch that moe_permute needs (per-chunk expert counts). */
 size_t moe_permute_workspace_size(int64_t T, int64_t E, int64_t k);
 
 /*
- * Stage 1-2: router GEMM, fp32 softmax over E, top-k (section 1 listing:
- * gate linear, softmax over dim 1, topk; no renormalisation follows).
+ * Stage 1-2: router GEMM, fp32 softmax over E, top-k (section 1: gate
+ * linear, softmax over the experts, topk; no renormalisation follows).
  *   x        [T, d]    bf16
  *   w_router [d, E]    bf16
  *   bias     [E]       fp32, or NULL for no bias
  *   topk_ids [T, k]    int32 out, slot j = j-th largest probability
  *   topk_w   [T, k]    fp32  out, the softmax probability of that expert
- *   workspace          device scratch of moe_route_workspace_size bytes,
- *                      16-byte aligned
- * Logits are accumulated in fp32 on the tensor cores (in a few slices of the
- * hidden dimension, summed in a fixed order) and never rounded to bf16.
+ *   workspace          device scratch of moe_route_workspace_size bytes
+ *                      (NULL when that is 0), 16-byte aligned
+ * One kernel: logits are accumulated in fp32 on the tensor cores over the
+ * whole hidden dimension, stay in tensor memory and are never rounded to
+ * bf16; softmax and top-k run in the same kernel's epilogue.
  * Selection compares the fp32 logits (softmax is monotone); ties go to the
  * lower expert index.
  */

@@ -49,8 +49,7 @@ def test_workspace_sizes(moe_lib):
     assert moe.workspace_size(8192, 2048, 128, 33, 768) == 0     # k > 32
     assert moe.workspace_size(0, 2048, 128, 8, 768) > 0
     assert moe.permute_workspace_size(8192, 128, 8) == (8192 // 64) * 128 * 4
-    assert moe.route_workspace_size(8192, 2048, 128) % 256 == 0
-    assert moe.route_workspace_size(8192, 2048, 128) >= 8192 * 128 * 4
+    assert moe.route_workspace_size(8192, 2048, 128) == 0   # logits stay on chip
     assert moe.route_workspace_size(8192, 2048, 12) == 0
 
 
@@ -67,8 +66,8 @@ def test_validation_happens_before_any_device_call(moe_lib):
     odd = ctypes.c_void_p(0x1001)
     assert L.moe_route(odd, odd, null, 16, 64, 8, 2, odd, odd, odd, 1 << 20, null) == moe.MOE_ERR_INVALID_ARG
     fake = ctypes.c_void_p(0x10000)
-    assert L.moe_route(fake, fake, null, 16, 64, 8, 2, fake, fake, fake, 16, null) == \
-        moe.MOE_ERR_WORKSPACE_TOO_SMALL
+    assert L.moe_permute(fake, fake, fake, 1000, 64, 8, 2, fake, fake, fake, fake, null, fake, fake, 16,
+                         null) == moe.MOE_ERR_WORKSPACE_TOO_SMALL
     # unknown flag bits
     assert L.moe_forward_ex(fake, fake, null, fake, fake, fake, 16, 64, 8, 2, 64, fake, null, null, fake, 1 << 30,
                             null, null, 0, 6) == moe.MOE_ERR_INVALID_ARG

@@ -156,12 +156,11 @@ def route(x, w_router, k, bias=None, topk_ids=None, topk_w=None, workspace=None)
     if topk_w is None:
         topk_w = torch.empty(T, k, dtype=torch.float32, device=x.device)
     need = route_workspace_size(T, d, E)
-    if need == 0 and T > 0:
-        raise MoEError(MOE_ERR_UNSUPPORTED_SHAPE, "moe_route_workspace_size")
-    if workspace is None or workspace.numel() < need:
+    if need > 0 and (workspace is None or workspace.numel() < need):
         workspace = _workspace(need, x.device)
+    ws_bytes = 0 if workspace is None else workspace.numel()
     _check(lib().moe_route(_ptr(x), _ptr(w_router), _ptr(bias), T, d, E, k, _ptr(topk_ids),
-                           _ptr(topk_w), _ptr(workspace), workspace.numel(), _stream()), "moe_route")
+                           _ptr(topk_w), _ptr(workspace), ws_bytes, _stream()), "moe_route")
     return topk_ids, topk_w
 
 

@@ -112,7 +112,12 @@ int setup_device(DeviceState** out)
                 g_encode = reinterpret_cast<EncodeTiledFn>(fn);
             }
             cudaError_t e = cudaSuccess;
-            e = e ? e : cudaFuncSetAttribute(moe::route::logits_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
+            e = e ? e : cudaFuncSetAttribute(moe::route::route_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
+            e = e ? e : cudaFuncSetAttribute(moe::route::route_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
+            e = e ? e : cudaFuncSetAttribute(moe::route::route_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
+            e = e ? e : cudaFuncSetAttribute(moe::route::route_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
+            e = e ? e : cudaFuncSetAttribute(moe::route::route_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
+            e = e ? e : cudaFuncSetAttribute(moe::route::route_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
             e = e ? e : cudaFuncSetAttribute(moe::gemm::grouped_gemm_kernel<moe::gemm::kSwiGLU, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
             e = e ? e : cudaFuncSetAttribute(moe::gemm::grouped_gemm_kernel<moe::gemm::kSwiGLU, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
             e = e ? e : cudaFuncSetAttribute(moe::gemm::grouped_gemm_kernel<moe::gemm::kWeighted, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
@@ -193,36 +198,17 @@ int make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, u
 inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
 // ---------------------------------------------------------- work shapes
-// Router: CTAs own 128 tokens and one of `slices` parts of the hidden
-// dimension.  The split aims at about two CTAs per SM of a 148-SM B200 and
-// keeps at least four 64-wide k-blocks per CTA.  It depends on the shape
-// only, so workspace sizes can be computed without a device.
-constexpr int64_t kRouterTargetCtas = 296;
-
-int router_slices(int64_t T, int64_t d)
-{
-    const int64_t tiles = (T + moe::route::kBM - 1) / moe::route::kBM;
-    const int64_t num_kb = d / moe::route::kBK;
-    int64_t s = tiles > 0 ? kRouterTargetCtas / tiles : 1;
-    int64_t cap = num_kb / 4 > 0 ? num_kb / 4 : 1;
-    if (cap > moe::route::kMaxSlices) cap = moe::route::kMaxSlices;
-    if (s > cap) s = cap;
-    if (s < 1) s = 1;
-    return (int)s;
-}
-
 inline int64_t token_chunks(int64_t T) { return (T + moe::permute::kTokensPerChunk - 1) / moe::permute::kTokensPerChunk; }
 
-size_t route_ws_bytes(int64_t T, int64_t d, int64_t E)
-{
-    return align256((size_t)router_slices(T, d) * (size_t)T * (size_t)E * 4);
-}
+// The router keeps its logits on chip and needs no scratch; the workspace
+// argument of moe_route stays in the ABI for a future split-K router.
+size_t route_ws_bytes(int64_t, int64_t, int64_t) { return 0; }
 
 size_t permute_ws_bytes(int64_t T, int64_t E) { return align256((size_t)token_chunks(T) * (size_t)E * 4); }
 
 // Workspace carve-up for moe_forward.
 struct Layout {
-    size_t ids, wts, counts, offsets, chunk, part, perm, inv, w_perm, x_perm, h, y, total;
+    size_t ids, wts, counts, offsets, chunk, perm, inv, w_perm, x_perm, h, y, total;
 };
 
 Layout plan(int64_t T, int64_t d, int64_t E, int64_t k, int64_t f)
@@ -235,7 +221,6 @@ Layout plan(int64_t T, int64_t d, int64_t E, int64_t k, int64_t f)
     L.counts = o;  o += align256((size_t)E * 4);
     L.offsets = o; o += align256((size_t)(E + 1) * 4);
     L.chunk = o;   o += permute_ws_bytes(T, E);
-    L.part = o;    o += route_ws_bytes(T, d, E);
     L.perm = o;    o += align256(M * 4);
     L.inv = o;     o += align256(M * 4);
     L.w_perm = o;  o += align256(M * 4);
@@ -247,11 +232,23 @@ Layout plan(int64_t T, int64_t d, int64_t E, int64_t k, int64_t f)
 }
 
 // ------------------------------------------------------------ launchers
-// Router GEMM (partial logits into `part`) and the softmax / top-k.  With
-// chunk_counts set, the softmax kernel also fills the per-chunk expert
-// histogram the permutation needs.
+// Router GEMM, softmax and top-k in one kernel.  With chunk_counts set, it
+// also writes the per-chunk expert histogram the permutation needs.
+template <int KMAX>
+int launch_route(const CUtensorMap& tx, const CUtensorMap& tw, moe::route::Params p, unsigned tiles,
+                 cudaStream_t s)
+{
+    using moe::route::smem_bytes;
+    // one CTA per SM: the deepest ring that fits (2 to 8 stages)
+    p.stages = moe::route::kMaxStages;
+    while (p.stages > 2 && smem_bytes<KMAX>(p.n_chunks, p.stages, p.E) > (size_t)kMaxDynSmem) --p.stages;
+    const size_t smem = smem_bytes<KMAX>(p.n_chunks, p.stages, p.E);
+    moe::route::route_kernel<KMAX><<<tiles, moe::route::Shape<KMAX>::threads, smem, s>>>(tx, tw, p);
+    return launch_status();
+}
+
 int run_route(const moe_bf16* x, const moe_bf16* w_router, const float* bias, int64_t T, int64_t d, int64_t E,
-              int64_t k, int32_t* ids, float* wts, float* part, int32_t* chunk_counts, cudaStream_t s)
+              int64_t k, int32_t* ids, float* wts, int32_t* chunk_counts, cudaStream_t s)
 {
     if (T == 0) return MOE_OK;
     CUtensorMap tx, tw;
@@ -259,42 +256,32 @@ int run_route(const moe_bf16* x, const moe_bf16* w_router, const float* bias, in
     if (rc) return rc;
     rc = make_map(&tw, w_router, (uint64_t)E, (uint64_t)d, 64, 64);
     if (rc) return rc;
+    int kmax = 1;
+    while (kmax < k) kmax <<= 1;
     moe::route::Params p;
-    p.part = part;
+    p.bias = bias;
+    p.ids = ids;
+    p.wts = wts;
+    p.chunk_counts = chunk_counts;
+    p.n_tchunks = (int)token_chunks(T);
     p.T = (int)T;
     p.d = (int)d;
     p.E = (int)E;
+    p.k = (int)k;
     p.n_chunks = (int)((E + 63) / 64);
-    p.slices = router_slices(T, d);
-    p.zero = chunk_counts;
-    p.zero_count = chunk_counts ? (int64_t)E * token_chunks(T) : 0;
-    // deepest ring that still lets two CTAs share an SM (at least 2 stages)
-    p.stages = 4;
-    while (p.stages > 2 && moe::route::smem_bytes(p.n_chunks, p.stages) > (size_t)(113 * 1024)) --p.stages;
+    p.stages = 0;  // set per list length
     uint32_t cols = 64;
     while (cols < (uint32_t)(64 * p.n_chunks)) cols <<= 1;
     p.tmem_cols = cols;
-    const size_t smem = moe::route::smem_bytes(p.n_chunks, p.stages);
-    const int64_t tiles = (T + moe::route::kBM - 1) / moe::route::kBM;
-    moe::route::logits_kernel<<<(unsigned)(tiles * p.slices), moe::route::kThreads, smem, s>>>(tx, tw, p);
-    if (launch_status()) return MOE_ERR_CUDA;
-
-    const int64_t nch = token_chunks(T);
-    const size_t hist_smem = 0;
-    const unsigned blocks = (unsigned)((T + moe::route::kSoftmaxWarps - 1) / moe::route::kSoftmaxWarps);
-    const int threads = moe::route::kSoftmaxWarps * 32;
-    const int vpl = (int)((E + 31) / 32);
-    if (vpl <= 1)
-        moe::route::softmax_topk_kernel<1><<<blocks, threads, hist_smem, s>>>(part, bias, (int)T, (int)E, (int)k, p.slices, ids, wts, chunk_counts, (int)nch);
-    else if (vpl <= 2)
-        moe::route::softmax_topk_kernel<2><<<blocks, threads, hist_smem, s>>>(part, bias, (int)T, (int)E, (int)k, p.slices, ids, wts, chunk_counts, (int)nch);
-    else if (vpl <= 4)
-        moe::route::softmax_topk_kernel<4><<<blocks, threads, hist_smem, s>>>(part, bias, (int)T, (int)E, (int)k, p.slices, ids, wts, chunk_counts, (int)nch);
-    else if (vpl <= 8)
-        moe::route::softmax_topk_kernel<8><<<blocks, threads, hist_smem, s>>>(part, bias, (int)T, (int)E, (int)k, p.slices, ids, wts, chunk_counts, (int)nch);
-    else
-        moe::route::softmax_topk_kernel<16><<<blocks, threads, hist_smem, s>>>(part, bias, (int)T, (int)E, (int)k, p.slices, ids, wts, chunk_counts, (int)nch);
-    return launch_status();
+    const unsigned tiles = (unsigned)((T + moe::route::kBM - 1) / moe::route::kBM);
+    switch (kmax) {
+        case 1: return launch_route<1>(tx, tw, p, tiles, s);
+        case 2: return launch_route<2>(tx, tw, p, tiles, s);
+        case 4: return launch_route<4>(tx, tw, p, tiles, s);
+        case 8: return launch_route<8>(tx, tw, p, tiles, s);
+        case 16: return launch_route<16>(tx, tw, p, tiles, s);
+        default: return launch_route<32>(tx, tw, p, tiles, s);
+    }
 }
 
 // Grouping by expert.  have_hist: chunk_em already holds the per-chunk
@@ -444,7 +431,6 @@ int forward_impl(const moe_bf16* x, const moe_bf16* w_router, const float* bias,
     int32_t* counts = reinterpret_cast<int32_t*>(w + L.counts);
     int32_t* offsets = reinterpret_cast<int32_t*>(w + L.offsets);
     int32_t* chunk = reinterpret_cast<int32_t*>(w + L.chunk);
-    float* part = reinterpret_cast<float*>(w + L.part);
     int32_t* perm = reinterpret_cast<int32_t*>(w + L.perm);
     int32_t* inv = reinterpret_cast<int32_t*>(w + L.inv);
     float* w_perm = reinterpret_cast<float*>(w + L.w_perm);
@@ -453,7 +439,7 @@ int forward_impl(const moe_bf16* x, const moe_bf16* w_router, const float* bias,
     float* y = reinterpret_cast<float*>(w + L.y);
     const bool gather = (flags & MOE_FLAG_FUSED_GATHER) != 0;
 
-    if ((rc = run_route(x, w_router, bias, T, d, E, k, ids, wts, part, chunk, s))) return rc;
+    if ((rc = run_route(x, w_router, bias, T, d, E, k, ids, wts, chunk, s))) return rc;
     if ((rc = rec(1))) return rc;
     if ((rc = run_permute(x, ids, wts, T, d, E, k, counts, offsets, perm, inv, gather ? nullptr : x_perm, w_perm,
                           chunk, true, s)))
@@ -551,11 +537,9 @@ int moe_route(const moe_bf16* x, const moe_bf16* w_router, const float* bias, in
         !aligned(topk_w, 4) || !aligned(workspace, 16))
         return MOE_ERR_INVALID_ARG;
     if (workspace_bytes < route_ws_bytes(T, d, E)) return MOE_ERR_WORKSPACE_TOO_SMALL;
-    if (T > 0 && !workspace) return MOE_ERR_INVALID_ARG;
     DeviceState* st = nullptr;
     if ((rc = setup_device(&st))) return rc;
-    return run_route(x, w_router, bias, T, d, E, k, topk_ids, topk_w, static_cast<float*>(workspace), nullptr,
-                     stream);
+    return run_route(x, w_router, bias, T, d, E, k, topk_ids, topk_w, nullptr, stream);
 }
 
 int moe_permute(const moe_bf16* x, const int32_t* topk_ids, const float* topk_w, int64_t T, int64_t d, int64_t E,
