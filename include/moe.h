@@ -4,7 +4,7 @@
  * The operation is the forward pass of a top-k routed MoE block as defined by
  * the article "Qwen3MoeSparseMoeBlock performance optimisation in practice"
  * (parallelising a sparse mixture-of-experts system), section 1: the forward()
- * listing and the four-stage workflow above it (router linear + softmax,
+ * code and the four-stage workflow above it (router linear + softmax,
  * top-k selection, per-expert computation, routing-weighted aggregation),
  * restaged in its section 2.2 as route -> sort tokens by expert -> batched
  * expert compute -> scatter back.  Notation: T tokens, d hidden size, E
@@ -17,19 +17,24 @@
  *                 equal values rank the lower expert index first
  *   w[t,j]      = p[t, ids[t,j]]                      (NOT renormalised)
  *   h           = silu(x[t] . W_gate[e]) * (x[t] . W_up[e]),  silu(z) = z/(1+e^-z)
- *   y[t,j]      = w[t,j] * (h . W_down[e]),  e = ids[t,j]      (fp32)
+ *   y[t,j]      = w[t,j] * (h . W_down[e]),  e = ids[t,j]      (fp32, stored fp16)
  *   out[t]      = sum_j y[t,j]                                  (fp32)
  * Precision: bf16 inputs, fp32 accumulation everywhere.  h is rounded to
- * bf16 once, because it is the operand of the second bf16 tensor-core GEMM;
- * y and out are never rounded below fp32.
+ * bf16 once, because it is the operand of the second bf16 tensor-core GEMM.
+ * Each slot's contribution y is computed in fp32 and stored once as IEEE
+ * fp16 (11-bit significand, relative error <= 2^-11): it is the block's
+ * largest intermediate, and fp16 keeps the output within its tolerance
+ * where bf16 would not.  The k-way sum and out stay fp32.  A y outside the
+ * fp16 range (|y| >= 65520) or NaN is stored as inf / NaN and reported as
+ * MOE_ERR_DEVICE_RANGE.
  * The optional per-expert bias follows the gate G(x) = Softmax(W_g x + b_g)
  * of the Hunyuan-Large overview page, section 2.1.
  *
  * Conventions shared by every entry point
  * ---------------------------------------
  * - Pointers named x, w_*, h, x_perm are DEVICE pointers to bf16 (IEEE
- *   bfloat16 bit patterns, type moe_bf16); y and out are DEVICE pointers to
- *   fp32.  All are row-major, contiguous and 16-byte aligned.  Other int32 /
+ *   bfloat16 bit patterns, type moe_bf16); y is a DEVICE pointer to IEEE
+ *   fp16 bit patterns (type moe_f16); out is a DEVICE pointer to fp32.  All are row-major, contiguous and 16-byte aligned.  Other int32 /
  *   fp32 arrays are device pointers, 4-byte aligned.
  *   The caller owns every buffer; the library never allocates, frees or
  *   synchronises (except moe_get_status), in line with the article's
@@ -37,7 +42,8 @@
  * - Work is enqueued on `stream` and runs asynchronously; a return value of
  *   MOE_OK means the arguments were valid and every launch was accepted.
  * - Errors detected on the device (an expert id out of range, corrupt group
- *   offsets, a pipeline wait that ran past its time limit) are written to a
+ *   offsets, a pipeline wait that ran past its time limit, a y value outside
+ *   the fp16 range) are written to a
  *   per-device status word and reported by moe_get_status.  The kernel that
  *   detects one skips the offending access and finishes without faulting.
  * - Shapes (MOE_ERR_UNSUPPORTED_SHAPE otherwise):
@@ -61,6 +67,8 @@ extern "C" {
 
 /* IEEE bfloat16 bit pattern. */
 typedef uint16_t moe_bf16;
+/* IEEE binary16 (fp16) bit pattern. */
+typedef uint16_t moe_f16;
 
 typedef enum {
     MOE_OK = 0,
@@ -71,7 +79,8 @@ typedef enum {
     MOE_ERR_DEVICE_TIMEOUT = 5,      /* device: a pipeline wait ran past its limit */
     MOE_ERR_DEVICE_BOUNDS = 6,       /* device: index data out of range (ids, offsets, inv) */
     MOE_ERR_UNSUPPORTED_DEVICE = 7,  /* not a compute-capability 10.0 GPU */
-    MOE_ERR_STATIC_SCRATCH_TOO_SMALL = 8 /* moe_permute_static: E * ceil(T/64) > 262144 */
+    MOE_ERR_STATIC_SCRATCH_TOO_SMALL = 8, /* moe_permute_static: E * ceil(T/64) > 262144 */
+    MOE_ERR_DEVICE_RANGE = 9         /* device: a y value outside the fp16 range, or NaN */
 } moe_status_t;
 
 /* Human-readable name of a status code (static string, never NULL). */
@@ -84,7 +93,7 @@ int moe_version(void);
  * Bytes of scratch that moe_forward needs for these sizes (0 if the shape is
  * unsupported).  The pieces, each 256-byte aligned, are: topk ids and
  * weights [M], counts [E], offsets [E+1], per-chunk group bases, perm / inv /
- * w_perm [M], h [M,f] bf16 and y [M,d] fp32.  (moe_forward never builds
+ * w_perm [M], h [M,f] bf16 and y [M,d] fp16.  (moe_forward never builds
  * x_perm: its gate/up GEMM gathers the rows of x through perm directly.)
  */
 size_t moe_workspace_size(int64_t T, int64_t d, int64_t E, int64_t k, int64_t f);
@@ -175,24 +184,25 @@ int moe_permute_static(const moe_bf16* x, const int32_t* topk_ids, const float* 
  * for offsets[e] <= pos < offsets[e+1].
  *   x_perm  [M, d] bf16,  w_perm [M] fp32,  offsets [E+1] int32 (device)
  *   w_gate, w_up [E, d, f] bf16;  w_down [E, f, d] bf16
- *   h [M, f] bf16 out (also the caller's scratch),  y [M, d] fp32 out
+ *   h [M, f] bf16 out (also the caller's scratch),  y [M, d] fp16 out
  * offsets must be non-decreasing with offsets[0] = 0 and offsets[E] = M;
  * otherwise MOE_ERR_DEVICE_BOUNDS is reported and nothing is written.
  */
 int moe_expert_ffn(const moe_bf16* x_perm, const float* w_perm, const int32_t* offsets,
                    const moe_bf16* w_gate, const moe_bf16* w_up, const moe_bf16* w_down,
                    int64_t M, int64_t d, int64_t E, int64_t f,
-                   moe_bf16* h, float* y, cudaStream_t stream);
+                   moe_bf16* h, moe_f16* y, cudaStream_t stream);
 
 /*
  * Weighted aggregation back to token order (section 1, stage 4; section 2.2
  * scatter_outputs), without atomics:
  *   out[t] = sum_{j = 0..k-1} y[inv[t*k + j]]   (fp32 sum in slot order)
- *   y [T*k, d] fp32 (already multiplied by the routing weight),
+ *   y [T*k, d] fp16 (already multiplied by the routing weight; widened to
+ *   fp32 before the sum),
  *   inv [T*k] int32 (entries outside [0, T*k) are reported as
  *   MOE_ERR_DEVICE_BOUNDS and skipped), out [T, d] fp32.
  */
-int moe_combine(const float* y, const int32_t* inv, int64_t T, int64_t d, int64_t k,
+int moe_combine(const moe_f16* y, const int32_t* inv, int64_t T, int64_t d, int64_t k,
                 float* out, cudaStream_t stream);
 
 /*

@@ -30,3 +30,22 @@ def test_wait_limit_setting_roundtrip():
     d = gc.on_device(gc.inputs(cfg))
     moe.forward(d["x"], d["w_router"], d["w_gate"], d["w_up"], d["w_down"], 2)
     assert moe.get_status() == moe.MOE_OK
+
+
+def test_y_outside_fp16_range_is_reported():
+    """y is stored as fp16.  A block whose contributions exceed the fp16 range
+    (here W_down scaled by 2^30, so |y| reaches about 1e6) stores inf and
+    reports MOE_ERR_DEVICE_RANGE;
+    the context stays usable and an in-range call is clean again."""
+    cfg = gc.small_cfg(256, 128, 8, 2, 128)
+    d = gc.on_device(gc.inputs(cfg))
+    assert moe.get_status() == moe.MOE_OK
+    big = (d["w_down"].float() * 2.0 ** 30).to(torch.bfloat16)
+    out = moe.forward(d["x"], d["w_router"], d["w_gate"], d["w_up"], big, 2)
+    torch.cuda.synchronize()
+    assert moe.get_status() == moe.MOE_ERR_DEVICE_RANGE
+    assert not torch.isfinite(out).all().item()
+    out = moe.forward(d["x"], d["w_router"], d["w_gate"], d["w_up"], d["w_down"], 2)
+    torch.cuda.synchronize()
+    assert moe.get_status() == moe.MOE_OK
+    assert torch.isfinite(out).all().item()

@@ -63,11 +63,12 @@ def test_ffn_and_combine_small(cfg):
 
 
 def test_combine_exact_fp32_sum():
-    """The combine is an fp32 sum in slot order: an fp32 numpy sum of the same
-    rows in the same order matches bit for bit."""
+    """The combine widens the fp16 rows to fp32 and sums them in slot order:
+    an fp32 numpy sum of the same widened rows in the same order matches bit
+    for bit."""
     cfg = gc.small_cfg(777, 192, 16, 4, 64)
     inp, d, ids, w, pm, h, y, out = _stages(cfg)
-    yf = y.cpu().numpy()
+    yf = y.cpu().numpy().astype(np.float32)   # fp16 -> fp32 is exact
     inv = pm["inv"].cpu().numpy().reshape(cfg.T, cfg.k)
     acc = np.zeros((cfg.T, cfg.d), np.float32)
     for j in range(cfg.k):

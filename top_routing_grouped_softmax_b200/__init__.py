@@ -31,6 +31,7 @@ MOE_ERR_DEVICE_TIMEOUT = 5
 MOE_ERR_DEVICE_BOUNDS = 6
 MOE_ERR_UNSUPPORTED_DEVICE = 7
 MOE_ERR_STATIC_SCRATCH_TOO_SMALL = 8
+MOE_ERR_DEVICE_RANGE = 9
 
 # Every symbol include/moe.h declares.
 ABI_SYMBOLS = (
@@ -191,7 +192,7 @@ def permute(x, topk_ids, topk_w, E, gather=True):
 
 
 def expert_ffn(x_perm, w_perm, offsets, w_gate, w_up, w_down, h=None, y=None):
-    """Grouped gate/up + SwiGLU and grouped down + routing weight; returns (h bf16, y fp32)."""
+    """Grouped gate/up + SwiGLU and grouped down + routing weight; returns (h bf16, y fp16)."""
     _need(x_perm, "x_perm", torch.bfloat16, 2)
     _need(w_perm, "w_perm", torch.float32, 1)
     _need(offsets, "offsets", torch.int32, 1)
@@ -202,16 +203,16 @@ def expert_ffn(x_perm, w_perm, offsets, w_gate, w_up, w_down, h=None, y=None):
     if h is None:
         h = torch.empty(M, f, dtype=torch.bfloat16, device=x_perm.device)
     if y is None:
-        y = torch.empty(M, d, dtype=torch.float32, device=x_perm.device)
-    _need(y, "y", torch.float32, 2)
+        y = torch.empty(M, d, dtype=torch.float16, device=x_perm.device)
+    _need(y, "y", torch.float16, 2)
     _check(lib().moe_expert_ffn(_ptr(x_perm), _ptr(w_perm), _ptr(offsets), _ptr(w_gate), _ptr(w_up),
                                 _ptr(w_down), M, d, E, f, _ptr(h), _ptr(y), _stream()), "moe_expert_ffn")
     return h, y
 
 
 def combine(y, inv, T, k, out=None):
-    """out[t] = sum_j y[inv[t*k+j]] (fp32 rows, fp32 sum, fp32 result)."""
-    _need(y, "y", torch.float32, 2)
+    """out[t] = sum_j y[inv[t*k+j]] (fp16 rows widened to fp32, fp32 sum, fp32 result)."""
+    _need(y, "y", torch.float16, 2)
     _need(inv, "inv", torch.int32, 1)
     d = y.shape[1]
     if out is None:

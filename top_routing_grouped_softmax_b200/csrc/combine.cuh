@@ -4,10 +4,13 @@
 // (section 1: expert outputs summed per token, weighted by the routing
 // weights; section 2.2 scatter_outputs).  The weight is already folded into
 // y by the down-projection epilogue, so each token gathers its k grouped
-// fp32 rows through inv and sums them in fp32 in slot order -- a gather, not
-// a scatter-add, so no atomics and a deterministic result.  The output stays
-// fp32: the accumulation is never rounded to a narrower type.
+// fp16 rows through inv, widens them to fp32 and sums them in fp32 in slot
+// order -- a gather, not a scatter-add, so no atomics and a deterministic
+// result.  The output stays fp32: the accumulation is never rounded to a
+// narrower type.
 #pragma once
+
+#include <cuda_fp16.h>
 
 #include "status.cuh"
 
@@ -16,8 +19,9 @@ namespace combine {
 
 constexpr int kMaxK = 32;
 
-// One block per token; thread v handles 4 consecutive columns (16 bytes).
-__global__ void __launch_bounds__(256) combine_kernel(const float4* __restrict__ y, const int32_t* __restrict__ inv,
+// One block per token; thread v handles 8 consecutive columns (16 bytes of
+// y, 32 bytes of out).
+__global__ void __launch_bounds__(256) combine_kernel(const uint4* __restrict__ y, const int32_t* __restrict__ inv,
                                                       int64_t n, int nvec, int k, float4* __restrict__ out)
 {
     __shared__ int s_pos[kMaxK];
@@ -32,19 +36,26 @@ __global__ void __launch_bounds__(256) combine_kernel(const float4* __restrict__
     }
     __syncthreads();
     for (int v = threadIdx.x; v < nvec; v += blockDim.x) {
-        float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        float acc[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
 #pragma unroll 4
         for (int j = 0; j < k; ++j) {
             const int p = s_pos[j];
             if (p >= 0) {
-                const float4 q = __ldg(y + (int64_t)p * nvec + v);
-                acc.x += q.x;
-                acc.y += q.y;
-                acc.z += q.z;
-                acc.w += q.w;
+                const uint4 q = __ldg(y + (int64_t)p * nvec + v);
+                const __half2* h = reinterpret_cast<const __half2*>(&q);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float2 f = __half22float2(h[i]);
+                    acc[2 * i] += f.x;
+                    acc[2 * i + 1] += f.y;
+                }
             }
         }
-        out[t * nvec + v] = acc;
+        float4* o = out + (t * nvec + v) * 2;
+        o[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        o[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
     }
 }
 

@@ -42,15 +42,21 @@
 //   kSwiGLU   : B columns 0..127 come from W_gate, 128..255 from W_up for the
 //               same 128 output columns; h = silu(g) * u, silu(z) = z/(1+e^-z),
 //               stored as bf16 (h is the next GEMM's bf16 operand)
-//   kWeighted : y = w_perm[row] * acc in fp32 (the routing weight applied
-//               after the down projection; y stays fp32 so that the k-way sum
-//               in the combine is an fp32 accumulation of unrounded terms).
-//               Each warp stages 32 rows x 16 columns in shared memory and
+//   kWeighted : y = w_perm[row] * acc, computed in fp32 and stored as IEEE
+//               fp16 (the routing weight applied after the down projection).
+//               One rounding to an 11-bit significand (relative error
+//               <= 2^-11) keeps the combine's fp32 k-way sum well inside the
+//               output tolerance, where bf16 (8 bits) would not, at half the
+//               bytes of fp32 -- y is the largest stream of the block.  A value
+//               that fp16 cannot hold (|y| >= 65520, or NaN) is stored as is
+//               (inf / NaN) and reported as a range error.
+//               Each warp stages 32 rows x 32 columns in shared memory and
 //               writes them with one TMA store, so global writes are whole
 //               64-byte row segments instead of per-thread scattered stores.
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include "ptx.cuh"
 
@@ -80,8 +86,8 @@ constexpr int kBBytes = 4 * kChunkBytes;    // 32 KB
 constexpr int kStageBytes = kABytes + kBBytes;
 constexpr uint32_t kTmemCols = 512;         // 2 accumulators x 256 columns
 constexpr int kMaxE = 512;
-constexpr int kSlabCols = 16;               // fp32 columns per TMA-store slab (64 B rows)
-constexpr int kSlabBytes = 32 * kSlabCols * 4;     // 32 rows x 16 fp32 = 2 KB
+constexpr int kSlabCols = 32;               // fp16 columns per TMA-store slab (64 B rows)
+constexpr int kSlabBytes = 32 * kSlabCols * 2;     // 32 rows x 32 fp16 = 2 KB
 constexpr int kStoreBytes = kEpiWarps * 2 * kSlabBytes;  // 2 buffers per epilogue warp
 
 // Ring depth and store staging per epilogue: the down GEMM gives up one
@@ -100,7 +106,7 @@ struct Params {
     const int32_t* perm;     // [M] grouped row -> flat assignment t*k + j (GATHER)
     const __nv_bfloat16* x;  // [T, ldx] token matrix the A rows are gathered from (GATHER)
     int64_t ldx;             // row length of x in elements (= K for the gate/up GEMM)
-    void* out;               // [M, n_out]: bf16 h (kSwiGLU) or fp32 y (kWeighted)
+    void* out;               // [M, n_out]: bf16 h (kSwiGLU) or fp16 y (kWeighted)
     int E;
     int M;        // grouped rows
     int K;        // reduction length (multiple of 64)
@@ -207,6 +213,16 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b)
 
 __device__ __forceinline__ float silu(float z) { return z / (1.0f + __expf(-z)); }
 
+// fp16 pair of w * a, w * b (round to nearest even); `bad` is set when either
+// product is outside the fp16 range (|v| >= 65520 rounds to inf) or NaN.
+__device__ __forceinline__ uint32_t scaled_f16x2(float w, uint32_t a, uint32_t b, bool& bad)
+{
+    const float va = w * __uint_as_float(a), vb = w * __uint_as_float(b);
+    bad |= !(fabsf(va) < 65520.0f) || !(fabsf(vb) < 65520.0f);
+    const __half2 h = __floats2half2_rn(va, vb);
+    return *reinterpret_cast<const uint32_t*>(&h);
+}
+
 // Token row of x for grouped row r (clamped into range; rows past the group
 // end only feed accumulator rows that are never stored).
 __device__ __forceinline__ int gather_token(const Params& p, int r)
@@ -267,36 +283,46 @@ __device__ __forceinline__ void epilogue_tile(const Params& p, const CUtensorMap
             tmem_ld_wait();
         }
     } else {
-        // this warp: columns [cbeg, cbeg + 256 / kColGroups) of the tile, in slabs of 16
+        // this warp: columns [cbeg, cbeg + 256 / kColGroups) of the tile, in
+        // slabs of 32 (two 16-column TMEM loads, the next slab in flight)
         constexpr int kIters = kBN / kColGroups / kSlabCols;
         const int cbeg = hf * (kBN / kColGroups);
         const float wgt = valid ? __ldg(p.w_perm + row) : 0.0f;
         const int wrow0 = row0 + q * 32;                   // first row of this warp's slab
         const bool whole = wrow0 + 31 < row_end;           // all 32 rows belong to the group
-        float* orow = static_cast<float*>(p.out) + (int64_t)row * p.n_out + nt * kBN;
+        __half* orow = static_cast<__half*>(p.out) + (int64_t)row * p.n_out + nt * kBN;
         const int ncols = min(kBN, p.n_out - nt * kBN);
-        uint32_t a[2][16];
-        tmem_ld16(tbase + cbeg, a[0]);
+        bool bad = false;
+        uint32_t lo[2][16], hi[2][16];  // columns 0..15 and 16..31 of a slab
+        tmem_ld16(tbase + cbeg, lo[0]);
+        tmem_ld16(tbase + cbeg + 16, hi[0]);
         tmem_ld_wait();
 #pragma unroll
         for (int it = 0; it < kIters; ++it) {
             const int c0 = cbeg + kSlabCols * it;
-            if (it + 1 < kIters) tmem_ld16(tbase + c0 + kSlabCols, a[(it + 1) & 1]);
-            const uint32_t* av = a[it & 1];
-            if (c0 < ncols) {  // warp-uniform
+            if (it + 1 < kIters) {
+                tmem_ld16(tbase + c0 + kSlabCols, lo[(it + 1) & 1]);
+                tmem_ld16(tbase + c0 + kSlabCols + 16, hi[(it + 1) & 1]);
+            }
+            const uint32_t* al = lo[it & 1];
+            const uint32_t* ah = hi[it & 1];
+            if (c0 < ncols) {  // warp-uniform (n_out % 64 == 0)
+                uint32_t pk[16];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    pk[i] = scaled_f16x2(wgt, al[2 * i], al[2 * i + 1], bad);
+                    pk[8 + i] = scaled_f16x2(wgt, ah[2 * i], ah[2 * i + 1], bad);
+                }
                 if (whole) {
-                    float* buf = slab + slab_buf * (kSlabBytes / 4);
+                    uint32_t* buf = reinterpret_cast<uint32_t*>(slab) + slab_buf * (kSlabBytes / 4);
                     if (lane == 0) bulk_wait_group_read<1>();  // the store that last read `buf` is done
                     __syncwarp();
                     // row `lane` of the slab: 4 x 16 B chunks, 64-byte swizzle
-                    float4* rowp = reinterpret_cast<float4*>(buf + lane * kSlabCols);
+                    uint4* rowp = reinterpret_cast<uint4*>(buf + lane * (kSlabCols / 2));
                     const int sw = (lane >> 1) & 3;
 #pragma unroll
                     for (int v = 0; v < 4; ++v)
-                        rowp[v ^ sw] = make_float4(wgt * __uint_as_float(av[4 * v]),
-                                                   wgt * __uint_as_float(av[4 * v + 1]),
-                                                   wgt * __uint_as_float(av[4 * v + 2]),
-                                                   wgt * __uint_as_float(av[4 * v + 3]));
+                        rowp[v ^ sw] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
                     fence_proxy_async_smem();
                     __syncwarp();
                     if (lane == 0) {
@@ -305,16 +331,14 @@ __device__ __forceinline__ void epilogue_tile(const Params& p, const CUtensorMap
                     }
                     slab_buf ^= 1;
                 } else if (valid) {
-                    float4* dst = reinterpret_cast<float4*>(orow + c0);
+                    uint4* dst = reinterpret_cast<uint4*>(orow + c0);
 #pragma unroll
-                    for (int v = 0; v < 4; ++v)
-                        dst[v] = make_float4(wgt * __uint_as_float(av[4 * v]), wgt * __uint_as_float(av[4 * v + 1]),
-                                             wgt * __uint_as_float(av[4 * v + 2]),
-                                             wgt * __uint_as_float(av[4 * v + 3]));
+                    for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
                 }
             }
             tmem_ld_wait();
         }
+        if (__any_sync(0xffffffffu, bad && valid) && lane == 0) record_status(kStatusDeviceRange);
     }
 }
 

@@ -226,7 +226,7 @@ Layout plan(int64_t T, int64_t d, int64_t E, int64_t k, int64_t f)
     L.w_perm = o;  o += align256(M * 4);
     L.x_perm = o;  o += align256(M * (size_t)d * 2);
     L.h = o;       o += align256(M * (size_t)f * 2);
-    L.y = o;       o += align256(M * (size_t)d * 4);
+    L.y = o;       o += align256(M * (size_t)d * 2);
     L.total = o;
     return L;
 }
@@ -316,7 +316,7 @@ int run_permute(const moe_bf16* x, const int32_t* ids, const float* wts, int64_t
 int run_ffn(const DeviceState& st, const moe_bf16* x_perm, const moe_bf16* x_gather, const int32_t* perm,
             int64_t T, int64_t k, const float* w_perm, const int32_t* offsets, const moe_bf16* w_gate,
             const moe_bf16* w_up, const moe_bf16* w_down, int64_t M, int64_t d, int64_t E, int64_t f, moe_bf16* h,
-            float* y, cudaStream_t s, cudaEvent_t mid_event)
+            moe_f16* y, cudaStream_t s, cudaEvent_t mid_event)
 {
     if (M == 0) {
         if (mid_event && cudaEventRecord(mid_event, s) != cudaSuccess) return MOE_ERR_CUDA;
@@ -333,7 +333,7 @@ int run_ffn(const DeviceState& st, const moe_bf16* x_perm, const moe_bf16* x_gat
     rc = rc ? rc : make_map(&tu, w_up, (uint64_t)f, (uint64_t)(E * d), 64, 64);
     rc = rc ? rc : make_map(&ta2, h, (uint64_t)f, (uint64_t)M, 64, kBM);
     rc = rc ? rc : make_map(&td, w_down, (uint64_t)d, (uint64_t)(E * f), 64, 64);
-    rc = rc ? rc : make_map(&ty, y, (uint64_t)d, (uint64_t)M, kSlabCols, 32, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4,
+    rc = rc ? rc : make_map(&ty, y, (uint64_t)d, (uint64_t)M, kSlabCols, 32, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
                             CU_TENSOR_MAP_SWIZZLE_64B);
     if (rc) return rc;
     const size_t smem1 = smem_bytes<kSwiGLU>();
@@ -388,12 +388,12 @@ int run_ffn(const DeviceState& st, const moe_bf16* x_perm, const moe_bf16* x_gat
     return launch_status();
 }
 
-int run_combine(const float* y, const int32_t* inv, int64_t T, int64_t d, int64_t k, float* out, cudaStream_t s)
+int run_combine(const moe_f16* y, const int32_t* inv, int64_t T, int64_t d, int64_t k, float* out, cudaStream_t s)
 {
     if (T == 0) return MOE_OK;
-    const int nvec = (int)(d / 4);
+    const int nvec = (int)(d / 8);
     const int threads = nvec < 256 ? ((nvec + 31) / 32) * 32 : 256;
-    moe::combine::combine_kernel<<<(unsigned)T, threads, 0, s>>>(reinterpret_cast<const float4*>(y), inv, T * k,
+    moe::combine::combine_kernel<<<(unsigned)T, threads, 0, s>>>(reinterpret_cast<const uint4*>(y), inv, T * k,
                                                                  nvec, (int)k, reinterpret_cast<float4*>(out));
     return launch_status();
 }
@@ -436,7 +436,7 @@ int forward_impl(const moe_bf16* x, const moe_bf16* w_router, const float* bias,
     float* w_perm = reinterpret_cast<float*>(w + L.w_perm);
     moe_bf16* x_perm = reinterpret_cast<moe_bf16*>(w + L.x_perm);
     moe_bf16* h = reinterpret_cast<moe_bf16*>(w + L.h);
-    float* y = reinterpret_cast<float*>(w + L.y);
+    moe_f16* y = reinterpret_cast<moe_f16*>(w + L.y);
     const bool gather = (flags & MOE_FLAG_FUSED_GATHER) != 0;
 
     if ((rc = run_route(x, w_router, bias, T, d, E, k, ids, wts, chunk, s))) return rc;
@@ -502,11 +502,13 @@ const char* moe_strerror(int status)
         case MOE_ERR_UNSUPPORTED_DEVICE: return "MOE_ERR_UNSUPPORTED_DEVICE: needs a compute capability 10.0 GPU";
         case MOE_ERR_STATIC_SCRATCH_TOO_SMALL:
             return "MOE_ERR_STATIC_SCRATCH_TOO_SMALL: moe_permute_static needs E * ceil(T / 64) <= 262144";
+        case MOE_ERR_DEVICE_RANGE:
+            return "MOE_ERR_DEVICE_RANGE: a y value outside the fp16 range (|y| >= 65520) or NaN on the device";
         default: return "unknown moe status";
     }
 }
 
-int moe_version(void) { return 100; }
+int moe_version(void) { return 200; }
 
 size_t moe_workspace_size(int64_t T, int64_t d, int64_t E, int64_t k, int64_t f)
 {
@@ -589,7 +591,7 @@ int moe_permute_static(const moe_bf16* x, const int32_t* topk_ids, const float* 
 
 int moe_expert_ffn(const moe_bf16* x_perm, const float* w_perm, const int32_t* offsets, const moe_bf16* w_gate,
                    const moe_bf16* w_up, const moe_bf16* w_down, int64_t M, int64_t d, int64_t E, int64_t f,
-                   moe_bf16* h, float* y, cudaStream_t stream)
+                   moe_bf16* h, moe_f16* y, cudaStream_t stream)
 {
     if (M < 0 || d <= 0 || E <= 0) return MOE_ERR_INVALID_ARG;
     int rc = check_common(M, d, E, 1);
@@ -606,7 +608,7 @@ int moe_expert_ffn(const moe_bf16* x_perm, const float* w_perm, const int32_t* o
                    stream, nullptr);
 }
 
-int moe_combine(const float* y, const int32_t* inv, int64_t T, int64_t d, int64_t k, float* out,
+int moe_combine(const moe_f16* y, const int32_t* inv, int64_t T, int64_t d, int64_t k, float* out,
                 cudaStream_t stream)
 {
     if (T < 0 || d <= 0 || k <= 0) return MOE_ERR_INVALID_ARG;
