@@ -348,7 +348,7 @@ def run_gpu(args, cfg):
             "tflops": alg["flops"] / (ms * 1e-3) / 1e12,
             "grouped_gemm_tflops": (alg["gateup_flops"] + alg["down_flops"]) /
                                    ((stage_ms["gateup_gemm"] + stage_ms["down_gemm"]) * 1e-3) / 1e12,
-            "roofline": {"bound": "tensor", "kernel": "grouped_gemm_kernel<SwiGLU> (gate/up + SwiGLU)",
+            "roofline": {"bound": "tensor", "kernel": "grouped_gemm_pair_kernel<SwiGLU> (gate/up + SwiGLU)",
                          "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                          "frac": achieved / peaks["bf16_tflops"], "traffic": traffic,
                          "peak_source": f"{peaks['source']} burst bf16"},

@@ -41,7 +41,7 @@ def _hash(flags) -> str:
     return h.hexdigest()
 
 
-def kernel_hash(files=("grouped_gemm.cuh", "ptx.cuh")) -> str:
+def kernel_hash(files=("grouped_gemm.cuh", "grouped_gemm_pair.cuh", "ptx.cuh", "status.cuh")) -> str:
     """Hash of the grouped-GEMM kernel sources and the build flags: ties a
     profiler measurement to the kernel version it was taken on."""
     h = hashlib.sha256()
