@@ -116,7 +116,6 @@ int setup_device(DeviceState** out)
             e = e ? e : cudaFuncSetAttribute(moe::route::route_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
             e = e ? e : cudaFuncSetAttribute(moe::route::route_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
             e = e ? e : cudaFuncSetAttribute(moe::route::route_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
-            e = e ? e : cudaFuncSetAttribute(moe::route::route_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
             e = e ? e : cudaFuncSetAttribute(moe::route::route_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
             e = e ? e : cudaFuncSetAttribute(moe::gemm::grouped_gemm_kernel<moe::gemm::kSwiGLU, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
             e = e ? e : cudaFuncSetAttribute(moe::gemm::grouped_gemm_kernel<moe::gemm::kSwiGLU, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
@@ -241,14 +240,26 @@ int launch_route(const CUtensorMap& tx, const CUtensorMap& tw, moe::route::Param
     using moe::route::smem_bytes;
     // one CTA per SM: the deepest ring that fits (2 to 8 stages)
     p.stages = moe::route::kMaxStages;
-    while (p.stages > 2 && smem_bytes<KMAX>(p.n_chunks, p.stages, p.E) > (size_t)kMaxDynSmem) --p.stages;
-    const size_t smem = smem_bytes<KMAX>(p.n_chunks, p.stages, p.E);
-    moe::route::route_kernel<KMAX><<<tiles, moe::route::Shape<KMAX>::threads, smem, s>>>(tx, tw, p);
-    return launch_status();
+    while (p.stages > 2 && smem_bytes(p.n_chunks, p.stages, p.E, p.split, p.passes) > (size_t)kMaxDynSmem)
+        --p.stages;
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)p.split;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(tiles * (unsigned)p.split);
+    cfg.blockDim = dim3(moe::route::kThreads);
+    cfg.dynamicSmemBytes = smem_bytes(p.n_chunks, p.stages, p.E, p.split, p.passes);
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = p.split > 1 ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, moe::route::route_kernel<KMAX>, tx, tw, p) == cudaSuccess ? MOE_OK
+                                                                                              : MOE_ERR_CUDA;
 }
 
-int run_route(const moe_bf16* x, const moe_bf16* w_router, const float* bias, int64_t T, int64_t d, int64_t E,
-              int64_t k, int32_t* ids, float* wts, int32_t* chunk_counts, cudaStream_t s)
+int run_route(const DeviceState& st, const moe_bf16* x, const moe_bf16* w_router, const float* bias, int64_t T,
+              int64_t d, int64_t E, int64_t k, int32_t* ids, float* wts, int32_t* chunk_counts, cudaStream_t s)
 {
     if (T == 0) return MOE_OK;
     CUtensorMap tx, tw;
@@ -256,8 +267,7 @@ int run_route(const moe_bf16* x, const moe_bf16* w_router, const float* bias, in
     if (rc) return rc;
     rc = make_map(&tw, w_router, (uint64_t)E, (uint64_t)d, 64, 64);
     if (rc) return rc;
-    int kmax = 1;
-    while (kmax < k) kmax <<= 1;
+    const int64_t tiles = (T + moe::route::kBM - 1) / moe::route::kBM;
     moe::route::Params p;
     p.bias = bias;
     p.ids = ids;
@@ -269,19 +279,24 @@ int run_route(const moe_bf16* x, const moe_bf16* w_router, const float* bias, in
     p.E = (int)E;
     p.k = (int)k;
     p.n_chunks = (int)((E + 63) / 64);
-    p.stages = 0;  // set per list length
+    p.stages = 0;  // set by the launcher
     uint32_t cols = 64;
     while (cols < (uint32_t)(64 * p.n_chunks)) cols <<= 1;
     p.tmem_cols = cols;
-    const unsigned tiles = (unsigned)((T + moe::route::kBM - 1) / moe::route::kBM);
-    switch (kmax) {
-        case 1: return launch_route<1>(tx, tw, p, tiles, s);
-        case 2: return launch_route<2>(tx, tw, p, tiles, s);
-        case 4: return launch_route<4>(tx, tw, p, tiles, s);
-        case 8: return launch_route<8>(tx, tw, p, tiles, s);
-        case 16: return launch_route<16>(tx, tw, p, tiles, s);
-        default: return launch_route<32>(tx, tw, p, tiles, s);
-    }
+    // Split K over a CTA pair while the pairs of all tiles can be resident
+    // at once: more SMs stream x.  The exchange buffer of a pair holds
+    // 128 x E fp32 partials, which fits the ring for E <= 256.
+    const int64_t pairs = st.max_pairs > 0 ? st.max_pairs : st.sm_count / 2;
+    p.split = (E <= 256 && d >= 2 * moe::route::kBK && tiles <= pairs) ? 2 : 1;
+    p.passes = (p.split == 1 && E > 256) ? 2 : 1;
+    // top-k list length: the power of two >= k for lane groups (k <= 8), or
+    // the whole-warp rounds (k > 8)
+    const unsigned ut = (unsigned)tiles;
+    if (k <= 1) return launch_route<1>(tx, tw, p, ut, s);
+    if (k <= 2) return launch_route<2>(tx, tw, p, ut, s);
+    if (k <= 4) return launch_route<4>(tx, tw, p, ut, s);
+    if (k <= 8) return launch_route<8>(tx, tw, p, ut, s);
+    return launch_route<32>(tx, tw, p, ut, s);
 }
 
 // Grouping by expert.  have_hist: chunk_em already holds the per-chunk
@@ -439,7 +454,7 @@ int forward_impl(const moe_bf16* x, const moe_bf16* w_router, const float* bias,
     moe_f16* y = reinterpret_cast<moe_f16*>(w + L.y);
     const bool gather = (flags & MOE_FLAG_FUSED_GATHER) != 0;
 
-    if ((rc = run_route(x, w_router, bias, T, d, E, k, ids, wts, chunk, s))) return rc;
+    if ((rc = run_route(*st, x, w_router, bias, T, d, E, k, ids, wts, chunk, s))) return rc;
     if ((rc = rec(1))) return rc;
     if ((rc = run_permute(x, ids, wts, T, d, E, k, counts, offsets, perm, inv, gather ? nullptr : x_perm, w_perm,
                           chunk, true, s)))
@@ -541,7 +556,7 @@ int moe_route(const moe_bf16* x, const moe_bf16* w_router, const float* bias, in
     if (workspace_bytes < route_ws_bytes(T, d, E)) return MOE_ERR_WORKSPACE_TOO_SMALL;
     DeviceState* st = nullptr;
     if ((rc = setup_device(&st))) return rc;
-    return run_route(x, w_router, bias, T, d, E, k, topk_ids, topk_w, nullptr, stream);
+    return run_route(*st, x, w_router, bias, T, d, E, k, topk_ids, topk_w, nullptr, stream);
 }
 
 int moe_permute(const moe_bf16* x, const int32_t* topk_ids, const float* topk_w, int64_t T, int64_t d, int64_t E,

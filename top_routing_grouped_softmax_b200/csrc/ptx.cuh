@@ -284,6 +284,12 @@ __device__ __forceinline__ uint32_t mapa_shared(const void* p, uint32_t rank)
     return r;
 }
 
+// Store to shared memory of any CTA of the cluster (address from mapa_shared).
+__device__ __forceinline__ void st_cluster_f32(uint32_t cluster_addr, float v)
+{
+    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(cluster_addr), "f"(v) : "memory");
+}
+
 // Arrive on an mbarrier that may live in another CTA of the cluster.
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr)
 {

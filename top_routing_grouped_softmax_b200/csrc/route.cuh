@@ -5,24 +5,38 @@
 // experts, topk; the routing weights are the top-k probabilities, not
 // renormalised).
 //
-// One CTA owns 128 tokens and the whole hidden dimension.  TMA streams
-// x[128 tokens, 64 k] (K-major) and W_router[64 k, E] (E contiguous,
-// MN-major) through a shared-memory ring; one thread issues tcgen05.mma into
-// a 128 x E fp32 accumulator in TMEM (token m -> TMEM lane m, expert e ->
-// column e).  The logits never leave the SM and are never rounded below fp32.
+// A tile is 128 tokens.  TMA streams x[128 tokens, 64 k] (K-major) and
+// W_router[64 k, E] (E contiguous, MN-major) through a shared-memory ring;
+// one thread issues tcgen05.mma into a 128 x E fp32 accumulator in TMEM
+// (token m -> TMEM lane m, expert e -> column e).  The logits are never
+// rounded below fp32.
 //
-// Epilogue, 4 * NG warps.  Warp w may only read TMEM lane quarter w % 4 (32
-// tokens), so it takes column group w / 4: NG threads share each token, one
-// NG-th of the experts each.  Each thread adds the bias, keeps its maximum
-// and a sorted top-KMAX list of (logit, expert) in registers (ranking
-// compares fp32 logits -- softmax is monotone -- and equal logits rank the
-// lower expert index first), then sums exp(l - max) over its columns.  The
-// NG partial results meet in shared memory; one thread per token combines
-// them: overall maximum, the partial sums rescaled by exp(m_g - max) in group
-// order, and an NG-way merge of the sorted lists for the k winners.  The
-// winners' probabilities exp(l - max) / sum are the routing weights.  The same thread counts its winners into the CTA's two
-// 64-token chunk histograms, which the permutation needs and which the CTA
-// writes out whole (expert-major table, no global atomics, no zeroing).
+// Split K over a CTA pair.  When the batch has few tiles (fewer than half the
+// SMs), a cluster of two CTAs shares a tile: CTA r accumulates k-blocks
+// [r*nkb/2, (r+1)*nkb/2), and CTA r owns token rows [64r, 64r+64) of the
+// tile.  After both mainloops, each CTA copies its partial logits from TMEM
+// into the owner's shared memory (distributed shared memory stores), one
+// buffer slot per sender; the owner adds the slots in rank order, so the
+// result does not depend on timing.  With one CTA per tile the same code
+// runs with a single slot (and, for E > 256, in two passes of 64 rows so
+// the buffer fits).
+//
+// Softmax and top-k.  For k <= 8, a group of L lanes of one warp takes a
+// token (L = 8 when a CTA owns 128 rows, 16 when it owns 64, so all 32 warps
+// are busy).  Lane j of the group visits experts j, j + L, j + 2L, ... in
+// ascending order, keeps the maximum and a sorted top-KMAX list of
+// (logit, expert) in registers, and later sums exp(l - max) over the same
+// experts; the group's maximum and sum are butterfly reductions in a fixed
+// order, and log2(L) butterfly rounds of a bitonic merge give every lane of
+// the group the token's sorted top-KMAX.  For k > 8, a whole warp takes a
+// token and picks the winners in k rounds of a butterfly arg-max.  Both
+// rank by the (value, index) order -- larger logit first, equal logits rank
+// the lower expert index first -- on fp32 logits (softmax is monotone).
+// Lane j < k of the token's group writes slot j: the expert and its
+// probability exp(l - max) / sum.  The same lanes count their experts into
+// the tile's 64-token chunk histograms, which the permutation needs and
+// which the CTA writes out whole (expert-major table, no global atomics, no
+// zeroing).
 #pragma once
 
 #include <cuda_bf16.h>
@@ -32,12 +46,14 @@
 namespace moe {
 namespace route {
 
-constexpr int kBM = 128;                    // tokens per CTA = TMEM lanes
+constexpr int kBM = 128;                    // tokens per tile = TMEM lanes
 constexpr int kBK = 64;                     // K per pipeline stage (128 B of bf16)
+constexpr int kThreads = 1024;              // 32 warps
+constexpr int kWarps = kThreads / 32;
 constexpr int kABytes = kBM * kBK * 2;      // 16 KB token tile
 constexpr int kChunkBytes = 64 * kBK * 2;   // 8 KB: 64 experts x 64 k
 constexpr int kTokensPerChunk = 64;         // permutation chunk (tokens)
-constexpr int kChunksPerTile = kBM / kTokensPerChunk;
+constexpr int kColGroups = kWarps / 4;      // warps sharing a TMEM lane quarter
 constexpr int kMaxStages = 8;
 
 struct Params {
@@ -50,108 +66,266 @@ struct Params {
     int n_chunks;            // ceil(E / 64): 64-expert column chunks of W_router
     int stages;              // pipeline depth
     uint32_t tmem_cols;      // power of two >= 64 * n_chunks
+    int split;               // CTAs per tile: 1, or 2 (cluster of two, split K)
+    int passes;              // row passes of the exchange buffer (1, or 2 when split == 1 and E > 256)
 };
 
 __host__ __device__ inline int stage_bytes(int n_chunks) { return kABytes + n_chunks * kChunkBytes; }
 
-// Column groups (threads per token) for a top-KMAX list: eight keep 32
-// warps busy while the short lists fit 64 registers; longer lists need the
-// registers of a 16-warp CTA.
-template <int KMAX>
-struct Shape {
-    static constexpr int groups = KMAX <= 8 ? 8 : 4;
-    static constexpr int threads = 128 * groups;
-};
-
-// Columns per group: a multiple of 16 (the TMEM load width) such that the
-// groups cover all E columns.  Groups past E are empty; a 16-column load
-// that starts below E (a multiple of 8) ends at or below 64 * n_chunks.
-__host__ __device__ inline int group_cols(int E, int groups)
+// Token rows one CTA owns in one pass, and the exchange buffer
+// [split slots][E][pitch] fp32 with pitch = own + 32 / L (own is a multiple
+// of 32, so pitch = 32 / L mod 32 banks).  A warp writing 32 rows of one
+// column hits 32 consecutive words; a warp reading, for 32 / L tokens, the
+// columns j + L m of its L lanes hits bank (32 / L) * j + token: distinct.
+__host__ __device__ inline int own_rows(int split, int passes) { return kBM / (split * passes); }
+__host__ __device__ inline int group_lanes(int own) { return kThreads / own; }  // 8 or 16
+__host__ __device__ inline int buffer_pitch(int own) { return own + 32 / group_lanes(own); }
+__host__ __device__ inline size_t buffer_bytes(int E, int split, int passes)
 {
-    return ((E + groups * 16 - 1) / (groups * 16)) * 16;
+    return (size_t)split * E * buffer_pitch(own_rows(split, passes)) * 4;
 }
 
-// Epilogue scratch (reuses the stage ring once every MMA has completed):
-// the groups' lists [group][j][token] (values, then indices), their maxima
-// and sums [group][token], and the winners [token][j] (ids, then weights).
-__host__ __device__ inline size_t epi_bytes(int kmax, int groups)
-{
-    return (size_t)4 * kBM * (2 * groups * kmax + 2 * groups + 2 * kmax);
-}
-
-__host__ __device__ inline size_t region_bytes(int n_chunks, int stages, int kmax, int groups)
+__host__ __device__ inline size_t region_bytes(int n_chunks, int stages, int E, int split, int passes)
 {
     const size_t ring = (size_t)stages * stage_bytes(n_chunks);
-    const size_t epi = epi_bytes(kmax, groups);
-    return ring > epi ? ring : epi;
+    const size_t buf = buffer_bytes(E, split, passes);
+    return ring > buf ? ring : buf;
 }
 
-// Dynamic shared memory: 1 KB alignment slack, ring/scratch region,
+// Dynamic shared memory: 1 KB alignment slack, ring / exchange region,
 // barriers, TMEM slot, abort flag, bias [E], chunk histograms [2][E].
-template <int KMAX>
-__host__ inline size_t smem_bytes(int n_chunks, int stages, int E)
+__host__ inline size_t smem_bytes(int n_chunks, int stages, int E, int split, int passes)
 {
-    return 1024 + region_bytes(n_chunks, stages, KMAX, Shape<KMAX>::groups) + (size_t)(2 * stages + 1) * 8 + 16 +
+    return 1024 + region_bytes(n_chunks, stages, E, split, passes) + (size_t)(2 * stages + 1) * 8 + 16 +
            (size_t)3 * E * 4;
 }
+
+// Columns per warp column group: a multiple of 16 (the TMEM load width) such
+// that the groups cover all E columns.  Groups past E are empty; a 16-column
+// load that starts below E (a multiple of 8) ends at or below 64 * n_chunks.
+__host__ __device__ inline int group_cols(int E) { return ((E + kColGroups * 16 - 1) / (kColGroups * 16)) * 16; }
 
 // (value, index) order of the top-k: larger logit first; equal logits rank
 // the lower expert index first.
 __device__ __forceinline__ bool ranks_before(float v, int i, float w, int j) { return v > w || (v == w && i < j); }
 
-// Insert (x, col) into a list sorted by ranks_before, dropping its last
-// entry.  The caller visits its columns in ascending index order, so every
-// entry already in the list has a lower index than col and x ranks before
-// entry j exactly when x > v[j].  All KMAX comparisons are independent and
-// every slot takes its new value by selection (no branches, no dependent
-// chain): slot j keeps its entry, takes x, or takes the old entry j-1.
+// Softmax and top-k of one token by a whole warp (k > 8).  `col(j)` is the
+// logit of expert lane + 32 j (called only for lane + 32 j < E).  Lane
+// j < k receives slot j.
+template <int VPL, typename Logit>
+__device__ __forceinline__ void warp_topk(int E, int k, int lane, Logit col, int& my_id, float& my_w)
+{
+    float v[VPL];
+    unsigned taken = 0;  // bit j: value j is not a candidate
+#pragma unroll
+    for (int j = 0; j < VPL; ++j) {
+        const int c = lane + 32 * j;
+        if (c < E) {
+            v[j] = col(j);
+        } else {
+            v[j] = -INFINITY;
+            taken |= 1u << j;
+        }
+    }
+    float mx = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < VPL; ++j) mx = fmaxf(mx, v[j]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    float sum = 0.0f;
+#pragma unroll
+    for (int j = 0; j < VPL; ++j)
+        if (!((taken >> j) & 1u)) sum += expf(v[j] - mx);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    my_id = 0;
+    my_w = 0.0f;
+    for (int slot = 0; slot < k; ++slot) {
+        float bv = -INFINITY;
+        int bi = 0x7fffffff;
+#pragma unroll
+        for (int j = 0; j < VPL; ++j) {
+            const int c = lane + 32 * j;
+            if (!((taken >> j) & 1u) && ranks_before(v[j], c, bv, bi)) {
+                bv = v[j];
+                bi = c;
+            }
+        }
+        // a strict total order: both partners of every exchange keep the
+        // same winner, so all lanes end with the token's best
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+            const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+            if (ranks_before(ov, oi, bv, bi)) {
+                bv = ov;
+                bi = oi;
+            }
+        }
+        if ((bi & 31) == lane) taken |= 1u << ((bi >> 5) & 31);
+        if (lane == slot) {
+            my_id = bi;
+            my_w = expf(bv - mx) / sum;
+        }
+    }
+}
+
+// Insert (x, col) into a list sorted by the (value, index) order, dropping
+// its last entry.  The caller visits its experts in ascending index order,
+// so every entry already in the list has a lower index than col and x
+// ranks before entry m exactly when x > v[m].  The comparisons are
+// independent and every slot takes its new value by selection: it keeps
+// its entry, takes x, or takes the old entry m-1.
 template <int KMAX>
-__device__ __forceinline__ void topk_insert_ascending(float (&v)[KMAX], int (&ix)[KMAX], float x, int col)
+__device__ __forceinline__ void insert_ascending(float (&v)[KMAX], int (&ix)[KMAX], float x, int col)
 {
     bool gt[KMAX];
 #pragma unroll
-    for (int j = 0; j < KMAX; ++j) gt[j] = x > v[j];
+    for (int m = 0; m < KMAX; ++m) gt[m] = x > v[m];
 #pragma unroll
-    for (int j = KMAX - 1; j > 0; --j) {
-        v[j] = gt[j - 1] ? v[j - 1] : (gt[j] ? x : v[j]);
-        ix[j] = gt[j - 1] ? ix[j - 1] : (gt[j] ? col : ix[j]);
+    for (int m = KMAX - 1; m > 0; --m) {
+        v[m] = gt[m - 1] ? v[m - 1] : (gt[m] ? x : v[m]);
+        ix[m] = gt[m - 1] ? ix[m - 1] : (gt[m] ? col : ix[m]);
     }
     v[0] = gt[0] ? x : v[0];
     ix[0] = gt[0] ? col : ix[0];
 }
 
+// Merge the sorted list of lane (lane ^ o) into this lane's, keeping the
+// KMAX best: the better of v[m] and the partner's [KMAX-1-m] leaves the KMAX
+// best of both lists as a bitonic sequence, which half-cleaners sort.  Both
+// partners end with the same list (the order is total; only identical
+// (-inf, sentinel) entries can compare equal).
 template <int KMAX>
-__global__ void __launch_bounds__(Shape<KMAX>::threads, 1)
+__device__ __forceinline__ void merge_partner(float (&v)[KMAX], int (&ix)[KMAX], int o)
+{
+    float ov[KMAX];
+    int oi[KMAX];
+#pragma unroll
+    for (int m = 0; m < KMAX; ++m) {
+        ov[m] = __shfl_xor_sync(0xffffffffu, v[m], o);
+        oi[m] = __shfl_xor_sync(0xffffffffu, ix[m], o);
+    }
+#pragma unroll
+    for (int m = 0; m < KMAX; ++m) {
+        const float bv = ov[KMAX - 1 - m];
+        const int bi = oi[KMAX - 1 - m];
+        if (ranks_before(bv, bi, v[m], ix[m])) {
+            v[m] = bv;
+            ix[m] = bi;
+        }
+    }
+#pragma unroll
+    for (int stride = KMAX / 2; stride > 0; stride >>= 1) {
+#pragma unroll
+        for (int m = 0; m < KMAX; ++m) {
+            if ((m & stride) == 0 && ranks_before(v[m + stride], ix[m + stride], v[m], ix[m])) {
+                const float tv = v[m];
+                const int ti = ix[m];
+                v[m] = v[m + stride];
+                ix[m] = ix[m + stride];
+                v[m + stride] = tv;
+                ix[m + stride] = ti;
+            }
+        }
+    }
+}
+
+// Softmax and top-k of one token by a group of L lanes (lane j of the group
+// = lane % L); `logit(c)` is expert c's logit.  Lane j < k receives slot j.
+template <int L, int KMAX, typename Logit>
+__device__ __forceinline__ void group_topk(int E, int j, Logit logit, int& my_id, float& my_w)
+{
+    float v[KMAX];
+    int ix[KMAX];
+#pragma unroll
+    for (int m = 0; m < KMAX; ++m) {
+        v[m] = -INFINITY;
+        ix[m] = 0x7fffffff;
+    }
+    float mx = -INFINITY;
+    for (int c = j; c < E; c += L) {
+        const float l = logit(c);
+        mx = fmaxf(mx, l);
+        insert_ascending<KMAX>(v, ix, l, c);
+    }
+#pragma unroll
+    for (int o = L / 2; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    float sum = 0.0f;
+    for (int c = j; c < E; c += L) sum += __expf(logit(c) - mx);
+#pragma unroll
+    for (int o = L / 2; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+#pragma unroll
+    for (int o = 1; o < L; o <<= 1) merge_partner<KMAX>(v, ix, o);
+    my_id = ix[0];
+    float w = v[0];
+#pragma unroll
+    for (int m = 1; m < KMAX; ++m)
+        if (m == j) {
+            my_id = ix[m];
+            w = v[m];
+        }
+    my_w = __expf(w - mx) / sum;
+}
+
+// One pass of softmax + top-k over the `own` buffered rows, L lanes per
+// token (32 / L tokens per warp).
+template <int L, int KMAX>
+__device__ __forceinline__ void topk_rows(const Params& p, const float* buf, const float* s_bias, int* s_hist,
+                                          int S, int own, int pitch, int tile0, int row0, bool ok, int warp,
+                                          int lane)
+{
+    const int E = p.E;
+    const int j = lane % L;
+    for (int i = warp * (32 / L) + lane / L; i - lane / L < own; i += kWarps * (32 / L)) {
+        // i < own for every group of the warp: own is a multiple of 32 / L
+        const int64_t t = (int64_t)tile0 + row0 + i;
+        int my_id;
+        float my_w;
+        group_topk<L, KMAX>(E, j, [&](int c) {
+            const float* col = buf + (size_t)c * pitch + i;
+            float l = col[0];
+            for (int s = 1; s < S; ++s) l += col[(size_t)s * E * pitch];
+            return l + s_bias[c];
+        }, my_id, my_w);
+        if (ok && t < p.T && j < p.k) {
+            p.ids[t * p.k + j] = my_id;
+            p.wts[t * p.k + j] = my_w;
+            if (p.chunk_counts && (unsigned)my_id < (unsigned)E)
+                atomicAdd(&s_hist[((row0 + i) / kTokensPerChunk) * E + my_id], 1);
+        }
+    }
+}
+
+template <int KMAX>
+__global__ void __launch_bounds__(kThreads, 1)
     route_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w, Params p)
 {
-    constexpr int kGroups = Shape<KMAX>::groups;
-    constexpr int kThreads = Shape<KMAX>::threads;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int S = p.split;
     const int sbytes = stage_bytes(p.n_chunks);
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + region_bytes(p.n_chunks, p.stages, KMAX, kGroups));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + region_bytes(p.n_chunks, p.stages, p.E, S, p.passes));
     uint64_t* empty = full + p.stages;
     uint64_t* done = empty + p.stages;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     float* s_bias = reinterpret_cast<float*>(tmem_slot + 4);
     int* s_hist = reinterpret_cast<int*>(s_bias + p.E);  // [2][E]
-    // epilogue scratch, valid once every MMA has completed
-    float* s_lval = reinterpret_cast<float*>(smem);                       // [groups][KMAX][128]
-    int* s_lidx = reinterpret_cast<int*>(s_lval + kGroups * KMAX * kBM);  // [groups][KMAX][128]
-    float* s_gmax = reinterpret_cast<float*>(s_lidx + kGroups * KMAX * kBM);  // [groups][128]
-    float* s_gsum = s_gmax + kGroups * kBM;                                   // [groups][128]
-    int* s_oid = reinterpret_cast<int*>(s_gsum + kGroups * kBM);              // [128][KMAX]
-    float* s_ow = reinterpret_cast<float*>(s_oid + kBM * KMAX);               // [128][KMAX]
+    float* buf = reinterpret_cast<float*>(smem);         // exchange buffer, once the ring is idle
 
     const int warp = threadIdx.x / 32;
     const int lane = threadIdx.x % 32;
     const uint64_t limit = g_wait_limit_ns;
-    const int tile0 = blockIdx.x * kBM;
-    const int num_kb = p.d / kBK;
+    const uint32_t r = S > 1 ? cluster_ctarank() : 0u;
+    const int tile0 = (int)(blockIdx.x / S) * kBM;
+    const int nkb = p.d / kBK;
+    const int kb0 = (int)((int64_t)nkb * r / S);
+    const int kb1 = (int)((int64_t)nkb * (r + 1) / S);
+    const int E = p.E;
 
-    for (int e = threadIdx.x; e < p.E; e += kThreads) s_bias[e] = p.bias ? p.bias[e] : 0.0f;
-    for (int e = threadIdx.x; e < kChunksPerTile * p.E; e += kThreads) s_hist[e] = 0;
+    for (int e = threadIdx.x; e < E; e += kThreads) s_bias[e] = p.bias ? p.bias[e] : 0.0f;
+    for (int e = threadIdx.x; e < 2 * E; e += kThreads) s_hist[e] = 0;
     if (threadIdx.x == 0) {
         for (int s = 0; s < p.stages; ++s) {
             mbar_init(&full[s], 1);
@@ -175,11 +349,12 @@ __global__ void __launch_bounds__(Shape<KMAX>::threads, 1)
 
     if (warp == 0) {
         if (lane == 0) {
-            // TMA producer
+            // TMA producer over this CTA's k-blocks
             int issued = 0;
-            for (int kb = 0; kb < num_kb; ++kb) {
-                const int s = kb % p.stages;
-                const uint32_t ph = (uint32_t)(kb / p.stages) & 1u;
+            for (int kb = kb0; kb < kb1; ++kb) {
+                const int i = kb - kb0;
+                const int s = i % p.stages;
+                const uint32_t ph = (uint32_t)(i / p.stages) & 1u;
                 if (!mbar_wait(&empty[s], ph ^ 1u, limit)) {
                     *abort_flag = 1;
                     break;
@@ -201,9 +376,10 @@ __global__ void __launch_bounds__(Shape<KMAX>::threads, 1)
     } else if (warp == 1) {
         if (lane == 0) {
             // MMA issuer: up to two N <= 256 MMAs per k-step cover all experts.
-            for (int kb = 0; kb < num_kb; ++kb) {
-                const int s = kb % p.stages;
-                const uint32_t ph = (uint32_t)(kb / p.stages) & 1u;
+            for (int kb = kb0; kb < kb1; ++kb) {
+                const int i = kb - kb0;
+                const int s = i % p.stages;
+                const uint32_t ph = (uint32_t)(i / p.stages) & 1u;
                 if (!mbar_wait(&full[s], ph, limit)) {
                     *abort_flag = 1;
                     break;
@@ -219,7 +395,7 @@ __global__ void __launch_bounds__(Shape<KMAX>::threads, 1)
                         const uint64_t bdesc =
                             smem_desc_sw128(b_base + m * 4 * kChunkBytes + kk * 2048, kChunkBytes, 1024);
                         mma_bf16_ss(tmem + m * 256, adesc, bdesc, idesc_bf16_f32(128, 64 * chunks, false, true),
-                                    (kb | kk) != 0);
+                                    (i | kk) != 0);
                     }
                 }
                 mma_commit(&empty[s]);
@@ -230,119 +406,97 @@ __global__ void __launch_bounds__(Shape<KMAX>::threads, 1)
     }
     __syncthreads();
 
-    // ------------------------------------------------------------ epilogue
+    // ---------------------------------------------------------- epilogue
     bool have = true;
     if (lane == 0) have = mbar_wait(done, 0, limit);
     have = __shfl_sync(0xffffffffu, have ? 1 : 0, 0) != 0;
     tc_fence_after_sync();
     // a timed-out wait already recorded the device status; every thread of
-    // the CTA reaches the same decision from the flag and its warp's wait
+    // the CTA reaches the same decision, and every thread of both CTAs of a
+    // pair still takes part in every cluster barrier below
     const bool ok = __syncthreads_and(have && *abort_flag == 0) != 0;
     const int q = warp & 3;          // TMEM lane quarter
     const int g = warp >> 2;         // column group
-    const int row = q * 32 + lane;   // token within the tile
-    if (ok) {
-        const int cg = group_cols(p.E, kGroups);
-        const int c_begin = g * cg;
-        const int c_end = min(p.E, c_begin + cg);
-        const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16);
-        float v[KMAX];
-        int ix[KMAX];
+    const int cg = group_cols(E);
+    const int c_begin = g * cg;
+    const int c_end = min(E, c_begin + cg);
+    const uint32_t trow = tmem + ((uint32_t)(q * 32) << 16);
+    const int own = own_rows(S, p.passes);
+    const int pitch = buffer_pitch(own);
+
+    for (int pass = 0; pass < p.passes; ++pass) {
+        // the ring (and the previous pass's buffer) is idle in every CTA of the tile
+        if (S > 1)
+            cluster_sync();
+        else
+            __syncthreads();
+        // stage this CTA's partial logits for the rows of this pass into the
+        // owner's buffer slot r: buf[r][col][row - owner's first row]
+        const int qrow = q * 32;
+        const int owner = S > 1 ? qrow / own : 0;
+        const int first = S > 1 ? owner * own : pass * own;
+        const bool stage = ok && qrow >= first && qrow < first + own;  // warp-uniform
+        if (stage) {
+            float* dst = buf + (size_t)r * E * pitch + (qrow + lane - first);
+            for (int c0 = c_begin; c0 < c_end; c0 += 16) {  // warp-uniform bounds
+                uint32_t acc[16];
+                tmem_ld16(trow + c0, acc);
+                tmem_ld_wait();
 #pragma unroll
-        for (int j = 0; j < KMAX; ++j) {
-            v[j] = -INFINITY;
-            ix[j] = 0x7fffffff;
-        }
-        float mx = -INFINITY;
-        for (int c0 = c_begin; c0 < c_end; c0 += 16) {  // warp-uniform bounds
-            uint32_t acc[16];
-            tmem_ld16(trow + c0, acc);
-            tmem_ld_wait();
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const int col = c0 + i;
-                if (col < c_end) {
-                    const float l = __uint_as_float(acc[i]) + s_bias[col];
-                    mx = fmaxf(mx, l);
-                    topk_insert_ascending<KMAX>(v, ix, l, col);
-                }
-            }
-        }
-        float sum = 0.0f;
-        for (int c0 = c_begin; c0 < c_end; c0 += 16) {
-            uint32_t acc[16];
-            tmem_ld16(trow + c0, acc);
-            tmem_ld_wait();
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const int col = c0 + i;
-                if (col < c_end) sum += expf(__uint_as_float(acc[i]) + s_bias[col] - mx);
-            }
-        }
-#pragma unroll
-        for (int j = 0; j < KMAX; ++j) {
-            s_lval[(g * KMAX + j) * kBM + row] = v[j];
-            s_lidx[(g * KMAX + j) * kBM + row] = ix[j];
-        }
-        s_gmax[g * kBM + row] = mx;
-        s_gsum[g * kBM + row] = sum;
-    }
-    __syncthreads();
-    const int64_t t = (int64_t)tile0 + row;
-    if (ok && g == 0 && t < p.T) {
-        float mx = s_gmax[row];
-        for (int h = 1; h < kGroups; ++h) mx = fmaxf(mx, s_gmax[h * kBM + row]);
-        float sum = 0.0f;
-        for (int h = 0; h < kGroups; ++h) {
-            const float mh = s_gmax[h * kBM + row];
-            if (mh != -INFINITY) sum += s_gsum[h * kBM + row] * expf(mh - mx);
-        }
-        // kGroups-way merge: each list is sorted and holds its group's
-        // KMAX >= k best, so the k best overall are among the heads
-        int head[kGroups];
-#pragma unroll
-        for (int h = 0; h < kGroups; ++h) head[h] = 0;
-        const int hc = row / kTokensPerChunk;
-        for (int j = 0; j < p.k; ++j) {
-            int bg = -1;
-            float bv = -INFINITY;
-            int bi = 0x7fffffff;
-#pragma unroll
-            for (int h = 0; h < kGroups; ++h) {
-                if (head[h] < KMAX) {
-                    const float hv = s_lval[(h * KMAX + head[h]) * kBM + row];
-                    const int hi = s_lidx[(h * KMAX + head[h]) * kBM + row];
-                    if (hi < p.E && (bg < 0 || ranks_before(hv, hi, bv, bi))) {
-                        bg = h;
-                        bv = hv;
-                        bi = hi;
+                for (int i = 0; i < 16; ++i) {
+                    const int col = c0 + i;
+                    if (col < c_end) {
+                        float* a = dst + (size_t)col * pitch;
+                        if (S > 1)
+                            st_cluster_f32(mapa_shared(a, (uint32_t)owner), __uint_as_float(acc[i]));
+                        else
+                            *a = __uint_as_float(acc[i]);
                     }
                 }
             }
-#pragma unroll
-            for (int h = 0; h < kGroups; ++h)
-                if (h == bg) ++head[h];
-            s_oid[row * KMAX + j] = bi;
-            s_ow[row * KMAX + j] = expf(bv - mx) / sum;
-            if (p.chunk_counts && bg >= 0) atomicAdd(&s_hist[hc * p.E + bi], 1);
+        }
+        if (S > 1)
+            cluster_sync();  // every slot of this CTA's buffer is written
+        else
+            __syncthreads();
+        // softmax + top-k of the rows this CTA owns in this pass
+        const int row0 = S > 1 ? (int)r * own : pass * own;
+        if (KMAX <= 8) {
+            if (own == 128)
+                topk_rows<8, KMAX>(p, buf, s_bias, s_hist, S, own, pitch, tile0, row0, ok, warp, lane);
+            else
+                topk_rows<16, KMAX>(p, buf, s_bias, s_hist, S, own, pitch, tile0, row0, ok, warp, lane);
+        } else {
+            for (int i = warp; i < own; i += kWarps) {
+                const int64_t t = (int64_t)tile0 + row0 + i;
+                if (t >= p.T) break;  // warp-uniform; later rows are past the end too
+                int my_id;
+                float my_w;
+                warp_topk<16>(E, p.k, lane, [&](int jj) {
+                    const int c = lane + 32 * jj;
+                    const float* col = buf + (size_t)c * pitch + i;
+                    float l = col[0];
+                    for (int s = 1; s < S; ++s) l += col[(size_t)s * E * pitch];
+                    return l + s_bias[c];
+                }, my_id, my_w);
+                if (ok && lane < p.k) {
+                    p.ids[t * p.k + lane] = my_id;
+                    p.wts[t * p.k + lane] = my_w;
+                    if (p.chunk_counts && (unsigned)my_id < (unsigned)E)
+                        atomicAdd(&s_hist[((row0 + i) / kTokensPerChunk) * E + my_id], 1);
+                }
+            }
         }
     }
     __syncthreads();
-    if (ok) {
-        // the tile's ids and weights are contiguous in [T, k]: coalesced copy
-        const int n_tok = min(kBM, p.T - tile0);
-        for (int i = threadIdx.x; i < n_tok * p.k; i += kThreads) {
-            const int r = i / p.k, j = i % p.k;
-            p.ids[(int64_t)tile0 * p.k + i] = s_oid[r * KMAX + j];
-            p.wts[(int64_t)tile0 * p.k + i] = s_ow[r * KMAX + j];
-        }
-        if (p.chunk_counts) {
-            const int chunk0 = tile0 / kTokensPerChunk;
-            for (int i = threadIdx.x; i < kChunksPerTile * p.E; i += kThreads) {
-                const int hc = i / p.E, e = i % p.E;
-                if (chunk0 + hc < p.n_tchunks)
-                    p.chunk_counts[(int64_t)e * p.n_tchunks + chunk0 + hc] = s_hist[i];
-            }
+    if (ok && p.chunk_counts) {
+        // chunks whose tokens this CTA ranked: both of the tile (one CTA), or
+        // chunk r (pair)
+        const int chunk0 = tile0 / kTokensPerChunk;
+        for (int i = threadIdx.x; i < 2 * E; i += kThreads) {
+            const int hc = i / E, e = i % E;
+            if ((S == 1 || hc == (int)r) && chunk0 + hc < p.n_tchunks)
+                p.chunk_counts[(int64_t)e * p.n_tchunks + chunk0 + hc] = s_hist[i];
         }
     }
     tc_fence_before_sync();
