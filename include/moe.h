@@ -229,9 +229,16 @@ int moe_forward(const moe_bf16* x, const moe_bf16* w_router, const float* bias,
  * moe_forward with options.  events (may be NULL): n_events >= 6
  * caller-created CUDA events recorded on `stream` before routing, after
  * routing, after the permutation, after the gate/up GEMM, after the down
- * GEMM and after the combine, for timing stages.  flags: 0 or
- * MOE_FLAG_FUSED_GATHER (other bits: MOE_ERR_INVALID_ARG).  The arithmetic
- * is identical to moe_forward.
+ * GEMM and after the combine, for timing stages; a NULL entry skips that
+ * boundary.  A recorded event makes the next kernel wait for the previous
+ * one to finish (it cannot begin its launch early), so record only the
+ * boundaries you need.  flags: 0 or MOE_FLAG_FUSED_GATHER (other bits:
+ * MOE_ERR_INVALID_ARG).  The arithmetic is identical to moe_forward.
+ *
+ * Every kernel of the library is launched with programmatic dependent
+ * launch: it may begin launching while the previous kernel on the stream
+ * drains, and waits for that kernel's completion before its first global
+ * memory access.
  */
 int moe_forward_ex(const moe_bf16* x, const moe_bf16* w_router, const float* bias,
                    const moe_bf16* w_gate, const moe_bf16* w_up, const moe_bf16* w_down,

@@ -241,9 +241,9 @@ def forward(x, w_router, w_gate, w_up, w_down, k, bias=None, out=None, workspace
             topk_ids=None, topk_w=None, events=None, flags=None):
     """The whole MoE block; returns out [T, d] fp32.
 
-    ``events`` (optional): a list of >= 6 torch.cuda.Event objects recorded at
-    the stage boundaries (before route, after route, after permute, after
-    gate/up, after down, after combine).  ``flags`` (optional):
+    ``events`` (optional): a list of >= 6 torch.cuda.Event objects (or None
+    to skip a boundary) recorded at the stage boundaries (before route, after
+    route, after permute, after gate/up, after down, after combine).  ``flags`` (optional):
     MOE_FLAG_FUSED_GATHER selects the variant whose gate/up GEMM gathers the
     rows of x itself; both variants give identical results.
     """
@@ -266,6 +266,8 @@ def forward(x, w_router, w_gate, w_up, w_down, k, bias=None, out=None, workspace
         if events is not None:
             arr = (ctypes.c_void_p * len(events))()
             for i, ev in enumerate(events):
+                if ev is None:
+                    continue
                 if ev.cuda_event == 0:
                     ev.record()  # the event handle is created lazily by torch
                 arr[i] = ev.cuda_event

@@ -12,7 +12,7 @@
 
 #include <cuda_fp16.h>
 
-#include "status.cuh"
+#include "ptx.cuh"
 
 namespace moe {
 namespace combine {
@@ -26,6 +26,8 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint4* __restrict__ 
 {
     __shared__ int s_pos[kMaxK];
     const int64_t t = blockIdx.x;
+    pdl_trigger();
+    pdl_wait();
     if (threadIdx.x < k) {
         int p = __ldg(inv + t * k + threadIdx.x);
         if ((unsigned)p >= (unsigned long long)n) {

@@ -359,8 +359,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint64_t limit = g_wait_limit_ns;
     const int E = p.E;
 
-    // ---- tile list from the device offsets (validated) ----
-    build_tile_list<kBM>(p.offsets, E, p.M, c.off, c.tp, &c.total_mtiles, &c.bad);
     if (threadIdx.x == 32) {
         for (int s = 0; s < kStages; ++s) {
             // GATHER: the TMA arrival plus one cp.async completion per lane
@@ -388,6 +386,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after_sync();
     const uint32_t tmem = c.tmem_slot;
+    // the offsets and A rows come from earlier kernels on the stream
+    pdl_trigger();
+    pdl_wait();
+    // ---- tile list from the device offsets (validated) ----
+    build_tile_list<kBM>(p.offsets, E, p.M, c.off, c.tp, &c.total_mtiles, &c.bad);
+    __syncthreads();
     const int64_t total_work = c.bad ? 0 : (int64_t)c.total_mtiles * p.n_tiles;
     const int num_kb = p.K / kBK;
 

@@ -72,7 +72,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int64_t pair = cluster_id_x();
     const int64_t npairs = num_clusters_x();
 
-    build_tile_list<kPairRows>(p.offsets, E, p.M, c.off, c.tp, &c.total_mtiles, &c.bad);
     if (threadIdx.x == 32) {
         for (int s = 0; s < kPairStages; ++s) {
             mbar_init(&c.full[s], 1);
@@ -99,6 +98,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     cluster_sync();  // both CTAs' barriers initialised and TMEM allocated
     tc_fence_after_sync();
     const uint32_t tmem = c.tmem_slot;
+    // the offsets and operands come from earlier kernels on the stream
+    pdl_trigger();
+    pdl_wait();
+    build_tile_list<kPairRows>(p.offsets, E, p.M, c.off, c.tp, &c.total_mtiles, &c.bad);
+    __syncthreads();
     const int64_t total_work = c.bad ? 0 : (int64_t)c.total_mtiles * p.n_tiles;
     const int num_kb = p.K / kBK;
 

@@ -63,6 +63,43 @@ constexpr unsigned kDefaultForwardFlags = 0;
 #define MOE_GEMM_PAIR 1
 #endif
 
+// Programmatic dependent launch for every kernel of the library: a launch
+// may begin while the previous kernel on the stream drains; each kernel
+// waits (griddepcontrol.wait) before its first global-memory access.
+#ifndef MOE_PDL
+#define MOE_PDL 1
+#endif
+
+// cudaLaunchKernelEx with the PDL attribute and, for cluster > 1, a 1-D
+// cluster of that many CTAs.
+template <typename... KArgs, typename... Args>
+int launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, unsigned cluster,
+           Args... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[2];
+    unsigned n = 0;
+    if (cluster > 1) {
+        attr[n].id = cudaLaunchAttributeClusterDimension;
+        attr[n].val.clusterDim.x = cluster;
+        attr[n].val.clusterDim.y = 1;
+        attr[n].val.clusterDim.z = 1;
+        ++n;
+    }
+    if (MOE_PDL) {
+        attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[n].val.programmaticStreamSerializationAllowed = 1;
+        ++n;
+    }
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = n;
+    return cudaLaunchKernelEx(&cfg, kernel, args...) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
 template <int EPI>
 int launch_pair_gemm(const DeviceState& st, int64_t work, const CUtensorMap& ta, const CUtensorMap& tb0,
                      const CUtensorMap& tb1, const CUtensorMap& tout, const moe::gemm::Params& p, cudaStream_t s)
@@ -70,21 +107,8 @@ int launch_pair_gemm(const DeviceState& st, int64_t work, const CUtensorMap& ta,
     int64_t pairs = st.max_pairs > 0 ? st.max_pairs : st.sm_count / 2;
     if (work < pairs) pairs = work;
     if (pairs < 1) pairs = 1;
-    cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.gridDim = dim3((unsigned)(2 * pairs));
-    cfg.blockDim = dim3(moe::gemm::kThreads);
-    cfg.dynamicSmemBytes = moe::gemm::pair_smem_bytes<EPI>();
-    cfg.stream = s;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, moe::gemm::grouped_gemm_pair_kernel<EPI>, ta, tb0, tb1, tout, p) == cudaSuccess
-               ? MOE_OK
-               : MOE_ERR_CUDA;
+    return launch(moe::gemm::grouped_gemm_pair_kernel<EPI>, dim3((unsigned)(2 * pairs)), dim3(moe::gemm::kThreads),
+                  moe::gemm::pair_smem_bytes<EPI>(), s, 2u, ta, tb0, tb1, tout, p);
 }
 
 int setup_device(DeviceState** out)
@@ -242,20 +266,8 @@ int launch_route(const CUtensorMap& tx, const CUtensorMap& tw, moe::route::Param
     p.stages = moe::route::kMaxStages;
     while (p.stages > 2 && smem_bytes(p.n_chunks, p.stages, p.E, p.split, p.passes) > (size_t)kMaxDynSmem)
         --p.stages;
-    cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = (unsigned)p.split;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.gridDim = dim3(tiles * (unsigned)p.split);
-    cfg.blockDim = dim3(moe::route::kThreads);
-    cfg.dynamicSmemBytes = smem_bytes(p.n_chunks, p.stages, p.E, p.split, p.passes);
-    cfg.stream = s;
-    cfg.attrs = attr;
-    cfg.numAttrs = p.split > 1 ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, moe::route::route_kernel<KMAX>, tx, tw, p) == cudaSuccess ? MOE_OK
-                                                                                              : MOE_ERR_CUDA;
+    return launch(moe::route::route_kernel<KMAX>, dim3(tiles * (unsigned)p.split), dim3(moe::route::kThreads),
+                  smem_bytes(p.n_chunks, p.stages, p.E, p.split, p.passes), s, (unsigned)p.split, tx, tw, p);
 }
 
 int run_route(const DeviceState& st, const moe_bf16* x, const moe_bf16* w_router, const float* bias, int64_t T,
@@ -313,16 +325,25 @@ int run_permute(const moe_bf16* x, const int32_t* ids, const float* wts, int64_t
     }
     using namespace moe::permute;
     const int nch = (int)token_chunks(T);
-    if (!have_hist) hist_kernel<<<nch, kThreads, 0, s>>>(ids, T, (int)k, (int)E, chunk_em, nch);
-    chunk_scan_kernel<<<(unsigned)E, kThreads, 0, s>>>(chunk_em, nch, counts);
-    rank_kernel<<<nch, kThreads, 0, s>>>(ids, wts, T, (int)k, (int)E, chunk_em, nch, counts, offsets, perm, inv,
-                                         w_perm);
+    const int32_t* cids = ids;
+    const float* cw = wts;
+    const int ik = (int)k, iE = (int)E;
+    if (!have_hist && launch(hist_kernel, dim3(nch), dim3(kThreads), 0, s, 1u, cids, T, ik, iE, chunk_em, nch))
+        return MOE_ERR_CUDA;
+    if (launch(chunk_scan_kernel, dim3((unsigned)E), dim3(kThreads), 0, s, 1u, chunk_em, nch, counts))
+        return MOE_ERR_CUDA;
+    if (launch(rank_kernel, dim3(nch), dim3(kThreads), 0, s, 1u, cids, cw, T, ik, iE,
+               static_cast<const int32_t*>(chunk_em), nch, static_cast<const int32_t*>(counts), offsets, perm, inv,
+               w_perm))
+        return MOE_ERR_CUDA;
     if (x_perm) {
         const int64_t n = T * k;
-        gather_kernel<<<(unsigned)((n + kWarps - 1) / kWarps), kThreads, 0, s>>>(
-            reinterpret_cast<const uint4*>(x), perm, n, (int)(d / 8), (int)k, reinterpret_cast<uint4*>(x_perm));
+        if (launch(gather_kernel, dim3((unsigned)((n + kWarps - 1) / kWarps)), dim3(kThreads), 0, s, 1u,
+                   reinterpret_cast<const uint4*>(x), static_cast<const int32_t*>(perm), n, (int)(d / 8), ik,
+                   reinterpret_cast<uint4*>(x_perm)))
+            return MOE_ERR_CUDA;
     }
-    return launch_status();
+    return MOE_OK;
 }
 
 // The two grouped GEMMs.  With x_gather/perm set, the gate/up GEMM reads its
@@ -373,11 +394,14 @@ int run_ffn(const DeviceState& st, const moe_bf16* x_perm, const moe_bf16* x_gat
     const int64_t max_pair_tiles = (M + kPairRows - 1) / kPairRows + E;
     if (MOE_GEMM_PAIR && !gather) {
         if (launch_pair_gemm<kSwiGLU>(st, max_pair_tiles * p1.n_tiles, ta1, tg, tu, ty, p1, s)) return MOE_ERR_CUDA;
-    } else if (gather)
-        grouped_gemm_kernel<kSwiGLU, true><<<grid1, kThreads, smem1, s>>>(ta1, tg, tu, ty, p1);
-    else
-        grouped_gemm_kernel<kSwiGLU, false><<<grid1, kThreads, smem1, s>>>(ta1, tg, tu, ty, p1);
-    if (launch_status()) return MOE_ERR_CUDA;
+    } else if (gather) {
+        if (launch(grouped_gemm_kernel<kSwiGLU, true>, dim3(grid1), dim3(kThreads), smem1, s, 1u, ta1, tg, tu, ty, p1))
+            return MOE_ERR_CUDA;
+    } else {
+        if (launch(grouped_gemm_kernel<kSwiGLU, false>, dim3(grid1), dim3(kThreads), smem1, s, 1u, ta1, tg, tu, ty,
+                   p1))
+            return MOE_ERR_CUDA;
+    }
     if (mid_event && cudaEventRecord(mid_event, s) != cudaSuccess) return MOE_ERR_CUDA;
 
     Params p2;
@@ -395,12 +419,9 @@ int run_ffn(const DeviceState& st, const moe_bf16* x_perm, const moe_bf16* x_gat
     p2.k_top = 1;
     const int64_t work2 = max_mtiles * p2.n_tiles;
     const unsigned grid2 = (unsigned)(work2 < st.sm_count ? work2 : st.sm_count);
-    if (MOE_GEMM_PAIR) {
-        if (launch_pair_gemm<kWeighted>(st, max_pair_tiles * p2.n_tiles, ta2, td, td, ty, p2, s)) return MOE_ERR_CUDA;
-        return launch_status();
-    }
-    grouped_gemm_kernel<kWeighted, false><<<grid2, kThreads, smem2, s>>>(ta2, td, td, ty, p2);
-    return launch_status();
+    if (MOE_GEMM_PAIR) return launch_pair_gemm<kWeighted>(st, max_pair_tiles * p2.n_tiles, ta2, td, td, ty, p2, s);
+    return launch(grouped_gemm_kernel<kWeighted, false>, dim3(grid2), dim3(kThreads), smem2, s, 1u, ta2, td, td, ty,
+                  p2);
 }
 
 int run_combine(const moe_f16* y, const int32_t* inv, int64_t T, int64_t d, int64_t k, float* out, cudaStream_t s)
@@ -408,9 +429,8 @@ int run_combine(const moe_f16* y, const int32_t* inv, int64_t T, int64_t d, int6
     if (T == 0) return MOE_OK;
     const int nvec = (int)(d / 8);
     const int threads = nvec < 256 ? ((nvec + 31) / 32) * 32 : 256;
-    moe::combine::combine_kernel<<<(unsigned)T, threads, 0, s>>>(reinterpret_cast<const uint4*>(y), inv, T * k,
-                                                                 nvec, (int)k, reinterpret_cast<float4*>(out));
-    return launch_status();
+    return launch(moe::combine::combine_kernel, dim3((unsigned)T), dim3(threads), 0, s, 1u,
+                  reinterpret_cast<const uint4*>(y), inv, T * k, nvec, (int)k, reinterpret_cast<float4*>(out));
 }
 
 int forward_impl(const moe_bf16* x, const moe_bf16* w_router, const float* bias, const moe_bf16* w_gate,
@@ -433,7 +453,9 @@ int forward_impl(const moe_bf16* x, const moe_bf16* w_router, const float* bias,
     if (ws_bytes < L.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
     DeviceState* st = nullptr;
     if ((rc = setup_device(&st))) return rc;
-    auto rec = [&](int i) { return (ev && cudaEventRecord(ev[i], s) != cudaSuccess) ? MOE_ERR_CUDA : MOE_OK; };
+    auto rec = [&](int i) {
+        return (ev && ev[i] && cudaEventRecord(ev[i], s) != cudaSuccess) ? MOE_ERR_CUDA : MOE_OK;
+    };
     if ((rc = rec(0))) return rc;
     if (T == 0) {
         for (int i = 1; i < 6; ++i)

@@ -22,7 +22,7 @@
 
 #include <cuda_bf16.h>
 
-#include "status.cuh"
+#include "ptx.cuh"
 
 namespace moe {
 namespace permute {
@@ -37,6 +37,8 @@ __global__ void __launch_bounds__(kThreads) hist_kernel(const int32_t* __restric
                                                         int32_t* __restrict__ counts_em, int n_tchunks)
 {
     __shared__ int s_hist[kMaxE];
+    pdl_trigger();
+    pdl_wait();
     for (int e = threadIdx.x; e < E; e += kThreads) s_hist[e] = 0;
     __syncthreads();
     const int64_t a0 = (int64_t)blockIdx.x * kTokensPerChunk * k;
@@ -59,6 +61,8 @@ __global__ void __launch_bounds__(kThreads) chunk_scan_kernel(int32_t* __restric
                                                               int32_t* __restrict__ totals)
 {
     __shared__ int s_warp[32];
+    pdl_trigger();
+    pdl_wait();
     int32_t* row = counts_em + (int64_t)blockIdx.x * n_tchunks;
     const int tid = threadIdx.x, lane = tid % 32, warp = tid / 32;
     int carry = 0;
@@ -118,6 +122,8 @@ __global__ void __launch_bounds__(kThreads) rank_kernel(const int32_t* __restric
     __shared__ int s_warp[32];
     const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
     const int chunk = blockIdx.x;
+    pdl_trigger();
+    pdl_wait();
 
     // group offsets = exclusive scan of the totals (E <= 512 <= 4 * 256)
     for (int e = tid; e < E; e += kThreads) s_off[e] = totals[e];
@@ -213,6 +219,8 @@ __global__ void __launch_bounds__(kThreads) gather_kernel(const uint4* __restric
 {
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const int64_t row = (int64_t)blockIdx.x * kWarps + warp;
+    pdl_trigger();
+    pdl_wait();
     if (row >= n) return;
     const int a = __ldg(perm + row);
     if ((unsigned)a >= (unsigned long long)n) {

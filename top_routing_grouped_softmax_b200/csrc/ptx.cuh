@@ -284,6 +284,16 @@ __device__ __forceinline__ uint32_t mapa_shared(const void* p, uint32_t rank)
     return r;
 }
 
+// ------------------------------------------ programmatic dependent launch
+// Let the next kernel on the stream start launching (its own prologue then
+// waits in pdl_wait), and wait until every kernel this one depends on has
+// completed with its memory visible.  Both are no-ops for a launch without
+// the programmatic-serialisation attribute.  Every kernel of the library
+// calls pdl_wait before its first global-memory access, so completion
+// chains through the whole stream.
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // Store to shared memory of any CTA of the cluster (address from mapa_shared).
 __device__ __forceinline__ void st_cluster_f32(uint32_t cluster_addr, float v)
 {

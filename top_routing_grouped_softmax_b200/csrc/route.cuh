@@ -324,8 +324,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int kb1 = (int)((int64_t)nkb * (r + 1) / S);
     const int E = p.E;
 
-    for (int e = threadIdx.x; e < E; e += kThreads) s_bias[e] = p.bias ? p.bias[e] : 0.0f;
-    for (int e = threadIdx.x; e < 2 * E; e += kThreads) s_hist[e] = 0;
     if (threadIdx.x == 0) {
         for (int s = 0; s < p.stages; ++s) {
             mbar_init(&full[s], 1);
@@ -346,6 +344,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after_sync();
     const uint32_t tmem = *tmem_slot;
+    // x may come from an earlier kernel on the stream, and earlier kernels
+    // may still read the ids, weights and histograms this launch writes
+    pdl_trigger();
+    pdl_wait();
+    for (int e = threadIdx.x; e < E; e += kThreads) s_bias[e] = p.bias ? p.bias[e] : 0.0f;
+    for (int e = threadIdx.x; e < 2 * E; e += kThreads) s_hist[e] = 0;
+    __syncthreads();
 
     if (warp == 0) {
         if (lane == 0) {
