@@ -7,11 +7,14 @@ One step = one moe_forward (router GEMM + softmax + top-k, permutation,
 grouped gate/up + SwiGLU GEMM, grouped down GEMM + routing weight, combine)
 over one batch of T tokens of the named workload, with every input already
 resident in HBM.  L2 is flushed (a 256 MiB write) between timed steps, and
-each step is timed with CUDA events on the launching stream; the stage
-boundaries inside a step are timed with events the library records on the
-same stream.  `e2e` repeats the measurement through the public API with the
-token batch copied host->device from pinned memory and the output copied
-back inside the timed region.
+each step is timed with CUDA events on the launching stream; inside a step
+the library records events only around the gate/up GEMM (the roofline
+kernel), because a recorded event stops the next kernel from launching
+early.  A second pass of the same steps records every stage boundary for
+the stage breakdown.  `e2e` repeats the measurement through the public API
+with the token batch copied host->device from pinned memory and the output
+copied back inside the timed region.  SM clocks and throttle reasons are
+sampled through NVML during the timed region.
 
 Multi-GPU: one process per GPU (torchrun); every rank runs its own replica
 on its own batch (the block is independent per token, so the path shards by
@@ -24,9 +27,7 @@ import argparse
 import json
 import os
 import statistics
-import subprocess
 import sys
-import tempfile
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -85,56 +86,70 @@ def algorithmic(cfg, active_experts=None):
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle sampling while the timed region runs."""
+    """SM clock / throttle-reason sampling while the timed region runs.
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    Reads NVML every few milliseconds from a background thread (read-only
+    queries; no clock or power setting is touched); without NVML the summary
+    says "unsampled".  The device is matched by its PCI bus id, so
+    CUDA_VISIBLE_DEVICES does not matter.
+    """
+
+    REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40), ("sw_thermal_slowdown", 0x20),
+               ("sw_power_cap", 0x4))
+    PERIOD_S = 0.004
 
     def __init__(self, device_index: int):
         self.dev = device_index
-        self.proc = None
-        self.path = None
+        self.samples = []   # (sm_mhz, max_mhz, power_w, reasons_bitmask)
+        self.stop = None
+        self.thread = None
+
+    def _handle(self):
+        import pynvml
+        import torch
+        pynvml.nvmlInit()
+        prop = torch.cuda.get_device_properties(self.dev)
+        bus = f"{prop.pci_domain_id:08x}:{prop.pci_bus_id:02x}:{prop.pci_device_id:02x}.0"
+        try:
+            return pynvml, pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+        except pynvml.NVMLError:
+            return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.dev)
+
+    def _run(self, nv, h):
+        while not self.stop.is_set():
+            try:
+                self.samples.append((nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM),
+                                     nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM),
+                                     nv.nvmlDeviceGetPowerUsage(h) / 1000.0,
+                                     nv.nvmlDeviceGetCurrentClocksEventReasons(h)))
+            except Exception:
+                pass
+            time.sleep(self.PERIOD_S)
 
     def __enter__(self):
-        fd, self.path = tempfile.mkstemp(suffix=".csv")
-        os.close(fd)
+        import threading
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100",
-                 "-i", str(self.dev)], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
-        except OSError:
-            self.proc = None
-        time.sleep(0.3)
+            nv, h = self._handle()
+        except Exception:
+            return self
+        self.stop = threading.Event()
+        self.thread = threading.Thread(target=self._run, args=(nv, h), daemon=True)
+        self.thread.start()
         return self
 
     def __exit__(self, *exc):
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
+        if self.thread is not None:
+            self.stop.set()
+            self.thread.join(timeout=5)
 
     def summary(self):
-        rows = []
-        if self.path and os.path.exists(self.path):
-            for line in open(self.path):
-                parts = [p.strip() for p in line.split(",")]
-                if len(parts) < 9:
-                    continue
-                try:
-                    rows.append((float(parts[1]), float(parts[2]), float(parts[3]), parts[5:9]))
-                except ValueError:
-                    continue
-            os.unlink(self.path)
+        rows = self.samples
         if not rows:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
-        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
-        reasons = sorted({names[i] for r in rows for i, v in enumerate(r[3]) if v.lower() == "active"})
-        loaded = [r for r in rows if r[2] > 250.0] or rows
-        return {"sm_mhz": statistics.median(r[0] for r in loaded), "sm_max_mhz": max(r[1] for r in rows),
-                "power_w_max": max(r[2] for r in rows), "samples": len(rows), "reasons": reasons}
+        reasons = sorted({name for r in rows for name, bit in self.REASONS if r[3] & bit})
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_mhz_min": min(r[0] for r in rows),
+                "sm_max_mhz": max(r[1] for r in rows), "power_w_max": max(r[2] for r in rows),
+                "samples": len(rows), "source": "NVML, every 4 ms during the timed region", "reasons": reasons}
 
 
 # ------------------------------------------------------------ CPU oracle
@@ -386,7 +401,7 @@ def run_gpu(args, cfg):
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default="qwen")

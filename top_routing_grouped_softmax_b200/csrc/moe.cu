@@ -337,9 +337,8 @@ int run_permute(const moe_bf16* x, const int32_t* ids, const float* wts, int64_t
                w_perm))
         return MOE_ERR_CUDA;
     if (x_perm) {
-        const int64_t n = T * k;
-        if (launch(gather_kernel, dim3((unsigned)((n + kWarps - 1) / kWarps)), dim3(kThreads), 0, s, 1u,
-                   reinterpret_cast<const uint4*>(x), static_cast<const int32_t*>(perm), n, (int)(d / 8), ik,
+        if (launch(gather_kernel, dim3((unsigned)((T + kWarps - 1) / kWarps)), dim3(kThreads), 0, s, 1u,
+                   reinterpret_cast<const uint4*>(x), static_cast<const int32_t*>(inv), T, ik, (int)(d / 8),
                    reinterpret_cast<uint4*>(x_perm)))
             return MOE_ERR_CUDA;
     }

@@ -16,8 +16,8 @@
 //                lane among same-expert lanes, so every group lists its
 //                assignments in ascending a -- deterministic, no global
 //                atomics.
-//   gather     : x_perm[pos] = x[perm[pos] / k], one warp per row, 16-byte
-//                vectors, many rows in flight per SM.
+//   gather     : x_perm[inv[t*k + j]] = x[t]: one warp per token reads the
+//                row once and writes its k copies (16-byte vectors).
 #pragma once
 
 #include <cuda_bf16.h>
@@ -212,25 +212,48 @@ __global__ void __launch_bounds__(kThreads) rank_kernel(const int32_t* __restric
     }
 }
 
-// x_perm[pos] = x[perm[pos] / k]; one warp per grouped row.
+// x_perm[inv[t*k + j]] = x[t] for every slot j: one warp per token reads the
+// token's row once (16-byte vectors, eight in flight per lane) and writes it
+// to its k grouped positions, so x is read from HBM once and every write is
+// a whole contiguous row.
 __global__ void __launch_bounds__(kThreads) gather_kernel(const uint4* __restrict__ x,
-                                                          const int32_t* __restrict__ perm, int64_t n, int nvec,
-                                                          int k, uint4* __restrict__ x_perm)
+                                                          const int32_t* __restrict__ inv, int64_t T, int k,
+                                                          int nvec, uint4* __restrict__ x_perm)
 {
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    const int64_t row = (int64_t)blockIdx.x * kWarps + warp;
+    const int64_t t = (int64_t)blockIdx.x * kWarps + warp;
     pdl_trigger();
     pdl_wait();
-    if (row >= n) return;
-    const int a = __ldg(perm + row);
-    if ((unsigned)a >= (unsigned long long)n) {
-        record_status(kStatusDeviceBounds);
-        return;
+    if (t >= T) return;
+    const int64_t n = T * k;
+    int pos = -1;
+    if (lane < k) {
+        pos = __ldg(inv + t * k + lane);
+        if ((unsigned long long)(unsigned)pos >= (unsigned long long)n) {
+            record_status(kStatusDeviceBounds);
+            pos = -1;
+        }
     }
-    const uint4* src = x + (int64_t)(a / k) * nvec;
-    uint4* dst = x_perm + row * nvec;
-#pragma unroll 8
-    for (int v = lane; v < nvec; v += 32) dst[v] = __ldg(src + v);
+    const uint4* src = x + t * nvec;
+    constexpr int kUnroll = 8;
+    for (int v0 = 0; v0 < nvec; v0 += 32 * kUnroll) {
+        uint4 buf[kUnroll];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const int v = v0 + u * 32 + lane;
+            if (v < nvec) buf[u] = __ldg(src + v);
+        }
+        for (int j = 0; j < k; ++j) {
+            const int pj = __shfl_sync(0xffffffffu, pos, j);  // warp-uniform
+            if (pj < 0) continue;
+            uint4* dst = x_perm + (int64_t)pj * nvec;
+#pragma unroll
+            for (int u = 0; u < kUnroll; ++u) {
+                const int v = v0 + u * 32 + lane;
+                if (v < nvec) dst[v] = buf[u];
+            }
+        }
+    }
 }
 
 }  // namespace permute
