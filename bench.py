@@ -82,7 +82,21 @@ def algorithmic(cfg, active_experts=None):
     nact = E if active_experts is None else active_experts
     # x read + out write (fp32) + router weights + weights of the experts in use
     compulsory = T * d * 2 + T * d * 4 + d * E * 2 + nact * 3 * d * f * 2
-    return {"flops": flops, "gateup_flops": gateup_flops, "down_flops": down_flops, "bytes": compulsory}
+    # per-stage algorithmic HBM bytes: route reads x and W_router and writes
+    # ids + weights; permute reads x and writes x_perm (+ 12 B per
+    # assignment of indices and weights); combine reads y (fp16), writes out
+    stage_bytes = {
+        "route": T * d * 2 + d * E * 2 + T * k * 8,
+        "permute": T * d * 2 + T * k * d * 2 + T * k * 12,
+        "combine": T * k * d * 2 + T * d * 4,
+    }
+    return {"flops": flops, "gateup_flops": gateup_flops, "down_flops": down_flops, "bytes": compulsory,
+            "stage_bytes": stage_bytes}
+
+
+# Datasheet figures for a B200 (dense bf16, HBM3e), for the second fraction
+# of the forward roofline; the primary fraction uses the measured peaks.
+DATASHEET = {"bf16_tflops": 2250.0, "hbm_gbs": 8000.0}
 
 
 class ClockSampler:
@@ -175,11 +189,25 @@ def time_oracle(cfg, n_tokens: int, seed: int, inp=None):
     return time.perf_counter() - t0, n_tokens
 
 
+def host_cpu():
+    """CPU model and logical core count of the host the oracle runs on."""
+    model = "unknown"
+    try:
+        with open("/proc/cpuinfo") as fh:
+            for line in fh:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"cpu_model": model, "host_logical_cpus": os.cpu_count()}
+
+
 def cpu_baseline(cfg, n_tokens: int, seed: int, inp=None):
     secs, n = time_oracle(cfg, n_tokens, seed, inp)
     return {"value": n / secs, "unit": UNIT, "cores": 1, "kind": "oracle",
             "sample": f"first {n} of {cfg.T} tokens of the {cfg.name} workload, full block "
-                      f"(route, permute, expert MLPs, combine), fp64, one thread"}
+                      f"(route, permute, expert MLPs, combine), fp64, one thread", **host_cpu()}
 
 
 # ------------------------------------------------------------- reference
@@ -201,7 +229,8 @@ def run_reference(args, cfg):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": workload_config(cfg, extra={"tokens_per_step": n}),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
-                         "sample": f"first {n} of {cfg.T} tokens per step, full block, fp64, one thread"},
+                         "sample": f"first {n} of {cfg.T} tokens per step, full block, fp64, one thread",
+                         **host_cpu()},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -314,8 +343,10 @@ def run_gpu(args, cfg):
     # expert load statistics of the batch
     counts = torch.bincount(ids.flatten().long(), minlength=cfg.E).cpu()
     active = int((counts > 0).sum())
-    tiles = int(((counts + 127) // 128).sum())
-    padding = 1.0 - cfg.T * cfg.k / (tiles * 128)
+    # the grouped GEMMs run 256-row CTA-pair tiles: rows past a group's end
+    # are computed and not stored
+    tiles = int(((counts + 255) // 256).sum())
+    padding = 1.0 - cfg.T * cfg.k / (tiles * 256)
 
     # ---- end to end through the public API, host buffers, copies timed
     x_host = inp.x.pin_memory()
@@ -359,6 +390,7 @@ def run_gpu(args, cfg):
         roof_flops = alg["gateup_flops"] + (alg["down_flops"] if args.path == "stages" else 0)
         achieved = roof_flops / (gateup_ms_max * 1e-3) / 1e12
         roof_time = max(alg["flops"] / (peaks["bf16_tflops"] * 1e12), alg["bytes"] / (peaks["hbm_gbs"] * 1e9))
+        roof_ds = max(alg["flops"] / (DATASHEET["bf16_tflops"] * 1e12), alg["bytes"] / (DATASHEET["hbm_gbs"] * 1e9))
         traffic = None
         tpath = os.path.join(ROOT, "profiles", "gateup_traffic.json")
         if os.path.exists(tpath):
@@ -375,6 +407,8 @@ def run_gpu(args, cfg):
             "tflops": alg["flops"] / (ms * 1e-3) / 1e12,
             "grouped_gemm_tflops": (alg["gateup_flops"] + alg["down_flops"]) /
                                    ((stage_ms["gateup_gemm"] + stage_ms["down_gemm"]) * 1e-3) / 1e12,
+            "grouped_gemm_tflops_padded": (alg["gateup_flops"] + alg["down_flops"]) / (1.0 - padding) /
+                                          ((stage_ms["gateup_gemm"] + stage_ms["down_gemm"]) * 1e-3) / 1e12,
             "roofline": {"bound": "tensor",
                          "kernel": ("grouped_gemm_pair_kernel<SwiGLU> (gate/up + SwiGLU)" if args.path == "fused"
                                     else "moe_expert_ffn (gate/up + down GEMMs)"),
@@ -382,11 +416,16 @@ def run_gpu(args, cfg):
                          "frac": achieved / peaks["bf16_tflops"], "traffic": traffic,
                          "peak_source": f"{peaks['source']} burst bf16"},
             "forward_roofline": {"roofline_ms": roof_time * 1e3, "frac": roof_time / (ms * 1e-3),
-                                 "flops": alg["flops"], "compulsory_bytes": alg["bytes"]},
+                                 "flops": alg["flops"], "compulsory_bytes": alg["bytes"],
+                                 "peaks": "of measured (MEASURED_PEAKS.json)",
+                                 "frac_of_datasheet": roof_ds / (ms * 1e-3),
+                                 "datasheet_peaks": "2250 TFLOP/s dense bf16, 8000 GB/s"},
+            "stage_gbs": {st: alg["stage_bytes"][st] / (stage_ms[st] * 1e-3) / 1e9
+                          for st in ("route", "permute", "combine")},
             "stage_ms": stage_ms,
             "stage_ms_note": "second pass of the same steps with every stage boundary recorded",
             "experts": {"active": active, "max_count": int(counts.max()), "min_count": int(counts.min()),
-                        "tile_padding": padding},
+                        "pair_tile_padding": padding},
             "e2e": {"value": whole_job_rate(cfg.T * args.steps, world, [e2e_s]), "unit": UNIT,
                     "h2d_bytes_per_step": cfg.T * cfg.d * 2, "d2h_bytes_per_step": cfg.T * cfg.d * 4},
             "gpu_launches": KERNELS_PER_FORWARD * args.steps,
