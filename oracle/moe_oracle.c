@@ -134,6 +134,23 @@ int oracle_route(const uint16_t* x, const uint16_t* w_router, const float* bias,
 }
 
 /*
+ * Optional variant (not in the article's listing, which keeps the top-k
+ * probabilities as they are): renormalised routing weights,
+ *   w[t][j] <- w[t][j] / sum_{m = 0..k-1} w[t][m]   (sum over m ascending),
+ * so that each token's k weights sum to one.  In place.
+ */
+int oracle_renormalize(double* weights, int64_t T, int64_t k)
+{
+    if (!weights || T < 0 || k < 1) return ORACLE_BAD_ARG;
+    for (int64_t t = 0; t < T; ++t) {
+        double s = 0.0;
+        for (int64_t j = 0; j < k; ++j) s += weights[t * k + j];
+        for (int64_t j = 0; j < k; ++j) weights[t * k + j] /= s;
+    }
+    return ORACLE_OK;
+}
+
+/*
  * Grouping of the T*k assignments by expert (the "token reordering" step of
  * the article's section 2.2: sort_tokens_by_expert, then gather).
  *   counts  [E]    assignments per expert

@@ -62,12 +62,13 @@ class Oracle:
         lib.oracle_permute.argtypes = [_P, _I64, _I64, _I64, _P, _P, _P, _P]
         lib.oracle_expert_rows.argtypes = [_P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64,
                                            _P, _P, _I64, _P, _P, _P, _P]
-        for fn in (lib.oracle_route, lib.oracle_permute, lib.oracle_expert_rows):
+        lib.oracle_renormalize.argtypes = [_P, _I64, _I64]
+        for fn in (lib.oracle_route, lib.oracle_permute, lib.oracle_expert_rows, lib.oracle_renormalize):
             fn.restype = ctypes.c_int
         self.lib = lib
 
     # -- stage 1 + 2 ------------------------------------------------------
-    def route(self, x, w_router, bias, k, want_logits=False, want_probs=True):
+    def route(self, x, w_router, bias, k, want_logits=False, want_probs=True, renormalize=False):
         x = np.ascontiguousarray(x, dtype=np.uint16)
         w_router = np.ascontiguousarray(w_router, dtype=np.uint16)
         T, d = x.shape
@@ -82,6 +83,10 @@ class Oracle:
                                    _ptr(logits), _ptr(probs), _ptr(ids), _ptr(w))
         if rc != 0:
             raise ValueError(f"oracle_route failed ({rc})")
+        if renormalize:
+            rc = self.lib.oracle_renormalize(_ptr(w), T, k)
+            if rc != 0:
+                raise ValueError(f"oracle_renormalize failed ({rc})")
         return RouteResult(ids=ids, weights=w, probs=probs, logits=logits)
 
     # -- grouping -----------------------------------------------------------
@@ -124,9 +129,9 @@ class Oracle:
 
     # -- whole block ----------------------------------------------------------
     def forward(self, x, w_router, bias, w_gate, w_up, w_down, k, rows=None,
-                want_y=False, want_h=False):
+                want_y=False, want_h=False, renormalize=False):
         """Route every token; evaluate the expert MLPs for ``rows`` (all if None)."""
-        r = self.route(x, w_router, bias, k)
+        r = self.route(x, w_router, bias, k, renormalize=renormalize)
         if rows is None:
             rows = np.arange(x.shape[0], dtype=np.int64)
         ex = self.expert_rows(x, w_gate, w_up, w_down, r.ids, r.weights, rows,

@@ -267,8 +267,27 @@ def check_expert_rows_outputs(o):
         assert np.allclose(ex.out[i], ex.y[i].sum(axis=0), rtol=1e-13, atol=1e-15)
 
 
+def check_renormalize(o):
+    """Renormalised routing weights equal a softmax over the k selected
+    logits only (scipy, from the numpy logits) -- a different formula for
+    the same quantity; they sum to one; with k = E they are the plain
+    probabilities; the selected ids do not change."""
+    inp = _rand_case(48, 64, 16, 4, 32, seed=31, bias=True)
+    x, wr, b = inp.bits("x"), inp.bits("W_router"), inp.bias_np()
+    plain = o.route(x, wr, b, 4)
+    r = o.route(x, wr, b, 4, renormalize=True)
+    assert np.array_equal(r.ids, plain.ids)
+    logits = widen(x) @ widen(wr) + b.astype(np.float64)[None, :]
+    sel = np.take_along_axis(logits, r.ids.astype(np.int64), axis=1)
+    np.testing.assert_allclose(r.weights, sps.softmax(sel, axis=1), rtol=1e-12, atol=0)
+    np.testing.assert_allclose(r.weights.sum(axis=1), 1.0, rtol=0, atol=1e-14)
+    full = o.route(x, wr, b, 16, renormalize=True)
+    np.testing.assert_allclose(full.weights, o.route(x, wr, b, 16).weights, rtol=1e-14, atol=0)
+
+
 ALL_CHECKS = [
     check_brute_force, check_softmax_library, check_topk_library_sort, check_topk_of_logits,
     check_exact_ties, check_dense_special_case, check_all_experts_identical, check_zero_expert,
     check_scale_down, check_permute_library, check_page_listing_torch, check_expert_rows_outputs,
+    check_renormalize,
 ]

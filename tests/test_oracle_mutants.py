@@ -28,6 +28,9 @@ MUTANTS = [
     ("softmax_no_norm", "for (int64_t e = 0; e < E; ++e) prob[e] /= s;", "for (int64_t e = 0; e < E; ++e) prob[e] /= 1.0;"),
     ("weights_from_wrong_slot", "weights[t * k + j] = ranked[j].p;", "weights[t * k + j] = ranked[0].p;"),
     ("sum_only_first_slot", "orow[c] += yc;", "orow[c] += (j == 0) ? yc : 0.0;"),
+    ("renorm_no_divide", "weights[t * k + j] /= s;", "weights[t * k + j] /= 1.0;"),
+    ("renorm_partial_sum", "for (int64_t j = 0; j < k; ++j) s += weights[t * k + j];",
+     "for (int64_t j = 0; j + 1 < k; ++j) s += weights[t * k + j];"),
 ]
 
 
