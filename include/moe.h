@@ -127,6 +127,24 @@ int moe_route(const moe_bf16* x, const moe_bf16* w_router, const float* bias,
               int32_t* topk_ids, float* topk_w,
               void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
+/* Flag of moe_route_ex and moe_forward_ex: renormalise the routing
+ * weights, w[t,j] = p[t,ids[t,j]] / sum_m p[t,ids[t,m]] (each token's k
+ * weights sum to one).  Not part of the article's listing, which keeps the
+ * top-k probabilities as they are; the default (no flag) follows the
+ * listing. */
+#define MOE_FLAG_RENORMALIZE 2u
+
+/*
+ * moe_route with flags: 0 or MOE_FLAG_RENORMALIZE (other bits:
+ * MOE_ERR_INVALID_ARG).  Same ids as moe_route; with the flag each weight
+ * is exp(l - max) divided by the sum of exp(l_m - max) over the token's k
+ * selected experts.
+ */
+int moe_route_ex(const moe_bf16* x, const moe_bf16* w_router, const float* bias,
+                 int64_t T, int64_t d, int64_t E, int64_t k,
+                 int32_t* topk_ids, float* topk_w,
+                 void* workspace, size_t workspace_bytes, cudaStream_t stream, unsigned flags);
+
 /*
  * Token reordering by expert (section 2.2: sort_tokens_by_expert, then
  * gather hidden states and routing weights in that order).
@@ -232,8 +250,9 @@ int moe_forward(const moe_bf16* x, const moe_bf16* w_router, const float* bias,
  * GEMM and after the combine, for timing stages; a NULL entry skips that
  * boundary.  A recorded event makes the next kernel wait for the previous
  * one to finish (it cannot begin its launch early), so record only the
- * boundaries you need.  flags: 0 or MOE_FLAG_FUSED_GATHER (other bits:
- * MOE_ERR_INVALID_ARG).  The arithmetic is identical to moe_forward.
+ * boundaries you need.  flags: any of MOE_FLAG_FUSED_GATHER and
+ * MOE_FLAG_RENORMALIZE (other bits: MOE_ERR_INVALID_ARG).  Without
+ * MOE_FLAG_RENORMALIZE the arithmetic is identical to moe_forward.
  *
  * Every kernel of the library is launched with programmatic dependent
  * launch: it may begin launching while the previous kernel on the stream

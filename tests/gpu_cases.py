@@ -61,3 +61,15 @@ def oracle_rows(cfg: MoEConfig, n: int):
 
 SAMPLES = {"tiny": 256, "qwen": 384, "fine": 384, "coarse": 24, "skew": 256}
 FULL = [CONFIGS[n] for n in ("tiny", "qwen", "fine", "coarse", "skew")]
+
+
+def near_tie_masks(cfg: MoEConfig):
+    """(excluded, inner) token masks of the oracle routing: a k-th / (k+1)-th
+    probability gap below the tie threshold (left out), and a near tie
+    inside the selected set (ids compared as a set)."""
+    from oracle.oracle import inner_gap, topk_gap
+    from tests.parity import TIE_EPS
+    probs = oracle_route(cfg).probs
+    excluded = topk_gap(probs, cfg.k) < TIE_EPS
+    inner = (inner_gap(probs, cfg.k) < TIE_EPS) & ~excluded
+    return excluded, inner

@@ -130,3 +130,25 @@ def test_forward_profiled_events():
     assert all(t >= 0 for t in times)
     ref, _, _ = _forward(cfg, d)
     assert torch.equal(out, ref)
+
+
+@pytest.mark.parametrize("cfg", [SMALL[0], SMALL[1], gc.small_cfg(257, 128, 64, 16, 128)], ids=lambda c: c.name)
+def test_forward_renormalized(cfg):
+    """MOE_FLAG_RENORMALIZE end to end, every token, against the oracle with
+    renormalised weights (k = 16 runs the whole-warp top-k)."""
+    d = gc.on_device(gc.inputs(cfg))
+    out, ids, w = _forward(cfg, d, moe.MOE_FLAG_RENORMALIZE)
+    inp = gc.inputs(cfg)
+    o = gc.default_oracle()
+    r = o.route(inp.bits("x"), inp.bits("W_router"), inp.bias_np(), cfg.k, renormalize=True)
+    excluded, inner = gc.near_tie_masks(cfg)
+    g = ids.cpu().numpy()
+    exact = ~excluded & ~inner
+    assert np.array_equal(g[exact], r.ids[exact])
+    assert np.array_equal(np.sort(g[inner], axis=1), np.sort(r.ids[inner], axis=1))
+    rows = np.arange(cfg.T, dtype=np.int64)
+    ex = o.expert_rows(inp.bits("x"), inp.bits("W_gate"), inp.bits("W_up"), inp.bits("W_down"), r.ids, r.weights,
+                       rows)
+    keep = ~excluded
+    value_check(out.double().cpu().numpy()[keep], ex.out[keep], f"out[{cfg.name}, renormalised]")
+    np.testing.assert_allclose(w.cpu().numpy().sum(axis=1), 1.0, rtol=0, atol=cfg.k * 5e-5)

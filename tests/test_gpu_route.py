@@ -8,7 +8,7 @@ import torch
 
 import top_routing_grouped_softmax_b200 as moe
 from tests import gpu_cases as gc
-from tests.parity import route_check
+from tests.parity import W_REL, route_check
 
 pytestmark = pytest.mark.gpu
 
@@ -70,3 +70,30 @@ def test_route_rejects_bad_shapes():
     with pytest.raises(moe.MoEError) as e:
         moe.route(x, wr, 9)
     assert e.value.status == moe.MOE_ERR_UNSUPPORTED_SHAPE
+
+
+RENORM = [SMALL[0], SMALL[4], SMALL[5], SMALL[6]]   # group top-k, whole-warp top-k (k = 32), k = E, bias
+
+
+@pytest.mark.parametrize("cfg", RENORM, ids=lambda c: c.name)
+def test_route_renormalized(cfg):
+    """MOE_FLAG_RENORMALIZE: the same ids; each weight is the oracle's
+    probability divided by the sum over the token's selected experts."""
+    d = gc.on_device(gc.inputs(cfg))
+    ids_t, w_t = moe.route(d["x"], d["w_router"], cfg.k, bias=d["bias"], renormalize=True)
+    ids_p, _ = moe.route(d["x"], d["w_router"], cfg.k, bias=d["bias"])
+    torch.cuda.synchronize()
+    assert moe.get_status() == moe.MOE_OK
+    assert torch.equal(ids_t, ids_p)
+    ids, w = ids_t.cpu().numpy(), w_t.cpu().numpy().astype(np.float64)
+    r = gc.oracle_route(cfg)
+    p_sel = np.take_along_axis(r.probs, ids.astype(np.int64), axis=1)
+    want = p_sel / p_sel.sum(axis=1, keepdims=True)
+    worst = float(np.max(np.abs(w - want) / want))
+    assert worst <= W_REL, f"renormalised weight relative error {worst:.3e}"
+    np.testing.assert_allclose(w.sum(axis=1), 1.0, rtol=0, atol=k_sum_tol(cfg.k))
+
+
+def k_sum_tol(k):
+    """fp32 sum of k weights that each carry relative error <= W_REL."""
+    return k * W_REL

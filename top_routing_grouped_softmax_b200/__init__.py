@@ -38,7 +38,7 @@ ABI_SYMBOLS = (
     "moe_strerror", "moe_version", "moe_workspace_size", "moe_route_workspace_size",
     "moe_permute_workspace_size", "moe_route", "moe_permute", "moe_expert_ffn", "moe_combine", "moe_forward",
     "moe_forward_ex", "moe_get_status", "moe_set_wait_limit_ns", "moe_selftest_wait_timeout",
-    "moe_permute_static",
+    "moe_permute_static", "moe_route_ex",
 )
 
 
@@ -75,6 +75,7 @@ def lib() -> ctypes.CDLL:
         L.moe_permute_workspace_size.restype = _SZ
         L.moe_permute_workspace_size.argtypes = [_I64] * 3
         L.moe_route.argtypes = [_P, _P, _P, _I64, _I64, _I64, _I64, _P, _P, _P, _SZ, _P]
+        L.moe_route_ex.argtypes = [_P, _P, _P, _I64, _I64, _I64, _I64, _P, _P, _P, _SZ, _P, ctypes.c_uint]
         L.moe_permute.argtypes = [_P, _P, _P, _I64, _I64, _I64, _I64, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]
         L.moe_permute_static.argtypes = [_P, _P, _P, _I64, _I64, _I64, _I64, _P, _P, _P, _P, _P, _P, _P]
         L.moe_expert_ffn.argtypes = [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _P, _P, _P]
@@ -86,7 +87,7 @@ def lib() -> ctypes.CDLL:
         L.moe_selftest_wait_timeout.argtypes = [_I64, _P]
         for name in ("moe_route", "moe_permute", "moe_expert_ffn", "moe_combine", "moe_forward",
                      "moe_forward_ex", "moe_get_status", "moe_set_wait_limit_ns",
-                     "moe_selftest_wait_timeout", "moe_permute_static"):
+                     "moe_selftest_wait_timeout", "moe_permute_static", "moe_route_ex"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -144,8 +145,11 @@ def _workspace(nbytes: int, device) -> torch.Tensor:
 
 
 # ----------------------------------------------------------------- stages
-def route(x, w_router, k, bias=None, topk_ids=None, topk_w=None, workspace=None):
-    """Router GEMM + fp32 softmax + top-k; returns (topk_ids int32 [T,k], topk_w fp32 [T,k])."""
+def route(x, w_router, k, bias=None, topk_ids=None, topk_w=None, workspace=None, renormalize=False):
+    """Router GEMM + fp32 softmax + top-k; returns (topk_ids int32 [T,k], topk_w fp32 [T,k]).
+
+    ``renormalize``: divide each token's k weights by their sum
+    (MOE_FLAG_RENORMALIZE); by default they are the softmax probabilities."""
     _need(x, "x", torch.bfloat16, 2)
     _need(w_router, "w_router", torch.bfloat16, 2)
     T, d = x.shape
@@ -160,8 +164,9 @@ def route(x, w_router, k, bias=None, topk_ids=None, topk_w=None, workspace=None)
     if need > 0 and (workspace is None or workspace.numel() < need):
         workspace = _workspace(need, x.device)
     ws_bytes = 0 if workspace is None else workspace.numel()
-    _check(lib().moe_route(_ptr(x), _ptr(w_router), _ptr(bias), T, d, E, k, _ptr(topk_ids),
-                           _ptr(topk_w), _ptr(workspace), ws_bytes, _stream()), "moe_route")
+    flags = MOE_FLAG_RENORMALIZE if renormalize else 0
+    _check(lib().moe_route_ex(_ptr(x), _ptr(w_router), _ptr(bias), T, d, E, k, _ptr(topk_ids),
+                              _ptr(topk_w), _ptr(workspace), ws_bytes, _stream(), flags), "moe_route_ex")
     return topk_ids, topk_w
 
 
@@ -235,6 +240,7 @@ def _forward_args(x, w_router, w_gate, w_up, w_down, bias):
 
 
 MOE_FLAG_FUSED_GATHER = 1
+MOE_FLAG_RENORMALIZE = 2
 
 
 def forward(x, w_router, w_gate, w_up, w_down, k, bias=None, out=None, workspace=None,
@@ -245,7 +251,8 @@ def forward(x, w_router, w_gate, w_up, w_down, k, bias=None, out=None, workspace
     to skip a boundary) recorded at the stage boundaries (before route, after
     route, after permute, after gate/up, after down, after combine).  ``flags`` (optional):
     MOE_FLAG_FUSED_GATHER selects the variant whose gate/up GEMM gathers the
-    rows of x itself; both variants give identical results.
+    rows of x itself (identical results); MOE_FLAG_RENORMALIZE divides each
+    token's k routing weights by their sum.
     """
     T, d, E, f = _forward_args(x, w_router, w_gate, w_up, w_down, bias)
     if out is None:
@@ -292,9 +299,10 @@ def selftest_wait_timeout(limit_ns: int):
 class MoEBlock:
     """Weights of one MoE block on the GPU plus a reusable workspace."""
 
-    def __init__(self, w_router, w_gate, w_up, w_down, k, bias=None):
+    def __init__(self, w_router, w_gate, w_up, w_down, k, bias=None, renormalize=False):
         self.w_router, self.w_gate, self.w_up, self.w_down = w_router, w_gate, w_up, w_down
         self.bias = bias
+        self.renormalize = bool(renormalize)
         self.k = int(k)
         self.E, self.d, self.f = w_gate.shape
         self._ws = None
@@ -306,6 +314,8 @@ class MoEBlock:
         return self._ws
 
     def __call__(self, x, out=None, topk_ids=None, topk_w=None, events=None, flags=None):
+        if self.renormalize:
+            flags = (flags or 0) | MOE_FLAG_RENORMALIZE
         return forward(x, self.w_router, self.w_gate, self.w_up, self.w_down, self.k, bias=self.bias,
                        out=out, workspace=self.workspace(x.shape[0]), topk_ids=topk_ids, topk_w=topk_w,
                        events=events, flags=flags)
@@ -313,7 +323,7 @@ class MoEBlock:
 
 __all__ = [
     "lib", "strerror", "MoEError", "ABI_SYMBOLS", "workspace_size", "route_workspace_size",
-    "permute_workspace_size", "MOE_FLAG_FUSED_GATHER", "route",
+    "permute_workspace_size", "MOE_FLAG_FUSED_GATHER", "MOE_FLAG_RENORMALIZE", "route",
     "permute", "expert_ffn", "combine", "forward", "get_status", "set_wait_limit_ns",
     "selftest_wait_timeout", "MoEBlock",
 ]

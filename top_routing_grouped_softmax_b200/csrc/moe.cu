@@ -271,7 +271,8 @@ int launch_route(const CUtensorMap& tx, const CUtensorMap& tw, moe::route::Param
 }
 
 int run_route(const DeviceState& st, const moe_bf16* x, const moe_bf16* w_router, const float* bias, int64_t T,
-              int64_t d, int64_t E, int64_t k, int32_t* ids, float* wts, int32_t* chunk_counts, cudaStream_t s)
+              int64_t d, int64_t E, int64_t k, int32_t* ids, float* wts, int32_t* chunk_counts, bool renorm,
+              cudaStream_t s)
 {
     if (T == 0) return MOE_OK;
     CUtensorMap tx, tw;
@@ -301,6 +302,7 @@ int run_route(const DeviceState& st, const moe_bf16* x, const moe_bf16* w_router
     const int64_t pairs = st.max_pairs > 0 ? st.max_pairs : st.sm_count / 2;
     p.split = (E <= 256 && d >= 2 * moe::route::kBK && tiles <= pairs) ? 2 : 1;
     p.passes = (p.split == 1 && E > 256) ? 2 : 1;
+    p.renorm = renorm ? 1 : 0;
     // top-k list length: the power of two >= k for lane groups (k <= 8), or
     // the whole-warp rounds (k > 8)
     const unsigned ut = (unsigned)tiles;
@@ -440,7 +442,7 @@ int forward_impl(const moe_bf16* x, const moe_bf16* w_router, const float* bias,
     int rc = check_common(T, d, E, k);
     if (rc) return rc;
     if ((rc = check_f(f))) return rc;
-    if (flags & ~(unsigned)MOE_FLAG_FUSED_GATHER) return MOE_ERR_INVALID_ARG;
+    if (flags & ~(unsigned)(MOE_FLAG_FUSED_GATHER | MOE_FLAG_RENORMALIZE)) return MOE_ERR_INVALID_ARG;
     if (T > 0 && (!x || !w_router || !w_gate || !w_up || !w_down || !out)) return MOE_ERR_INVALID_ARG;
     if (!aligned(x, 16) || !aligned(w_router, 16) || !aligned(w_gate, 16) || !aligned(w_up, 16) ||
         !aligned(w_down, 16) || !aligned(out, 16) || !aligned(bias, 4) || !aligned(ids_out, 4) ||
@@ -475,7 +477,9 @@ int forward_impl(const moe_bf16* x, const moe_bf16* w_router, const float* bias,
     moe_f16* y = reinterpret_cast<moe_f16*>(w + L.y);
     const bool gather = (flags & MOE_FLAG_FUSED_GATHER) != 0;
 
-    if ((rc = run_route(*st, x, w_router, bias, T, d, E, k, ids, wts, chunk, s))) return rc;
+    if ((rc = run_route(*st, x, w_router, bias, T, d, E, k, ids, wts, chunk, (flags & MOE_FLAG_RENORMALIZE) != 0,
+                        s)))
+        return rc;
     if ((rc = rec(1))) return rc;
     if ((rc = run_permute(x, ids, wts, T, d, E, k, counts, offsets, perm, inv, gather ? nullptr : x_perm, w_perm,
                           chunk, true, s)))
@@ -544,7 +548,7 @@ const char* moe_strerror(int status)
     }
 }
 
-int moe_version(void) { return 200; }
+int moe_version(void) { return 201; }
 
 size_t moe_workspace_size(int64_t T, int64_t d, int64_t E, int64_t k, int64_t f)
 {
@@ -568,6 +572,14 @@ int moe_route(const moe_bf16* x, const moe_bf16* w_router, const float* bias, in
               int64_t k, int32_t* topk_ids, float* topk_w, void* workspace, size_t workspace_bytes,
               cudaStream_t stream)
 {
+    return moe_route_ex(x, w_router, bias, T, d, E, k, topk_ids, topk_w, workspace, workspace_bytes, stream, 0u);
+}
+
+int moe_route_ex(const moe_bf16* x, const moe_bf16* w_router, const float* bias, int64_t T, int64_t d, int64_t E,
+                 int64_t k, int32_t* topk_ids, float* topk_w, void* workspace, size_t workspace_bytes,
+                 cudaStream_t stream, unsigned flags)
+{
+    if (flags & ~(unsigned)MOE_FLAG_RENORMALIZE) return MOE_ERR_INVALID_ARG;
     int rc = check_common(T, d, E, k);
     if (rc) return rc;
     if (T > 0 && (!x || !w_router || !topk_ids || !topk_w)) return MOE_ERR_INVALID_ARG;
@@ -577,7 +589,8 @@ int moe_route(const moe_bf16* x, const moe_bf16* w_router, const float* bias, in
     if (workspace_bytes < route_ws_bytes(T, d, E)) return MOE_ERR_WORKSPACE_TOO_SMALL;
     DeviceState* st = nullptr;
     if ((rc = setup_device(&st))) return rc;
-    return run_route(*st, x, w_router, bias, T, d, E, k, topk_ids, topk_w, nullptr, stream);
+    return run_route(*st, x, w_router, bias, T, d, E, k, topk_ids, topk_w, nullptr,
+                     (flags & MOE_FLAG_RENORMALIZE) != 0, stream);
 }
 
 int moe_permute(const moe_bf16* x, const int32_t* topk_ids, const float* topk_w, int64_t T, int64_t d, int64_t E,

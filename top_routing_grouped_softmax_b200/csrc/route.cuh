@@ -33,7 +33,8 @@
 // rank by the (value, index) order -- larger logit first, equal logits rank
 // the lower expert index first -- on fp32 logits (softmax is monotone).
 // Lane j < k of the token's group writes slot j: the expert and its
-// probability exp(l - max) / sum.  The same lanes count their experts into
+// probability exp(l - max) / sum -- or, with renorm, exp(l - max) divided by
+// the sum over the k selected experts only (weights summing to one).  The same lanes count their experts into
 // the tile's 64-token chunk histograms, which the permutation needs and
 // which the CTA writes out whole (expert-major table, no global atomics, no
 // zeroing).
@@ -68,6 +69,7 @@ struct Params {
     uint32_t tmem_cols;      // power of two >= 64 * n_chunks
     int split;               // CTAs per tile: 1, or 2 (cluster of two, split K)
     int passes;              // row passes of the exchange buffer (1, or 2 when split == 1 and E > 256)
+    int renorm;              // 1: divide each token's k weights by their sum
 };
 
 __host__ __device__ inline int stage_bytes(int n_chunks) { return kABytes + n_chunks * kChunkBytes; }
@@ -113,7 +115,7 @@ __device__ __forceinline__ bool ranks_before(float v, int i, float w, int j) { r
 // logit of expert lane + 32 j (called only for lane + 32 j < E).  Lane
 // j < k receives slot j.
 template <int VPL, typename Logit>
-__device__ __forceinline__ void warp_topk(int E, int k, int lane, Logit col, int& my_id, float& my_w)
+__device__ __forceinline__ void warp_topk(int E, int k, bool renorm, int lane, Logit col, int& my_id, float& my_w)
 {
     float v[VPL];
     unsigned taken = 0;  // bit j: value j is not a candidate
@@ -165,9 +167,16 @@ __device__ __forceinline__ void warp_topk(int E, int k, int lane, Logit col, int
         if ((bi & 31) == lane) taken |= 1u << ((bi >> 5) & 31);
         if (lane == slot) {
             my_id = bi;
-            my_w = expf(bv - mx) / sum;
+            my_w = expf(bv - mx);
         }
     }
+    if (renorm) {
+        // the selected terms only (lanes >= k hold 0), in a fixed order
+        sum = my_w;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    }
+    my_w /= sum;
 }
 
 // Insert (x, col) into a list sorted by the (value, index) order, dropping
@@ -234,7 +243,7 @@ __device__ __forceinline__ void merge_partner(float (&v)[KMAX], int (&ix)[KMAX],
 // Softmax and top-k of one token by a group of L lanes (lane j of the group
 // = lane % L); `logit(c)` is expert c's logit.  Lane j < k receives slot j.
 template <int L, int KMAX, typename Logit>
-__device__ __forceinline__ void group_topk(int E, int j, Logit logit, int& my_id, float& my_w)
+__device__ __forceinline__ void group_topk(int E, int k, bool renorm, int j, Logit logit, int& my_id, float& my_w)
 {
     float v[KMAX];
     int ix[KMAX];
@@ -265,6 +274,13 @@ __device__ __forceinline__ void group_topk(int E, int j, Logit logit, int& my_id
             my_id = ix[m];
             w = v[m];
         }
+    if (renorm) {
+        // every lane of the group holds the same sorted list: the same sum
+        sum = 0.0f;
+#pragma unroll
+        for (int m = 0; m < KMAX; ++m)
+            if (m < k) sum += __expf(v[m] - mx);
+    }
     my_w = __expf(w - mx) / sum;
 }
 
@@ -282,7 +298,7 @@ __device__ __forceinline__ void topk_rows(const Params& p, const float* buf, con
         const int64_t t = (int64_t)tile0 + row0 + i;
         int my_id;
         float my_w;
-        group_topk<L, KMAX>(E, j, [&](int c) {
+        group_topk<L, KMAX>(E, p.k, p.renorm != 0, j, [&](int c) {
             const float* col = buf + (size_t)c * pitch + i;
             float l = col[0];
             for (int s = 1; s < S; ++s) l += col[(size_t)s * E * pitch];
@@ -477,7 +493,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (t >= p.T) break;  // warp-uniform; later rows are past the end too
                 int my_id;
                 float my_w;
-                warp_topk<16>(E, p.k, lane, [&](int jj) {
+                warp_topk<16>(E, p.k, p.renorm != 0, lane, [&](int jj) {
                     const int c = lane + 32 * jj;
                     const float* col = buf + (size_t)c * pitch + i;
                     float l = col[0];
