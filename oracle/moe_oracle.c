@@ -264,3 +264,43 @@ int oracle_expert_rows(const uint16_t* x, const uint16_t* w_gate, const uint16_t
     free(xrow); free(g); free(u); free(h); free(o);
     return status;
 }
+
+/*
+ * Optional variant: shared experts, SwiGLU experts that every token passes
+ * through with weight one, on top of its k routed experts (the "shared
+ * expert" routing of the Hunyuan-Large overview page, section 2.1; the page
+ * gives no formula, so the reading is: out[t] += sum_s shared_s(x[t])).
+ *   w_gate_s, w_up_s [n_s][d][f_s], w_down_s [n_s][f_s][d]
+ *   out [n_rows][d]  in/out: out[r] += sum_{s ascending} shared_s(x[rows[r]])
+ *                    (call after oracle_expert_rows on the same rows)
+ */
+int oracle_shared_rows(const uint16_t* x, const uint16_t* w_gate_s, const uint16_t* w_up_s,
+                       const uint16_t* w_down_s, int64_t T, int64_t d, int64_t n_s, int64_t f_s,
+                       int64_t n_rows, const int64_t* rows, double* out)
+{
+    if (!x || !w_gate_s || !w_up_s || !w_down_s || !rows || !out || T < 0 || d < 1 || n_s < 1 ||
+        f_s < 1 || n_rows < 0)
+        return ORACLE_BAD_ARG;
+    double* xrow = (double*)malloc(sizeof(double) * d);
+    double* g = (double*)malloc(sizeof(double) * f_s);
+    double* u = (double*)malloc(sizeof(double) * f_s);
+    double* h = (double*)malloc(sizeof(double) * f_s);
+    double* o = (double*)malloc(sizeof(double) * d);
+    if (!xrow || !g || !u || !h || !o) {
+        free(xrow); free(g); free(u); free(h); free(o);
+        return ORACLE_NO_MEMORY;
+    }
+    int status = ORACLE_OK;
+    for (int64_t r = 0; r < n_rows; ++r) {
+        const int64_t t = rows[r];
+        if (t < 0 || t >= T) { status = ORACLE_BAD_ARG; break; }
+        for (int64_t i = 0; i < d; ++i) xrow[i] = bf16_to_double(x[t * d + i]);
+        for (int64_t sidx = 0; sidx < n_s; ++sidx) {
+            expert_swiglu(xrow, w_gate_s + sidx * d * f_s, w_up_s + sidx * d * f_s,
+                          w_down_s + sidx * f_s * d, d, f_s, g, u, h, o);
+            for (int64_t c = 0; c < d; ++c) out[r * d + c] += o[c];
+        }
+    }
+    free(xrow); free(g); free(u); free(h); free(o);
+    return status;
+}

@@ -63,6 +63,8 @@ class Oracle:
         lib.oracle_expert_rows.argtypes = [_P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64,
                                            _P, _P, _I64, _P, _P, _P, _P]
         lib.oracle_renormalize.argtypes = [_P, _I64, _I64]
+        lib.oracle_shared_rows.argtypes = [_P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64, _P, _P]
+        lib.oracle_shared_rows.restype = ctypes.c_int
         for fn in (lib.oracle_route, lib.oracle_permute, lib.oracle_expert_rows, lib.oracle_renormalize):
             fn.restype = ctypes.c_int
         self.lib = lib
@@ -127,15 +129,36 @@ class Oracle:
             raise ValueError(f"oracle_expert_rows failed ({rc})")
         return ExpertResult(out=out, y=y, h=h)
 
+    # -- shared experts -------------------------------------------------------
+    def shared_rows(self, x, w_gate_s, w_up_s, w_down_s, rows, out):
+        """out + sum over shared experts s of SwiGLU_s(x[rows]) (a new array)."""
+        x = np.ascontiguousarray(x, dtype=np.uint16)
+        w_gate_s = np.ascontiguousarray(w_gate_s, dtype=np.uint16)
+        w_up_s = np.ascontiguousarray(w_up_s, dtype=np.uint16)
+        w_down_s = np.ascontiguousarray(w_down_s, dtype=np.uint16)
+        rows = np.ascontiguousarray(rows, dtype=np.int64)
+        res = np.array(out, dtype=np.float64, copy=True, order="C")
+        T, d = x.shape
+        n_s, _, f_s = w_gate_s.shape
+        rc = self.lib.oracle_shared_rows(_ptr(x), _ptr(w_gate_s), _ptr(w_up_s), _ptr(w_down_s), T, d, n_s, f_s,
+                                         rows.shape[0], _ptr(rows), _ptr(res))
+        if rc != 0:
+            raise ValueError(f"oracle_shared_rows failed ({rc})")
+        return res
+
     # -- whole block ----------------------------------------------------------
     def forward(self, x, w_router, bias, w_gate, w_up, w_down, k, rows=None,
-                want_y=False, want_h=False, renormalize=False):
-        """Route every token; evaluate the expert MLPs for ``rows`` (all if None)."""
+                want_y=False, want_h=False, renormalize=False, shared=None):
+        """Route every token; evaluate the expert MLPs for ``rows`` (all if
+        None).  ``shared``: optional (W_gate_s, W_up_s, W_down_s) bit arrays of
+        shared experts, added to ``out`` with weight one."""
         r = self.route(x, w_router, bias, k, renormalize=renormalize)
         if rows is None:
             rows = np.arange(x.shape[0], dtype=np.int64)
         ex = self.expert_rows(x, w_gate, w_up, w_down, r.ids, r.weights, rows,
                               want_y=want_y, want_h=want_h)
+        if shared is not None:
+            ex = ExpertResult(out=self.shared_rows(x, *shared, rows, ex.out), y=ex.y, h=ex.h)
         return r, ex
 
 

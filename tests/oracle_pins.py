@@ -285,9 +285,32 @@ def check_renormalize(o):
     np.testing.assert_allclose(full.weights, o.route(x, wr, b, 16).weights, rtol=1e-14, atol=0)
 
 
+def check_shared_experts(o):
+    """Shared experts: the oracle's output equals the dense brute force plus
+    every shared SwiGLU evaluated densely with numpy matmuls (weight one);
+    zero shared down-projections leave the output bit-identical."""
+    from top_routing_grouped_softmax_b200.synth import MoEConfig, make_shared_weights
+    inp = _rand_case(40, 64, 8, 2, 32, seed=41, bias=True)
+    sw = make_shared_weights(MoEConfig("pin", T=40, d=64, E=8, k=2, f=32, sigma=0.05, seed=41), 2, 48)
+    shared = tuple(bf16_bits(sw[n]) for n in ("W_gate_s", "W_up_s", "W_down_s"))
+    x = inp.bits("x")
+    _, ex = o.forward(*_args(inp), 2, shared=shared)
+    ref, _, _, _ = dense_reference(*_args(inp), 2)
+    X = widen(x)
+    for s_idx in range(2):
+        G = X @ widen(shared[0][s_idx])
+        U = X @ widen(shared[1][s_idx])
+        ref = ref + (G * sps.expit(G) * U) @ widen(shared[2][s_idx])
+    assert _rel(ex.out, ref) < 1e-12, _rel(ex.out, ref)
+    zero = (shared[0], shared[1], np.zeros_like(shared[2]))
+    _, ex0 = o.forward(*_args(inp), 2, shared=zero)
+    _, plain = o.forward(*_args(inp), 2)
+    assert np.array_equal(ex0.out, plain.out)
+
+
 ALL_CHECKS = [
     check_brute_force, check_softmax_library, check_topk_library_sort, check_topk_of_logits,
     check_exact_ties, check_dense_special_case, check_all_experts_identical, check_zero_expert,
     check_scale_down, check_permute_library, check_page_listing_torch, check_expert_rows_outputs,
-    check_renormalize,
+    check_renormalize, check_shared_experts,
 ]

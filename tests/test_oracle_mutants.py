@@ -29,6 +29,10 @@ MUTANTS = [
     ("weights_from_wrong_slot", "weights[t * k + j] = ranked[j].p;", "weights[t * k + j] = ranked[0].p;"),
     ("sum_only_first_slot", "orow[c] += yc;", "orow[c] += (j == 0) ? yc : 0.0;"),
     ("renorm_no_divide", "weights[t * k + j] /= s;", "weights[t * k + j] /= 1.0;"),
+    ("shared_first_only", "for (int64_t sidx = 0; sidx < n_s; ++sidx) {",
+     "for (int64_t sidx = 0; sidx < 1; ++sidx) {"),
+    ("shared_half_weight", "for (int64_t c = 0; c < d; ++c) out[r * d + c] += o[c];",
+     "for (int64_t c = 0; c < d; ++c) out[r * d + c] += 0.5 * o[c];"),
     ("renorm_partial_sum", "for (int64_t j = 0; j < k; ++j) s += weights[t * k + j];",
      "for (int64_t j = 0; j + 1 < k; ++j) s += weights[t * k + j];"),
 ]

@@ -137,6 +137,29 @@ def make_inputs(cfg: MoEConfig | str, **overrides) -> MoEInputs:
     return MoEInputs(cfg, x, W_router, W_gate, W_up, W_down, bias)
 
 
+def make_shared_weights(cfg: MoEConfig, n_shared: int, f_shared: int | None = None) -> dict:
+    """Weights of ``n_shared`` shared experts (every token passes through
+    them with weight one): bf16 W_gate_s, W_up_s [n_shared, d, f_s] and
+    W_down_s [n_shared, f_s, d], f_s = f_shared or cfg.f.  Drawn like the
+    routed experts (fp32 randn * sigma, rounded to bf16; gate of every
+    shared expert, then up, then down) from their own generator seeded with
+    seed + 100000, so adding shared experts leaves the other inputs of the
+    workload unchanged."""
+    fs = cfg.f if f_shared is None else f_shared
+    gen = torch.Generator(device="cpu")
+    gen.manual_seed(cfg.seed + 100000)
+    W_gate_s = torch.empty(n_shared, cfg.d, fs, dtype=torch.bfloat16)
+    W_up_s = torch.empty(n_shared, cfg.d, fs, dtype=torch.bfloat16)
+    W_down_s = torch.empty(n_shared, fs, cfg.d, dtype=torch.bfloat16)
+    for s in range(n_shared):
+        W_gate_s[s] = _randn_bf16(gen, (cfg.d, fs), cfg.sigma)
+    for s in range(n_shared):
+        W_up_s[s] = _randn_bf16(gen, (cfg.d, fs), cfg.sigma)
+    for s in range(n_shared):
+        W_down_s[s] = _randn_bf16(gen, (fs, cfg.d), cfg.sigma)
+    return {"W_gate_s": W_gate_s, "W_up_s": W_up_s, "W_down_s": W_down_s}
+
+
 def sample_tokens(T: int, n: int, seed: int, must_include=()) -> np.ndarray:
     """A seeded, sorted, duplicate-free sample of n token indices in [0, T).
 
@@ -157,5 +180,5 @@ def sample_tokens(T: int, n: int, seed: int, must_include=()) -> np.ndarray:
 
 __all__ = [
     "MoEConfig", "MoEInputs", "CONFIGS", "make_inputs", "bf16_bits", "bits_to_bf16",
-    "zipf_bias", "sample_tokens",
+    "zipf_bias", "sample_tokens", "make_shared_weights",
 ]
