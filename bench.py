@@ -73,15 +73,17 @@ def load_peaks():
     return dict(FALLBACK_PEAKS, source="fallback")
 
 
-def algorithmic(cfg, active_experts=None):
-    """FLOPs and compulsory HBM bytes of one forward, and of its gate/up GEMM."""
+def algorithmic(cfg, active_experts=None, n_shared=0):
+    """FLOPs and compulsory HBM bytes of one forward, and of its gate/up GEMM
+    (n_shared shared experts of size f add 2*T*3*d*f FLOPs and their weights
+    each)."""
     T, d, E, k, f = cfg.T, cfg.d, cfg.E, cfg.k, cfg.f
-    flops = 2 * T * (d * E + 3 * k * d * f)
+    flops = 2 * T * (d * E + 3 * k * d * f) + n_shared * 2 * T * 3 * d * f
     gateup_flops = 2 * T * k * d * 2 * f
     down_flops = 2 * T * k * f * d
     nact = E if active_experts is None else active_experts
     # x read + out write (fp32) + router weights + weights of the experts in use
-    compulsory = T * d * 2 + T * d * 4 + d * E * 2 + nact * 3 * d * f * 2
+    compulsory = T * d * 2 + T * d * 4 + d * E * 2 + (nact + n_shared) * 3 * d * f * 2
     # per-stage algorithmic HBM bytes: route reads x and W_router and writes
     # ids + weights; permute reads x and writes x_perm (+ 12 B per
     # assignment of indices and weights); combine reads y (fp16), writes out
@@ -295,11 +297,30 @@ def run_gpu(args, cfg):
             moe.combine(y_, pm["inv"], cfg.T, cfg.k, out=out)
             rec(5)
             ids.copy_(st_ids)
+
+        def fwd(xin, events=None, topk_ids=None):  # e2e leg: the public fused call
+            blk(xin, out=out, topk_ids=topk_ids, events=events)
     else:
         flags = moe.MOE_FLAG_FUSED_GATHER if args.gather else 0
+        if args.shared > 0:
+            from top_routing_grouped_softmax_b200.synth import make_shared_weights
+            sw = {n: t.to(dev) for n, t in make_shared_weights(cfg, args.shared).items()}
+            ws_sh = None
+
+            def fwd(xin, events=None, topk_ids=None):
+                nonlocal ws_sh
+                if ws_sh is None:
+                    nb = moe.lib().moe_workspace_size_shared(cfg.T, cfg.d, cfg.E, cfg.k, cfg.f, args.shared, cfg.f)
+                    ws_sh = torch.empty(int(nb), dtype=torch.uint8, device=dev)
+                moe.forward_shared(xin, w["W_router"], w["W_gate"], w["W_up"], w["W_down"], sw["W_gate_s"],
+                                   sw["W_up_s"], sw["W_down_s"], cfg.k, bias=bias, out=out, workspace=ws_sh,
+                                   topk_ids=topk_ids, events=events, flags=flags)
+        else:
+            def fwd(xin, events=None, topk_ids=None):
+                blk(xin, out=out, topk_ids=topk_ids, events=events, flags=flags)
 
         def step(events=None):
-            blk(x, out=out, topk_ids=ids, events=events, flags=flags)
+            fwd(x, events, ids)
 
     for _ in range(args.warmup):
         step()
@@ -355,7 +376,7 @@ def run_gpu(args, cfg):
     e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     for _ in range(2):
         x_dev.copy_(x_host, non_blocking=True)
-        blk(x_dev, out=out)
+        fwd(x_dev)
         out_host.copy_(out, non_blocking=True)
     torch.cuda.synchronize()
     if world > 1:
@@ -364,7 +385,7 @@ def run_gpu(args, cfg):
         flush.zero_()
         e2e_ev[i][0].record(stream)
         x_dev.copy_(x_host, non_blocking=True)
-        blk(x_dev, out=out)
+        fwd(x_dev)
         out_host.copy_(out, non_blocking=True)
         e2e_ev[i][1].record(stream)
     torch.cuda.synchronize()
@@ -383,7 +404,7 @@ def run_gpu(args, cfg):
     result = None
     if rank == 0:
         peaks = load_peaks()
-        alg = algorithmic(cfg, active)
+        alg = algorithmic(cfg, active, args.shared)
         ms = 1e3 * total_s / args.steps
         tok_s = whole_job_rate(cfg.T * args.steps, world, [total_s])
         # --path stages times both GEMMs together (moe_expert_ffn is one call)
@@ -403,7 +424,9 @@ def run_gpu(args, cfg):
             "metric": METRIC, "value": tok_s, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": workload_config(cfg, extra={"out_dtype": "fp32"}),
+            "config": workload_config(cfg, extra={"out_dtype": "fp32", **({"shared_experts": args.shared,
+                                                                             "f_shared": cfg.f}
+                                                                          if args.shared else {})}),
             "tflops": alg["flops"] / (ms * 1e-3) / 1e12,
             "grouped_gemm_tflops": (alg["gateup_flops"] + alg["down_flops"]) /
                                    ((stage_ms["gateup_gemm"] + stage_ms["down_gemm"]) * 1e-3) / 1e12,
@@ -428,7 +451,7 @@ def run_gpu(args, cfg):
                         "pair_tile_padding": padding},
             "e2e": {"value": whole_job_rate(cfg.T * args.steps, world, [e2e_s]), "unit": UNIT,
                     "h2d_bytes_per_step": cfg.T * cfg.d * 2, "d2h_bytes_per_step": cfg.T * cfg.d * 4},
-            "gpu_launches": KERNELS_PER_FORWARD * args.steps,
+            "gpu_launches": (KERNELS_PER_FORWARD + 2 * args.shared) * args.steps,
             "clocks": clocks,
             "wall_s_timed_region": wall,
         }
@@ -446,6 +469,8 @@ def main(argv=None):
     ap.add_argument("--workload", default="qwen")
     ap.add_argument("--path", choices=("fused", "stages"), default="fused",
                     help="fused: moe_forward; stages: moe_route/permute/expert_ffn/combine one by one")
+    ap.add_argument("--shared", type=int, default=0,
+                    help="add this many shared experts (weight one, every token, intermediate size f)")
     ap.add_argument("--gather", action="store_true",
                     help="fused path: the gate/up GEMM gathers x rows itself (MOE_FLAG_FUSED_GATHER)")
     ap.add_argument("--cpu-tokens", type=int, default=384,

@@ -267,6 +267,49 @@ int moe_forward_ex(const moe_bf16* x, const moe_bf16* w_router, const float* bia
                    cudaEvent_t* events, int n_events, unsigned flags);
 
 /*
+ * Shared experts (optional; not in the article's block).  n_shared SwiGLU
+ * experts that every token passes through with weight one, on top of its k
+ * routed experts -- the "shared expert" routing of the Hunyuan-Large
+ * overview page, section 2.1:
+ *   out[t] = sum_j y[t,j] + sum_{s = 0..n_shared-1} down_s(silu(gate_s x[t]) * up_s x[t])
+ * with the shared sum added after the routed slots, in ascending s, in fp32.
+ *   w_gate_s, w_up_s [n_shared, d, f_shared] bf16;  w_down_s [n_shared, f_shared, d] bf16
+ *   1 <= n_shared <= 8; f_shared follows the rules for f.
+ * Each shared expert runs through the same grouped GEMMs as one group of all
+ * T rows of x (no permutation).
+ */
+
+/* Bytes of scratch for moe_forward_shared (0 if a shape is unsupported). */
+size_t moe_workspace_size_shared(int64_t T, int64_t d, int64_t E, int64_t k, int64_t f,
+                                 int64_t n_shared, int64_t f_shared);
+
+/* Stage: y_s[s][t] = down_s(silu(gate_s x[t]) * up_s x[t]) for every shared
+ * expert s, stored fp16 (range errors as for y).  h_s [T, f_shared] bf16 is
+ * the caller's scratch; y_s is [n_shared, T, d] fp16. */
+int moe_shared_ffn(const moe_bf16* x, const moe_bf16* w_gate_s, const moe_bf16* w_up_s,
+                   const moe_bf16* w_down_s, int64_t T, int64_t d, int64_t n_shared, int64_t f_shared,
+                   moe_bf16* h_s, moe_f16* y_s, cudaStream_t stream);
+
+/* Stage: moe_combine plus the shared rows: out[t] = sum_j y[inv[t*k+j]] +
+ * sum_s y_s[s][t] (fp32, routed slots first, then ascending s).
+ * n_shared = 0 is moe_combine (y_s may then be NULL). */
+int moe_combine_shared(const moe_f16* y, const int32_t* inv, const moe_f16* y_s, int64_t n_shared,
+                       int64_t T, int64_t d, int64_t k, float* out, cudaStream_t stream);
+
+/* The whole block with shared experts: moe_forward_ex's stages, with the
+ * shared GEMMs after the routed down GEMM (inside the "after down" event)
+ * and moe_combine_shared; workspace of moe_workspace_size_shared bytes.
+ * events and flags as for moe_forward_ex. */
+int moe_forward_shared(const moe_bf16* x, const moe_bf16* w_router, const float* bias,
+                       const moe_bf16* w_gate, const moe_bf16* w_up, const moe_bf16* w_down,
+                       const moe_bf16* w_gate_s, const moe_bf16* w_up_s, const moe_bf16* w_down_s,
+                       int64_t T, int64_t d, int64_t E, int64_t k, int64_t f,
+                       int64_t n_shared, int64_t f_shared,
+                       float* out, int32_t* topk_ids_out, float* topk_w_out,
+                       void* workspace, size_t workspace_bytes, cudaStream_t stream,
+                       cudaEvent_t* events, int n_events, unsigned flags);
+
+/*
  * Synchronises `stream`, then returns and clears the current device's status
  * word (MOE_OK if no device-side error was recorded since the last call).
  */

@@ -34,7 +34,7 @@ def test_library_exports_every_declared_symbol(moe_lib):
 
 
 def test_strerror_and_version(moe_lib):
-    assert moe_lib.moe_version() == 201
+    assert moe_lib.moe_version() == 202
     for code in range(10):
         assert moe.strerror(code).startswith("MOE_")
 
@@ -93,3 +93,20 @@ def test_product_never_touches_the_oracle():
                 text = open(os.path.join(dirpath, fn)).read()
                 assert "import oracle" not in text and "from oracle" not in text, fn
                 assert "moe_oracle" not in text and "liboracle" not in text, fn
+
+
+def test_shared_expert_validation(moe_lib):
+    """Shared-expert entry points reject bad counts and sizes on the host."""
+    L = moe_lib
+    null = ctypes.c_void_p(0)
+    assert moe.lib().moe_workspace_size_shared(8192, 2048, 128, 8, 768, 1, 768) > \
+        moe.workspace_size(8192, 2048, 128, 8, 768)
+    assert L.moe_workspace_size_shared(8192, 2048, 128, 8, 768, 9, 768) == 0     # more than 8 shared experts
+    assert L.moe_workspace_size_shared(8192, 2048, 128, 8, 768, 1, 700) == 0     # f_shared % 64 != 0
+    fake = ctypes.c_void_p(0x10000)
+    args = [fake] * 9 + [16, 64, 8, 2, 64]
+    assert L.moe_forward_shared(*args, 0, 64, fake, null, null, fake, 1 << 30, null, null, 0, 0) == \
+        moe.MOE_ERR_INVALID_ARG                                                    # n_shared = 0
+    assert L.moe_forward_shared(*args, 9, 64, fake, null, null, fake, 1 << 30, null, null, 0, 0) == \
+        moe.MOE_ERR_UNSUPPORTED_SHAPE
+    assert L.moe_combine_shared(fake, fake, null, 1, 4, 64, 2, fake, null) == moe.MOE_ERR_INVALID_ARG

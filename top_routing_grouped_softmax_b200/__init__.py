@@ -38,7 +38,8 @@ ABI_SYMBOLS = (
     "moe_strerror", "moe_version", "moe_workspace_size", "moe_route_workspace_size",
     "moe_permute_workspace_size", "moe_route", "moe_permute", "moe_expert_ffn", "moe_combine", "moe_forward",
     "moe_forward_ex", "moe_get_status", "moe_set_wait_limit_ns", "moe_selftest_wait_timeout",
-    "moe_permute_static", "moe_route_ex",
+    "moe_permute_static", "moe_route_ex", "moe_workspace_size_shared", "moe_shared_ffn", "moe_combine_shared",
+    "moe_forward_shared",
 )
 
 
@@ -82,12 +83,19 @@ def lib() -> ctypes.CDLL:
         L.moe_combine.argtypes = [_P, _P, _I64, _I64, _I64, _P, _P]
         L.moe_forward.argtypes = [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64, _P, _P, _P, _P, _SZ, _P]
         L.moe_forward_ex.argtypes = L.moe_forward.argtypes + [_P, ctypes.c_int, ctypes.c_uint]
+        L.moe_workspace_size_shared.restype = _SZ
+        L.moe_workspace_size_shared.argtypes = [_I64] * 7
+        L.moe_shared_ffn.argtypes = [_P, _P, _P, _P, _I64, _I64, _I64, _I64, _P, _P, _P]
+        L.moe_combine_shared.argtypes = [_P, _P, _P, _I64, _I64, _I64, _I64, _P, _P]
+        L.moe_forward_shared.argtypes = ([_P] * 9 + [_I64] * 7 + [_P, _P, _P, _P, _SZ, _P, _P, ctypes.c_int,
+                                                                   ctypes.c_uint])
         L.moe_get_status.argtypes = [_P]
         L.moe_set_wait_limit_ns.argtypes = [_I64]
         L.moe_selftest_wait_timeout.argtypes = [_I64, _P]
         for name in ("moe_route", "moe_permute", "moe_expert_ffn", "moe_combine", "moe_forward",
                      "moe_forward_ex", "moe_get_status", "moe_set_wait_limit_ns",
-                     "moe_selftest_wait_timeout", "moe_permute_static", "moe_route_ex"):
+                     "moe_selftest_wait_timeout", "moe_permute_static", "moe_route_ex", "moe_shared_ffn",
+                     "moe_combine_shared", "moe_forward_shared"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -215,6 +223,60 @@ def expert_ffn(x_perm, w_perm, offsets, w_gate, w_up, w_down, h=None, y=None):
     return h, y
 
 
+def shared_ffn(x, w_gate_s, w_up_s, w_down_s, h_s=None, y_s=None):
+    """Shared experts on every token; returns (h_s bf16 [T, f_s] scratch, y_s fp16 [n_s, T, d])."""
+    _need(x, "x", torch.bfloat16, 2)
+    for n, t in (("w_gate_s", w_gate_s), ("w_up_s", w_up_s), ("w_down_s", w_down_s)):
+        _need(t, n, torch.bfloat16, 3)
+    T, d = x.shape
+    n_s, _, f_s = w_gate_s.shape
+    if h_s is None:
+        h_s = torch.empty(T, f_s, dtype=torch.bfloat16, device=x.device)
+    if y_s is None:
+        y_s = torch.empty(n_s, T, d, dtype=torch.float16, device=x.device)
+    _need(y_s, "y_s", torch.float16, 3)
+    _check(lib().moe_shared_ffn(_ptr(x), _ptr(w_gate_s), _ptr(w_up_s), _ptr(w_down_s), T, d, n_s, f_s, _ptr(h_s),
+                                _ptr(y_s), _stream()), "moe_shared_ffn")
+    return h_s, y_s
+
+
+def combine_shared(y, inv, y_s, T, k, out=None):
+    """out[t] = sum_j y[inv[t*k+j]] + sum_s y_s[s, t] (fp32 sum: routed slots, then ascending s)."""
+    _need(y, "y", torch.float16, 2)
+    _need(inv, "inv", torch.int32, 1)
+    _need(y_s, "y_s", torch.float16, 3)
+    d = y.shape[1]
+    if out is None:
+        out = torch.empty(T, d, dtype=torch.float32, device=y.device)
+    _need(out, "out", torch.float32, 2)
+    _check(lib().moe_combine_shared(_ptr(y), _ptr(inv), _ptr(y_s), y_s.shape[0], T, d, k, _ptr(out), _stream()),
+           "moe_combine_shared")
+    return out
+
+
+def forward_shared(x, w_router, w_gate, w_up, w_down, w_gate_s, w_up_s, w_down_s, k, bias=None, out=None,
+                   workspace=None, topk_ids=None, topk_w=None, events=None, flags=0):
+    """The MoE block plus shared experts (weight one on every token); returns out [T, d] fp32."""
+    T, d, E, f = _forward_args(x, w_router, w_gate, w_up, w_down, bias)
+    for n, t in (("w_gate_s", w_gate_s), ("w_up_s", w_up_s), ("w_down_s", w_down_s)):
+        _need(t, n, torch.bfloat16, 3)
+    n_s, _, f_s = w_gate_s.shape
+    if out is None:
+        out = torch.empty(T, d, dtype=torch.float32, device=x.device)
+    _need(out, "out", torch.float32, 2)
+    nbytes = int(lib().moe_workspace_size_shared(T, d, E, k, f, n_s, f_s))
+    if nbytes == 0:
+        raise MoEError(MOE_ERR_UNSUPPORTED_SHAPE, "moe_workspace_size_shared")
+    if workspace is None or workspace.numel() < nbytes:
+        workspace = _workspace(nbytes, x.device)
+    arr, n = _event_array(events)
+    _check(lib().moe_forward_shared(_ptr(x), _ptr(w_router), _ptr(bias), _ptr(w_gate), _ptr(w_up), _ptr(w_down),
+                                    _ptr(w_gate_s), _ptr(w_up_s), _ptr(w_down_s), T, d, E, k, f, n_s, f_s,
+                                    _ptr(out), _ptr(topk_ids), _ptr(topk_w), _ptr(workspace), workspace.numel(),
+                                    _stream(), arr, n, int(flags or 0)), "moe_forward_shared")
+    return out
+
+
 def combine(y, inv, T, k, out=None):
     """out[t] = sum_j y[inv[t*k+j]] (fp16 rows widened to fp32, fp32 sum, fp32 result)."""
     _need(y, "y", torch.float16, 2)
@@ -268,19 +330,23 @@ def forward(x, w_router, w_gate, w_up, w_down, k, bias=None, out=None, workspace
     if events is None and flags is None:
         _check(lib().moe_forward(*args), "moe_forward")
     else:
-        arr = None
-        n = 0
-        if events is not None:
-            arr = (ctypes.c_void_p * len(events))()
-            for i, ev in enumerate(events):
-                if ev is None:
-                    continue
-                if ev.cuda_event == 0:
-                    ev.record()  # the event handle is created lazily by torch
-                arr[i] = ev.cuda_event
-            n = len(events)
+        arr, n = _event_array(events)
         _check(lib().moe_forward_ex(*args, arr, n, int(flags or 0)), "moe_forward_ex")
     return out
+
+
+def _event_array(events):
+    """ctypes array of cudaEvent_t handles (None entries stay NULL), and its length."""
+    if events is None:
+        return None, 0
+    arr = (ctypes.c_void_p * len(events))()
+    for i, ev in enumerate(events):
+        if ev is None:
+            continue
+        if ev.cuda_event == 0:
+            ev.record()  # the event handle is created lazily by torch
+        arr[i] = ev.cuda_event
+    return arr, len(events)
 
 
 def get_status() -> int:
@@ -324,6 +390,7 @@ class MoEBlock:
 __all__ = [
     "lib", "strerror", "MoEError", "ABI_SYMBOLS", "workspace_size", "route_workspace_size",
     "permute_workspace_size", "MOE_FLAG_FUSED_GATHER", "MOE_FLAG_RENORMALIZE", "route",
-    "permute", "expert_ffn", "combine", "forward", "get_status", "set_wait_limit_ns",
+    "permute", "expert_ffn", "combine", "forward", "shared_ffn", "combine_shared", "forward_shared",
+    "get_status", "set_wait_limit_ns",
     "selftest_wait_timeout", "MoEBlock",
 ]

@@ -19,10 +19,25 @@ namespace combine {
 
 constexpr int kMaxK = 32;
 
+// Widen eight fp16 values and add them to acc.
+__device__ __forceinline__ void add_f16x8(float (&acc)[8], const uint4& q)
+{
+    const __half2* h = reinterpret_cast<const __half2*>(&q);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 f = __half22float2(h[i]);
+        acc[2 * i] += f.x;
+        acc[2 * i + 1] += f.y;
+    }
+}
+
 // One block per token; thread v handles 8 consecutive columns (16 bytes of
-// y, 32 bytes of out).
+// y, 32 bytes of out).  With shared experts (n_s > 0), their rows
+// y_s[s][t] (weight one, already applied) are added after the k routed
+// slots, in ascending s.
 __global__ void __launch_bounds__(256) combine_kernel(const uint4* __restrict__ y, const int32_t* __restrict__ inv,
-                                                      int64_t n, int nvec, int k, float4* __restrict__ out)
+                                                      int64_t n, int nvec, int k, const uint4* __restrict__ y_s,
+                                                      int n_s, int64_t T, float4* __restrict__ out)
 {
     __shared__ int s_pos[kMaxK];
     const int64_t t = blockIdx.x;
@@ -44,17 +59,9 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint4* __restrict__ 
 #pragma unroll 4
         for (int j = 0; j < k; ++j) {
             const int p = s_pos[j];
-            if (p >= 0) {
-                const uint4 q = __ldg(y + (int64_t)p * nvec + v);
-                const __half2* h = reinterpret_cast<const __half2*>(&q);
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const float2 f = __half22float2(h[i]);
-                    acc[2 * i] += f.x;
-                    acc[2 * i + 1] += f.y;
-                }
-            }
+            if (p >= 0) add_f16x8(acc, __ldg(y + (int64_t)p * nvec + v));
         }
+        for (int sh = 0; sh < n_s; ++sh) add_f16x8(acc, __ldg(y_s + ((int64_t)sh * T + t) * nvec + v));
         float4* o = out + (t * nvec + v) * 2;
         o[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
         o[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);

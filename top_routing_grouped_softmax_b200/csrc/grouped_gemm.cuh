@@ -101,8 +101,8 @@ struct Stages {
 enum EpiKind { kSwiGLU = 0, kWeighted = 1 };
 
 struct Params {
-    const int32_t* offsets;  // [E+1] group boundaries (device)
-    const float* w_perm;     // [M] routing weight per grouped row (kWeighted)
+    const int32_t* offsets;  // [E+1] group boundaries (device), or nullptr: one group of M rows
+    const float* w_perm;     // [M] routing weight per grouped row (kWeighted), or nullptr: weight one
     const int32_t* perm;     // [M] grouped row -> flat assignment t*k + j (GATHER)
     const __nv_bfloat16* x;  // [T, ldx] token matrix the A rows are gathered from (GATHER)
     int64_t ldx;             // row length of x in elements (= K for the gate/up GEMM)
@@ -173,7 +173,8 @@ __device__ __forceinline__ void build_tile_list(const int32_t* offsets, int E, i
                                                 int* total, int* bad_out)
 {
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    for (int i = threadIdx.x; i <= E; i += blockDim.x) off[i] = offsets[i];
+    // offsets == nullptr: a single group of all M rows (E == 1)
+    for (int i = threadIdx.x; i <= E; i += blockDim.x) off[i] = offsets ? offsets[i] : (i == 0 ? 0 : M);
     __syncthreads();
     if (warp == 0) {
         int run = 0;
@@ -287,7 +288,7 @@ __device__ __forceinline__ void epilogue_tile(const Params& p, const CUtensorMap
         // slabs of 32 (two 16-column TMEM loads, the next slab in flight)
         constexpr int kIters = kBN / kColGroups / kSlabCols;
         const int cbeg = hf * (kBN / kColGroups);
-        const float wgt = valid ? __ldg(p.w_perm + row) : 0.0f;
+        const float wgt = valid ? (p.w_perm ? __ldg(p.w_perm + row) : 1.0f) : 0.0f;  // no weights: one
         const int wrow0 = row0 + q * 32;                   // first row of this warp's slab
         const bool whole = wrow0 + 31 < row_end;           // all 32 rows belong to the group
         __half* orow = static_cast<__half*>(p.out) + (int64_t)row * p.n_out + nt * kBN;

@@ -231,10 +231,12 @@ size_t permute_ws_bytes(int64_t T, int64_t E) { return align256((size_t)token_ch
 
 // Workspace carve-up for moe_forward.
 struct Layout {
-    size_t ids, wts, counts, offsets, chunk, perm, inv, w_perm, x_perm, h, y, total;
+    size_t ids, wts, counts, offsets, chunk, perm, inv, w_perm, x_perm, h, y, h_s, y_s, total;
 };
 
-Layout plan(int64_t T, int64_t d, int64_t E, int64_t k, int64_t f)
+// n_s shared experts of intermediate size f_s add h_s [T, f_s] bf16 (reused
+// by every shared expert) and y_s [n_s, T, d] fp16.
+Layout plan(int64_t T, int64_t d, int64_t E, int64_t k, int64_t f, int64_t n_s = 0, int64_t f_s = 0)
 {
     const size_t M = (size_t)(T * k);
     Layout L{};
@@ -250,6 +252,8 @@ Layout plan(int64_t T, int64_t d, int64_t E, int64_t k, int64_t f)
     L.x_perm = o;  o += align256(M * (size_t)d * 2);
     L.h = o;       o += align256(M * (size_t)f * 2);
     L.y = o;       o += align256(M * (size_t)d * 2);
+    L.h_s = o;     o += n_s > 0 ? align256((size_t)T * (size_t)f_s * 2) : 0;
+    L.y_s = o;     o += align256((size_t)n_s * (size_t)T * (size_t)d * 2);
     L.total = o;
     return L;
 }
@@ -425,23 +429,58 @@ int run_ffn(const DeviceState& st, const moe_bf16* x_perm, const moe_bf16* x_gat
                   p2);
 }
 
-int run_combine(const moe_f16* y, const int32_t* inv, int64_t T, int64_t d, int64_t k, float* out, cudaStream_t s)
+int run_combine(const moe_f16* y, const int32_t* inv, int64_t T, int64_t d, int64_t k, float* out, cudaStream_t s,
+                const moe_f16* y_s = nullptr, int64_t n_s = 0)
 {
     if (T == 0) return MOE_OK;
     const int nvec = (int)(d / 8);
     const int threads = nvec < 256 ? ((nvec + 31) / 32) * 32 : 256;
     return launch(moe::combine::combine_kernel, dim3((unsigned)T), dim3(threads), 0, s, 1u,
-                  reinterpret_cast<const uint4*>(y), inv, T * k, nvec, (int)k, reinterpret_cast<float4*>(out));
+                  reinterpret_cast<const uint4*>(y), inv, T * k, nvec, (int)k, reinterpret_cast<const uint4*>(y_s),
+                  (int)n_s, T, reinterpret_cast<float4*>(out));
+}
+
+// Shared experts: each is one group of all T rows of x (no permutation, no
+// gather, weight one) through the same grouped GEMMs: h_s = SwiGLU input
+// projections of shared expert s, y_s[s] = h_s . W_down_s[s] in fp16.
+int run_shared(const DeviceState& st, const moe_bf16* x, const moe_bf16* w_gate_s, const moe_bf16* w_up_s,
+               const moe_bf16* w_down_s, int64_t T, int64_t d, int64_t n_s, int64_t f_s, moe_bf16* h_s, moe_f16* y_s,
+               cudaStream_t s)
+{
+    for (int64_t i = 0; i < n_s; ++i) {
+        const int rc = run_ffn(st, x, nullptr, nullptr, T, 1, nullptr, nullptr, w_gate_s + i * d * f_s,
+                               w_up_s + i * d * f_s, w_down_s + i * f_s * d, T, d, 1, f_s, h_s, y_s + i * T * d, s,
+                               nullptr);
+        if (rc) return rc;
+    }
+    return MOE_OK;
+}
+
+constexpr int64_t kMaxShared = 8;
+
+int check_shared(const moe_bf16* w_gate_s, const moe_bf16* w_up_s, const moe_bf16* w_down_s, int64_t T,
+                 int64_t n_s, int64_t f_s)
+{
+    if (n_s < 0 || n_s > kMaxShared) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (n_s == 0) return MOE_OK;
+    int rc = check_f(f_s);
+    if (rc) return rc;
+    if (T > 0 && (!w_gate_s || !w_up_s || !w_down_s)) return MOE_ERR_INVALID_ARG;
+    if (!aligned(w_gate_s, 16) || !aligned(w_up_s, 16) || !aligned(w_down_s, 16)) return MOE_ERR_INVALID_ARG;
+    return MOE_OK;
 }
 
 int forward_impl(const moe_bf16* x, const moe_bf16* w_router, const float* bias, const moe_bf16* w_gate,
                  const moe_bf16* w_up, const moe_bf16* w_down, int64_t T, int64_t d, int64_t E, int64_t k, int64_t f,
                  float* out, int32_t* ids_out, float* w_out, void* ws, size_t ws_bytes, cudaStream_t s,
-                 cudaEvent_t* ev, int n_ev, unsigned flags)
+                 cudaEvent_t* ev, int n_ev, unsigned flags, const moe_bf16* w_gate_s = nullptr,
+                 const moe_bf16* w_up_s = nullptr, const moe_bf16* w_down_s = nullptr, int64_t n_s = 0,
+                 int64_t f_s = 0)
 {
     int rc = check_common(T, d, E, k);
     if (rc) return rc;
     if ((rc = check_f(f))) return rc;
+    if ((rc = check_shared(w_gate_s, w_up_s, w_down_s, T, n_s, f_s))) return rc;
     if (flags & ~(unsigned)(MOE_FLAG_FUSED_GATHER | MOE_FLAG_RENORMALIZE)) return MOE_ERR_INVALID_ARG;
     if (T > 0 && (!x || !w_router || !w_gate || !w_up || !w_down || !out)) return MOE_ERR_INVALID_ARG;
     if (!aligned(x, 16) || !aligned(w_router, 16) || !aligned(w_gate, 16) || !aligned(w_up, 16) ||
@@ -449,7 +488,7 @@ int forward_impl(const moe_bf16* x, const moe_bf16* w_router, const float* bias,
         !aligned(w_out, 4))
         return MOE_ERR_INVALID_ARG;
     if (ev && n_ev < 6) return MOE_ERR_INVALID_ARG;
-    const Layout L = plan(T, d, E, k, f);
+    const Layout L = plan(T, d, E, k, f, n_s, f_s);
     if (T > 0 && (!ws || !aligned(ws, 256))) return MOE_ERR_INVALID_ARG;
     if (ws_bytes < L.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
     DeviceState* st = nullptr;
@@ -488,8 +527,12 @@ int forward_impl(const moe_bf16* x, const moe_bf16* w_router, const float* bias,
     if ((rc = run_ffn(*st, gather ? nullptr : x_perm, gather ? x : nullptr, perm, T, k, w_perm, offsets, w_gate,
                       w_up, w_down, T * k, d, E, f, h, y, s, ev ? ev[3] : nullptr)))
         return rc;
+    moe_f16* y_s = reinterpret_cast<moe_f16*>(w + L.y_s);
+    if (n_s > 0 && (rc = run_shared(*st, x, w_gate_s, w_up_s, w_down_s, T, d, n_s, f_s,
+                                    reinterpret_cast<moe_bf16*>(w + L.h_s), y_s, s)))
+        return rc;
     if ((rc = rec(4))) return rc;
-    if ((rc = run_combine(y, inv, T, d, k, out, s))) return rc;
+    if ((rc = run_combine(y, inv, T, d, k, out, s, y_s, n_s))) return rc;
     return rec(5);
 }
 
@@ -548,12 +591,20 @@ const char* moe_strerror(int status)
     }
 }
 
-int moe_version(void) { return 201; }
+int moe_version(void) { return 202; }
 
 size_t moe_workspace_size(int64_t T, int64_t d, int64_t E, int64_t k, int64_t f)
 {
     if (check_common(T, d, E, k) || check_f(f)) return 0;
     return plan(T, d, E, k, f).total;
+}
+
+size_t moe_workspace_size_shared(int64_t T, int64_t d, int64_t E, int64_t k, int64_t f, int64_t n_shared,
+                                 int64_t f_shared)
+{
+    if (check_common(T, d, E, k) || check_f(f) || n_shared < 1 || n_shared > kMaxShared || check_f(f_shared))
+        return 0;
+    return plan(T, d, E, k, f, n_shared, f_shared).total;
 }
 
 size_t moe_route_workspace_size(int64_t T, int64_t d, int64_t E)
@@ -668,6 +719,49 @@ int moe_combine(const moe_f16* y, const int32_t* inv, int64_t T, int64_t d, int6
     int rc = setup_device(&st);
     if (rc) return rc;
     return run_combine(y, inv, T, d, k, out, stream);
+}
+
+int moe_shared_ffn(const moe_bf16* x, const moe_bf16* w_gate_s, const moe_bf16* w_up_s, const moe_bf16* w_down_s,
+                   int64_t T, int64_t d, int64_t n_shared, int64_t f_shared, moe_bf16* h_s, moe_f16* y_s,
+                   cudaStream_t stream)
+{
+    if (T < 0 || d <= 0 || n_shared < 1) return MOE_ERR_INVALID_ARG;
+    if (d % 64 != 0 || d > 32768 || T >= (int64_t(1) << 31)) return MOE_ERR_UNSUPPORTED_SHAPE;
+    int rc;
+    if ((rc = check_shared(w_gate_s, w_up_s, w_down_s, T, n_shared, f_shared))) return rc;
+    if (T > 0 && (!x || !h_s || !y_s)) return MOE_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(h_s, 16) || !aligned(y_s, 16)) return MOE_ERR_INVALID_ARG;
+    if (T == 0) return MOE_OK;
+    DeviceState* st = nullptr;
+    if ((rc = setup_device(&st))) return rc;
+    return run_shared(*st, x, w_gate_s, w_up_s, w_down_s, T, d, n_shared, f_shared, h_s, y_s, stream);
+}
+
+int moe_combine_shared(const moe_f16* y, const int32_t* inv, const moe_f16* y_s, int64_t n_shared, int64_t T,
+                       int64_t d, int64_t k, float* out, cudaStream_t stream)
+{
+    if (T < 0 || d <= 0 || k <= 0 || n_shared < 0) return MOE_ERR_INVALID_ARG;
+    if (d % 64 != 0 || d > 32768 || k > 32 || T * k >= (int64_t(1) << 31) || n_shared > kMaxShared)
+        return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (T > 0 && (!y || !inv || !out || (n_shared > 0 && !y_s))) return MOE_ERR_INVALID_ARG;
+    if (!aligned(y, 16) || !aligned(out, 16) || !aligned(inv, 4) || !aligned(y_s, 16)) return MOE_ERR_INVALID_ARG;
+    DeviceState* st = nullptr;
+    int rc = setup_device(&st);
+    if (rc) return rc;
+    return run_combine(y, inv, T, d, k, out, stream, y_s, n_shared);
+}
+
+int moe_forward_shared(const moe_bf16* x, const moe_bf16* w_router, const float* bias, const moe_bf16* w_gate,
+                       const moe_bf16* w_up, const moe_bf16* w_down, const moe_bf16* w_gate_s,
+                       const moe_bf16* w_up_s, const moe_bf16* w_down_s, int64_t T, int64_t d, int64_t E, int64_t k,
+                       int64_t f, int64_t n_shared, int64_t f_shared, float* out, int32_t* topk_ids_out,
+                       float* topk_w_out, void* workspace, size_t workspace_bytes, cudaStream_t stream,
+                       cudaEvent_t* events, int n_events, unsigned flags)
+{
+    if (n_shared < 1) return MOE_ERR_INVALID_ARG;
+    return forward_impl(x, w_router, bias, w_gate, w_up, w_down, T, d, E, k, f, out, topk_ids_out, topk_w_out,
+                        workspace, workspace_bytes, stream, events, n_events, flags, w_gate_s, w_up_s, w_down_s,
+                        n_shared, f_shared);
 }
 
 int moe_forward(const moe_bf16* x, const moe_bf16* w_router, const float* bias, const moe_bf16* w_gate,
