@@ -304,3 +304,129 @@ int oracle_shared_rows(const uint16_t* x, const uint16_t* w_gate_s, const uint16
     free(xrow); free(g); free(u); free(h); free(o);
     return status;
 }
+
+/*
+ * Optional variant: token rounding (the "token rounding" scheduling of the
+ * SonicMoE comparison page, core difference 3: adjust the number of tokens
+ * each expert receives so that the grouped GEMM needs no tile padding).  The
+ * page's pseudocode is garbled; the reading implemented here, per expert e
+ * and independently of the other experts, starting from the top-k routing:
+ *   c = number of tokens routed to e, r = c mod R (R = the tile rows);
+ *   r == 0        : unchanged;
+ *   2 r <= R      : drop the r routed tokens with the smallest p[t][e]
+ *                   (equal p: the larger token index is dropped first);
+ *   2 r >  R      : add the a = R - r unrouted tokens with the largest
+ *                   p[t][e] (equal p: the smaller token index first), if
+ *                   T - c >= a; otherwise drop r as above.
+ * Every count becomes a multiple of R.  A token's weight for each expert it
+ * keeps or gains is its softmax probability p[t][e]; a token may end with
+ * fewer or more than k experts.
+ *   probs [T][E] fp64 (oracle_route's probs_out), ids [T][k]
+ *   mask_out [T][E] (1: token t goes to expert e after rounding), counts_out [E]
+ */
+typedef struct {
+    double p;
+    int64_t t;
+} cand_t;
+
+/* ascending p; equal p: larger t first (the order in which tokens are dropped) */
+static int drop_order(const void* a, const void* b)
+{
+    const cand_t* x = (const cand_t*)a;
+    const cand_t* y = (const cand_t*)b;
+    if (x->p < y->p) return -1;
+    if (x->p > y->p) return 1;
+    return (x->t < y->t) - (x->t > y->t);
+}
+
+/* descending p; equal p: smaller t first (the order in which tokens are added) */
+static int add_order(const void* a, const void* b)
+{
+    const cand_t* x = (const cand_t*)a;
+    const cand_t* y = (const cand_t*)b;
+    if (x->p > y->p) return -1;
+    if (x->p < y->p) return 1;
+    return (x->t > y->t) - (x->t < y->t);
+}
+
+int oracle_round_tokens(const double* probs, const int32_t* ids, int64_t T, int64_t E, int64_t k, int64_t R,
+                        uint8_t* mask_out, int32_t* counts_out)
+{
+    if (!probs || !ids || !mask_out || !counts_out || T < 0 || E < 1 || k < 1 || k > E || R < 1)
+        return ORACLE_BAD_ARG;
+    memset(mask_out, 0, (size_t)(T * E));
+    for (int64_t a = 0; a < T * k; ++a) {
+        const int32_t e = ids[a];
+        if (e < 0 || e >= E) return ORACLE_BAD_ARG;
+        mask_out[(a / k) * E + e] = 1;
+    }
+    cand_t* in = (cand_t*)malloc(sizeof(cand_t) * (size_t)(T > 0 ? T : 1));
+    cand_t* out = (cand_t*)malloc(sizeof(cand_t) * (size_t)(T > 0 ? T : 1));
+    if (!in || !out) {
+        free(in); free(out);
+        return ORACLE_NO_MEMORY;
+    }
+    for (int64_t e = 0; e < E; ++e) {
+        int64_t n_in = 0, n_out = 0;
+        for (int64_t t = 0; t < T; ++t) {
+            cand_t cd = {probs[t * E + e], t};
+            if (mask_out[t * E + e]) in[n_in++] = cd; else out[n_out++] = cd;
+        }
+        const int64_t r = n_in % R;
+        int64_t count = n_in;
+        if (r != 0) {
+            const int64_t add = R - r;
+            if (2 * r > R && n_out >= add) {
+                qsort(out, (size_t)n_out, sizeof(cand_t), add_order);
+                for (int64_t i = 0; i < add; ++i) mask_out[out[i].t * E + e] = 1;
+                count += add;
+            } else {
+                qsort(in, (size_t)n_in, sizeof(cand_t), drop_order);
+                for (int64_t i = 0; i < r; ++i) mask_out[in[i].t * E + e] = 0;
+                count -= r;
+            }
+        }
+        counts_out[e] = (int32_t)count;
+    }
+    free(in); free(out);
+    return ORACLE_OK;
+}
+
+/*
+ * Stages 3 and 4 for a routing given as a mask (token rounding):
+ *   out[r] = sum_{e ascending, mask[t][e] = 1} probs[t][e] * expert_e(x[t]), t = rows[r].
+ */
+int oracle_masked_rows(const uint16_t* x, const uint16_t* w_gate, const uint16_t* w_up,
+                       const uint16_t* w_down, int64_t T, int64_t d, int64_t E, int64_t f,
+                       const uint8_t* mask, const double* probs, int64_t n_rows, const int64_t* rows,
+                       double* out)
+{
+    if (!x || !w_gate || !w_up || !w_down || !mask || !probs || !rows || !out || T < 0 || d < 1 ||
+        E < 1 || f < 1 || n_rows < 0)
+        return ORACLE_BAD_ARG;
+    double* xrow = (double*)malloc(sizeof(double) * d);
+    double* g = (double*)malloc(sizeof(double) * f);
+    double* u = (double*)malloc(sizeof(double) * f);
+    double* h = (double*)malloc(sizeof(double) * f);
+    double* o = (double*)malloc(sizeof(double) * d);
+    if (!xrow || !g || !u || !h || !o) {
+        free(xrow); free(g); free(u); free(h); free(o);
+        return ORACLE_NO_MEMORY;
+    }
+    int status = ORACLE_OK;
+    for (int64_t r = 0; r < n_rows; ++r) {
+        const int64_t t = rows[r];
+        if (t < 0 || t >= T) { status = ORACLE_BAD_ARG; break; }
+        for (int64_t i = 0; i < d; ++i) xrow[i] = bf16_to_double(x[t * d + i]);
+        double* orow = out + r * d;
+        for (int64_t c = 0; c < d; ++c) orow[c] = 0.0;
+        for (int64_t e = 0; e < E; ++e) {
+            if (!mask[t * E + e]) continue;
+            expert_swiglu(xrow, w_gate + e * d * f, w_up + e * d * f, w_down + e * f * d, d, f, g, u, h, o);
+            const double we = probs[t * E + e];
+            for (int64_t c = 0; c < d; ++c) orow[c] += we * o[c];
+        }
+    }
+    free(xrow); free(g); free(u); free(h); free(o);
+    return status;
+}

@@ -65,6 +65,10 @@ class Oracle:
         lib.oracle_renormalize.argtypes = [_P, _I64, _I64]
         lib.oracle_shared_rows.argtypes = [_P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64, _P, _P]
         lib.oracle_shared_rows.restype = ctypes.c_int
+        lib.oracle_round_tokens.argtypes = [_P, _P, _I64, _I64, _I64, _I64, _P, _P]
+        lib.oracle_round_tokens.restype = ctypes.c_int
+        lib.oracle_masked_rows.argtypes = [_P, _P, _P, _P, _I64, _I64, _I64, _I64, _P, _P, _I64, _P, _P]
+        lib.oracle_masked_rows.restype = ctypes.c_int
         for fn in (lib.oracle_route, lib.oracle_permute, lib.oracle_expert_rows, lib.oracle_renormalize):
             fn.restype = ctypes.c_int
         self.lib = lib
@@ -145,6 +149,39 @@ class Oracle:
         if rc != 0:
             raise ValueError(f"oracle_shared_rows failed ({rc})")
         return res
+
+    # -- token rounding -------------------------------------------------------
+    def round_tokens(self, probs, ids, tile):
+        """Token rounding of the top-k routing to multiples of ``tile`` rows per
+        expert; returns (mask [T, E] bool, counts [E] int32)."""
+        probs = np.ascontiguousarray(probs, dtype=np.float64)
+        ids = np.ascontiguousarray(ids, dtype=np.int32)
+        T, E = probs.shape
+        k = ids.shape[1]
+        mask = np.empty((T, E), np.uint8)
+        counts = np.empty(E, np.int32)
+        rc = self.lib.oracle_round_tokens(_ptr(probs), _ptr(ids), T, E, k, tile, _ptr(mask), _ptr(counts))
+        if rc != 0:
+            raise ValueError(f"oracle_round_tokens failed ({rc})")
+        return mask.astype(bool), counts
+
+    def masked_rows(self, x, w_gate, w_up, w_down, mask, probs, rows):
+        """out[r] = sum over experts e (ascending) with mask[t, e] of probs[t, e] * expert_e(x[t])."""
+        x = np.ascontiguousarray(x, dtype=np.uint16)
+        w_gate = np.ascontiguousarray(w_gate, dtype=np.uint16)
+        w_up = np.ascontiguousarray(w_up, dtype=np.uint16)
+        w_down = np.ascontiguousarray(w_down, dtype=np.uint16)
+        m = np.ascontiguousarray(mask, dtype=np.uint8)
+        probs = np.ascontiguousarray(probs, dtype=np.float64)
+        rows = np.ascontiguousarray(rows, dtype=np.int64)
+        T, d = x.shape
+        E, _, f = w_gate.shape
+        out = np.empty((rows.shape[0], d), np.float64)
+        rc = self.lib.oracle_masked_rows(_ptr(x), _ptr(w_gate), _ptr(w_up), _ptr(w_down), T, d, E, f, _ptr(m),
+                                         _ptr(probs), rows.shape[0], _ptr(rows), _ptr(out))
+        if rc != 0:
+            raise ValueError(f"oracle_masked_rows failed ({rc})")
+        return out
 
     # -- whole block ----------------------------------------------------------
     def forward(self, x, w_router, bias, w_gate, w_up, w_down, k, rows=None,

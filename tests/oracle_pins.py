@@ -308,9 +308,80 @@ def check_shared_experts(o):
     assert np.array_equal(ex0.out, plain.out)
 
 
+def _rounding_ok(probs, mask0, mask, tile):
+    """Order-statistic characterisation of token rounding, expert by expert:
+    the count becomes a multiple of the tile; a dropped token ranks below
+    every kept one by (p, then the smaller index kept); an added token ranks
+    above every unrouted one left out (p, then the smaller index added)."""
+    T, E = probs.shape
+    for e in range(E):
+        m0, m1 = mask0[:, e], mask[:, e]
+        c, r = int(m0.sum()), int(m0.sum()) % tile
+        n = int(m1.sum())
+        added, dropped = np.nonzero(m1 & ~m0)[0], np.nonzero(m0 & ~m1)[0]
+        assert added.size == 0 or dropped.size == 0, f"expert {e} both gains and loses tokens"
+        if r == 0:
+            assert n == c
+            continue
+        if added.size:
+            assert 2 * r > tile and n == c + tile - r, (e, c, n)
+            rest = np.nonzero(~m0 & ~m1)[0]
+            for a in added:
+                assert np.all((probs[a, e] > probs[rest, e]) | ((probs[a, e] == probs[rest, e]) & (a < rest)))
+        else:
+            assert (2 * r <= tile or T - c < tile - r) and n == c - r, (e, c, n)
+            kept = np.nonzero(m1)[0]
+            for dd in dropped:
+                assert np.all((probs[dd, e] < probs[kept, e]) | ((probs[dd, e] == probs[kept, e]) & (dd > kept)))
+
+
+def check_token_rounding(o):
+    """Token rounding: tile 1 changes nothing; on random routing every
+    expert's count becomes a tile multiple by the order-statistic rule; the
+    masked block output equals a dense numpy evaluation with the rounded
+    mask; exact ties drop the larger and add the smaller token index."""
+    inp = _rand_case(300, 64, 8, 2, 32, seed=53, bias=True)
+    x, wr, b = inp.bits("x"), inp.bits("W_router"), inp.bias_np()
+    r = o.route(x, wr, b, 2)
+    mask0 = np.zeros((300, 8), bool)
+    np.put_along_axis(mask0, r.ids.astype(np.int64), True, axis=1)
+    same, c1 = o.round_tokens(r.probs, r.ids, 1)
+    assert np.array_equal(same, mask0) and np.array_equal(c1, mask0.sum(0))
+    for tile in (16, 48):
+        mask, counts = o.round_tokens(r.probs, r.ids, tile)
+        assert np.array_equal(counts, mask.sum(0))
+        _rounding_ok(r.probs, mask0, mask, tile)
+    mask, _ = o.round_tokens(r.probs, r.ids, 16)
+    rows = np.arange(300, dtype=np.int64)
+    got = o.masked_rows(x, inp.bits("W_gate"), inp.bits("W_up"), inp.bits("W_down"), mask, r.probs, rows)
+    X = widen(x)
+    ref = np.zeros_like(got)
+    for e in range(8):
+        G = X @ widen(inp.bits("W_gate")[e])
+        U = X @ widen(inp.bits("W_up")[e])
+        ref += (mask[:, e] * r.probs[:, e])[:, None] * ((G * sps.expit(G) * U) @ widen(inp.bits("W_down")[e]))
+    assert _rel(got, ref) < 1e-12, _rel(got, ref)
+    # exact ties: tokens 0..19 prefer expert 0, tokens 20..39 expert 1, all
+    # with the same probability pair
+    T = 40
+    v = widen(inp.bits("x")[0, :64])
+    xs = np.vstack([np.tile(v, (20, 1)), np.tile(-v, (20, 1))])
+    wcol = widen(inp.bits("W_router")[:, 0])
+    wr2 = np.stack([wcol, -wcol], axis=1)
+    xb, wb = bf16_bits(torch.from_numpy(xs).to(torch.bfloat16)), bf16_bits(torch.from_numpy(wr2).to(torch.bfloat16))
+    rt = o.route(xb, wb, None, 1)
+    assert set(rt.ids[:20, 0]) == {0} and set(rt.ids[20:, 0]) == {1}
+    m16, _ = o.round_tokens(rt.probs, rt.ids, 16)      # 20 each, r = 4: drop the 4 largest indices
+    assert np.array_equal(np.nonzero(m16[:, 0])[0], np.arange(16))
+    assert np.array_equal(np.nonzero(m16[:, 1])[0], np.arange(20, 36))
+    m24, _ = o.round_tokens(rt.probs, rt.ids, 24)      # r = 20 > 12: add the 4 smallest unrouted indices
+    assert np.array_equal(np.nonzero(m24[:, 0])[0], np.arange(24))
+    assert np.array_equal(np.nonzero(m24[:, 1])[0], np.concatenate([np.arange(4), np.arange(20, 40)]))
+
+
 ALL_CHECKS = [
     check_brute_force, check_softmax_library, check_topk_library_sort, check_topk_of_logits,
     check_exact_ties, check_dense_special_case, check_all_experts_identical, check_zero_expert,
     check_scale_down, check_permute_library, check_page_listing_torch, check_expert_rows_outputs,
-    check_renormalize, check_shared_experts,
+    check_renormalize, check_shared_experts, check_token_rounding,
 ]

@@ -29,6 +29,14 @@ MUTANTS = [
     ("weights_from_wrong_slot", "weights[t * k + j] = ranked[j].p;", "weights[t * k + j] = ranked[0].p;"),
     ("sum_only_first_slot", "orow[c] += yc;", "orow[c] += (j == 0) ? yc : 0.0;"),
     ("renorm_no_divide", "weights[t * k + j] /= s;", "weights[t * k + j] /= 1.0;"),
+    ("round_drops_largest", "qsort(in, (size_t)n_in, sizeof(cand_t), drop_order);",
+     "qsort(in, (size_t)n_in, sizeof(cand_t), add_order);"),
+    ("round_adds_smallest", "qsort(out, (size_t)n_out, sizeof(cand_t), add_order);",
+     "qsort(out, (size_t)n_out, sizeof(cand_t), drop_order);"),
+    ("round_drop_tie_smaller_index", "return (x->t < y->t) - (x->t > y->t);",
+     "return (x->t > y->t) - (x->t < y->t);"),
+    ("round_one_short", "const int64_t add = R - r;", "const int64_t add = R - r - 1;"),
+    ("masked_weight_one", "const double we = probs[t * E + e];", "const double we = 1.0;"),
     ("shared_first_only", "for (int64_t sidx = 0; sidx < n_s; ++sidx) {",
      "for (int64_t sidx = 0; sidx < 1; ++sidx) {"),
     ("shared_half_weight", "for (int64_t c = 0; c < d; ++c) out[r * d + c] += o[c];",
