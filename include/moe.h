@@ -310,6 +310,44 @@ int moe_forward_shared(const moe_bf16* x, const moe_bf16* w_router, const float*
                        cudaEvent_t* events, int n_events, unsigned flags);
 
 /*
+ * Token rounding (optional; an approximation, not the article's block): the
+ * "token rounding" scheduling of the SonicMoE comparison page (core
+ * difference 3), which adjusts how many tokens each expert receives so the
+ * grouped GEMMs need no tile padding.  The page's pseudocode is garbled; the
+ * rule implemented, per expert e and independently of the other experts,
+ * starting from the top-k routing (c tokens routed to e, r = c mod tile):
+ *   r == 0         unchanged;
+ *   2 r <= tile    drop the r routed tokens with the smallest p[t,e]
+ *                  (equal p: the larger token index first);
+ *   2 r >  tile    add the tile - r unrouted tokens with the largest p[t,e]
+ *                  (equal p: the smaller token index first) when there are
+ *                  that many, else drop r as above.
+ * Every count becomes a multiple of `tile` (256 matches the CTA-pair GEMM
+ * tile, leaving it no padding).  A token's weight for each expert it keeps or
+ * gains is the softmax probability p[t,e]; a token can end with more or
+ * fewer than k experts (or none):
+ *   out[t] = sum over its experts e, ascending, of p[t,e] * expert_e(x[t]).
+ * Limits: T <= 2^20, 1 <= tile <= 65536, T*k + E*(tile-1) < 2^31.
+ */
+
+/* Bytes of scratch for moe_forward_rounded (0 if a shape is unsupported). */
+size_t moe_workspace_size_rounded(int64_t T, int64_t d, int64_t E, int64_t k, int64_t f, int64_t tile);
+
+/*
+ * The block with token rounding.  out [T, d] fp32.  counts_out [E] int32 (or
+ * NULL): the rounded token count of every expert.  rows_out [T, E] int32 (or
+ * NULL): the grouped row of (t, e), -1 where token t does not go to expert e
+ * (so rows_out >= 0 is the rounded routing mask).  events as for
+ * moe_forward_ex (the "after permute" event follows the rounding).
+ */
+int moe_forward_rounded(const moe_bf16* x, const moe_bf16* w_router, const float* bias,
+                        const moe_bf16* w_gate, const moe_bf16* w_up, const moe_bf16* w_down,
+                        int64_t T, int64_t d, int64_t E, int64_t k, int64_t f, int64_t tile,
+                        float* out, int32_t* counts_out, int32_t* rows_out,
+                        void* workspace, size_t workspace_bytes, cudaStream_t stream,
+                        cudaEvent_t* events, int n_events);
+
+/*
  * Synchronises `stream`, then returns and clears the current device's status
  * word (MOE_OK if no device-side error was recorded since the last call).
  */

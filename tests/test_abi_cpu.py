@@ -34,7 +34,7 @@ def test_library_exports_every_declared_symbol(moe_lib):
 
 
 def test_strerror_and_version(moe_lib):
-    assert moe_lib.moe_version() == 202
+    assert moe_lib.moe_version() == 203
     for code in range(10):
         assert moe.strerror(code).startswith("MOE_")
 

@@ -39,7 +39,7 @@ ABI_SYMBOLS = (
     "moe_permute_workspace_size", "moe_route", "moe_permute", "moe_expert_ffn", "moe_combine", "moe_forward",
     "moe_forward_ex", "moe_get_status", "moe_set_wait_limit_ns", "moe_selftest_wait_timeout",
     "moe_permute_static", "moe_route_ex", "moe_workspace_size_shared", "moe_shared_ffn", "moe_combine_shared",
-    "moe_forward_shared",
+    "moe_forward_shared", "moe_workspace_size_rounded", "moe_forward_rounded",
 )
 
 
@@ -87,6 +87,9 @@ def lib() -> ctypes.CDLL:
         L.moe_workspace_size_shared.argtypes = [_I64] * 7
         L.moe_shared_ffn.argtypes = [_P, _P, _P, _P, _I64, _I64, _I64, _I64, _P, _P, _P]
         L.moe_combine_shared.argtypes = [_P, _P, _P, _I64, _I64, _I64, _I64, _P, _P]
+        L.moe_workspace_size_rounded.restype = _SZ
+        L.moe_workspace_size_rounded.argtypes = [_I64] * 6
+        L.moe_forward_rounded.argtypes = [_P] * 6 + [_I64] * 6 + [_P, _P, _P, _P, _SZ, _P, _P, ctypes.c_int]
         L.moe_forward_shared.argtypes = ([_P] * 9 + [_I64] * 7 + [_P, _P, _P, _P, _SZ, _P, _P, ctypes.c_int,
                                                                    ctypes.c_uint])
         L.moe_get_status.argtypes = [_P]
@@ -95,7 +98,7 @@ def lib() -> ctypes.CDLL:
         for name in ("moe_route", "moe_permute", "moe_expert_ffn", "moe_combine", "moe_forward",
                      "moe_forward_ex", "moe_get_status", "moe_set_wait_limit_ns",
                      "moe_selftest_wait_timeout", "moe_permute_static", "moe_route_ex", "moe_shared_ffn",
-                     "moe_combine_shared", "moe_forward_shared"):
+                     "moe_combine_shared", "moe_forward_shared", "moe_forward_rounded"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -277,6 +280,32 @@ def forward_shared(x, w_router, w_gate, w_up, w_down, w_gate_s, w_up_s, w_down_s
     return out
 
 
+def forward_rounded(x, w_router, w_gate, w_up, w_down, k, tile=256, bias=None, out=None, workspace=None,
+                    counts=None, rows=None, events=None):
+    """The block with token rounding (every expert's token count rounded to a
+    multiple of ``tile``); returns (out fp32 [T, d], counts int32 [E], rows).
+    ``rows`` (optional int32 [T, E] output): the grouped row of (t, e), -1
+    where token t does not go to expert e."""
+    T, d, E, f = _forward_args(x, w_router, w_gate, w_up, w_down, bias)
+    if out is None:
+        out = torch.empty(T, d, dtype=torch.float32, device=x.device)
+    _need(out, "out", torch.float32, 2)
+    if counts is None:
+        counts = torch.empty(E, dtype=torch.int32, device=x.device)
+    if rows is not None:
+        _need(rows, "rows", torch.int32, 2)
+    nbytes = int(lib().moe_workspace_size_rounded(T, d, E, k, f, tile))
+    if nbytes == 0:
+        raise MoEError(MOE_ERR_UNSUPPORTED_SHAPE, "moe_workspace_size_rounded")
+    if workspace is None or workspace.numel() < nbytes:
+        workspace = _workspace(nbytes, x.device)
+    arr, n = _event_array(events)
+    _check(lib().moe_forward_rounded(_ptr(x), _ptr(w_router), _ptr(bias), _ptr(w_gate), _ptr(w_up), _ptr(w_down),
+                                     T, d, E, k, f, tile, _ptr(out), _ptr(counts), _ptr(rows), _ptr(workspace),
+                                     workspace.numel(), _stream(), arr, n), "moe_forward_rounded")
+    return out, counts, rows
+
+
 def combine(y, inv, T, k, out=None):
     """out[t] = sum_j y[inv[t*k+j]] (fp16 rows widened to fp32, fp32 sum, fp32 result)."""
     _need(y, "y", torch.float16, 2)
@@ -390,7 +419,7 @@ class MoEBlock:
 __all__ = [
     "lib", "strerror", "MoEError", "ABI_SYMBOLS", "workspace_size", "route_workspace_size",
     "permute_workspace_size", "MOE_FLAG_FUSED_GATHER", "MOE_FLAG_RENORMALIZE", "route",
-    "permute", "expert_ffn", "combine", "forward", "shared_ffn", "combine_shared", "forward_shared",
+    "permute", "expert_ffn", "combine", "forward", "shared_ffn", "combine_shared", "forward_shared", "forward_rounded",
     "get_status", "set_wait_limit_ns",
     "selftest_wait_timeout", "MoEBlock",
 ]

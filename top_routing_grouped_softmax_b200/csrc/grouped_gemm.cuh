@@ -113,6 +113,7 @@ struct Params {
     int n_out;    // output columns (multiple of 64)
     int n_tiles;  // N tiles per M tile
     int k_top;    // experts per token (GATHER: token = perm[row] / k_top)
+    int m_capacity;  // 0: offsets[E] must equal M; 1: M is a capacity, offsets[E] <= M
 };
 
 // Shared memory after the stage ring and the store staging buffers.
@@ -170,7 +171,7 @@ __device__ __forceinline__ void decode(int64_t w, int n_tiles, const Ctrl& c, in
 // Contains __syncthreads: every thread of the block must call it.
 template <int TILE_ROWS>
 __device__ __forceinline__ void build_tile_list(const int32_t* offsets, int E, int M, int* off, int* tp,
-                                                int* total, int* bad_out)
+                                                int* total, int* bad_out, bool capacity = false)
 {
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     // offsets == nullptr: a single group of all M rows (E == 1)
@@ -199,7 +200,7 @@ __device__ __forceinline__ void build_tile_list(const int32_t* offsets, int E, i
         bad = __any_sync(0xffffffffu, bad);
         if (lane == 0) {
             tp[E] = run;
-            *bad_out = (bad || off[0] != 0 || off[E] != M) ? 1 : 0;
+            *bad_out = (bad || off[0] != 0 || (capacity ? off[E] > M : off[E] != M)) ? 1 : 0;
             *total = run;
             if (*bad_out && blockIdx.x == 0) record_status(kStatusDeviceBounds);
         }
@@ -391,7 +392,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     pdl_trigger();
     pdl_wait();
     // ---- tile list from the device offsets (validated) ----
-    build_tile_list<kBM>(p.offsets, E, p.M, c.off, c.tp, &c.total_mtiles, &c.bad);
+    build_tile_list<kBM>(p.offsets, E, p.M, c.off, c.tp, &c.total_mtiles, &c.bad, p.m_capacity != 0);
     __syncthreads();
     const int64_t total_work = c.bad ? 0 : (int64_t)c.total_mtiles * p.n_tiles;
     const int num_kb = p.K / kBK;

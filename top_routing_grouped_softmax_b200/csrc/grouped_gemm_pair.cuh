@@ -101,7 +101,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // the offsets and operands come from earlier kernels on the stream
     pdl_trigger();
     pdl_wait();
-    build_tile_list<kPairRows>(p.offsets, E, p.M, c.off, c.tp, &c.total_mtiles, &c.bad);
+    build_tile_list<kPairRows>(p.offsets, E, p.M, c.off, c.tp, &c.total_mtiles, &c.bad, p.m_capacity != 0);
     __syncthreads();
     const int64_t total_work = c.bad ? 0 : (int64_t)c.total_mtiles * p.n_tiles;
     const int num_kb = p.K / kBK;

@@ -13,6 +13,7 @@
 #include "status.cuh"
 #include "ptx.cuh"
 #include "route.cuh"
+#include "rounding.cuh"
 #include "permute.cuh"
 #include "grouped_gemm.cuh"
 #include "grouped_gemm_pair.cuh"
@@ -141,6 +142,7 @@ int setup_device(DeviceState** out)
             e = e ? e : cudaFuncSetAttribute(moe::route::route_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
             e = e ? e : cudaFuncSetAttribute(moe::route::route_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
             e = e ? e : cudaFuncSetAttribute(moe::route::route_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
+            e = e ? e : cudaFuncSetAttribute(moe::rounding::round_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
             e = e ? e : cudaFuncSetAttribute(moe::gemm::grouped_gemm_kernel<moe::gemm::kSwiGLU, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
             e = e ? e : cudaFuncSetAttribute(moe::gemm::grouped_gemm_kernel<moe::gemm::kSwiGLU, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
             e = e ? e : cudaFuncSetAttribute(moe::gemm::grouped_gemm_kernel<moe::gemm::kWeighted, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
@@ -276,7 +278,7 @@ int launch_route(const CUtensorMap& tx, const CUtensorMap& tw, moe::route::Param
 
 int run_route(const DeviceState& st, const moe_bf16* x, const moe_bf16* w_router, const float* bias, int64_t T,
               int64_t d, int64_t E, int64_t k, int32_t* ids, float* wts, int32_t* chunk_counts, bool renorm,
-              cudaStream_t s)
+              cudaStream_t s, float* probs_t = nullptr)
 {
     if (T == 0) return MOE_OK;
     CUtensorMap tx, tw;
@@ -307,6 +309,7 @@ int run_route(const DeviceState& st, const moe_bf16* x, const moe_bf16* w_router
     p.split = (E <= 256 && d >= 2 * moe::route::kBK && tiles <= pairs) ? 2 : 1;
     p.passes = (p.split == 1 && E > 256) ? 2 : 1;
     p.renorm = renorm ? 1 : 0;
+    p.probs_t = probs_t;
     // top-k list length: the power of two >= k for lane groups (k <= 8), or
     // the whole-warp rounds (k > 8)
     const unsigned ut = (unsigned)tiles;
@@ -357,7 +360,7 @@ int run_permute(const moe_bf16* x, const int32_t* ids, const float* wts, int64_t
 int run_ffn(const DeviceState& st, const moe_bf16* x_perm, const moe_bf16* x_gather, const int32_t* perm,
             int64_t T, int64_t k, const float* w_perm, const int32_t* offsets, const moe_bf16* w_gate,
             const moe_bf16* w_up, const moe_bf16* w_down, int64_t M, int64_t d, int64_t E, int64_t f, moe_bf16* h,
-            moe_f16* y, cudaStream_t s, cudaEvent_t mid_event)
+            moe_f16* y, cudaStream_t s, cudaEvent_t mid_event, bool m_capacity = false)
 {
     if (M == 0) {
         if (mid_event && cudaEventRecord(mid_event, s) != cudaSuccess) return MOE_ERR_CUDA;
@@ -394,6 +397,7 @@ int run_ffn(const DeviceState& st, const moe_bf16* x_perm, const moe_bf16* x_gat
     p1.n_out = (int)f;
     p1.n_tiles = (int)((f + 127) / 128);
     p1.k_top = (int)k;
+    p1.m_capacity = m_capacity ? 1 : 0;
     const int64_t work1 = max_mtiles * p1.n_tiles;
     const unsigned grid1 = (unsigned)(work1 < st.sm_count ? work1 : st.sm_count);
     const int64_t max_pair_tiles = (M + kPairRows - 1) / kPairRows + E;
@@ -422,6 +426,7 @@ int run_ffn(const DeviceState& st, const moe_bf16* x_perm, const moe_bf16* x_gat
     p2.n_out = (int)d;
     p2.n_tiles = (int)((d + kBN - 1) / kBN);
     p2.k_top = 1;
+    p2.m_capacity = m_capacity ? 1 : 0;
     const int64_t work2 = max_mtiles * p2.n_tiles;
     const unsigned grid2 = (unsigned)(work2 < st.sm_count ? work2 : st.sm_count);
     if (MOE_GEMM_PAIR) return launch_pair_gemm<kWeighted>(st, max_pair_tiles * p2.n_tiles, ta2, td, td, ty, p2, s);
@@ -536,6 +541,136 @@ int forward_impl(const moe_bf16* x, const moe_bf16* w_router, const float* bias,
     return rec(5);
 }
 
+// ------------------------------------------------------------ token rounding
+// Rows of the rounded grouping: every expert gains fewer than `tile` rows.
+inline int64_t round_capacity(int64_t T, int64_t E, int64_t k, int64_t tile) { return T * k + E * (tile - 1); }
+
+int check_rounding(int64_t T, int64_t E, int64_t k, int64_t tile)
+{
+    if (tile < 1) return MOE_ERR_INVALID_ARG;
+    if (tile > 65536 || T > moe::rounding::kMaxTokens || round_capacity(T, E, k, tile) >= (int64_t(1) << 31))
+        return MOE_ERR_UNSUPPORTED_SHAPE;
+    return MOE_OK;
+}
+
+struct RLayout {
+    size_t ids, wts, counts, offsets, chunk, perm, inv, w_perm, probs_t, bitmaps, new_counts, offsets2, tok, w2,
+        posmap, x_perm, h, y, total;
+};
+
+RLayout plan_rounded(int64_t T, int64_t d, int64_t E, int64_t k, int64_t f, int64_t tile)
+{
+    const size_t M = (size_t)(T * k);
+    const size_t cap = (size_t)round_capacity(T, E, k, tile);
+    RLayout L{};
+    size_t o = 0;
+    L.ids = o;        o += align256(M * 4);
+    L.wts = o;        o += align256(M * 4);
+    L.counts = o;     o += align256((size_t)E * 4);
+    L.offsets = o;    o += align256((size_t)(E + 1) * 4);
+    L.chunk = o;      o += permute_ws_bytes(T, E);
+    L.perm = o;       o += align256(M * 4);
+    L.inv = o;        o += align256(M * 4);
+    L.w_perm = o;     o += align256(M * 4);
+    L.probs_t = o;    o += align256((size_t)E * (size_t)T * 4);
+    L.bitmaps = o;    o += align256((size_t)E * (size_t)moe::rounding::bitmap_words((int)T) * 4);
+    L.new_counts = o; o += align256((size_t)E * 4);
+    L.offsets2 = o;   o += align256((size_t)(E + 1) * 4);
+    L.tok = o;        o += align256(cap * 4);
+    L.w2 = o;         o += align256(cap * 4);
+    L.posmap = o;     o += align256((size_t)T * (size_t)E * 4);
+    L.x_perm = o;     o += align256(cap * (size_t)d * 2);
+    L.h = o;          o += align256(cap * (size_t)f * 2);
+    L.y = o;          o += align256(cap * (size_t)d * 2);
+    L.total = o;
+    return L;
+}
+
+int forward_rounded_impl(const moe_bf16* x, const moe_bf16* w_router, const float* bias, const moe_bf16* w_gate,
+                         const moe_bf16* w_up, const moe_bf16* w_down, int64_t T, int64_t d, int64_t E, int64_t k,
+                         int64_t f, int64_t tile, float* out, int32_t* counts_out, int32_t* posmap_out, void* ws,
+                         size_t ws_bytes, cudaStream_t s, cudaEvent_t* ev, int n_ev)
+{
+    int rc = check_common(T, d, E, k);
+    if (rc) return rc;
+    if ((rc = check_f(f))) return rc;
+    if ((rc = check_rounding(T, E, k, tile))) return rc;
+    if (T > 0 && (!x || !w_router || !w_gate || !w_up || !w_down || !out)) return MOE_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(w_router, 16) || !aligned(w_gate, 16) || !aligned(w_up, 16) ||
+        !aligned(w_down, 16) || !aligned(out, 16) || !aligned(bias, 4) || !aligned(counts_out, 4) ||
+        !aligned(posmap_out, 4))
+        return MOE_ERR_INVALID_ARG;
+    if (ev && n_ev < 6) return MOE_ERR_INVALID_ARG;
+    const RLayout L = plan_rounded(T, d, E, k, f, tile);
+    if (T > 0 && (!ws || !aligned(ws, 256))) return MOE_ERR_INVALID_ARG;
+    if (ws_bytes < L.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
+    DeviceState* st = nullptr;
+    if ((rc = setup_device(&st))) return rc;
+    auto rec = [&](int i) {
+        return (ev && ev[i] && cudaEventRecord(ev[i], s) != cudaSuccess) ? MOE_ERR_CUDA : MOE_OK;
+    };
+    if ((rc = rec(0))) return rc;
+    if (T == 0) {
+        if (counts_out && cudaMemsetAsync(counts_out, 0, (size_t)E * 4, s) != cudaSuccess) return MOE_ERR_CUDA;
+        for (int i = 1; i < 6; ++i)
+            if ((rc = rec(i))) return rc;
+        return MOE_OK;
+    }
+    uint8_t* w = static_cast<uint8_t*>(ws);
+    auto at = [&](size_t off) { return static_cast<void*>(w + off); };
+    int32_t* ids = static_cast<int32_t*>(at(L.ids));
+    float* wts = static_cast<float*>(at(L.wts));
+    int32_t* counts = static_cast<int32_t*>(at(L.counts));
+    int32_t* offsets = static_cast<int32_t*>(at(L.offsets));
+    int32_t* chunk = static_cast<int32_t*>(at(L.chunk));
+    int32_t* perm = static_cast<int32_t*>(at(L.perm));
+    int32_t* inv = static_cast<int32_t*>(at(L.inv));
+    float* w_perm = static_cast<float*>(at(L.w_perm));
+    float* probs_t = static_cast<float*>(at(L.probs_t));
+    uint32_t* bitmaps = static_cast<uint32_t*>(at(L.bitmaps));
+    int32_t* new_counts = counts_out ? counts_out : static_cast<int32_t*>(at(L.new_counts));
+    int32_t* offsets2 = static_cast<int32_t*>(at(L.offsets2));
+    int32_t* tok = static_cast<int32_t*>(at(L.tok));
+    float* w2 = static_cast<float*>(at(L.w2));
+    int32_t* posmap = posmap_out ? posmap_out : static_cast<int32_t*>(at(L.posmap));
+    moe_bf16* x_perm = static_cast<moe_bf16*>(at(L.x_perm));
+    moe_bf16* h = static_cast<moe_bf16*>(at(L.h));
+    moe_f16* y = static_cast<moe_f16*>(at(L.y));
+    const int64_t cap = round_capacity(T, E, k, tile);
+    using namespace moe::rounding;
+
+    if ((rc = run_route(*st, x, w_router, bias, T, d, E, k, ids, wts, chunk, false, s, probs_t))) return rc;
+    if ((rc = rec(1))) return rc;
+    if ((rc = run_permute(x, ids, wts, T, d, E, k, counts, offsets, perm, inv, nullptr, w_perm, chunk, true, s)))
+        return rc;
+    const int iT = (int)T, iE = (int)E;
+    if (launch(round_kernel, dim3((unsigned)E), dim3(kThreads), round_smem_bytes(iT), s, 1u,
+               static_cast<const int32_t*>(offsets), static_cast<const int32_t*>(perm), (int)k,
+               static_cast<const float*>(probs_t), iT, iE, (int)tile, bitmaps, new_counts))
+        return MOE_ERR_CUDA;
+    if (launch(scan_kernel, dim3(1), dim3(kThreads), 0, s, 1u, static_cast<const int32_t*>(new_counts), iE, offsets2))
+        return MOE_ERR_CUDA;
+    if (launch(place_kernel, dim3((unsigned)E), dim3(kThreads), 0, s, 1u, static_cast<const uint32_t*>(bitmaps),
+               static_cast<const int32_t*>(offsets2), static_cast<const float*>(probs_t), iT, iE, cap, tok, w2,
+               posmap))
+        return MOE_ERR_CUDA;
+    if (launch(gather_rows_kernel, dim3((unsigned)((cap + 7) / 8)), dim3(256), 0, s, 1u,
+               reinterpret_cast<const uint4*>(x), static_cast<const int32_t*>(tok),
+               static_cast<const int32_t*>(offsets2), iE, T, cap, (int)(d / 8), reinterpret_cast<uint4*>(x_perm)))
+        return MOE_ERR_CUDA;
+    if ((rc = rec(2))) return rc;
+    if ((rc = run_ffn(*st, x_perm, nullptr, nullptr, T, k, w2, offsets2, w_gate, w_up, w_down, cap, d, E, f, h, y, s,
+                      ev ? ev[3] : nullptr, true)))
+        return rc;
+    if ((rc = rec(4))) return rc;
+    const int nvec = (int)(d / 8);
+    const int threads = nvec < 256 ? ((nvec + 31) / 32) * 32 : 256;
+    if (launch(combine_masked_kernel, dim3((unsigned)T), dim3(threads), 0, s, 1u, reinterpret_cast<const uint4*>(y),
+               static_cast<const int32_t*>(posmap), iE, cap, nvec, reinterpret_cast<float4*>(out)))
+        return MOE_ERR_CUDA;
+    return rec(5);
+}
+
 // ------------------------------------------- fixed scratch for moe_permute_static
 // Some callers cannot allocate device memory when they run the permutation:
 // for example a plugin inside an inference engine that plans all device
@@ -591,7 +726,7 @@ const char* moe_strerror(int status)
     }
 }
 
-int moe_version(void) { return 202; }
+int moe_version(void) { return 203; }
 
 size_t moe_workspace_size(int64_t T, int64_t d, int64_t E, int64_t k, int64_t f)
 {
@@ -762,6 +897,22 @@ int moe_forward_shared(const moe_bf16* x, const moe_bf16* w_router, const float*
     return forward_impl(x, w_router, bias, w_gate, w_up, w_down, T, d, E, k, f, out, topk_ids_out, topk_w_out,
                         workspace, workspace_bytes, stream, events, n_events, flags, w_gate_s, w_up_s, w_down_s,
                         n_shared, f_shared);
+}
+
+size_t moe_workspace_size_rounded(int64_t T, int64_t d, int64_t E, int64_t k, int64_t f, int64_t tile)
+{
+    if (check_common(T, d, E, k) || check_f(f) || check_rounding(T, E, k, tile)) return 0;
+    return plan_rounded(T, d, E, k, f, tile).total;
+}
+
+int moe_forward_rounded(const moe_bf16* x, const moe_bf16* w_router, const float* bias, const moe_bf16* w_gate,
+                        const moe_bf16* w_up, const moe_bf16* w_down, int64_t T, int64_t d, int64_t E, int64_t k,
+                        int64_t f, int64_t tile, float* out, int32_t* counts_out, int32_t* rows_out,
+                        void* workspace, size_t workspace_bytes, cudaStream_t stream, cudaEvent_t* events,
+                        int n_events)
+{
+    return forward_rounded_impl(x, w_router, bias, w_gate, w_up, w_down, T, d, E, k, f, tile, out, counts_out,
+                                rows_out, workspace, workspace_bytes, stream, events, n_events);
 }
 
 int moe_forward(const moe_bf16* x, const moe_bf16* w_router, const float* bias, const moe_bf16* w_gate,

@@ -70,6 +70,7 @@ struct Params {
     int split;               // CTAs per tile: 1, or 2 (cluster of two, split K)
     int passes;              // row passes of the exchange buffer (1, or 2 when split == 1 and E > 256)
     int renorm;              // 1: divide each token's k weights by their sum
+    float* probs_t;          // [E][T]: every expert's probability (token rounding), or nullptr
 };
 
 __host__ __device__ inline int stage_bytes(int n_chunks) { return kABytes + n_chunks * kChunkBytes; }
@@ -115,7 +116,8 @@ __device__ __forceinline__ bool ranks_before(float v, int i, float w, int j) { r
 // logit of expert lane + 32 j (called only for lane + 32 j < E).  Lane
 // j < k receives slot j.
 template <int VPL, typename Logit>
-__device__ __forceinline__ void warp_topk(int E, int k, bool renorm, int lane, Logit col, int& my_id, float& my_w)
+__device__ __forceinline__ void warp_topk(int E, int k, bool renorm, int lane, Logit col, int& my_id, float& my_w,
+                                          float* pcol, int64_t pstride)
 {
     float v[VPL];
     unsigned taken = 0;  // bit j: value j is not a candidate
@@ -140,6 +142,11 @@ __device__ __forceinline__ void warp_topk(int E, int k, bool renorm, int lane, L
         if (!((taken >> j) & 1u)) sum += expf(v[j] - mx);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    if (pcol) {  // every expert's probability, by the same formula as the weights below
+#pragma unroll
+        for (int j = 0; j < VPL; ++j)
+            if (!((taken >> j) & 1u)) pcol[(int64_t)(lane + 32 * j) * pstride] = expf(v[j] - mx) / sum;
+    }
     my_id = 0;
     my_w = 0.0f;
     for (int slot = 0; slot < k; ++slot) {
@@ -243,7 +250,8 @@ __device__ __forceinline__ void merge_partner(float (&v)[KMAX], int (&ix)[KMAX],
 // Softmax and top-k of one token by a group of L lanes (lane j of the group
 // = lane % L); `logit(c)` is expert c's logit.  Lane j < k receives slot j.
 template <int L, int KMAX, typename Logit>
-__device__ __forceinline__ void group_topk(int E, int k, bool renorm, int j, Logit logit, int& my_id, float& my_w)
+__device__ __forceinline__ void group_topk(int E, int k, bool renorm, int j, Logit logit, int& my_id, float& my_w,
+                                           float* pcol, int64_t pstride)
 {
     float v[KMAX];
     int ix[KMAX];
@@ -264,6 +272,8 @@ __device__ __forceinline__ void group_topk(int E, int k, bool renorm, int j, Log
     for (int c = j; c < E; c += L) sum += __expf(logit(c) - mx);
 #pragma unroll
     for (int o = L / 2; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    if (pcol)  // every expert's probability, by the same formula as the weights below
+        for (int c = j; c < E; c += L) pcol[c * pstride] = __expf(logit(c) - mx) / sum;
 #pragma unroll
     for (int o = 1; o < L; o <<= 1) merge_partner<KMAX>(v, ix, o);
     my_id = ix[0];
@@ -303,7 +313,7 @@ __device__ __forceinline__ void topk_rows(const Params& p, const float* buf, con
             float l = col[0];
             for (int s = 1; s < S; ++s) l += col[(size_t)s * E * pitch];
             return l + s_bias[c];
-        }, my_id, my_w);
+        }, my_id, my_w, (p.probs_t && ok && t < p.T) ? p.probs_t + t : nullptr, (int64_t)p.T);
         if (ok && t < p.T && j < p.k) {
             p.ids[t * p.k + j] = my_id;
             p.wts[t * p.k + j] = my_w;
@@ -499,7 +509,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     float l = col[0];
                     for (int s = 1; s < S; ++s) l += col[(size_t)s * E * pitch];
                     return l + s_bias[c];
-                }, my_id, my_w);
+                }, my_id, my_w, (p.probs_t && ok) ? p.probs_t + t : nullptr, (int64_t)p.T);
                 if (ok && lane < p.k) {
                     p.ids[t * p.k + lane] = my_id;
                     p.wts[t * p.k + lane] = my_w;
