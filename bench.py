@@ -302,7 +302,18 @@ def run_gpu(args, cfg):
             blk(xin, out=out, topk_ids=topk_ids, events=events)
     else:
         flags = moe.MOE_FLAG_FUSED_GATHER if args.gather else 0
-        if args.shared > 0:
+        if args.round > 0:
+            ws_rd = None
+            counts_rd = torch.empty(cfg.E, dtype=torch.int32, device=dev)
+
+            def fwd(xin, events=None, topk_ids=None):
+                nonlocal ws_rd
+                if ws_rd is None:
+                    nb = moe.lib().moe_workspace_size_rounded(cfg.T, cfg.d, cfg.E, cfg.k, cfg.f, args.round)
+                    ws_rd = torch.empty(int(nb), dtype=torch.uint8, device=dev)
+                moe.forward_rounded(xin, w["W_router"], w["W_gate"], w["W_up"], w["W_down"], cfg.k, tile=args.round,
+                                    bias=bias, out=out, workspace=ws_rd, counts=counts_rd, events=events)
+        elif args.shared > 0:
             from top_routing_grouped_softmax_b200.synth import make_shared_weights
             sw = {n: t.to(dev) for n, t in make_shared_weights(cfg, args.shared).items()}
             ws_sh = None
@@ -362,12 +373,17 @@ def run_gpu(args, cfg):
     total_s = sum(step_ms) / 1e3
 
     # expert load statistics of the batch
+    rounded_rows = None
+    if args.round > 0:
+        moe.route(x, w["W_router"], cfg.k, bias=bias, topk_ids=ids)   # top-k ids for the report (untimed)
+        rounded_rows = int(counts_rd.sum().item())
     counts = torch.bincount(ids.flatten().long(), minlength=cfg.E).cpu()
     active = int((counts > 0).sum())
     # the grouped GEMMs run 256-row CTA-pair tiles: rows past a group's end
     # are computed and not stored
-    tiles = int(((counts + 255) // 256).sum())
-    padding = 1.0 - cfg.T * cfg.k / (tiles * 256)
+    gemm_counts = counts_rd.cpu() if args.round > 0 else counts
+    tiles = int(((gemm_counts + 255) // 256).sum())
+    padding = 1.0 - int(gemm_counts.sum()) / max(1, tiles * 256)
 
     # ---- end to end through the public API, host buffers, copies timed
     x_host = inp.x.pin_memory()
@@ -405,6 +421,12 @@ def run_gpu(args, cfg):
     if rank == 0:
         peaks = load_peaks()
         alg = algorithmic(cfg, active, args.shared)
+        if rounded_rows is not None:
+            # token rounding changes the number of (token, expert) rows the GEMMs compute
+            scale = rounded_rows / (cfg.T * cfg.k)
+            alg["gateup_flops"] = int(alg["gateup_flops"] * scale)
+            alg["down_flops"] = int(alg["down_flops"] * scale)
+            alg["flops"] = 2 * cfg.T * cfg.d * cfg.E + alg["gateup_flops"] + alg["down_flops"]
         ms = 1e3 * total_s / args.steps
         tok_s = whole_job_rate(cfg.T * args.steps, world, [total_s])
         # --path stages times both GEMMs together (moe_expert_ffn is one call)
@@ -424,7 +446,11 @@ def run_gpu(args, cfg):
             "metric": METRIC, "value": tok_s, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": workload_config(cfg, extra={"out_dtype": "fp32", **({"shared_experts": args.shared,
+            "config": workload_config(cfg, extra={"out_dtype": "fp32",
+                                                  **({"routing": f"token rounding to {args.round}-row tiles "
+                                                                 "(an approximation of the block)",
+                                                      "rounded_rows": rounded_rows} if args.round else {}),
+                                                  **({"shared_experts": args.shared,
                                                                              "f_shared": cfg.f}
                                                                           if args.shared else {})}),
             "tflops": alg["flops"] / (ms * 1e-3) / 1e12,
@@ -451,7 +477,7 @@ def run_gpu(args, cfg):
                         "pair_tile_padding": padding},
             "e2e": {"value": whole_job_rate(cfg.T * args.steps, world, [e2e_s]), "unit": UNIT,
                     "h2d_bytes_per_step": cfg.T * cfg.d * 2, "d2h_bytes_per_step": cfg.T * cfg.d * 4},
-            "gpu_launches": (KERNELS_PER_FORWARD + 2 * args.shared) * args.steps,
+            "gpu_launches": (KERNELS_PER_FORWARD + 2 * args.shared + (3 if args.round else 0)) * args.steps,
             "clocks": clocks,
             "wall_s_timed_region": wall,
         }
@@ -469,6 +495,8 @@ def main(argv=None):
     ap.add_argument("--workload", default="qwen")
     ap.add_argument("--path", choices=("fused", "stages"), default="fused",
                     help="fused: moe_forward; stages: moe_route/permute/expert_ffn/combine one by one")
+    ap.add_argument("--round", type=int, default=0,
+                    help="token rounding to this tile (e.g. 256): an approximation of the block, reported apart")
     ap.add_argument("--shared", type=int, default=0,
                     help="add this many shared experts (weight one, every token, intermediate size f)")
     ap.add_argument("--gather", action="store_true",

@@ -554,7 +554,7 @@ int check_rounding(int64_t T, int64_t E, int64_t k, int64_t tile)
 }
 
 struct RLayout {
-    size_t ids, wts, counts, offsets, chunk, perm, inv, w_perm, probs_t, bitmaps, new_counts, offsets2, tok, w2,
+    size_t ids, wts, counts, offsets, chunk, perm, inv, w_perm, probs_t, bitmaps, new_counts, offsets2, w2,
         posmap, x_perm, h, y, total;
 };
 
@@ -576,7 +576,6 @@ RLayout plan_rounded(int64_t T, int64_t d, int64_t E, int64_t k, int64_t f, int6
     L.bitmaps = o;    o += align256((size_t)E * (size_t)moe::rounding::bitmap_words((int)T) * 4);
     L.new_counts = o; o += align256((size_t)E * 4);
     L.offsets2 = o;   o += align256((size_t)(E + 1) * 4);
-    L.tok = o;        o += align256(cap * 4);
     L.w2 = o;         o += align256(cap * 4);
     L.posmap = o;     o += align256((size_t)T * (size_t)E * 4);
     L.x_perm = o;     o += align256(cap * (size_t)d * 2);
@@ -630,7 +629,6 @@ int forward_rounded_impl(const moe_bf16* x, const moe_bf16* w_router, const floa
     uint32_t* bitmaps = static_cast<uint32_t*>(at(L.bitmaps));
     int32_t* new_counts = counts_out ? counts_out : static_cast<int32_t*>(at(L.new_counts));
     int32_t* offsets2 = static_cast<int32_t*>(at(L.offsets2));
-    int32_t* tok = static_cast<int32_t*>(at(L.tok));
     float* w2 = static_cast<float*>(at(L.w2));
     int32_t* posmap = posmap_out ? posmap_out : static_cast<int32_t*>(at(L.posmap));
     moe_bf16* x_perm = static_cast<moe_bf16*>(at(L.x_perm));
@@ -650,13 +648,14 @@ int forward_rounded_impl(const moe_bf16* x, const moe_bf16* w_router, const floa
         return MOE_ERR_CUDA;
     if (launch(scan_kernel, dim3(1), dim3(kThreads), 0, s, 1u, static_cast<const int32_t*>(new_counts), iE, offsets2))
         return MOE_ERR_CUDA;
+    if (cudaMemsetAsync(posmap, 0xff, (size_t)T * (size_t)E * 4, s) != cudaSuccess) return MOE_ERR_CUDA;  // -1
     if (launch(place_kernel, dim3((unsigned)E), dim3(kThreads), 0, s, 1u, static_cast<const uint32_t*>(bitmaps),
-               static_cast<const int32_t*>(offsets2), static_cast<const float*>(probs_t), iT, iE, cap, tok, w2,
+               static_cast<const int32_t*>(offsets2), static_cast<const float*>(probs_t), iT, iE, cap, w2,
                posmap))
         return MOE_ERR_CUDA;
-    if (launch(gather_rows_kernel, dim3((unsigned)((cap + 7) / 8)), dim3(256), 0, s, 1u,
-               reinterpret_cast<const uint4*>(x), static_cast<const int32_t*>(tok),
-               static_cast<const int32_t*>(offsets2), iE, T, cap, (int)(d / 8), reinterpret_cast<uint4*>(x_perm)))
+    if (launch(gather_rows_kernel, dim3((unsigned)((T + 7) / 8)), dim3(256), 0, s, 1u,
+               reinterpret_cast<const uint4*>(x), static_cast<const int32_t*>(posmap), iE, T, cap, (int)(d / 8),
+               reinterpret_cast<uint4*>(x_perm)))
         return MOE_ERR_CUDA;
     if ((rc = rec(2))) return rc;
     if ((rc = run_ffn(*st, x_perm, nullptr, nullptr, T, k, w2, offsets2, w_gate, w_up, w_down, cap, d, E, f, h, y, s,

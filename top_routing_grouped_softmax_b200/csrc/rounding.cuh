@@ -23,9 +23,10 @@
 //                 with the new count.
 //   scan_kernel   exclusive scan of the new counts -> group offsets.
 //   place_kernel  one CTA per expert: walks its bitmap in token order and
-//                 writes the grouped rows (token, weight) and posmap[t][e]
-//                 (the row of (t, e), or -1).
-//   gather_rows   x_perm[pos] = x[tok[pos]] in row order (warp per row).
+//                 writes the grouped rows' weights and posmap[t][e]
+//                 (the row of (t, e); -1, set by a memset, elsewhere).
+//   gather_rows   x_perm[posmap[t][e]] = x[t]: a warp per token reads its row
+//                 once and writes it to each of the token's rows.
 //   combine_kernel_masked: out[t] = sum over e ascending with posmap[t][e] >= 0
 //                 of y[posmap[t][e]] (fp16 rows widened, fp32 sum).
 #pragma once
@@ -43,8 +44,15 @@ constexpr int kMaxTokens = 1 << 20;   // bitmap of one expert: 128 KB of shared 
 
 __host__ __device__ inline int bitmap_words(int T) { return (T + 31) / 32; }
 
-// Shared memory of round_kernel: 64 B of scratch, 256 histogram bins, bitmap words.
-__host__ inline size_t round_smem_bytes(int T) { return (size_t)bitmap_words(T) * 4 + 256 * 4 + 64; }
+// Shared memory of round_kernel: 64 B of scratch, 256 histogram bins, bitmap
+// words and, when T <= kCachedTokens, the expert's probability row (read by
+// all eight radix passes).
+constexpr int kCachedTokens = 40960;
+__host__ __device__ inline bool round_caches_row(int T) { return T <= kCachedTokens; }
+__host__ inline size_t round_smem_bytes(int T)
+{
+    return 64 + 256 * 4 + (size_t)bitmap_words(T) * 4 + (round_caches_row(T) ? (size_t)T * 4 : 0);
+}
 
 __device__ __forceinline__ uint64_t round_key(float p, int t)
 {
@@ -63,10 +71,16 @@ __device__ uint64_t select_kth(int n, int m, Cand cand, int* hist, unsigned long
         const uint64_t hi_mask = shift == 56 ? 0ull : (~0ull << (shift + 8));
         for (int i = threadIdx.x; i < 256; i += kThreads) hist[i] = 0;
         __syncthreads();
-        for (int i = threadIdx.x; i < n; i += kThreads) {
-            uint64_t key;
-            if (!cand(i, key)) continue;
-            if ((key & hi_mask) == (prefix & hi_mask)) atomicAdd(&hist[(key >> shift) & 255u], 1);
+        // warp-aggregated: the lanes with the same digit add once (most keys
+        // share their top bytes, so per-lane atomics would serialise)
+        const int lane = threadIdx.x & 31;
+        for (int i0 = threadIdx.x - lane; i0 < n; i0 += kThreads) {
+            const int i = i0 + lane;
+            uint64_t key = 0;
+            const bool live = i < n && cand(i, key) && (key & hi_mask) == (prefix & hi_mask);
+            const int digit = live ? (int)((key >> shift) & 255u) : -1;
+            const unsigned peers = __match_any_sync(0xffffffffu, digit);
+            if (live && (__ffs(peers) - 1) == lane) atomicAdd(&hist[digit], __popc(peers));
         }
         __syncthreads();
         if (threadIdx.x < 32) {
@@ -117,10 +131,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     unsigned long long* sh = reinterpret_cast<unsigned long long*>(smem_raw);  // 8 words (64 B), 8-byte aligned
     int* hist = reinterpret_cast<int*>(smem_raw + 64);                        // 256 bins
     uint32_t* bits = reinterpret_cast<uint32_t*>(smem_raw + 64 + 256 * 4);    // nw words
+    float* s_p = reinterpret_cast<float*>(bits + nw);                          // T floats when cached
+    const bool cached = round_caches_row(T);
     const int e = blockIdx.x;
     pdl_trigger();
     pdl_wait();
     for (int i = threadIdx.x; i < nw; i += kThreads) bits[i] = 0u;
+    if (cached)
+        for (int t = threadIdx.x; t < T; t += kThreads) s_p[t] = __ldg(probs_t + (int64_t)e * T + t);
     __syncthreads();
     const int g0 = __ldg(offsets + e), g1 = __ldg(offsets + e + 1);
     const int c = g1 - g0;
@@ -140,7 +158,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = threadIdx.x; i < nw; i += kThreads) bits[i] = 0u;
         __syncthreads();
     }
-    const float* pe = probs_t + (int64_t)e * T;
+    const float* pe = cached ? s_p : probs_t + (int64_t)e * T;
     const int r = bad ? 0 : c % R;
     const int add = R - r;
     if (r != 0) {
@@ -149,23 +167,23 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int n = T - c;
             const uint64_t kth = select_kth(T, n - add + 1, [&](int t, uint64_t& key) {
                 if ((bits[t >> 5] >> (t & 31)) & 1u) return false;
-                key = round_key(__ldg(pe + t), t);
+                key = round_key(pe[t], t);
                 return true;
             }, hist, sh);
             __syncthreads();
             for (int t = threadIdx.x; t < T; t += kThreads)
-                if (!((bits[t >> 5] >> (t & 31)) & 1u) && round_key(__ldg(pe + t), t) >= kth)
+                if (!((bits[t >> 5] >> (t & 31)) & 1u) && round_key(pe[t], t) >= kth)
                     atomicOr(&bits[t >> 5], 1u << (t & 31));
         } else {
             const uint64_t kth = select_kth(c, r, [&](int i, uint64_t& key) {
                 const int t = __ldg(perm + g0 + i) / k;
-                key = round_key(__ldg(pe + t), t);
+                key = round_key(pe[t], t);
                 return true;
             }, hist, sh);
             __syncthreads();
             for (int i = threadIdx.x; i < c; i += kThreads) {
                 const int t = __ldg(perm + g0 + i) / k;
-                if (round_key(__ldg(pe + t), t) <= kth) atomicAnd(&bits[t >> 5], ~(1u << (t & 31)));
+                if (round_key(pe[t], t) <= kth) atomicAnd(&bits[t >> 5], ~(1u << (t & 31)));
             }
         }
     }
@@ -219,14 +237,13 @@ __global__ void __launch_bounds__(kThreads) scan_kernel(const int32_t* __restric
     if (tid == 0) offsets[E] = s_warp[kWarps - 1];
 }
 
-// One CTA per expert: group e's rows, in token order.  tok[pos] = t,
-// w[pos] = p[t][e], posmap[t * E + e] = pos (or -1 for every token not in
-// the group).
+// One CTA per expert: group e's rows, in token order: w[pos] = p[t][e] and
+// posmap[t * E + e] = pos (the caller fills posmap with -1 first).
 __global__ void __launch_bounds__(kThreads) place_kernel(const uint32_t* __restrict__ bitmaps,
                                                           const int32_t* __restrict__ offsets,
                                                           const float* __restrict__ probs_t, int T, int E,
-                                                          int64_t capacity, int32_t* __restrict__ tok,
-                                                          float* __restrict__ w, int32_t* __restrict__ posmap)
+                                                          int64_t capacity, float* __restrict__ w,
+                                                          int32_t* __restrict__ posmap)
 {
     __shared__ int s_warp[kWarps];
     __shared__ int s_carry;
@@ -267,14 +284,13 @@ __global__ void __launch_bounds__(kThreads) place_kernel(const uint32_t* __restr
             for (int b = 0; b < 32; ++b) {
                 const int t = wi * 32 + b;
                 if (t >= T) break;
-                if (((word >> b) & 1u) && (unsigned long long)(unsigned)pos < (unsigned long long)capacity) {
-                    tok[pos] = t;
-                    w[pos] = __ldg(pe + t);
+                if (!((word >> b) & 1u)) continue;  // posmap was filled with -1 beforehand
+                if ((unsigned long long)(unsigned)pos < (unsigned long long)capacity) {
+                    w[pos] = pe[t];
                     posmap[(int64_t)t * E + e] = pos;
                     ++pos;
                 } else {
-                    if ((word >> b) & 1u) record_status(kStatusDeviceBounds);
-                    posmap[(int64_t)t * E + e] = -1;
+                    record_status(kStatusDeviceBounds);
                 }
             }
         }
@@ -284,25 +300,48 @@ __global__ void __launch_bounds__(kThreads) place_kernel(const uint32_t* __restr
     }
 }
 
-// x_perm[pos] = x[tok[pos]] for pos < offsets[E]; one warp per row.
-__global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restrict__ x, const int32_t* __restrict__ tok,
-                                                           const int32_t* __restrict__ offsets, int E, int64_t T,
+// x_perm[posmap[t][e]] = x[t] for every row of token t: one warp per token
+// reads the row once (16-byte vectors, eight in flight per lane) and writes
+// it to each of the token's rows, found 32 experts at a time with a ballot.
+__global__ void __launch_bounds__(256) gather_rows_kernel(const uint4* __restrict__ x,
+                                                           const int32_t* __restrict__ posmap, int E, int64_t T,
                                                            int64_t capacity, int nvec, uint4* __restrict__ x_perm)
 {
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    const int64_t row = (int64_t)blockIdx.x * 8 + warp;   // the launch covers `capacity` rows
+    const int64_t t = (int64_t)blockIdx.x * 8 + warp;
     pdl_trigger();
     pdl_wait();
-    if (row >= capacity || row >= __ldg(offsets + E)) return;
-    const int t = __ldg(tok + row);
-    if ((unsigned long long)(unsigned)t >= (unsigned long long)T) {
-        record_status(kStatusDeviceBounds);
-        return;
+    if (t >= T) return;
+    const uint4* src = x + t * nvec;
+    constexpr int kUnroll = 8;
+    for (int v0 = 0; v0 < nvec; v0 += 32 * kUnroll) {
+        uint4 buf[kUnroll];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const int v = v0 + u * 32 + lane;
+            if (v < nvec) buf[u] = __ldg(src + v);
+        }
+        for (int e0 = 0; e0 < E; e0 += 32) {
+            const int e = e0 + lane;
+            int pos = e < E ? __ldg(posmap + t * E + e) : -1;
+            if (pos >= 0 && (unsigned long long)pos >= (unsigned long long)capacity) {
+                record_status(kStatusDeviceBounds);
+                pos = -1;
+            }
+            unsigned m = __ballot_sync(0xffffffffu, pos >= 0);
+            while (m) {  // warp-uniform
+                const int src_lane = __ffs(m) - 1;
+                m &= m - 1;
+                const int pj = __shfl_sync(0xffffffffu, pos, src_lane);
+                uint4* dst = x_perm + (int64_t)pj * nvec;
+#pragma unroll
+                for (int u = 0; u < kUnroll; ++u) {
+                    const int v = v0 + u * 32 + lane;
+                    if (v < nvec) dst[v] = buf[u];
+                }
+            }
+        }
     }
-    const uint4* src = x + (int64_t)t * nvec;
-    uint4* dst = x_perm + row * nvec;
-#pragma unroll 8
-    for (int v = lane; v < nvec; v += 32) dst[v] = __ldg(src + v);
 }
 
 // out[t] = sum over experts e ascending with posmap[t][e] >= 0 of y[row]
@@ -313,28 +352,45 @@ __global__ void __launch_bounds__(256) combine_masked_kernel(const uint4* __rest
                                                               int64_t rows, int nvec, float4* __restrict__ out)
 {
     __shared__ int s_pos[512];
-    __shared__ int s_n;
+    __shared__ int s_chunk[17];  // per 32-expert chunk: its row count, then the exclusive prefix; [16]: total
     const int64_t t = blockIdx.x;
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int nwarps = blockDim.x / 32;
+    const int nchunks = (E + 31) / 32;
     pdl_trigger();
     pdl_wait();
-    if (threadIdx.x < 32) {
-        const int lane = threadIdx.x;
-        int n = 0;
-        for (int e0 = 0; e0 < E; e0 += 32) {
-            const int e = e0 + lane;
-            int p = e < E ? __ldg(posmap + t * E + e) : -1;
-            if (p >= 0 && (unsigned long long)p >= (unsigned long long)rows) {
-                record_status(kStatusDeviceBounds);
-                p = -1;
-            }
-            const unsigned m = __ballot_sync(0xffffffffu, p >= 0);
-            if (p >= 0) s_pos[n + __popc(m & ((1u << lane) - 1u))] = p;
-            n += __popc(m);
+    auto row_of = [&](int e) {
+        int p = e < E ? __ldg(posmap + t * E + e) : -1;
+        if (p >= 0 && (unsigned long long)p >= (unsigned long long)rows) {
+            record_status(kStatusDeviceBounds);
+            p = -1;
         }
-        if (lane == 0) s_n = n;
+        return p;
+    };
+    // the token's rows, compacted in ascending expert order by all warps:
+    // chunk counts, their prefix, then each chunk writes at its offset
+    for (int ch = warp; ch < nchunks; ch += nwarps) {
+        const unsigned m = __ballot_sync(0xffffffffu, row_of(ch * 32 + lane) >= 0);
+        if (lane == 0) s_chunk[ch] = __popc(m);
     }
     __syncthreads();
-    const int n = s_n;
+    if (threadIdx.x == 0) {
+        int run = 0;
+        for (int ch = 0; ch < nchunks; ++ch) {
+            const int c = s_chunk[ch];
+            s_chunk[ch] = run;
+            run += c;
+        }
+        s_chunk[16] = run;
+    }
+    __syncthreads();
+    for (int ch = warp; ch < nchunks; ch += nwarps) {
+        const int p = row_of(ch * 32 + lane);
+        const unsigned m = __ballot_sync(0xffffffffu, p >= 0);
+        if (p >= 0) s_pos[s_chunk[ch] + __popc(m & ((1u << lane) - 1u))] = p;
+    }
+    __syncthreads();
+    const int n = s_chunk[16];
     for (int v = threadIdx.x; v < nvec; v += blockDim.x) {
         float acc[8];
 #pragma unroll
