@@ -301,6 +301,7 @@ __device__ __forceinline__ void topk_rows(const Params& p, const float* buf, con
                                           int S, int own, int pitch, int tile0, int row0, bool ok, int warp,
                                           int lane)
 {
+    static_assert(L >= KMAX, "lane j of a group writes slot j: a group needs at least k lanes");
     const int E = p.E;
     const int j = lane % L;
     for (int i = warp * (32 / L) + lane / L; i - lane / L < own; i += kWarps * (32 / L)) {
@@ -492,7 +493,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncthreads();
         // softmax + top-k of the rows this CTA owns in this pass
         const int row0 = S > 1 ? (int)r * own : pass * own;
-        if (KMAX <= 8) {
+        if constexpr (KMAX <= 8) {
             if (own == 128)
                 topk_rows<8, KMAX>(p, buf, s_bias, s_hist, S, own, pitch, tile0, row0, ok, warp, lane);
             else
