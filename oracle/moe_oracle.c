@@ -36,6 +36,11 @@
  *   x [T][d], W_router [d][E], bias [E] (fp32, may be NULL),
  *   W_gate [E][d][f], W_up [E][d][f], W_down [E][f][d].
  *
+ * Optional variants, each off the article's path and pinned like the rest:
+ * oracle_renormalize (renormalised top-k weights), oracle_shared_rows
+ * (shared experts), oracle_round_tokens and oracle_masked_rows (token
+ * rounding).
+ *
  * Parity status: every function here is pinned by CPU tests against
  * independent computations (brute force, library routines, invariants and
  * special cases); nothing is "parity unpinned".

@@ -152,3 +152,31 @@ def test_forward_renormalized(cfg):
     keep = ~excluded
     value_check(out.double().cpu().numpy()[keep], ex.out[keep], f"out[{cfg.name}, renormalised]")
     np.testing.assert_allclose(w.cpu().numpy().sum(axis=1), 1.0, rtol=0, atol=cfg.k * 5e-5)
+
+
+def test_forward_cuda_graph_replay_equals_eager():
+    """moe_forward captured in a CUDA graph (its launches carry the
+    programmatic-dependent-launch attribute) replays bit-identically to the
+    eager call, also after the input changes in place."""
+    cfg = SMALL[0]
+    d = gc.on_device(gc.inputs(cfg))
+    blk = moe.MoEBlock(d["w_router"], d["w_gate"], d["w_up"], d["w_down"], cfg.k, bias=d["bias"])
+    x = d["x"].clone()
+    out = torch.empty(cfg.T, cfg.d, dtype=torch.float32, device="cuda")
+    blk(x, out=out)                                   # eager: sets up the device and the workspace
+    torch.cuda.synchronize()
+    ref = out.clone()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        blk(x, out=out)
+    out.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    assert moe.get_status() == moe.MOE_OK
+    assert torch.equal(out, ref)
+    x2 = torch.flip(d["x"], dims=[0]).contiguous()
+    x.copy_(x2)
+    g.replay()
+    eager = blk(x2)
+    torch.cuda.synchronize()
+    assert torch.equal(out, eager)

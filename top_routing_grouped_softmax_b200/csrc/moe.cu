@@ -225,8 +225,10 @@ inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 // ---------------------------------------------------------- work shapes
 inline int64_t token_chunks(int64_t T) { return (T + moe::permute::kTokensPerChunk - 1) / moe::permute::kTokensPerChunk; }
 
-// The router keeps its logits on chip and needs no scratch; the workspace
-// argument of moe_route stays in the ABI for a future split-K router.
+// The router keeps its logits on chip (a CTA pair that splits K exchanges
+// its partial logits through distributed shared memory) and needs no
+// scratch; moe_route keeps its workspace argument so that every stage entry
+// point is sized the same way.
 size_t route_ws_bytes(int64_t, int64_t, int64_t) { return 0; }
 
 size_t permute_ws_bytes(int64_t T, int64_t E) { return align256((size_t)token_chunks(T) * (size_t)E * 4); }
