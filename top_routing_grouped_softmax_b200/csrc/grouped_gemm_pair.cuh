@@ -6,10 +6,12 @@
 // and a 256-column N tile.  Each CTA loads its own 128 rows of A and its own
 // half of the B tile (128 columns), so per SM a pipeline stage is 32 KB
 // instead of 48 KB for the same tensor work: less shared-memory fill and
-// L2->SM traffic per flop, and a deeper ring (6 stages).  The even CTA
-// issues the pair MMAs (M=256, N=256, K=16); each CTA's TMEM receives its own
-// 128 rows of the accumulator, so each CTA's epilogue drains its own rows
-// exactly like the single-CTA kernel.
+// L2->SM traffic per flop, and a deeper ring (6 stages).  The B half is
+// fetched by one 3-D copy (two 64-column chunks), so a CTA issues two
+// copies per stage.  The even CTA issues the pair MMAs (M=256, N=256,
+// K=16); each CTA's TMEM receives its own 128 rows of the accumulator, so
+// each CTA's epilogue drains its own rows exactly like the single-CTA
+// kernel.
 //
 // Synchronisation across the pair:
 //   full[s]      lives in the even CTA; both CTAs' TMA loads complete on it
@@ -129,16 +131,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint32_t bar = mapa_shared(&c.full[s], 0);
                     const int kr = krow0 + kb * kBK;
                     tma_load_2d_pair(sa, &tm_a, bar, kb * kBK, arow);
+                    // 128 weight columns as two 64-column chunks in one copy (the
+                    // weight maps view [K, N] as [N/64][K][64])
                     if (EPI == kSwiGLU) {
                         // even CTA: the gate columns, odd CTA: the matching up columns
                         const CUtensorMap* tb = leader ? &tm_b0 : &tm_b1;
-                        const int n0 = nt * 128;
-                        tma_load_2d_pair(sb, tb, bar, n0, kr);
-                        tma_load_2d_pair(sb + kChunkBytes, tb, bar, n0 + 64, kr);
+                        tma_load_3d_pair(sb, tb, bar, 0, kr, nt * 2);
                     } else {
-                        const int n0 = nt * kBN + (int)rank * 128;
-                        tma_load_2d_pair(sb, &tm_b0, bar, n0, kr);
-                        tma_load_2d_pair(sb + kChunkBytes, &tm_b0, bar, n0 + 64, kr);
+                        tma_load_3d_pair(sb, &tm_b0, bar, 0, kr, nt * (kBN / 64) + (int)rank * 2);
                     }
                     ++issued;
                     if (++s == kPairStages) {

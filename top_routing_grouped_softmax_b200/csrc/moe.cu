@@ -220,6 +220,22 @@ int make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, u
     return r == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
 }
 
+// A bf16 weight matrix [rows = k, cols] viewed as [cols/64][rows][64]
+// (64-column chunks outermost), 128-byte swizzle, box of 64 rows x two
+// chunks: one copy fetches 128 columns as the two 8 KB chunks an MN-major
+// operand uses.  Chunks past the last column read zeros.
+int make_weight_chunk_map(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows)
+{
+    cuuint64_t dims[3] = {64, rows, (cols + 63) / 64};
+    cuuint64_t strides[2] = {cols * 2, 128};
+    cuuint32_t box[3] = {64, 64, 2};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
+}
+
 inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
 // ---------------------------------------------------------- work shapes
@@ -381,6 +397,11 @@ int run_ffn(const DeviceState& st, const moe_bf16* x_perm, const moe_bf16* x_gat
     rc = rc ? rc : make_map(&td, w_down, (uint64_t)d, (uint64_t)(E * f), 64, 64);
     rc = rc ? rc : make_map(&ty, y, (uint64_t)d, (uint64_t)M, kSlabCols, 32, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
                             CU_TENSOR_MAP_SWIZZLE_64B);
+    // the CTA-pair kernels fetch weight columns in 128-column copies
+    CUtensorMap tg3, tu3, td3;
+    rc = rc ? rc : make_weight_chunk_map(&tg3, w_gate, (uint64_t)f, (uint64_t)(E * d));
+    rc = rc ? rc : make_weight_chunk_map(&tu3, w_up, (uint64_t)f, (uint64_t)(E * d));
+    rc = rc ? rc : make_weight_chunk_map(&td3, w_down, (uint64_t)d, (uint64_t)(E * f));
     if (rc) return rc;
     const size_t smem1 = smem_bytes<kSwiGLU>();
     const size_t smem2 = smem_bytes<kWeighted>();
@@ -404,7 +425,7 @@ int run_ffn(const DeviceState& st, const moe_bf16* x_perm, const moe_bf16* x_gat
     const unsigned grid1 = (unsigned)(work1 < st.sm_count ? work1 : st.sm_count);
     const int64_t max_pair_tiles = (M + kPairRows - 1) / kPairRows + E;
     if (MOE_GEMM_PAIR && !gather) {
-        if (launch_pair_gemm<kSwiGLU>(st, max_pair_tiles * p1.n_tiles, ta1, tg, tu, ty, p1, s)) return MOE_ERR_CUDA;
+        if (launch_pair_gemm<kSwiGLU>(st, max_pair_tiles * p1.n_tiles, ta1, tg3, tu3, ty, p1, s)) return MOE_ERR_CUDA;
     } else if (gather) {
         if (launch(grouped_gemm_kernel<kSwiGLU, true>, dim3(grid1), dim3(kThreads), smem1, s, 1u, ta1, tg, tu, ty, p1))
             return MOE_ERR_CUDA;
@@ -431,7 +452,7 @@ int run_ffn(const DeviceState& st, const moe_bf16* x_perm, const moe_bf16* x_gat
     p2.m_capacity = m_capacity ? 1 : 0;
     const int64_t work2 = max_mtiles * p2.n_tiles;
     const unsigned grid2 = (unsigned)(work2 < st.sm_count ? work2 : st.sm_count);
-    if (MOE_GEMM_PAIR) return launch_pair_gemm<kWeighted>(st, max_pair_tiles * p2.n_tiles, ta2, td, td, ty, p2, s);
+    if (MOE_GEMM_PAIR) return launch_pair_gemm<kWeighted>(st, max_pair_tiles * p2.n_tiles, ta2, td3, td3, ty, p2, s);
     return launch(grouped_gemm_kernel<kWeighted, false>, dim3(grid2), dim3(kThreads), smem2, s, 1u, ta2, td, td, ty,
                   p2);
 }
