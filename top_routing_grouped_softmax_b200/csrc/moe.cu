@@ -282,8 +282,8 @@ Layout plan(int64_t T, int64_t d, int64_t E, int64_t k, int64_t f, int64_t n_s =
 // Router GEMM, softmax and top-k in one kernel.  With chunk_counts set, it
 // also writes the per-chunk expert histogram the permutation needs.
 template <int KMAX>
-int launch_route(const CUtensorMap& tx, const CUtensorMap& tw, moe::route::Params p, unsigned tiles,
-                 cudaStream_t s)
+int launch_route(const CUtensorMap& tx, const CUtensorMap& tw, const CUtensorMap& tw3, moe::route::Params p,
+                 unsigned tiles, cudaStream_t s)
 {
     using moe::route::smem_bytes;
     // one CTA per SM: the deepest ring that fits (2 to 8 stages)
@@ -291,7 +291,7 @@ int launch_route(const CUtensorMap& tx, const CUtensorMap& tw, moe::route::Param
     while (p.stages > 2 && smem_bytes(p.n_chunks, p.stages, p.E, p.split, p.passes) > (size_t)kMaxDynSmem)
         --p.stages;
     return launch(moe::route::route_kernel<KMAX>, dim3(tiles * (unsigned)p.split), dim3(moe::route::kThreads),
-                  smem_bytes(p.n_chunks, p.stages, p.E, p.split, p.passes), s, (unsigned)p.split, tx, tw, p);
+                  smem_bytes(p.n_chunks, p.stages, p.E, p.split, p.passes), s, (unsigned)p.split, tx, tw, tw3, p);
 }
 
 int run_route(const DeviceState& st, const moe_bf16* x, const moe_bf16* w_router, const float* bias, int64_t T,
@@ -304,6 +304,21 @@ int run_route(const DeviceState& st, const moe_bf16* x, const moe_bf16* w_router
     if (rc) return rc;
     rc = make_map(&tw, w_router, (uint64_t)E, (uint64_t)d, 64, 64);
     if (rc) return rc;
+    // E a multiple of 64: every expert chunk of a k-block in one 3-D copy
+    // (W_router viewed as [E/64][d][64]); otherwise one copy per chunk, the
+    // last one zero-filled past E
+    CUtensorMap tw3 = tw;
+    const bool w_one_copy = E % 64 == 0 && E / 64 <= 16;
+    if (w_one_copy) {
+        cuuint64_t dims[3] = {64, (cuuint64_t)d, (cuuint64_t)(E / 64)};
+        cuuint64_t strides[2] = {(cuuint64_t)E * 2, 128};
+        cuuint32_t box[3] = {64, 64, (cuuint32_t)(E / 64)};
+        cuuint32_t estr[3] = {1, 1, 1};
+        if (g_encode(&tw3, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<moe_bf16*>(w_router), dims, strides, box,
+                     estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return MOE_ERR_CUDA;
+    }
     const int64_t tiles = (T + moe::route::kBM - 1) / moe::route::kBM;
     moe::route::Params p;
     p.bias = bias;
@@ -316,6 +331,7 @@ int run_route(const DeviceState& st, const moe_bf16* x, const moe_bf16* w_router
     p.E = (int)E;
     p.k = (int)k;
     p.n_chunks = (int)((E + 63) / 64);
+    p.w_one_copy = w_one_copy ? 1 : 0;
     p.stages = 0;  // set by the launcher
     uint32_t cols = 64;
     while (cols < (uint32_t)(64 * p.n_chunks)) cols <<= 1;
@@ -331,11 +347,11 @@ int run_route(const DeviceState& st, const moe_bf16* x, const moe_bf16* w_router
     // top-k list length: the power of two >= k for lane groups (k <= 8), or
     // the whole-warp rounds (k > 8)
     const unsigned ut = (unsigned)tiles;
-    if (k <= 1) return launch_route<1>(tx, tw, p, ut, s);
-    if (k <= 2) return launch_route<2>(tx, tw, p, ut, s);
-    if (k <= 4) return launch_route<4>(tx, tw, p, ut, s);
-    if (k <= 8) return launch_route<8>(tx, tw, p, ut, s);
-    return launch_route<32>(tx, tw, p, ut, s);
+    if (k <= 1) return launch_route<1>(tx, tw, tw3, p, ut, s);
+    if (k <= 2) return launch_route<2>(tx, tw, tw3, p, ut, s);
+    if (k <= 4) return launch_route<4>(tx, tw, tw3, p, ut, s);
+    if (k <= 8) return launch_route<8>(tx, tw, tw3, p, ut, s);
+    return launch_route<32>(tx, tw, tw3, p, ut, s);
 }
 
 // Grouping by expert.  have_hist: chunk_em already holds the per-chunk

@@ -65,6 +65,7 @@ struct Params {
     int n_tchunks;
     int T, d, E, k;
     int n_chunks;            // ceil(E / 64): 64-expert column chunks of W_router
+    int w_one_copy;          // 1: all chunks of a k-block come in one 3-D copy (E % 64 == 0)
     int stages;              // pipeline depth
     uint32_t tmem_cols;      // power of two >= 64 * n_chunks
     int split;               // CTAs per tile: 1, or 2 (cluster of two, split K)
@@ -326,7 +327,8 @@ __device__ __forceinline__ void topk_rows(const Params& p, const float* buf, con
 
 template <int KMAX>
 __global__ void __launch_bounds__(kThreads, 1)
-    route_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w, Params p)
+    route_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
+                 const __grid_constant__ CUtensorMap tm_w3, Params p)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -360,7 +362,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         *abort_flag = 0;
         fence_mbar_init();
         tma_prefetch_map(&tm_x);
-        tma_prefetch_map(&tm_w);
+        tma_prefetch_map(p.w_one_copy ? &tm_w3 : &tm_w);
     }
     if (warp == 1) {
         __syncwarp();
@@ -394,8 +396,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 uint8_t* sa = smem + (size_t)s * sbytes;
                 mbar_arrive_expect_tx(&full[s], (uint32_t)sbytes);
                 tma_load_2d(sa, &tm_x, &full[s], kb * kBK, tile0);
-                for (int c = 0; c < p.n_chunks; ++c)
-                    tma_load_2d(sa + kABytes + c * kChunkBytes, &tm_w, &full[s], c * 64, kb * kBK);
+                if (p.w_one_copy) {
+                    // W_router viewed as [E/64][d][64]: every 64-expert chunk of the k-block
+                    tma_load_3d(sa + kABytes, &tm_w3, &full[s], 0, kb * kBK, 0);
+                } else {
+                    for (int c = 0; c < p.n_chunks; ++c)
+                        tma_load_2d(sa + kABytes + c * kChunkBytes, &tm_w, &full[s], c * 64, kb * kBK);
+                }
                 ++issued;
             }
             // Never leave the CTA with a copy still landing in its shared memory.
