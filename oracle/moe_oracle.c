@@ -39,7 +39,8 @@
  * Optional variants, each off the article's path and pinned like the rest:
  * oracle_renormalize (renormalised top-k weights), oracle_shared_rows
  * (shared experts), oracle_round_tokens and oracle_masked_rows (token
- * rounding).
+ * rounding), and oracle_backward (the gradient of the block, for the
+ * backward that recomputes the expert activations).
  *
  * Parity status: every function here is pinned by CPU tests against
  * independent computations (brute force, library routines, invariants and
@@ -434,4 +435,150 @@ int oracle_masked_rows(const uint16_t* x, const uint16_t* w_gate, const uint16_t
     }
     free(xrow); free(g); free(u); free(h); free(o);
     return status;
+}
+
+/*
+ * Backward of the block (the next row after the forward): the exact gradient
+ * of L = sum_t sum_c dout[t][c] * out[t][c] with respect to x, W_router, the
+ * router bias and the three expert weight tensors.  The SonicMoE comparison
+ * page, section "core differences", item 1 (memory management), stores only
+ * the gating outputs and the final expert outputs for the backward and
+ * recomputes the rest; that changes what a GPU keeps, not the gradient, so
+ * this oracle recomputes everything from the inputs, like the forward.
+ *
+ * For token t with routing (ids, w) from oracle_route (plus
+ * oracle_renormalize when renormalize != 0), for each slot j, e = ids[t][j]:
+ *   g, u, h = silu(g) * u, z = h . W_down[e]          (as the forward)
+ *   dw_j     = dout[t] . z                            (gradient of the weight)
+ *   dz       = w_j * dout[t]
+ *   dW_down[e][n][c] += h[n] * dz[c]
+ *   dh[n]    = sum_c dz[c] * W_down[e][n][c]
+ *   du[n]    = dh[n] * silu(g[n])
+ *   dg[n]    = dh[n] * u[n] * s(g[n]) * (1 + g[n] * (1 - s(g[n]))),  s = 1/(1+e^-x)
+ *              (the derivative of silu(z) = z * s(z))
+ *   dW_gate[e][i][n] += x[t][i] * dg[n],  dW_up[e][i][n] += x[t][i] * du[n]
+ *   dx[t][i] += sum_n dg[n] * W_gate[e][i][n] + du[n] * W_up[e][i][n]
+ * Router (the top-k choice itself is piecewise constant and passes no
+ * gradient): with p the softmax of the logits,
+ *   dp[e]      = dw_j for e = ids[t][j], 0 for the other experts
+ *                (renormalised weights w_j = p_j / S, S = sum_m p_m over the
+ *                 slots: dp[ids[t][m]] = (dw_m - sum_j dw_j * w_j) / S)
+ *   dlogit[e]  = p[e] * (dp[e] - sum_i p[i] * dp[i])   (softmax Jacobian)
+ *   dW_router[i][e] += x[t][i] * dlogit[e],  dbias[e] += dlogit[e]
+ *   dx[t][i]  += sum_e dlogit[e] * W_router[i][e]
+ * Every sum runs in ascending index order in fp64; tokens accumulate into
+ * the weight gradients in ascending t, slots in ascending j.
+ *
+ * Outputs (fp64, overwritten): dx [T][d], dw_router [d][E], dbias [E],
+ * dw_gate [E][d][f], dw_up [E][d][f], dw_down [E][f][d].  dout is [T][d].
+ */
+int oracle_backward(const uint16_t* x, const uint16_t* w_router, const float* bias,
+                    const uint16_t* w_gate, const uint16_t* w_up, const uint16_t* w_down,
+                    int64_t T, int64_t d, int64_t E, int64_t k, int64_t f, int renormalize,
+                    const double* dout, double* dx, double* dw_router, double* dbias,
+                    double* dw_gate, double* dw_up, double* dw_down)
+{
+    if (!x || !w_router || !w_gate || !w_up || !w_down || !dout || !dx || !dw_router || !dbias ||
+        !dw_gate || !dw_up || !dw_down || T < 0 || d < 1 || E < 1 || k < 1 || k > E || f < 1)
+        return ORACLE_BAD_ARG;
+    int32_t* ids = (int32_t*)malloc(sizeof(int32_t) * (size_t)(T * k + 1));
+    double* w = (double*)malloc(sizeof(double) * (size_t)(T * k + 1));
+    double* probs = (double*)malloc(sizeof(double) * (size_t)(T * E + 1));
+    double* xrow = (double*)malloc(sizeof(double) * (size_t)d);
+    double* g = (double*)malloc(sizeof(double) * (size_t)f);
+    double* u = (double*)malloc(sizeof(double) * (size_t)f);
+    double* h = (double*)malloc(sizeof(double) * (size_t)f);
+    double* z = (double*)malloc(sizeof(double) * (size_t)d);
+    double* dz = (double*)malloc(sizeof(double) * (size_t)d);
+    double* dh = (double*)malloc(sizeof(double) * (size_t)f);
+    double* dg = (double*)malloc(sizeof(double) * (size_t)f);
+    double* du = (double*)malloc(sizeof(double) * (size_t)f);
+    double* dwj = (double*)malloc(sizeof(double) * (size_t)k);
+    double* dp = (double*)malloc(sizeof(double) * (size_t)E);
+    double* dl = (double*)malloc(sizeof(double) * (size_t)E);
+    int rc = ORACLE_NO_MEMORY;
+    if (!ids || !w || !probs || !xrow || !g || !u || !h || !z || !dz || !dh || !dg || !du || !dwj || !dp || !dl)
+        goto done;
+    rc = oracle_route(x, w_router, bias, T, d, E, k, NULL, probs, ids, w);
+    if (rc != ORACLE_OK) goto done;
+    if (renormalize) {
+        rc = oracle_renormalize(w, T, k);
+        if (rc != ORACLE_OK) goto done;
+    }
+    memset(dx, 0, sizeof(double) * (size_t)(T * d));
+    memset(dw_router, 0, sizeof(double) * (size_t)(d * E));
+    memset(dbias, 0, sizeof(double) * (size_t)E);
+    memset(dw_gate, 0, sizeof(double) * (size_t)(E * d * f));
+    memset(dw_up, 0, sizeof(double) * (size_t)(E * d * f));
+    memset(dw_down, 0, sizeof(double) * (size_t)(E * f * d));
+    for (int64_t t = 0; t < T; ++t) {
+        for (int64_t i = 0; i < d; ++i) xrow[i] = bf16_to_double(x[t * d + i]);
+        const double* drow_out = dout + t * d;
+        for (int64_t j = 0; j < k; ++j) {
+            const int64_t e = ids[t * k + j];
+            const double wj = w[t * k + j];
+            const uint16_t* wg = w_gate + e * d * f;
+            const uint16_t* wu = w_up + e * d * f;
+            const uint16_t* wd = w_down + e * f * d;
+            expert_swiglu(xrow, wg, wu, wd, d, f, g, u, h, z);
+            double s = 0.0;
+            for (int64_t c = 0; c < d; ++c) s += drow_out[c] * z[c];
+            dwj[j] = s;
+            for (int64_t c = 0; c < d; ++c) dz[c] = wj * drow_out[c];
+            double* gdown = dw_down + e * f * d;
+            for (int64_t n = 0; n < f; ++n) {
+                double acc = 0.0;
+                for (int64_t c = 0; c < d; ++c) {
+                    gdown[n * d + c] += h[n] * dz[c];
+                    acc += dz[c] * bf16_to_double(wd[n * d + c]);
+                }
+                dh[n] = acc;
+            }
+            for (int64_t n = 0; n < f; ++n) {
+                const double sg = 1.0 / (1.0 + exp(-g[n]));
+                du[n] = dh[n] * (g[n] * sg);
+                dg[n] = dh[n] * u[n] * sg * (1.0 + g[n] * (1.0 - sg));
+            }
+            double* ggate = dw_gate + e * d * f;
+            double* gup = dw_up + e * d * f;
+            for (int64_t i = 0; i < d; ++i) {
+                double acc = 0.0;
+                for (int64_t n = 0; n < f; ++n) {
+                    ggate[i * f + n] += xrow[i] * dg[n];
+                    gup[i * f + n] += xrow[i] * du[n];
+                    acc += dg[n] * bf16_to_double(wg[i * f + n]) + du[n] * bf16_to_double(wu[i * f + n]);
+                }
+                dx[t * d + i] += acc;
+            }
+        }
+        /* router: routing-weight gradients -> probabilities -> logits */
+        for (int64_t e = 0; e < E; ++e) dp[e] = 0.0;
+        if (renormalize) {
+            double ssum = 0.0, dot = 0.0;
+            for (int64_t j = 0; j < k; ++j) ssum += probs[t * E + ids[t * k + j]];
+            for (int64_t j = 0; j < k; ++j) dot += dwj[j] * w[t * k + j];
+            for (int64_t j = 0; j < k; ++j) dp[ids[t * k + j]] = (dwj[j] - dot) / ssum;
+        } else {
+            for (int64_t j = 0; j < k; ++j) dp[ids[t * k + j]] = dwj[j];
+        }
+        const double* p = probs + t * E;
+        double pdp = 0.0;
+        for (int64_t e = 0; e < E; ++e) pdp += p[e] * dp[e];
+        for (int64_t e = 0; e < E; ++e) dl[e] = p[e] * (dp[e] - pdp);
+        for (int64_t e = 0; e < E; ++e) dbias[e] += dl[e];
+        for (int64_t i = 0; i < d; ++i) {
+            double acc = 0.0;
+            const uint16_t* wrow = w_router + i * E;
+            for (int64_t e = 0; e < E; ++e) {
+                dw_router[i * E + e] += xrow[i] * dl[e];
+                acc += dl[e] * bf16_to_double(wrow[e]);
+            }
+            dx[t * d + i] += acc;
+        }
+    }
+    rc = ORACLE_OK;
+done:
+    free(ids); free(w); free(probs); free(xrow); free(g); free(u); free(h); free(z); free(dz);
+    free(dh); free(dg); free(du); free(dwj); free(dp); free(dl);
+    return rc;
 }

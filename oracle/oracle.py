@@ -69,6 +69,9 @@ class Oracle:
         lib.oracle_round_tokens.restype = ctypes.c_int
         lib.oracle_masked_rows.argtypes = [_P, _P, _P, _P, _I64, _I64, _I64, _I64, _P, _P, _I64, _P, _P]
         lib.oracle_masked_rows.restype = ctypes.c_int
+        lib.oracle_backward.argtypes = [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64, ctypes.c_int,
+                                        _P, _P, _P, _P, _P, _P, _P]
+        lib.oracle_backward.restype = ctypes.c_int
         for fn in (lib.oracle_route, lib.oracle_permute, lib.oracle_expert_rows, lib.oracle_renormalize):
             fn.restype = ctypes.c_int
         self.lib = lib
@@ -197,6 +200,42 @@ class Oracle:
         if shared is not None:
             ex = ExpertResult(out=self.shared_rows(x, *shared, rows, ex.out), y=ex.y, h=ex.h)
         return r, ex
+
+    # -- backward ---------------------------------------------------------------
+    def backward(self, x, w_router, bias, w_gate, w_up, w_down, k, dout, renormalize=False):
+        """Gradient of sum(dout * out) with respect to x, W_router, the bias
+        and the expert weights (fp64; the routing choice passes no gradient)."""
+        x = np.ascontiguousarray(x, dtype=np.uint16)
+        w_router = np.ascontiguousarray(w_router, dtype=np.uint16)
+        w_gate = np.ascontiguousarray(w_gate, dtype=np.uint16)
+        w_up = np.ascontiguousarray(w_up, dtype=np.uint16)
+        w_down = np.ascontiguousarray(w_down, dtype=np.uint16)
+        dout = np.ascontiguousarray(dout, dtype=np.float64)
+        T, d = x.shape
+        E = w_router.shape[1]
+        f = w_gate.shape[2]
+        assert w_gate.shape == (E, d, f) and w_up.shape == (E, d, f) and w_down.shape == (E, f, d)
+        assert dout.shape == (T, d)
+        b = None if bias is None else np.ascontiguousarray(bias, dtype=np.float32)
+        g = BackwardResult(dx=np.empty((T, d)), dw_router=np.empty((d, E)), dbias=np.empty(E),
+                           dw_gate=np.empty((E, d, f)), dw_up=np.empty((E, d, f)), dw_down=np.empty((E, f, d)))
+        rc = self.lib.oracle_backward(_ptr(x), _ptr(w_router), _ptr(b), _ptr(w_gate), _ptr(w_up), _ptr(w_down),
+                                      T, d, E, k, f, 1 if renormalize else 0, _ptr(dout), _ptr(g.dx),
+                                      _ptr(g.dw_router), _ptr(g.dbias), _ptr(g.dw_gate), _ptr(g.dw_up),
+                                      _ptr(g.dw_down))
+        if rc != 0:
+            raise ValueError(f"oracle_backward failed ({rc})")
+        return g
+
+
+@dataclass
+class BackwardResult:
+    dx: np.ndarray         # [T, d]
+    dw_router: np.ndarray  # [d, E]
+    dbias: np.ndarray      # [E]
+    dw_gate: np.ndarray    # [E, d, f]
+    dw_up: np.ndarray      # [E, d, f]
+    dw_down: np.ndarray    # [E, f, d]
 
 
 @dataclass

@@ -14,7 +14,12 @@ The independent computations used here:
     scipy.special.expit (for silu(z) = z * expit(z)), numpy's stable argsort;
   * special cases with closed forms: E = 1, k = 1 is a dense SwiGLU MLP;
     k = E with identical experts is that MLP times sum(p) = 1; exact ties;
-  * invariants: counts sum to T*k, the permutation is a bijection, etc.
+  * invariants: counts sum to T*k, the permutation is a bijection, etc.;
+  * for the backward: torch autograd through an fp64 torch rendering of the
+    forward (a library differentiator, independent of the oracle's
+    hand-derived chain rule), central finite differences of a numpy forward
+    that is itself checked against the oracle's forward, and the softmax
+    gradient's zero sum over experts.
 """
 from __future__ import annotations
 
@@ -379,9 +384,124 @@ def check_token_rounding(o):
     assert np.array_equal(np.nonzero(m24[:, 1])[0], np.concatenate([np.arange(4), np.arange(20, 40)]))
 
 
+# --------------------------------------------------------------- backward
+def _torch_block_grads(x, wr, bias, wg, wu, wd, k, dout, renormalize):
+    """Gradients of sum(dout * out) by torch autograd (fp64) through a dense
+    torch rendering of the block; the top-k choice is numpy's lexsort over
+    scipy's softmax (no gradient flows through a selection)."""
+    _, _, top, _ = dense_reference(x, wr, bias, wg, wu, wd, k)
+    X = torch.tensor(widen(x), requires_grad=True)
+    Wr = torch.tensor(widen(wr), requires_grad=True)
+    E = Wr.shape[1]
+    b = torch.tensor(np.zeros(E) if bias is None else bias.astype(np.float64), requires_grad=True)
+    Wg = torch.tensor(widen(wg), requires_grad=True)
+    Wu = torch.tensor(widen(wu), requires_grad=True)
+    Wd = torch.tensor(widen(wd), requires_grad=True)
+    ids = torch.tensor(top.astype(np.int64))
+    p = torch.softmax(X @ Wr + b, dim=1)
+    w = torch.gather(p, 1, ids)
+    if renormalize:
+        w = w / w.sum(dim=1, keepdim=True)
+    out = torch.zeros_like(X)
+    for j in range(k):
+        e = ids[:, j]
+        G = torch.einsum("td,tdf->tf", X, Wg[e])
+        U = torch.einsum("td,tdf->tf", X, Wu[e])
+        H = torch.nn.functional.silu(G) * U
+        out = out + w[:, j:j + 1] * torch.einsum("tf,tfd->td", H, Wd[e])
+    (out * torch.tensor(dout)).sum().backward()
+    return {"dx": X.grad.numpy(), "dw_router": Wr.grad.numpy(), "dbias": b.grad.numpy(),
+            "dw_gate": Wg.grad.numpy(), "dw_up": Wu.grad.numpy(), "dw_down": Wd.grad.numpy()}
+
+
+_BWD_CASES = [(24, 32, 6, 2, 16, 21, False, False), (17, 16, 8, 3, 24, 22, True, False),
+              (20, 32, 5, 5, 8, 23, False, True), (9, 16, 1, 1, 16, 24, False, False),
+              (16, 24, 8, 4, 16, 25, True, True)]
+
+
+def _dout(T, d, seed):
+    return np.random.default_rng(seed).standard_normal((T, d))
+
+
+def check_backward_autograd(o):
+    for (T, d, E, k, f, seed, bias, renorm) in _BWD_CASES:
+        inp = _rand_case(T, d, E, k, f, seed, bias=bias, sigma=0.2)
+        dout = _dout(T, d, seed)
+        g = o.backward(*_args(inp), k, dout, renormalize=renorm)
+        ref = _torch_block_grads(*_args(inp), k, dout, renorm)
+        for name, want in ref.items():
+            got = getattr(g, name)
+            assert got.shape == want.shape, (name, got.shape, want.shape)
+            assert _rel(got, want) < 1e-10 or np.abs(want).max() < 1e-300, ("autograd", name, T, d, E, k, f, renorm)
+
+
+def _np_block(X, Wr, b, Wg, Wu, Wd, ids, renormalize):
+    """Plain fp64 numpy forward with a fixed expert choice (for finite differences)."""
+    p = sps.softmax(X @ Wr + b[None, :], axis=1)
+    w = np.take_along_axis(p, ids, axis=1)
+    if renormalize:
+        w = w / w.sum(axis=1, keepdims=True)
+    out = np.zeros_like(X)
+    for t in range(X.shape[0]):
+        for j in range(ids.shape[1]):
+            e = ids[t, j]
+            G = X[t] @ Wg[e]
+            H = G * sps.expit(G) * (X[t] @ Wu[e])
+            out[t] += w[t, j] * (H @ Wd[e])
+    return out
+
+
+def check_backward_finite_differences(o):
+    for (T, d, E, k, f, seed, bias, renorm) in _BWD_CASES[:3]:
+        inp = _rand_case(T, d, E, k, f, seed, bias=bias, sigma=0.2)
+        args = _args(inp)
+        dout = _dout(T, d, seed)
+        r, ex = o.forward(*args, k, renormalize=renorm)
+        base = [widen(args[0]), widen(args[1]),
+                np.zeros(E) if args[2] is None else args[2].astype(np.float64),
+                widen(args[3]), widen(args[4]), widen(args[5])]
+        ids = r.ids.astype(np.int64)
+        # the numpy forward is the oracle's forward at the bf16 point
+        assert _rel(_np_block(*base, ids, renorm), ex.out) < 1e-12, ("numpy forward", T, E, k)
+        g = o.backward(*args, k, dout, renormalize=renorm)
+        grads = [g.dx, g.dw_router, g.dbias, g.dw_gate, g.dw_up, g.dw_down]
+        rng = np.random.default_rng(seed + 1)
+        for pos in range(6):
+            v = rng.standard_normal(base[pos].shape)
+            eps = 1e-6 * max(1.0, float(np.abs(base[pos]).max()))
+
+            def loss(sign):
+                pts = list(base)
+                pts[pos] = base[pos] + sign * eps * v
+                return float(np.sum(_np_block(*pts, ids, renorm) * dout))
+
+            fd = (loss(1.0) - loss(-1.0)) / (2 * eps)
+            an = float(np.sum(grads[pos] * v))
+            assert abs(fd - an) <= 1e-6 * max(1.0, abs(an)), ("finite differences", pos, fd, an)
+
+
+def check_backward_invariants(o):
+    # the softmax gradient sums to zero over experts, so do dbias and each row of dW_router
+    inp = _rand_case(24, 32, 8, 3, 16, 31, bias=True, sigma=0.2)
+    dout = _dout(24, 32, 31)
+    g = o.backward(*_args(inp), 3, dout)
+    assert abs(g.dbias.sum()) <= 1e-12 * np.abs(g.dbias).sum()
+    assert np.all(np.abs(g.dw_router.sum(axis=1)) <= 1e-12 * np.abs(g.dw_router).sum(axis=1) + 1e-300)
+    # experts no token selects get exactly zero weight gradients
+    r, _ = o.forward(*_args(inp), 3)
+    unused = np.setdiff1d(np.arange(8), r.ids.ravel())
+    for e in unused:
+        assert not g.dw_gate[e].any() and not g.dw_up[e].any() and not g.dw_down[e].any()
+    # linear in dout: doubling it doubles every gradient exactly
+    g2 = o.backward(*_args(inp), 3, 2.0 * dout)
+    for name in ("dx", "dw_router", "dbias", "dw_gate", "dw_up", "dw_down"):
+        assert np.array_equal(getattr(g2, name), 2.0 * getattr(g, name)), name
+
+
 ALL_CHECKS = [
     check_brute_force, check_softmax_library, check_topk_library_sort, check_topk_of_logits,
     check_exact_ties, check_dense_special_case, check_all_experts_identical, check_zero_expert,
     check_scale_down, check_permute_library, check_page_listing_torch, check_expert_rows_outputs,
-    check_renormalize, check_shared_experts, check_token_rounding,
+    check_renormalize, check_shared_experts, check_token_rounding, check_backward_autograd,
+    check_backward_finite_differences, check_backward_invariants,
 ]

@@ -43,6 +43,17 @@ MUTANTS = [
      "for (int64_t c = 0; c < d; ++c) out[r * d + c] += 0.5 * o[c];"),
     ("renorm_partial_sum", "for (int64_t j = 0; j < k; ++j) s += weights[t * k + j];",
      "for (int64_t j = 0; j + 1 < k; ++j) s += weights[t * k + j];"),
+    ("bwd_silu_derivative_short", "dg[n] = dh[n] * u[n] * sg * (1.0 + g[n] * (1.0 - sg));",
+     "dg[n] = dh[n] * u[n] * sg;"),
+    ("bwd_no_routing_weight", "for (int64_t c = 0; c < d; ++c) dz[c] = wj * drow_out[c];",
+     "for (int64_t c = 0; c < d; ++c) dz[c] = drow_out[c];"),
+    ("bwd_softmax_no_centering", "for (int64_t e = 0; e < E; ++e) dl[e] = p[e] * (dp[e] - pdp);",
+     "for (int64_t e = 0; e < E; ++e) dl[e] = p[e] * dp[e];"),
+    ("bwd_dx_without_router", "acc += dl[e] * bf16_to_double(wrow[e]);", "acc += 0.0 * dl[e] * bf16_to_double(wrow[e]);"),
+    ("bwd_up_grad_uses_gate", "du[n] = dh[n] * (g[n] * sg);", "du[n] = dh[n] * g[n];"),
+    ("bwd_renorm_no_dot", "dp[ids[t * k + j]] = (dwj[j] - dot) / ssum;", "dp[ids[t * k + j]] = dwj[j] / ssum;"),
+    ("bwd_down_transposed", "acc += dz[c] * bf16_to_double(wd[n * d + c]);",
+     "acc += dz[c] * bf16_to_double(wd[c * f + n]);"),
 ]
 
 
