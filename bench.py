@@ -212,6 +212,28 @@ def cpu_baseline(cfg, n_tokens: int, seed: int, inp=None):
                       f"(route, permute, expert MLPs, combine), fp64, one thread", **host_cpu()}
 
 
+def route_parity(cfg, ids_gpu, seed):
+    """Expert ids of the timed batch against the oracle's routing of every
+    token (part of the CPU-oracle leg): tokens whose k-th and (k+1)-th
+    probabilities differ by less than 1e-6 are counted and left out; tokens
+    with a near tie between two selected slots are compared as sets."""
+    import numpy as np
+    from oracle.oracle import default_oracle, inner_gap, topk_gap
+    from top_routing_grouped_softmax_b200.synth import make_inputs
+
+    inp = make_inputs(cfg.with_(seed=seed))
+    r = default_oracle().route(inp.bits("x"), inp.bits("W_router"), inp.bias_np(), cfg.k)
+    excluded = topk_gap(r.probs, cfg.k) < 1e-6
+    inner = (inner_gap(r.probs, cfg.k) < 1e-6) & ~excluded
+    exact = ~excluded & ~inner
+    mism_exact = int(np.any(ids_gpu[exact] != r.ids[exact], axis=1).sum())
+    mism_inner = int(np.any(np.sort(ids_gpu[inner], 1) != np.sort(r.ids[inner], 1), axis=1).sum())
+    return {"tokens": int(cfg.T), "ids_mismatch": mism_exact + mism_inner, "excluded_near_tie": int(excluded.sum()),
+            "inner_near_tie": int(inner.sum()),
+            "rule": "ids bit-exact per slot; tokens with p_(k) - p_(k+1) < 1e-6 excluded; tokens with a "
+                    "gap < 1e-6 between two selected slots compared as sets"}
+
+
 # ------------------------------------------------------------- reference
 def run_reference(args, cfg):
     rank, _, world = dist_env()
@@ -459,11 +481,16 @@ def run_gpu(args, cfg):
             "grouped_gemm_tflops_padded": (alg["gateup_flops"] + alg["down_flops"]) / (1.0 - padding) /
                                           ((stage_ms["gateup_gemm"] + stage_ms["down_gemm"]) * 1e-3) / 1e12,
             "roofline": {"bound": "tensor",
+                         "scope": "kernel: the dominant kernel alone (achieved, frac, traffic); "
+                                  "the whole forward is in `forward`",
                          "kernel": ("grouped_gemm_pair_kernel<SwiGLU> (gate/up + SwiGLU)" if args.path == "fused"
                                     else "moe_expert_ffn (gate/up + down GEMMs)"),
                          "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                          "frac": achieved / peaks["bf16_tflops"], "traffic": traffic,
-                         "peak_source": f"{peaks['source']} burst bf16"},
+                         "peak_source": f"{peaks['source']} burst bf16",
+                         "forward": {"frac": roof_time / (ms * 1e-3), "roofline_ms": roof_time * 1e3,
+                                     "ms_per_step": ms, "frac_of_datasheet": roof_ds / (ms * 1e-3),
+                                     "bound": "max(FLOPs / bf16 peak, compulsory bytes / HBM peak)"}},
             "forward_roofline": {"roofline_ms": roof_time * 1e3, "frac": roof_time / (ms * 1e-3),
                                  "flops": alg["flops"], "compulsory_bytes": alg["bytes"],
                                  "peaks": "of measured (MEASURED_PEAKS.json)",
@@ -480,10 +507,78 @@ def run_gpu(args, cfg):
             "gpu_launches": (KERNELS_PER_FORWARD + 2 * args.shared + (3 if args.round else 0)) * args.steps,
             "clocks": clocks,
             "wall_s_timed_region": wall,
+            "_topk_ids": ids.cpu().numpy(),
         }
     if world > 1:
         dist.destroy_process_group()
     return result
+
+
+def time_workload(name, args, dev):
+    """Time moe_forward on another of the workloads (fused path, N = 1) with
+    the headline's rules -- inputs resident in HBM, L2 flushed between timed
+    steps, CUDA events on the launching stream, NVML clocks sampled during
+    the timed region -- and return its figures for the `workloads` object."""
+    import torch
+
+    import top_routing_grouped_softmax_b200 as moe
+    from top_routing_grouped_softmax_b200.synth import CONFIGS, make_inputs
+
+    cfg = CONFIGS[name]
+    inp = make_inputs(cfg)
+    x = inp.x.to(dev)
+    w = {n: getattr(inp, n).to(dev) for n in ("W_router", "W_gate", "W_up", "W_down")}
+    bias = None if inp.bias is None else inp.bias.to(dev)
+    del inp
+    blk = moe.MoEBlock(w["W_router"], w["W_gate"], w["W_up"], w["W_down"], cfg.k, bias=bias)
+    out = torch.empty(cfg.T, cfg.d, dtype=torch.float32, device=dev)
+    ids = torch.empty(cfg.T, cfg.k, dtype=torch.int32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    for _ in range(max(args.warmup, 3)):
+        blk(x, out=out, topk_ids=ids)
+    torch.cuda.synchronize()
+    n_ev = 6
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
+    with ClockSampler(dev.index) as clk:
+        for i in range(args.steps):
+            flush.zero_()
+            e = evs[i]
+            blk(x, out=out, topk_ids=ids, events=[e[0], None, e[2], e[3], None, e[5]])
+        torch.cuda.synchronize()
+    sev = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush.zero_()
+        blk(x, out=out, topk_ids=ids, events=sev[i])
+    torch.cuda.synchronize()
+    status = moe.get_status()
+    assert status == moe.MOE_OK, moe.strerror(status)
+    ms = statistics.mean(e[0].elapsed_time(e[n_ev - 1]) for e in evs)
+    gateup_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
+    stage_ms = {s: statistics.mean(e[i].elapsed_time(e[i + 1]) for e in sev) for i, s in enumerate(STAGES)}
+    counts = torch.bincount(ids.flatten().long(), minlength=cfg.E).cpu()
+    active = int((counts > 0).sum())
+    tiles = int(((counts + 255) // 256).sum())
+    peaks = load_peaks()
+    alg = algorithmic(cfg, active)
+    roof = max(alg["flops"] / (peaks["bf16_tflops"] * 1e12), alg["bytes"] / (peaks["hbm_gbs"] * 1e9))
+    roof_ds = max(alg["flops"] / (DATASHEET["bf16_tflops"] * 1e12), alg["bytes"] / (DATASHEET["hbm_gbs"] * 1e9))
+    gateup = alg["gateup_flops"] / (gateup_ms * 1e-3) / 1e12
+    res = {
+        "config": workload_config(cfg, extra={"out_dtype": "fp32"}),
+        "ms_per_step": ms, "tokens_per_s": cfg.T / (ms * 1e-3), "steps": args.steps,
+        "tflops": alg["flops"] / (ms * 1e-3) / 1e12,
+        "forward_roofline": {"frac": roof / (ms * 1e-3), "roofline_ms": roof * 1e3,
+                             "frac_of_datasheet": roof_ds / (ms * 1e-3)},
+        "gateup": {"achieved_tflops": gateup, "frac": gateup / peaks["bf16_tflops"],
+                   "peak_source": f"{peaks['source']} burst bf16"},
+        "stage_ms": stage_ms,
+        "experts": {"active": active, "max_count": int(counts.max()), "min_count": int(counts.min()),
+                    "pair_tile_padding": 1.0 - int(counts.sum()) / max(1, tiles * 256)},
+        "clocks": clk.summary(),
+    }
+    del blk, x, w, out, ids, flush
+    torch.cuda.empty_cache()
+    return res
 
 
 def main(argv=None):
@@ -505,6 +600,9 @@ def main(argv=None):
                     help="tokens of the workload the CPU-oracle baseline leg evaluates")
     ap.add_argument("--ref-tokens", type=int, default=32, help="tokens per step of the reference arm")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workloads", default="coarse,fine,skew",
+                    help="other workloads to time at N=1 (fused path) into the line's `workloads` object; "
+                         "empty to skip")
     args = ap.parse_args(argv)
 
     from top_routing_grouped_softmax_b200.synth import CONFIGS
@@ -517,8 +615,19 @@ def main(argv=None):
     res = run_gpu(args, cfg)
     rank, _, world = dist_env()
     if rank == 0 and res is not None:
+        ids_gpu = res.pop("_topk_ids", None)
+        extra = [n for n in args.workloads.split(",") if n and n != cfg.name]
+        if world == 1 and extra and args.path == "fused" and not (args.round or args.shared or args.gather):
+            import torch
+            dev = torch.device("cuda", torch.cuda.current_device())
+            wl = {n: time_workload(n, args, dev) for n in extra}
+            res["workloads"] = wl
+            res["roofline"]["forward_by_workload"] = {
+                cfg.name: res["roofline"]["forward"]["frac"], **{n: v["forward_roofline"]["frac"] for n, v in wl.items()}}
         if world == 1 and not args.no_cpu_baseline:
             res["cpu_baseline"] = cpu_baseline(cfg, args.cpu_tokens, replica_seed(cfg.seed, 0))
+            if ids_gpu is not None and not args.round:
+                res["cpu_baseline"]["route_parity"] = route_parity(cfg, ids_gpu, replica_seed(cfg.seed, 0))
         print(json.dumps(res), flush=True)
     return 0
 

@@ -27,6 +27,12 @@
  * where bf16 would not.  The k-way sum and out stay fp32.  A y outside the
  * fp16 range (|y| >= 65520) or NaN is stored as inf / NaN and reported as
  * MOE_ERR_DEVICE_RANGE.
+ * Types at the boundary: out is fp32 and y fp16, where a bf16 interface
+ * would round both to bf16.  Rounding out to bf16 alone puts the worst
+ * element at about 0.024 x RMS from the exact fp64 result on the
+ * Qwen3-shaped layer (a CPU emulation of the rounding points), above the
+ * block's 0.02 x RMS tolerance; a bf16 y alone gives 0.022 x RMS; fp16 y
+ * with fp32 out gives 0.012 x RMS.
  * The optional per-expert bias follows the gate G(x) = Softmax(W_g x + b_g)
  * of the Hunyuan-Large overview page, section 2.1.
  *
@@ -93,8 +99,11 @@ int moe_version(void);
  * Bytes of scratch that moe_forward needs for these sizes (0 if the shape is
  * unsupported).  The pieces, each 256-byte aligned, are: topk ids and
  * weights [M], counts [E], offsets [E+1], per-chunk group bases, perm / inv /
- * w_perm [M], h [M,f] bf16 and y [M,d] fp16.  (moe_forward never builds
- * x_perm: its gate/up GEMM gathers the rows of x through perm directly.)
+ * w_perm [M], x_perm [M,d] bf16 (the rows of x in grouped order, which the
+ * gate/up GEMM reads; moe_forward builds it), h [M,f] bf16 and y [M,d] fp16.
+ * Only moe_forward_ex with MOE_FLAG_FUSED_GATHER leaves x_perm unwritten
+ * (its gate/up GEMM gathers the rows of x through perm itself); the size
+ * still includes it.
  */
 size_t moe_workspace_size(int64_t T, int64_t d, int64_t E, int64_t k, int64_t f);
 
@@ -182,7 +191,9 @@ int moe_permute(const moe_bf16* x, const int32_t* topk_ids, const float* topk_w,
  *          sizes return MOE_ERR_STATIC_SCRATCH_TOO_SMALL.
  *   The call allocates nothing and calls no allocating routine.  The first
  *   call on each device looks up the array's device address (a one-time
- *   set-up for that device); make that first call before any stream capture.
+ *   set-up for that device, repeated once in a new context if the caller
+ *   destroyed the old one with cudaDeviceReset); make that first call before
+ *   any stream capture.
  *   All calls share the one array and it keeps the last call's contents;
  *   each call writes every entry it later reads, so nothing needs clearing,
  *   but calls whose work overlaps on the GPU (for example on two streams)
@@ -357,7 +368,10 @@ int moe_get_status(cudaStream_t stream);
  * Upper bound, in nanoseconds, on any single pipeline wait inside the
  * library's kernels on the current device (default 1e9).  A wait that runs
  * past it records MOE_ERR_DEVICE_TIMEOUT and the kernel winds down
- * without faulting.  Values <= 0 restore the default.
+ * without faulting: before it frees its tensor memory or exits, each CTA
+ * waits for its own copies and MMAs still in flight, for up to the larger of
+ * this limit and one second.  Values <= 0 restore the default; values below
+ * 1e6 (1 ms) are raised to 1e6.
  */
 int moe_set_wait_limit_ns(int64_t limit_ns);
 

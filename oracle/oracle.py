@@ -262,7 +262,9 @@ class ExpertResult:
 
 
 def topk_gap(probs: np.ndarray, k: int) -> np.ndarray:
-    """p_(k) - p_(k+1) per token (inf when k == E): the near-tie margin."""
+    """p_(k-1) - p_(k) per token, with p_(0) >= p_(1) >= ... the probabilities
+    sorted in descending order: the margin between the last selected expert
+    and the best unselected one (inf when k >= E)."""
     T, E = probs.shape
     if k >= E:
         return np.full(T, np.inf)
@@ -271,10 +273,12 @@ def topk_gap(probs: np.ndarray, k: int) -> np.ndarray:
 
 
 def inner_gap(probs: np.ndarray, k: int) -> np.ndarray:
-    """Smallest gap between consecutive probabilities among the top k+... slots.
+    """Smallest gap between consecutive probabilities inside the top k, per token.
 
-    min over j < k-1 of p_(j) - p_(j+1): a near tie here may swap the order of
-    two selected slots without changing the selected set.
+    min over j < k-1 of p_(j) - p_(j+1), with p_(0) >= p_(1) >= ... the
+    probabilities sorted in descending order (inf when k < 2): a near tie
+    here may swap the order of two selected slots without changing the
+    selected set.
     """
     T, E = probs.shape
     if k < 2:

@@ -38,7 +38,11 @@ def oracle_route(cfg: MoEConfig):
 
 def sample_for(cfg: MoEConfig, n: int):
     """Sampled tokens, always including one token of the largest and of the
-    smallest non-empty expert group."""
+    smallest non-empty expert group, and, for every non-empty expert, the
+    last token routed to it.  Groups list their tokens in ascending order, so
+    that token's grouped row is the group's last row: it lies in the group's
+    last (usually partial) 256-row GEMM tile, where the epilogue masks the
+    rows past the group's end."""
     r = oracle_route(cfg)
     counts = np.bincount(r.ids.ravel(), minlength=cfg.E)
     big = int(np.argmax(counts))
@@ -46,7 +50,26 @@ def sample_for(cfg: MoEConfig, n: int):
     small = int(nz[np.argmin(counts[nz])])
     t_big = int(np.nonzero((r.ids == big).any(axis=1))[0][0])
     t_small = int(np.nonzero((r.ids == small).any(axis=1))[0][0])
-    return sample_tokens(cfg.T, n, cfg.seed, must_include=(t_big, t_small, 0, cfg.T - 1))
+    last = [int(np.nonzero((r.ids == e).any(axis=1))[0][-1]) for e in nz]
+    return sample_tokens(cfg.T, n, cfg.seed, must_include=(t_big, t_small, 0, cfg.T - 1, *last))
+
+
+def expert_rows_parallel(inp, ids, weights, rows, workers: int = 0):
+    """The oracle's expert rows for ``rows``, evaluated in chunks on host
+    threads.  The oracle is single-threaded C called through ctypes (which
+    releases the GIL) and keeps no global state, so chunks run side by side;
+    each row is computed exactly as in one call, so the result is identical."""
+    import os
+    from concurrent.futures import ThreadPoolExecutor
+    o = default_oracle()
+    args = (inp.bits("x"), inp.bits("W_gate"), inp.bits("W_up"), inp.bits("W_down"))
+    workers = workers or max(1, min(16, (os.cpu_count() or 1)))
+    chunks = [c for c in np.array_split(np.asarray(rows, dtype=np.int64), workers) if c.size]
+    if len(chunks) <= 1:
+        return o.expert_rows(*args, ids, weights, rows).out
+    with ThreadPoolExecutor(max_workers=len(chunks)) as pool:
+        parts = list(pool.map(lambda c: o.expert_rows(*args, ids, weights, c).out, chunks))
+    return np.concatenate(parts, axis=0)
 
 
 @functools.lru_cache(maxsize=8)
@@ -54,12 +77,10 @@ def oracle_rows(cfg: MoEConfig, n: int):
     inp = inputs(cfg)
     r = oracle_route(cfg)
     rows = sample_for(cfg, n)
-    ex = default_oracle().expert_rows(inp.bits("x"), inp.bits("W_gate"), inp.bits("W_up"), inp.bits("W_down"),
-                                      r.ids, r.weights, rows)
-    return rows, ex.out
+    return rows, expert_rows_parallel(inp, r.ids, r.weights, rows)
 
 
-SAMPLES = {"tiny": 256, "qwen": 384, "fine": 384, "coarse": 24, "skew": 256}
+SAMPLES = {"tiny": 256, "qwen": 384, "fine": 384, "coarse": 160, "skew": 256}
 FULL = [CONFIGS[n] for n in ("tiny", "qwen", "fine", "coarse", "skew")]
 
 

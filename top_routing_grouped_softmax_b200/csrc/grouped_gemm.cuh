@@ -469,7 +469,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             for (int q = 0; q < kStages; ++q) {
                 const int64_t cnt = issued / kStages + (q < issued % kStages ? 1 : 0);
-                if (cnt > 0) mbar_wait(&c.full[q], (uint32_t)(cnt - 1) & 1u, limit);
+                if (cnt > 0) mbar_wait(&c.full[q], (uint32_t)(cnt - 1) & 1u, drain_limit(limit));
             }
         }
         __syncwarp(pmask);
@@ -522,7 +522,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             mma_commit(&c.done);
-            mbar_wait(&c.done, 0, limit);
+            mbar_wait(&c.done, 0, drain_limit(limit));
         }
         __syncwarp();
     } else {

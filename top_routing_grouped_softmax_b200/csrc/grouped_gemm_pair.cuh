@@ -157,7 +157,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             // only after the stage's bytes arrived).
             for (int q = 0; q < kPairStages; ++q) {
                 const int64_t cnt = issued / kPairStages + (q < issued % kPairStages ? 1 : 0);
-                if (cnt > 0) mbar_wait(leader ? &c.full[q] : &c.empty[q], (uint32_t)(cnt - 1) & 1u, limit);
+                if (cnt > 0)
+                    mbar_wait(leader ? &c.full[q] : &c.empty[q], (uint32_t)(cnt - 1) & 1u, drain_limit(limit));
             }
         }
         __syncwarp();
@@ -208,7 +209,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             mma_commit_pair(&c.done);
-            mbar_wait(&c.done, 0, limit);
+            mbar_wait(&c.done, 0, drain_limit(limit));
         }
         __syncwarp();
     } else {

@@ -42,16 +42,58 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
 
 constexpr int kMaxDevices = 64;
 
+// Per-device state lives as long as the context it was set up in: kernel
+// attributes and symbol addresses belong to a context, and a caller may
+// destroy the device's primary context (cudaDeviceReset) and carry on in a
+// new one.  Each entry records the unique id of its context and is set up
+// again when the current context's id differs.
 struct DeviceState {
     bool init = false;
     bool supported = false;
     int sm_count = 0;
     int max_pairs = 0;  // co-resident 2-CTA clusters of the pair GEMM
+    unsigned long long ctx_id = 0;
 };
 
 std::mutex g_mu;
 DeviceState g_dev[kMaxDevices];
 EncodeTiledFn g_encode = nullptr;
+
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+CtxGetCurrentFn g_ctx_get_current = nullptr;
+CtxGetIdFn g_ctx_get_id = nullptr;
+
+// Process-unique id of the calling thread's current context on device `dev`
+// (its primary context is made current first if the thread has none).
+// Called with g_mu held.
+int current_context_id(int dev, unsigned long long* id)
+{
+    cudaDriverEntryPointQueryResult q;
+    if (!g_ctx_get_current) {
+        void* fn = nullptr;
+        if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &fn, 12000, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || !fn)
+            return MOE_ERR_CUDA;
+        g_ctx_get_current = reinterpret_cast<CtxGetCurrentFn>(fn);
+    }
+    if (!g_ctx_get_id) {
+        void* fn = nullptr;
+        if (cudaGetDriverEntryPointByVersion("cuCtxGetId", &fn, 12000, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || !fn)
+            return MOE_ERR_CUDA;
+        g_ctx_get_id = reinterpret_cast<CtxGetIdFn>(fn);
+    }
+    CUcontext ctx = nullptr;
+    if (g_ctx_get_current(&ctx) != CUDA_SUCCESS) return MOE_ERR_CUDA;
+    if (!ctx) {
+        // no context current on this thread yet: cudaSetDevice initialises the
+        // device's primary context and makes it current
+        if (cudaSetDevice(dev) != cudaSuccess || g_ctx_get_current(&ctx) != CUDA_SUCCESS || !ctx)
+            return MOE_ERR_CUDA;
+    }
+    return g_ctx_get_id(ctx, id) == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
+}
 
 constexpr int kMaxDynSmem = 227 * 1024;
 
@@ -118,6 +160,9 @@ int setup_device(DeviceState** out)
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MOE_ERR_CUDA;
     std::lock_guard<std::mutex> lock(g_mu);
     DeviceState& st = g_dev[dev];
+    unsigned long long ctx_id = 0;
+    if (current_context_id(dev, &ctx_id)) return MOE_ERR_CUDA;
+    if (st.init && st.ctx_id != ctx_id) st = DeviceState{};  // a new context: set up again
     if (!st.init) {
         int major = 0, minor = 0, sms = 0;
         if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
@@ -172,6 +217,7 @@ int setup_device(DeviceState** out)
             }
             if (e != cudaSuccess) return MOE_ERR_CUDA;
         }
+        st.ctx_id = ctx_id;
         st.init = true;
     }
     if (!st.supported) return MOE_ERR_UNSUPPORTED_DEVICE;
@@ -722,19 +768,24 @@ constexpr int64_t kStaticPermuteScratchInts = int64_t(1) << 18;
 static __device__ __align__(256) int32_t g_static_permute_scratch[kStaticPermuteScratchInts];
 
 int32_t* g_static_scratch_addr[kMaxDevices] = {};
+unsigned long long g_static_scratch_ctx[kMaxDevices] = {};
 
 // The array's device address for the current device.  In host code the
 // symbol name is only a host-side stand-in, so the address is looked up once
-// per device with that device current, checked, and cached.
+// per device (and context) with that device current, checked, and cached;
+// a new context on the device (after cudaDeviceReset) gets a new lookup.
 int static_permute_scratch(int32_t** out)
 {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MOE_ERR_CUDA;
     std::lock_guard<std::mutex> lock(g_mu);
-    if (!g_static_scratch_addr[dev]) {
+    unsigned long long ctx_id = 0;
+    if (current_context_id(dev, &ctx_id)) return MOE_ERR_CUDA;
+    if (!g_static_scratch_addr[dev] || g_static_scratch_ctx[dev] != ctx_id) {
         void* addr = nullptr;
         if (cudaGetSymbolAddress(&addr, g_static_permute_scratch) != cudaSuccess || !addr) return MOE_ERR_CUDA;
         g_static_scratch_addr[dev] = static_cast<int32_t*>(addr);
+        g_static_scratch_ctx[dev] = ctx_id;
     }
     *out = g_static_scratch_addr[dev];
     return MOE_OK;
@@ -983,7 +1034,9 @@ int moe_get_status(cudaStream_t stream)
 
 int moe_set_wait_limit_ns(int64_t limit_ns)
 {
-    const unsigned long long v = limit_ns > 0 ? (unsigned long long)limit_ns : 1000000000ull;
+    // <= 0: the default (1 s); otherwise at least 1 ms
+    const unsigned long long v =
+        limit_ns <= 0 ? 1000000000ull : (limit_ns < 1000000 ? 1000000ull : (unsigned long long)limit_ns);
     return cudaMemcpyToSymbol(moe::g_wait_limit_ns, &v, sizeof(v)) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 

@@ -75,6 +75,16 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64
     }
 }
 
+// Limit for the waits of the wind-down after an abort: a CTA waits for its
+// own copies and MMAs in flight before it frees TMEM or exits, for at least
+// one second whatever the (caller-tunable) pipeline wait limit is, so a small
+// limit can end a pipeline early but never leaves an async write landing in
+// memory the CTA has given up.
+__device__ __forceinline__ uint64_t drain_limit(uint64_t limit_ns)
+{
+    return limit_ns > 1000000000ull ? limit_ns : 1000000000ull;
+}
+
 // -------------------------------------------------------------------- TMA
 // 2-D tiled bulk tensor load global -> shared, completion counted in bytes
 // on `bar`.  c0 is the innermost (contiguous) coordinate in elements.

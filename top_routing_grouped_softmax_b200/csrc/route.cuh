@@ -408,7 +408,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // Never leave the CTA with a copy still landing in its shared memory.
             for (int s = 0; s < p.stages; ++s) {
                 const int cnt = issued / p.stages + (s < issued % p.stages ? 1 : 0);
-                if (cnt > 0) mbar_wait(&full[s], (uint32_t)(cnt - 1) & 1u, limit);
+                if (cnt > 0) mbar_wait(&full[s], (uint32_t)(cnt - 1) & 1u, drain_limit(limit));
             }
         }
         __syncwarp();
@@ -447,7 +447,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     // ---------------------------------------------------------- epilogue
     bool have = true;
-    if (lane == 0) have = mbar_wait(done, 0, limit);
+    if (lane == 0) have = mbar_wait(done, 0, drain_limit(limit));
     have = __shfl_sync(0xffffffffu, have ? 1 : 0, 0) != 0;
     tc_fence_after_sync();
     // a timed-out wait already recorded the device status; every thread of
