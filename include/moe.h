@@ -359,6 +359,41 @@ int moe_forward_rounded(const moe_bf16* x, const moe_bf16* w_router, const float
                         cudaEvent_t* events, int n_events);
 
 /*
+ * Backward of the block (optional; the article's block is forward only): the
+ * gradient of L = sum_t dout[t] . out[t] with respect to x, W_router, the
+ * bias and the three expert weight tensors, following the memory rule of
+ * the SonicMoE comparison page ("SonicMoE vs conventional MoE", core
+ * difference 1): nothing from the forward is kept beyond the inputs; the
+ * routing, the permutation and the expert activations g, u and h are
+ * recomputed.  With e = ids[t][j], w = w[t][j], s = 1/(1+e^-g):
+ *   dh          = w * dout[t] . W_down[e]^T
+ *   dg          = dh * u * s * (1 + g * (1 - s)),   du = dh * g * s
+ *   dW_down[e] += (w h)^T dout[t],  dW_gate[e] += x[t]^T dg,  dW_up[e] += x[t]^T du
+ *   dx[t]      += dg . W_gate[e]^T + du . W_up[e]^T
+ *   dw_j        = dout[t] . (h . W_down[e])          (the routing weight's gradient)
+ *   dp[e]       = dw_j at e = ids[t][j], else 0      (with MOE_FLAG_RENORMALIZE:
+ *                 (dw_j - sum_m w_m dw_m) / S, S = sum of the k probabilities)
+ *   dlogit      = p * (dp - sum_e p_e dp_e)
+ *   dW_router  += x[t]^T dlogit,  dbias += dlogit,  dx[t] += dlogit . W_router^T
+ * The top-k choice itself passes no gradient.
+ *   dout [T, d] fp32 in; dx [T, d] fp32 out; dw_router [d, E], dbias [E]
+ *   (NULL to skip), dw_gate / dw_up [E, d, f], dw_down [E, f, d]: fp32 out,
+ *   overwritten (experts no token selects get zeros).  All 16-byte aligned.
+ * Precision: the GEMM operands are bf16 (x, the weights, dout, dg, du, w h
+ * and dlogit rounded once each), every sum fp32.  flags: 0 or
+ * MOE_FLAG_RENORMALIZE (the routing the forward used).  Workspace:
+ * moe_backward_workspace_size bytes, 256-byte aligned; grouped rows are
+ * padded so that each expert's group starts on a 64-row boundary.
+ */
+size_t moe_backward_workspace_size(int64_t T, int64_t d, int64_t E, int64_t k, int64_t f);
+
+int moe_backward(const moe_bf16* x, const moe_bf16* w_router, const float* bias,
+                 const moe_bf16* w_gate, const moe_bf16* w_up, const moe_bf16* w_down, const float* dout,
+                 int64_t T, int64_t d, int64_t E, int64_t k, int64_t f,
+                 float* dx, float* dw_router, float* dbias, float* dw_gate, float* dw_up, float* dw_down,
+                 void* workspace, size_t workspace_bytes, cudaStream_t stream, unsigned flags);
+
+/*
  * Synchronises `stream`, then returns and clears the current device's status
  * word (MOE_OK if no device-side error was recorded since the last call).
  */

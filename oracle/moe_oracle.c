@@ -582,3 +582,170 @@ done:
     free(dh); free(dg); free(du); free(dwj); free(dp); free(dl);
     return rc;
 }
+
+/*
+ * The backward restricted to what a sampled check at full size needs; each
+ * follows oracle_backward's arithmetic and summation order, so its results
+ * equal the corresponding entries of oracle_backward's outputs.
+ *
+ * oracle_backward_rows: dx_rows[r] = dx[rows[r]] (fp64 [n_rows][d]).  dx[t]
+ * depends only on token t (its routing, its k expert evaluations and its
+ * router gradient), so each row is computed from that token alone.
+ */
+int oracle_backward_rows(const uint16_t* x, const uint16_t* w_router, const float* bias,
+                         const uint16_t* w_gate, const uint16_t* w_up, const uint16_t* w_down,
+                         int64_t T, int64_t d, int64_t E, int64_t k, int64_t f, int renormalize,
+                         const double* dout, int64_t n_rows, const int64_t* rows, double* dx_rows)
+{
+    if (!x || !w_router || !w_gate || !w_up || !w_down || !dout || !rows || !dx_rows || T < 0 || d < 1 ||
+        E < 1 || k < 1 || k > E || f < 1 || n_rows < 0)
+        return ORACLE_BAD_ARG;
+    int32_t* ids = (int32_t*)malloc(sizeof(int32_t) * (size_t)k);
+    double* w = (double*)malloc(sizeof(double) * (size_t)k);
+    double* probs = (double*)malloc(sizeof(double) * (size_t)E);
+    double* xrow = (double*)malloc(sizeof(double) * (size_t)d);
+    double* g = (double*)malloc(sizeof(double) * (size_t)f);
+    double* u = (double*)malloc(sizeof(double) * (size_t)f);
+    double* h = (double*)malloc(sizeof(double) * (size_t)f);
+    double* z = (double*)malloc(sizeof(double) * (size_t)d);
+    double* dz = (double*)malloc(sizeof(double) * (size_t)d);
+    double* dh = (double*)malloc(sizeof(double) * (size_t)f);
+    double* dg = (double*)malloc(sizeof(double) * (size_t)f);
+    double* du = (double*)malloc(sizeof(double) * (size_t)f);
+    double* dwj = (double*)malloc(sizeof(double) * (size_t)k);
+    double* dp = (double*)malloc(sizeof(double) * (size_t)E);
+    double* dl = (double*)malloc(sizeof(double) * (size_t)E);
+    int rc = ORACLE_NO_MEMORY;
+    if (!ids || !w || !probs || !xrow || !g || !u || !h || !z || !dz || !dh || !dg || !du || !dwj || !dp || !dl)
+        goto done;
+    rc = ORACLE_OK;
+    for (int64_t r = 0; r < n_rows && rc == ORACLE_OK; ++r) {
+        const int64_t t = rows[r];
+        if (t < 0 || t >= T) { rc = ORACLE_BAD_ARG; break; }
+        rc = oracle_route(x + t * d, w_router, bias, 1, d, E, k, NULL, probs, ids, w);
+        if (rc != ORACLE_OK) break;
+        if (renormalize && (rc = oracle_renormalize(w, 1, k)) != ORACLE_OK) break;
+        double* dxr = dx_rows + r * d;
+        for (int64_t i = 0; i < d; ++i) { xrow[i] = bf16_to_double(x[t * d + i]); dxr[i] = 0.0; }
+        const double* drow_out = dout + t * d;
+        for (int64_t j = 0; j < k; ++j) {
+            const int64_t e = ids[j];
+            const uint16_t* wg = w_gate + e * d * f;
+            const uint16_t* wu = w_up + e * d * f;
+            const uint16_t* wd = w_down + e * f * d;
+            expert_swiglu(xrow, wg, wu, wd, d, f, g, u, h, z);
+            double s = 0.0;
+            for (int64_t c = 0; c < d; ++c) s += drow_out[c] * z[c];
+            dwj[j] = s;
+            for (int64_t c = 0; c < d; ++c) dz[c] = w[j] * drow_out[c];
+            for (int64_t n = 0; n < f; ++n) {
+                double acc = 0.0;
+                for (int64_t c = 0; c < d; ++c) acc += dz[c] * bf16_to_double(wd[n * d + c]);
+                dh[n] = acc;
+            }
+            for (int64_t n = 0; n < f; ++n) {
+                const double sg = 1.0 / (1.0 + exp(-g[n]));
+                du[n] = dh[n] * (g[n] * sg);
+                dg[n] = dh[n] * u[n] * sg * (1.0 + g[n] * (1.0 - sg));
+            }
+            for (int64_t i = 0; i < d; ++i) {
+                double acc = 0.0;
+                for (int64_t n = 0; n < f; ++n)
+                    acc += dg[n] * bf16_to_double(wg[i * f + n]) + du[n] * bf16_to_double(wu[i * f + n]);
+                dxr[i] += acc;
+            }
+        }
+        for (int64_t e = 0; e < E; ++e) dp[e] = 0.0;
+        if (renormalize) {
+            double ssum = 0.0, dot = 0.0;
+            for (int64_t j = 0; j < k; ++j) ssum += probs[ids[j]];
+            for (int64_t j = 0; j < k; ++j) dot += dwj[j] * w[j];
+            for (int64_t j = 0; j < k; ++j) dp[ids[j]] = (dwj[j] - dot) / ssum;
+        } else {
+            for (int64_t j = 0; j < k; ++j) dp[ids[j]] = dwj[j];
+        }
+        double pdp = 0.0;
+        for (int64_t e = 0; e < E; ++e) pdp += probs[e] * dp[e];
+        for (int64_t e = 0; e < E; ++e) dl[e] = probs[e] * (dp[e] - pdp);
+        for (int64_t i = 0; i < d; ++i) {
+            double acc = 0.0;
+            const uint16_t* wrow = w_router + i * E;
+            for (int64_t e = 0; e < E; ++e) acc += dl[e] * bf16_to_double(wrow[e]);
+            dxr[i] += acc;
+        }
+    }
+done:
+    free(ids); free(w); free(probs); free(xrow); free(g); free(u); free(h); free(z); free(dz);
+    free(dh); free(dg); free(du); free(dwj); free(dp); free(dl);
+    return rc;
+}
+
+/*
+ * oracle_backward_expert: the weight gradients of one expert e_sel,
+ * dw_gate_e, dw_up_e [d][f] and dw_down_e [f][d] (fp64, overwritten): the
+ * contributions of the (token, slot) pairs routed to e_sel, tokens in
+ * ascending order, exactly as oracle_backward accumulates dW[e_sel].
+ */
+int oracle_backward_expert(const uint16_t* x, const uint16_t* w_router, const float* bias,
+                           const uint16_t* w_gate, const uint16_t* w_up, const uint16_t* w_down,
+                           int64_t T, int64_t d, int64_t E, int64_t k, int64_t f, int renormalize,
+                           const double* dout, int64_t e_sel, double* dw_gate_e, double* dw_up_e,
+                           double* dw_down_e)
+{
+    if (!x || !w_router || !w_gate || !w_up || !w_down || !dout || !dw_gate_e || !dw_up_e || !dw_down_e ||
+        T < 0 || d < 1 || E < 1 || k < 1 || k > E || f < 1 || e_sel < 0 || e_sel >= E)
+        return ORACLE_BAD_ARG;
+    int32_t* ids = (int32_t*)malloc(sizeof(int32_t) * (size_t)(T * k + 1));
+    double* w = (double*)malloc(sizeof(double) * (size_t)(T * k + 1));
+    double* xrow = (double*)malloc(sizeof(double) * (size_t)d);
+    double* g = (double*)malloc(sizeof(double) * (size_t)f);
+    double* u = (double*)malloc(sizeof(double) * (size_t)f);
+    double* h = (double*)malloc(sizeof(double) * (size_t)f);
+    double* z = (double*)malloc(sizeof(double) * (size_t)d);
+    double* dz = (double*)malloc(sizeof(double) * (size_t)d);
+    double* dh = (double*)malloc(sizeof(double) * (size_t)f);
+    double* dg = (double*)malloc(sizeof(double) * (size_t)f);
+    double* du = (double*)malloc(sizeof(double) * (size_t)f);
+    int rc = ORACLE_NO_MEMORY;
+    if (!ids || !w || !xrow || !g || !u || !h || !z || !dz || !dh || !dg || !du) goto done;
+    rc = oracle_route(x, w_router, bias, T, d, E, k, NULL, NULL, ids, w);
+    if (rc != ORACLE_OK) goto done;
+    if (renormalize && (rc = oracle_renormalize(w, T, k)) != ORACLE_OK) goto done;
+    memset(dw_gate_e, 0, sizeof(double) * (size_t)(d * f));
+    memset(dw_up_e, 0, sizeof(double) * (size_t)(d * f));
+    memset(dw_down_e, 0, sizeof(double) * (size_t)(f * d));
+    const uint16_t* wg = w_gate + e_sel * d * f;
+    const uint16_t* wu = w_up + e_sel * d * f;
+    const uint16_t* wd = w_down + e_sel * f * d;
+    for (int64_t t = 0; t < T; ++t) {
+        for (int64_t j = 0; j < k; ++j) {
+            if (ids[t * k + j] != e_sel) continue;
+            for (int64_t i = 0; i < d; ++i) xrow[i] = bf16_to_double(x[t * d + i]);
+            const double* drow_out = dout + t * d;
+            expert_swiglu(xrow, wg, wu, wd, d, f, g, u, h, z);
+            for (int64_t c = 0; c < d; ++c) dz[c] = w[t * k + j] * drow_out[c];
+            for (int64_t n = 0; n < f; ++n) {
+                double acc = 0.0;
+                for (int64_t c = 0; c < d; ++c) {
+                    dw_down_e[n * d + c] += h[n] * dz[c];
+                    acc += dz[c] * bf16_to_double(wd[n * d + c]);
+                }
+                dh[n] = acc;
+            }
+            for (int64_t n = 0; n < f; ++n) {
+                const double sg = 1.0 / (1.0 + exp(-g[n]));
+                du[n] = dh[n] * (g[n] * sg);
+                dg[n] = dh[n] * u[n] * sg * (1.0 + g[n] * (1.0 - sg));
+            }
+            for (int64_t i = 0; i < d; ++i)
+                for (int64_t n = 0; n < f; ++n) {
+                    dw_gate_e[i * f + n] += xrow[i] * dg[n];
+                    dw_up_e[i * f + n] += xrow[i] * du[n];
+                }
+        }
+    }
+    rc = ORACLE_OK;
+done:
+    free(ids); free(w); free(xrow); free(g); free(u); free(h); free(z); free(dz); free(dh); free(dg); free(du);
+    return rc;
+}

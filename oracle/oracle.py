@@ -72,6 +72,12 @@ class Oracle:
         lib.oracle_backward.argtypes = [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64, ctypes.c_int,
                                         _P, _P, _P, _P, _P, _P, _P]
         lib.oracle_backward.restype = ctypes.c_int
+        lib.oracle_backward_rows.argtypes = [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64, ctypes.c_int,
+                                             _P, _I64, _P, _P]
+        lib.oracle_backward_rows.restype = ctypes.c_int
+        lib.oracle_backward_expert.argtypes = [_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64,
+                                               ctypes.c_int, _P, _I64, _P, _P, _P]
+        lib.oracle_backward_expert.restype = ctypes.c_int
         for fn in (lib.oracle_route, lib.oracle_permute, lib.oracle_expert_rows, lib.oracle_renormalize):
             fn.restype = ctypes.c_int
         self.lib = lib
@@ -226,6 +232,47 @@ class Oracle:
         if rc != 0:
             raise ValueError(f"oracle_backward failed ({rc})")
         return g
+
+
+    def _bwd_args(self, x, w_router, bias, w_gate, w_up, w_down, dout):
+        x = np.ascontiguousarray(x, dtype=np.uint16)
+        w_router = np.ascontiguousarray(w_router, dtype=np.uint16)
+        w_gate = np.ascontiguousarray(w_gate, dtype=np.uint16)
+        w_up = np.ascontiguousarray(w_up, dtype=np.uint16)
+        w_down = np.ascontiguousarray(w_down, dtype=np.uint16)
+        dout = np.ascontiguousarray(dout, dtype=np.float64)
+        b = None if bias is None else np.ascontiguousarray(bias, dtype=np.float32)
+        return x, w_router, b, w_gate, w_up, w_down, dout
+
+    def backward_rows(self, x, w_router, bias, w_gate, w_up, w_down, k, dout, rows, renormalize=False):
+        """dx of the chosen tokens only ([len(rows), d] fp64), equal to the
+        corresponding rows of backward()'s dx."""
+        x, w_router, b, w_gate, w_up, w_down, dout = self._bwd_args(x, w_router, bias, w_gate, w_up, w_down, dout)
+        rows = np.ascontiguousarray(rows, dtype=np.int64)
+        T, d = x.shape
+        E = w_router.shape[1]
+        f = w_gate.shape[2]
+        out = np.empty((rows.shape[0], d), np.float64)
+        rc = self.lib.oracle_backward_rows(_ptr(x), _ptr(w_router), _ptr(b), _ptr(w_gate), _ptr(w_up), _ptr(w_down),
+                                           T, d, E, k, f, 1 if renormalize else 0, _ptr(dout), rows.shape[0],
+                                           _ptr(rows), _ptr(out))
+        if rc != 0:
+            raise ValueError(f"oracle_backward_rows failed ({rc})")
+        return out
+
+    def backward_expert(self, x, w_router, bias, w_gate, w_up, w_down, k, dout, e, renormalize=False):
+        """(dW_gate[e], dW_up[e], dW_down[e]) in fp64, equal to backward()'s."""
+        x, w_router, b, w_gate, w_up, w_down, dout = self._bwd_args(x, w_router, bias, w_gate, w_up, w_down, dout)
+        T, d = x.shape
+        E = w_router.shape[1]
+        f = w_gate.shape[2]
+        gg, gu, gd = np.empty((d, f)), np.empty((d, f)), np.empty((f, d))
+        rc = self.lib.oracle_backward_expert(_ptr(x), _ptr(w_router), _ptr(b), _ptr(w_gate), _ptr(w_up),
+                                             _ptr(w_down), T, d, E, k, f, 1 if renormalize else 0, _ptr(dout), e,
+                                             _ptr(gg), _ptr(gu), _ptr(gd))
+        if rc != 0:
+            raise ValueError(f"oracle_backward_expert failed ({rc})")
+        return gg, gu, gd
 
 
 @dataclass

@@ -469,10 +469,25 @@ def check_backward_invariants(o):
         assert np.array_equal(getattr(g2, name), 2.0 * getattr(g, name)), name
 
 
+def check_backward_restricted(o):
+    """The per-token dx and per-expert weight gradients (for sampled checks
+    at full size) equal the corresponding entries of the whole backward."""
+    for (T, d, E, k, f, seed, bias, ren) in [(24, 32, 8, 3, 16, 31, True, False), (30, 64, 8, 2, 32, 5, False, True)]:
+        inp = _rand_case(T, d, E, k, f, seed, bias=bias, sigma=0.2)
+        dout = _dout(T, d, seed)
+        g = o.backward(*_args(inp), k, dout, renormalize=ren)
+        rows = np.array([0, T // 2, T - 1])
+        assert np.array_equal(o.backward_rows(*_args(inp), k, dout, rows, renormalize=ren), g.dx[rows]), "dx rows"
+        for e in range(E):
+            gg, gu, gd = o.backward_expert(*_args(inp), k, dout, e, renormalize=ren)
+            assert np.array_equal(gg, g.dw_gate[e]) and np.array_equal(gu, g.dw_up[e]), ("expert", e)
+            assert np.array_equal(gd, g.dw_down[e]), ("expert down", e)
+
+
 ALL_CHECKS = [
     check_brute_force, check_softmax_library, check_topk_library_sort, check_topk_of_logits,
     check_exact_ties, check_dense_special_case, check_all_experts_identical, check_zero_expert,
     check_scale_down, check_permute_library, check_expert_rows_outputs,
     check_renormalize, check_shared_experts, check_token_rounding, check_backward_autograd,
-    check_backward_finite_differences, check_backward_invariants,
+    check_backward_finite_differences, check_backward_invariants, check_backward_restricted,
 ]

@@ -54,13 +54,23 @@ MUTANTS = [
     ("bwd_renorm_no_dot", "dp[ids[t * k + j]] = (dwj[j] - dot) / ssum;", "dp[ids[t * k + j]] = dwj[j] / ssum;"),
     ("bwd_down_transposed", "acc += dz[c] * bf16_to_double(wd[n * d + c]);",
      "acc += dz[c] * bf16_to_double(wd[c * f + n]);"),
+    ("bwd_rows_without_router", "            for (int64_t e = 0; e < E; ++e) acc += dl[e] * bf16_to_double(wrow[e]);\n            dxr[i] += acc;",
+     "            for (int64_t e = 0; e < E; ++e) acc += 0.0 * dl[e] * bf16_to_double(wrow[e]);\n            dxr[i] += acc;"),
+    ("bwd_rows_no_routing_weight", "for (int64_t c = 0; c < d; ++c) dz[c] = w[j] * drow_out[c];",
+     "for (int64_t c = 0; c < d; ++c) dz[c] = drow_out[c];"),
+    ("bwd_expert_no_routing_weight", "for (int64_t c = 0; c < d; ++c) dz[c] = w[t * k + j] * drow_out[c];",
+     "for (int64_t c = 0; c < d; ++c) dz[c] = drow_out[c];"),
+    ("bwd_expert_up_uses_gate", "                    dw_up_e[i * f + n] += xrow[i] * du[n];",
+     "                    dw_up_e[i * f + n] += xrow[i] * dg[n];"),
 ]
 
 
 @pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
 def test_pins_catch_mutant(tmp_path, name, old, new):
     src = open(SRC).read()
-    assert src.count(old) == 1, f"mutation site for {name} not found exactly once"
+    # the per-token and per-expert restrictions of the backward repeat some of
+    # its lines; a slip in such a line is planted in every copy of it
+    assert src.count(old) >= 1, f"mutation site for {name} not found"
     mut_src = tmp_path / f"mut_{name}.c"
     mut_src.write_text(src.replace(old, new))
     lib = compile_oracle(str(mut_src), str(tmp_path / f"lib_{name}.so"), force=True)

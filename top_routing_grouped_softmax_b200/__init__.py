@@ -8,8 +8,9 @@ CUDA stream.  There is no CPU or PyTorch fallback: if the library is missing
 or the device is not a B200, the calls raise.
 
 Functions mirror the ABI entry points:
-  route, permute, expert_ffn, combine, forward (and forward_profiled),
-  workspace_size, permute_workspace_size, get_status, set_wait_limit_ns.
+  route, permute, expert_ffn, combine, forward, backward, the shared-expert
+  and token-rounding variants, the *_workspace_size queries, get_status,
+  set_wait_limit_ns.
 ``MoEBlock`` keeps the weights and a reusable workspace for repeated calls.
 """
 from __future__ import annotations
@@ -40,6 +41,7 @@ ABI_SYMBOLS = (
     "moe_forward_ex", "moe_get_status", "moe_set_wait_limit_ns", "moe_selftest_wait_timeout",
     "moe_permute_static", "moe_route_ex", "moe_workspace_size_shared", "moe_shared_ffn", "moe_combine_shared",
     "moe_forward_shared", "moe_workspace_size_rounded", "moe_forward_rounded",
+    "moe_backward_workspace_size", "moe_backward",
 )
 
 
@@ -92,13 +94,16 @@ def lib() -> ctypes.CDLL:
         L.moe_forward_rounded.argtypes = [_P] * 6 + [_I64] * 6 + [_P, _P, _P, _P, _SZ, _P, _P, ctypes.c_int]
         L.moe_forward_shared.argtypes = ([_P] * 9 + [_I64] * 7 + [_P, _P, _P, _P, _SZ, _P, _P, ctypes.c_int,
                                                                    ctypes.c_uint])
+        L.moe_backward_workspace_size.restype = _SZ
+        L.moe_backward_workspace_size.argtypes = [_I64] * 5
+        L.moe_backward.argtypes = [_P] * 7 + [_I64] * 5 + [_P] * 7 + [_SZ, _P, ctypes.c_uint]
         L.moe_get_status.argtypes = [_P]
         L.moe_set_wait_limit_ns.argtypes = [_I64]
         L.moe_selftest_wait_timeout.argtypes = [_I64, _P]
         for name in ("moe_route", "moe_permute", "moe_expert_ffn", "moe_combine", "moe_forward",
                      "moe_forward_ex", "moe_get_status", "moe_set_wait_limit_ns",
                      "moe_selftest_wait_timeout", "moe_permute_static", "moe_route_ex", "moe_shared_ffn",
-                     "moe_combine_shared", "moe_forward_shared", "moe_forward_rounded"):
+                     "moe_combine_shared", "moe_forward_shared", "moe_forward_rounded", "moe_backward"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -364,6 +369,39 @@ def forward(x, w_router, w_gate, w_up, w_down, k, bias=None, out=None, workspace
     return out
 
 
+def backward_workspace_size(T: int, d: int, E: int, k: int, f: int) -> int:
+    return int(lib().moe_backward_workspace_size(T, d, E, k, f))
+
+
+def backward(x, w_router, w_gate, w_up, w_down, k, dout, bias=None, workspace=None, renormalize=False,
+             want_dbias=True):
+    """Gradient of sum(dout * out) of the block (moe_backward): returns a dict
+    of fp32 tensors dx [T, d], dw_router [d, E], dbias [E] (None unless
+    want_dbias), dw_gate / dw_up [E, d, f], dw_down [E, f, d]."""
+    T, d, E, f = _forward_args(x, w_router, w_gate, w_up, w_down, bias)
+    _need(dout, "dout", torch.float32, 2)
+    dev = x.device
+    g = {
+        "dx": torch.empty(T, d, dtype=torch.float32, device=dev),
+        "dw_router": torch.empty(d, E, dtype=torch.float32, device=dev),
+        "dbias": torch.empty(E, dtype=torch.float32, device=dev) if want_dbias else None,
+        "dw_gate": torch.empty(E, d, f, dtype=torch.float32, device=dev),
+        "dw_up": torch.empty(E, d, f, dtype=torch.float32, device=dev),
+        "dw_down": torch.empty(E, f, d, dtype=torch.float32, device=dev),
+    }
+    nbytes = backward_workspace_size(T, d, E, k, f)
+    if nbytes == 0:
+        raise MoEError(MOE_ERR_UNSUPPORTED_SHAPE, "moe_backward_workspace_size")
+    if workspace is None:
+        workspace = _workspace(nbytes, dev)
+    flags = MOE_FLAG_RENORMALIZE if renormalize else 0
+    _check(lib().moe_backward(_ptr(x), _ptr(w_router), _ptr(bias), _ptr(w_gate), _ptr(w_up), _ptr(w_down),
+                              _ptr(dout), T, d, E, k, f, _ptr(g["dx"]), _ptr(g["dw_router"]), _ptr(g["dbias"]),
+                              _ptr(g["dw_gate"]), _ptr(g["dw_up"]), _ptr(g["dw_down"]), _ptr(workspace),
+                              workspace.numel(), _stream(), flags), "moe_backward")
+    return g
+
+
 def _event_array(events):
     """ctypes array of cudaEvent_t handles (None entries stay NULL), and its length."""
     if events is None:
@@ -420,6 +458,6 @@ __all__ = [
     "lib", "strerror", "MoEError", "ABI_SYMBOLS", "workspace_size", "route_workspace_size",
     "permute_workspace_size", "MOE_FLAG_FUSED_GATHER", "MOE_FLAG_RENORMALIZE", "route",
     "permute", "expert_ffn", "combine", "forward", "shared_ffn", "combine_shared", "forward_shared", "forward_rounded",
-    "get_status", "set_wait_limit_ns",
+    "get_status", "set_wait_limit_ns", "backward", "backward_workspace_size",
     "selftest_wait_timeout", "MoEBlock",
 ]

@@ -1,0 +1,512 @@
+// grouped_gemm_bwd.cuh -- the grouped GEMMs of the MoE block's backward on
+// CTA pairs (tcgen05 cta_group::2), with their epilogues fused in.
+//
+// The backward follows the memory rule of the SonicMoE comparison page ("SonicMoE
+// vs conventional MoE", core difference 1): only the routing is kept, and the
+// expert activations g, u and h are recomputed from the grouped rows of x.
+// Rows are grouped by expert with every group starting on a 64-row boundary
+// (the rows between a group's end and the next boundary are zero in every
+// row operand), so a group's rows can also serve as the reduction axis of
+// the weight gradients in whole 64-row blocks.
+//
+// Four kinds share one pipeline (the CTA-pair ring of the forward's grouped
+// GEMM: TMA producer, one MMA thread in the even CTA issuing M=256 N=256 K=16
+// pair MMAs, four epilogue warps per CTA over a double-buffered accumulator):
+//
+//   kGU  g, u = x_perm . W_gate[e], x_perm . W_up[e]      (recompute)
+//        A = x_perm rows (K-major), B = weight columns (MN-major): the even
+//        CTA loads W_gate's 128 columns, the odd CTA the matching W_up ones,
+//        so accumulator columns 0..127 are g and 128..255 are u.  Stored bf16.
+//   kDH  dh = w . (dout_perm . W_down[e]^T), then the SwiGLU derivative:
+//          s = 1/(1+e^-g),  h = g s u,
+//          dg = dh u s (1 + g (1 - s)),  du = dh g s,
+//        and the routing-weight gradient's partial dot products
+//          dwp[row][nt] = sum over this tile's columns of (dh / w) h
+//        (dh / w is the unweighted accumulator: dout . (h W_down) = (dout W_down^T) . h).
+//        A = dout_perm rows (K-major), B = W_down[e] rows (K-major: W_down[e] is
+//        [f][d], its rows are the output columns).  Stores dg, du and
+//        hw = w h (the operand of the W_down gradient) as bf16.
+//   kDX  out = A1 . B1^T + A2 . B2^T with K split in two halves (the first
+//        k_split 64-blocks read A1/B1, the rest A2/B2), fp32 store:
+//        dx_perm = dg . W_gate[e]^T + du . W_up[e]^T, and (one group, one half)
+//        the router's dx = dlogit . W_router^T.
+//   kDW  out[e] = A_e^T . B_e, reduced over the rows of group e:
+//        A = the group's rows read MN-major (x_perm or hw, or x), B likewise
+//        (dg | du split over the pair, or dout_perm / dlogit).  One work item
+//        is (expert, 256-row M tile, 256-column N tile); an empty group writes
+//        zeros.  fp32 store.
+//
+// No TMA load uses multicast.  Every wait is bounded (see ptx.cuh).
+#pragma once
+
+#include "grouped_gemm_pair.cuh"
+
+namespace moe {
+namespace bwd {
+
+using gemm::kABytes;
+using gemm::kBK;
+using gemm::kBM;
+using gemm::kBN;
+using gemm::kChunkBytes;
+using gemm::kEpiWarps;
+using gemm::kMaxE;
+using gemm::kPairRows;
+using gemm::kPairStageBytes;
+using gemm::kPairStages;
+using gemm::kThreads;
+using gemm::kTmemCols;
+
+enum Kind { kGU = 0, kDH = 1, kDX = 2, kDW = 3 };
+
+struct Params {
+    const int32_t* offsets;  // [E+1] group starts; nullptr: one group of M rows
+    const float* w_perm;     // kDH: routing weight of each grouped row
+    const __nv_bfloat16* g;  // kDH: recomputed g, u [rows][ld_f]
+    const __nv_bfloat16* u;
+    __nv_bfloat16* out_g;    // kGU: g;  kDH: dg        [rows][ld_f]
+    __nv_bfloat16* out_u;    // kGU: u;  kDH: du
+    __nv_bfloat16* out_hw;   // kDH: w * h
+    float* dwp;              // kDH: [rows][n_tiles] partial dot products
+    float* out0;             // kDX: [rows][ld_out];  kDW: [E][m_total][ld_out] (gate part when split)
+    float* out1;             // kDW split: the up part
+    int64_t ld_f;            // row length of g, u, dg, du, hw
+    int64_t ld_out;          // row length of out0 / out1
+    int E;
+    int M;                   // grouped rows (capacity: offsets[E] <= M)
+    int K;                   // kGU, kDH, kDX: reduction length (kDX: both halves)
+    int k_split;             // kDX: 64-blocks read from A1/B1 below this, A2/B2 from it on
+    int n_out;               // output columns
+    int n_tiles;             // N tiles per item (kGU: 128 output columns each, else 256)
+    int b_rows;              // kGU: weight rows per expert (d); kDH, kDX: B rows per expert (f, d)
+    int m_total;             // kDW: output rows per expert
+    int m_tiles;             // kDW: 256-row M tiles per expert
+    int split_b;             // kDW: 1 = B halves from two tensors (dg | du), two outputs
+};
+
+struct alignas(8) Ctrl {
+    uint64_t full[kPairStages];
+    uint64_t empty[kPairStages];
+    uint64_t acc_full[2];
+    uint64_t acc_empty[2];
+    uint64_t done;
+    uint32_t tmem_slot;
+    volatile int abort_flag;
+    int bad;
+    int total_mtiles;
+    int off[kMaxE + 1];
+    int tp[kMaxE + 1];
+};
+
+__host__ inline size_t smem_bytes() { return 1024 + (size_t)kPairStages * kPairStageBytes + sizeof(Ctrl); }
+
+// One work item of kind KIND: the expert, the first grouped row (M-grouped
+// kinds) or M tile (kDW), the group's row range, the N tile and the number
+// of 64-row k-blocks.
+struct Item {
+    int e, row0, row_end, nt, mt, kstart, num_kb;
+};
+
+template <int KIND>
+__device__ __forceinline__ Item decode_item(int64_t w, const Params& p, const Ctrl& c)
+{
+    Item it;
+    if constexpr (KIND == kDW) {
+        const int64_t per_e = (int64_t)p.m_tiles * p.n_tiles;
+        it.e = (int)(w / per_e);
+        const int rem = (int)(w - (int64_t)it.e * per_e);
+        it.mt = rem / p.n_tiles;
+        it.nt = rem - it.mt * p.n_tiles;
+        it.kstart = c.off[it.e];
+        it.num_kb = (c.off[it.e + 1] - c.off[it.e] + kBK - 1) / kBK;
+        it.row0 = it.kstart;
+        it.row_end = c.off[it.e + 1];
+    } else {
+        gemm::decode_tile<kPairRows>(w, p.n_tiles, c.tp, c.off, p.E, it.e, it.row0, it.row_end, it.nt);
+        it.mt = 0;
+        it.kstart = 0;
+        it.num_kb = p.K / kBK;
+    }
+    return it;
+}
+
+__device__ __forceinline__ float sigmoid(float z) { return 1.0f / (1.0f + __expf(-z)); }
+
+__device__ __forceinline__ void unpack_bf16x8(const uint4& q, float (&v)[8])
+{
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&q);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 f = __bfloat1622float2(h[i]);
+        v[2 * i] = f.x;
+        v[2 * i + 1] = f.y;
+    }
+}
+
+// Sixteen fp32 values to one row segment (four 16-byte stores).
+__device__ __forceinline__ void store_f32x16(float* dst, const uint32_t (&r)[16])
+{
+    float4* d4 = reinterpret_cast<float4*>(dst);
+#pragma unroll
+    for (int v = 0; v < 4; ++v)
+        d4[v] = make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]), __uint_as_float(r[4 * v + 2]),
+                            __uint_as_float(r[4 * v + 3]));
+}
+
+__device__ __forceinline__ void store_zero_f32x16(float* dst)
+{
+    float4* d4 = reinterpret_cast<float4*>(dst);
+#pragma unroll
+    for (int v = 0; v < 4; ++v) d4[v] = make_float4(0.f, 0.f, 0.f, 0.f);
+}
+
+// Drains one accumulator tile.  The calling warp reads TMEM lane quarter q:
+// row q*32 + lane of this CTA's 128 rows.  tbase addresses the accumulator
+// at this warp's lane quarter.
+template <int KIND>
+__device__ __forceinline__ void epilogue(const Params& p, const Item& it, uint32_t tbase, uint32_t rank, int q,
+                                         int lane)
+{
+    const int r = (int)rank * kBM + q * 32 + lane;  // row of the 256-row pair tile
+    if constexpr (KIND == kGU) {
+        const int row = it.row0 + r;
+        const bool valid = row < it.row_end;
+        const int c_base = it.nt * 128;
+        const int ncols = min(128, p.n_out - c_base);
+#pragma unroll 1
+        for (int c0 = 0; c0 < 128; c0 += 16) {
+            uint32_t g[16], u[16];
+            tmem_ld16(tbase + c0, g);
+            tmem_ld16(tbase + 128 + c0, u);
+            tmem_ld_wait();
+            if (valid && c0 < ncols) {
+                uint32_t pg[8], pu[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    pg[i] = gemm::pack_bf16x2(__uint_as_float(g[2 * i]), __uint_as_float(g[2 * i + 1]));
+                    pu[i] = gemm::pack_bf16x2(__uint_as_float(u[2 * i]), __uint_as_float(u[2 * i + 1]));
+                }
+                uint4* dg = reinterpret_cast<uint4*>(p.out_g + (int64_t)row * p.ld_f + c_base + c0);
+                uint4* du = reinterpret_cast<uint4*>(p.out_u + (int64_t)row * p.ld_f + c_base + c0);
+                dg[0] = make_uint4(pg[0], pg[1], pg[2], pg[3]);
+                dg[1] = make_uint4(pg[4], pg[5], pg[6], pg[7]);
+                du[0] = make_uint4(pu[0], pu[1], pu[2], pu[3]);
+                du[1] = make_uint4(pu[4], pu[5], pu[6], pu[7]);
+            }
+        }
+    } else if constexpr (KIND == kDH) {
+        const int row = it.row0 + r;
+        const bool valid = row < it.row_end;
+        const int c_base = it.nt * kBN;
+        const int ncols = min(kBN, p.n_out - c_base);
+        const float w = valid ? __ldg(p.w_perm + row) : 0.0f;
+        float dot = 0.0f;
+#pragma unroll 1
+        for (int c0 = 0; c0 < kBN; c0 += 16) {
+            uint32_t acc[16];
+            tmem_ld16(tbase + c0, acc);
+            tmem_ld_wait();
+            if (valid && c0 < ncols) {
+                const int64_t off = (int64_t)row * p.ld_f + c_base + c0;
+                const uint4* gp = reinterpret_cast<const uint4*>(p.g + off);
+                const uint4* up = reinterpret_cast<const uint4*>(p.u + off);
+                float g[16], u[16];
+                {
+                    float t[8];
+                    unpack_bf16x8(gp[0], t);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) g[i] = t[i];
+                    unpack_bf16x8(gp[1], t);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) g[8 + i] = t[i];
+                    unpack_bf16x8(up[0], t);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) u[i] = t[i];
+                    unpack_bf16x8(up[1], t);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) u[8 + i] = t[i];
+                }
+                uint32_t pdg[8], pdu[8], phw[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    float dgv[2], duv[2], hwv[2];
+#pragma unroll
+                    for (int h2 = 0; h2 < 2; ++h2) {
+                        const int c = 2 * i + h2;
+                        const float dhu = __uint_as_float(acc[c]);  // dout . W_down^T (unweighted)
+                        const float s = sigmoid(g[c]);
+                        const float gs = g[c] * s;
+                        const float h = gs * u[c];
+                        const float dh = w * dhu;
+                        dot += dhu * h;
+                        dgv[h2] = dh * u[c] * s * (1.0f + g[c] * (1.0f - s));
+                        duv[h2] = dh * gs;
+                        hwv[h2] = w * h;
+                    }
+                    pdg[i] = gemm::pack_bf16x2(dgv[0], dgv[1]);
+                    pdu[i] = gemm::pack_bf16x2(duv[0], duv[1]);
+                    phw[i] = gemm::pack_bf16x2(hwv[0], hwv[1]);
+                }
+                uint4* dgp = reinterpret_cast<uint4*>(p.out_g + off);
+                uint4* dup = reinterpret_cast<uint4*>(p.out_u + off);
+                uint4* hwp = reinterpret_cast<uint4*>(p.out_hw + off);
+                dgp[0] = make_uint4(pdg[0], pdg[1], pdg[2], pdg[3]);
+                dgp[1] = make_uint4(pdg[4], pdg[5], pdg[6], pdg[7]);
+                dup[0] = make_uint4(pdu[0], pdu[1], pdu[2], pdu[3]);
+                dup[1] = make_uint4(pdu[4], pdu[5], pdu[6], pdu[7]);
+                hwp[0] = make_uint4(phw[0], phw[1], phw[2], phw[3]);
+                hwp[1] = make_uint4(phw[4], phw[5], phw[6], phw[7]);
+            }
+        }
+        if (valid) p.dwp[(int64_t)row * p.n_tiles + it.nt] = dot;
+    } else if constexpr (KIND == kDX) {
+        const int row = it.row0 + r;
+        const bool valid = row < it.row_end;
+        const int c_base = it.nt * kBN;
+        const int ncols = min(kBN, p.n_out - c_base);
+#pragma unroll 1
+        for (int c0 = 0; c0 < kBN; c0 += 16) {
+            uint32_t acc[16];
+            tmem_ld16(tbase + c0, acc);
+            tmem_ld_wait();
+            if (valid && c0 < ncols) store_f32x16(p.out0 + (int64_t)row * p.ld_out + c_base + c0, acc);
+        }
+    } else {  // kDW
+        const int m = it.mt * kPairRows + r;
+        const bool valid = m < p.m_total;
+        const bool empty = it.num_kb == 0;
+        const int64_t obase = ((int64_t)it.e * p.m_total + m) * p.ld_out;
+#pragma unroll 1
+        for (int c0 = 0; c0 < kBN; c0 += 16) {
+            uint32_t acc[16];
+            tmem_ld16(tbase + c0, acc);
+            tmem_ld_wait();
+            if (!valid) continue;
+            float* dst;
+            int col;
+            if (p.split_b) {
+                col = it.nt * 128 + (c0 & 127);
+                dst = (c0 < 128 ? p.out0 : p.out1) + obase + col;
+            } else {
+                col = it.nt * kBN + c0;
+                dst = p.out0 + obase + col;
+            }
+            if (col >= p.n_out) continue;
+            if (col + 16 <= p.n_out) {
+                if (empty)
+                    store_zero_f32x16(dst);
+                else
+                    store_f32x16(dst, acc);
+            } else {
+                // a row that ends inside this 16-column chunk (n_out % 16 == 8)
+                const int n = p.n_out - col;
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    if (i < n) dst[i] = empty ? 0.0f : __uint_as_float(acc[i]);
+            }
+        }
+    }
+}
+
+template <int KIND>
+__global__ void __launch_bounds__(kThreads, 1)
+    pair_bwd_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_a2,
+                    const __grid_constant__ CUtensorMap tm_b0, const __grid_constant__ CUtensorMap tm_b1, Params p)
+{
+    constexpr bool kAMN = KIND == kDW;                   // A read MN-major
+    constexpr bool kBK_MAJOR = KIND == kDH || KIND == kDX;  // B read K-major
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    Ctrl& c = *reinterpret_cast<Ctrl*>(smem + (size_t)kPairStages * kPairStageBytes);
+
+    const int warp = threadIdx.x / 32;
+    const int lane = threadIdx.x % 32;
+    const uint64_t limit = g_wait_limit_ns;
+    const int E = p.E;
+    const uint32_t rank = cluster_ctarank();  // 0: issues the MMAs
+    const bool leader = rank == 0;
+    const int64_t pair = cluster_id_x();
+    const int64_t npairs = num_clusters_x();
+
+    if (threadIdx.x == 32) {
+        for (int s = 0; s < kPairStages; ++s) {
+            mbar_init(&c.full[s], 1);
+            mbar_init(&c.empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&c.acc_full[b], 1);
+            mbar_init(&c.acc_empty[b], 2 * kEpiWarps);
+        }
+        mbar_init(&c.done, 1);
+        c.abort_flag = 0;
+        fence_mbar_init();
+        tma_prefetch_map(&tm_a);
+        tma_prefetch_map(&tm_b0);
+        if (KIND == kDX) tma_prefetch_map(&tm_a2);
+        if (KIND == kGU || KIND == kDX || KIND == kDW) tma_prefetch_map(&tm_b1);
+    }
+    if (warp == 1) {
+        __syncwarp();
+        tmem_alloc_pair(&c.tmem_slot, kTmemCols);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before_sync();
+    cluster_sync();
+    tc_fence_after_sync();
+    const uint32_t tmem = c.tmem_slot;
+    pdl_trigger();
+    pdl_wait();
+    gemm::build_tile_list<kPairRows>(p.offsets, E, p.M, c.off, c.tp, &c.total_mtiles, &c.bad, true);
+    __syncthreads();
+    int64_t total_work = 0;
+    if (!c.bad) total_work = KIND == kDW ? (int64_t)E * p.m_tiles * p.n_tiles : (int64_t)c.total_mtiles * p.n_tiles;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ------------------------------------------------ TMA producer (both CTAs)
+            int s = 0;
+            uint32_t ph = 0;
+            int64_t issued = 0;
+            for (int64_t w = pair; w < total_work && !c.abort_flag; w += npairs) {
+                const Item it = decode_item<KIND>(w, p, c);
+                bool ok = true;
+                for (int kb = 0; kb < it.num_kb; ++kb) {
+                    if (!mbar_wait(&c.empty[s], ph ^ 1u, limit)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t* sa = smem + (size_t)s * kPairStageBytes;
+                    uint8_t* sb = sa + kABytes;
+                    if (leader) mbar_arrive_expect_tx(&c.full[s], (uint32_t)(2 * kPairStageBytes));
+                    const uint32_t bar = mapa_shared(&c.full[s], 0);
+                    if constexpr (KIND == kGU) {
+                        tma_load_2d_pair(sa, &tm_a, bar, kb * kBK, it.row0 + (int)rank * kBM);
+                        tma_load_3d_pair(sb, leader ? &tm_b0 : &tm_b1, bar, 0, it.e * p.b_rows + kb * kBK, it.nt * 2);
+                    } else if constexpr (KIND == kDH) {
+                        tma_load_2d_pair(sa, &tm_a, bar, kb * kBK, it.row0 + (int)rank * kBM);
+                        tma_load_2d_pair(sb, &tm_b0, bar, kb * kBK, it.e * p.b_rows + it.nt * kBN + (int)rank * kBM);
+                    } else if constexpr (KIND == kDX) {
+                        const bool second = kb >= p.k_split;
+                        const int kc = (second ? kb - p.k_split : kb) * kBK;
+                        tma_load_2d_pair(sa, second ? &tm_a2 : &tm_a, bar, kc, it.row0 + (int)rank * kBM);
+                        tma_load_2d_pair(sb, second ? &tm_b1 : &tm_b0, bar, kc,
+                                         it.e * p.b_rows + it.nt * kBN + (int)rank * kBM);
+                    } else {
+                        const int kr = it.kstart + kb * kBK;
+                        tma_load_3d_pair(sa, &tm_a, bar, 0, kr, (it.mt * kPairRows + (int)rank * kBM) / 64);
+                        if (p.split_b)
+                            tma_load_3d_pair(sb, leader ? &tm_b0 : &tm_b1, bar, 0, kr, it.nt * 2);
+                        else
+                            tma_load_3d_pair(sb, &tm_b0, bar, 0, kr, it.nt * (kBN / 64) + (int)rank * 2);
+                    }
+                    ++issued;
+                    if (++s == kPairStages) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
+                }
+                if (!ok) {
+                    c.abort_flag = 1;
+                    break;
+                }
+            }
+            for (int qq = 0; qq < kPairStages; ++qq) {
+                const int64_t cnt = issued / kPairStages + (qq < issued % kPairStages ? 1 : 0);
+                if (cnt > 0)
+                    mbar_wait(leader ? &c.full[qq] : &c.empty[qq], (uint32_t)(cnt - 1) & 1u, drain_limit(limit));
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        if (lane == 0 && leader) {
+            // ------------------------------------------------ MMA issuer (even CTA)
+            constexpr uint32_t idesc = idesc_bf16_f32(kPairRows, kBN, kAMN, !kBK_MAJOR);
+            int s = 0;
+            uint32_t ph = 0;
+            int acc = 0;
+            uint32_t acc_ph = 0;
+            for (int64_t w = pair; w < total_work && !c.abort_flag; w += npairs) {
+                const Item it = decode_item<KIND>(w, p, c);
+                if (!mbar_wait(&c.acc_empty[acc], acc_ph ^ 1u, limit)) {
+                    c.abort_flag = 1;
+                    break;
+                }
+                tc_fence_after_sync();
+                const uint32_t d_tmem = tmem + (uint32_t)(acc * kBN);
+                bool ok = true;
+                for (int kb = 0; kb < it.num_kb; ++kb) {
+                    if (!mbar_wait(&c.full[s], ph, limit)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after_sync();
+                    const uint32_t a_base = smem_u32(smem + (size_t)s * kPairStageBytes);
+                    const uint32_t b_base = a_base + kABytes;
+#pragma unroll
+                    for (int kk = 0; kk < kBK / 16; ++kk) {
+                        const uint64_t adesc = kAMN ? smem_desc_sw128(a_base + kk * 2048, kChunkBytes, 1024)
+                                                    : smem_desc_sw128(a_base + kk * 32, 16, 1024);
+                        const uint64_t bdesc = kBK_MAJOR ? smem_desc_sw128(b_base + kk * 32, 16, 1024)
+                                                         : smem_desc_sw128(b_base + kk * 2048, kChunkBytes, 1024);
+                        mma_bf16_ss_pair(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
+                    }
+                    mma_commit_pair_multicast(&c.empty[s], 0x3);
+                    if (++s == kPairStages) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
+                }
+                if (!ok) {
+                    c.abort_flag = 1;
+                    break;
+                }
+                // an empty group issues no MMA: the commit still arrives (once
+                // the earlier MMAs are done) and the epilogue writes zeros
+                mma_commit_pair_multicast(&c.acc_full[acc], 0x3);
+                if (++acc == 2) {
+                    acc = 0;
+                    acc_ph ^= 1u;
+                }
+            }
+            mma_commit_pair(&c.done);
+            mbar_wait(&c.done, 0, drain_limit(limit));
+        }
+        __syncwarp();
+    } else {
+        // ---------------------------------------------------- epilogue (both CTAs)
+        const int q = warp & 3;
+        int acc = 0;
+        uint32_t acc_ph = 0;
+        for (int64_t w = pair; w < total_work; w += npairs) {
+            const Item it = decode_item<KIND>(w, p, c);
+            bool ready = true;
+            if (lane == 0) ready = mbar_wait(&c.acc_full[acc], acc_ph, limit);
+            ready = __shfl_sync(0xffffffffu, ready ? 1 : 0, 0) != 0;
+            if (!ready) {
+                c.abort_flag = 1;
+                break;
+            }
+            tc_fence_after_sync();
+            const uint32_t tbase = tmem + (uint32_t)(acc * kBN) + ((uint32_t)(q * 32) << 16);
+            epilogue<KIND>(p, it, tbase, rank, q, lane);
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(mapa_shared(&c.acc_empty[acc], 0));
+            if (++acc == 2) {
+                acc = 0;
+                acc_ph ^= 1u;
+            }
+        }
+        __syncwarp();
+    }
+
+    tc_fence_before_sync();
+    cluster_sync();
+    if (warp == 1) {
+        tc_fence_after_sync();
+        tmem_dealloc_pair(tmem, kTmemCols);
+    }
+}
+
+}  // namespace bwd
+}  // namespace moe

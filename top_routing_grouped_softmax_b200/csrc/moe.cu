@@ -18,6 +18,8 @@
 #include "grouped_gemm.cuh"
 #include "grouped_gemm_pair.cuh"
 #include "combine.cuh"
+#include "grouped_gemm_bwd.cuh"
+#include "backward.cuh"
 
 namespace {
 
@@ -193,6 +195,10 @@ int setup_device(DeviceState** out)
             e = e ? e : cudaFuncSetAttribute(moe::gemm::grouped_gemm_kernel<moe::gemm::kWeighted, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
             e = e ? e : cudaFuncSetAttribute(moe::gemm::grouped_gemm_pair_kernel<moe::gemm::kSwiGLU>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
             e = e ? e : cudaFuncSetAttribute(moe::gemm::grouped_gemm_pair_kernel<moe::gemm::kWeighted>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
+            e = e ? e : cudaFuncSetAttribute(moe::bwd::pair_bwd_kernel<moe::bwd::kGU>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
+            e = e ? e : cudaFuncSetAttribute(moe::bwd::pair_bwd_kernel<moe::bwd::kDH>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
+            e = e ? e : cudaFuncSetAttribute(moe::bwd::pair_bwd_kernel<moe::bwd::kDX>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
+            e = e ? e : cudaFuncSetAttribute(moe::bwd::pair_bwd_kernel<moe::bwd::kDW>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
             if (e == cudaSuccess) {
                 // CTA pairs that can be resident at once (clusters need two
                 // SMs of one GPC, so this can be below sm_count / 2)
@@ -342,7 +348,7 @@ int launch_route(const CUtensorMap& tx, const CUtensorMap& tw, const CUtensorMap
 
 int run_route(const DeviceState& st, const moe_bf16* x, const moe_bf16* w_router, const float* bias, int64_t T,
               int64_t d, int64_t E, int64_t k, int32_t* ids, float* wts, int32_t* chunk_counts, bool renorm,
-              cudaStream_t s, float* probs_t = nullptr)
+              cudaStream_t s, float* probs_t = nullptr, float* probs_tm = nullptr)
 {
     if (T == 0) return MOE_OK;
     CUtensorMap tx, tw;
@@ -389,7 +395,10 @@ int run_route(const DeviceState& st, const moe_bf16* x, const moe_bf16* w_router
     p.split = (E <= 256 && d >= 2 * moe::route::kBK && tiles <= pairs) ? 2 : 1;
     p.passes = (p.split == 1 && E > 256) ? 2 : 1;
     p.renorm = renorm ? 1 : 0;
-    p.probs_t = probs_t;
+    // every expert's probability, [E][T] (token rounding) or [T][E] (backward)
+    p.probs = probs_t ? probs_t : probs_tm;
+    p.probs_tstride = probs_t ? 1 : E;
+    p.probs_estride = probs_t ? T : 1;
     // top-k list length: the power of two >= k for lane groups (k <= 8), or
     // the whole-warp rounds (k > 8)
     const unsigned ut = (unsigned)tiles;
@@ -421,13 +430,13 @@ int run_permute(const moe_bf16* x, const int32_t* ids, const float* wts, int64_t
         return MOE_ERR_CUDA;
     if (launch(chunk_scan_kernel, dim3((unsigned)E), dim3(kThreads), 0, s, 1u, chunk_em, nch, counts))
         return MOE_ERR_CUDA;
-    if (launch(rank_kernel, dim3(nch), dim3(kThreads), 0, s, 1u, cids, cw, T, ik, iE,
+    if (launch(rank_kernel<false>, dim3(nch), dim3(kThreads), 0, s, 1u, cids, cw, T, ik, iE,
                static_cast<const int32_t*>(chunk_em), nch, static_cast<const int32_t*>(counts), offsets, perm, inv,
                w_perm))
         return MOE_ERR_CUDA;
     if (x_perm) {
         if (launch(gather_kernel, dim3((unsigned)((T + kWarps - 1) / kWarps)), dim3(kThreads), 0, s, 1u,
-                   reinterpret_cast<const uint4*>(x), static_cast<const int32_t*>(inv), T, ik, (int)(d / 8),
+                   reinterpret_cast<const uint4*>(x), static_cast<const int32_t*>(inv), T, ik, (int)(d / 8), T * k,
                    reinterpret_cast<uint4*>(x_perm)))
             return MOE_ERR_CUDA;
     }
@@ -755,6 +764,320 @@ int forward_rounded_impl(const moe_bf16* x, const moe_bf16* w_router, const floa
     return rec(5);
 }
 
+// ------------------------------------------------------------ backward
+// Workspace of moe_backward.  Grouped rows are padded: every expert group
+// starts on a 64-row boundary, so the grouped buffers hold up to
+// T*k + 63*E rows.
+struct BLayout {
+    size_t ids, wts, probs, counts, offsets, chunk, perm, inv, w_perm, x_perm, dout_perm, g, u, hw, dwp, dx_perm,
+        dlogit, db_part, dx_router, total;
+    int64_t rows;    // padded row capacity
+    int64_t e_pad;   // E rounded up to 64 (row length of dlogit)
+    int n_tiles_f;   // 256-column tiles over f (the down-projection gradient's partial dots)
+};
+
+BLayout plan_backward(int64_t T, int64_t d, int64_t E, int64_t k, int64_t f)
+{
+    const size_t M = (size_t)(T * k);
+    BLayout L{};
+    L.rows = (int64_t)M + 63 * E;
+    L.e_pad = (E + 63) / 64 * 64;
+    L.n_tiles_f = (int)((f + moe::gemm::kBN - 1) / moe::gemm::kBN);
+    const size_t R = (size_t)L.rows;
+    size_t o = 0;
+    L.ids = o;       o += align256(M * 4);
+    L.wts = o;       o += align256(M * 4);
+    L.probs = o;     o += align256((size_t)T * (size_t)E * 4);
+    L.counts = o;    o += align256((size_t)E * 4);
+    L.offsets = o;   o += align256((size_t)(E + 1) * 4);
+    L.chunk = o;     o += permute_ws_bytes(T, E);
+    L.perm = o;      o += align256(R * 4);
+    L.inv = o;       o += align256(M * 4);
+    L.w_perm = o;    o += align256(R * 4);
+    L.x_perm = o;    o += align256(R * (size_t)d * 2);
+    L.dout_perm = o; o += align256(R * (size_t)d * 2);
+    L.g = o;         o += align256(R * (size_t)f * 2);   // g, then dg in place
+    L.u = o;         o += align256(R * (size_t)f * 2);   // u, then du in place
+    L.hw = o;        o += align256(R * (size_t)f * 2);
+    L.dwp = o;       o += align256(R * (size_t)L.n_tiles_f * 4);
+    L.dx_perm = o;   o += align256(R * (size_t)d * 4);
+    L.dlogit = o;    o += align256((size_t)T * (size_t)L.e_pad * 2);
+    L.db_part = o;   o += align256((size_t)((T + moe::bwd::kRowWarps - 1) / moe::bwd::kRowWarps) * (size_t)E * 4);
+    L.dx_router = o; o += align256((size_t)T * (size_t)d * 4);
+    L.total = o;
+    return L;
+}
+
+template <int KIND>
+int launch_pair_bwd(const DeviceState& st, int64_t work, const CUtensorMap& ta, const CUtensorMap& ta2,
+                    const CUtensorMap& tb0, const CUtensorMap& tb1, const moe::bwd::Params& p, cudaStream_t s)
+{
+    int64_t pairs = st.max_pairs > 0 ? st.max_pairs : st.sm_count / 2;
+    if (work < pairs) pairs = work;
+    if (pairs < 1) pairs = 1;
+    return launch(moe::bwd::pair_bwd_kernel<KIND>, dim3((unsigned)(2 * pairs)), dim3(moe::gemm::kThreads),
+                  moe::bwd::smem_bytes(), s, 2u, ta, ta2, tb0, tb1, p);
+}
+
+moe::bwd::Params bwd_params()
+{
+    moe::bwd::Params p;
+    std::memset(&p, 0, sizeof(p));
+    return p;
+}
+
+int backward_impl(const moe_bf16* x, const moe_bf16* w_router, const float* bias, const moe_bf16* w_gate,
+                  const moe_bf16* w_up, const moe_bf16* w_down, const float* dout, int64_t T, int64_t d, int64_t E,
+                  int64_t k, int64_t f, float* dx, float* dw_router, float* dbias, float* dw_gate, float* dw_up,
+                  float* dw_down, void* ws, size_t ws_bytes, cudaStream_t s, unsigned flags)
+{
+    int rc = check_common(T, d, E, k);
+    if (rc) return rc;
+    if ((rc = check_f(f))) return rc;
+    if (flags & ~(unsigned)MOE_FLAG_RENORMALIZE) return MOE_ERR_INVALID_ARG;
+    if (!w_router || !w_gate || !w_up || !w_down || !dw_router || !dw_gate || !dw_up || !dw_down)
+        return MOE_ERR_INVALID_ARG;
+    if (T > 0 && (!x || !dout || !dx)) return MOE_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(w_router, 16) || !aligned(w_gate, 16) || !aligned(w_up, 16) ||
+        !aligned(w_down, 16) || !aligned(dout, 16) || !aligned(dx, 16) || !aligned(dw_router, 16) ||
+        !aligned(dw_gate, 16) || !aligned(dw_up, 16) || !aligned(dw_down, 16) || !aligned(bias, 4) ||
+        !aligned(dbias, 4))
+        return MOE_ERR_INVALID_ARG;
+    const BLayout L = plan_backward(T, d, E, k, f);
+    if (L.rows >= (int64_t(1) << 31)) return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (T > 0 && (!ws || !aligned(ws, 256))) return MOE_ERR_INVALID_ARG;
+    if (T > 0 && ws_bytes < L.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
+    DeviceState* st = nullptr;
+    if ((rc = setup_device(&st))) return rc;
+    if (T == 0) {
+        // no tokens: every weight gradient is zero
+        const size_t we = (size_t)E * (size_t)d * (size_t)f * 4;
+        if (cudaMemsetAsync(dw_gate, 0, we, s) != cudaSuccess || cudaMemsetAsync(dw_up, 0, we, s) != cudaSuccess ||
+            cudaMemsetAsync(dw_down, 0, we, s) != cudaSuccess ||
+            cudaMemsetAsync(dw_router, 0, (size_t)d * (size_t)E * 4, s) != cudaSuccess ||
+            (dbias && cudaMemsetAsync(dbias, 0, (size_t)E * 4, s) != cudaSuccess))
+            return MOE_ERR_CUDA;
+        return MOE_OK;
+    }
+    using namespace moe::bwd;
+    uint8_t* w = static_cast<uint8_t*>(ws);
+    auto at = [&](size_t off) { return static_cast<void*>(w + off); };
+    int32_t* ids = static_cast<int32_t*>(at(L.ids));
+    float* wts = static_cast<float*>(at(L.wts));
+    float* probs = static_cast<float*>(at(L.probs));
+    int32_t* counts = static_cast<int32_t*>(at(L.counts));
+    int32_t* offsets = static_cast<int32_t*>(at(L.offsets));
+    int32_t* chunk = static_cast<int32_t*>(at(L.chunk));
+    int32_t* perm = static_cast<int32_t*>(at(L.perm));
+    int32_t* inv = static_cast<int32_t*>(at(L.inv));
+    float* w_perm = static_cast<float*>(at(L.w_perm));
+    moe_bf16* x_perm = static_cast<moe_bf16*>(at(L.x_perm));
+    moe_bf16* dout_perm = static_cast<moe_bf16*>(at(L.dout_perm));
+    moe_bf16* g = static_cast<moe_bf16*>(at(L.g));
+    moe_bf16* u = static_cast<moe_bf16*>(at(L.u));
+    moe_bf16* hw = static_cast<moe_bf16*>(at(L.hw));
+    float* dwp = static_cast<float*>(at(L.dwp));
+    float* dx_perm = static_cast<float*>(at(L.dx_perm));
+    moe_bf16* dlogit = static_cast<moe_bf16*>(at(L.dlogit));
+    float* db_part = static_cast<float*>(at(L.db_part));
+    float* dx_router = static_cast<float*>(at(L.dx_router));
+    const int64_t R = L.rows;
+    const int iE = (int)E, ik = (int)k;
+    const bool renorm = (flags & MOE_FLAG_RENORMALIZE) != 0;
+
+    // 1. routing again (ids, weights, every probability [T][E], chunk histograms)
+    if ((rc = run_route(*st, x, w_router, bias, T, d, E, k, ids, wts, chunk, renorm, s, nullptr, probs))) return rc;
+    // 2. grouping with 64-row aligned groups, x_perm, dout_perm, zero padding
+    {
+        using namespace moe::permute;
+        const int nch = (int)token_chunks(T);
+        if (launch(chunk_scan_kernel, dim3((unsigned)E), dim3(moe::permute::kThreads), 0, s, 1u, chunk, nch, counts))
+            return MOE_ERR_CUDA;
+        if (launch(rank_kernel<true>, dim3(nch), dim3(moe::permute::kThreads), 0, s, 1u,
+                   static_cast<const int32_t*>(ids), static_cast<const float*>(wts), T, ik, iE,
+                   static_cast<const int32_t*>(chunk), nch, static_cast<const int32_t*>(counts), offsets, perm, inv,
+                   w_perm))
+            return MOE_ERR_CUDA;
+        if (launch(gather_kernel, dim3((unsigned)((T + moe::permute::kWarps - 1) / moe::permute::kWarps)),
+                   dim3(moe::permute::kThreads), 0, s, 1u, reinterpret_cast<const uint4*>(x),
+                   static_cast<const int32_t*>(inv), T, ik, (int)(d / 8), R, reinterpret_cast<uint4*>(x_perm)))
+            return MOE_ERR_CUDA;
+    }
+    if (launch(gather_dout_kernel, dim3((unsigned)((T + kRowWarps - 1) / kRowWarps)), dim3(kRowThreads), 0, s, 1u,
+               reinterpret_cast<const float4*>(dout), static_cast<const int32_t*>(inv), T, ik, (int)(d / 8), R,
+               reinterpret_cast<uint4*>(dout_perm)))
+        return MOE_ERR_CUDA;
+    if (launch(zero_pad_kernel, dim3((unsigned)E), dim3(kRowThreads), 0, s, 1u, static_cast<const int32_t*>(offsets),
+               static_cast<const int32_t*>(counts), (int)(d / 8), reinterpret_cast<uint4*>(x_perm),
+               reinterpret_cast<uint4*>(dout_perm), w_perm))
+        return MOE_ERR_CUDA;
+
+    using moe::gemm::kBN;
+    using moe::gemm::kBM;
+    using moe::gemm::kPairRows;
+    const int64_t max_mtiles = (R + kPairRows - 1) / kPairRows + E;
+    // 3. recompute g, u = x_perm . [W_gate | W_up]
+    {
+        CUtensorMap ta, tg3, tu3;
+        rc = make_map(&ta, x_perm, (uint64_t)d, (uint64_t)R, 64, kBM);
+        rc = rc ? rc : make_weight_chunk_map(&tg3, w_gate, (uint64_t)f, (uint64_t)(E * d));
+        rc = rc ? rc : make_weight_chunk_map(&tu3, w_up, (uint64_t)f, (uint64_t)(E * d));
+        if (rc) return rc;
+        Params p = bwd_params();
+        p.offsets = offsets;
+        p.out_g = reinterpret_cast<__nv_bfloat16*>(g);
+        p.out_u = reinterpret_cast<__nv_bfloat16*>(u);
+        p.ld_f = f;
+        p.E = iE;
+        p.M = (int)R;
+        p.K = (int)d;
+        p.n_out = (int)f;
+        p.n_tiles = (int)((f + 127) / 128);
+        p.b_rows = (int)d;
+        if (launch_pair_bwd<kGU>(*st, max_mtiles * p.n_tiles, ta, ta, tg3, tu3, p, s)) return MOE_ERR_CUDA;
+    }
+    // 4. dh = w . dout_perm . W_down^T and the SwiGLU derivative: dg, du (in place of g, u), w h, partial dots
+    {
+        CUtensorMap ta, tb;
+        rc = make_map(&ta, dout_perm, (uint64_t)d, (uint64_t)R, 64, kBM);
+        rc = rc ? rc : make_map(&tb, w_down, (uint64_t)d, (uint64_t)(E * f), 64, kBM);
+        if (rc) return rc;
+        Params p = bwd_params();
+        p.offsets = offsets;
+        p.w_perm = w_perm;
+        p.g = reinterpret_cast<const __nv_bfloat16*>(g);
+        p.u = reinterpret_cast<const __nv_bfloat16*>(u);
+        p.out_g = reinterpret_cast<__nv_bfloat16*>(g);
+        p.out_u = reinterpret_cast<__nv_bfloat16*>(u);
+        p.out_hw = reinterpret_cast<__nv_bfloat16*>(hw);
+        p.dwp = dwp;
+        p.ld_f = f;
+        p.E = iE;
+        p.M = (int)R;
+        p.K = (int)d;
+        p.n_out = (int)f;
+        p.n_tiles = L.n_tiles_f;
+        p.b_rows = (int)f;
+        if (launch_pair_bwd<kDH>(*st, max_mtiles * p.n_tiles, ta, ta, tb, tb, p, s)) return MOE_ERR_CUDA;
+    }
+    // 5. dx_perm = dg . W_gate^T + du . W_up^T (fp32)
+    {
+        CUtensorMap ta, ta2, tb0, tb1;
+        rc = make_map(&ta, g, (uint64_t)f, (uint64_t)R, 64, kBM);
+        rc = rc ? rc : make_map(&ta2, u, (uint64_t)f, (uint64_t)R, 64, kBM);
+        rc = rc ? rc : make_map(&tb0, w_gate, (uint64_t)f, (uint64_t)(E * d), 64, kBM);
+        rc = rc ? rc : make_map(&tb1, w_up, (uint64_t)f, (uint64_t)(E * d), 64, kBM);
+        if (rc) return rc;
+        Params p = bwd_params();
+        p.offsets = offsets;
+        p.out0 = dx_perm;
+        p.ld_out = d;
+        p.E = iE;
+        p.M = (int)R;
+        p.K = (int)(2 * f);
+        p.k_split = (int)(f / 64);
+        p.n_out = (int)d;
+        p.n_tiles = (int)((d + kBN - 1) / kBN);
+        p.b_rows = (int)d;
+        if (launch_pair_bwd<kDX>(*st, max_mtiles * p.n_tiles, ta, ta2, tb0, tb1, p, s)) return MOE_ERR_CUDA;
+    }
+    // 6. dW_gate[e], dW_up[e] = x_perm_e^T . dg_e, x_perm_e^T . du_e
+    {
+        CUtensorMap ta, tb0, tb1;
+        rc = make_weight_chunk_map(&ta, x_perm, (uint64_t)d, (uint64_t)R);
+        rc = rc ? rc : make_weight_chunk_map(&tb0, g, (uint64_t)f, (uint64_t)R);
+        rc = rc ? rc : make_weight_chunk_map(&tb1, u, (uint64_t)f, (uint64_t)R);
+        if (rc) return rc;
+        Params p = bwd_params();
+        p.offsets = offsets;
+        p.out0 = dw_gate;
+        p.out1 = dw_up;
+        p.ld_out = f;
+        p.E = iE;
+        p.M = (int)R;
+        p.n_out = (int)f;
+        p.n_tiles = (int)((f + 127) / 128);
+        p.m_total = (int)d;
+        p.m_tiles = (int)((d + kPairRows - 1) / kPairRows);
+        p.split_b = 1;
+        if (launch_pair_bwd<kDW>(*st, E * p.m_tiles * p.n_tiles, ta, ta, tb0, tb1, p, s)) return MOE_ERR_CUDA;
+    }
+    // 7. dW_down[e] = (w h)_e^T . dout_perm_e
+    {
+        CUtensorMap ta, tb;
+        rc = make_weight_chunk_map(&ta, hw, (uint64_t)f, (uint64_t)R);
+        rc = rc ? rc : make_weight_chunk_map(&tb, dout_perm, (uint64_t)d, (uint64_t)R);
+        if (rc) return rc;
+        Params p = bwd_params();
+        p.offsets = offsets;
+        p.out0 = dw_down;
+        p.ld_out = d;
+        p.E = iE;
+        p.M = (int)R;
+        p.n_out = (int)d;
+        p.n_tiles = (int)((d + kBN - 1) / kBN);
+        p.m_total = (int)f;
+        p.m_tiles = (int)((f + kPairRows - 1) / kPairRows);
+        p.split_b = 0;
+        if (launch_pair_bwd<kDW>(*st, E * p.m_tiles * p.n_tiles, ta, ta, tb, tb, p, s)) return MOE_ERR_CUDA;
+    }
+    // 8. router: dlogit (bf16 [T][E_pad]) and the bias gradient
+    const unsigned nblk = (unsigned)((T + kRowWarps - 1) / kRowWarps);
+    if (launch(route_bwd_kernel, dim3(nblk), dim3(kRowThreads), 0, s, 1u, static_cast<const float*>(probs),
+               static_cast<const int32_t*>(ids), static_cast<const float*>(wts), static_cast<const int32_t*>(inv),
+               static_cast<const float*>(dwp), L.n_tiles_f, R, T, iE, ik, renorm ? 1 : 0,
+               reinterpret_cast<__nv_bfloat16*>(dlogit), dbias ? db_part : nullptr, (int)L.e_pad))
+        return MOE_ERR_CUDA;
+    if (dbias && launch(colsum_kernel, dim3((unsigned)((E + kRowThreads - 1) / kRowThreads)), dim3(kRowThreads), 0, s,
+                        1u, static_cast<const float*>(db_part), (int)nblk, iE, dbias))
+        return MOE_ERR_CUDA;
+    // 9. dW_router = x^T . dlogit (one group of T rows)
+    {
+        CUtensorMap ta, tb;
+        rc = make_weight_chunk_map(&ta, x, (uint64_t)d, (uint64_t)T);
+        rc = rc ? rc : make_weight_chunk_map(&tb, dlogit, (uint64_t)L.e_pad, (uint64_t)T);
+        if (rc) return rc;
+        Params p = bwd_params();
+        p.offsets = nullptr;
+        p.out0 = dw_router;
+        p.ld_out = E;
+        p.E = 1;
+        p.M = (int)T;
+        p.n_out = iE;
+        p.n_tiles = (int)((E + kBN - 1) / kBN);
+        p.m_total = (int)d;
+        p.m_tiles = (int)((d + kPairRows - 1) / kPairRows);
+        p.split_b = 0;
+        if (launch_pair_bwd<kDW>(*st, p.m_tiles * p.n_tiles, ta, ta, tb, tb, p, s)) return MOE_ERR_CUDA;
+    }
+    // 10. dx_router = dlogit . W_router^T (fp32)
+    {
+        CUtensorMap ta, tb;
+        rc = make_map(&ta, dlogit, (uint64_t)L.e_pad, (uint64_t)T, 64, kBM);
+        rc = rc ? rc : make_map(&tb, w_router, (uint64_t)E, (uint64_t)d, 64, kBM);
+        if (rc) return rc;
+        Params p = bwd_params();
+        p.offsets = nullptr;
+        p.out0 = dx_router;
+        p.ld_out = d;
+        p.E = 1;
+        p.M = (int)T;
+        p.K = (int)L.e_pad;
+        p.k_split = (int)(L.e_pad / 64);
+        p.n_out = (int)d;
+        p.n_tiles = (int)((d + kBN - 1) / kBN);
+        p.b_rows = 0;
+        if (launch_pair_bwd<kDX>(*st, ((T + kPairRows - 1) / kPairRows) * p.n_tiles, ta, ta, tb, tb, p, s))
+            return MOE_ERR_CUDA;
+    }
+    // 11. dx = dx_router + sum over slots of dx_perm (fp32)
+    if (launch(combine_dx_kernel, dim3((unsigned)T), dim3(kRowThreads), 0, s, 1u,
+               reinterpret_cast<const float4*>(dx_perm), reinterpret_cast<const float4*>(dx_router),
+               static_cast<const int32_t*>(inv), R, ik, (int)(d / 4), reinterpret_cast<float4*>(dx)))
+        return MOE_ERR_CUDA;
+    return MOE_OK;
+}
+
 // ------------------------------------------- fixed scratch for moe_permute_static
 // Some callers cannot allocate device memory when they run the permutation:
 // for example a plugin inside an inference engine that plans all device
@@ -1020,6 +1343,23 @@ int moe_forward_ex(const moe_bf16* x, const moe_bf16* w_router, const float* bia
 {
     return forward_impl(x, w_router, bias, w_gate, w_up, w_down, T, d, E, k, f, out, topk_ids_out, topk_w_out,
                         workspace, workspace_bytes, stream, events, n_events, flags);
+}
+
+size_t moe_backward_workspace_size(int64_t T, int64_t d, int64_t E, int64_t k, int64_t f)
+{
+    if (check_common(T, d, E, k) || check_f(f)) return 0;
+    const BLayout L = plan_backward(T, d, E, k, f);
+    if (L.rows >= (int64_t(1) << 31)) return 0;
+    return L.total;
+}
+
+int moe_backward(const moe_bf16* x, const moe_bf16* w_router, const float* bias, const moe_bf16* w_gate,
+                 const moe_bf16* w_up, const moe_bf16* w_down, const float* dout, int64_t T, int64_t d, int64_t E,
+                 int64_t k, int64_t f, float* dx, float* dw_router, float* dbias, float* dw_gate, float* dw_up,
+                 float* dw_down, void* workspace, size_t workspace_bytes, cudaStream_t stream, unsigned flags)
+{
+    return backward_impl(x, w_router, bias, w_gate, w_up, w_down, dout, T, d, E, k, f, dx, dw_router, dbias, dw_gate,
+                         dw_up, dw_down, workspace, workspace_bytes, stream, flags);
 }
 
 int moe_get_status(cudaStream_t stream)

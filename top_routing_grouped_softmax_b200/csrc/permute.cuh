@@ -107,9 +107,20 @@ __global__ void __launch_bounds__(kThreads) chunk_scan_kernel(int32_t* __restric
     if (tid == 0) totals[blockIdx.x] = carry;
 }
 
+// Rows a group occupies: its size, or (PAD64) its size rounded up to a
+// multiple of 64, so that every group starts on a 64-row boundary.
+template <bool PAD64>
+__device__ __forceinline__ int group_span(int n)
+{
+    return PAD64 ? (n + 63) & ~63 : n;
+}
+
 // One block per 64-token chunk.  chunk_base_em[e][c] holds the chunk's first
 // position inside group e (relative to the group start); totals[e] the group
-// sizes.  Block 0 also writes offsets[0..E].
+// sizes.  Block 0 also writes offsets[0..E] (the group starts; with PAD64
+// each group's rows are followed by padding up to the next multiple of 64,
+// which this kernel leaves unwritten).
+template <bool PAD64>
 __global__ void __launch_bounds__(kThreads) rank_kernel(const int32_t* __restrict__ ids,
                                                         const float* __restrict__ wts, int64_t T, int k, int E,
                                                         const int32_t* __restrict__ chunk_base_em, int n_tchunks,
@@ -133,7 +144,7 @@ __global__ void __launch_bounds__(kThreads) rank_kernel(const int32_t* __restric
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const int idx = tid * 4 + i;
-            v[i] = idx < E ? s_off[idx] : 0;
+            v[i] = idx < E ? group_span<PAD64>(s_off[idx]) : 0;
             local += v[i];
         }
         int incl = local;
@@ -215,17 +226,18 @@ __global__ void __launch_bounds__(kThreads) rank_kernel(const int32_t* __restric
 // x_perm[inv[t*k + j]] = x[t] for every slot j: one warp per token reads the
 // token's row once (16-byte vectors, eight in flight per lane) and writes it
 // to its k grouped positions, so x is read from HBM once and every write is
-// a whole contiguous row.
+// a whole contiguous row.  rows: the rows x_perm holds (T*k, or more when
+// the groups are padded); a position outside is reported and skipped.
 __global__ void __launch_bounds__(kThreads) gather_kernel(const uint4* __restrict__ x,
                                                           const int32_t* __restrict__ inv, int64_t T, int k,
-                                                          int nvec, uint4* __restrict__ x_perm)
+                                                          int nvec, int64_t rows, uint4* __restrict__ x_perm)
 {
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const int64_t t = (int64_t)blockIdx.x * kWarps + warp;
     pdl_trigger();
     pdl_wait();
     if (t >= T) return;
-    const int64_t n = T * k;
+    const int64_t n = rows;
     int pos = -1;
     if (lane < k) {
         pos = __ldg(inv + t * k + lane);

@@ -71,7 +71,9 @@ struct Params {
     int split;               // CTAs per tile: 1, or 2 (cluster of two, split K)
     int passes;              // row passes of the exchange buffer (1, or 2 when split == 1 and E > 256)
     int renorm;              // 1: divide each token's k weights by their sum
-    float* probs_t;          // [E][T]: every expert's probability (token rounding), or nullptr
+    float* probs;            // every expert's probability, or nullptr: p[t][e] at t * probs_tstride + e * probs_estride
+    int64_t probs_tstride;   // [E][T] for token rounding (1, T); [T][E] for the backward (E, 1)
+    int64_t probs_estride;
 };
 
 __host__ __device__ inline int stage_bytes(int n_chunks) { return kABytes + n_chunks * kChunkBytes; }
@@ -315,7 +317,7 @@ __device__ __forceinline__ void topk_rows(const Params& p, const float* buf, con
             float l = col[0];
             for (int s = 1; s < S; ++s) l += col[(size_t)s * E * pitch];
             return l + s_bias[c];
-        }, my_id, my_w, (p.probs_t && ok && t < p.T) ? p.probs_t + t : nullptr, (int64_t)p.T);
+        }, my_id, my_w, (p.probs && ok && t < p.T) ? p.probs + t * p.probs_tstride : nullptr, p.probs_estride);
         if (ok && t < p.T && j < p.k) {
             p.ids[t * p.k + j] = my_id;
             p.wts[t * p.k + j] = my_w;
@@ -517,7 +519,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     float l = col[0];
                     for (int s = 1; s < S; ++s) l += col[(size_t)s * E * pitch];
                     return l + s_bias[c];
-                }, my_id, my_w, (p.probs_t && ok) ? p.probs_t + t : nullptr, (int64_t)p.T);
+                }, my_id, my_w, (p.probs && ok) ? p.probs + t * p.probs_tstride : nullptr, p.probs_estride);
                 if (ok && lane < p.k) {
                     p.ids[t * p.k + lane] = my_id;
                     p.wts[t * p.k + lane] = my_w;

@@ -160,6 +160,15 @@ def make_shared_weights(cfg: MoEConfig, n_shared: int, f_shared: int | None = No
     return {"W_gate_s": W_gate_s, "W_up_s": W_up_s, "W_down_s": W_down_s}
 
 
+def make_dout(T: int, d: int, seed: int) -> torch.Tensor:
+    """The output gradient for a backward check: fp32 [T, d], N(0, 1), drawn
+    from its own generator (seed + 200000) so the forward inputs of the
+    same seed are unchanged."""
+    gen = torch.Generator(device="cpu")
+    gen.manual_seed(seed + 200000)
+    return torch.randn(T, d, generator=gen, dtype=torch.float32)
+
+
 def sample_tokens(T: int, n: int, seed: int, must_include=()) -> np.ndarray:
     """A seeded, sorted, duplicate-free sample of n token indices in [0, T).
 
@@ -180,5 +189,5 @@ def sample_tokens(T: int, n: int, seed: int, must_include=()) -> np.ndarray:
 
 __all__ = [
     "MoEConfig", "MoEInputs", "CONFIGS", "make_inputs", "bf16_bits", "bits_to_bf16",
-    "zipf_bias", "sample_tokens", "make_shared_weights",
+    "zipf_bias", "sample_tokens", "make_shared_weights", "make_dout",
 ]
