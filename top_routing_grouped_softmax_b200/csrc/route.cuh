@@ -24,11 +24,12 @@
 // Softmax and top-k.  For k <= 8, a group of L lanes of one warp takes a
 // token (L = 8 when a CTA owns 128 rows, 16 when it owns 64, so all 32 warps
 // are busy).  Lane j of the group visits experts j, j + L, j + 2L, ... in
-// ascending order, keeps the maximum and a sorted top-KMAX list of
-// (logit, expert) in registers, and later sums exp(l - max) over the same
-// experts; the group's maximum and sum are butterfly reductions in a fixed
-// order, and log2(L) butterfly rounds of a bitonic merge give every lane of
-// the group the token's sorted top-KMAX.  For k > 8, a whole warp takes a
+// ascending order: it adds the split-K partials and the bias once, writes
+// the logit back to shared memory, and keeps its maximum and its best
+// (logit, expert); the group's maximum and the sum of exp(l - max) are
+// butterfly reductions in a fixed order.  k rounds of a butterfly arg-max
+// over the lanes' best candidates then pick the winners in order; the lane
+// that owned a winner marks it taken and rescans its experts.  For k > 8, a whole warp takes a
 // token and picks the winners in k rounds of a butterfly arg-max.  Both
 // rank by the (value, index) order -- larger logit first, equal logits rank
 // the lower expert index first -- on fp32 logits (softmax is monotone).
@@ -189,118 +190,86 @@ __device__ __forceinline__ void warp_topk(int E, int k, bool renorm, int lane, L
     my_w /= sum;
 }
 
-// Insert (x, col) into a list sorted by the (value, index) order, dropping
-// its last entry.  The caller visits its experts in ascending index order,
-// so every entry already in the list has a lower index than col and x
-// ranks before entry m exactly when x > v[m].  The comparisons are
-// independent and every slot takes its new value by selection: it keeps
-// its entry, takes x, or takes the old entry m-1.
-template <int KMAX>
-__device__ __forceinline__ void insert_ascending(float (&v)[KMAX], int (&ix)[KMAX], float x, int col)
-{
-    bool gt[KMAX];
-#pragma unroll
-    for (int m = 0; m < KMAX; ++m) gt[m] = x > v[m];
-#pragma unroll
-    for (int m = KMAX - 1; m > 0; --m) {
-        v[m] = gt[m - 1] ? v[m - 1] : (gt[m] ? x : v[m]);
-        ix[m] = gt[m - 1] ? ix[m - 1] : (gt[m] ? col : ix[m]);
-    }
-    v[0] = gt[0] ? x : v[0];
-    ix[0] = gt[0] ? col : ix[0];
-}
-
-// Merge the sorted list of lane (lane ^ o) into this lane's, keeping the
-// KMAX best: the better of v[m] and the partner's [KMAX-1-m] leaves the KMAX
-// best of both lists as a bitonic sequence, which half-cleaners sort.  Both
-// partners end with the same list (the order is total; only identical
-// (-inf, sentinel) entries can compare equal).
-template <int KMAX>
-__device__ __forceinline__ void merge_partner(float (&v)[KMAX], int (&ix)[KMAX], int o)
-{
-    float ov[KMAX];
-    int oi[KMAX];
-#pragma unroll
-    for (int m = 0; m < KMAX; ++m) {
-        ov[m] = __shfl_xor_sync(0xffffffffu, v[m], o);
-        oi[m] = __shfl_xor_sync(0xffffffffu, ix[m], o);
-    }
-#pragma unroll
-    for (int m = 0; m < KMAX; ++m) {
-        const float bv = ov[KMAX - 1 - m];
-        const int bi = oi[KMAX - 1 - m];
-        if (ranks_before(bv, bi, v[m], ix[m])) {
-            v[m] = bv;
-            ix[m] = bi;
-        }
-    }
-#pragma unroll
-    for (int stride = KMAX / 2; stride > 0; stride >>= 1) {
-#pragma unroll
-        for (int m = 0; m < KMAX; ++m) {
-            if ((m & stride) == 0 && ranks_before(v[m + stride], ix[m + stride], v[m], ix[m])) {
-                const float tv = v[m];
-                const int ti = ix[m];
-                v[m] = v[m + stride];
-                ix[m] = ix[m + stride];
-                v[m + stride] = tv;
-                ix[m + stride] = ti;
-            }
-        }
-    }
-}
-
 // Softmax and top-k of one token by a group of L lanes (lane j of the group
-// = lane % L); `logit(c)` is expert c's logit.  Lane j < k receives slot j.
-template <int L, int KMAX, typename Logit>
-__device__ __forceinline__ void group_topk(int E, int k, bool renorm, int j, Logit logit, int& my_id, float& my_w,
-                                           float* pcol, int64_t pstride)
+// = lane % L).  Lane j owns experts j, j + L, j + 2L, ...  `combine(c)` returns
+// expert c's logit (the sum of the split-K partials plus the bias) and
+// `cell(c)` is a shared-memory slot for it: the first pass writes the
+// combined logits there, tracks the lane's maximum and its best (value,
+// index), and the group's maximum and sum follow by butterfly reductions in
+// a fixed order.  Then k rounds of a butterfly arg-max over the lanes' best
+// candidates pick the winners in (value, index) order; the lane that owned
+// a winner marks it taken (-inf in its slot) and rescans its experts for its
+// next best.  Lane j < k receives slot j.
+template <int L, typename Combine, typename Cell>
+__device__ __forceinline__ void group_topk(int E, int k, bool renorm, int j, Combine combine, Cell cell, int& my_id,
+                                           float& my_w, float* pcol, int64_t pstride)
 {
-    float v[KMAX];
-    int ix[KMAX];
-#pragma unroll
-    for (int m = 0; m < KMAX; ++m) {
-        v[m] = -INFINITY;
-        ix[m] = 0x7fffffff;
-    }
-    float mx = -INFINITY;
+    float mx = -INFINITY, bv = -INFINITY;
+    int bc = 0x7fffffff;
     for (int c = j; c < E; c += L) {
-        const float l = logit(c);
+        const float l = combine(c);
+        cell(c) = l;
         mx = fmaxf(mx, l);
-        insert_ascending<KMAX>(v, ix, l, c);
+        if (l > bv) {  // ascending c: among equal values the lower index stays
+            bv = l;
+            bc = c;
+        }
     }
 #pragma unroll
     for (int o = L / 2; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
     float sum = 0.0f;
-    for (int c = j; c < E; c += L) sum += __expf(logit(c) - mx);
+    for (int c = j; c < E; c += L) sum += __expf(cell(c) - mx);
 #pragma unroll
     for (int o = L / 2; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
     if (pcol)  // every expert's probability, by the same formula as the weights below
-        for (int c = j; c < E; c += L) pcol[c * pstride] = __expf(logit(c) - mx) / sum;
+        for (int c = j; c < E; c += L) pcol[c * pstride] = __expf(cell(c) - mx) / sum;
+    float my_v = -INFINITY;
+    my_id = 0;
+    for (int slot = 0; slot < k; ++slot) {
+        float wv = bv;
+        int wc = bc;
 #pragma unroll
-    for (int o = 1; o < L; o <<= 1) merge_partner<KMAX>(v, ix, o);
-    my_id = ix[0];
-    float w = v[0];
-#pragma unroll
-    for (int m = 1; m < KMAX; ++m)
-        if (m == j) {
-            my_id = ix[m];
-            w = v[m];
+        for (int o = L / 2; o > 0; o >>= 1) {
+            const float ov = __shfl_xor_sync(0xffffffffu, wv, o);
+            const int oc = __shfl_xor_sync(0xffffffffu, wc, o);
+            if (ranks_before(ov, oc, wv, wc)) {
+                wv = ov;
+                wc = oc;
+            }
         }
-    if (renorm) {
-        // every lane of the group holds the same sorted list: the same sum
-        sum = 0.0f;
-#pragma unroll
-        for (int m = 0; m < KMAX; ++m)
-            if (m < k) sum += __expf(v[m] - mx);
+        if (j == slot) {
+            my_id = wc;
+            my_v = wv;
+        }
+        // this lane owned the winner: take it, find the next best (a lane with
+        // no candidate left -- NaN logits -- holds the sentinel, never an index)
+        if (wc == bc && wc < E) {
+            cell(wc) = -INFINITY;
+            bv = -INFINITY;
+            bc = 0x7fffffff;
+            for (int c = j; c < E; c += L) {
+                const float l = cell(c);
+                if (l > bv) {
+                    bv = l;
+                    bc = c;
+                }
+            }
+        }
     }
-    my_w = __expf(w - mx) / sum;
+    if (renorm) {
+        // the selected terms only (lanes >= k hold 0), in a fixed order
+        float s = j < k ? __expf(my_v - mx) : 0.0f;
+#pragma unroll
+        for (int o = L / 2; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+        sum = s;
+    }
+    my_w = __expf(my_v - mx) / sum;
 }
 
 // One pass of softmax + top-k over the `own` buffered rows, L lanes per
 // token (32 / L tokens per warp).
 template <int L, int KMAX>
-__device__ __forceinline__ void topk_rows(const Params& p, const float* buf, const float* s_bias, int* s_hist,
+__device__ __forceinline__ void topk_rows(const Params& p, float* buf, const float* s_bias, int* s_hist,
                                           int S, int own, int pitch, int tile0, int row0, bool ok, int warp,
                                           int lane)
 {
@@ -312,12 +281,16 @@ __device__ __forceinline__ void topk_rows(const Params& p, const float* buf, con
         const int64_t t = (int64_t)tile0 + row0 + i;
         int my_id;
         float my_w;
-        group_topk<L, KMAX>(E, p.k, p.renorm != 0, j, [&](int c) {
-            const float* col = buf + (size_t)c * pitch + i;
-            float l = col[0];
-            for (int s = 1; s < S; ++s) l += col[(size_t)s * E * pitch];
-            return l + s_bias[c];
-        }, my_id, my_w, (p.probs && ok && t < p.T) ? p.probs + t * p.probs_tstride : nullptr, p.probs_estride);
+        group_topk<L>(
+            E, p.k, p.renorm != 0, j,
+            [&](int c) {
+                const float* col = buf + (size_t)c * pitch + i;
+                float l = col[0];
+                for (int s = 1; s < S; ++s) l += col[(size_t)s * E * pitch];
+                return l + s_bias[c];
+            },
+            [&](int c) -> float& { return buf[(size_t)c * pitch + i]; }, my_id, my_w,
+            (p.probs && ok && t < p.T) ? p.probs + t * p.probs_tstride : nullptr, p.probs_estride);
         if (ok && t < p.T && j < p.k) {
             p.ids[t * p.k + j] = my_id;
             p.wts[t * p.k + j] = my_w;
