@@ -581,6 +581,69 @@ def time_workload(name, args, dev):
     return res
 
 
+def backward_flops(cfg):
+    """FLOPs of one moe_backward: the recomputed gate/up GEMM, dh, dx_perm,
+    the three expert weight gradients and the router's three T x d x E
+    products (logits again, dW_router, dx_router)."""
+    T, d, E, k, f = cfg.T, cfg.d, cfg.E, cfg.k, cfg.f
+    expert = 2 * T * k * d * f
+    return 2 * expert + expert + 2 * expert + 2 * expert + expert + 3 * 2 * T * d * E
+
+
+def run_backward(args, cfg):
+    """Time moe_backward on one GPU (inputs resident, L2 flushed between
+    steps, CUDA events on the launching stream) and print its JSON line."""
+    import torch
+
+    import top_routing_grouped_softmax_b200 as moe
+    from top_routing_grouped_softmax_b200.synth import make_dout, make_inputs
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    inp = make_inputs(cfg)
+    x = inp.x.to(dev)
+    w = {n: getattr(inp, n).to(dev) for n in ("W_router", "W_gate", "W_up", "W_down")}
+    bias = None if inp.bias is None else inp.bias.to(dev)
+    dout = make_dout(cfg.T, cfg.d, cfg.seed).to(dev)
+    ws = torch.empty(moe.backward_workspace_size(cfg.T, cfg.d, cfg.E, cfg.k, cfg.f), dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def step():
+        return moe.backward(x, w["W_router"], w["W_gate"], w["W_up"], w["W_down"], cfg.k, dout, bias=bias,
+                            workspace=ws)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    with ClockSampler(0) as clk:
+        for a, b in evs:
+            flush.zero_()
+            a.record()
+            step()
+            b.record()
+        torch.cuda.synchronize()
+    status = moe.get_status()
+    assert status == moe.MOE_OK, moe.strerror(status)
+    ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
+    peaks = load_peaks()
+    flops = backward_flops(cfg)
+    tflops = flops / (ms * 1e-3) / 1e12
+    line = {
+        "metric": "MoE-layer bwd tokens/s & TFLOP/s vs roofline, 1xB200", "value": cfg.T / (ms * 1e-3),
+        "unit": "tokens/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": workload_config(cfg, extra={"pass": "backward (activations recomputed)", "grads_dtype": "fp32"}),
+        "roofline": {"bound": "tensor", "scope": "the whole backward", "achieved": tflops,
+                     "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": tflops / peaks["bf16_tflops"],
+                     "traffic": None, "flops": flops, "peak_source": f"{peaks['source']} burst bf16"},
+        "gpu_launches": 16 * args.steps,  # 6 routing and grouping, 7 GEMMs, router step, bias sum, combine
+        "clocks": clk.summary(),
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -600,6 +663,8 @@ def main(argv=None):
                     help="tokens of the workload the CPU-oracle baseline leg evaluates")
     ap.add_argument("--ref-tokens", type=int, default=32, help="tokens per step of the reference arm")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--backward", action="store_true",
+                    help="time moe_backward (gradients of the block, activations recomputed) on one GPU instead")
     ap.add_argument("--workloads", default="coarse,fine,skew",
                     help="other workloads to time at N=1 (fused path) into the line's `workloads` object; "
                          "empty to skip")
@@ -612,6 +677,8 @@ def main(argv=None):
 
     from top_routing_grouped_softmax_b200 import _build
     _build.build_library()
+    if args.backward:
+        return run_backward(args, cfg)
     res = run_gpu(args, cfg)
     rank, _, world = dist_env()
     if rank == 0 and res is not None:

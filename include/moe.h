@@ -394,6 +394,20 @@ int moe_backward(const moe_bf16* x, const moe_bf16* w_router, const float* bias,
                  void* workspace, size_t workspace_bytes, cudaStream_t stream, unsigned flags);
 
 /*
+ * Row gather for moving grouped rows between layouts (the expert-parallel
+ * dispatch regroups the rows it receives by local expert and returns them in
+ * the order they came; the pages' hierarchical all-to-all of the
+ * Hunyuan-Large overview, section 5.1, leaves the layout open):
+ *   dst[i] = src[idx[i]] for i < n, whole rows of row_bytes bytes
+ *   src [n_src rows], dst [n rows]: device; row_bytes % 4 == 0; 16-byte
+ *   aligned when row_bytes % 16 == 0 (copied in 16-byte vectors), else 4-byte
+ *   idx [n] int32 device; an index outside [0, n_src) is reported as
+ *   MOE_ERR_DEVICE_BOUNDS and its row is zero-filled.
+ */
+int moe_gather_rows(const void* src, const int32_t* idx, int64_t n_src, int64_t n, int64_t row_bytes, void* dst,
+                    cudaStream_t stream);
+
+/*
  * Synchronises `stream`, then returns and clears the current device's status
  * word (MOE_OK if no device-side error was recorded since the last call).
  */

@@ -41,7 +41,7 @@ ABI_SYMBOLS = (
     "moe_forward_ex", "moe_get_status", "moe_set_wait_limit_ns", "moe_selftest_wait_timeout",
     "moe_permute_static", "moe_route_ex", "moe_workspace_size_shared", "moe_shared_ffn", "moe_combine_shared",
     "moe_forward_shared", "moe_workspace_size_rounded", "moe_forward_rounded",
-    "moe_backward_workspace_size", "moe_backward",
+    "moe_backward_workspace_size", "moe_backward", "moe_gather_rows",
 )
 
 
@@ -97,13 +97,14 @@ def lib() -> ctypes.CDLL:
         L.moe_backward_workspace_size.restype = _SZ
         L.moe_backward_workspace_size.argtypes = [_I64] * 5
         L.moe_backward.argtypes = [_P] * 7 + [_I64] * 5 + [_P] * 7 + [_SZ, _P, ctypes.c_uint]
+        L.moe_gather_rows.argtypes = [_P, _P, _I64, _I64, _I64, _P, _P]
         L.moe_get_status.argtypes = [_P]
         L.moe_set_wait_limit_ns.argtypes = [_I64]
         L.moe_selftest_wait_timeout.argtypes = [_I64, _P]
         for name in ("moe_route", "moe_permute", "moe_expert_ffn", "moe_combine", "moe_forward",
                      "moe_forward_ex", "moe_get_status", "moe_set_wait_limit_ns",
                      "moe_selftest_wait_timeout", "moe_permute_static", "moe_route_ex", "moe_shared_ffn",
-                     "moe_combine_shared", "moe_forward_shared", "moe_forward_rounded", "moe_backward"):
+                     "moe_combine_shared", "moe_forward_shared", "moe_forward_rounded", "moe_backward", "moe_gather_rows"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -369,6 +370,23 @@ def forward(x, w_router, w_gate, w_up, w_down, k, bias=None, out=None, workspace
     return out
 
 
+def gather_rows(src, idx, out=None):
+    """out[i] = src[idx[i]] (whole rows) on the GPU; src is 1-D or 2-D and
+    contiguous, each row a multiple of 4 bytes; idx int32 on the same device."""
+    if not (src.is_cuda and src.is_contiguous() and src.dim() in (1, 2)):
+        raise ValueError("src: contiguous 1-D or 2-D CUDA tensor expected")
+    if src.dim() == 1:
+        return gather_rows(src.view(-1, 1), idx, None if out is None else out.view(-1, 1)).view(-1)
+    _need(idx, "idx", torch.int32, 1)
+    n = idx.shape[0]
+    if out is None:
+        out = torch.empty(n, src.shape[1], dtype=src.dtype, device=src.device)
+    row_bytes = src.shape[1] * src.element_size()
+    _check(lib().moe_gather_rows(_ptr(src), _ptr(idx), src.shape[0], n, row_bytes, _ptr(out), _stream()),
+           "moe_gather_rows")
+    return out
+
+
 def backward_workspace_size(T: int, d: int, E: int, k: int, f: int) -> int:
     return int(lib().moe_backward_workspace_size(T, d, E, k, f))
 
@@ -458,6 +476,6 @@ __all__ = [
     "lib", "strerror", "MoEError", "ABI_SYMBOLS", "workspace_size", "route_workspace_size",
     "permute_workspace_size", "MOE_FLAG_FUSED_GATHER", "MOE_FLAG_RENORMALIZE", "route",
     "permute", "expert_ffn", "combine", "forward", "shared_ffn", "combine_shared", "forward_shared", "forward_rounded",
-    "get_status", "set_wait_limit_ns", "backward", "backward_workspace_size",
+    "get_status", "set_wait_limit_ns", "backward", "backward_workspace_size", "gather_rows",
     "selftest_wait_timeout", "MoEBlock",
 ]

@@ -1345,6 +1345,31 @@ int moe_forward_ex(const moe_bf16* x, const moe_bf16* w_router, const float* bia
                         workspace, workspace_bytes, stream, events, n_events, flags);
 }
 
+int moe_gather_rows(const void* src, const int32_t* idx, int64_t n_src, int64_t n, int64_t row_bytes, void* dst,
+                    cudaStream_t stream)
+{
+    if (n_src < 0 || n < 0 || row_bytes <= 0) return MOE_ERR_INVALID_ARG;
+    if (row_bytes % 4 != 0 || row_bytes / 4 > (int64_t(1) << 24) || n >= (int64_t(1) << 31) ||
+        n * (row_bytes / 4) >= (int64_t(1) << 40))
+        return MOE_ERR_UNSUPPORTED_SHAPE;
+    if (n > 0 && (!src || !idx || !dst)) return MOE_ERR_INVALID_ARG;
+    const bool wide = row_bytes % 16 == 0;
+    if (!aligned(src, wide ? 16 : 4) || !aligned(dst, wide ? 16 : 4) || !aligned(idx, 4)) return MOE_ERR_INVALID_ARG;
+    if (n == 0) return MOE_OK;
+    DeviceState* st = nullptr;
+    int rc = setup_device(&st);
+    if (rc) return rc;
+    using namespace moe::permute;
+    if (wide)
+        return launch(gather_rows_idx_kernel, dim3((unsigned)((n + kWarps - 1) / kWarps)), dim3(kThreads), 0, stream,
+                      1u, static_cast<const uint4*>(src), idx, n, n_src, (int)(row_bytes / 16),
+                      static_cast<uint4*>(dst));
+    const int64_t words = n * (row_bytes / 4);
+    return launch(gather_words_idx_kernel, dim3((unsigned)((words + kThreads - 1) / kThreads)), dim3(kThreads), 0,
+                  stream, 1u, static_cast<const uint32_t*>(src), idx, n, n_src, (int)(row_bytes / 4),
+                  static_cast<uint32_t*>(dst));
+}
+
 size_t moe_backward_workspace_size(int64_t T, int64_t d, int64_t E, int64_t k, int64_t f)
 {
     if (check_common(T, d, E, k) || check_f(f)) return 0;

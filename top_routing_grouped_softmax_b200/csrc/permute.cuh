@@ -268,5 +268,42 @@ __global__ void __launch_bounds__(kThreads) gather_kernel(const uint4* __restric
     }
 }
 
+// dst[i] = src[idx[i]] for whole rows of nvec 16-byte vectors: one warp per
+// row.  An index outside [0, n_src) is reported and its row is zero-filled.
+__global__ void __launch_bounds__(kThreads) gather_rows_idx_kernel(const uint4* __restrict__ src,
+                                                                   const int32_t* __restrict__ idx, int64_t n,
+                                                                   int64_t n_src, int nvec, uint4* __restrict__ dst)
+{
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int64_t i = (int64_t)blockIdx.x * kWarps + warp;
+    pdl_trigger();
+    pdl_wait();
+    if (i >= n) return;
+    const int r = __ldg(idx + i);
+    const bool ok = r >= 0 && (int64_t)r < n_src;
+    if (!ok && lane == 0) record_status(kStatusDeviceBounds);
+    const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+    for (int v = lane; v < nvec; v += 32) dst[i * nvec + v] = ok ? __ldg(src + (int64_t)r * nvec + v) : z;
+}
+
+// The same for rows of nword 4-byte words (rows that are not a multiple of
+// 16 bytes, such as one routing weight per row).
+__global__ void __launch_bounds__(kThreads) gather_words_idx_kernel(const uint32_t* __restrict__ src,
+                                                                    const int32_t* __restrict__ idx, int64_t n,
+                                                                    int64_t n_src, int nword, uint32_t* __restrict__ dst)
+{
+    const int64_t i0 = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+    pdl_trigger();
+    pdl_wait();
+    const int64_t total = n * nword;
+    if (i0 >= total) return;
+    const int64_t i = i0 / nword;
+    const int wd = (int)(i0 - i * nword);
+    const int r = __ldg(idx + i);
+    const bool ok = r >= 0 && (int64_t)r < n_src;
+    if (!ok && wd == 0) record_status(kStatusDeviceBounds);
+    dst[i0] = ok ? __ldg(src + (int64_t)r * nword + wd) : 0u;
+}
+
 }  // namespace permute
 }  // namespace moe
