@@ -19,7 +19,7 @@
 //                 dlogit = p (dp - sum_e p_e dp_e) (the softmax Jacobian);
 //                 stores dlogit in bf16 (the operand of the two router GEMMs)
 //                 and the block's fp32 sums of dlogit for the bias gradient
-//   colsum        dbias[e] = sum over blocks of those sums, in block order
+//   colsum        dbias[e] = sum over blocks of those sums, in a fixed order
 //   combine_dx    dx[t] = dx_router[t] + sum_j dx_perm[inv[t*k+j]]  (fp32)
 #pragma once
 
@@ -92,7 +92,8 @@ __global__ void __launch_bounds__(kRowThreads) zero_pad_kernel(const int32_t* __
 
 // One warp per token, eight tokens per block.  probs [T][E] fp32 (the
 // router's probabilities, recomputed), ids / wts [T][k], inv [T*k], dwp
-// [rows][n_tiles] (the down GEMM's partial dot products).  Writes dlogit
+// [rows][n_tiles] (the down GEMM's partial dot products; n_tiles counts
+// them per row).  Writes dlogit
 // [T][ld_dl] bf16 (columns past E zero) and, per block, the fp32 sum of its tokens' dlogit rows
 // (db_part [gridDim.x][E], added in warp order).
 __global__ void __launch_bounds__(kRowThreads) route_bwd_kernel(
@@ -159,17 +160,25 @@ __global__ void __launch_bounds__(kRowThreads) route_bwd_kernel(
         }
 }
 
-// dbias[e] = sum over blocks b (ascending) of db_part[b][e].
+// dbias[e] = sum over blocks b of db_part[b][e]: one block per expert;
+// thread i sums blocks i, i + 256, ... in order, then a fixed tree adds the
+// 256 partial sums (the same order on every run).
 __global__ void __launch_bounds__(kRowThreads) colsum_kernel(const float* __restrict__ db_part, int nblk, int E,
                                                              float* __restrict__ dbias)
 {
-    const int e = blockIdx.x * kRowThreads + threadIdx.x;
+    __shared__ float s_part[kRowThreads];
+    const int e = blockIdx.x;
     pdl_trigger();
     pdl_wait();
-    if (e >= E) return;
     float acc = 0.0f;
-    for (int b = 0; b < nblk; ++b) acc += __ldg(db_part + (int64_t)b * E + e);
-    dbias[e] = acc;
+    for (int b = threadIdx.x; b < nblk; b += kRowThreads) acc += __ldg(db_part + (int64_t)b * E + e);
+    s_part[threadIdx.x] = acc;
+    __syncthreads();
+    for (int w = kRowThreads / 2; w > 0; w >>= 1) {
+        if (threadIdx.x < w) s_part[threadIdx.x] += s_part[threadIdx.x + w];
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) dbias[e] = s_part[0];
 }
 
 // dx[t] = dx_router[t] + sum_j dx_perm[inv[t*k+j]] (fp32, slots in order):

@@ -21,7 +21,7 @@
 //          s = 1/(1+e^-g),  h = g s u,
 //          dg = dh u s (1 + g (1 - s)),  du = dh g s,
 //        and the routing-weight gradient's partial dot products
-//          dwp[row][nt] = sum over this tile's columns of (dh / w) h
+//          dwp[row][2 nt + half] = sum over that half of the tile's columns of (dh / w) h
 //        (dh / w is the unweighted accumulator: dout . (h W_down) = (dout W_down^T) . h).
 //        A = dout_perm rows (K-major), B = W_down[e] rows (K-major: W_down[e] is
 //        [f][d], its rows are the output columns).  Stores dg, du and
@@ -49,15 +49,21 @@ using gemm::kBK;
 using gemm::kBM;
 using gemm::kBN;
 using gemm::kChunkBytes;
-using gemm::kEpiWarps;
 using gemm::kMaxE;
 using gemm::kPairRows;
 using gemm::kPairStageBytes;
 using gemm::kPairStages;
-using gemm::kThreads;
 using gemm::kTmemCols;
 
 enum Kind { kGU = 0, kDH = 1, kDX = 2, kDW = 3 };
+
+// Eight epilogue warps: two per TMEM lane quarter, each taking half of the
+// tile's columns.  The backward's epilogues do more per element than the
+// forward's (kDH reads g and u and writes three bf16 outputs; kDW and kDX
+// write fp32), so they need the issue slots of eight warps to keep pace
+// with the MMAs.
+constexpr int kEpiWarps = 8;
+constexpr int kThreads = 64 + kEpiWarps * 32;
 
 struct Params {
     const int32_t* offsets;  // [E+1] group starts; nullptr: one group of M rows
@@ -67,7 +73,7 @@ struct Params {
     __nv_bfloat16* out_g;    // kGU: g;  kDH: dg        [rows][ld_f]
     __nv_bfloat16* out_u;    // kGU: u;  kDH: du
     __nv_bfloat16* out_hw;   // kDH: w * h
-    float* dwp;              // kDH: [rows][n_tiles] partial dot products
+    float* dwp;              // kDH: [rows][2 * n_tiles] partial dot products (two column halves per tile)
     float* out0;             // kDX: [rows][ld_out];  kDW: [E][m_total][ld_out] (gate part when split)
     float* out1;             // kDW split: the up part
     int64_t ld_f;            // row length of g, u, dg, du, hw
@@ -98,7 +104,18 @@ struct alignas(8) Ctrl {
     int tp[kMaxE + 1];
 };
 
-__host__ inline size_t smem_bytes() { return 1024 + (size_t)kPairStages * kPairStageBytes + sizeof(Ctrl); }
+// Ring depth per kind: kDW gives two stages to the staging slabs of its
+// TMA-store epilogue (eight warps x two 32 x 32 fp32 slabs).
+constexpr int kSlabBytes = 32 * 32 * 4;
+constexpr int kStoreBytes = kEpiWarps * 2 * kSlabBytes;
+__host__ __device__ constexpr int stages_for(int kind) { return kind == kDW ? 4 : kPairStages; }
+__host__ __device__ constexpr int store_bytes_for(int kind) { return kind == kDW ? kStoreBytes : 0; }
+
+template <int KIND>
+__host__ inline size_t smem_bytes()
+{
+    return 1024 + (size_t)stages_for(KIND) * kPairStageBytes + store_bytes_for(KIND) + sizeof(Ctrl);
+}
 
 // One work item of kind KIND: the expert, the first grouped row (M-grouped
 // kinds) or M tile (kDW), the group's row range, the N tile and the number
@@ -130,7 +147,9 @@ __device__ __forceinline__ Item decode_item(int64_t w, const Params& p, const Ct
     return it;
 }
 
-__device__ __forceinline__ float sigmoid(float z) { return 1.0f / (1.0f + __expf(-z)); }
+// 1 / (1 + e^-z) with the fast reciprocal division (about 2 ulp in fp32; the
+// results are rounded to bf16).
+__device__ __forceinline__ float sigmoid(float z) { return __fdividef(1.0f, 1.0f + __expf(-z)); }
 
 __device__ __forceinline__ void unpack_bf16x8(const uint4& q, float (&v)[8])
 {
@@ -163,9 +182,15 @@ __device__ __forceinline__ void store_zero_f32x16(float* dst)
 // Drains one accumulator tile.  The calling warp reads TMEM lane quarter q:
 // row q*32 + lane of this CTA's 128 rows.  tbase addresses the accumulator
 // at this warp's lane quarter.
+// `half` selects the columns this warp drains: half of the tile's output
+// columns (kGU: 64 of 128; the others: 128 of 256).  kDW stages its output
+// in `slab` (two 4 KB buffers of this warp, alternated by slab_buf) and
+// stores it with TMA through tm_o0 / tm_o1 ([E][m_total][n_out] fp32 views;
+// rows past m_total and columns past n_out are not written).
 template <int KIND>
 __device__ __forceinline__ void epilogue(const Params& p, const Item& it, uint32_t tbase, uint32_t rank, int q,
-                                         int lane)
+                                         int lane, int half, const CUtensorMap* tm_o0, const CUtensorMap* tm_o1,
+                                         float* slab, int& slab_buf)
 {
     const int r = (int)rank * kBM + q * 32 + lane;  // row of the 256-row pair tile
     if constexpr (KIND == kGU) {
@@ -174,7 +199,7 @@ __device__ __forceinline__ void epilogue(const Params& p, const Item& it, uint32
         const int c_base = it.nt * 128;
         const int ncols = min(128, p.n_out - c_base);
 #pragma unroll 1
-        for (int c0 = 0; c0 < 128; c0 += 16) {
+        for (int c0 = half * 64; c0 < half * 64 + 64; c0 += 16) {
             uint32_t g[16], u[16];
             tmem_ld16(tbase + c0, g);
             tmem_ld16(tbase + 128 + c0, u);
@@ -200,32 +225,36 @@ __device__ __forceinline__ void epilogue(const Params& p, const Item& it, uint32
         const int c_base = it.nt * kBN;
         const int ncols = min(kBN, p.n_out - c_base);
         const float w = valid ? __ldg(p.w_perm + row) : 0.0f;
+        const int64_t row_off = (int64_t)row * p.ld_f + c_base;
         float dot = 0.0f;
-#pragma unroll 1
-        for (int c0 = 0; c0 < kBN; c0 += 16) {
+        // g and u of the next 16 columns are in flight while this chunk is
+        // processed (the loads are row-strided across the warp and would
+        // otherwise expose their latency once per chunk)
+        uint4 gq[2][2], uq[2][2];
+        auto fetch = [&](int c0, int b) {
+            if (valid && c0 < ncols) {
+                const uint4* gp = reinterpret_cast<const uint4*>(p.g + row_off + c0);
+                const uint4* up = reinterpret_cast<const uint4*>(p.u + row_off + c0);
+                gq[b][0] = __ldg(gp);
+                gq[b][1] = __ldg(gp + 1);
+                uq[b][0] = __ldg(up);
+                uq[b][1] = __ldg(up + 1);
+            }
+        };
+        fetch(half * 128, 0);
+#pragma unroll
+        for (int ci = 0; ci < 8; ++ci) {
+            const int c0 = half * 128 + ci * 16;
+            if (ci + 1 < 8) fetch(c0 + 16, (ci + 1) & 1);
             uint32_t acc[16];
             tmem_ld16(tbase + c0, acc);
             tmem_ld_wait();
             if (valid && c0 < ncols) {
-                const int64_t off = (int64_t)row * p.ld_f + c_base + c0;
-                const uint4* gp = reinterpret_cast<const uint4*>(p.g + off);
-                const uint4* up = reinterpret_cast<const uint4*>(p.u + off);
                 float g[16], u[16];
-                {
-                    float t[8];
-                    unpack_bf16x8(gp[0], t);
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) g[i] = t[i];
-                    unpack_bf16x8(gp[1], t);
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) g[8 + i] = t[i];
-                    unpack_bf16x8(up[0], t);
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) u[i] = t[i];
-                    unpack_bf16x8(up[1], t);
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) u[8 + i] = t[i];
-                }
+                unpack_bf16x8(gq[ci & 1][0], *reinterpret_cast<float(*)[8]>(&g[0]));
+                unpack_bf16x8(gq[ci & 1][1], *reinterpret_cast<float(*)[8]>(&g[8]));
+                unpack_bf16x8(uq[ci & 1][0], *reinterpret_cast<float(*)[8]>(&u[0]));
+                unpack_bf16x8(uq[ci & 1][1], *reinterpret_cast<float(*)[8]>(&u[8]));
                 uint32_t pdg[8], pdu[8], phw[8];
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
@@ -234,12 +263,12 @@ __device__ __forceinline__ void epilogue(const Params& p, const Item& it, uint32
                     for (int h2 = 0; h2 < 2; ++h2) {
                         const int c = 2 * i + h2;
                         const float dhu = __uint_as_float(acc[c]);  // dout . W_down^T (unweighted)
-                        const float s = sigmoid(g[c]);
-                        const float gs = g[c] * s;
+                        const float sg = sigmoid(g[c]);
+                        const float gs = g[c] * sg;
                         const float h = gs * u[c];
                         const float dh = w * dhu;
                         dot += dhu * h;
-                        dgv[h2] = dh * u[c] * s * (1.0f + g[c] * (1.0f - s));
+                        dgv[h2] = dh * u[c] * sg * (1.0f + g[c] * (1.0f - sg));
                         duv[h2] = dh * gs;
                         hwv[h2] = w * h;
                     }
@@ -247,9 +276,9 @@ __device__ __forceinline__ void epilogue(const Params& p, const Item& it, uint32
                     pdu[i] = gemm::pack_bf16x2(duv[0], duv[1]);
                     phw[i] = gemm::pack_bf16x2(hwv[0], hwv[1]);
                 }
-                uint4* dgp = reinterpret_cast<uint4*>(p.out_g + off);
-                uint4* dup = reinterpret_cast<uint4*>(p.out_u + off);
-                uint4* hwp = reinterpret_cast<uint4*>(p.out_hw + off);
+                uint4* dgp = reinterpret_cast<uint4*>(p.out_g + row_off + c0);
+                uint4* dup = reinterpret_cast<uint4*>(p.out_u + row_off + c0);
+                uint4* hwp = reinterpret_cast<uint4*>(p.out_hw + row_off + c0);
                 dgp[0] = make_uint4(pdg[0], pdg[1], pdg[2], pdg[3]);
                 dgp[1] = make_uint4(pdg[4], pdg[5], pdg[6], pdg[7]);
                 dup[0] = make_uint4(pdu[0], pdu[1], pdu[2], pdu[3]);
@@ -258,52 +287,50 @@ __device__ __forceinline__ void epilogue(const Params& p, const Item& it, uint32
                 hwp[1] = make_uint4(phw[4], phw[5], phw[6], phw[7]);
             }
         }
-        if (valid) p.dwp[(int64_t)row * p.n_tiles + it.nt] = dot;
+        if (valid) p.dwp[(int64_t)row * (2 * p.n_tiles) + 2 * it.nt + half] = dot;
     } else if constexpr (KIND == kDX) {
         const int row = it.row0 + r;
         const bool valid = row < it.row_end;
         const int c_base = it.nt * kBN;
         const int ncols = min(kBN, p.n_out - c_base);
 #pragma unroll 1
-        for (int c0 = 0; c0 < kBN; c0 += 16) {
+        for (int c0 = half * 128; c0 < half * 128 + 128; c0 += 16) {
             uint32_t acc[16];
             tmem_ld16(tbase + c0, acc);
             tmem_ld_wait();
             if (valid && c0 < ncols) store_f32x16(p.out0 + (int64_t)row * p.ld_out + c_base + c0, acc);
         }
-    } else {  // kDW
-        const int m = it.mt * kPairRows + r;
-        const bool valid = m < p.m_total;
+    } else {  // kDW: 32 x 32 fp32 slabs staged in shared memory, written by TMA
         const bool empty = it.num_kb == 0;
-        const int64_t obase = ((int64_t)it.e * p.m_total + m) * p.ld_out;
+        const int m0 = it.mt * kPairRows + (int)rank * kBM + q * 32;  // first row of this warp's slabs
 #pragma unroll 1
-        for (int c0 = 0; c0 < kBN; c0 += 16) {
-            uint32_t acc[16];
-            tmem_ld16(tbase + c0, acc);
+        for (int c0 = half * 128; c0 < half * 128 + 128; c0 += 32) {
+            uint32_t lo[16], hi[16];
+            tmem_ld16(tbase + c0, lo);
+            tmem_ld16(tbase + c0 + 16, hi);
             tmem_ld_wait();
-            if (!valid) continue;
-            float* dst;
-            int col;
-            if (p.split_b) {
-                col = it.nt * 128 + (c0 & 127);
-                dst = (c0 < 128 ? p.out0 : p.out1) + obase + col;
-            } else {
-                col = it.nt * kBN + c0;
-                dst = p.out0 + obase + col;
-            }
-            if (col >= p.n_out) continue;
-            if (col + 16 <= p.n_out) {
-                if (empty)
-                    store_zero_f32x16(dst);
-                else
-                    store_f32x16(dst, acc);
-            } else {
-                // a row that ends inside this 16-column chunk (n_out % 16 == 8)
-                const int n = p.n_out - col;
+            uint32_t* buf = reinterpret_cast<uint32_t*>(slab) + slab_buf * (kSlabBytes / 4);
+            if (lane == 0) bulk_wait_group_read<1>();  // the store that last read `buf` is done
+            __syncwarp();
+            // row `lane` of the slab: 8 x 16 B chunks, 128-byte swizzle
+            uint4* rowp = reinterpret_cast<uint4*>(buf + lane * 32);
+            const int sw = lane & 7;
 #pragma unroll
-                for (int i = 0; i < 16; ++i)
-                    if (i < n) dst[i] = empty ? 0.0f : __uint_as_float(acc[i]);
+            for (int v = 0; v < 4; ++v) {
+                rowp[v ^ sw] = empty ? make_uint4(0u, 0u, 0u, 0u)
+                                     : make_uint4(lo[4 * v], lo[4 * v + 1], lo[4 * v + 2], lo[4 * v + 3]);
+                rowp[(4 + v) ^ sw] = empty ? make_uint4(0u, 0u, 0u, 0u)
+                                           : make_uint4(hi[4 * v], hi[4 * v + 1], hi[4 * v + 2], hi[4 * v + 3]);
             }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                const bool second = p.split_b && c0 >= 128;
+                const int col = p.split_b ? it.nt * 128 + (c0 & 127) : it.nt * kBN + c0;
+                tma_store_3d(second ? tm_o1 : tm_o0, buf, col, m0, it.e);
+                bulk_commit_group();
+            }
+            slab_buf ^= 1;
         }
     }
 }
@@ -311,13 +338,16 @@ __device__ __forceinline__ void epilogue(const Params& p, const Item& it, uint32
 template <int KIND>
 __global__ void __launch_bounds__(kThreads, 1)
     pair_bwd_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_a2,
-                    const __grid_constant__ CUtensorMap tm_b0, const __grid_constant__ CUtensorMap tm_b1, Params p)
+                    const __grid_constant__ CUtensorMap tm_b0, const __grid_constant__ CUtensorMap tm_b1,
+                    const __grid_constant__ CUtensorMap tm_o0, const __grid_constant__ CUtensorMap tm_o1, Params p)
 {
     constexpr bool kAMN = KIND == kDW;                   // A read MN-major
     constexpr bool kBK_MAJOR = KIND == kDH || KIND == kDX;  // B read K-major
+    constexpr int kStages = stages_for(KIND);
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    Ctrl& c = *reinterpret_cast<Ctrl*>(smem + (size_t)kPairStages * kPairStageBytes);
+    uint8_t* stage_out = smem + (size_t)kStages * kPairStageBytes;
+    Ctrl& c = *reinterpret_cast<Ctrl*>(stage_out + store_bytes_for(KIND));
 
     const int warp = threadIdx.x / 32;
     const int lane = threadIdx.x % 32;
@@ -329,7 +359,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int64_t npairs = num_clusters_x();
 
     if (threadIdx.x == 32) {
-        for (int s = 0; s < kPairStages; ++s) {
+        for (int s = 0; s < kStages; ++s) {
             mbar_init(&c.full[s], 1);
             mbar_init(&c.empty[s], 1);
         }
@@ -344,6 +374,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_prefetch_map(&tm_b0);
         if (KIND == kDX) tma_prefetch_map(&tm_a2);
         if (KIND == kGU || KIND == kDX || KIND == kDW) tma_prefetch_map(&tm_b1);
+        if (KIND == kDW) {
+            tma_prefetch_map(&tm_o0);
+            tma_prefetch_map(&tm_o1);
+        }
     }
     if (warp == 1) {
         __syncwarp();
@@ -400,7 +434,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             tma_load_3d_pair(sb, &tm_b0, bar, 0, kr, it.nt * (kBN / 64) + (int)rank * 2);
                     }
                     ++issued;
-                    if (++s == kPairStages) {
+                    if (++s == kStages) {
                         s = 0;
                         ph ^= 1u;
                     }
@@ -410,8 +444,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     break;
                 }
             }
-            for (int qq = 0; qq < kPairStages; ++qq) {
-                const int64_t cnt = issued / kPairStages + (qq < issued % kPairStages ? 1 : 0);
+            for (int qq = 0; qq < kStages; ++qq) {
+                const int64_t cnt = issued / kStages + (qq < issued % kStages ? 1 : 0);
                 if (cnt > 0)
                     mbar_wait(leader ? &c.full[qq] : &c.empty[qq], (uint32_t)(cnt - 1) & 1u, drain_limit(limit));
             }
@@ -451,7 +485,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         mma_bf16_ss_pair(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
                     }
                     mma_commit_pair_multicast(&c.empty[s], 0x3);
-                    if (++s == kPairStages) {
+                    if (++s == kStages) {
                         s = 0;
                         ph ^= 1u;
                     }
@@ -474,7 +508,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
     } else {
         // ---------------------------------------------------- epilogue (both CTAs)
-        const int q = warp & 3;
+        const int q = warp & 3;                 // TMEM lane quarter
+        const int half = (warp - 2) >> 2;       // column half: warps 2-5 and 6-9
+        float* slab = reinterpret_cast<float*>(stage_out + (warp - 2) * 2 * kSlabBytes);
+        int slab_buf = 0;
         int acc = 0;
         uint32_t acc_ph = 0;
         for (int64_t w = pair; w < total_work; w += npairs) {
@@ -488,7 +525,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             tc_fence_after_sync();
             const uint32_t tbase = tmem + (uint32_t)(acc * kBN) + ((uint32_t)(q * 32) << 16);
-            epilogue<KIND>(p, it, tbase, rank, q, lane);
+            epilogue<KIND>(p, it, tbase, rank, q, lane, half, &tm_o0, &tm_o1, slab, slab_buf);
             tc_fence_before_sync();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(mapa_shared(&c.acc_empty[acc], 0));
@@ -497,6 +534,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 acc_ph ^= 1u;
             }
         }
+        if (KIND == kDW && lane == 0) bulk_wait_group_all();
         __syncwarp();
     }
 

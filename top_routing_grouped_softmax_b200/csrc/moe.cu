@@ -799,7 +799,7 @@ BLayout plan_backward(int64_t T, int64_t d, int64_t E, int64_t k, int64_t f)
     L.g = o;         o += align256(R * (size_t)f * 2);   // g, then dg in place
     L.u = o;         o += align256(R * (size_t)f * 2);   // u, then du in place
     L.hw = o;        o += align256(R * (size_t)f * 2);
-    L.dwp = o;       o += align256(R * (size_t)L.n_tiles_f * 4);
+    L.dwp = o;       o += align256(R * (size_t)(2 * L.n_tiles_f) * 4);
     L.dx_perm = o;   o += align256(R * (size_t)d * 4);
     L.dlogit = o;    o += align256((size_t)T * (size_t)L.e_pad * 2);
     L.db_part = o;   o += align256((size_t)((T + moe::bwd::kRowWarps - 1) / moe::bwd::kRowWarps) * (size_t)E * 4);
@@ -808,15 +808,32 @@ BLayout plan_backward(int64_t T, int64_t d, int64_t E, int64_t k, int64_t f)
     return L;
 }
 
+// to0 / to1: the fp32 output views of the weight-gradient kind (kDW); the
+// other kinds ignore them.
 template <int KIND>
 int launch_pair_bwd(const DeviceState& st, int64_t work, const CUtensorMap& ta, const CUtensorMap& ta2,
-                    const CUtensorMap& tb0, const CUtensorMap& tb1, const moe::bwd::Params& p, cudaStream_t s)
+                    const CUtensorMap& tb0, const CUtensorMap& tb1, const moe::bwd::Params& p, cudaStream_t s,
+                    const CUtensorMap* to0 = nullptr, const CUtensorMap* to1 = nullptr)
 {
     int64_t pairs = st.max_pairs > 0 ? st.max_pairs : st.sm_count / 2;
     if (work < pairs) pairs = work;
     if (pairs < 1) pairs = 1;
-    return launch(moe::bwd::pair_bwd_kernel<KIND>, dim3((unsigned)(2 * pairs)), dim3(moe::gemm::kThreads),
-                  moe::bwd::smem_bytes(), s, 2u, ta, ta2, tb0, tb1, p);
+    return launch(moe::bwd::pair_bwd_kernel<KIND>, dim3((unsigned)(2 * pairs)), dim3(moe::bwd::kThreads),
+                  moe::bwd::smem_bytes<KIND>(), s, 2u, ta, ta2, tb0, tb1, to0 ? *to0 : ta, to1 ? *to1 : ta, p);
+}
+
+// fp32 [groups][rows][cols] viewed for 32 x 32 TMA stores (128-byte swizzle);
+// elements outside the extents are clipped by the store.
+int make_out3_map(CUtensorMap* m, float* base, uint64_t cols, uint64_t rows, uint64_t groups)
+{
+    cuuint64_t dims[3] = {cols, rows, groups};
+    cuuint64_t strides[2] = {cols * 4, rows * cols * 4};
+    cuuint32_t box[3] = {32, 32, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
 }
 
 moe::bwd::Params bwd_params()
@@ -983,10 +1000,12 @@ int backward_impl(const moe_bf16* x, const moe_bf16* w_router, const float* bias
     }
     // 6. dW_gate[e], dW_up[e] = x_perm_e^T . dg_e, x_perm_e^T . du_e
     {
-        CUtensorMap ta, tb0, tb1;
+        CUtensorMap ta, tb0, tb1, to0, to1;
         rc = make_weight_chunk_map(&ta, x_perm, (uint64_t)d, (uint64_t)R);
         rc = rc ? rc : make_weight_chunk_map(&tb0, g, (uint64_t)f, (uint64_t)R);
         rc = rc ? rc : make_weight_chunk_map(&tb1, u, (uint64_t)f, (uint64_t)R);
+        rc = rc ? rc : make_out3_map(&to0, dw_gate, (uint64_t)f, (uint64_t)d, (uint64_t)E);
+        rc = rc ? rc : make_out3_map(&to1, dw_up, (uint64_t)f, (uint64_t)d, (uint64_t)E);
         if (rc) return rc;
         Params p = bwd_params();
         p.offsets = offsets;
@@ -1000,13 +1019,15 @@ int backward_impl(const moe_bf16* x, const moe_bf16* w_router, const float* bias
         p.m_total = (int)d;
         p.m_tiles = (int)((d + kPairRows - 1) / kPairRows);
         p.split_b = 1;
-        if (launch_pair_bwd<kDW>(*st, E * p.m_tiles * p.n_tiles, ta, ta, tb0, tb1, p, s)) return MOE_ERR_CUDA;
+        if (launch_pair_bwd<kDW>(*st, E * p.m_tiles * p.n_tiles, ta, ta, tb0, tb1, p, s, &to0, &to1))
+            return MOE_ERR_CUDA;
     }
     // 7. dW_down[e] = (w h)_e^T . dout_perm_e
     {
-        CUtensorMap ta, tb;
+        CUtensorMap ta, tb, to0;
         rc = make_weight_chunk_map(&ta, hw, (uint64_t)f, (uint64_t)R);
         rc = rc ? rc : make_weight_chunk_map(&tb, dout_perm, (uint64_t)d, (uint64_t)R);
+        rc = rc ? rc : make_out3_map(&to0, dw_down, (uint64_t)d, (uint64_t)f, (uint64_t)E);
         if (rc) return rc;
         Params p = bwd_params();
         p.offsets = offsets;
@@ -1019,23 +1040,25 @@ int backward_impl(const moe_bf16* x, const moe_bf16* w_router, const float* bias
         p.m_total = (int)f;
         p.m_tiles = (int)((f + kPairRows - 1) / kPairRows);
         p.split_b = 0;
-        if (launch_pair_bwd<kDW>(*st, E * p.m_tiles * p.n_tiles, ta, ta, tb, tb, p, s)) return MOE_ERR_CUDA;
+        if (launch_pair_bwd<kDW>(*st, E * p.m_tiles * p.n_tiles, ta, ta, tb, tb, p, s, &to0, &to0))
+            return MOE_ERR_CUDA;
     }
     // 8. router: dlogit (bf16 [T][E_pad]) and the bias gradient
     const unsigned nblk = (unsigned)((T + kRowWarps - 1) / kRowWarps);
     if (launch(route_bwd_kernel, dim3(nblk), dim3(kRowThreads), 0, s, 1u, static_cast<const float*>(probs),
                static_cast<const int32_t*>(ids), static_cast<const float*>(wts), static_cast<const int32_t*>(inv),
-               static_cast<const float*>(dwp), L.n_tiles_f, R, T, iE, ik, renorm ? 1 : 0,
+               static_cast<const float*>(dwp), 2 * L.n_tiles_f, R, T, iE, ik, renorm ? 1 : 0,
                reinterpret_cast<__nv_bfloat16*>(dlogit), dbias ? db_part : nullptr, (int)L.e_pad))
         return MOE_ERR_CUDA;
-    if (dbias && launch(colsum_kernel, dim3((unsigned)((E + kRowThreads - 1) / kRowThreads)), dim3(kRowThreads), 0, s,
-                        1u, static_cast<const float*>(db_part), (int)nblk, iE, dbias))
+    if (dbias && launch(colsum_kernel, dim3((unsigned)E), dim3(kRowThreads), 0, s, 1u,
+                        static_cast<const float*>(db_part), (int)nblk, iE, dbias))
         return MOE_ERR_CUDA;
     // 9. dW_router = x^T . dlogit (one group of T rows)
     {
-        CUtensorMap ta, tb;
+        CUtensorMap ta, tb, to0;
         rc = make_weight_chunk_map(&ta, x, (uint64_t)d, (uint64_t)T);
         rc = rc ? rc : make_weight_chunk_map(&tb, dlogit, (uint64_t)L.e_pad, (uint64_t)T);
+        rc = rc ? rc : make_out3_map(&to0, dw_router, (uint64_t)E, (uint64_t)d, 1);
         if (rc) return rc;
         Params p = bwd_params();
         p.offsets = nullptr;
@@ -1048,7 +1071,7 @@ int backward_impl(const moe_bf16* x, const moe_bf16* w_router, const float* bias
         p.m_total = (int)d;
         p.m_tiles = (int)((d + kPairRows - 1) / kPairRows);
         p.split_b = 0;
-        if (launch_pair_bwd<kDW>(*st, p.m_tiles * p.n_tiles, ta, ta, tb, tb, p, s)) return MOE_ERR_CUDA;
+        if (launch_pair_bwd<kDW>(*st, p.m_tiles * p.n_tiles, ta, ta, tb, tb, p, s, &to0, &to0)) return MOE_ERR_CUDA;
     }
     // 10. dx_router = dlogit . W_router^T (fp32)
     {
