@@ -73,14 +73,24 @@ def _inputs():
     return cfg, make_inputs(cfg)
 
 
-def _worker(rank, world, port, q):
+def _token_ranges(T, world, uneven):
+    """Each rank's token slice: equal shares, or uneven ones (rank r gets
+    r + 1 parts) so that ranks send and receive different row counts."""
+    w = [r + 1 for r in range(world)] if uneven else [1] * world
+    cuts = [0]
+    for r in range(world):
+        cuts.append(cuts[-1] + T * w[r] // sum(w) if r < world - 1 else T)
+    return [(cuts[r], cuts[r + 1]) for r in range(world)]
+
+
+def _worker(rank, world, port, q, uneven=False):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=rank, world_size=world)
     from oracle.oracle import default_oracle
     cfg, inp = _inputs()
     e0, e1 = owner_block(cfg.E, world, rank)
-    T_r = cfg.T // world
-    x = inp.x[rank * T_r:(rank + 1) * T_r].contiguous()
+    t0, t1 = _token_ranges(cfg.T, world, uneven)[rank]
+    x = inp.x[t0:t1].contiguous()
     blk = ExpertParallelMoE(inp.W_router, inp.W_gate[e0:e1].contiguous(), inp.W_up[e0:e1].contiguous(),
                             inp.W_down[e0:e1].contiguous(), cfg.k, bias=inp.bias,
                             stages=CpuStages(default_oracle(), cfg.E))
@@ -89,6 +99,45 @@ def _worker(rank, world, port, q):
     dist.barrier()
     dist.destroy_process_group()
     q.put((rank, out, plan.recv_counts, plan.offsets))
+
+
+def _run_ranks(world, port, uneven):
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_worker, args=(r, world, port, q, uneven)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = sorted((q.get(timeout=150) for _ in range(world)), key=lambda r: r[0])
+    for p in procs:
+        p.join(timeout=30)
+        assert p.exitcode == 0
+    return res
+
+
+def _single_process_reference():
+    from oracle.oracle import default_oracle
+    cfg, inp = _inputs()
+    st = CpuStages(default_oracle(), cfg.E)
+    ids, w = st.route(inp.x, inp.W_router, cfg.k, inp.bias)
+    pm = st.permute(inp.x, ids, w, cfg.E)
+    y = st.expert_ffn(pm["x_perm"], pm["w_perm"], pm["offsets"], inp.W_gate, inp.W_up, inp.W_down)
+    return cfg, ids.numpy(), st.combine(y, pm["inv"], cfg.T, cfg.k).numpy()
+
+
+@pytest.mark.timeout(240)
+def test_four_ranks_uneven_tokens_match_single_process():
+    """Four ranks (two experts each) with uneven token shares: different
+    send and receive counts on every rank; the outputs still equal the
+    single-process forward, rank by rank."""
+    world = 4
+    res = _run_ranks(world, 29541, uneven=True)
+    cfg, ids, ref = _single_process_reference()
+    counts = np.bincount(ids.ravel(), minlength=cfg.E)
+    for (rank, out, recv_counts, offsets), (t0, t1) in zip(res, _token_ranges(cfg.T, world, True)):
+        np.testing.assert_allclose(out, ref[t0:t1], rtol=1e-12, atol=1e-14)
+        e0, e1 = owner_block(cfg.E, world, rank)
+        assert recv_counts.shape == (world, e1 - e0)
+        assert recv_counts.sum(axis=0).tolist() == counts[e0:e1].tolist()
 
 
 @pytest.mark.timeout(180)

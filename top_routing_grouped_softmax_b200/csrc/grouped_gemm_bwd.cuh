@@ -11,7 +11,7 @@
 //
 // Four kinds share one pipeline (the CTA-pair ring of the forward's grouped
 // GEMM: TMA producer, one MMA thread in the even CTA issuing M=256 N=256 K=16
-// pair MMAs, four epilogue warps per CTA over a double-buffered accumulator):
+// pair MMAs, eight epilogue warps per CTA over a double-buffered accumulator):
 //
 //   kGU  g, u = x_perm . W_gate[e], x_perm . W_up[e]      (recompute)
 //        A = x_perm rows (K-major), B = weight columns (MN-major): the even
@@ -27,14 +27,16 @@
 //        [f][d], its rows are the output columns).  Stores dg, du and
 //        hw = w h (the operand of the W_down gradient) as bf16.
 //   kDX  out = A1 . B1^T + A2 . B2^T with K split in two halves (the first
-//        k_split 64-blocks read A1/B1, the rest A2/B2), fp32 store:
+//        k_split 64-blocks read A1/B1, the rest A2/B2), fp32 out:
 //        dx_perm = dg . W_gate[e]^T + du . W_up[e]^T, and (one group, one half)
-//        the router's dx = dlogit . W_router^T.
+//        the router's dx = dlogit . W_router^T.  Whole 32-row slabs go out by
+//        TMA store; a slab that crosses the group's end is stored row by row.
 //   kDW  out[e] = A_e^T . B_e, reduced over the rows of group e:
 //        A = the group's rows read MN-major (x_perm or hw, or x), B likewise
 //        (dg | du split over the pair, or dout_perm / dlogit).  One work item
 //        is (expert, 256-row M tile, 256-column N tile); an empty group writes
-//        zeros.  fp32 store.
+//        zeros.  fp32 out by 3-D TMA store ([E][rows][cols] views clip the
+//        partial tiles).
 //
 // No TMA load uses multicast.  Every wait is bounded (see ptx.cuh).
 #pragma once
@@ -104,12 +106,12 @@ struct alignas(8) Ctrl {
     int tp[kMaxE + 1];
 };
 
-// Ring depth per kind: kDW gives two stages to the staging slabs of its
-// TMA-store epilogue (eight warps x two 32 x 32 fp32 slabs).
+// Ring depth per kind: kDW and kDX give two stages to the staging slabs of
+// their TMA-store epilogues (eight warps x two 32 x 32 fp32 slabs).
 constexpr int kSlabBytes = 32 * 32 * 4;
 constexpr int kStoreBytes = kEpiWarps * 2 * kSlabBytes;
-__host__ __device__ constexpr int stages_for(int kind) { return kind == kDW ? 4 : kPairStages; }
-__host__ __device__ constexpr int store_bytes_for(int kind) { return kind == kDW ? kStoreBytes : 0; }
+__host__ __device__ constexpr int stages_for(int kind) { return (kind == kDW || kind == kDX) ? 4 : kPairStages; }
+__host__ __device__ constexpr int store_bytes_for(int kind) { return (kind == kDW || kind == kDX) ? kStoreBytes : 0; }
 
 template <int KIND>
 __host__ inline size_t smem_bytes()
@@ -183,10 +185,11 @@ __device__ __forceinline__ void store_zero_f32x16(float* dst)
 // row q*32 + lane of this CTA's 128 rows.  tbase addresses the accumulator
 // at this warp's lane quarter.
 // `half` selects the columns this warp drains: half of the tile's output
-// columns (kGU: 64 of 128; the others: 128 of 256).  kDW stages its output
-// in `slab` (two 4 KB buffers of this warp, alternated by slab_buf) and
-// stores it with TMA through tm_o0 / tm_o1 ([E][m_total][n_out] fp32 views;
-// rows past m_total and columns past n_out are not written).
+// columns (kGU: 64 of 128; the others: 128 of 256).  kDW and kDX stage their
+// output in `slab` (two 4 KB buffers of this warp, alternated by slab_buf)
+// and store it with TMA: kDW through tm_o0 / tm_o1 ([E][m_total][n_out]
+// fp32 views; rows past m_total and columns past n_out are not written),
+// kDX through tm_o0 ([1][rows][n_out]).
 template <int KIND>
 __device__ __forceinline__ void epilogue(const Params& p, const Item& it, uint32_t tbase, uint32_t rank, int q,
                                          int lane, int half, const CUtensorMap* tm_o0, const CUtensorMap* tm_o1,
@@ -289,16 +292,46 @@ __device__ __forceinline__ void epilogue(const Params& p, const Item& it, uint32
         }
         if (valid) p.dwp[(int64_t)row * (2 * p.n_tiles) + 2 * it.nt + half] = dot;
     } else if constexpr (KIND == kDX) {
+        // 32 x 32 fp32 slabs written by TMA when all 32 rows of this warp
+        // belong to the group (the rows past a group's end belong to the next
+        // group and are left alone); a warp with a partial slab stores its
+        // valid rows itself
         const int row = it.row0 + r;
         const bool valid = row < it.row_end;
         const int c_base = it.nt * kBN;
         const int ncols = min(kBN, p.n_out - c_base);
+        const int wrow0 = it.row0 + (int)rank * kBM + q * 32;
+        const bool whole = wrow0 + 31 < it.row_end;  // warp-uniform
 #pragma unroll 1
-        for (int c0 = half * 128; c0 < half * 128 + 128; c0 += 16) {
-            uint32_t acc[16];
-            tmem_ld16(tbase + c0, acc);
+        for (int c0 = half * 128; c0 < half * 128 + 128; c0 += 32) {
+            uint32_t lo[16], hi[16];
+            tmem_ld16(tbase + c0, lo);
+            tmem_ld16(tbase + c0 + 16, hi);
             tmem_ld_wait();
-            if (valid && c0 < ncols) store_f32x16(p.out0 + (int64_t)row * p.ld_out + c_base + c0, acc);
+            if (c0 >= ncols) continue;  // warp-uniform (n_out % 64 == 0)
+            if (whole) {
+                uint32_t* buf = reinterpret_cast<uint32_t*>(slab) + slab_buf * (kSlabBytes / 4);
+                if (lane == 0) bulk_wait_group_read<1>();
+                __syncwarp();
+                uint4* rowp = reinterpret_cast<uint4*>(buf + lane * 32);
+                const int sw = lane & 7;
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                    rowp[v ^ sw] = make_uint4(lo[4 * v], lo[4 * v + 1], lo[4 * v + 2], lo[4 * v + 3]);
+                    rowp[(4 + v) ^ sw] = make_uint4(hi[4 * v], hi[4 * v + 1], hi[4 * v + 2], hi[4 * v + 3]);
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    tma_store_3d(tm_o0, buf, c_base + c0, wrow0, 0);
+                    bulk_commit_group();
+                }
+                slab_buf ^= 1;
+            } else if (valid) {
+                float* dst = p.out0 + (int64_t)row * p.ld_out + c_base + c0;
+                store_f32x16(dst, lo);
+                store_f32x16(dst + 16, hi);
+            }
         }
     } else {  // kDW: 32 x 32 fp32 slabs staged in shared memory, written by TMA
         const bool empty = it.num_kb == 0;
@@ -374,7 +407,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_prefetch_map(&tm_b0);
         if (KIND == kDX) tma_prefetch_map(&tm_a2);
         if (KIND == kGU || KIND == kDX || KIND == kDW) tma_prefetch_map(&tm_b1);
-        if (KIND == kDW) {
+        if (KIND == kDW || KIND == kDX) {
             tma_prefetch_map(&tm_o0);
             tma_prefetch_map(&tm_o1);
         }
@@ -534,7 +567,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 acc_ph ^= 1u;
             }
         }
-        if (KIND == kDW && lane == 0) bulk_wait_group_all();
+        if ((KIND == kDW || KIND == kDX) && lane == 0) bulk_wait_group_all();
         __syncwarp();
     }
 

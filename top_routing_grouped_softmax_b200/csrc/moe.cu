@@ -979,11 +979,12 @@ int backward_impl(const moe_bf16* x, const moe_bf16* w_router, const float* bias
     }
     // 5. dx_perm = dg . W_gate^T + du . W_up^T (fp32)
     {
-        CUtensorMap ta, ta2, tb0, tb1;
+        CUtensorMap ta, ta2, tb0, tb1, to0;
         rc = make_map(&ta, g, (uint64_t)f, (uint64_t)R, 64, kBM);
         rc = rc ? rc : make_map(&ta2, u, (uint64_t)f, (uint64_t)R, 64, kBM);
         rc = rc ? rc : make_map(&tb0, w_gate, (uint64_t)f, (uint64_t)(E * d), 64, kBM);
         rc = rc ? rc : make_map(&tb1, w_up, (uint64_t)f, (uint64_t)(E * d), 64, kBM);
+        rc = rc ? rc : make_out3_map(&to0, dx_perm, (uint64_t)d, (uint64_t)R, 1);
         if (rc) return rc;
         Params p = bwd_params();
         p.offsets = offsets;
@@ -996,7 +997,8 @@ int backward_impl(const moe_bf16* x, const moe_bf16* w_router, const float* bias
         p.n_out = (int)d;
         p.n_tiles = (int)((d + kBN - 1) / kBN);
         p.b_rows = (int)d;
-        if (launch_pair_bwd<kDX>(*st, max_mtiles * p.n_tiles, ta, ta2, tb0, tb1, p, s)) return MOE_ERR_CUDA;
+        if (launch_pair_bwd<kDX>(*st, max_mtiles * p.n_tiles, ta, ta2, tb0, tb1, p, s, &to0, &to0))
+            return MOE_ERR_CUDA;
     }
     // 6. dW_gate[e], dW_up[e] = x_perm_e^T . dg_e, x_perm_e^T . du_e
     {
@@ -1075,9 +1077,10 @@ int backward_impl(const moe_bf16* x, const moe_bf16* w_router, const float* bias
     }
     // 10. dx_router = dlogit . W_router^T (fp32)
     {
-        CUtensorMap ta, tb;
+        CUtensorMap ta, tb, to0;
         rc = make_map(&ta, dlogit, (uint64_t)L.e_pad, (uint64_t)T, 64, kBM);
         rc = rc ? rc : make_map(&tb, w_router, (uint64_t)E, (uint64_t)d, 64, kBM);
+        rc = rc ? rc : make_out3_map(&to0, dx_router, (uint64_t)d, (uint64_t)T, 1);
         if (rc) return rc;
         Params p = bwd_params();
         p.offsets = nullptr;
@@ -1090,7 +1093,8 @@ int backward_impl(const moe_bf16* x, const moe_bf16* w_router, const float* bias
         p.n_out = (int)d;
         p.n_tiles = (int)((d + kBN - 1) / kBN);
         p.b_rows = 0;
-        if (launch_pair_bwd<kDX>(*st, ((T + kPairRows - 1) / kPairRows) * p.n_tiles, ta, ta, tb, tb, p, s))
+        if (launch_pair_bwd<kDX>(*st, ((T + kPairRows - 1) / kPairRows) * p.n_tiles, ta, ta, tb, tb, p, s, &to0,
+                                 &to0))
             return MOE_ERR_CUDA;
     }
     // 11. dx = dx_router + sum over slots of dx_perm (fp32)
