@@ -12,8 +12,10 @@ the library records events only around the gate/up GEMM (the roofline
 kernel), because a recorded event stops the next kernel from launching
 early.  A second pass of the same steps records every stage boundary for
 the stage breakdown.  `e2e` repeats the measurement through the public API
-with the token batch copied host->device from pinned memory and the output
-copied back inside the timed region.  SM clocks and throttle reasons are
+with each step's token batch copied host->device from pinned memory and its
+output copied back inside the timed region; consecutive steps overlap their
+copies with the neighbouring step's compute on separate streams, as a
+serving loop would.  SM clocks and throttle reasons are
 sampled through NVML during the timed region.
 
 Multi-GPU: one process per GPU (torchrun); every rank runs its own replica
@@ -407,27 +409,61 @@ def run_gpu(args, cfg):
     tiles = int(((gemm_counts + 255) // 256).sum())
     padding = 1.0 - int(gemm_counts.sum()) / max(1, tiles * 256)
 
-    # ---- end to end through the public API, host buffers, copies timed
+    # ---- end to end through the public API, host buffers, copies timed.
+    # Consecutive batches are pipelined the way a serving loop runs them: the
+    # host->device copy of batch i+1 and the device->host copy of batch i-1
+    # run on their own streams while batch i computes (two device buffers of
+    # each).  Every step still copies its whole token batch in and its whole
+    # output back inside the timed region.
     x_host = inp.x.pin_memory()
-    out_host = torch.empty(cfg.T, cfg.d, dtype=torch.float32).pin_memory()
-    x_dev = torch.empty_like(x)
-    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    for _ in range(2):
-        x_dev.copy_(x_host, non_blocking=True)
-        fwd(x_dev)
-        out_host.copy_(out, non_blocking=True)
+    pipelined = args.path == "fused" and not (args.round or args.shared or args.gather)
+    nbuf = 2 if pipelined else 1
+    out_host = [torch.empty(cfg.T, cfg.d, dtype=torch.float32).pin_memory() for _ in range(nbuf)]
+    x_dev = [torch.empty_like(x) for _ in range(nbuf)]
+    out_dev = [out] + [torch.empty_like(out) for _ in range(nbuf - 1)]
+    s_in = torch.cuda.Stream(dev) if pipelined else stream
+    s_out = torch.cuda.Stream(dev) if pipelined else stream
+
+    def e2e_run(n_steps, t0=None, t1=None):
+        in_done = [torch.cuda.Event() for _ in range(nbuf)]
+        comp_done = [torch.cuda.Event() for _ in range(nbuf)]
+        out_done = [torch.cuda.Event() for _ in range(nbuf)]
+        if t0 is not None:
+            t0.record(stream)
+            s_in.wait_event(t0)
+        for i in range(n_steps):
+            b = i % nbuf
+            if i >= nbuf:
+                s_in.wait_event(comp_done[b])        # x_dev[b] no longer read
+            with torch.cuda.stream(s_in):
+                x_dev[b].copy_(x_host, non_blocking=True)
+                in_done[b].record(s_in)
+            stream.wait_event(in_done[b])
+            if i >= nbuf:
+                stream.wait_event(out_done[b])       # out_dev[b] copied out
+            flush.zero_()
+            if pipelined:
+                blk(x_dev[b], out=out_dev[b])
+            else:
+                fwd(x_dev[b])
+            comp_done[b].record(stream)
+            s_out.wait_event(comp_done[b])
+            with torch.cuda.stream(s_out):
+                out_host[b].copy_(out_dev[b], non_blocking=True)
+                out_done[b].record(s_out)
+        stream.wait_stream(s_in)
+        stream.wait_stream(s_out)
+        if t1 is not None:
+            t1.record(stream)
+
+    e2e_run(2)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    for i in range(args.steps):
-        flush.zero_()
-        e2e_ev[i][0].record(stream)
-        x_dev.copy_(x_host, non_blocking=True)
-        fwd(x_dev)
-        out_host.copy_(out, non_blocking=True)
-        e2e_ev[i][1].record(stream)
+    e2e_t0, e2e_t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2e_run(args.steps, e2e_t0, e2e_t1)
     torch.cuda.synchronize()
-    e2e_s = sum(a.elapsed_time(b) for a, b in e2e_ev) / 1e3
+    e2e_s = e2e_t0.elapsed_time(e2e_t1) / 1e3
     if world > 1:
         dist.barrier()
 
@@ -503,7 +539,9 @@ def run_gpu(args, cfg):
             "experts": {"active": active, "max_count": int(counts.max()), "min_count": int(counts.min()),
                         "pair_tile_padding": padding},
             "e2e": {"value": whole_job_rate(cfg.T * args.steps, world, [e2e_s]), "unit": UNIT,
-                    "h2d_bytes_per_step": cfg.T * cfg.d * 2, "d2h_bytes_per_step": cfg.T * cfg.d * 4},
+                    "h2d_bytes_per_step": cfg.T * cfg.d * 2, "d2h_bytes_per_step": cfg.T * cfg.d * 4,
+                    "copies": ("pinned host buffers; batch i+1 in and batch i-1 out on their own streams while "
+                               "batch i computes" if pipelined else "pinned host buffers, in order on one stream")},
             "gpu_launches": (KERNELS_PER_FORWARD + 2 * args.shared + (3 if args.round else 0)) * args.steps,
             "clocks": clocks,
             "wall_s_timed_region": wall,
