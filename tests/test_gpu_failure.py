@@ -49,3 +49,22 @@ def test_y_outside_fp16_range_is_reported():
     torch.cuda.synchronize()
     assert moe.get_status() == moe.MOE_OK
     assert torch.isfinite(out).all().item()
+
+
+def test_tiny_wait_limit_is_raised_to_one_millisecond():
+    """A limit below 1 ms is raised to 1 ms: with a 1 ns limit taken as is,
+    nearly every pipeline wait would give up; raised, a small forward and
+    backward finish cleanly (their waits last microseconds)."""
+    cfg = gc.small_cfg(256, 128, 8, 2, 128)
+    d = gc.on_device(gc.inputs(cfg))
+    assert moe.get_status() == moe.MOE_OK
+    moe.set_wait_limit_ns(1)
+    try:
+        out = moe.forward(d["x"], d["w_router"], d["w_gate"], d["w_up"], d["w_down"], 2)
+        dout = torch.ones(cfg.T, cfg.d, dtype=torch.float32, device="cuda")
+        moe.backward(d["x"], d["w_router"], d["w_gate"], d["w_up"], d["w_down"], 2, dout)
+        torch.cuda.synchronize()
+        assert moe.get_status() == moe.MOE_OK
+        assert torch.isfinite(out).all().item()
+    finally:
+        moe.set_wait_limit_ns(0)
