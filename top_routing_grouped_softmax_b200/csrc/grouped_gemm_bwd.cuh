@@ -230,10 +230,10 @@ __device__ __forceinline__ void epilogue(const Params& p, const Item& it, uint32
         const float w = valid ? __ldg(p.w_perm + row) : 0.0f;
         const int64_t row_off = (int64_t)row * p.ld_f + c_base;
         float dot = 0.0f;
-        // g and u of the next 16 columns are in flight while this chunk is
-        // processed (the loads are row-strided across the warp and would
-        // otherwise expose their latency once per chunk)
-        uint4 gq[2][2], uq[2][2];
+        // g and u of the next two 16-column chunks are in flight while this
+        // chunk is processed (the loads are row-strided across the warp and
+        // would otherwise expose their latency once per chunk)
+        uint4 gq[3][2], uq[3][2];
         auto fetch = [&](int c0, int b) {
             if (valid && c0 < ncols) {
                 const uint4* gp = reinterpret_cast<const uint4*>(p.g + row_off + c0);
@@ -245,19 +245,20 @@ __device__ __forceinline__ void epilogue(const Params& p, const Item& it, uint32
             }
         };
         fetch(half * 128, 0);
+        fetch(half * 128 + 16, 1);
 #pragma unroll
         for (int ci = 0; ci < 8; ++ci) {
             const int c0 = half * 128 + ci * 16;
-            if (ci + 1 < 8) fetch(c0 + 16, (ci + 1) & 1);
+            if (ci + 2 < 8) fetch(c0 + 32, (ci + 2) % 3);
             uint32_t acc[16];
             tmem_ld16(tbase + c0, acc);
             tmem_ld_wait();
             if (valid && c0 < ncols) {
                 float g[16], u[16];
-                unpack_bf16x8(gq[ci & 1][0], *reinterpret_cast<float(*)[8]>(&g[0]));
-                unpack_bf16x8(gq[ci & 1][1], *reinterpret_cast<float(*)[8]>(&g[8]));
-                unpack_bf16x8(uq[ci & 1][0], *reinterpret_cast<float(*)[8]>(&u[0]));
-                unpack_bf16x8(uq[ci & 1][1], *reinterpret_cast<float(*)[8]>(&u[8]));
+                unpack_bf16x8(gq[ci % 3][0], *reinterpret_cast<float(*)[8]>(&g[0]));
+                unpack_bf16x8(gq[ci % 3][1], *reinterpret_cast<float(*)[8]>(&g[8]));
+                unpack_bf16x8(uq[ci % 3][0], *reinterpret_cast<float(*)[8]>(&u[0]));
+                unpack_bf16x8(uq[ci % 3][1], *reinterpret_cast<float(*)[8]>(&u[8]));
                 uint32_t pdg[8], pdu[8], phw[8];
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
