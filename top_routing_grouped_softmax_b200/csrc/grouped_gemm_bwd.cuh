@@ -246,13 +246,18 @@ __device__ __forceinline__ void epilogue(const Params& p, const Item& it, uint32
         };
         fetch(half * 128, 0);
         fetch(half * 128 + 16, 1);
+        // the accumulator of the next chunk is read from TMEM while this one
+        // is processed (tcgen05.wait::ld waits for all of a thread's loads,
+        // so the wait comes after the math)
+        uint32_t accb[2][16];
+        tmem_ld16(tbase + half * 128, accb[0]);
+        tmem_ld_wait();
 #pragma unroll
         for (int ci = 0; ci < 8; ++ci) {
             const int c0 = half * 128 + ci * 16;
             if (ci + 2 < 8) fetch(c0 + 32, (ci + 2) % 3);
-            uint32_t acc[16];
-            tmem_ld16(tbase + c0, acc);
-            tmem_ld_wait();
+            if (ci + 1 < 8) tmem_ld16(tbase + c0 + 16, accb[(ci + 1) & 1]);
+            const uint32_t* acc = accb[ci & 1];
             if (valid && c0 < ncols) {
                 float g[16], u[16];
                 unpack_bf16x8(gq[ci % 3][0], *reinterpret_cast<float(*)[8]>(&g[0]));
@@ -290,6 +295,7 @@ __device__ __forceinline__ void epilogue(const Params& p, const Item& it, uint32
                 hwp[0] = make_uint4(phw[0], phw[1], phw[2], phw[3]);
                 hwp[1] = make_uint4(phw[4], phw[5], phw[6], phw[7]);
             }
+            tmem_ld_wait();
         }
         if (valid) p.dwp[(int64_t)row * (2 * p.n_tiles) + 2 * it.nt + half] = dot;
     } else if constexpr (KIND == kDX) {
@@ -303,14 +309,20 @@ __device__ __forceinline__ void epilogue(const Params& p, const Item& it, uint32
         const int ncols = min(kBN, p.n_out - c_base);
         const int wrow0 = it.row0 + (int)rank * kBM + q * 32;
         const bool whole = wrow0 + 31 < it.row_end;  // warp-uniform
-#pragma unroll 1
-        for (int c0 = half * 128; c0 < half * 128 + 128; c0 += 32) {
-            uint32_t lo[16], hi[16];
-            tmem_ld16(tbase + c0, lo);
-            tmem_ld16(tbase + c0 + 16, hi);
-            tmem_ld_wait();
-            if (c0 >= ncols) continue;  // warp-uniform (n_out % 64 == 0)
-            if (whole) {
+        uint32_t lob[2][16], hib[2][16];  // this slab and the next one in flight
+        tmem_ld16(tbase + half * 128, lob[0]);
+        tmem_ld16(tbase + half * 128 + 16, hib[0]);
+        tmem_ld_wait();
+#pragma unroll
+        for (int si = 0; si < 4; ++si) {
+            const int c0 = half * 128 + si * 32;
+            if (si + 1 < 4) {
+                tmem_ld16(tbase + c0 + 32, lob[(si + 1) & 1]);
+                tmem_ld16(tbase + c0 + 48, hib[(si + 1) & 1]);
+            }
+            const uint32_t(&lo)[16] = lob[si & 1];
+            const uint32_t(&hi)[16] = hib[si & 1];
+            if (c0 < ncols && whole) {  // c0 < ncols is warp-uniform (n_out % 64 == 0)
                 uint32_t* buf = reinterpret_cast<uint32_t*>(slab) + slab_buf * (kSlabBytes / 4);
                 if (lane == 0) bulk_wait_group_read<1>();
                 __syncwarp();
@@ -328,21 +340,29 @@ __device__ __forceinline__ void epilogue(const Params& p, const Item& it, uint32
                     bulk_commit_group();
                 }
                 slab_buf ^= 1;
-            } else if (valid) {
+            } else if (c0 < ncols && valid) {
                 float* dst = p.out0 + (int64_t)row * p.ld_out + c_base + c0;
                 store_f32x16(dst, lo);
                 store_f32x16(dst + 16, hi);
             }
+            tmem_ld_wait();
         }
     } else {  // kDW: 32 x 32 fp32 slabs staged in shared memory, written by TMA
         const bool empty = it.num_kb == 0;
         const int m0 = it.mt * kPairRows + (int)rank * kBM + q * 32;  // first row of this warp's slabs
-#pragma unroll 1
-        for (int c0 = half * 128; c0 < half * 128 + 128; c0 += 32) {
-            uint32_t lo[16], hi[16];
-            tmem_ld16(tbase + c0, lo);
-            tmem_ld16(tbase + c0 + 16, hi);
-            tmem_ld_wait();
+        uint32_t lob[2][16], hib[2][16];  // this slab and the next one in flight
+        tmem_ld16(tbase + half * 128, lob[0]);
+        tmem_ld16(tbase + half * 128 + 16, hib[0]);
+        tmem_ld_wait();
+#pragma unroll
+        for (int si = 0; si < 4; ++si) {
+            const int c0 = half * 128 + si * 32;
+            if (si + 1 < 4) {
+                tmem_ld16(tbase + c0 + 32, lob[(si + 1) & 1]);
+                tmem_ld16(tbase + c0 + 48, hib[(si + 1) & 1]);
+            }
+            const uint32_t(&lo)[16] = lob[si & 1];
+            const uint32_t(&hi)[16] = hib[si & 1];
             uint32_t* buf = reinterpret_cast<uint32_t*>(slab) + slab_buf * (kSlabBytes / 4);
             if (lane == 0) bulk_wait_group_read<1>();  // the store that last read `buf` is done
             __syncwarp();
@@ -365,6 +385,7 @@ __device__ __forceinline__ void epilogue(const Params& p, const Item& it, uint32
                 bulk_commit_group();
             }
             slab_buf ^= 1;
+            tmem_ld_wait();
         }
     }
 }
