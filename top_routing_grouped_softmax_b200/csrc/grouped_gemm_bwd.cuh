@@ -108,9 +108,22 @@ struct alignas(8) Ctrl {
 
 // Ring depth per kind: kDW and kDX give two stages to the staging slabs of
 // their TMA-store epilogues (eight warps x two 32 x 32 fp32 slabs).
+// Tuning constants (overridable at build time for measurements): staging
+// slabs per epilogue warp and the ring depth of the TMA-store kinds.
+#ifndef MOE_BWD_SLAB_BUFS
+#define MOE_BWD_SLAB_BUFS 2
+#endif
+#ifndef MOE_BWD_STORE_STAGES
+#define MOE_BWD_STORE_STAGES 4
+#endif
+constexpr int kSlabBufs = MOE_BWD_SLAB_BUFS;
 constexpr int kSlabBytes = 32 * 32 * 4;
-constexpr int kStoreBytes = kEpiWarps * 2 * kSlabBytes;
-__host__ __device__ constexpr int stages_for(int kind) { return (kind == kDW || kind == kDX) ? 4 : kPairStages; }
+constexpr int kStoreBytes = kEpiWarps * kSlabBufs * kSlabBytes;
+static_assert(kSlabBufs == 1 || kSlabBufs == 2, "staging slabs per warp");
+__host__ __device__ constexpr int stages_for(int kind)
+{
+    return (kind == kDW || kind == kDX) ? MOE_BWD_STORE_STAGES : kPairStages;
+}
 __host__ __device__ constexpr int store_bytes_for(int kind) { return (kind == kDW || kind == kDX) ? kStoreBytes : 0; }
 
 template <int KIND>
@@ -186,7 +199,7 @@ __device__ __forceinline__ void store_zero_f32x16(float* dst)
 // at this warp's lane quarter.
 // `half` selects the columns this warp drains: half of the tile's output
 // columns (kGU: 64 of 128; the others: 128 of 256).  kDW and kDX stage their
-// output in `slab` (two 4 KB buffers of this warp, alternated by slab_buf)
+// output in `slab` (kSlabBufs 4 KB buffers of this warp, taken in turn)
 // and store it with TMA: kDW through tm_o0 / tm_o1 ([E][m_total][n_out]
 // fp32 views; rows past m_total and columns past n_out are not written),
 // kDX through tm_o0 ([1][rows][n_out]).
@@ -324,7 +337,7 @@ __device__ __forceinline__ void epilogue(const Params& p, const Item& it, uint32
             const uint32_t(&hi)[16] = hib[si & 1];
             if (c0 < ncols && whole) {  // c0 < ncols is warp-uniform (n_out % 64 == 0)
                 uint32_t* buf = reinterpret_cast<uint32_t*>(slab) + slab_buf * (kSlabBytes / 4);
-                if (lane == 0) bulk_wait_group_read<1>();
+                if (lane == 0) bulk_wait_group_read<kSlabBufs - 1>();
                 __syncwarp();
                 uint4* rowp = reinterpret_cast<uint4*>(buf + lane * 32);
                 const int sw = lane & 7;
@@ -339,7 +352,7 @@ __device__ __forceinline__ void epilogue(const Params& p, const Item& it, uint32
                     tma_store_3d(tm_o0, buf, c_base + c0, wrow0, 0);
                     bulk_commit_group();
                 }
-                slab_buf ^= 1;
+                slab_buf = (slab_buf + 1) % kSlabBufs;
             } else if (c0 < ncols && valid) {
                 float* dst = p.out0 + (int64_t)row * p.ld_out + c_base + c0;
                 store_f32x16(dst, lo);
@@ -364,7 +377,7 @@ __device__ __forceinline__ void epilogue(const Params& p, const Item& it, uint32
             const uint32_t(&lo)[16] = lob[si & 1];
             const uint32_t(&hi)[16] = hib[si & 1];
             uint32_t* buf = reinterpret_cast<uint32_t*>(slab) + slab_buf * (kSlabBytes / 4);
-            if (lane == 0) bulk_wait_group_read<1>();  // the store that last read `buf` is done
+            if (lane == 0) bulk_wait_group_read<kSlabBufs - 1>();  // the store that last read `buf` is done
             __syncwarp();
             // row `lane` of the slab: 8 x 16 B chunks, 128-byte swizzle
             uint4* rowp = reinterpret_cast<uint4*>(buf + lane * 32);
@@ -384,7 +397,7 @@ __device__ __forceinline__ void epilogue(const Params& p, const Item& it, uint32
                 tma_store_3d(second ? tm_o1 : tm_o0, buf, col, m0, it.e);
                 bulk_commit_group();
             }
-            slab_buf ^= 1;
+            slab_buf = (slab_buf + 1) % kSlabBufs;
             tmem_ld_wait();
         }
     }
@@ -565,7 +578,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ---------------------------------------------------- epilogue (both CTAs)
         const int q = warp & 3;                 // TMEM lane quarter
         const int half = (warp - 2) >> 2;       // column half: warps 2-5 and 6-9
-        float* slab = reinterpret_cast<float*>(stage_out + (warp - 2) * 2 * kSlabBytes);
+        float* slab = reinterpret_cast<float*>(stage_out + (warp - 2) * kSlabBufs * kSlabBytes);
         int slab_buf = 0;
         int acc = 0;
         uint32_t acc_ph = 0;
