@@ -16,7 +16,8 @@
 //   kGU  g, u = x_perm . W_gate[e], x_perm . W_up[e]      (recompute)
 //        A = x_perm rows (K-major), B = weight columns (MN-major): the even
 //        CTA loads W_gate's 128 columns, the odd CTA the matching W_up ones,
-//        so accumulator columns 0..127 are g and 128..255 are u.  Stored bf16.
+//        so accumulator columns 0..127 are g and 128..255 are u.  Stores g, u
+//        and hw = w silu(g) u (the operand of the W_down gradient), bf16.
 //   kDH  dh = w . (dout_perm . W_down[e]^T), then the SwiGLU derivative:
 //          s = 1/(1+e^-g),  h = g s u,
 //          dg = dh u s (1 + g (1 - s)),  du = dh g s,
@@ -24,8 +25,8 @@
 //          dwp[row][2 nt + half] = sum over that half of the tile's columns of (dh / w) h
 //        (dh / w is the unweighted accumulator: dout . (h W_down) = (dout W_down^T) . h).
 //        A = dout_perm rows (K-major), B = W_down[e] rows (K-major: W_down[e] is
-//        [f][d], its rows are the output columns).  Stores dg, du and
-//        hw = w h (the operand of the W_down gradient) as bf16.
+//        [f][d], its rows are the output columns).  Stores dg and du as bf16
+//        (in place of g and u).
 //   kDX  out = A1 . B1^T + A2 . B2^T with K split in two halves (the first
 //        k_split 64-blocks read A1/B1, the rest A2/B2), fp32 out:
 //        dx_perm = dg . W_gate[e]^T + du . W_up[e]^T, and (one group, one half)
@@ -69,12 +70,12 @@ constexpr int kThreads = 64 + kEpiWarps * 32;
 
 struct Params {
     const int32_t* offsets;  // [E+1] group starts; nullptr: one group of M rows
-    const float* w_perm;     // kDH: routing weight of each grouped row
+    const float* w_perm;     // kGU, kDH: routing weight of each grouped row
     const __nv_bfloat16* g;  // kDH: recomputed g, u [rows][ld_f]
     const __nv_bfloat16* u;
     __nv_bfloat16* out_g;    // kGU: g;  kDH: dg        [rows][ld_f]
     __nv_bfloat16* out_u;    // kGU: u;  kDH: du
-    __nv_bfloat16* out_hw;   // kDH: w * h
+    __nv_bfloat16* out_hw;   // kGU: w * h
     float* dwp;              // kDH: [rows][2 * n_tiles] partial dot products (two column halves per tile)
     float* out0;             // kDX: [rows][ld_out];  kDW: [E][m_total][ld_out] (gate part when split)
     float* out1;             // kDW split: the up part
@@ -213,10 +214,13 @@ __device__ __forceinline__ void epilogue(const Params& p, const Item& it, uint32
 {
     const int r = (int)rank * kBM + q * 32 + lane;  // row of the 256-row pair tile
     if constexpr (KIND == kGU) {
+        // g and u (bf16, for the dh epilogue) and w h = w silu(g) u (bf16,
+        // the A operand of the W_down gradient) from the fp32 accumulators
         const int row = it.row0 + r;
         const bool valid = row < it.row_end;
         const int c_base = it.nt * 128;
         const int ncols = min(128, p.n_out - c_base);
+        const float w = valid ? __ldg(p.w_perm + row) : 0.0f;
 #pragma unroll 1
         for (int c0 = half * 64; c0 < half * 64 + 64; c0 += 16) {
             uint32_t g[16], u[16];
@@ -224,18 +228,25 @@ __device__ __forceinline__ void epilogue(const Params& p, const Item& it, uint32
             tmem_ld16(tbase + 128 + c0, u);
             tmem_ld_wait();
             if (valid && c0 < ncols) {
-                uint32_t pg[8], pu[8];
+                uint32_t pg[8], pu[8], ph[8];
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
-                    pg[i] = gemm::pack_bf16x2(__uint_as_float(g[2 * i]), __uint_as_float(g[2 * i + 1]));
-                    pu[i] = gemm::pack_bf16x2(__uint_as_float(u[2 * i]), __uint_as_float(u[2 * i + 1]));
+                    const float g0 = __uint_as_float(g[2 * i]), g1 = __uint_as_float(g[2 * i + 1]);
+                    const float u0 = __uint_as_float(u[2 * i]), u1 = __uint_as_float(u[2 * i + 1]);
+                    pg[i] = gemm::pack_bf16x2(g0, g1);
+                    pu[i] = gemm::pack_bf16x2(u0, u1);
+                    ph[i] = gemm::pack_bf16x2(w * (g0 * sigmoid(g0) * u0), w * (g1 * sigmoid(g1) * u1));
                 }
-                uint4* dg = reinterpret_cast<uint4*>(p.out_g + (int64_t)row * p.ld_f + c_base + c0);
-                uint4* du = reinterpret_cast<uint4*>(p.out_u + (int64_t)row * p.ld_f + c_base + c0);
+                const int64_t off = (int64_t)row * p.ld_f + c_base + c0;
+                uint4* dg = reinterpret_cast<uint4*>(p.out_g + off);
+                uint4* du = reinterpret_cast<uint4*>(p.out_u + off);
+                uint4* dh = reinterpret_cast<uint4*>(p.out_hw + off);
                 dg[0] = make_uint4(pg[0], pg[1], pg[2], pg[3]);
                 dg[1] = make_uint4(pg[4], pg[5], pg[6], pg[7]);
                 du[0] = make_uint4(pu[0], pu[1], pu[2], pu[3]);
                 du[1] = make_uint4(pu[4], pu[5], pu[6], pu[7]);
+                dh[0] = make_uint4(ph[0], ph[1], ph[2], ph[3]);
+                dh[1] = make_uint4(ph[4], ph[5], ph[6], ph[7]);
             }
         }
     } else if constexpr (KIND == kDH) {
@@ -280,36 +291,30 @@ __device__ __forceinline__ void epilogue(const Params& p, const Item& it, uint32
                 unpack_bf16x8(gq[ci % 3][1], *reinterpret_cast<float(*)[8]>(&g[8]));
                 unpack_bf16x8(uq[ci % 3][0], *reinterpret_cast<float(*)[8]>(&u[0]));
                 unpack_bf16x8(uq[ci % 3][1], *reinterpret_cast<float(*)[8]>(&u[8]));
-                uint32_t pdg[8], pdu[8], phw[8];
+                uint32_t pdg[8], pdu[8];
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
-                    float dgv[2], duv[2], hwv[2];
+                    float dgv[2], duv[2];
 #pragma unroll
                     for (int h2 = 0; h2 < 2; ++h2) {
                         const int c = 2 * i + h2;
                         const float dhu = __uint_as_float(acc[c]);  // dout . W_down^T (unweighted)
                         const float sg = sigmoid(g[c]);
                         const float gs = g[c] * sg;
-                        const float h = gs * u[c];
                         const float dh = w * dhu;
-                        dot += dhu * h;
+                        dot += dhu * (gs * u[c]);
                         dgv[h2] = dh * u[c] * sg * (1.0f + g[c] * (1.0f - sg));
                         duv[h2] = dh * gs;
-                        hwv[h2] = w * h;
                     }
                     pdg[i] = gemm::pack_bf16x2(dgv[0], dgv[1]);
                     pdu[i] = gemm::pack_bf16x2(duv[0], duv[1]);
-                    phw[i] = gemm::pack_bf16x2(hwv[0], hwv[1]);
                 }
                 uint4* dgp = reinterpret_cast<uint4*>(p.out_g + row_off + c0);
                 uint4* dup = reinterpret_cast<uint4*>(p.out_u + row_off + c0);
-                uint4* hwp = reinterpret_cast<uint4*>(p.out_hw + row_off + c0);
                 dgp[0] = make_uint4(pdg[0], pdg[1], pdg[2], pdg[3]);
                 dgp[1] = make_uint4(pdg[4], pdg[5], pdg[6], pdg[7]);
                 dup[0] = make_uint4(pdu[0], pdu[1], pdu[2], pdu[3]);
                 dup[1] = make_uint4(pdu[4], pdu[5], pdu[6], pdu[7]);
-                hwp[0] = make_uint4(phw[0], phw[1], phw[2], phw[3]);
-                hwp[1] = make_uint4(phw[4], phw[5], phw[6], phw[7]);
             }
             tmem_ld_wait();
         }

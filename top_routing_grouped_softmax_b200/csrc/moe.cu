@@ -933,7 +933,7 @@ int backward_impl(const moe_bf16* x, const moe_bf16* w_router, const float* bias
     using moe::gemm::kBM;
     using moe::gemm::kPairRows;
     const int64_t max_mtiles = (R + kPairRows - 1) / kPairRows + E;
-    // 3. recompute g, u = x_perm . [W_gate | W_up]
+    // 3. recompute g, u = x_perm . [W_gate | W_up], and w h for the W_down gradient
     {
         CUtensorMap ta, tg3, tu3;
         rc = make_map(&ta, x_perm, (uint64_t)d, (uint64_t)R, 64, kBM);
@@ -942,8 +942,10 @@ int backward_impl(const moe_bf16* x, const moe_bf16* w_router, const float* bias
         if (rc) return rc;
         Params p = bwd_params();
         p.offsets = offsets;
+        p.w_perm = w_perm;
         p.out_g = reinterpret_cast<__nv_bfloat16*>(g);
         p.out_u = reinterpret_cast<__nv_bfloat16*>(u);
+        p.out_hw = reinterpret_cast<__nv_bfloat16*>(hw);
         p.ld_f = f;
         p.E = iE;
         p.M = (int)R;
@@ -953,7 +955,7 @@ int backward_impl(const moe_bf16* x, const moe_bf16* w_router, const float* bias
         p.b_rows = (int)d;
         if (launch_pair_bwd<kGU>(*st, max_mtiles * p.n_tiles, ta, ta, tg3, tu3, p, s)) return MOE_ERR_CUDA;
     }
-    // 4. dh = w . dout_perm . W_down^T and the SwiGLU derivative: dg, du (in place of g, u), w h, partial dots
+    // 4. dh = w . dout_perm . W_down^T and the SwiGLU derivative: dg, du (in place of g, u), partial dots
     {
         CUtensorMap ta, tb;
         rc = make_map(&ta, dout_perm, (uint64_t)d, (uint64_t)R, 64, kBM);
@@ -966,7 +968,6 @@ int backward_impl(const moe_bf16* x, const moe_bf16* w_router, const float* bias
         p.u = reinterpret_cast<const __nv_bfloat16*>(u);
         p.out_g = reinterpret_cast<__nv_bfloat16*>(g);
         p.out_u = reinterpret_cast<__nv_bfloat16*>(u);
-        p.out_hw = reinterpret_cast<__nv_bfloat16*>(hw);
         p.dwp = dwp;
         p.ld_f = f;
         p.E = iE;
