@@ -29,7 +29,8 @@
 // (logit, expert); the group's maximum and the sum of exp(l - max) are
 // butterfly reductions in a fixed order.  k rounds of a butterfly arg-max
 // over the lanes' best candidates then pick the winners in order; the lane
-// that owned a winner marks it taken and rescans its experts.  For k > 8, a whole warp takes a
+// that owned a winner marks it taken and rescans its experts (from a
+// register copy when a lane has at most 16).  For k > 8, a whole warp takes a
 // token and picks the winners in k rounds of a butterfly arg-max.  Both
 // rank by the (value, index) order -- larger logit first, equal logits rank
 // the lower expert index first -- on fp32 logits (softmax is monotone).
@@ -199,8 +200,11 @@ __device__ __forceinline__ void warp_topk(int E, int k, bool renorm, int lane, L
 // a fixed order.  Then k rounds of a butterfly arg-max over the lanes' best
 // candidates pick the winners in (value, index) order; the lane that owned
 // a winner marks it taken (-inf in its slot) and rescans its experts for its
-// next best.  Lane j < k receives slot j.
-template <int L, typename Combine, typename Cell>
+// next best.  Lane j < k receives slot j.  With VPL > 0 (E <= L * VPL) the
+// rescans run over a register copy of the lane's logits, unrolled, instead
+// of the shared-memory cells; the passes before stay rolled loops, because
+// the epilogue runs once per CTA and unrolled code there is fetched cold.
+template <int L, int VPL, typename Combine, typename Cell>
 __device__ __forceinline__ void group_topk(int E, int k, bool renorm, int j, Combine combine, Cell cell, int& my_id,
                                            float& my_w, float* pcol, int64_t pstride)
 {
@@ -223,6 +227,13 @@ __device__ __forceinline__ void group_topk(int E, int k, bool renorm, int j, Com
     for (int o = L / 2; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
     if (pcol)  // every expert's probability, by the same formula as the weights below
         for (int c = j; c < E; c += L) pcol[c * pstride] = __expf(cell(c) - mx) / sum;
+    // VPL > 0: a register copy of the lane's logits (slots at or past E hold
+    // -inf, never a candidate) serves the rescans below
+    float v[VPL > 0 ? VPL : 1];
+    if constexpr (VPL > 0) {
+#pragma unroll
+        for (int m = 0; m < VPL; ++m) v[m] = j + L * m < E ? cell(j + L * m) : -INFINITY;
+    }
     float my_v = -INFINITY;
     my_id = 0;
     for (int slot = 0; slot < k; ++slot) {
@@ -244,14 +255,26 @@ __device__ __forceinline__ void group_topk(int E, int k, bool renorm, int j, Com
         // this lane owned the winner: take it, find the next best (a lane with
         // no candidate left -- NaN logits -- holds the sentinel, never an index)
         if (wc == bc && wc < E) {
-            cell(wc) = -INFINITY;
             bv = -INFINITY;
             bc = 0x7fffffff;
-            for (int c = j; c < E; c += L) {
-                const float l = cell(c);
-                if (l > bv) {
-                    bv = l;
-                    bc = c;
+            if constexpr (VPL > 0) {
+#pragma unroll
+                for (int m = 0; m < VPL; ++m) {
+                    const int c = j + L * m;
+                    if (c == wc) v[m] = -INFINITY;
+                    if (v[m] > bv) {
+                        bv = v[m];
+                        bc = c;
+                    }
+                }
+            } else {
+                cell(wc) = -INFINITY;
+                for (int c = j; c < E; c += L) {
+                    const float l = cell(c);
+                    if (l > bv) {
+                        bv = l;
+                        bc = c;
+                    }
                 }
             }
         }
@@ -267,8 +290,10 @@ __device__ __forceinline__ void group_topk(int E, int k, bool renorm, int j, Com
 }
 
 // One pass of softmax + top-k over the `own` buffered rows, L lanes per
-// token (32 / L tokens per warp).
-template <int L, int KMAX>
+// token (32 / L tokens per warp).  VPL > 0: the rescans of the top-k rounds
+// over VPL registers per lane (E <= L * VPL); VPL == 0: over the
+// shared-memory buffer cells (any E).
+template <int L, int KMAX, int VPL>
 __device__ __forceinline__ void topk_rows(const Params& p, float* buf, const float* s_bias, int* s_hist,
                                           int S, int own, int pitch, int tile0, int row0, bool ok, int warp,
                                           int lane)
@@ -281,16 +306,16 @@ __device__ __forceinline__ void topk_rows(const Params& p, float* buf, const flo
         const int64_t t = (int64_t)tile0 + row0 + i;
         int my_id;
         float my_w;
-        group_topk<L>(
-            E, p.k, p.renorm != 0, j,
-            [&](int c) {
-                const float* col = buf + (size_t)c * pitch + i;
-                float l = col[0];
-                for (int s = 1; s < S; ++s) l += col[(size_t)s * E * pitch];
-                return l + s_bias[c];
-            },
-            [&](int c) -> float& { return buf[(size_t)c * pitch + i]; }, my_id, my_w,
-            (p.probs && ok && t < p.T) ? p.probs + t * p.probs_tstride : nullptr, p.probs_estride);
+        const auto combine = [&](int c) {
+            const float* col = buf + (size_t)c * pitch + i;
+            float l = col[0];
+            for (int s = 1; s < S; ++s) l += col[(size_t)s * E * pitch];
+            return l + s_bias[c];
+        };
+        float* const pcol = (p.probs && ok && t < p.T) ? p.probs + t * p.probs_tstride : nullptr;
+        group_topk<L, VPL>(
+            E, p.k, p.renorm != 0, j, combine, [&](int c) -> float& { return buf[(size_t)c * pitch + i]; }, my_id,
+            my_w, pcol, p.probs_estride);
         if (ok && t < p.T && j < p.k) {
             p.ids[t * p.k + j] = my_id;
             p.wts[t * p.k + j] = my_w;
@@ -298,6 +323,28 @@ __device__ __forceinline__ void topk_rows(const Params& p, float* buf, const flo
                 atomicAdd(&s_hist[((row0 + i) / kTokensPerChunk) * E + my_id], 1);
         }
     }
+}
+
+// topk_rows with the smallest register count per lane that holds the
+// lane's ceil(E / L) experts (up to 16), else the shared-memory version.
+template <int L, int KMAX>
+__device__ __forceinline__ void topk_rows_any(const Params& p, float* buf, const float* s_bias, int* s_hist,
+                                              int S, int own, int pitch, int tile0, int row0, bool ok, int warp,
+                                              int lane)
+{
+    const int vpl = (p.E + L - 1) / L;
+    if (vpl <= 1)
+        topk_rows<L, KMAX, 1>(p, buf, s_bias, s_hist, S, own, pitch, tile0, row0, ok, warp, lane);
+    else if (vpl <= 2)
+        topk_rows<L, KMAX, 2>(p, buf, s_bias, s_hist, S, own, pitch, tile0, row0, ok, warp, lane);
+    else if (vpl <= 4)
+        topk_rows<L, KMAX, 4>(p, buf, s_bias, s_hist, S, own, pitch, tile0, row0, ok, warp, lane);
+    else if (vpl <= 8)
+        topk_rows<L, KMAX, 8>(p, buf, s_bias, s_hist, S, own, pitch, tile0, row0, ok, warp, lane);
+    else if (vpl <= 16)
+        topk_rows<L, KMAX, 16>(p, buf, s_bias, s_hist, S, own, pitch, tile0, row0, ok, warp, lane);
+    else
+        topk_rows<L, KMAX, 0>(p, buf, s_bias, s_hist, S, own, pitch, tile0, row0, ok, warp, lane);
 }
 
 template <int KMAX>
@@ -477,9 +524,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int row0 = S > 1 ? (int)r * own : pass * own;
         if constexpr (KMAX <= 8) {
             if (own == 128)
-                topk_rows<8, KMAX>(p, buf, s_bias, s_hist, S, own, pitch, tile0, row0, ok, warp, lane);
+                topk_rows_any<8, KMAX>(p, buf, s_bias, s_hist, S, own, pitch, tile0, row0, ok, warp, lane);
             else
-                topk_rows<16, KMAX>(p, buf, s_bias, s_hist, S, own, pitch, tile0, row0, ok, warp, lane);
+                topk_rows_any<16, KMAX>(p, buf, s_bias, s_hist, S, own, pitch, tile0, row0, ok, warp, lane);
         } else {
             for (int i = warp; i < own; i += kWarps) {
                 const int64_t t = (int64_t)tile0 + row0 + i;
