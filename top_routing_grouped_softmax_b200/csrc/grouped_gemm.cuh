@@ -32,9 +32,12 @@
 //                3x slower here: too many small TMA requests per stage.)
 //   warp 1       TMEM allocation + single-thread tcgen05.mma issuer,
 //                M=128 N=256 K=16 per instruction, fp32 accumulators
-//   warps 2..5   epilogue: tcgen05.ld of the 128 x 256 accumulator, one row
-//                per thread, fused math, stores.  (With 8 warps the two warps
-//                of a lane quarter split the columns; 4 measured faster.)
+//   warps 2..9   epilogue: tcgen05.ld of the 128 x 256 accumulator, one row
+//                per thread, fused math, stores; the two warps of a TMEM lane
+//                quarter split the columns.  (Eight warps against four: the
+//                same time where the MMA bounds the tile, and 7 % off the
+//                fine-grained layer, f = 256, whose short K leaves each tile's
+//                epilogue longer than its MMAs.)
 // Two accumulator buffers (2 x 256 TMEM columns) let the epilogue of one
 // tile overlap the MMAs of the next.
 //
@@ -67,11 +70,12 @@ constexpr int kBM = 128;
 constexpr int kBN = 256;
 constexpr int kBK = 64;
 constexpr int kMaxStages = 4;
-// Tuning constants (overridable at build time for measurements).  Measured
-// on the Qwen3-shaped layer: 4 epilogue warps beat 8, and 4 down-GEMM stages
-// beat 3 stages with double store buffers for 8 warps.
+// Tuning constants (overridable at build time for measurements).  The CTA
+// pair kernels (the default path) take 8 epilogue warps: even with 4 where
+// the MMA bounds the tile, 7 % faster on the fine-grained layer.  For the
+// single-CTA kernel, 4 down-GEMM stages beat 3 with more store staging.
 #ifndef MOE_GEMM_EPI_WARPS
-#define MOE_GEMM_EPI_WARPS 4
+#define MOE_GEMM_EPI_WARPS 8
 #endif
 #ifndef MOE_GEMM_DOWN_STAGES
 #define MOE_GEMM_DOWN_STAGES 4
@@ -88,7 +92,8 @@ constexpr uint32_t kTmemCols = 512;         // 2 accumulators x 256 columns
 constexpr int kMaxE = 512;
 constexpr int kSlabCols = 32;               // fp16 columns per TMA-store slab (64 B rows)
 constexpr int kSlabBytes = 32 * kSlabCols * 2;     // 32 rows x 32 fp16 = 2 KB
-constexpr int kStoreBytes = kEpiWarps * 2 * kSlabBytes;  // 2 buffers per epilogue warp
+constexpr int kSlabBufs = kEpiWarps == 8 ? 1 : 2;  // y staging slabs per epilogue warp
+constexpr int kStoreBytes = kEpiWarps * kSlabBufs * kSlabBytes;
 
 // Ring depth and store staging per epilogue: the down GEMM gives up one
 // stage to the staging buffers its TMA stores read from.
@@ -137,6 +142,12 @@ __host__ inline size_t smem_bytes()
 {
     return 1024 + (size_t)Stages<EPI>::value * kStageBytes + Stages<EPI>::store_bytes + sizeof(Ctrl);
 }
+static_assert(1024 + (size_t)Stages<kSwiGLU>::value * kStageBytes + Stages<kSwiGLU>::store_bytes + sizeof(Ctrl) <=
+                  227 * 1024,
+              "gate/up ring, staging and control exceed 227 KB of shared memory");
+static_assert(1024 + (size_t)Stages<kWeighted>::value * kStageBytes + Stages<kWeighted>::store_bytes + sizeof(Ctrl) <=
+                  227 * 1024,
+              "down ring, staging and control exceed 227 KB of shared memory");
 
 // Work item -> (expert, first row, group end, N tile), for M tiles of
 // TILE_ROWS rows: tp[e] is the exclusive prefix of M tiles per group.
@@ -242,7 +253,10 @@ __device__ __forceinline__ int gather_token(const Params& p, int r)
 // calling warp reads TMEM lane quarter q (rows q*32 .. +31 of the tile, row
 // row0 + r for thread r) and column group hf; rows at or past row_end are
 // not stored.  tbase addresses the accumulator at this warp's lane quarter.
-template <int EPI>
+// kWeighted stages y through NBUF slab buffers of this warp (slab, in turn
+// by slab_buf): a buffer is rewritten once the store that last read it is
+// done, so up to NBUF stores per warp are in flight.
+template <int EPI, int NBUF = 2>
 __device__ __forceinline__ void epilogue_tile(const Params& p, const CUtensorMap* tm_out, uint32_t tbase, int row0,
                                               int row_end, int nt, int q, int lane, int hf, float* slab,
                                               int& slab_buf)
@@ -317,7 +331,7 @@ __device__ __forceinline__ void epilogue_tile(const Params& p, const CUtensorMap
                 }
                 if (whole) {
                     uint32_t* buf = reinterpret_cast<uint32_t*>(slab) + slab_buf * (kSlabBytes / 4);
-                    if (lane == 0) bulk_wait_group_read<1>();  // the store that last read `buf` is done
+                    if (lane == 0) bulk_wait_group_read<NBUF - 1>();  // the store that last read `buf` is done
                     __syncwarp();
                     // row `lane` of the slab: 4 x 16 B chunks, 64-byte swizzle
                     uint4* rowp = reinterpret_cast<uint4*>(buf + lane * (kSlabCols / 2));
@@ -331,7 +345,7 @@ __device__ __forceinline__ void epilogue_tile(const Params& p, const CUtensorMap
                         tma_store_2d(tm_out, buf, nt * kBN + c0, wrow0);
                         bulk_commit_group();
                     }
-                    slab_buf ^= 1;
+                    slab_buf = slab_buf + 1 == NBUF ? 0 : slab_buf + 1;
                 } else if (valid) {
                     uint4* dst = reinterpret_cast<uint4*>(orow + c0);
 #pragma unroll
@@ -532,7 +546,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int ew = warp - 2;            // 0..7
         const int q = warp & 3;             // TMEM lane quarter
         const int hf = ew >> 2;             // column group (0 when kColGroups == 1)
-        float* slab = reinterpret_cast<float*>(stage_out + ew * 2 * kSlabBytes);
+        float* slab = reinterpret_cast<float*>(stage_out + ew * kSlabBufs * kSlabBytes);
         int slab_buf = 0;
         int acc = 0;
         uint32_t acc_ph = 0;
@@ -551,7 +565,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             tc_fence_after_sync();
             const uint32_t tbase = tmem + (uint32_t)(acc * kBN) + ((uint32_t)(q * 32) << 16);
-            epilogue_tile<EPI>(p, &tm_out, tbase, row0, row_end, nt, q, lane, hf, slab, slab_buf);
+            epilogue_tile<EPI, kSlabBufs>(p, &tm_out, tbase, row0, row_end, nt, q, lane, hf, slab, slab_buf);
             tc_fence_before_sync();
             mbar_arrive(&c.acc_empty[acc]);
             if (++acc == 2) {

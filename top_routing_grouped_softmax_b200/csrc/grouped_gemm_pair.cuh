@@ -18,7 +18,7 @@
 //                (the even CTA's producer expects the bytes of both halves)
 //   empty[s]     one per CTA; the MMA commit is multicast to both
 //   acc_full[b]  one per CTA; multicast commit
-//   acc_empty[b] lives in the even CTA; the four epilogue warps of each CTA
+//   acc_empty[b] lives in the even CTA; the epilogue warps of each CTA
 //                arrive on it (remotely, for the odd CTA)
 // The pair meets at a cluster barrier after set-up and before releasing TMEM.
 // No TMA load uses multicast.
@@ -33,6 +33,32 @@ constexpr int kPairRows = 256;                        // M rows per CTA pair
 constexpr int kPairBHalfBytes = 2 * kChunkBytes;      // 128 columns x 64 k
 constexpr int kPairStageBytes = kABytes + kPairBHalfBytes;  // 32 KB per CTA
 constexpr int kPairStages = 6;
+// Ring depth of the down-projection (kWeighted) kernel and y staging slabs
+// per epilogue warp: build-time tuning constants (the ring and the slabs
+// share the 227 KB of shared memory).  Six stages and one slab per warp for
+// eight epilogue warps measured the same as five stages with two or three
+// slabs on the fine-grained layer and 4 us faster on the Qwen3-shaped one.
+#ifndef MOE_PAIR_DOWN_STAGES
+#define MOE_PAIR_DOWN_STAGES 6
+#endif
+#ifndef MOE_PAIR_SLAB_BUFS
+#define MOE_PAIR_SLAB_BUFS 1
+#endif
+constexpr int kPairSlabBufs = MOE_PAIR_SLAB_BUFS;
+static_assert(MOE_PAIR_DOWN_STAGES >= 2 && MOE_PAIR_DOWN_STAGES <= kPairStages, "down ring depth");
+static_assert(kPairSlabBufs >= 1 && kPairSlabBufs <= 8, "slab buffers per epilogue warp");
+
+template <int EPI>
+__host__ __device__ constexpr int pair_stages()
+{
+    return EPI == kWeighted ? MOE_PAIR_DOWN_STAGES : kPairStages;
+}
+
+template <int EPI>
+__host__ __device__ constexpr int pair_store_bytes()
+{
+    return EPI == kWeighted ? kEpiWarps * kPairSlabBufs * kSlabBytes : 0;
+}
 
 struct alignas(8) PairCtrl {
     uint64_t full[kPairStages];
@@ -51,8 +77,13 @@ struct alignas(8) PairCtrl {
 template <int EPI>
 __host__ inline size_t pair_smem_bytes()
 {
-    return 1024 + (size_t)kPairStages * kPairStageBytes + Stages<EPI>::store_bytes + sizeof(PairCtrl);
+    return 1024 + (size_t)pair_stages<EPI>() * kPairStageBytes + pair_store_bytes<EPI>() + sizeof(PairCtrl);
 }
+static_assert(1024 + (size_t)pair_stages<kSwiGLU>() * kPairStageBytes + sizeof(PairCtrl) <= 227 * 1024,
+              "gate/up pair ring and control exceed 227 KB of shared memory");
+static_assert(1024 + (size_t)pair_stages<kWeighted>() * kPairStageBytes + pair_store_bytes<kWeighted>() +
+                      sizeof(PairCtrl) <= 227 * 1024,
+              "down pair ring, staging and control exceed 227 KB of shared memory");
 
 template <int EPI>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -62,8 +93,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t* stage_out = smem + (size_t)kPairStages * kPairStageBytes;
-    PairCtrl& c = *reinterpret_cast<PairCtrl*>(stage_out + Stages<EPI>::store_bytes);
+    constexpr int NS = pair_stages<EPI>();
+    uint8_t* stage_out = smem + (size_t)NS * kPairStageBytes;
+    PairCtrl& c = *reinterpret_cast<PairCtrl*>(stage_out + pair_store_bytes<EPI>());
 
     const int warp = threadIdx.x / 32;
     const int lane = threadIdx.x % 32;
@@ -75,7 +107,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int64_t npairs = num_clusters_x();
 
     if (threadIdx.x == 32) {
-        for (int s = 0; s < kPairStages; ++s) {
+        for (int s = 0; s < NS; ++s) {
             mbar_init(&c.full[s], 1);
             mbar_init(&c.empty[s], 1);
         }
@@ -141,7 +173,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tma_load_3d_pair(sb, &tm_b0, bar, 0, kr, nt * (kBN / 64) + (int)rank * 2);
                     }
                     ++issued;
-                    if (++s == kPairStages) {
+                    if (++s == NS) {
                         s = 0;
                         ph ^= 1u;
                     }
@@ -155,8 +187,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             // barriers count both CTAs' copies; the odd CTA instead waits until
             // the MMAs that read each of its stages released it (which they do
             // only after the stage's bytes arrived).
-            for (int q = 0; q < kPairStages; ++q) {
-                const int64_t cnt = issued / kPairStages + (q < issued % kPairStages ? 1 : 0);
+            for (int q = 0; q < NS; ++q) {
+                const int64_t cnt = issued / NS + (q < issued % NS ? 1 : 0);
                 if (cnt > 0)
                     mbar_wait(leader ? &c.full[q] : &c.empty[q], (uint32_t)(cnt - 1) & 1u, drain_limit(limit));
             }
@@ -193,7 +225,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         mma_bf16_ss_pair(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
                     }
                     mma_commit_pair_multicast(&c.empty[s], 0x3);  // frees the stage in both CTAs
-                    if (++s == kPairStages) {
+                    if (++s == NS) {
                         s = 0;
                         ph ^= 1u;
                     }
@@ -217,7 +249,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int ew = warp - 2;
         const int q = warp & 3;
         const int hf = ew >> 2;
-        float* slab = reinterpret_cast<float*>(stage_out + ew * 2 * kSlabBytes);
+        float* slab = reinterpret_cast<float*>(stage_out + ew * kPairSlabBufs * kSlabBytes);
         int slab_buf = 0;
         int acc = 0;
         uint32_t acc_ph = 0;
@@ -233,7 +265,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             tc_fence_after_sync();
             const uint32_t tbase = tmem + (uint32_t)(acc * kBN) + ((uint32_t)(q * 32) << 16);
-            epilogue_tile<EPI>(p, &tm_out, tbase, row0 + (int)rank * kBM, row_end, nt, q, lane, hf, slab, slab_buf);
+            epilogue_tile<EPI, kPairSlabBufs>(p, &tm_out, tbase, row0 + (int)rank * kBM, row_end, nt, q, lane, hf, slab,
+                                              slab_buf);
             tc_fence_before_sync();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(mapa_shared(&c.acc_empty[acc], 0));
