@@ -15,8 +15,10 @@ the stage breakdown.  `e2e` repeats the measurement through the public API
 with each step's token batch copied host->device from pinned memory and its
 output copied back inside the timed region; consecutive steps overlap their
 copies with the neighbouring step's compute on separate streams, as a
-serving loop would.  SM clocks and throttle reasons are
-sampled through NVML during the timed region.
+serving loop would.  `e2e_f16out` is the same loop with the block's fp16
+output option (MOE_FLAG_OUT_F16: the fp32 result rounded once, half the
+bytes read back); `value` and `e2e` keep the fp32 output.  SM clocks and
+throttle reasons are sampled through NVML during the timed region.
 
 Multi-GPU: one process per GPU (torchrun); every rank runs its own replica
 on its own batch (the block is independent per token, so the path shards by
@@ -423,8 +425,13 @@ def run_gpu(args, cfg):
     out_dev = [out] + [torch.empty_like(out) for _ in range(nbuf - 1)]
     s_in = torch.cuda.Stream(dev) if pipelined else stream
     s_out = torch.cuda.Stream(dev) if pipelined else stream
+    # the same loop with the block's fp16-output option (MOE_FLAG_OUT_F16):
+    # half the bytes read back
+    out_host16 = [torch.empty(cfg.T, cfg.d, dtype=torch.float16).pin_memory() for _ in range(nbuf)]
+    out_dev16 = [torch.empty(cfg.T, cfg.d, dtype=torch.float16, device=dev) for _ in range(nbuf)]
 
-    def e2e_run(n_steps, t0=None, t1=None):
+    def e2e_run(n_steps, t0=None, t1=None, f16=False):
+        o_dev, o_host = (out_dev16, out_host16) if f16 else (out_dev, out_host)
         in_done = [torch.cuda.Event() for _ in range(nbuf)]
         comp_done = [torch.cuda.Event() for _ in range(nbuf)]
         out_done = [torch.cuda.Event() for _ in range(nbuf)]
@@ -443,13 +450,13 @@ def run_gpu(args, cfg):
                 stream.wait_event(out_done[b])       # out_dev[b] copied out
             flush.zero_()
             if pipelined:
-                blk(x_dev[b], out=out_dev[b])
+                blk(x_dev[b], out=o_dev[b], flags=moe.MOE_FLAG_OUT_F16 if f16 else None)
             else:
                 fwd(x_dev[b])
             comp_done[b].record(stream)
             s_out.wait_event(comp_done[b])
             with torch.cuda.stream(s_out):
-                out_host[b].copy_(out_dev[b], non_blocking=True)
+                o_host[b].copy_(o_dev[b], non_blocking=True)
                 out_done[b].record(s_out)
         stream.wait_stream(s_in)
         stream.wait_stream(s_out)
@@ -466,12 +473,24 @@ def run_gpu(args, cfg):
     e2e_s = e2e_t0.elapsed_time(e2e_t1) / 1e3
     if world > 1:
         dist.barrier()
+    e2e16_s = 0.0
+    if pipelined:
+        e2e_run(2, f16=True)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        e2e_t0, e2e_t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e2e_run(args.steps, e2e_t0, e2e_t1, f16=True)
+        torch.cuda.synchronize()
+        e2e16_s = e2e_t0.elapsed_time(e2e_t1) / 1e3
+        if world > 1:
+            dist.barrier()
 
     # max over ranks
     if world > 1:
-        t = torch.tensor([total_s, e2e_s, gateup_ms], dtype=torch.float64, device=dev)
+        t = torch.tensor([total_s, e2e_s, gateup_ms, e2e16_s], dtype=torch.float64, device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_s, e2e_s, gateup_ms_max = t.tolist()
+        total_s, e2e_s, gateup_ms_max, e2e16_s = t.tolist()
     else:
         gateup_ms_max = gateup_ms
 
@@ -542,6 +561,11 @@ def run_gpu(args, cfg):
                     "h2d_bytes_per_step": cfg.T * cfg.d * 2, "d2h_bytes_per_step": cfg.T * cfg.d * 4,
                     "copies": ("pinned host buffers; batch i+1 in and batch i-1 out on their own streams while "
                                "batch i computes" if pipelined else "pinned host buffers, in order on one stream")},
+            "e2e_f16out": ({"value": whole_job_rate(cfg.T * args.steps, world, [e2e16_s]), "unit": UNIT,
+                            "h2d_bytes_per_step": cfg.T * cfg.d * 2, "d2h_bytes_per_step": cfg.T * cfg.d * 2,
+                            "out": "fp16: the fp32 sum rounded once (MOE_FLAG_OUT_F16); out16 == fp16(out32) bit "
+                                   "for bit, within the out criteria of the oracle",
+                            "copies": "as e2e"} if pipelined else None),
             "gpu_launches": (KERNELS_PER_FORWARD + 2 * args.shared + (3 if args.round else 0)) * args.steps,
             "clocks": clocks,
             "wall_s_timed_region": wall,

@@ -254,6 +254,16 @@ int moe_forward(const moe_bf16* x, const moe_bf16* w_router, const float* bias,
  * materialised x_perm.  Same results bit for bit. */
 #define MOE_FLAG_FUSED_GATHER 1u
 
+/* moe_forward_ex flag: `out` is [T, d] fp16 instead of fp32.  The combine
+ * sums in fp32 exactly as without the flag and rounds each sum to fp16
+ * (round to nearest even) once, at the store, so the result equals the
+ * fp32 output rounded to fp16 bit for bit; it halves the bytes written and
+ * read back.  An output whose rounding leaves the fp16 range (|v| >= 65520)
+ * or is NaN is stored as such and reported as MOE_ERR_DEVICE_RANGE.  The
+ * article's block returns bf16 (section 1); fp16 keeps three more mantissa
+ * bits.  Accepted by moe_forward_ex only. */
+#define MOE_FLAG_OUT_F16 4u
+
 /*
  * moe_forward with options.  events (may be NULL): n_events >= 6
  * caller-created CUDA events recorded on `stream` before routing, after
@@ -261,9 +271,12 @@ int moe_forward(const moe_bf16* x, const moe_bf16* w_router, const float* bias,
  * GEMM and after the combine, for timing stages; a NULL entry skips that
  * boundary.  A recorded event makes the next kernel wait for the previous
  * one to finish (it cannot begin its launch early), so record only the
- * boundaries you need.  flags: any of MOE_FLAG_FUSED_GATHER and
- * MOE_FLAG_RENORMALIZE (other bits: MOE_ERR_INVALID_ARG).  Without
- * MOE_FLAG_RENORMALIZE the arithmetic is identical to moe_forward.
+ * boundaries you need.  flags: any of MOE_FLAG_FUSED_GATHER,
+ * MOE_FLAG_RENORMALIZE and MOE_FLAG_OUT_F16 (other bits:
+ * MOE_ERR_INVALID_ARG).  out: fp32 [T, d], or fp16 [T, d] with
+ * MOE_FLAG_OUT_F16 (16-byte aligned either way).  Without
+ * MOE_FLAG_RENORMALIZE and MOE_FLAG_OUT_F16 the arithmetic is identical to
+ * moe_forward.
  *
  * Every kernel of the library is launched with programmatic dependent
  * launch: it may begin launching while the previous kernel on the stream
@@ -273,7 +286,7 @@ int moe_forward(const moe_bf16* x, const moe_bf16* w_router, const float* bias,
 int moe_forward_ex(const moe_bf16* x, const moe_bf16* w_router, const float* bias,
                    const moe_bf16* w_gate, const moe_bf16* w_up, const moe_bf16* w_down,
                    int64_t T, int64_t d, int64_t E, int64_t k, int64_t f,
-                   float* out, int32_t* topk_ids_out, float* topk_w_out,
+                   void* out, int32_t* topk_ids_out, float* topk_w_out,
                    void* workspace, size_t workspace_bytes, cudaStream_t stream,
                    cudaEvent_t* events, int n_events, unsigned flags);
 
@@ -310,7 +323,8 @@ int moe_combine_shared(const moe_f16* y, const int32_t* inv, const moe_f16* y_s,
 /* The whole block with shared experts: moe_forward_ex's stages, with the
  * shared GEMMs after the routed down GEMM (inside the "after down" event)
  * and moe_combine_shared; workspace of moe_workspace_size_shared bytes.
- * events and flags as for moe_forward_ex. */
+ * events and flags as for moe_forward_ex, except MOE_FLAG_OUT_F16 (out stays
+ * fp32; the flag gives MOE_ERR_INVALID_ARG). */
 int moe_forward_shared(const moe_bf16* x, const moe_bf16* w_router, const float* bias,
                        const moe_bf16* w_gate, const moe_bf16* w_up, const moe_bf16* w_down,
                        const moe_bf16* w_gate_s, const moe_bf16* w_up_s, const moe_bf16* w_down_s,

@@ -23,6 +23,11 @@ def test_header_matches_binding_list():
     assert set(_declared()) == set(moe.ABI_SYMBOLS)
 
 
+def test_flag_values_match_header():
+    flags = dict(re.findall(r"#define\s+(MOE_FLAG_[A-Z0-9_]+)\s+(\d+)u", open(HEADER).read()))
+    assert flags and {k: int(v) for k, v in flags.items()} == {k: getattr(moe, k) for k in flags}
+
+
 def test_library_exports_every_declared_symbol(moe_lib):
     out = subprocess.run(["nm", "-D", "--defined-only", moe.LIB_PATH], capture_output=True, text=True,
                          check=True).stdout
@@ -70,7 +75,10 @@ def test_validation_happens_before_any_device_call(moe_lib):
                          null) == moe.MOE_ERR_WORKSPACE_TOO_SMALL
     # unknown flag bits
     assert L.moe_forward_ex(fake, fake, null, fake, fake, fake, 16, 64, 8, 2, 64, fake, null, null, fake, 1 << 30,
-                            null, null, 0, 6) == moe.MOE_ERR_INVALID_ARG
+                            null, null, 0, 8) == moe.MOE_ERR_INVALID_ARG
+    # fp16 output is an option of moe_forward_ex only
+    assert L.moe_forward_shared(null, null, null, null, null, null, null, null, null, 16, 64, 8, 2, 64, 1, 64, null,
+                                null, null, null, 0, null, null, 0, moe.MOE_FLAG_OUT_F16) == moe.MOE_ERR_INVALID_ARG
     assert L.moe_combine(null, null, 4, 64, 2, null, null) == moe.MOE_ERR_INVALID_ARG
     assert L.moe_combine(null, null, 4, 65, 2, null, null) == moe.MOE_ERR_UNSUPPORTED_SHAPE
     # workspace too small is caught on the host

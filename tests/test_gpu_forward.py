@@ -180,3 +180,62 @@ def test_forward_cuda_graph_replay_equals_eager():
     eager = blk(x2)
     torch.cuda.synchronize()
     assert torch.equal(out, eager)
+
+
+@pytest.mark.parametrize("cfg", SMALL, ids=lambda c: c.name)
+def test_forward_f16_out_small_all_tokens(cfg):
+    """MOE_FLAG_OUT_F16: the fp32 output rounded to fp16 bit for bit, and every
+    token within the out criteria of the oracle."""
+    d = gc.on_device(gc.inputs(cfg))
+    out32, _, _ = _forward(cfg, d)
+    out16, ids, w = _forward(cfg, d, moe.MOE_FLAG_OUT_F16)
+    assert out16.dtype == torch.float16 and out16.shape == out32.shape
+    assert torch.equal(out16, out32.half())
+    rows, ref = gc.oracle_rows(cfg, cfg.T)
+    _check(cfg, out16, ids, w, rows, ref)
+
+
+def test_forward_f16_out_full_size_is_rounded_fp32():
+    """The Qwen3-shaped layer in the launch configuration the benchmark's
+    fp16-output leg times: out16 == fp16(out32), sampled tokens against the
+    oracle."""
+    cfg = gc.FULL[1]
+    d = gc.on_device(gc.inputs(cfg))
+    out32, _, _ = _forward(cfg, d)
+    out16, ids, w = _forward(cfg, d, moe.MOE_FLAG_OUT_F16)
+    assert torch.equal(out16, out32.half())
+    rows, ref = gc.oracle_rows(cfg, gc.SAMPLES[cfg.name])
+    _check(cfg, out16, ids, w, rows, ref)
+
+
+def test_forward_f16_out_range_is_reported():
+    """Eight identical experts, all selected (k = E) with equal weights 1/8
+    (a zero router): out is the expert's output o and each y row is o / 8.
+    W_down scaled by a power of two so that max|o| lands in [65520, 131040):
+    the fp32 call is clean (y stays in range), the fp16 call stores inf and
+    reports MOE_ERR_DEVICE_RANGE, and the context stays usable."""
+    import math
+    cfg = gc.small_cfg(256, 128, 8, 8, 128)
+    d = gc.on_device(gc.inputs(cfg))
+    wr = torch.zeros_like(d["w_router"])
+    wg = d["w_gate"][:1].expand_as(d["w_gate"]).contiguous()
+    wu = d["w_up"][:1].expand_as(d["w_up"]).contiguous()
+    wd = d["w_down"][:1].expand_as(d["w_down"]).contiguous()
+    o = moe.forward(d["x"], wr, wg, wu, wd, 8)
+    torch.cuda.synchronize()
+    assert moe.get_status() == moe.MOE_OK
+    n = math.ceil(math.log2(65520.0 / o.abs().max().item()))
+    wd2 = (wd.float() * 2.0 ** n).to(torch.bfloat16)
+    o2 = moe.forward(d["x"], wr, wg, wu, wd2, 8)
+    torch.cuda.synchronize()
+    assert moe.get_status() == moe.MOE_OK
+    assert 65520.0 <= o2.abs().max().item() < 131040.0
+    o16 = moe.forward(d["x"], wr, wg, wu, wd2, 8, flags=moe.MOE_FLAG_OUT_F16)
+    torch.cuda.synchronize()
+    assert moe.get_status() == moe.MOE_ERR_DEVICE_RANGE
+    assert torch.isinf(o16).any().item()
+    assert torch.equal(o16, o2.half())
+    o16 = moe.forward(d["x"], wr, wg, wu, wd, 8, flags=moe.MOE_FLAG_OUT_F16)
+    torch.cuda.synchronize()
+    assert moe.get_status() == moe.MOE_OK
+    assert torch.equal(o16, o.half())

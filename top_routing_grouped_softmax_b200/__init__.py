@@ -338,23 +338,26 @@ def _forward_args(x, w_router, w_gate, w_up, w_down, bias):
 
 MOE_FLAG_FUSED_GATHER = 1
 MOE_FLAG_RENORMALIZE = 2
+MOE_FLAG_OUT_F16 = 4
 
 
 def forward(x, w_router, w_gate, w_up, w_down, k, bias=None, out=None, workspace=None,
             topk_ids=None, topk_w=None, events=None, flags=None):
-    """The whole MoE block; returns out [T, d] fp32.
+    """The whole MoE block; returns out [T, d] fp32 (fp16 with MOE_FLAG_OUT_F16).
 
     ``events`` (optional): a list of >= 6 torch.cuda.Event objects (or None
     to skip a boundary) recorded at the stage boundaries (before route, after
     route, after permute, after gate/up, after down, after combine).  ``flags`` (optional):
     MOE_FLAG_FUSED_GATHER selects the variant whose gate/up GEMM gathers the
     rows of x itself (identical results); MOE_FLAG_RENORMALIZE divides each
-    token's k routing weights by their sum.
+    token's k routing weights by their sum; MOE_FLAG_OUT_F16 stores out as
+    fp16 (the fp32 result rounded once).
     """
     T, d, E, f = _forward_args(x, w_router, w_gate, w_up, w_down, bias)
+    out_dtype = torch.float16 if (flags or 0) & MOE_FLAG_OUT_F16 else torch.float32
     if out is None:
-        out = torch.empty(T, d, dtype=torch.float32, device=x.device)
-    _need(out, "out", torch.float32, 2)
+        out = torch.empty(T, d, dtype=out_dtype, device=x.device)
+    _need(out, "out", out_dtype, 2)
     nbytes = workspace_size(T, d, E, k, f)
     if nbytes == 0:
         raise MoEError(MOE_ERR_UNSUPPORTED_SHAPE, "moe_workspace_size")
@@ -474,7 +477,7 @@ class MoEBlock:
 
 __all__ = [
     "lib", "strerror", "MoEError", "ABI_SYMBOLS", "workspace_size", "route_workspace_size",
-    "permute_workspace_size", "MOE_FLAG_FUSED_GATHER", "MOE_FLAG_RENORMALIZE", "route",
+    "permute_workspace_size", "MOE_FLAG_FUSED_GATHER", "MOE_FLAG_RENORMALIZE", "MOE_FLAG_OUT_F16", "route",
     "permute", "expert_ffn", "combine", "forward", "shared_ffn", "combine_shared", "forward_shared", "forward_rounded",
     "get_status", "set_wait_limit_ns", "backward", "backward_workspace_size", "gather_rows",
     "selftest_wait_timeout", "MoEBlock",

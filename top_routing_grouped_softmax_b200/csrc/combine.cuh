@@ -34,10 +34,14 @@ __device__ __forceinline__ void add_f16x8(float (&acc)[8], const uint4& q)
 // One block per token; thread v handles 8 consecutive columns (16 bytes of
 // y, 32 bytes of out).  With shared experts (n_s > 0), their rows
 // y_s[s][t] (weight one, already applied) are added after the k routed
-// slots, in ascending s.
+// slots, in ascending s.  F16OUT: the fp32 sum is rounded to fp16 once, at
+// the store (16 bytes of out per thread); a value whose rounding leaves the
+// fp16 range (|v| >= 65520, or NaN) is stored as such and reported as
+// kStatusDeviceRange, as for y.
+template <bool F16OUT>
 __global__ void __launch_bounds__(256) combine_kernel(const uint4* __restrict__ y, const int32_t* __restrict__ inv,
                                                       int64_t n, int nvec, int k, const uint4* __restrict__ y_s,
-                                                      int n_s, int64_t T, float4* __restrict__ out)
+                                                      int n_s, int64_t T, void* __restrict__ out_)
 {
     __shared__ int s_pos[kMaxK];
     const int64_t t = blockIdx.x;
@@ -62,9 +66,22 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint4* __restrict__ 
             if (p >= 0) add_f16x8(acc, __ldg(y + (int64_t)p * nvec + v));
         }
         for (int sh = 0; sh < n_s; ++sh) add_f16x8(acc, __ldg(y_s + ((int64_t)sh * T + t) * nvec + v));
-        float4* o = out + (t * nvec + v) * 2;
-        o[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
-        o[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+        if constexpr (F16OUT) {
+            bool bad = false;
+            uint32_t pk[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                bad |= !(fabsf(acc[2 * i]) < 65520.0f) || !(fabsf(acc[2 * i + 1]) < 65520.0f);
+                const __half2 h2 = __floats2half2_rn(acc[2 * i], acc[2 * i + 1]);
+                pk[i] = *reinterpret_cast<const uint32_t*>(&h2);
+            }
+            static_cast<uint4*>(out_)[t * nvec + v] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            if (bad) record_status(kStatusDeviceRange);
+        } else {
+            float4* o = static_cast<float4*>(out_) + (t * nvec + v) * 2;
+            o[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+            o[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+        }
     }
 }
 

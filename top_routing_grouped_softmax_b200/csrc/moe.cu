@@ -528,15 +528,20 @@ int run_ffn(const DeviceState& st, const moe_bf16* x_perm, const moe_bf16* x_gat
                   p2);
 }
 
-int run_combine(const moe_f16* y, const int32_t* inv, int64_t T, int64_t d, int64_t k, float* out, cudaStream_t s,
-                const moe_f16* y_s = nullptr, int64_t n_s = 0)
+// out: fp32 [T, d], or fp16 [T, d] with f16_out.
+int run_combine(const moe_f16* y, const int32_t* inv, int64_t T, int64_t d, int64_t k, void* out, cudaStream_t s,
+                const moe_f16* y_s = nullptr, int64_t n_s = 0, bool f16_out = false)
 {
     if (T == 0) return MOE_OK;
     const int nvec = (int)(d / 8);
     const int threads = nvec < 256 ? ((nvec + 31) / 32) * 32 : 256;
-    return launch(moe::combine::combine_kernel, dim3((unsigned)T), dim3(threads), 0, s, 1u,
+    if (f16_out)
+        return launch(moe::combine::combine_kernel<true>, dim3((unsigned)T), dim3(threads), 0, s, 1u,
+                      reinterpret_cast<const uint4*>(y), inv, T * k, nvec, (int)k,
+                      reinterpret_cast<const uint4*>(y_s), (int)n_s, T, out);
+    return launch(moe::combine::combine_kernel<false>, dim3((unsigned)T), dim3(threads), 0, s, 1u,
                   reinterpret_cast<const uint4*>(y), inv, T * k, nvec, (int)k, reinterpret_cast<const uint4*>(y_s),
-                  (int)n_s, T, reinterpret_cast<float4*>(out));
+                  (int)n_s, T, out);
 }
 
 // Shared experts: each is one group of all T rows of x (no permutation, no
@@ -571,7 +576,7 @@ int check_shared(const moe_bf16* w_gate_s, const moe_bf16* w_up_s, const moe_bf1
 
 int forward_impl(const moe_bf16* x, const moe_bf16* w_router, const float* bias, const moe_bf16* w_gate,
                  const moe_bf16* w_up, const moe_bf16* w_down, int64_t T, int64_t d, int64_t E, int64_t k, int64_t f,
-                 float* out, int32_t* ids_out, float* w_out, void* ws, size_t ws_bytes, cudaStream_t s,
+                 void* out, int32_t* ids_out, float* w_out, void* ws, size_t ws_bytes, cudaStream_t s,
                  cudaEvent_t* ev, int n_ev, unsigned flags, const moe_bf16* w_gate_s = nullptr,
                  const moe_bf16* w_up_s = nullptr, const moe_bf16* w_down_s = nullptr, int64_t n_s = 0,
                  int64_t f_s = 0)
@@ -580,7 +585,8 @@ int forward_impl(const moe_bf16* x, const moe_bf16* w_router, const float* bias,
     if (rc) return rc;
     if ((rc = check_f(f))) return rc;
     if ((rc = check_shared(w_gate_s, w_up_s, w_down_s, T, n_s, f_s))) return rc;
-    if (flags & ~(unsigned)(MOE_FLAG_FUSED_GATHER | MOE_FLAG_RENORMALIZE)) return MOE_ERR_INVALID_ARG;
+    if (flags & ~(unsigned)(MOE_FLAG_FUSED_GATHER | MOE_FLAG_RENORMALIZE | MOE_FLAG_OUT_F16))
+        return MOE_ERR_INVALID_ARG;
     if (T > 0 && (!x || !w_router || !w_gate || !w_up || !w_down || !out)) return MOE_ERR_INVALID_ARG;
     if (!aligned(x, 16) || !aligned(w_router, 16) || !aligned(w_gate, 16) || !aligned(w_up, 16) ||
         !aligned(w_down, 16) || !aligned(out, 16) || !aligned(bias, 4) || !aligned(ids_out, 4) ||
@@ -631,7 +637,7 @@ int forward_impl(const moe_bf16* x, const moe_bf16* w_router, const float* bias,
                                     reinterpret_cast<moe_bf16*>(w + L.h_s), y_s, s)))
         return rc;
     if ((rc = rec(4))) return rc;
-    if ((rc = run_combine(y, inv, T, d, k, out, s, y_s, n_s))) return rc;
+    if ((rc = run_combine(y, inv, T, d, k, out, s, y_s, n_s, (flags & MOE_FLAG_OUT_F16) != 0))) return rc;
     return rec(5);
 }
 
@@ -1333,7 +1339,7 @@ int moe_forward_shared(const moe_bf16* x, const moe_bf16* w_router, const float*
                        float* topk_w_out, void* workspace, size_t workspace_bytes, cudaStream_t stream,
                        cudaEvent_t* events, int n_events, unsigned flags)
 {
-    if (n_shared < 1) return MOE_ERR_INVALID_ARG;
+    if (n_shared < 1 || (flags & MOE_FLAG_OUT_F16)) return MOE_ERR_INVALID_ARG;
     return forward_impl(x, w_router, bias, w_gate, w_up, w_down, T, d, E, k, f, out, topk_ids_out, topk_w_out,
                         workspace, workspace_bytes, stream, events, n_events, flags, w_gate_s, w_up_s, w_down_s,
                         n_shared, f_shared);
@@ -1366,7 +1372,7 @@ int moe_forward(const moe_bf16* x, const moe_bf16* w_router, const float* bias, 
 
 int moe_forward_ex(const moe_bf16* x, const moe_bf16* w_router, const float* bias, const moe_bf16* w_gate,
                    const moe_bf16* w_up, const moe_bf16* w_down, int64_t T, int64_t d, int64_t E, int64_t k,
-                   int64_t f, float* out, int32_t* topk_ids_out, float* topk_w_out, void* workspace,
+                   int64_t f, void* out, int32_t* topk_ids_out, float* topk_w_out, void* workspace,
                    size_t workspace_bytes, cudaStream_t stream, cudaEvent_t* events, int n_events, unsigned flags)
 {
     return forward_impl(x, w_router, bias, w_gate, w_up, w_down, T, d, E, k, f, out, topk_ids_out, topk_w_out,
