@@ -30,6 +30,21 @@ def on_device(inp):
     }
 
 
+@functools.lru_cache(maxsize=4)
+def logit_error(cfg: MoEConfig):
+    """logit_error_bound of a configuration's inputs: from
+    sum_i |x[t, i]| |W_router[i, e]| + |b_e| in fp64 ([T, E])."""
+    from tests.parity import logit_error_bound, widen
+    inp = inputs(cfg)
+    ax = np.abs(widen(inp.bits("x")).reshape(cfg.T, cfg.d))
+    aw = np.abs(widen(inp.bits("W_router")).reshape(cfg.d, cfg.E))
+    scale = ax @ aw
+    b = inp.bias_np()
+    if b is not None:
+        scale += np.abs(b.astype(np.float64))[None, :]
+    return logit_error_bound(scale, cfg.d)
+
+
 @functools.lru_cache(maxsize=8)
 def oracle_route(cfg: MoEConfig):
     inp = inputs(cfg)

@@ -9,7 +9,9 @@ Tolerances (floating point; inputs bf16, fp32 accumulation, fp32 outputs):
   * o = h . W_down (y before the routing weight): each element within the
     worst-case effect of that one rounding of h plus fp32 accumulation,
     |gpu - oracle| <= (2^-8 + f * 2^-23) * sum_n |h_n| |W_down[n, c]|
-  * routing weights:            |w_gpu - w_oracle| <= W_REL * w_oracle
+  * routing weights:            |w_gpu - w_oracle| <= W_REL * w_oracle, and,
+                                where the caller passes the logits' magnitudes,
+                                within the a-priori bound of weight_bound
 Integer results (expert ids, counts, offsets, perm, inv) must be bit-exact,
 except for tokens whose k-th and (k+1)-th oracle probabilities differ by less
 than 1e-6: the fp32 logits of the GPU may order such a pair differently, so
@@ -35,6 +37,49 @@ MEAN_REL = 5e-3
 W_REL = 5e-5
 
 
+def logit_error_bound(abs_scale: np.ndarray, d: int) -> np.ndarray:
+    """A-priori bound on |l_gpu - l| per (token, expert) for fp32 logits.
+
+    abs_scale[t, e] = sum_i |x[t, i]| |W_router[i, e]| + |b_e| (fp64).  The
+    products of two bf16 values are exact in fp32; the d - 1 additions of the
+    dot product, the sum of the split-K partials and the bias add are at
+    most d + 1 roundings, in any order.  With unit roundoff u the classical
+    bound is gamma_n * abs_scale, gamma_n = n u / (1 - n u).  u = 2^-23, not
+    2^-24: neither the order nor the rounding mode inside the tensor-core
+    accumulation is specified, and 2^-23 also covers truncation.
+    """
+    u = 2.0 ** -23
+    n = d + 2
+    return (n * u / (1.0 - n * u)) * abs_scale
+
+
+def weight_bound(logit_err: np.ndarray, probs: np.ndarray, ids: np.ndarray) -> np.ndarray:
+    """A-priori bound on |w_gpu - p| / p for each selected slot [T, k].
+
+    With logit errors |delta_j| <= b_j, exp(l_e + delta_e - m) / sum_j
+    exp(l_j + delta_j - m) differs from p_e by a factor within
+    exp(+-(b_e + max_j b_j)).  The fp32 softmax adds: the rounding of l - m
+    and of (l - m) log2(e) before the exponential (relative error of the
+    term up to |l - m| 2^-23, with |l_e - m| = log(p_max / p_e), and, for the
+    sum, the p-weighted mean H of |l_j - m|), the approximate exponential
+    (2^-21 for the numerator and for the sum's terms), and the E-term sum plus
+    the division ((E + 1) 2^-24).  The first-order terms are added and the
+    total is scaled by 1.25 to cover the neglected second-order products.
+    """
+    T, E = probs.shape
+    ids = ids.astype(np.int64)
+    b_e = np.take_along_axis(logit_err, ids, axis=1)
+    b_max = logit_err.max(axis=1, keepdims=True)
+    p_max = probs.max(axis=1, keepdims=True)
+    p_e = np.take_along_axis(probs, ids, axis=1)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        r_e = np.log(p_max / p_e)
+        terms = np.where(probs > 0, probs * np.log(p_max / np.where(probs > 0, probs, 1.0)), 0.0)
+    H = terms.sum(axis=1, keepdims=True)
+    fp = (r_e + H) * 2.0 ** -23 + 2 * 2.0 ** -21 + (E + 1) * 2.0 ** -24
+    return 1.25 * (np.expm1(b_e + b_max) + fp)
+
+
 def widen(bits: np.ndarray) -> np.ndarray:
     return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
 
@@ -44,9 +89,12 @@ def bf16_tensor_to_f64(t) -> np.ndarray:
     return widen(t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16))
 
 
-def route_check(ids_gpu: np.ndarray, w_gpu: np.ndarray, probs: np.ndarray, oracle_ids: np.ndarray, k: int):
+def route_check(ids_gpu: np.ndarray, w_gpu: np.ndarray, probs: np.ndarray, oracle_ids: np.ndarray, k: int,
+                logit_err: np.ndarray | None = None):
     """Check GPU routing against the oracle's fp64 probabilities.
 
+    logit_err (optional, [T, E]): logit_error_bound of the inputs; the
+    weights must then also lie within weight_bound.
     Returns (excluded token mask, stats).  Raises AssertionError on mismatch.
     """
     T = probs.shape[0]
@@ -70,9 +118,15 @@ def route_check(ids_gpu: np.ndarray, w_gpu: np.ndarray, probs: np.ndarray, oracl
     err = np.abs(w_gpu.astype(np.float64) - p_sel)
     worst = float(np.max(err[ok] / p_sel[ok])) if ok.any() else 0.0
     assert worst <= W_REL, f"routing weight relative error {worst:.3e} > {W_REL}"
+    bound_use = None
+    if logit_err is not None:
+        bound = weight_bound(logit_err, probs, ids_gpu)
+        ratio = err / (p_sel * bound)
+        bound_use = float(ratio[ok].max()) if ok.any() else 0.0
+        assert bound_use <= 1.0, f"routing weight beyond its a-priori bound (x{bound_use:.3f})"
     assert np.all(np.diff(w_gpu, axis=1) <= 0), "slots not in descending probability order"
     stats = {"tokens": int(T), "excluded_near_tie": int(excluded.sum()), "inner_near_tie": int(inner.sum()),
-             "w_max_rel_err": worst}
+             "w_max_rel_err": worst, "w_bound_use": bound_use}
     return excluded, stats
 
 

@@ -34,7 +34,8 @@ def _forward(cfg, d, flags=0):
 
 def _check(cfg, out, ids, w, rows, ref_out):
     r = gc.oracle_route(cfg)
-    excluded, stats = route_check(ids.cpu().numpy(), w.cpu().numpy(), r.probs, r.ids, cfg.k)
+    excluded, stats = route_check(ids.cpu().numpy(), w.cpu().numpy(), r.probs, r.ids, cfg.k,
+                                  logit_err=gc.logit_error(cfg))
     keep = ~excluded[rows]
     got = out.double().cpu().numpy()[rows]
     return value_check(got[keep], ref_out[keep], f"out[{cfg.name}]"), stats

@@ -1,7 +1,7 @@
 """Router kernel (GEMM + fp32 softmax + top-k) against the oracle, on the GPU.
 
 Expert ids bit-exact (near ties excepted, see tests/parity.py), weights to
-1e-5 relative."""
+5e-5 relative and within their a-priori fp32 bound (tests/parity.py)."""
 import numpy as np
 import pytest
 import torch
@@ -35,14 +35,14 @@ def _route(cfg):
 def test_route_small(cfg):
     ids, w = _route(cfg)
     r = gc.oracle_route(cfg)
-    route_check(ids, w, r.probs, r.ids, cfg.k)
+    route_check(ids, w, r.probs, r.ids, cfg.k, logit_err=gc.logit_error(cfg))
 
 
 @pytest.mark.parametrize("cfg", gc.FULL, ids=lambda c: c.name)
 def test_route_full_size(cfg):
     ids, w = _route(cfg)
     r = gc.oracle_route(cfg)
-    excluded, stats = route_check(ids, w, r.probs, r.ids, cfg.k)
+    excluded, stats = route_check(ids, w, r.probs, r.ids, cfg.k, logit_err=gc.logit_error(cfg))
     print(cfg.name, stats)
     assert stats["excluded_near_tie"] < max(1, cfg.T // 100)
 

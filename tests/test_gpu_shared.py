@@ -39,7 +39,8 @@ def _run(cfg, d, sdev):
 def _check(cfg, out, ids, w, bits, rows):
     inp = gc.inputs(cfg)
     r = gc.oracle_route(cfg)
-    excluded, _ = route_check(ids.cpu().numpy(), w.cpu().numpy(), r.probs, r.ids, cfg.k)
+    excluded, _ = route_check(ids.cpu().numpy(), w.cpu().numpy(), r.probs, r.ids, cfg.k,
+                              logit_err=gc.logit_error(cfg))
     _, ex = gc.default_oracle().forward(inp.bits("x"), inp.bits("W_router"), inp.bias_np(), inp.bits("W_gate"),
                                         inp.bits("W_up"), inp.bits("W_down"), cfg.k, rows=rows, shared=bits)
     keep = ~excluded[rows]
