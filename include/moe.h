@@ -394,7 +394,9 @@ int moe_forward_rounded(const moe_bf16* x, const moe_bf16* w_router, const float
  *   (NULL to skip), dw_gate / dw_up [E, d, f], dw_down [E, f, d]: fp32 out,
  *   overwritten (experts no token selects get zeros).  All 16-byte aligned.
  * Precision: the GEMM operands are bf16 (x, the weights, dout, dg, du, w h
- * and dlogit rounded once each), every sum fp32.  flags: 0 or
+ * and dlogit rounded once each), every sum fp32; each slot's contribution
+ * to dx (dg . W_gate^T + du . W_up^T) is rounded to bf16 once before the
+ * fp32 sum over the token's k slots.  flags: 0 or
  * MOE_FLAG_RENORMALIZE (the routing the forward used).  Workspace:
  * moe_backward_workspace_size bytes, 256-byte aligned; grouped rows are
  * padded so that each expert's group starts on a 64-row boundary.

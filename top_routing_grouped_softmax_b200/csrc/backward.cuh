@@ -20,11 +20,12 @@
 //                 stores dlogit in bf16 (the operand of the two router GEMMs)
 //                 and the block's fp32 sums of dlogit for the bias gradient
 //   colsum        dbias[e] = sum over blocks of those sums, in a fixed order
-//   combine_dx    dx[t] = dx_router[t] + sum_j dx_perm[inv[t*k+j]]  (fp32)
+//   combine_dx    dx[t] = dx_router[t] + sum_j dx_perm[inv[t*k+j]]  (fp32 sums of bf16 dx_perm rows)
 #pragma once
 
 #include <cuda_bf16.h>
 
+#include "grouped_gemm_bwd.cuh"
 #include "ptx.cuh"
 
 namespace moe {
@@ -181,9 +182,10 @@ __global__ void __launch_bounds__(kRowThreads) colsum_kernel(const float* __rest
     if (threadIdx.x == 0) dbias[e] = s_part[0];
 }
 
-// dx[t] = dx_router[t] + sum_j dx_perm[inv[t*k+j]] (fp32, slots in order):
-// one block per token, four columns per thread.  nvec = d / 4.
-__global__ void __launch_bounds__(kRowThreads) combine_dx_kernel(const float4* __restrict__ dx_perm,
+// dx[t] = dx_router[t] + sum_j dx_perm[inv[t*k+j]] (fp32 sums, slots in
+// order; dx_perm bf16, widened exactly): one block per token, eight columns
+// per thread.  nvec = d / 8.
+__global__ void __launch_bounds__(kRowThreads) combine_dx_kernel(const uint4* __restrict__ dx_perm,
                                                                  const float4* __restrict__ dx_router,
                                                                  const int32_t* __restrict__ inv, int64_t rows, int k,
                                                                  int nvec, float4* __restrict__ dx)
@@ -202,17 +204,18 @@ __global__ void __launch_bounds__(kRowThreads) combine_dx_kernel(const float4* _
     }
     __syncthreads();
     for (int v = threadIdx.x; v < nvec; v += blockDim.x) {
-        float4 acc = __ldg(dx_router + t * nvec + v);
+        const float4 r0 = __ldg(dx_router + (t * nvec + v) * 2), r1 = __ldg(dx_router + (t * nvec + v) * 2 + 1);
+        float acc[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
         for (int j = 0; j < k; ++j) {
             const int p = s_pos[j];
             if (p < 0) continue;
-            const float4 a = __ldg(dx_perm + (int64_t)p * nvec + v);
-            acc.x += a.x;
-            acc.y += a.y;
-            acc.z += a.z;
-            acc.w += a.w;
+            float a[8];
+            unpack_bf16x8(__ldg(dx_perm + (int64_t)p * nvec + v), a);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) acc[i] += a[i];
         }
-        dx[t * nvec + v] = acc;
+        dx[(t * nvec + v) * 2] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        dx[(t * nvec + v) * 2 + 1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
     }
 }
 

@@ -91,6 +91,7 @@ struct Params {
     int m_total;             // kDW: output rows per expert
     int m_tiles;             // kDW: 256-row M tiles per expert
     int split_b;             // kDW: 1 = B halves from two tensors (dg | du), two outputs
+    int out_bf16;            // kDX: 1 = out0 holds bf16 values (rows of ld_out), stored through a 2-D map
 };
 
 struct alignas(8) Ctrl {
@@ -206,7 +207,8 @@ __device__ __forceinline__ void store_zero_f32x16(float* dst)
 // output in `slab` (kSlabBufs 4 KB buffers of this warp, taken in turn)
 // and store it with TMA: kDW through tm_o0 / tm_o1 ([E][m_total][n_out]
 // fp32 views; rows past m_total and columns past n_out are not written),
-// kDX through tm_o0 ([1][rows][n_out]).
+// kDX through tm_o0 ([1][rows][n_out] fp32, or with p.out_bf16 a 2-D
+// [rows][n_out] bf16 map whose 32 x 32 box is a 2 KB slab).
 template <int KIND>
 __device__ __forceinline__ void epilogue(const Params& p, const Item& it, uint32_t tbase, uint32_t rank, int q,
                                          int lane, int half, const CUtensorMap* tm_o0, const CUtensorMap* tm_o1,
@@ -343,7 +345,37 @@ __device__ __forceinline__ void epilogue(const Params& p, const Item& it, uint32
             }
             const uint32_t(&lo)[16] = lob[si & 1];
             const uint32_t(&hi)[16] = hib[si & 1];
-            if (c0 < ncols && whole) {  // c0 < ncols is warp-uniform (n_out % 64 == 0)
+            if (p.out_bf16) {
+                // bf16 rows: a 32 x 32 slab is 2 KB (64-byte rows, 64-byte swizzle)
+                uint32_t pk[16];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    pk[i] = gemm::pack_bf16x2(__uint_as_float(lo[2 * i]), __uint_as_float(lo[2 * i + 1]));
+                    pk[8 + i] = gemm::pack_bf16x2(__uint_as_float(hi[2 * i]), __uint_as_float(hi[2 * i + 1]));
+                }
+                if (c0 < ncols && whole) {
+                    uint32_t* buf = reinterpret_cast<uint32_t*>(slab) + slab_buf * (kSlabBytes / 4);
+                    if (lane == 0) bulk_wait_group_read<kSlabBufs - 1>();
+                    __syncwarp();
+                    uint4* rowp = reinterpret_cast<uint4*>(buf + lane * 16);
+                    const int sw = (lane >> 1) & 3;
+#pragma unroll
+                    for (int v = 0; v < 4; ++v)
+                        rowp[v ^ sw] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_2d(tm_o0, buf, c_base + c0, wrow0);
+                        bulk_commit_group();
+                    }
+                    slab_buf = (slab_buf + 1) % kSlabBufs;
+                } else if (c0 < ncols && valid) {
+                    uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.out0) +
+                                                          (int64_t)row * p.ld_out + c_base + c0);
+#pragma unroll
+                    for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+                }
+            } else if (c0 < ncols && whole) {  // c0 < ncols is warp-uniform (n_out % 64 == 0)
                 uint32_t* buf = reinterpret_cast<uint32_t*>(slab) + slab_buf * (kSlabBytes / 4);
                 if (lane == 0) bulk_wait_group_read<kSlabBufs - 1>();
                 __syncwarp();

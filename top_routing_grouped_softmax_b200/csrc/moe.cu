@@ -806,7 +806,7 @@ BLayout plan_backward(int64_t T, int64_t d, int64_t E, int64_t k, int64_t f)
     L.u = o;         o += align256(R * (size_t)f * 2);   // u, then du in place
     L.hw = o;        o += align256(R * (size_t)f * 2);
     L.dwp = o;       o += align256(R * (size_t)(2 * L.n_tiles_f) * 4);
-    L.dx_perm = o;   o += align256(R * (size_t)d * 4);
+    L.dx_perm = o;   o += align256(R * (size_t)d * 2);  // bf16
     L.dlogit = o;    o += align256((size_t)T * (size_t)L.e_pad * 2);
     L.db_part = o;   o += align256((size_t)((T + moe::bwd::kRowWarps - 1) / moe::bwd::kRowWarps) * (size_t)E * 4);
     L.dx_router = o; o += align256((size_t)T * (size_t)d * 4);
@@ -900,7 +900,7 @@ int backward_impl(const moe_bf16* x, const moe_bf16* w_router, const float* bias
     moe_bf16* u = static_cast<moe_bf16*>(at(L.u));
     moe_bf16* hw = static_cast<moe_bf16*>(at(L.hw));
     float* dwp = static_cast<float*>(at(L.dwp));
-    float* dx_perm = static_cast<float*>(at(L.dx_perm));
+    moe_bf16* dx_perm = static_cast<moe_bf16*>(at(L.dx_perm));
     moe_bf16* dlogit = static_cast<moe_bf16*>(at(L.dlogit));
     float* db_part = static_cast<float*>(at(L.db_part));
     float* dx_router = static_cast<float*>(at(L.dx_router));
@@ -984,18 +984,20 @@ int backward_impl(const moe_bf16* x, const moe_bf16* w_router, const float* bias
         p.b_rows = (int)f;
         if (launch_pair_bwd<kDH>(*st, max_mtiles * p.n_tiles, ta, ta, tb, tb, p, s)) return MOE_ERR_CUDA;
     }
-    // 5. dx_perm = dg . W_gate^T + du . W_up^T (fp32)
+    // 5. dx_perm = dg . W_gate^T + du . W_up^T (fp32 accumulators, stored bf16)
     {
         CUtensorMap ta, ta2, tb0, tb1, to0;
         rc = make_map(&ta, g, (uint64_t)f, (uint64_t)R, 64, kBM);
         rc = rc ? rc : make_map(&ta2, u, (uint64_t)f, (uint64_t)R, 64, kBM);
         rc = rc ? rc : make_map(&tb0, w_gate, (uint64_t)f, (uint64_t)(E * d), 64, kBM);
         rc = rc ? rc : make_map(&tb1, w_up, (uint64_t)f, (uint64_t)(E * d), 64, kBM);
-        rc = rc ? rc : make_out3_map(&to0, dx_perm, (uint64_t)d, (uint64_t)R, 1);
+        rc = rc ? rc : make_map(&to0, dx_perm, (uint64_t)d, (uint64_t)R, 32, 32, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                                CU_TENSOR_MAP_SWIZZLE_64B);
         if (rc) return rc;
         Params p = bwd_params();
         p.offsets = offsets;
-        p.out0 = dx_perm;
+        p.out0 = reinterpret_cast<float*>(dx_perm);
+        p.out_bf16 = 1;
         p.ld_out = d;
         p.E = iE;
         p.M = (int)R;
@@ -1104,10 +1106,10 @@ int backward_impl(const moe_bf16* x, const moe_bf16* w_router, const float* bias
                                  &to0))
             return MOE_ERR_CUDA;
     }
-    // 11. dx = dx_router + sum over slots of dx_perm (fp32)
+    // 11. dx = dx_router + sum over slots of dx_perm (fp32 sums)
     if (launch(combine_dx_kernel, dim3((unsigned)T), dim3(kRowThreads), 0, s, 1u,
-               reinterpret_cast<const float4*>(dx_perm), reinterpret_cast<const float4*>(dx_router),
-               static_cast<const int32_t*>(inv), R, ik, (int)(d / 4), reinterpret_cast<float4*>(dx)))
+               reinterpret_cast<const uint4*>(dx_perm), reinterpret_cast<const float4*>(dx_router),
+               static_cast<const int32_t*>(inv), R, ik, (int)(d / 8), reinterpret_cast<float4*>(dx)))
         return MOE_ERR_CUDA;
     return MOE_OK;
 }
