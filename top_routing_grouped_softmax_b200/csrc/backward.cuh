@@ -20,6 +20,7 @@
 //                 stores dlogit in bf16 (the operand of the two router GEMMs)
 //                 and the block's fp32 sums of dlogit for the bias gradient
 //   colsum        dbias[e] = sum over blocks of those sums, in a fixed order
+//   sum_partials  dW_router = the sum of its split-K partials, in a fixed order
 //   combine_dx    dx[t] = dx_router[t] + sum_j dx_perm[inv[t*k+j]]  (fp32 sums of bf16 dx_perm rows)
 #pragma once
 
@@ -180,6 +181,26 @@ __global__ void __launch_bounds__(kRowThreads) colsum_kernel(const float* __rest
         __syncthreads();
     }
     if (threadIdx.x == 0) dbias[e] = s_part[0];
+}
+
+// out[i] = sum over s = 0..S-1 of part[s][i], in ascending s (fp32): the
+// split-K partial products of the router's weight gradient.  n4 = elements / 4.
+__global__ void __launch_bounds__(kRowThreads) sum_partials_kernel(const float4* __restrict__ part, int S,
+                                                                   int64_t n4, float4* __restrict__ out)
+{
+    pdl_trigger();
+    pdl_wait();
+    for (int64_t i = blockIdx.x * (int64_t)kRowThreads + threadIdx.x; i < n4; i += (int64_t)gridDim.x * kRowThreads) {
+        float4 acc = __ldg(part + i);
+        for (int s = 1; s < S; ++s) {
+            const float4 a = __ldg(part + (int64_t)s * n4 + i);
+            acc.x += a.x;
+            acc.y += a.y;
+            acc.z += a.z;
+            acc.w += a.w;
+        }
+        out[i] = acc;
+    }
 }
 
 // dx[t] = dx_router[t] + sum_j dx_perm[inv[t*k+j]] (fp32 sums, slots in

@@ -92,6 +92,8 @@ struct Params {
     int m_tiles;             // kDW: 256-row M tiles per expert
     int split_b;             // kDW: 1 = B halves from two tensors (dg | du), two outputs
     int out_bf16;            // kDX: 1 = out0 holds bf16 values (rows of ld_out), stored through a 2-D map
+    int k_chunk;             // kDW: > 0 = group e is rows [e k_chunk, min((e + 1) k_chunk, M)) of one
+                             // M-row operand pair (split K; offsets unused), else the offsets' groups
 };
 
 struct alignas(8) Ctrl {
@@ -154,10 +156,15 @@ __device__ __forceinline__ Item decode_item(int64_t w, const Params& p, const Ct
         const int rem = (int)(w - (int64_t)it.e * per_e);
         it.mt = rem / p.n_tiles;
         it.nt = rem - it.mt * p.n_tiles;
-        it.kstart = c.off[it.e];
-        it.num_kb = (c.off[it.e + 1] - c.off[it.e] + kBK - 1) / kBK;
+        if (p.k_chunk > 0) {
+            it.kstart = it.e * p.k_chunk;
+            it.row_end = min(it.kstart + p.k_chunk, p.M);
+        } else {
+            it.kstart = c.off[it.e];
+            it.row_end = c.off[it.e + 1];
+        }
+        it.num_kb = (it.row_end - it.kstart + kBK - 1) / kBK;
         it.row0 = it.kstart;
-        it.row_end = c.off[it.e + 1];
     } else {
         gemm::decode_tile<kPairRows>(w, p.n_tiles, c.tp, c.off, p.E, it.e, it.row0, it.row_end, it.nt);
         it.mt = 0;

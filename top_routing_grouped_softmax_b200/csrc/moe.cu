@@ -774,9 +774,15 @@ int forward_rounded_impl(const moe_bf16* x, const moe_bf16* w_router, const floa
 // Workspace of moe_backward.  Grouped rows are padded: every expert group
 // starts on a 64-row boundary, so the grouped buffers hold up to
 // T*k + 63*E rows.
+// The router's weight gradient x^T . dlogit reduces over all T tokens into a
+// small d x E matrix: (d / 256) x (E / 256) output tiles, too few to fill the
+// GPU.  It is split over up to this many chunks of tokens, each writing a
+// partial product, summed afterwards in a fixed order.
+constexpr int64_t kRouterGradSplits = 16;
+
 struct BLayout {
     size_t ids, wts, probs, counts, offsets, chunk, perm, inv, w_perm, x_perm, dout_perm, g, u, hw, dwp, dx_perm,
-        dlogit, db_part, dx_router, total;
+        dlogit, db_part, dx_router, dwr_part, total;
     int64_t rows;    // padded row capacity
     int64_t e_pad;   // E rounded up to 64 (row length of dlogit)
     int n_tiles_f;   // 256-column tiles over f (the down-projection gradient's partial dots)
@@ -810,6 +816,7 @@ BLayout plan_backward(int64_t T, int64_t d, int64_t E, int64_t k, int64_t f)
     L.dlogit = o;    o += align256((size_t)T * (size_t)L.e_pad * 2);
     L.db_part = o;   o += align256((size_t)((T + moe::bwd::kRowWarps - 1) / moe::bwd::kRowWarps) * (size_t)E * 4);
     L.dx_router = o; o += align256((size_t)T * (size_t)d * 4);
+    L.dwr_part = o;  o += align256((size_t)kRouterGradSplits * (size_t)d * (size_t)E * 4);
     L.total = o;
     return L;
 }
@@ -1064,25 +1071,43 @@ int backward_impl(const moe_bf16* x, const moe_bf16* w_router, const float* bias
     if (dbias && launch(colsum_kernel, dim3((unsigned)E), dim3(kRowThreads), 0, s, 1u,
                         static_cast<const float*>(db_part), (int)nblk, iE, dbias))
         return MOE_ERR_CUDA;
-    // 9. dW_router = x^T . dlogit (one group of T rows)
+    // 9. dW_router = x^T . dlogit: the T rows in S chunks of a multiple of 64
+    //    rows (as many as fill one wave of CTA pairs, at most
+    //    kRouterGradSplits), one fp32 partial product per chunk, then their
+    //    sum in chunk order
     {
+        const int m_tiles = (int)((d + kPairRows - 1) / kPairRows);
+        const int n_tiles = (int)((E + kBN - 1) / kBN);
+        const int64_t pairs = st->max_pairs > 0 ? st->max_pairs : st->sm_count / 2;
+        int64_t S = pairs / ((int64_t)m_tiles * n_tiles);
+        S = S < 1 ? 1 : (S > kRouterGradSplits ? kRouterGradSplits : S);
+        const int64_t chunk = ((T + S - 1) / S + 63) / 64 * 64;
+        S = (T + chunk - 1) / chunk;
+        float* part = static_cast<float*>(at(L.dwr_part));
         CUtensorMap ta, tb, to0;
         rc = make_weight_chunk_map(&ta, x, (uint64_t)d, (uint64_t)T);
         rc = rc ? rc : make_weight_chunk_map(&tb, dlogit, (uint64_t)L.e_pad, (uint64_t)T);
-        rc = rc ? rc : make_out3_map(&to0, dw_router, (uint64_t)E, (uint64_t)d, 1);
+        rc = rc ? rc : make_out3_map(&to0, part, (uint64_t)E, (uint64_t)d, (uint64_t)S);
         if (rc) return rc;
         Params p = bwd_params();
         p.offsets = nullptr;
-        p.out0 = dw_router;
+        p.out0 = part;
         p.ld_out = E;
-        p.E = 1;
+        p.E = (int)S;
         p.M = (int)T;
+        p.k_chunk = (int)chunk;
         p.n_out = iE;
-        p.n_tiles = (int)((E + kBN - 1) / kBN);
+        p.n_tiles = n_tiles;
         p.m_total = (int)d;
-        p.m_tiles = (int)((d + kPairRows - 1) / kPairRows);
+        p.m_tiles = m_tiles;
         p.split_b = 0;
-        if (launch_pair_bwd<kDW>(*st, p.m_tiles * p.n_tiles, ta, ta, tb, tb, p, s, &to0, &to0)) return MOE_ERR_CUDA;
+        if (launch_pair_bwd<kDW>(*st, S * p.m_tiles * p.n_tiles, ta, ta, tb, tb, p, s, &to0, &to0))
+            return MOE_ERR_CUDA;
+        const int64_t n4 = d * E / 4;
+        const unsigned blocks = (unsigned)((n4 + kRowThreads - 1) / kRowThreads);
+        if (launch(sum_partials_kernel, dim3(blocks < 1184u ? blocks : 1184u), dim3(kRowThreads), 0, s, 1u,
+                   reinterpret_cast<const float4*>(part), (int)S, n4, reinterpret_cast<float4*>(dw_router)))
+            return MOE_ERR_CUDA;
     }
     // 10. dx_router = dlogit . W_router^T (fp32)
     {
