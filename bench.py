@@ -699,7 +699,7 @@ def run_backward(args, cfg):
         "roofline": {"bound": "tensor", "scope": "the whole backward", "achieved": tflops,
                      "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": tflops / peaks["bf16_tflops"],
                      "traffic": None, "flops": flops, "peak_source": f"{peaks['source']} burst bf16"},
-        "gpu_launches": 16 * args.steps,  # 6 routing and grouping, 7 GEMMs, router step, bias sum, combine
+        "gpu_launches": 17 * args.steps,  # 6 routing and grouping, 7 GEMMs, router step, bias sum, router-gradient sum, combine
         "clocks": clk.summary(),
     }
     print(json.dumps(line), flush=True)
