@@ -240,3 +240,17 @@ def test_forward_f16_out_range_is_reported():
     torch.cuda.synchronize()
     assert moe.get_status() == moe.MOE_OK
     assert torch.equal(o16, o.half())
+
+
+@pytest.mark.parametrize("flags", [moe.MOE_FLAG_RENORMALIZE, moe.MOE_FLAG_FUSED_GATHER,
+                                   moe.MOE_FLAG_RENORMALIZE | moe.MOE_FLAG_FUSED_GATHER],
+                         ids=["renorm", "fused_gather", "both"])
+def test_forward_f16_out_with_other_flags(flags):
+    """The fp16 output composes with the other flags: fp16 of the fp32 output
+    computed with the same flags, bit for bit."""
+    cfg = gc.small_cfg(1000, 256, 16, 4, 320, skew=True)
+    d = gc.on_device(gc.inputs(cfg))
+    out32, ids32, w32 = _forward(cfg, d, flags)
+    out16, ids16, w16 = _forward(cfg, d, flags | moe.MOE_FLAG_OUT_F16)
+    assert torch.equal(ids16, ids32) and torch.equal(w16, w32)
+    assert torch.equal(out16, out32.half())
