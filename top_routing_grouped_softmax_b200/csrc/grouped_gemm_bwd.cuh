@@ -127,17 +127,31 @@ constexpr int kSlabBufs = MOE_BWD_SLAB_BUFS;
 constexpr int kSlabBytes = 32 * 32 * 4;
 constexpr int kStoreBytes = kEpiWarps * kSlabBufs * kSlabBytes;
 static_assert(kSlabBufs == 1 || kSlabBufs == 2, "staging slabs per warp");
+// kDH stages each warp's 32-row x 16-column dg and du chunk in one 2 KB
+// slab (dg in the first KB, du in the second) for two 2-D TMA stores.
+constexpr int kDhSlabBytes = 2048;
+__host__ __device__ constexpr int slab_stride_for(int kind)
+{
+    return kind == kDH ? kDhSlabBytes : kSlabBufs * kSlabBytes;
+}
 __host__ __device__ constexpr int stages_for(int kind)
 {
     return (kind == kDW || kind == kDX) ? MOE_BWD_STORE_STAGES : kPairStages;
 }
-__host__ __device__ constexpr int store_bytes_for(int kind) { return (kind == kDW || kind == kDX) ? kStoreBytes : 0; }
+__host__ __device__ constexpr int store_bytes_for(int kind)
+{
+    return (kind == kDW || kind == kDX) ? kStoreBytes : (kind == kDH ? kEpiWarps * kDhSlabBytes : 0);
+}
 
 template <int KIND>
 __host__ inline size_t smem_bytes()
 {
     return 1024 + (size_t)stages_for(KIND) * kPairStageBytes + store_bytes_for(KIND) + sizeof(Ctrl);
 }
+static_assert(1024 + (size_t)stages_for(kDH) * kPairStageBytes + store_bytes_for(kDH) + sizeof(Ctrl) <= 227 * 1024,
+              "dh ring, staging and control exceed 227 KB of shared memory");
+static_assert(1024 + (size_t)stages_for(kDW) * kPairStageBytes + store_bytes_for(kDW) + sizeof(Ctrl) <= 227 * 1024,
+              "weight-gradient ring, staging and control exceed 227 KB of shared memory");
 
 // One work item of kind KIND: the expert, the first grouped row (M-grouped
 // kinds) or M tile (kDW), the group's row range, the N tile and the number
@@ -265,6 +279,8 @@ __device__ __forceinline__ void epilogue(const Params& p, const Item& it, uint32
         const int ncols = min(kBN, p.n_out - c_base);
         const float w = valid ? __ldg(p.w_perm + row) : 0.0f;
         const int64_t row_off = (int64_t)row * p.ld_f + c_base;
+        const int wrow0 = it.row0 + (int)rank * kBM + q * 32;
+        const bool whole = wrow0 + 31 < it.row_end;  // warp-uniform: all 32 rows belong to the group
         float dot = 0.0f;
         // g and u of the next two 16-column chunks are in flight while this
         // chunk is processed (the loads are row-strided across the warp and
@@ -318,12 +334,32 @@ __device__ __forceinline__ void epilogue(const Params& p, const Item& it, uint32
                     pdg[i] = gemm::pack_bf16x2(dgv[0], dgv[1]);
                     pdu[i] = gemm::pack_bf16x2(duv[0], duv[1]);
                 }
-                uint4* dgp = reinterpret_cast<uint4*>(p.out_g + row_off + c0);
-                uint4* dup = reinterpret_cast<uint4*>(p.out_u + row_off + c0);
-                dgp[0] = make_uint4(pdg[0], pdg[1], pdg[2], pdg[3]);
-                dgp[1] = make_uint4(pdg[4], pdg[5], pdg[6], pdg[7]);
-                dup[0] = make_uint4(pdu[0], pdu[1], pdu[2], pdu[3]);
-                dup[1] = make_uint4(pdu[4], pdu[5], pdu[6], pdu[7]);
+                if (whole) {
+                    // the warp's 32 x 16 chunk of dg and du through the slab:
+                    // two 2-D TMA stores instead of 64 row-strided 32-byte ones
+                    uint4* sg = reinterpret_cast<uint4*>(slab) + lane * 2;
+                    uint4* su = reinterpret_cast<uint4*>(slab) + 64 + lane * 2;
+                    if (lane == 0) bulk_wait_group_read<0>();  // the slab's last stores have read it
+                    __syncwarp();
+                    sg[0] = make_uint4(pdg[0], pdg[1], pdg[2], pdg[3]);
+                    sg[1] = make_uint4(pdg[4], pdg[5], pdg[6], pdg[7]);
+                    su[0] = make_uint4(pdu[0], pdu[1], pdu[2], pdu[3]);
+                    su[1] = make_uint4(pdu[4], pdu[5], pdu[6], pdu[7]);
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_2d(tm_o0, slab, c_base + c0, wrow0);
+                        tma_store_2d(tm_o1, reinterpret_cast<uint8_t*>(slab) + 1024, c_base + c0, wrow0);
+                        bulk_commit_group();
+                    }
+                } else {
+                    uint4* dgp = reinterpret_cast<uint4*>(p.out_g + row_off + c0);
+                    uint4* dup = reinterpret_cast<uint4*>(p.out_u + row_off + c0);
+                    dgp[0] = make_uint4(pdg[0], pdg[1], pdg[2], pdg[3]);
+                    dgp[1] = make_uint4(pdg[4], pdg[5], pdg[6], pdg[7]);
+                    dup[0] = make_uint4(pdu[0], pdu[1], pdu[2], pdu[3]);
+                    dup[1] = make_uint4(pdu[4], pdu[5], pdu[6], pdu[7]);
+                }
             }
             tmem_ld_wait();
         }
@@ -489,7 +525,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_prefetch_map(&tm_b0);
         if (KIND == kDX) tma_prefetch_map(&tm_a2);
         if (KIND == kGU || KIND == kDX || KIND == kDW) tma_prefetch_map(&tm_b1);
-        if (KIND == kDW || KIND == kDX) {
+        if (KIND == kDW || KIND == kDX || KIND == kDH) {
             tma_prefetch_map(&tm_o0);
             tma_prefetch_map(&tm_o1);
         }
@@ -625,7 +661,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ---------------------------------------------------- epilogue (both CTAs)
         const int q = warp & 3;                 // TMEM lane quarter
         const int half = (warp - 2) >> 2;       // column half: warps 2-5 and 6-9
-        float* slab = reinterpret_cast<float*>(stage_out + (warp - 2) * kSlabBufs * kSlabBytes);
+        float* slab = reinterpret_cast<float*>(stage_out + (warp - 2) * slab_stride_for(KIND));
         int slab_buf = 0;
         int acc = 0;
         uint32_t acc_ph = 0;
@@ -649,7 +685,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 acc_ph ^= 1u;
             }
         }
-        if ((KIND == kDW || KIND == kDX) && lane == 0) bulk_wait_group_all();
+        if ((KIND == kDW || KIND == kDX || KIND == kDH) && lane == 0) bulk_wait_group_all();
         __syncwarp();
     }
 

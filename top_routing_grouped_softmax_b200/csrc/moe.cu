@@ -970,9 +970,14 @@ int backward_impl(const moe_bf16* x, const moe_bf16* w_router, const float* bias
     }
     // 4. dh = w . dout_perm . W_down^T and the SwiGLU derivative: dg, du (in place of g, u), partial dots
     {
-        CUtensorMap ta, tb;
+        CUtensorMap ta, tb, tog, tou;
         rc = make_map(&ta, dout_perm, (uint64_t)d, (uint64_t)R, 64, kBM);
         rc = rc ? rc : make_map(&tb, w_down, (uint64_t)d, (uint64_t)(E * f), 64, kBM);
+        // dg and du (in place over g and u) for the epilogue's 32 x 16 TMA stores
+        rc = rc ? rc : make_map(&tog, g, (uint64_t)f, (uint64_t)R, 16, 32, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                                CU_TENSOR_MAP_SWIZZLE_NONE);
+        rc = rc ? rc : make_map(&tou, u, (uint64_t)f, (uint64_t)R, 16, 32, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                                CU_TENSOR_MAP_SWIZZLE_NONE);
         if (rc) return rc;
         Params p = bwd_params();
         p.offsets = offsets;
@@ -989,7 +994,7 @@ int backward_impl(const moe_bf16* x, const moe_bf16* w_router, const float* bias
         p.n_out = (int)f;
         p.n_tiles = L.n_tiles_f;
         p.b_rows = (int)f;
-        if (launch_pair_bwd<kDH>(*st, max_mtiles * p.n_tiles, ta, ta, tb, tb, p, s)) return MOE_ERR_CUDA;
+        if (launch_pair_bwd<kDH>(*st, max_mtiles * p.n_tiles, ta, ta, tb, tb, p, s, &tog, &tou)) return MOE_ERR_CUDA;
     }
     // 5. dx_perm = dg . W_gate^T + du . W_up^T (fp32 accumulators, stored bf16)
     {
