@@ -115,8 +115,22 @@ def qwen_grads():
     return cfg, _run(cfg)
 
 
-def test_backward_full_size_sampled_rows(qwen_grads):
-    cfg, got = qwen_grads
+@pytest.fixture(scope="module")
+def fine_grads():
+    cfg = CONFIGS["fine"]
+    return cfg, _run(cfg)
+
+
+@pytest.fixture(params=["qwen", "fine"])
+def full_grads(request):
+    """The Qwen3-shaped layer and the fine-grained one (E = 256, f = 256: a
+    short K for the dh and weight-gradient GEMMs, 256 experts in the router
+    gradient's split)."""
+    return request.getfixturevalue(f"{request.param}_grads")
+
+
+def test_backward_full_size_sampled_rows(full_grads):
+    cfg, got = full_grads
     inp = gc.inputs(cfg)
     r = gc.oracle_route(cfg)
     excluded = topk_gap(r.probs, cfg.k) < TIE_EPS
@@ -133,8 +147,8 @@ def test_backward_full_size_sampled_rows(qwen_grads):
     print("dx rows", grad_check(got["dx"][rows], ref, "dx (sampled rows)"))
 
 
-def test_backward_full_size_one_expert(qwen_grads):
-    cfg, got = qwen_grads
+def test_backward_full_size_one_expert(full_grads):
+    cfg, got = full_grads
     inp = gc.inputs(cfg)
     r = gc.oracle_route(cfg)
     counts = np.bincount(r.ids.ravel(), minlength=cfg.E)
