@@ -255,8 +255,10 @@ __device__ __forceinline__ int gather_token(const Params& p, int r)
 // not stored.  tbase addresses the accumulator at this warp's lane quarter.
 // kWeighted stages y through NBUF slab buffers of this warp (slab, in turn
 // by slab_buf): a buffer is rewritten once the store that last read it is
-// done, so up to NBUF stores per warp are in flight.
-template <int EPI, int NBUF = 2>
+// done, so up to NBUF stores per warp are in flight.  A slab is 32 rows x SC
+// fp16 columns (SC = 32: 64-byte rows, 64-byte swizzle; SC = 64: 128-byte
+// rows, 128-byte swizzle), the box of the caller's y map.
+template <int EPI, int NBUF = 2, int SC = kSlabCols>
 __device__ __forceinline__ void epilogue_tile(const Params& p, const CUtensorMap* tm_out, uint32_t tbase, int row0,
                                               int row_end, int nt, int q, int lane, int hf, float* slab,
                                               int& slab_buf)
@@ -300,8 +302,9 @@ __device__ __forceinline__ void epilogue_tile(const Params& p, const CUtensorMap
         }
     } else {
         // this warp: columns [cbeg, cbeg + 256 / kColGroups) of the tile, in
-        // slabs of 32 (two 16-column TMEM loads, the next slab in flight)
-        constexpr int kIters = kBN / kColGroups / kSlabCols;
+        // slabs of SC columns
+        constexpr int kIters = kBN / kColGroups / SC;
+        constexpr int kSlabB = 32 * SC * 2;
         const int cbeg = hf * (kBN / kColGroups);
         const float wgt = valid ? (p.w_perm ? __ldg(p.w_perm + row) : 1.0f) : 0.0f;  // no weights: one
         const int wrow0 = row0 + q * 32;                   // first row of this warp's slab
@@ -309,50 +312,94 @@ __device__ __forceinline__ void epilogue_tile(const Params& p, const CUtensorMap
         __half* orow = static_cast<__half*>(p.out) + (int64_t)row * p.n_out + nt * kBN;
         const int ncols = min(kBN, p.n_out - nt * kBN);
         bool bad = false;
-        uint32_t lo[2][16], hi[2][16];  // columns 0..15 and 16..31 of a slab
-        tmem_ld16(tbase + cbeg, lo[0]);
-        tmem_ld16(tbase + cbeg + 16, hi[0]);
-        tmem_ld_wait();
+        if constexpr (SC == 64) {
+#pragma unroll 1
+            for (int it = 0; it < kIters; ++it) {
+                const int c0 = cbeg + SC * it;
+                if (c0 < ncols) {  // warp-uniform (n_out % 64 == 0)
+                    uint32_t pk[32];
 #pragma unroll
-        for (int it = 0; it < kIters; ++it) {
-            const int c0 = cbeg + kSlabCols * it;
-            if (it + 1 < kIters) {
-                tmem_ld16(tbase + c0 + kSlabCols, lo[(it + 1) & 1]);
-                tmem_ld16(tbase + c0 + kSlabCols + 16, hi[(it + 1) & 1]);
-            }
-            const uint32_t* al = lo[it & 1];
-            const uint32_t* ah = hi[it & 1];
-            if (c0 < ncols) {  // warp-uniform (n_out % 64 == 0)
-                uint32_t pk[16];
+                    for (int h4 = 0; h4 < 4; h4 += 2) {
+                        uint32_t a0[16], a1[16];
+                        tmem_ld16(tbase + c0 + 16 * h4, a0);
+                        tmem_ld16(tbase + c0 + 16 * h4 + 16, a1);
+                        tmem_ld_wait();
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    pk[i] = scaled_f16x2(wgt, al[2 * i], al[2 * i + 1], bad);
-                    pk[8 + i] = scaled_f16x2(wgt, ah[2 * i], ah[2 * i + 1], bad);
-                }
-                if (whole) {
-                    uint32_t* buf = reinterpret_cast<uint32_t*>(slab) + slab_buf * (kSlabBytes / 4);
-                    if (lane == 0) bulk_wait_group_read<NBUF - 1>();  // the store that last read `buf` is done
-                    __syncwarp();
-                    // row `lane` of the slab: 4 x 16 B chunks, 64-byte swizzle
-                    uint4* rowp = reinterpret_cast<uint4*>(buf + lane * (kSlabCols / 2));
-                    const int sw = (lane >> 1) & 3;
-#pragma unroll
-                    for (int v = 0; v < 4; ++v)
-                        rowp[v ^ sw] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                    if (lane == 0) {
-                        tma_store_2d(tm_out, buf, nt * kBN + c0, wrow0);
-                        bulk_commit_group();
+                        for (int i = 0; i < 8; ++i) {
+                            pk[8 * h4 + i] = scaled_f16x2(wgt, a0[2 * i], a0[2 * i + 1], bad);
+                            pk[8 * h4 + 8 + i] = scaled_f16x2(wgt, a1[2 * i], a1[2 * i + 1], bad);
+                        }
                     }
-                    slab_buf = slab_buf + 1 == NBUF ? 0 : slab_buf + 1;
-                } else if (valid) {
-                    uint4* dst = reinterpret_cast<uint4*>(orow + c0);
+                    if (whole) {
+                        uint32_t* buf = reinterpret_cast<uint32_t*>(slab) + slab_buf * (kSlabB / 4);
+                        if (lane == 0) bulk_wait_group_read<NBUF - 1>();  // the store that last read `buf` is done
+                        __syncwarp();
+                        // row `lane` of the slab: 8 x 16 B chunks, 128-byte swizzle
+                        uint4* rowp = reinterpret_cast<uint4*>(buf + lane * (SC / 2));
+                        const int sw = lane & 7;
 #pragma unroll
-                    for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+                        for (int v = 0; v < 8; ++v)
+                            rowp[v ^ sw] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) {
+                            tma_store_2d(tm_out, buf, nt * kBN + c0, wrow0);
+                            bulk_commit_group();
+                        }
+                        slab_buf = slab_buf + 1 == NBUF ? 0 : slab_buf + 1;
+                    } else if (valid) {
+                        uint4* dst = reinterpret_cast<uint4*>(orow + c0);
+#pragma unroll
+                        for (int v = 0; v < 8; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+                    }
                 }
             }
+        } else {
+            uint32_t lo[2][16], hi[2][16];  // columns 0..15 and 16..31 of a slab
+            tmem_ld16(tbase + cbeg, lo[0]);
+            tmem_ld16(tbase + cbeg + 16, hi[0]);
             tmem_ld_wait();
+#pragma unroll
+            for (int it = 0; it < kIters; ++it) {
+                const int c0 = cbeg + SC * it;
+                if (it + 1 < kIters) {
+                    tmem_ld16(tbase + c0 + SC, lo[(it + 1) & 1]);
+                    tmem_ld16(tbase + c0 + SC + 16, hi[(it + 1) & 1]);
+                }
+                const uint32_t* al = lo[it & 1];
+                const uint32_t* ah = hi[it & 1];
+                if (c0 < ncols) {  // warp-uniform (n_out % 64 == 0)
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        pk[i] = scaled_f16x2(wgt, al[2 * i], al[2 * i + 1], bad);
+                        pk[8 + i] = scaled_f16x2(wgt, ah[2 * i], ah[2 * i + 1], bad);
+                    }
+                    if (whole) {
+                        uint32_t* buf = reinterpret_cast<uint32_t*>(slab) + slab_buf * (kSlabB / 4);
+                        if (lane == 0) bulk_wait_group_read<NBUF - 1>();  // the store that last read `buf` is done
+                        __syncwarp();
+                        // row `lane` of the slab: 4 x 16 B chunks, 64-byte swizzle
+                        uint4* rowp = reinterpret_cast<uint4*>(buf + lane * (SC / 2));
+                        const int sw = (lane >> 1) & 3;
+#pragma unroll
+                        for (int v = 0; v < 4; ++v)
+                            rowp[v ^ sw] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) {
+                            tma_store_2d(tm_out, buf, nt * kBN + c0, wrow0);
+                            bulk_commit_group();
+                        }
+                        slab_buf = slab_buf + 1 == NBUF ? 0 : slab_buf + 1;
+                    } else if (valid) {
+                        uint4* dst = reinterpret_cast<uint4*>(orow + c0);
+#pragma unroll
+                        for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+                    }
+                }
+                tmem_ld_wait();
+            }
         }
         if (__any_sync(0xffffffffu, bad && valid) && lane == 0) record_status(kStatusDeviceRange);
     }

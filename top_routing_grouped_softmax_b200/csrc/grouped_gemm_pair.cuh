@@ -48,16 +48,24 @@ constexpr int kPairSlabBufs = MOE_PAIR_SLAB_BUFS;
 static_assert(MOE_PAIR_DOWN_STAGES >= 2 && MOE_PAIR_DOWN_STAGES <= kPairStages, "down ring depth");
 static_assert(kPairSlabBufs >= 1 && kPairSlabBufs <= 8, "slab buffers per epilogue warp");
 
-template <int EPI>
+// The down kernel's y slabs are 32 x SC fp16: SC = 32 by default; SC = 64
+// (128-byte rows, half as many fences and stores per tile, with a five-stage
+// ring to make room) where the reduction is short (f <= kDownShortK), whose
+// tiles are bound by their epilogue: 7 % off that layer's down GEMM, while
+// a long K lost the ring stage (qwen's down GEMM 5 us slower).
+constexpr int kDownShortK = 512;
+constexpr int kDownShortKStages = 5;
+
+template <int EPI, int SC = kSlabCols>
 __host__ __device__ constexpr int pair_stages()
 {
-    return EPI == kWeighted ? MOE_PAIR_DOWN_STAGES : kPairStages;
+    return EPI == kWeighted ? (SC == 64 ? kDownShortKStages : MOE_PAIR_DOWN_STAGES) : kPairStages;
 }
 
-template <int EPI>
+template <int EPI, int SC = kSlabCols>
 __host__ __device__ constexpr int pair_store_bytes()
 {
-    return EPI == kWeighted ? kEpiWarps * kPairSlabBufs * kSlabBytes : 0;
+    return EPI == kWeighted ? kEpiWarps * kPairSlabBufs * (32 * SC * 2) : 0;
 }
 
 struct alignas(8) PairCtrl {
@@ -74,18 +82,21 @@ struct alignas(8) PairCtrl {
     int tp[kMaxE + 1];
 };
 
-template <int EPI>
+template <int EPI, int SC = kSlabCols>
 __host__ inline size_t pair_smem_bytes()
 {
-    return 1024 + (size_t)pair_stages<EPI>() * kPairStageBytes + pair_store_bytes<EPI>() + sizeof(PairCtrl);
+    return 1024 + (size_t)pair_stages<EPI, SC>() * kPairStageBytes + pair_store_bytes<EPI, SC>() + sizeof(PairCtrl);
 }
 static_assert(1024 + (size_t)pair_stages<kSwiGLU>() * kPairStageBytes + sizeof(PairCtrl) <= 227 * 1024,
               "gate/up pair ring and control exceed 227 KB of shared memory");
 static_assert(1024 + (size_t)pair_stages<kWeighted>() * kPairStageBytes + pair_store_bytes<kWeighted>() +
                       sizeof(PairCtrl) <= 227 * 1024,
               "down pair ring, staging and control exceed 227 KB of shared memory");
+static_assert(1024 + (size_t)pair_stages<kWeighted, 64>() * kPairStageBytes + pair_store_bytes<kWeighted, 64>() +
+                      sizeof(PairCtrl) <= 227 * 1024,
+              "down pair ring, staging and control exceed 227 KB of shared memory (short-K form)");
 
-template <int EPI>
+template <int EPI, int SC = kSlabCols>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b0,
                              const __grid_constant__ CUtensorMap tm_b1, const __grid_constant__ CUtensorMap tm_out,
@@ -93,9 +104,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    constexpr int NS = pair_stages<EPI>();
+    constexpr int NS = pair_stages<EPI, SC>();
     uint8_t* stage_out = smem + (size_t)NS * kPairStageBytes;
-    PairCtrl& c = *reinterpret_cast<PairCtrl*>(stage_out + pair_store_bytes<EPI>());
+    PairCtrl& c = *reinterpret_cast<PairCtrl*>(stage_out + pair_store_bytes<EPI, SC>());
 
     const int warp = threadIdx.x / 32;
     const int lane = threadIdx.x % 32;
@@ -249,7 +260,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int ew = warp - 2;
         const int q = warp & 3;
         const int hf = ew >> 2;
-        float* slab = reinterpret_cast<float*>(stage_out + ew * kPairSlabBufs * kSlabBytes);
+        float* slab = reinterpret_cast<float*>(stage_out + ew * kPairSlabBufs * (32 * SC * 2));
         int slab_buf = 0;
         int acc = 0;
         uint32_t acc_ph = 0;
@@ -265,8 +276,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             tc_fence_after_sync();
             const uint32_t tbase = tmem + (uint32_t)(acc * kBN) + ((uint32_t)(q * 32) << 16);
-            epilogue_tile<EPI, kPairSlabBufs>(p, &tm_out, tbase, row0 + (int)rank * kBM, row_end, nt, q, lane, hf, slab,
-                                              slab_buf);
+            epilogue_tile<EPI, kPairSlabBufs, SC>(p, &tm_out, tbase, row0 + (int)rank * kBM, row_end, nt, q, lane, hf,
+                                                  slab, slab_buf);
             tc_fence_before_sync();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(mapa_shared(&c.acc_empty[acc], 0));

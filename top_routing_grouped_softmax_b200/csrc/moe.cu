@@ -145,15 +145,15 @@ int launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStr
     return cudaLaunchKernelEx(&cfg, kernel, args...) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
-template <int EPI>
+template <int EPI, int SC = moe::gemm::kSlabCols>
 int launch_pair_gemm(const DeviceState& st, int64_t work, const CUtensorMap& ta, const CUtensorMap& tb0,
                      const CUtensorMap& tb1, const CUtensorMap& tout, const moe::gemm::Params& p, cudaStream_t s)
 {
     int64_t pairs = st.max_pairs > 0 ? st.max_pairs : st.sm_count / 2;
     if (work < pairs) pairs = work;
     if (pairs < 1) pairs = 1;
-    return launch(moe::gemm::grouped_gemm_pair_kernel<EPI>, dim3((unsigned)(2 * pairs)), dim3(moe::gemm::kThreads),
-                  moe::gemm::pair_smem_bytes<EPI>(), s, 2u, ta, tb0, tb1, tout, p);
+    return launch(moe::gemm::grouped_gemm_pair_kernel<EPI, SC>, dim3((unsigned)(2 * pairs)),
+                  dim3(moe::gemm::kThreads), moe::gemm::pair_smem_bytes<EPI, SC>(), s, 2u, ta, tb0, tb1, tout, p);
 }
 
 int setup_device(DeviceState** out)
@@ -195,6 +195,7 @@ int setup_device(DeviceState** out)
             e = e ? e : cudaFuncSetAttribute(moe::gemm::grouped_gemm_kernel<moe::gemm::kWeighted, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
             e = e ? e : cudaFuncSetAttribute(moe::gemm::grouped_gemm_pair_kernel<moe::gemm::kSwiGLU>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
             e = e ? e : cudaFuncSetAttribute(moe::gemm::grouped_gemm_pair_kernel<moe::gemm::kWeighted>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
+            e = e ? e : cudaFuncSetAttribute(moe::gemm::grouped_gemm_pair_kernel<moe::gemm::kWeighted, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
             e = e ? e : cudaFuncSetAttribute(moe::bwd::pair_bwd_kernel<moe::bwd::kGU>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
             e = e ? e : cudaFuncSetAttribute(moe::bwd::pair_bwd_kernel<moe::bwd::kDH>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
             e = e ? e : cudaFuncSetAttribute(moe::bwd::pair_bwd_kernel<moe::bwd::kDX>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
@@ -523,7 +524,16 @@ int run_ffn(const DeviceState& st, const moe_bf16* x_perm, const moe_bf16* x_gat
     p2.m_capacity = m_capacity ? 1 : 0;
     const int64_t work2 = max_mtiles * p2.n_tiles;
     const unsigned grid2 = (unsigned)(work2 < st.sm_count ? work2 : st.sm_count);
-    if (MOE_GEMM_PAIR) return launch_pair_gemm<kWeighted>(st, max_pair_tiles * p2.n_tiles, ta2, td3, td3, ty, p2, s);
+    if (MOE_GEMM_PAIR) {
+        if (f <= kDownShortK) {  // y through 32 x 64 slabs (128-byte rows)
+            CUtensorMap ty64;
+            if (make_map(&ty64, y, (uint64_t)d, (uint64_t)M, 64, 32, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+                         CU_TENSOR_MAP_SWIZZLE_128B))
+                return MOE_ERR_CUDA;
+            return launch_pair_gemm<kWeighted, 64>(st, max_pair_tiles * p2.n_tiles, ta2, td3, td3, ty64, p2, s);
+        }
+        return launch_pair_gemm<kWeighted>(st, max_pair_tiles * p2.n_tiles, ta2, td3, td3, ty, p2, s);
+    }
     return launch(grouped_gemm_kernel<kWeighted, false>, dim3(grid2), dim3(kThreads), smem2, s, 1u, ta2, td, td, ty,
                   p2);
 }
