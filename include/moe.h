@@ -278,10 +278,11 @@ int moe_forward(const moe_bf16* x, const moe_bf16* w_router, const float* bias,
  * MOE_FLAG_RENORMALIZE and MOE_FLAG_OUT_F16 the arithmetic is identical to
  * moe_forward.
  *
- * Every kernel of the library is launched with programmatic dependent
- * launch: it may begin launching while the previous kernel on the stream
- * drains, and waits for that kernel's completion before its first global
- * memory access.
+ * Every kernel of the library but the combine is launched with
+ * programmatic dependent launch: it may begin launching while the previous
+ * kernel on the stream drains, and waits for that kernel's completion before
+ * its first global memory access.  The combine starts after the down GEMM
+ * ends (waiting beside the GEMM's CTAs measured slower).
  */
 int moe_forward_ex(const moe_bf16* x, const moe_bf16* w_router, const float* bias,
                    const moe_bf16* w_gate, const moe_bf16* w_up, const moe_bf16* w_down,

@@ -32,7 +32,8 @@ __device__ __forceinline__ void add_f16x8(float (&acc)[8], const uint4& q)
 }
 
 // One block per token; thread v handles 8 consecutive columns (16 bytes of
-// y, 32 bytes of out).  With shared experts (n_s > 0), their rows
+// y, 32 bytes of out), with all k <= 8 row loads in flight at once.  The
+// kernel is launched after the down GEMM ends, not early beside its CTAs.  With shared experts (n_s > 0), their rows
 // y_s[s][t] (weight one, already applied) are added after the k routed
 // slots, in ascending s.  F16OUT: the fp32 sum is rounded to fp16 once, at
 // the store (16 bytes of out per thread); a value whose rounding leaves the
@@ -60,10 +61,23 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint4* __restrict__ 
         float acc[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
+        if (k <= 8) {
+            // every slot's load in flight before the sums (slot order kept)
+            uint4 q[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int p = j < k ? s_pos[j] : -1;
+                q[j] = p >= 0 ? __ldg(y + (int64_t)p * nvec + v) : make_uint4(0u, 0u, 0u, 0u);
+            }
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                if (j < k && s_pos[j] >= 0) add_f16x8(acc, q[j]);
+        } else {
 #pragma unroll 4
-        for (int j = 0; j < k; ++j) {
-            const int p = s_pos[j];
-            if (p >= 0) add_f16x8(acc, __ldg(y + (int64_t)p * nvec + v));
+            for (int j = 0; j < k; ++j) {
+                const int p = s_pos[j];
+                if (p >= 0) add_f16x8(acc, __ldg(y + (int64_t)p * nvec + v));
+            }
         }
         for (int sh = 0; sh < n_s; ++sh) add_f16x8(acc, __ldg(y_s + ((int64_t)sh * T + t) * nvec + v));
         if constexpr (F16OUT) {
