@@ -392,22 +392,29 @@ int moe_forward_rounded(const moe_bf16* x, const moe_bf16* w_router, const float
  *   dW_router  += x[t]^T dlogit,  dbias += dlogit,  dx[t] += dlogit . W_router^T
  * The top-k choice itself passes no gradient.
  *   dout [T, d] fp32 in; dx [T, d] fp32 out; dw_router [d, E], dbias [E]
- *   (NULL to skip), dw_gate / dw_up [E, d, f], dw_down [E, f, d]: fp32 out,
- *   overwritten (experts no token selects get zeros).  All 16-byte aligned.
+ *   (NULL to skip), dw_gate / dw_up [E, d, f], dw_down [E, f, d]: fp32 out
+ *   (with MOE_FLAG_GRAD_BF16: dw_router, dw_gate, dw_up and dw_down bf16,
+ *   each the fp32 result rounded once; dx and dbias stay fp32), overwritten
+ *   (experts no token selects get zeros).  All 16-byte aligned.
  * Precision: the GEMM operands are bf16 (x, the weights, dout, dg, du, w h
  * and dlogit rounded once each), every sum fp32; each slot's contribution
  * to dx (dg . W_gate^T + du . W_up^T) is rounded to bf16 once before the
- * fp32 sum over the token's k slots.  flags: 0 or
- * MOE_FLAG_RENORMALIZE (the routing the forward used).  Workspace:
+ * fp32 sum over the token's k slots.  flags: any of MOE_FLAG_RENORMALIZE
+ * (the routing the forward used) and MOE_FLAG_GRAD_BF16.  Workspace:
  * moe_backward_workspace_size bytes, 256-byte aligned; grouped rows are
  * padded so that each expert's group starts on a 64-row boundary.
  */
 size_t moe_backward_workspace_size(int64_t T, int64_t d, int64_t E, int64_t k, int64_t f);
 
+/* moe_backward flag: the weight gradients are bf16 (the fp32 accumulators
+ * rounded to nearest even once, at the store), half the bytes of the
+ * weight-gradient GEMMs' outputs, which bound those GEMMs' time. */
+#define MOE_FLAG_GRAD_BF16 8u
+
 int moe_backward(const moe_bf16* x, const moe_bf16* w_router, const float* bias,
                  const moe_bf16* w_gate, const moe_bf16* w_up, const moe_bf16* w_down, const float* dout,
                  int64_t T, int64_t d, int64_t E, int64_t k, int64_t f,
-                 float* dx, float* dw_router, float* dbias, float* dw_gate, float* dw_up, float* dw_down,
+                 float* dx, void* dw_router, float* dbias, void* dw_gate, void* dw_up, void* dw_down,
                  void* workspace, size_t workspace_bytes, cudaStream_t stream, unsigned flags);
 
 /*

@@ -180,3 +180,35 @@ def test_backward_full_size_properties(qwen_grads):
     # in fp32 from the unrounded dlogit) sums to zero up to fp32 rounding
     db = got["dbias"].astype(np.float64)
     assert abs(db.sum()) <= 2.0 ** -8 * np.abs(db).sum() + 1e-6
+
+
+def _run_dtype(cfg, grad_dtype):
+    inp = gc.inputs(cfg)
+    d = gc.on_device(inp)
+    dout = make_dout(cfg.T, cfg.d, cfg.seed).cuda()
+    g = moe.backward(d["x"], d["w_router"], d["w_gate"], d["w_up"], d["w_down"], cfg.k, dout, bias=d["bias"],
+                     grad_dtype=grad_dtype)
+    torch.cuda.synchronize()
+    assert moe.get_status() == moe.MOE_OK
+    return g
+
+
+@pytest.mark.parametrize("cfg", [SMALL[0][0], SMALL[1][0], CONFIGS["qwen"]], ids=lambda c: c.name)
+def test_backward_bf16_weight_gradients_are_rounded_fp32(cfg):
+    """MOE_FLAG_GRAD_BF16: each weight gradient is the fp32 one rounded to
+    bf16 once, bit for bit; dx and dbias are unchanged; the bf16 gradients
+    are within the backward's criteria of the oracle on a small shape."""
+    g32 = _run_dtype(cfg, torch.float32)
+    g16 = _run_dtype(cfg, torch.bfloat16)
+    for n in ("dw_router", "dw_gate", "dw_up", "dw_down"):
+        assert g16[n].dtype == torch.bfloat16
+        assert torch.equal(g16[n], g32[n].to(torch.bfloat16)), n
+    for n in ("dx", "dbias"):
+        assert torch.equal(g16[n], g32[n]), n
+    if cfg.T <= 1000:
+        inp = gc.inputs(cfg)
+        dout = make_dout(cfg.T, cfg.d, cfg.seed).numpy().astype(np.float64)
+        ref = default_oracle().backward(inp.bits("x"), inp.bits("W_router"), inp.bias_np(), inp.bits("W_gate"),
+                                        inp.bits("W_up"), inp.bits("W_down"), cfg.k, dout)
+        for n in ("dw_router", "dw_gate", "dw_up", "dw_down"):
+            grad_check(g16[n].float().cpu().numpy(), getattr(ref, n), f"{n} (bf16)")

@@ -339,6 +339,7 @@ def _forward_args(x, w_router, w_gate, w_up, w_down, bias):
 MOE_FLAG_FUSED_GATHER = 1
 MOE_FLAG_RENORMALIZE = 2
 MOE_FLAG_OUT_F16 = 4
+MOE_FLAG_GRAD_BF16 = 8
 
 
 def forward(x, w_router, w_gate, w_up, w_down, k, bias=None, out=None, workspace=None,
@@ -395,27 +396,32 @@ def backward_workspace_size(T: int, d: int, E: int, k: int, f: int) -> int:
 
 
 def backward(x, w_router, w_gate, w_up, w_down, k, dout, bias=None, workspace=None, renormalize=False,
-             want_dbias=True):
+             want_dbias=True, grad_dtype=torch.float32):
     """Gradient of sum(dout * out) of the block (moe_backward): returns a dict
-    of fp32 tensors dx [T, d], dw_router [d, E], dbias [E] (None unless
-    want_dbias), dw_gate / dw_up [E, d, f], dw_down [E, f, d]."""
+    of tensors dx [T, d] fp32, dw_router [d, E], dbias [E] fp32 (None unless
+    want_dbias), dw_gate / dw_up [E, d, f], dw_down [E, f, d].  The four
+    weight gradients are fp32, or bf16 with grad_dtype=torch.bfloat16
+    (MOE_FLAG_GRAD_BF16: the fp32 results rounded once)."""
     T, d, E, f = _forward_args(x, w_router, w_gate, w_up, w_down, bias)
     _need(dout, "dout", torch.float32, 2)
+    if grad_dtype not in (torch.float32, torch.bfloat16):
+        raise ValueError("grad_dtype: torch.float32 or torch.bfloat16")
     dev = x.device
+    gd = grad_dtype
     g = {
         "dx": torch.empty(T, d, dtype=torch.float32, device=dev),
-        "dw_router": torch.empty(d, E, dtype=torch.float32, device=dev),
+        "dw_router": torch.empty(d, E, dtype=gd, device=dev),
         "dbias": torch.empty(E, dtype=torch.float32, device=dev) if want_dbias else None,
-        "dw_gate": torch.empty(E, d, f, dtype=torch.float32, device=dev),
-        "dw_up": torch.empty(E, d, f, dtype=torch.float32, device=dev),
-        "dw_down": torch.empty(E, f, d, dtype=torch.float32, device=dev),
+        "dw_gate": torch.empty(E, d, f, dtype=gd, device=dev),
+        "dw_up": torch.empty(E, d, f, dtype=gd, device=dev),
+        "dw_down": torch.empty(E, f, d, dtype=gd, device=dev),
     }
     nbytes = backward_workspace_size(T, d, E, k, f)
     if nbytes == 0:
         raise MoEError(MOE_ERR_UNSUPPORTED_SHAPE, "moe_backward_workspace_size")
     if workspace is None:
         workspace = _workspace(nbytes, dev)
-    flags = MOE_FLAG_RENORMALIZE if renormalize else 0
+    flags = (MOE_FLAG_RENORMALIZE if renormalize else 0) | (MOE_FLAG_GRAD_BF16 if gd == torch.bfloat16 else 0)
     _check(lib().moe_backward(_ptr(x), _ptr(w_router), _ptr(bias), _ptr(w_gate), _ptr(w_up), _ptr(w_down),
                               _ptr(dout), T, d, E, k, f, _ptr(g["dx"]), _ptr(g["dw_router"]), _ptr(g["dbias"]),
                               _ptr(g["dw_gate"]), _ptr(g["dw_up"]), _ptr(g["dw_down"]), _ptr(workspace),
@@ -477,7 +483,7 @@ class MoEBlock:
 
 __all__ = [
     "lib", "strerror", "MoEError", "ABI_SYMBOLS", "workspace_size", "route_workspace_size",
-    "permute_workspace_size", "MOE_FLAG_FUSED_GATHER", "MOE_FLAG_RENORMALIZE", "MOE_FLAG_OUT_F16", "route",
+    "permute_workspace_size", "MOE_FLAG_FUSED_GATHER", "MOE_FLAG_RENORMALIZE", "MOE_FLAG_OUT_F16", "MOE_FLAG_GRAD_BF16", "route",
     "permute", "expert_ffn", "combine", "forward", "shared_ffn", "combine_shared", "forward_shared", "forward_rounded",
     "get_status", "set_wait_limit_ns", "backward", "backward_workspace_size", "gather_rows",
     "selftest_wait_timeout", "MoEBlock",

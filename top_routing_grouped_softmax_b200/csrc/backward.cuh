@@ -185,8 +185,10 @@ __global__ void __launch_bounds__(kRowThreads) colsum_kernel(const float* __rest
 
 // out[i] = sum over s = 0..S-1 of part[s][i], in ascending s (fp32): the
 // split-K partial products of the router's weight gradient.  n4 = elements / 4.
+// BF16OUT: the fp32 sum rounded to bf16 once.
+template <bool BF16OUT>
 __global__ void __launch_bounds__(kRowThreads) sum_partials_kernel(const float4* __restrict__ part, int S,
-                                                                   int64_t n4, float4* __restrict__ out)
+                                                                   int64_t n4, void* __restrict__ out)
 {
     pdl_trigger();
     pdl_wait();
@@ -199,7 +201,10 @@ __global__ void __launch_bounds__(kRowThreads) sum_partials_kernel(const float4*
             acc.z += a.z;
             acc.w += a.w;
         }
-        out[i] = acc;
+        if constexpr (BF16OUT)
+            static_cast<uint2*>(out)[i] = make_uint2(gemm::pack_bf16x2(acc.x, acc.y), gemm::pack_bf16x2(acc.z, acc.w));
+        else
+            static_cast<float4*>(out)[i] = acc;
     }
 }
 

@@ -91,7 +91,8 @@ struct Params {
     int m_total;             // kDW: output rows per expert
     int m_tiles;             // kDW: 256-row M tiles per expert
     int split_b;             // kDW: 1 = B halves from two tensors (dg | du), two outputs
-    int out_bf16;            // kDX: 1 = out0 holds bf16 values (rows of ld_out), stored through a 2-D map
+    int out_bf16;            // kDX: 1 = out0 holds bf16 values (rows of ld_out), stored through a 2-D map;
+                             // kDW: 1 = out0 / out1 hold bf16 values (32 x 32 slabs of 2 KB, 64-byte swizzle)
     int k_chunk;             // kDW: > 0 = group e is rows [e k_chunk, min((e + 1) k_chunk, M)) of one
                              // M-row operand pair (split K; offsets unused), else the offsets' groups
 };
@@ -462,15 +463,31 @@ __device__ __forceinline__ void epilogue(const Params& p, const Item& it, uint32
             uint32_t* buf = reinterpret_cast<uint32_t*>(slab) + slab_buf * (kSlabBytes / 4);
             if (lane == 0) bulk_wait_group_read<kSlabBufs - 1>();  // the store that last read `buf` is done
             __syncwarp();
-            // row `lane` of the slab: 8 x 16 B chunks, 128-byte swizzle
-            uint4* rowp = reinterpret_cast<uint4*>(buf + lane * 32);
-            const int sw = lane & 7;
+            if (p.out_bf16) {
+                // row `lane` of a 32 x 32 bf16 slab: 4 x 16 B chunks, 64-byte swizzle
+                uint32_t pk[16];
 #pragma unroll
-            for (int v = 0; v < 4; ++v) {
-                rowp[v ^ sw] = empty ? make_uint4(0u, 0u, 0u, 0u)
-                                     : make_uint4(lo[4 * v], lo[4 * v + 1], lo[4 * v + 2], lo[4 * v + 3]);
-                rowp[(4 + v) ^ sw] = empty ? make_uint4(0u, 0u, 0u, 0u)
-                                           : make_uint4(hi[4 * v], hi[4 * v + 1], hi[4 * v + 2], hi[4 * v + 3]);
+                for (int i = 0; i < 8; ++i) {
+                    pk[i] = empty ? 0u : gemm::pack_bf16x2(__uint_as_float(lo[2 * i]), __uint_as_float(lo[2 * i + 1]));
+                    pk[8 + i] = empty ? 0u
+                                      : gemm::pack_bf16x2(__uint_as_float(hi[2 * i]), __uint_as_float(hi[2 * i + 1]));
+                }
+                uint4* rowp = reinterpret_cast<uint4*>(buf + lane * 16);
+                const int sw = (lane >> 1) & 3;
+#pragma unroll
+                for (int v = 0; v < 4; ++v)
+                    rowp[v ^ sw] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+            } else {
+                // row `lane` of the slab: 8 x 16 B chunks, 128-byte swizzle
+                uint4* rowp = reinterpret_cast<uint4*>(buf + lane * 32);
+                const int sw = lane & 7;
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                    rowp[v ^ sw] = empty ? make_uint4(0u, 0u, 0u, 0u)
+                                         : make_uint4(lo[4 * v], lo[4 * v + 1], lo[4 * v + 2], lo[4 * v + 3]);
+                    rowp[(4 + v) ^ sw] = empty ? make_uint4(0u, 0u, 0u, 0u)
+                                               : make_uint4(hi[4 * v], hi[4 * v + 1], hi[4 * v + 2], hi[4 * v + 3]);
+                }
             }
             fence_proxy_async_smem();
             __syncwarp();

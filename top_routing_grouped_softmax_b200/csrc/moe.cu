@@ -865,6 +865,19 @@ int launch_pair_bwd(const DeviceState& st, int64_t work, const CUtensorMap& ta, 
 
 // fp32 [groups][rows][cols] viewed for 32 x 32 TMA stores (128-byte swizzle);
 // elements outside the extents are clipped by the store.
+// bf16 [groups][rows][cols] for the same 32 x 32 stores (2 KB, 64-byte swizzle).
+int make_out3_map_bf16(CUtensorMap* m, void* base, uint64_t cols, uint64_t rows, uint64_t groups)
+{
+    cuuint64_t dims[3] = {cols, rows, groups};
+    cuuint64_t strides[2] = {cols * 2, rows * cols * 2};
+    cuuint32_t box[3] = {32, 32, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
+}
+
 int make_out3_map(CUtensorMap* m, float* base, uint64_t cols, uint64_t rows, uint64_t groups)
 {
     cuuint64_t dims[3] = {cols, rows, groups};
@@ -886,13 +899,15 @@ moe::bwd::Params bwd_params()
 
 int backward_impl(const moe_bf16* x, const moe_bf16* w_router, const float* bias, const moe_bf16* w_gate,
                   const moe_bf16* w_up, const moe_bf16* w_down, const float* dout, int64_t T, int64_t d, int64_t E,
-                  int64_t k, int64_t f, float* dx, float* dw_router, float* dbias, float* dw_gate, float* dw_up,
-                  float* dw_down, void* ws, size_t ws_bytes, cudaStream_t s, unsigned flags)
+                  int64_t k, int64_t f, float* dx, void* dw_router, float* dbias, void* dw_gate, void* dw_up,
+                  void* dw_down, void* ws, size_t ws_bytes, cudaStream_t s, unsigned flags)
 {
     int rc = check_common(T, d, E, k);
     if (rc) return rc;
     if ((rc = check_f(f))) return rc;
-    if (flags & ~(unsigned)MOE_FLAG_RENORMALIZE) return MOE_ERR_INVALID_ARG;
+    if (flags & ~(unsigned)(MOE_FLAG_RENORMALIZE | MOE_FLAG_GRAD_BF16)) return MOE_ERR_INVALID_ARG;
+    const bool grad_bf16 = (flags & MOE_FLAG_GRAD_BF16) != 0;
+    const size_t gbytes = grad_bf16 ? 2 : 4;  // bytes per weight-gradient element
     if (!w_router || !w_gate || !w_up || !w_down || !dw_router || !dw_gate || !dw_up || !dw_down)
         return MOE_ERR_INVALID_ARG;
     if (T > 0 && (!x || !dout || !dx)) return MOE_ERR_INVALID_ARG;
@@ -909,10 +924,10 @@ int backward_impl(const moe_bf16* x, const moe_bf16* w_router, const float* bias
     if ((rc = setup_device(&st))) return rc;
     if (T == 0) {
         // no tokens: every weight gradient is zero
-        const size_t we = (size_t)E * (size_t)d * (size_t)f * 4;
+        const size_t we = (size_t)E * (size_t)d * (size_t)f * gbytes;
         if (cudaMemsetAsync(dw_gate, 0, we, s) != cudaSuccess || cudaMemsetAsync(dw_up, 0, we, s) != cudaSuccess ||
             cudaMemsetAsync(dw_down, 0, we, s) != cudaSuccess ||
-            cudaMemsetAsync(dw_router, 0, (size_t)d * (size_t)E * 4, s) != cudaSuccess ||
+            cudaMemsetAsync(dw_router, 0, (size_t)d * (size_t)E * gbytes, s) != cudaSuccess ||
             (dbias && cudaMemsetAsync(dbias, 0, (size_t)E * 4, s) != cudaSuccess))
             return MOE_ERR_CUDA;
         return MOE_OK;
@@ -1055,13 +1070,19 @@ int backward_impl(const moe_bf16* x, const moe_bf16* w_router, const float* bias
         rc = make_weight_chunk_map(&ta, x_perm, (uint64_t)d, (uint64_t)R);
         rc = rc ? rc : make_weight_chunk_map(&tb0, g, (uint64_t)f, (uint64_t)R);
         rc = rc ? rc : make_weight_chunk_map(&tb1, u, (uint64_t)f, (uint64_t)R);
-        rc = rc ? rc : make_out3_map(&to0, dw_gate, (uint64_t)f, (uint64_t)d, (uint64_t)E);
-        rc = rc ? rc : make_out3_map(&to1, dw_up, (uint64_t)f, (uint64_t)d, (uint64_t)E);
+        if (grad_bf16) {
+            rc = rc ? rc : make_out3_map_bf16(&to0, dw_gate, (uint64_t)f, (uint64_t)d, (uint64_t)E);
+            rc = rc ? rc : make_out3_map_bf16(&to1, dw_up, (uint64_t)f, (uint64_t)d, (uint64_t)E);
+        } else {
+            rc = rc ? rc : make_out3_map(&to0, static_cast<float*>(dw_gate), (uint64_t)f, (uint64_t)d, (uint64_t)E);
+            rc = rc ? rc : make_out3_map(&to1, static_cast<float*>(dw_up), (uint64_t)f, (uint64_t)d, (uint64_t)E);
+        }
         if (rc) return rc;
         Params p = bwd_params();
         p.offsets = offsets;
-        p.out0 = dw_gate;
-        p.out1 = dw_up;
+        p.out0 = static_cast<float*>(dw_gate);
+        p.out1 = static_cast<float*>(dw_up);
+        p.out_bf16 = grad_bf16 ? 1 : 0;
         p.ld_out = f;
         p.E = iE;
         p.M = (int)R;
@@ -1078,11 +1099,15 @@ int backward_impl(const moe_bf16* x, const moe_bf16* w_router, const float* bias
         CUtensorMap ta, tb, to0;
         rc = make_weight_chunk_map(&ta, hw, (uint64_t)f, (uint64_t)R);
         rc = rc ? rc : make_weight_chunk_map(&tb, dout_perm, (uint64_t)d, (uint64_t)R);
-        rc = rc ? rc : make_out3_map(&to0, dw_down, (uint64_t)d, (uint64_t)f, (uint64_t)E);
+        rc = rc ? rc
+                : (grad_bf16 ? make_out3_map_bf16(&to0, dw_down, (uint64_t)d, (uint64_t)f, (uint64_t)E)
+                             : make_out3_map(&to0, static_cast<float*>(dw_down), (uint64_t)d, (uint64_t)f,
+                                             (uint64_t)E));
         if (rc) return rc;
         Params p = bwd_params();
         p.offsets = offsets;
-        p.out0 = dw_down;
+        p.out0 = static_cast<float*>(dw_down);
+        p.out_bf16 = grad_bf16 ? 1 : 0;
         p.ld_out = d;
         p.E = iE;
         p.M = (int)R;
@@ -1138,8 +1163,11 @@ int backward_impl(const moe_bf16* x, const moe_bf16* w_router, const float* bias
             return MOE_ERR_CUDA;
         const int64_t n4 = d * E / 4;
         const unsigned blocks = (unsigned)((n4 + kRowThreads - 1) / kRowThreads);
-        if (launch(sum_partials_kernel, dim3(blocks < 1184u ? blocks : 1184u), dim3(kRowThreads), 0, s, 1u,
-                   reinterpret_cast<const float4*>(part), (int)S, n4, reinterpret_cast<float4*>(dw_router)))
+        const dim3 grid(blocks < 1184u ? blocks : 1184u);
+        if (grad_bf16 ? launch(sum_partials_kernel<true>, grid, dim3(kRowThreads), 0, s, 1u,
+                               reinterpret_cast<const float4*>(part), (int)S, n4, dw_router)
+                      : launch(sum_partials_kernel<false>, grid, dim3(kRowThreads), 0, s, 1u,
+                               reinterpret_cast<const float4*>(part), (int)S, n4, dw_router))
             return MOE_ERR_CUDA;
     }
     // 10. dx_router = dlogit . W_router^T (fp32)
@@ -1474,8 +1502,8 @@ size_t moe_backward_workspace_size(int64_t T, int64_t d, int64_t E, int64_t k, i
 
 int moe_backward(const moe_bf16* x, const moe_bf16* w_router, const float* bias, const moe_bf16* w_gate,
                  const moe_bf16* w_up, const moe_bf16* w_down, const float* dout, int64_t T, int64_t d, int64_t E,
-                 int64_t k, int64_t f, float* dx, float* dw_router, float* dbias, float* dw_gate, float* dw_up,
-                 float* dw_down, void* workspace, size_t workspace_bytes, cudaStream_t stream, unsigned flags)
+                 int64_t k, int64_t f, float* dx, void* dw_router, float* dbias, void* dw_gate, void* dw_up,
+                 void* dw_down, void* workspace, size_t workspace_bytes, cudaStream_t stream, unsigned flags)
 {
     return backward_impl(x, w_router, bias, w_gate, w_up, w_down, dout, T, d, E, k, f, dx, dw_router, dbias, dw_gate,
                          dw_up, dw_down, workspace, workspace_bytes, stream, flags);
