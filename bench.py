@@ -105,7 +105,8 @@ def algorithmic(cfg, active_experts=None, n_shared=0):
 
 
 # Datasheet figures for a B200 (dense bf16, HBM3e), for the second fraction
-# of the forward roofline; the primary fraction uses the measured peaks.
+# of the forward roofline; the primary fraction uses the measured peaks
+# (the fallback figures when the peaks file is absent).
 DATASHEET = {"bf16_tflops": 2250.0, "hbm_gbs": 8000.0}
 
 
@@ -553,7 +554,9 @@ def run_gpu(args, cfg):
                                      "bound": "max(FLOPs / bf16 peak, compulsory bytes / HBM peak)"}},
             "forward_roofline": {"roofline_ms": roof_time * 1e3, "frac": roof_time / (ms * 1e-3),
                                  "flops": alg["flops"], "compulsory_bytes": alg["bytes"],
-                                 "peaks": "of measured (MEASURED_PEAKS.json)",
+                                 "peaks": ("of measured (MEASURED_PEAKS.json)" if peaks["source"] == "measured"
+                                           else "of fallback (no MEASURED_PEAKS.json: "
+                                                f"{peaks['bf16_tflops']:.0f} TFLOP/s, {peaks['hbm_gbs']:.0f} GB/s)"),
                                  "frac_of_datasheet": roof_ds / (ms * 1e-3),
                                  "datasheet_peaks": "2250 TFLOP/s dense bf16, 8000 GB/s"},
             "stage_gbs": {st: alg["stage_bytes"][st] / (stage_ms[st] * 1e-3) / 1e9
