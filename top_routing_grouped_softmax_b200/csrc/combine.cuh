@@ -6,8 +6,8 @@
 // y by the down-projection epilogue, so each token gathers its k grouped
 // fp16 rows through inv, widens them to fp32 and sums them in fp32 in slot
 // order -- a gather, not a scatter-add, so no atomics and a deterministic
-// result.  The output stays fp32: the accumulation is never rounded to a
-// narrower type.
+// result.  The sum is fp32 and by default is stored as fp32; an output
+// option rounds it to fp16 once, at the store.
 #pragma once
 
 #include <cuda_fp16.h>
@@ -33,9 +33,9 @@ __device__ __forceinline__ void add_f16x8(float (&acc)[8], const uint4& q)
 
 // One block per token; thread v handles 8 consecutive columns (16 bytes of
 // y, 32 bytes of out), with all k <= 8 row loads in flight at once.  The
-// kernel is launched after the down GEMM ends, not early beside its CTAs.  With shared experts (n_s > 0), their rows
-// y_s[s][t] (weight one, already applied) are added after the k routed
-// slots, in ascending s.  F16OUT: the fp32 sum is rounded to fp16 once, at
+// kernel is launched after the down GEMM ends, not early beside its CTAs.
+// With shared experts (n_s > 0), their rows y_s[s][t] (weight one, already
+// applied) are added after the k routed slots, in ascending s.  F16OUT: the fp32 sum is rounded to fp16 once, at
 // the store (16 bytes of out per thread); a value whose rounding leaves the
 // fp16 range (|v| >= 65520, or NaN) is stored as such and reported as
 // kStatusDeviceRange, as for y.

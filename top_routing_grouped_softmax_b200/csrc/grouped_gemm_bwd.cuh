@@ -28,16 +28,20 @@
 //        [f][d], its rows are the output columns).  Stores dg and du as bf16
 //        (in place of g and u).
 //   kDX  out = A1 . B1^T + A2 . B2^T with K split in two halves (the first
-//        k_split 64-blocks read A1/B1, the rest A2/B2), fp32 out:
-//        dx_perm = dg . W_gate[e]^T + du . W_up[e]^T, and (one group, one half)
-//        the router's dx = dlogit . W_router^T.  Whole 32-row slabs go out by
-//        TMA store; a slab that crosses the group's end is stored row by row.
+//        k_split 64-blocks read A1/B1, the rest A2/B2):
+//        dx_perm = dg . W_gate[e]^T + du . W_up[e]^T (out rounded to bf16), and
+//        (one group, one half) the router's dx = dlogit . W_router^T (fp32 out).
+//        Whole 32-row slabs go out by TMA store; a slab that crosses the
+//        group's end is stored row by row.
 //   kDW  out[e] = A_e^T . B_e, reduced over the rows of group e:
 //        A = the group's rows read MN-major (x_perm or hw, or x), B likewise
 //        (dg | du split over the pair, or dout_perm / dlogit).  One work item
 //        is (expert, 256-row M tile, 256-column N tile); an empty group writes
-//        zeros.  fp32 out by 3-D TMA store ([E][rows][cols] views clip the
-//        partial tiles).
+//        zeros.  fp32 out (or, as an option, the fp32 result rounded to bf16)
+//        by 3-D TMA store ([E][rows][cols] views clip the partial tiles).  With
+//        k_chunk the "groups" are fixed chunks of one operand pair's rows, so a
+//        long reduction (the router's weight gradient over all tokens) is split
+//        over many CTA pairs and the partial results are summed afterwards.
 //
 // No TMA load uses multicast.  Every wait is bounded (see ptx.cuh).
 #pragma once

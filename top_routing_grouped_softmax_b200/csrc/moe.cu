@@ -849,8 +849,9 @@ BLayout plan_backward(int64_t T, int64_t d, int64_t E, int64_t k, int64_t f)
     return L;
 }
 
-// to0 / to1: the fp32 output views of the weight-gradient kind (kDW); the
-// other kinds ignore them.
+// to0 / to1: the output maps of the TMA-store epilogues: the two weight-gradient
+// views of kDW (fp32 or bf16), the bf16 dx_perm rows of kDX (to0), the dg
+// and du chunks of kDH (to0, to1); kGU ignores them.
 template <int KIND>
 int launch_pair_bwd(const DeviceState& st, int64_t work, const CUtensorMap& ta, const CUtensorMap& ta2,
                     const CUtensorMap& tb0, const CUtensorMap& tb1, const moe::bwd::Params& p, cudaStream_t s,
@@ -863,9 +864,8 @@ int launch_pair_bwd(const DeviceState& st, int64_t work, const CUtensorMap& ta, 
                   moe::bwd::smem_bytes<KIND>(), s, 2u, ta, ta2, tb0, tb1, to0 ? *to0 : ta, to1 ? *to1 : ta, p);
 }
 
-// fp32 [groups][rows][cols] viewed for 32 x 32 TMA stores (128-byte swizzle);
-// elements outside the extents are clipped by the store.
-// bf16 [groups][rows][cols] for the same 32 x 32 stores (2 KB, 64-byte swizzle).
+// bf16 [groups][rows][cols] viewed for 32 x 32 TMA stores (2 KB slabs,
+// 64-byte swizzle); elements outside the extents are clipped by the store.
 int make_out3_map_bf16(CUtensorMap* m, void* base, uint64_t cols, uint64_t rows, uint64_t groups)
 {
     cuuint64_t dims[3] = {cols, rows, groups};
@@ -878,6 +878,7 @@ int make_out3_map_bf16(CUtensorMap* m, void* base, uint64_t cols, uint64_t rows,
     return r == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
 }
 
+// The same for fp32 (4 KB slabs, 128-byte swizzle).
 int make_out3_map(CUtensorMap* m, float* base, uint64_t cols, uint64_t rows, uint64_t groups)
 {
     cuuint64_t dims[3] = {cols, rows, groups};
