@@ -324,20 +324,25 @@ __device__ __forceinline__ void epilogue(const Params& p, const Item& it, uint32
                 uint32_t pdg[8], pdu[8];
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
-                    float dgv[2], duv[2];
-#pragma unroll
-                    for (int h2 = 0; h2 < 2; ++h2) {
-                        const int c = 2 * i + h2;
-                        const float dhu = __uint_as_float(acc[c]);  // dout . W_down^T (unweighted)
-                        const float sg = sigmoid(g[c]);
-                        const float gs = g[c] * sg;
-                        const float dh = w * dhu;
-                        dot += dhu * (gs * u[c]);
-                        dgv[h2] = dh * u[c] * sg * (1.0f + g[c] * (1.0f - sg));
-                        duv[h2] = dh * gs;
-                    }
-                    pdg[i] = gemm::pack_bf16x2(dgv[0], dgv[1]);
-                    pdu[i] = gemm::pack_bf16x2(duv[0], duv[1]);
+                    // two columns at a time: packed fp32 multiplies and FMAs
+                    // (each lane rounded as the scalar operation would be);
+                    // dh = w dhu, where dhu = dout . W_down^T is the
+                    // unweighted accumulator, and dot is a serial sum
+                    const float2 dhu = make_float2(__uint_as_float(acc[2 * i]), __uint_as_float(acc[2 * i + 1]));
+                    const float2 gg = make_float2(g[2 * i], g[2 * i + 1]);
+                    const float2 uu = make_float2(u[2 * i], u[2 * i + 1]);
+                    const float2 sg = make_float2(sigmoid(gg.x), sigmoid(gg.y));
+                    const float2 gs = __fmul2_rn(gg, sg);
+                    const float2 dh = __fmul2_rn(make_float2(w, w), dhu);
+                    const float2 hu = __fmul2_rn(gs, uu);
+                    dot = fmaf(dhu.x, hu.x, dot);
+                    dot = fmaf(dhu.y, hu.y, dot);
+                    const float2 om = __ffma2_rn(sg, make_float2(-1.0f, -1.0f), make_float2(1.0f, 1.0f));
+                    const float2 t = __ffma2_rn(gg, om, make_float2(1.0f, 1.0f));
+                    const float2 dg = __fmul2_rn(__fmul2_rn(__fmul2_rn(dh, uu), sg), t);
+                    const float2 du = __fmul2_rn(dh, gs);
+                    pdg[i] = gemm::pack_bf16x2(dg.x, dg.y);
+                    pdu[i] = gemm::pack_bf16x2(du.x, du.y);
                 }
                 if (whole) {
                     // the warp's 32 x 16 chunk of dg and du through the slab:
