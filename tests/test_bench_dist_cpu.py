@@ -58,3 +58,15 @@ def test_algorithmic_counts():
     a = bench.algorithmic(CONFIGS["qwen"])
     assert a["flops"] == 2 * 8192 * (2048 * 128 + 3 * 8 * 2048 * 768)
     assert a["gateup_flops"] + a["down_flops"] + 2 * 8192 * 2048 * 128 == a["flops"]
+
+
+def test_peaks_source(monkeypatch, tmp_path):
+    """The roofline denominators come from the peaks file when it exists and
+    are labelled as the fallback figures when it does not."""
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    p = bench.load_peaks()
+    assert p["source"] == "fallback"
+    assert p["bf16_tflops"] == bench.FALLBACK_PEAKS["bf16_tflops"]
+    (tmp_path / "MEASURED_PEAKS.json").write_text('{"hbm_gbs": 6554.6, "bf16_tflops": 1657.0}')
+    p = bench.load_peaks()
+    assert p == {"hbm_gbs": 6554.6, "bf16_tflops": 1657.0, "bf16_tflops_sustained": 1657.0, "source": "measured"}
