@@ -162,6 +162,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 decode_tile<kPairRows>(w, p.n_tiles, c.tp, c.off, E, e, row0, row_end, nt);
                 const int krow0 = e * p.K;
                 const int arow = row0 + (int)rank * kBM;
+                // A tail tile of at most 128 rows: the odd CTA's rows all lie past
+                // the group's end (its accumulator rows are never stored), so it
+                // loads no A and the stage expects 16 KB less.  Both CTAs decode
+                // the same tile, so they agree on this.
+                const bool odd_idle = row0 + kBM >= row_end;
+                const uint32_t stage_tx = (uint32_t)(2 * kPairStageBytes - (odd_idle ? kABytes : 0));
                 bool ok = true;
                 for (int kb = 0; kb < num_kb; ++kb) {
                     if (!mbar_wait(&c.empty[s], ph ^ 1u, limit)) {
@@ -170,10 +176,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     uint8_t* sa = smem + (size_t)s * kPairStageBytes;
                     uint8_t* sb = sa + kABytes;
-                    if (leader) mbar_arrive_expect_tx(&c.full[s], (uint32_t)(2 * kPairStageBytes));
+                    if (leader) mbar_arrive_expect_tx(&c.full[s], stage_tx);
                     const uint32_t bar = mapa_shared(&c.full[s], 0);
                     const int kr = krow0 + kb * kBK;
-                    tma_load_2d_pair(sa, &tm_a, bar, kb * kBK, arow);
+                    if (leader || !odd_idle) tma_load_2d_pair(sa, &tm_a, bar, kb * kBK, arow);
                     // 128 weight columns as two 64-column chunks in one copy (the
                     // weight maps view [K, N] as [N/64][K][64])
                     if (EPI == kSwiGLU) {
