@@ -580,6 +580,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             int64_t issued = 0;
             for (int64_t w = pair; w < total_work && !c.abort_flag; w += npairs) {
                 const Item it = decode_item<KIND>(w, p, c);
+                // M-grouped kinds: on a tail tile whose odd half lies wholly past
+                // the group's end (rows never stored), the odd CTA loads no A
+                const bool odd_idle = KIND != kDW && it.row0 + kBM >= it.row_end;
+                const uint32_t stage_tx = (uint32_t)(2 * kPairStageBytes - (odd_idle ? kABytes : 0));
+                const bool load_a = leader || !odd_idle;
                 bool ok = true;
                 for (int kb = 0; kb < it.num_kb; ++kb) {
                     if (!mbar_wait(&c.empty[s], ph ^ 1u, limit)) {
@@ -588,18 +593,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     uint8_t* sa = smem + (size_t)s * kPairStageBytes;
                     uint8_t* sb = sa + kABytes;
-                    if (leader) mbar_arrive_expect_tx(&c.full[s], (uint32_t)(2 * kPairStageBytes));
+                    if (leader) mbar_arrive_expect_tx(&c.full[s], stage_tx);
                     const uint32_t bar = mapa_shared(&c.full[s], 0);
                     if constexpr (KIND == kGU) {
-                        tma_load_2d_pair(sa, &tm_a, bar, kb * kBK, it.row0 + (int)rank * kBM);
+                        if (load_a) tma_load_2d_pair(sa, &tm_a, bar, kb * kBK, it.row0 + (int)rank * kBM);
                         tma_load_3d_pair(sb, leader ? &tm_b0 : &tm_b1, bar, 0, it.e * p.b_rows + kb * kBK, it.nt * 2);
                     } else if constexpr (KIND == kDH) {
-                        tma_load_2d_pair(sa, &tm_a, bar, kb * kBK, it.row0 + (int)rank * kBM);
+                        if (load_a) tma_load_2d_pair(sa, &tm_a, bar, kb * kBK, it.row0 + (int)rank * kBM);
                         tma_load_2d_pair(sb, &tm_b0, bar, kb * kBK, it.e * p.b_rows + it.nt * kBN + (int)rank * kBM);
                     } else if constexpr (KIND == kDX) {
                         const bool second = kb >= p.k_split;
                         const int kc = (second ? kb - p.k_split : kb) * kBK;
-                        tma_load_2d_pair(sa, second ? &tm_a2 : &tm_a, bar, kc, it.row0 + (int)rank * kBM);
+                        if (load_a) tma_load_2d_pair(sa, second ? &tm_a2 : &tm_a, bar, kc, it.row0 + (int)rank * kBM);
                         tma_load_2d_pair(sb, second ? &tm_b1 : &tm_b0, bar, kc,
                                          it.e * p.b_rows + it.nt * kBN + (int)rank * kBM);
                     } else {
