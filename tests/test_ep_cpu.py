@@ -25,6 +25,8 @@ class CpuStages:
     """Test stand-ins for the kernels: fp64 routing / grouping from the oracle
     and numpy SwiGLU experts; y rows stay fp64."""
 
+    y_dtype = torch.float64
+
     def __init__(self, oracle, E_total):
         self.o = oracle
         self.E_total = E_total
@@ -74,8 +76,11 @@ def _inputs():
 
 
 def _token_ranges(T, world, uneven):
-    """Each rank's token slice: equal shares, or uneven ones (rank r gets
-    r + 1 parts) so that ranks send and receive different row counts."""
+    """Each rank's token slice: equal shares, uneven ones (rank r gets r + 1
+    parts) so that ranks send and receive different row counts, or
+    ("empty") every token on rank 0 and none on the others."""
+    if uneven == "empty":
+        return [(0, T)] + [(T, T)] * (world - 1)
     w = [r + 1 for r in range(world)] if uneven else [1] * world
     cuts = [0]
     for r in range(world):
@@ -138,6 +143,23 @@ def test_four_ranks_uneven_tokens_match_single_process():
         e0, e1 = owner_block(cfg.E, world, rank)
         assert recv_counts.shape == (world, e1 - e0)
         assert recv_counts.sum(axis=0).tolist() == counts[e0:e1].tolist()
+
+
+@pytest.mark.timeout(240)
+def test_rank_without_tokens():
+    """A rank with no tokens of its own still serves its experts: it sends
+    nothing, receives rank 0's rows for its experts, and returns an empty
+    output; rank 0's output equals the single-process forward."""
+    world = 2
+    res = _run_ranks(world, 29547, uneven="empty")
+    cfg, ids, ref = _single_process_reference()
+    counts = np.bincount(ids.ravel(), minlength=cfg.E)
+    (r0, out0, rc0, _), (r1, out1, rc1, off1) = res
+    np.testing.assert_allclose(out0, ref, rtol=1e-12, atol=1e-14)
+    assert out1.shape == (0, cfg.d)
+    e0, e1 = owner_block(cfg.E, world, 1)
+    assert rc1[1].sum() == 0 and rc1[0].tolist() == counts[e0:e1].tolist()
+    assert off1[-1] == counts[e0:e1].sum()
 
 
 @pytest.mark.timeout(180)

@@ -96,6 +96,8 @@ def plan_dispatch(recv_counts: np.ndarray) -> DispatchPlan:
 class CudaStages:
     """The library's kernels as the stages of the expert-parallel forward."""
 
+    y_dtype = torch.float16  # the grouped GEMM's y rows
+
     def __init__(self):
         import top_routing_grouped_softmax_b200 as moe
         self.moe = moe
@@ -122,7 +124,11 @@ def _exchange(t: torch.Tensor, out_rows: int, out_split, in_split, group) -> tor
     moves."""
     t = t.contiguous()
     packed = t.element_size() == 2
-    view = t.view(t.shape[0], -1).view(torch.int32) if packed else t
+    row = 1
+    for n in t.shape[1:]:
+        row *= int(n)
+    # an explicit row width: a rank may send no rows at all
+    view = t.view(t.shape[0], row).view(torch.int32) if packed else t
     out = torch.empty((out_rows,) + tuple(view.shape[1:]), dtype=view.dtype, device=view.device)
     dist.all_to_all_single(out, view, output_split_sizes=out_split, input_split_sizes=in_split, group=group)
     return out.view(t.dtype).view((out_rows,) + tuple(t.shape[1:])) if packed else out
@@ -184,7 +190,8 @@ class ExpertParallelMoE:
             y_grp = st.expert_ffn(x_grp, w_grp, offsets, self.w_gate, self.w_up, self.w_down)
             y_recv = st.gather_rows(y_grp, ungroup)
         else:
-            y_recv = torch.empty(0, x.shape[1], dtype=torch.float16, device=dev)
+            # no rows for this rank's experts: an empty block of the stages' y type
+            y_recv = torch.empty(0, x.shape[1], dtype=getattr(st, "y_dtype", torch.float16), device=dev)
         # 4. return: the reverse exchange puts every y row back at its grouped
         #    position on the rank that owns the token
         y_back = _exchange(y_recv, T * self.k, send_split, recv_split, self.group)
