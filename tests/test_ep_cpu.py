@@ -88,11 +88,21 @@ def _token_ranges(T, world, uneven):
     return [(cuts[r], cuts[r + 1]) for r in range(world)]
 
 
-def _worker(rank, world, port, q, uneven=False):
+def _cold_bias(cfg):
+    """A router bias that no expert of the upper half survives: their owner
+    ranks receive no rows at all."""
+    b = torch.zeros(cfg.E, dtype=torch.float32)
+    b[cfg.E // 2:] = -1.0e4
+    return b
+
+
+def _worker(rank, world, port, q, uneven=False, cold=False):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=rank, world_size=world)
     from oracle.oracle import default_oracle
     cfg, inp = _inputs()
+    if cold:
+        inp.bias = _cold_bias(cfg)
     e0, e1 = owner_block(cfg.E, world, rank)
     t0, t1 = _token_ranges(cfg.T, world, uneven)[rank]
     x = inp.x[t0:t1].contiguous()
@@ -106,10 +116,10 @@ def _worker(rank, world, port, q, uneven=False):
     q.put((rank, out, plan.recv_counts, plan.offsets))
 
 
-def _run_ranks(world, port, uneven):
+def _run_ranks(world, port, uneven, cold=False):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
-    procs = [ctx.Process(target=_worker, args=(r, world, port, q, uneven)) for r in range(world)]
+    procs = [ctx.Process(target=_worker, args=(r, world, port, q, uneven, cold)) for r in range(world)]
     for p in procs:
         p.start()
     res = sorted((q.get(timeout=150) for _ in range(world)), key=lambda r: r[0])
@@ -119,9 +129,11 @@ def _run_ranks(world, port, uneven):
     return res
 
 
-def _single_process_reference():
+def _single_process_reference(cold=False):
     from oracle.oracle import default_oracle
     cfg, inp = _inputs()
+    if cold:
+        inp.bias = _cold_bias(cfg)
     st = CpuStages(default_oracle(), cfg.E)
     ids, w = st.route(inp.x, inp.W_router, cfg.k, inp.bias)
     pm = st.permute(inp.x, ids, w, cfg.E)
@@ -160,6 +172,20 @@ def test_rank_without_tokens():
     e0, e1 = owner_block(cfg.E, world, 1)
     assert rc1[1].sum() == 0 and rc1[0].tolist() == counts[e0:e1].tolist()
     assert off1[-1] == counts[e0:e1].sum()
+
+
+@pytest.mark.timeout(240)
+def test_rank_whose_experts_get_no_rows():
+    """No token picks the experts of rank 1: it receives nothing, computes
+    nothing, and the return exchange still delivers every rank's rows."""
+    world = 2
+    res = _run_ranks(world, 29551, uneven=False, cold=True)
+    cfg, ids, ref = _single_process_reference(cold=True)
+    assert ids.max() < cfg.E // 2
+    for (rank, out, recv_counts, offsets), (t0, t1) in zip(res, _token_ranges(cfg.T, world, False)):
+        np.testing.assert_allclose(out, ref[t0:t1], rtol=1e-12, atol=1e-14)
+        if rank == 1:
+            assert recv_counts.sum() == 0 and offsets[-1] == 0
 
 
 @pytest.mark.timeout(180)
